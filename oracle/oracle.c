@@ -1,0 +1,1090 @@
+/*
+ * oracle.c -- reference implementation (the oracle) of the EntroPack-style lattice-rANS
+ * weight codec: encoder, blob writer and decoder.
+ *
+ * TEST INFRASTRUCTURE.  Only the test suite, the smoke check and the CPU-baseline leg of the
+ * benchmark load this library.  The product path (the CUDA library and its host encoder) never
+ * calls it, and the two share no code, header, table or constant.
+ *
+ * Plain, single-threaded C99 in double precision, written to be checked by eye against the
+ * method's description rather than to be fast.  Sources, cited by page title and section:
+ *
+ *   [ABS]  "EntroPack: Fast and Accurate Entropy-Coded Weight Compression at Arbitrary
+ *          Bitrates", arXiv abstract page (row-normalised E8 quantisation, conditional model,
+ *          sampled storage estimates, independently decodable tiles, BF16/FP16/FP8 containers).
+ *   [DOC]  "EntroPack lattice compression", documentation page Principles / Lattice-rANS:
+ *            DOC-0  opening paragraph (2-D tensors, target range [0.001, 11] bits per element,
+ *                   decompression keeps the input dtype);
+ *            DOC-LQ section "Lattice quantization and integer fields";
+ *            DOC-RS section "Rate selection and refinement";
+ *            DOC-ER section "Encoding and reconstruction";
+ *            DOC-U  section "Usage".
+ *   [ANS]  J. Duda, "Asymmetric numeral systems" (2009) -- the rANS coding step; cited in the
+ *          reference list of the Crossref record "Learned Lossless Image Compression with
+ *          Interleaved Parallel Inference and Irregular Causal Reasoning".
+ *   [CS]   J. H. Conway and N. J. A. Sloane, "Fast quantizing and decoding algorithms for lattice
+ *          quantizers and codes" (1982): nearest point of D8, and of E8 = D8 u (D8 + 1/2).
+ *   [OCP]  OCP 8-bit floating point specification: the E4M3 encoding (bias 7, no infinities,
+ *          largest finite 448).
+ *
+ * Where the pages leave a step open, the step is marked "reading:" and the same reading is
+ * listed in the design notes.  The format these functions write and read is the blob format
+ * described there; it is restated next to each writer below.
+ *
+ * Parity status of each function (which independent check pins it) is listed in the test
+ * suite's oracle pin file; every function here is pinned.
+ */
+#include <math.h>
+#include <stdint.h>
+#include <stdlib.h>
+#include <string.h>
+
+/* ------------------------------------------------------------------------------------------ */
+/* Constants of the format.                                                                    */
+/* ------------------------------------------------------------------------------------------ */
+
+enum { ORC_BF16 = 1, ORC_FP16 = 2, ORC_E4M3 = 3, ORC_F32 = 4 };
+
+#define ORC_R 127          /* reading: field alphabet [-R, R] coded directly, R = 127     */
+#define ORC_ESC 255        /* symbol that announces a raw 16-bit field value               */
+#define ORC_M 4096u        /* frequency totals are 12-bit: every table sums to 4096       */
+#define ORC_L 65536u       /* rANS lower bound 2^16, 32-bit state, 16-bit renormalisation */
+#define ORC_LANES 32       /* interleaved rANS states per tile                            */
+#define ORC_NCTX 17        /* context 0: coset; 1 + 8c + (j-1): field j given coset c     */
+#define ORC_HEADER 80      /* bytes in the fixed header                                   */
+#define ORC_CLAMP 32764.0  /* reading: |t| clamp, keeps every field inside int16          */
+
+/* ------------------------------------------------------------------------------------------ */
+/* Little-endian byte access.                                                                  */
+/* ------------------------------------------------------------------------------------------ */
+
+static void put16(uint8_t* p, uint32_t v) { p[0] = (uint8_t)v; p[1] = (uint8_t)(v >> 8); }
+static void put32(uint8_t* p, uint32_t v) { for (int i = 0; i < 4; i++) p[i] = (uint8_t)(v >> (8 * i)); }
+static void put64(uint8_t* p, uint64_t v) { for (int i = 0; i < 8; i++) p[i] = (uint8_t)(v >> (8 * i)); }
+static uint32_t get16(const uint8_t* p) { return (uint32_t)p[0] | ((uint32_t)p[1] << 8); }
+static uint32_t get32(const uint8_t* p) {
+    return (uint32_t)p[0] | ((uint32_t)p[1] << 8) | ((uint32_t)p[2] << 16) | ((uint32_t)p[3] << 24);
+}
+static uint64_t get64(const uint8_t* p) {
+    uint64_t v = 0;
+    for (int i = 7; i >= 0; i--) v = (v << 8) | p[i];
+    return v;
+}
+static uint64_t pad16(uint64_t n) { return (n + 15u) / 16u * 16u; }
+
+/* ------------------------------------------------------------------------------------------ */
+/* Number formats: reading each container exactly, and rounding to it.                        */
+/* [DOC-0]: the tensor is restored in the input's dtype; [ABS] lists BF16, FP16 and FP8.       */
+/* ------------------------------------------------------------------------------------------ */
+
+/* Exact value of one stored element of the given dtype. */
+double orc_dtype_to_f64(uint32_t bits, int dtype)
+{
+    if (dtype == ORC_BF16) {                       /* BF16 = the high half of an fp32 */
+        uint32_t w = bits << 16;
+        float f;
+        memcpy(&f, &w, 4);
+        return (double)f;
+    }
+    if (dtype == ORC_F32) {
+        float f;
+        memcpy(&f, &bits, 4);
+        return (double)f;
+    }
+    if (dtype == ORC_FP16) {                       /* IEEE binary16: 1 + 5 + 10 bits */
+        int s = (bits >> 15) & 1, e = (bits >> 10) & 31, m = bits & 1023;
+        double v;
+        if (e == 0) v = ldexp((double)m, -24);
+        else if (e == 31) v = m ? NAN : INFINITY;
+        else v = ldexp((double)(1024 + m), e - 25);
+        return s ? -v : v;
+    }
+    if (dtype == ORC_E4M3) {                       /* [OCP] E4M3: 1 + 4 + 3 bits, bias 7 */
+        int s = (bits >> 7) & 1, e = (bits >> 3) & 15, m = bits & 7;
+        double v;
+        if (e == 15 && m == 7) v = NAN;
+        else if (e == 0) v = ldexp((double)m, -9);
+        else v = ldexp((double)(8 + m), e - 10);
+        return s ? -v : v;
+    }
+    return NAN;
+}
+
+/*
+ * Round v to a binary format with p significand bits, smallest normal exponent emin and largest
+ * finite value maxf, ties to even.  v must be finite.  The quantum (the value of the last
+ * significand bit) is 2^(max(exponent(v), emin) - (p - 1)); v / quantum is exact because the
+ * quantum is a power of two, and rint() rounds it half-to-even in the default rounding mode.
+ */
+static double round_to_format(double v, int p, int emin, double maxf, int* overflow)
+{
+    *overflow = 0;
+    if (v == 0.0) return v;
+    int e;
+    frexp(v, &e);                                  /* v = m * 2^e with 0.5 <= |m| < 1 */
+    int lead = e - 1;                              /* exponent of the leading bit     */
+    if (lead < emin) lead = emin;                  /* subnormal range: fixed quantum  */
+    double quantum = ldexp(1.0, lead - (p - 1));
+    double r = rint(v / quantum) * quantum;
+    if (fabs(r) > maxf) *overflow = 1;
+    return r;
+}
+
+/* fp32 with round-to-nearest-even; returns the fp32 bit pattern. */
+uint32_t orc_round_f32(double v)
+{
+    uint32_t bits;
+    float f;
+    if (isnan(v)) { bits = 0x7FC00000u; return bits; }
+    if (isinf(v)) { f = (float)v; memcpy(&bits, &f, 4); return bits; }
+    int ovf;
+    double r = round_to_format(v, 24, -126, (double)3.4028234663852886e38, &ovf);
+    if (ovf) r = r > 0 ? INFINITY : -INFINITY;
+    f = (float)r;                                  /* exact: r is an fp32 value */
+    memcpy(&bits, &f, 4);
+    return bits;
+}
+
+/* fp32 bit pattern -> BF16 (8 significand bits, fp32 exponent range), RNE, overflow -> inf. */
+uint32_t orc_f32_to_bf16(uint32_t fbits)
+{
+    float f;
+    memcpy(&f, &fbits, 4);
+    uint32_t sign = (fbits >> 16) & 0x8000u;
+    if (isnan(f)) return sign | 0x7FC0u;
+    if (isinf(f)) return sign | 0x7F80u;
+    int ovf;
+    double r = round_to_format((double)f, 8, -126, ldexp(255.0, 120), &ovf);
+    if (ovf) return sign | 0x7F80u;
+    float g = (float)r;                            /* exact: r has 8 significant bits */
+    uint32_t gb;
+    memcpy(&gb, &g, 4);
+    return (gb >> 16) | sign;                      /* keeps the sign of a zero too */
+}
+
+/* fp32 bit pattern -> IEEE binary16, RNE with subnormals, overflow -> inf. */
+uint32_t orc_f32_to_f16(uint32_t fbits)
+{
+    float f;
+    memcpy(&f, &fbits, 4);
+    uint32_t sign = (fbits >> 16) & 0x8000u;
+    if (isnan(f)) return sign | 0x7E00u;
+    if (isinf(f)) return sign | 0x7C00u;
+    int ovf;
+    double r = fabs(round_to_format((double)f, 11, -14, 65504.0, &ovf));
+    if (ovf) return sign | 0x7C00u;
+    if (r < ldexp(1.0, -14)) return sign | (uint32_t)(r / ldexp(1.0, -24));   /* subnormal or 0 */
+    int e;
+    frexp(r, &e);
+    int lead = e - 1;                              /* -14 .. 15 */
+    uint32_t mant = (uint32_t)(r / ldexp(1.0, lead - 10)) - 1024u;
+    return sign | ((uint32_t)(lead + 15) << 10) | mant;
+}
+
+/* fp32 bit pattern -> OCP E4M3, RNE, saturating to +-448 (no infinities); NaN -> NaN. */
+uint32_t orc_f32_to_e4m3(uint32_t fbits)
+{
+    float f;
+    memcpy(&f, &fbits, 4);
+    uint32_t sign = (fbits >> 24) & 0x80u;
+    if (isnan(f)) return sign | 0x7Fu;
+    if (isinf(f)) return sign | 0x7Eu;            /* saturate */
+    int ovf;
+    double r = fabs(round_to_format((double)f, 4, -6, 448.0, &ovf));
+    if (ovf) return sign | 0x7Eu;                 /* saturate */
+    if (r < ldexp(1.0, -6)) return sign | (uint32_t)(r / ldexp(1.0, -9));     /* subnormal or 0 */
+    int e;
+    frexp(r, &e);
+    int lead = e - 1;                              /* -6 .. 8 */
+    uint32_t mant = (uint32_t)(r / ldexp(1.0, lead - 3)) - 8u;
+    return sign | ((uint32_t)(lead + 7) << 3) | mant;
+}
+
+/* Array form of the three conversions (used by the exhaustive conversion checks). */
+void orc_cvt_f32_array(const uint32_t* in, uint64_t n, int dtype_out, void* out)
+{
+    for (uint64_t i = 0; i < n; i++) {
+        if (dtype_out == ORC_BF16) ((uint16_t*)out)[i] = (uint16_t)orc_f32_to_bf16(in[i]);
+        else if (dtype_out == ORC_FP16) ((uint16_t*)out)[i] = (uint16_t)orc_f32_to_f16(in[i]);
+        else if (dtype_out == ORC_E4M3) ((uint8_t*)out)[i] = (uint8_t)orc_f32_to_e4m3(in[i]);
+        else ((uint32_t*)out)[i] = in[i];
+    }
+}
+
+/* Store one reconstructed value w (exact, double) into out[idx] of dtype dtype_out:
+ * first the fp32 product rounding, then the container rounding. */
+static void store_value(void* out, uint64_t idx, int dtype_out, double w)
+{
+    uint32_t fb = orc_round_f32(w);
+    if (dtype_out == ORC_BF16) ((uint16_t*)out)[idx] = (uint16_t)orc_f32_to_bf16(fb);
+    else if (dtype_out == ORC_FP16) ((uint16_t*)out)[idx] = (uint16_t)orc_f32_to_f16(fb);
+    else if (dtype_out == ORC_E4M3) ((uint8_t*)out)[idx] = (uint8_t)orc_f32_to_e4m3(fb);
+    else ((uint32_t*)out)[idx] = fb;
+}
+
+static int dtype_size(int dtype)
+{
+    return dtype == ORC_E4M3 ? 1 : dtype == ORC_F32 ? 4 : (dtype == ORC_BF16 || dtype == ORC_FP16) ? 2 : 0;
+}
+
+static uint32_t load_bits(const void* data, int dtype, uint64_t i)
+{
+    if (dtype == ORC_E4M3) return ((const uint8_t*)data)[i];
+    if (dtype == ORC_F32) return ((const uint32_t*)data)[i];
+    return ((const uint16_t*)data)[i];
+}
+
+/* ------------------------------------------------------------------------------------------ */
+/* E8 nearest point [CS], used as [DOC-LQ] describes: nearest point of a scaled E8.            */
+/* ------------------------------------------------------------------------------------------ */
+
+/*
+ * Nearest point of D8 = { z in Z^8 : sum z even } to u [CS]: round every coordinate to the
+ * nearest integer; if the sum of the rounded vector is odd, round the coordinate that was
+ * furthest from its integer the other way.
+ * reading: ties in rounding go away from zero (C round()); ties for the furthest coordinate go
+ * to the lowest index; when that coordinate is exactly an integer, "the other way" is +1.
+ */
+static void d8_nearest(const double u[8], double g[8])
+{
+    long long sum = 0;
+    for (int i = 0; i < 8; i++) {
+        g[i] = round(u[i]);
+        sum += (long long)g[i];
+    }
+    if (sum % 2 != 0) {
+        int k = 0;
+        double worst = -1.0;
+        for (int i = 0; i < 8; i++) {
+            double d = fabs(u[i] - g[i]);
+            if (d > worst) { worst = d; k = i; }
+        }
+        if (u[k] > g[k]) g[k] += 1.0;
+        else if (u[k] < g[k]) g[k] -= 1.0;
+        else g[k] += 1.0;
+    }
+}
+
+/*
+ * Nearest point of E8 = D8 u (D8 + 1/2) to t [CS]: take the nearest point of D8 and the nearest
+ * point of the half-integer coset (the D8 rule applied to t - 1/2, then + 1/2), and keep the
+ * nearer of the two.  The coset bit is 0 for the integer coset and 1 for the half-integer one
+ * ([DOC-LQ]: "E8 has integer-coordinate and half-integer-coordinate subsets, called cosets").
+ * reading: an exact tie in squared distance keeps coset 0.
+ */
+void orc_e8_nearest(const double t[8], double y[8], int* coset)
+{
+    double a[8], b[8], u[8];
+    d8_nearest(t, a);
+    for (int i = 0; i < 8; i++) u[i] = t[i] - 0.5;
+    d8_nearest(u, b);
+    for (int i = 0; i < 8; i++) b[i] += 0.5;
+    double da = 0.0, db = 0.0;
+    for (int i = 0; i < 8; i++) {
+        da += (t[i] - a[i]) * (t[i] - a[i]);
+        db += (t[i] - b[i]) * (t[i] - b[i]);
+    }
+    if (db < da) {
+        memcpy(y, b, sizeof b);
+        *coset = 1;
+    } else {
+        memcpy(y, a, sizeof a);
+        *coset = 0;
+    }
+}
+
+/* ------------------------------------------------------------------------------------------ */
+/* Coset bit + eight integer fields [DOC-LQ].                                                 */
+/* ------------------------------------------------------------------------------------------ */
+
+/*
+ * Lattice point -> fields.  z = y - c/2 lies in D8 (sum even).  f1..f7 = z1..z7, and the
+ * parity constraint compacts the last coordinate: with par = (z1 + ... + z7) mod 2 in {0, 1},
+ * z8 - par is even and f8 = (z8 - par) / 2 ([DOC-LQ]: "using the lattice's parity constraint
+ * to compact the final coordinate").
+ * reading: for coset 1 the half is subtracted (z = y - 1/2).
+ */
+void orc_point_to_fields(const double y[8], int coset, int32_t f[8])
+{
+    int32_t z[8];
+    for (int i = 0; i < 8; i++) z[i] = (int32_t)(y[i] - 0.5 * coset);
+    int32_t s7 = 0;
+    for (int i = 0; i < 7; i++) s7 += z[i];
+    int32_t par = ((s7 % 2) + 2) % 2;
+    for (int i = 0; i < 7; i++) f[i] = z[i];
+    f[7] = (z[7] - par) / 2;
+}
+
+/* Fields -> lattice point, the arithmetic inverse ([DOC-LQ]: "inverted arithmetically without a
+ * reconstruction codebook"): z8 = 2 f8 + par, y = z + c/2. */
+void orc_fields_to_point(int coset, const int32_t f[8], double y[8])
+{
+    int32_t z[8];
+    int32_t s7 = 0;
+    for (int i = 0; i < 7; i++) { z[i] = f[i]; s7 += f[i]; }
+    int32_t par = ((s7 % 2) + 2) % 2;
+    z[7] = 2 * f[7] + par;
+    for (int i = 0; i < 8; i++) y[i] = (double)z[i] + 0.5 * coset;
+}
+
+/* Field value -> symbol of the 256-letter alphabet.  reading: |f| <= 127 is coded as f + 127
+ * (symbols 0..254); anything else is the escape symbol 255 followed by the raw 16-bit value. */
+static int field_symbol(int32_t f) { return (f >= -ORC_R && f <= ORC_R) ? f + ORC_R : ORC_ESC; }
+
+/* ------------------------------------------------------------------------------------------ */
+/* Probability tables with 12-bit totals.                                                     */
+/* ------------------------------------------------------------------------------------------ */
+
+/*
+ * Quantise symbol counts n[0..255] to frequencies q[] summing to 4096.
+ * reading: q_s = max(1, round_half_up(4096 n_s / N)) for n_s > 0, else 0; then, while the sum
+ * exceeds 4096, decrement the largest q (> 1; lowest symbol on ties); while it is below 4096,
+ * increment the symbol with the largest count (lowest symbol on ties).  N = 0 gives all zeros.
+ */
+void orc_quantize_table(const uint64_t n[256], uint16_t q[256])
+{
+    uint64_t N = 0;
+    for (int s = 0; s < 256; s++) N += n[s];
+    for (int s = 0; s < 256; s++) q[s] = 0;
+    if (N == 0) return;
+    long sum = 0;
+    for (int s = 0; s < 256; s++) {
+        if (n[s] == 0) continue;
+        uint64_t v = (2u * ORC_M * n[s] + N) / (2u * N);      /* round half up */
+        if (v < 1) v = 1;
+        q[s] = (uint16_t)v;
+        sum += (long)v;
+    }
+    while (sum > (long)ORC_M) {
+        int best = -1;
+        for (int s = 0; s < 256; s++)
+            if (q[s] > 1 && (best < 0 || q[s] > q[best])) best = s;
+        q[best]--;
+        sum--;
+    }
+    while (sum < (long)ORC_M) {
+        int best = -1;
+        for (int s = 0; s < 256; s++)
+            if (n[s] > 0 && (best < 0 || n[s] > n[best])) best = s;
+        q[best]++;
+        sum++;
+    }
+}
+
+/* Cumulative frequencies: cum[s] = q[0] + ... + q[s-1]. */
+static void cumulate(const uint16_t q[256], uint32_t cum[257])
+{
+    cum[0] = 0;
+    for (int s = 0; s < 256; s++) cum[s + 1] = cum[s] + q[s];
+}
+
+/* Context index of sub-step u (0 = coset, 1..8 = field u) of a vector with coset c. */
+static int context_of(int u, int c) { return u == 0 ? 0 : 1 + 8 * c + (u - 1); }
+
+/* ------------------------------------------------------------------------------------------ */
+/* Tiled, 32-way interleaved rANS [ANS] with the word order of the format ([DOC-ER]: "encoded   */
+/* with rANS in independently decodable tiles").                                               */
+/*                                                                                            */
+/* One tile holds up to 32*S consecutive vectors; lane l at step k owns vector 32k + l of the  */
+/* tile.  Each vector is 9 symbols: the coset (context 0) and f1..f8 (context 1 + 8c + j - 1).  */
+/* Decode order: for each step k, for each sub-step u = 0..8, lanes 0..31 in turn decode their */
+/* symbol and, if the 32-bit state fell below 2^16, read the next 16-bit word; after sub-step 8 */
+/* the raw words of escaped fields follow, ordered by field j = 1..8, then lane.               */
+/* Tile bytes: 32 little-endian u32 initial states (lane order), the u16 words in decode order, */
+/* zero padding to a multiple of 16 bytes.  Every lane ends in state 2^16.                     */
+/* ------------------------------------------------------------------------------------------ */
+
+typedef struct {
+    uint16_t* w;
+    uint64_t n, cap;
+} wordbuf;
+
+static int push_word(wordbuf* b, uint32_t v)
+{
+    if (b->n == b->cap) {
+        uint64_t nc = b->cap ? 2 * b->cap : 1024;
+        uint16_t* nw = (uint16_t*)realloc(b->w, nc * sizeof(uint16_t));
+        if (!nw) return -1;
+        b->w = nw;
+        b->cap = nc;
+    }
+    b->w[b->n++] = (uint16_t)v;
+    return 0;
+}
+
+/*
+ * Encode one tile.  sym9[v*9 + u] is the symbol of sub-step u of vector v, raw8[v*8 + j-1] the raw
+ * value of field j (used when its symbol is the escape).  q17 holds the 17 context tables
+ * (17 x 256 frequencies).  Returns the tile size in bytes (written to out when out != NULL and
+ * cap is large enough), or 0 on failure.
+ *
+ * rANS encode of symbol s with frequency q and cumulative cum [ANS]: while x >= q * 2^20,
+ * emit the low 16 bits of x and shift them out; then x <- floor(x / q) * 4096 + (x mod q) + cum.
+ * The encoder runs in reverse decode order and the emitted words are reversed at the end.
+ */
+uint64_t orc_encode_tile(const uint8_t* sym9, const int16_t* raw8, int64_t nvec,
+                         const uint16_t* q17, uint8_t* out, uint64_t cap)
+{
+    uint32_t cum[ORC_NCTX][257];
+    for (int c = 0; c < ORC_NCTX; c++) cumulate(q17 + 256 * c, cum[c]);
+    uint32_t x[ORC_LANES];
+    for (int l = 0; l < ORC_LANES; l++) x[l] = ORC_L;
+    wordbuf wb = {0, 0, 0};
+    int64_t nsteps = (nvec + ORC_LANES - 1) / ORC_LANES;
+    for (int64_t k = nsteps - 1; k >= 0; k--) {
+        for (int j = 8; j >= 1; j--)
+            for (int l = ORC_LANES - 1; l >= 0; l--) {
+                int64_t v = k * ORC_LANES + l;
+                if (v < nvec && sym9[v * 9 + j] == ORC_ESC)
+                    if (push_word(&wb, (uint16_t)raw8[v * 8 + (j - 1)])) goto fail;
+            }
+        for (int u = 8; u >= 0; u--)
+            for (int l = ORC_LANES - 1; l >= 0; l--) {
+                int64_t v = k * ORC_LANES + l;
+                if (v >= nvec) continue;
+                int s = sym9[v * 9 + u];
+                int ctx = context_of(u, sym9[v * 9]);
+                uint32_t q = q17[256 * ctx + s];
+                if (q == 0) goto fail;
+                if ((uint64_t)x[l] >= ((uint64_t)q << 20)) {
+                    if (push_word(&wb, x[l] & 0xFFFFu)) goto fail;
+                    x[l] >>= 16;
+                }
+                x[l] = (x[l] / q) * ORC_M + (x[l] % q) + cum[ctx][s];
+            }
+    }
+    uint64_t bytes = pad16(4u * ORC_LANES + 2u * wb.n);
+    if (out && cap >= bytes) {
+        memset(out, 0, bytes);
+        for (int l = 0; l < ORC_LANES; l++) put32(out + 4 * l, x[l]);
+        for (uint64_t i = 0; i < wb.n; i++)                      /* reversed emission order */
+            put16(out + 4 * ORC_LANES + 2 * i, wb.w[wb.n - 1 - i]);
+    }
+    free(wb.w);
+    return bytes;
+fail:
+    free(wb.w);
+    return 0;
+}
+
+/* Decoding tables of the 17 contexts: cumulative frequencies and the symbol of every slot. */
+typedef struct {
+    const uint16_t* q17;
+    uint32_t cum[ORC_NCTX][257];
+    uint8_t slot_sym[ORC_NCTX][ORC_M];
+} dtables;
+
+static void build_dtables(const uint16_t* q17, dtables* T)
+{
+    T->q17 = q17;
+    for (int c = 0; c < ORC_NCTX; c++) {
+        cumulate(q17 + 256 * c, T->cum[c]);
+        memset(T->slot_sym[c], 0, ORC_M);
+        for (int s = 0; s < 256; s++)
+            for (uint32_t i = T->cum[c][s]; i < T->cum[c][s + 1] && i < ORC_M; i++) T->slot_sym[c][i] = (uint8_t)s;
+    }
+}
+
+/*
+ * Decode one tile of nvec vectors with prepared tables.  Writes sym9 / raw8 as orc_encode_tile
+ * reads them and the 32 final states.  rANS decode [ANS]: slot = x mod 4096, s = the symbol with
+ * cum[s] <= slot < cum[s+1], x <- q_s * floor(x / 4096) + slot - cum[s]; if x < 2^16,
+ * x <- x * 2^16 + next word.  Returns 0 when the tile is consistent (every state back at 2^16 and
+ * every word used, up to the zero padding), 1 when it is not, -1 when the words ran out.
+ */
+static int decode_tile(const uint8_t* tile, uint64_t nbytes, int64_t nvec, const dtables* T,
+                       uint8_t* sym9, int16_t* raw8, uint32_t* final_states)
+{
+    if (nbytes < 4u * ORC_LANES) return -1;
+    uint32_t x[ORC_LANES];
+    for (int l = 0; l < ORC_LANES; l++) x[l] = get32(tile + 4 * l);
+    const uint8_t* words = tile + 4 * ORC_LANES;
+    uint64_t nwords = (nbytes - 4u * ORC_LANES) / 2u, pos = 0;
+    int64_t nsteps = (nvec + ORC_LANES - 1) / ORC_LANES;
+    for (int64_t k = 0; k < nsteps; k++) {
+        for (int u = 0; u <= 8; u++)
+            for (int l = 0; l < ORC_LANES; l++) {
+                int64_t v = k * ORC_LANES + l;
+                if (v >= nvec) continue;
+                int ctx = context_of(u, u == 0 ? 0 : sym9[v * 9]);
+                uint32_t slot = x[l] & (ORC_M - 1);
+                int s = T->slot_sym[ctx][slot];
+                uint32_t q = T->q17[256 * ctx + s];
+                x[l] = q * (x[l] >> 12) + slot - T->cum[ctx][s];
+                sym9[v * 9 + u] = (uint8_t)s;
+                if (x[l] < ORC_L) {
+                    if (pos >= nwords) return -1;
+                    x[l] = (x[l] << 16) | get16(words + 2 * pos++);
+                }
+            }
+        for (int j = 1; j <= 8; j++)
+            for (int l = 0; l < ORC_LANES; l++) {
+                int64_t v = k * ORC_LANES + l;
+                if (v < nvec && sym9[v * 9 + j] == ORC_ESC) {
+                    if (pos >= nwords) return -1;
+                    raw8[v * 8 + (j - 1)] = (int16_t)get16(words + 2 * pos++);
+                }
+            }
+    }
+    int bad = 0;
+    for (int l = 0; l < ORC_LANES; l++) {
+        if (final_states) final_states[l] = x[l];
+        if (x[l] != ORC_L) bad = 1;
+    }
+    if (nbytes - 4u * ORC_LANES - 2u * pos >= 16u) bad = 1;
+    return bad;
+}
+
+/* Decode one tile given the 17 x 256 frequency tables (exposed for the rANS checks). */
+int orc_decode_tile(const uint8_t* tile, uint64_t nbytes, int64_t nvec, const uint16_t* q17,
+                    uint8_t* sym9, int16_t* raw8, uint32_t* final_states)
+{
+    dtables* T = (dtables*)malloc(sizeof(dtables));
+    if (!T) return -2;
+    build_dtables(q17, T);
+    int rc = decode_tile(tile, nbytes, nvec, T, sym9, raw8, final_states);
+    free(T);
+    return rc;
+}
+
+/* ------------------------------------------------------------------------------------------ */
+/* The encoder: normalise, quantise, choose the scale, fit row scales, code ([DOC-LQ/RS/ER]).  */
+/* ------------------------------------------------------------------------------------------ */
+
+typedef struct {
+    int dtype;
+    int64_t rows, cols, cols_p, vpr;   /* vpr = vectors per row = cols_p / 8 */
+    double* w;                         /* rows x cols, exact values            */
+    double* rms;                       /* per-row root mean square             */
+} matrix;
+
+/* reading: columns are padded with zeros to a multiple of 8; the padding is quantised with the
+ * row but is excluded from the RMS and least-squares sums and never written back. */
+static double elem(const matrix* m, int64_t r, int64_t c) { return c < m->cols ? m->w[r * m->cols + c] : 0.0; }
+
+/* [DOC-LQ]: "normalizes each row by its root mean square". */
+static void row_rms(matrix* m)
+{
+    for (int64_t r = 0; r < m->rows; r++) {
+        double acc = 0.0;
+        for (int64_t c = 0; c < m->cols; c++) acc += m->w[r * m->cols + c] * m->w[r * m->cols + c];
+        m->rms[r] = sqrt(acc / (double)m->cols);
+    }
+}
+
+/*
+ * Quantise vector k of row r at shared scale s: t = clamp(x_hat / s, +-32764) with x_hat the
+ * RMS-normalised row, then the E8 nearest point ([DOC-LQ]: "groups the normalized values into
+ * eight-dimensional vectors ... nearest point on a scaled E8 lattice"; "a shared quantization
+ * scale controls the spacing").  An all-zero row (RMS 0) maps every vector to the origin.
+ */
+static void quantise_vector(const matrix* m, int64_t r, int64_t k, double s, double y[8], int* coset)
+{
+    double t[8];
+    for (int i = 0; i < 8; i++) {
+        double xh = m->rms[r] > 0.0 ? elem(m, r, 8 * k + i) / m->rms[r] : 0.0;
+        double v = xh / s;
+        if (v > ORC_CLAMP) v = ORC_CLAMP;
+        if (v < -ORC_CLAMP) v = -ORC_CLAMP;
+        t[i] = v;
+    }
+    orc_e8_nearest(t, y, coset);
+}
+
+/* The nine symbols of a quantised vector and the raw values of escaped fields. */
+static void vector_symbols(const double y[8], int coset, uint8_t sym[9], int16_t raw[8])
+{
+    int32_t f[8];
+    orc_point_to_fields(y, coset, f);
+    sym[0] = (uint8_t)coset;
+    for (int j = 0; j < 8; j++) {
+        sym[1 + j] = (uint8_t)field_symbol(f[j]);
+        raw[j] = (int16_t)f[j];
+    }
+}
+
+/* reading: S = clamp(next_pow2(ceil(128 / target)), 16, 1024) steps per tile, unless given. */
+static int64_t default_steps(double target)
+{
+    double want = ceil(128.0 / target);
+    int64_t s = 1;
+    while ((double)s < want) s *= 2;
+    if (s < 16) s = 16;
+    if (s > 1024) s = 1024;
+    return s;
+}
+
+/* Bytes of the serialised table section for the given 17 tables (unpadded). */
+static uint64_t table_section_bytes(const uint16_t* q17)
+{
+    uint64_t bytes = 4;                                   /* coset q0, q1 */
+    for (int ctx = 1; ctx < ORC_NCTX; ctx++) {
+        const uint16_t* q = q17 + 256 * ctx;
+        int lo = -1, hi = -1;
+        for (int s = 0; s < ORC_ESC; s++)
+            if (q[s]) { if (lo < 0) lo = s; hi = s; }
+        bytes += 4 + (lo < 0 ? 0 : 2u * (uint64_t)(hi - lo + 1));
+    }
+    return bytes;
+}
+
+/*
+ * Estimated blob size in bits per element at scale s from the sampled rows ([DOC-RS]: "For each
+ * candidate scale, it estimates the coded field size and the metadata needed for decoding").
+ * reading: n_s = min(rows, 256) rows at floor(i * rows / n_s); tables are quantised from the
+ * sample's counts; coded size = sum over contexts and symbols of n * -log2(q / 4096) bits plus
+ * 16 bits per escape, scaled by rows / n_s; metadata = exact header, table, row-scale and
+ * tile-offset bytes, plus 128 state bytes and 8 padding bytes per tile.
+ * With full_sample != 0 every row is used (n_s = rows).
+ */
+static double estimate_bpp(const matrix* m, double s, int64_t S, int full_sample)
+{
+    int64_t ns = full_sample ? m->rows : (m->rows < 256 ? m->rows : 256);
+    uint64_t* cnt = (uint64_t*)calloc(ORC_NCTX * 256, sizeof(uint64_t));
+    uint64_t nesc = 0;
+    for (int64_t i = 0; i < ns; i++) {
+        int64_t r = (int64_t)((i * m->rows) / ns);
+        for (int64_t k = 0; k < m->vpr; k++) {
+            double y[8];
+            int c;
+            uint8_t sym[9];
+            int16_t raw[8];
+            quantise_vector(m, r, k, s, y, &c);
+            vector_symbols(y, c, sym, raw);
+            for (int u = 0; u <= 8; u++) {
+                cnt[256 * context_of(u, c) + sym[u]]++;
+                if (u > 0 && sym[u] == ORC_ESC) nesc++;
+            }
+        }
+    }
+    uint16_t q17[ORC_NCTX * 256];
+    for (int ctx = 0; ctx < ORC_NCTX; ctx++) orc_quantize_table(cnt + 256 * ctx, q17 + 256 * ctx);
+    double bits = 0.0;
+    for (int ctx = 0; ctx < ORC_NCTX; ctx++)
+        for (int sy = 0; sy < 256; sy++)
+            if (cnt[256 * ctx + sy]) bits += (double)cnt[256 * ctx + sy] * -log2((double)q17[256 * ctx + sy] / 4096.0);
+    double payload = ((double)m->rows / (double)ns) * (bits / 8.0 + 2.0 * (double)nesc);
+    int64_t V = m->rows * m->vpr;
+    int64_t ntiles = (V + 32 * S - 1) / (32 * S);
+    double meta = (double)(ORC_HEADER + pad16(table_section_bytes(q17)) + pad16(4u * (uint64_t)m->rows) +
+                           pad16(4u * (uint64_t)(ntiles + 1))) +
+                  (double)ntiles * (128.0 + 8.0);
+    free(cnt);
+    return 8.0 * (meta + payload) / ((double)m->rows * (double)m->cols);
+}
+
+/*
+ * Choose the shared scale ([DOC-RS]: "searches for a quantization scale using sampled rows";
+ * [DOC-LQ]: finer spacing costs more bits).
+ * reading: the finest scale whose estimate meets the target, by 48 bisection steps on log2 s
+ * over [-24, 8]; if even 2^8 misses the target, 2^8 (the actual size is reported as it is,
+ * [DOC-ER]: "the achieved bitrate can differ from the requested target").
+ */
+static double choose_scale(const matrix* m, double target, int64_t S)
+{
+    double lo = -24.0, hi = 8.0;
+    if (estimate_bpp(m, exp2(hi), S, 0) > target) return exp2(hi);
+    if (estimate_bpp(m, exp2(lo), S, 0) <= target) return exp2(lo);
+    for (int it = 0; it < 48; it++) {
+        double mid = 0.5 * (lo + hi);
+        if (estimate_bpp(m, exp2(mid), S, 0) <= target) hi = mid;
+        else lo = mid;
+    }
+    return exp2(hi);
+}
+
+static int load_matrix(matrix* m, const void* data, int dtype, int64_t rows, int64_t cols)
+{
+    if (rows <= 0 || cols <= 0 || dtype_size(dtype) == 0) return -1;
+    m->dtype = dtype;
+    m->rows = rows;
+    m->cols = cols;
+    m->cols_p = (cols + 7) / 8 * 8;
+    m->vpr = m->cols_p / 8;
+    m->w = (double*)malloc((size_t)(rows * cols) * sizeof(double));
+    m->rms = (double*)malloc((size_t)rows * sizeof(double));
+    if (!m->w || !m->rms) return -2;
+    for (int64_t i = 0; i < rows * cols; i++) {
+        m->w[i] = orc_dtype_to_f64(load_bits(data, dtype, (uint64_t)i), dtype);
+        if (!isfinite(m->w[i])) return -3;
+    }
+    row_rms(m);
+    return 0;
+}
+
+static void free_matrix(matrix* m)
+{
+    free(m->w);
+    free(m->rms);
+}
+
+/* Estimated bits per element at a given scale (exposed for the size-estimate check). */
+double orc_estimate_bpp(const void* data, int dtype, int64_t rows, int64_t cols, double scale,
+                        int64_t S, int full_sample)
+{
+    matrix m;
+    memset(&m, 0, sizeof m);
+    if (load_matrix(&m, data, dtype, rows, cols)) { free_matrix(&m); return -1.0; }
+    double b = estimate_bpp(&m, scale, S, full_sample);
+    free_matrix(&m);
+    return b;
+}
+
+/*
+ * Compress a rows x cols matrix stored as dtype bits.  steps_per_tile = 0 selects the default S;
+ * scale_override > 0 skips the search.  On success *blob is a malloc'd byte string of *len bytes.
+ *
+ * Blob layout (little-endian, every section 16-byte aligned; [DOC-ER]: "the representation also
+ * stores the probability tables, row scales, and tile metadata"):
+ *   header (80 bytes): "EPK1", u16 version 1, u8 dtype, u8 R, u64 rows, u64 cols, u32 S,
+ *     u32 n_tiles, f64 s, u64 total bytes, u64 offsets of the table, row-scale, tile-offset
+ *     and stream sections;
+ *   tables: u16 q(coset 0), u16 q(coset 1); then for c = 0,1 and j = 1..8: u16 q(escape),
+ *     u8 lo, u8 n, u16 q[lo .. lo+n-1] (symbols 0..254);
+ *   row scales: f32 per row;
+ *   tile offsets: u32[n_tiles + 1], in 16-byte units from the stream section start;
+ *   stream: the tiles.
+ */
+int orc_compress(const void* data, int dtype, int64_t rows, int64_t cols, double target_bpp,
+                 int64_t steps_per_tile, double scale_override, uint8_t** blob, uint64_t* len)
+{
+    *blob = NULL;
+    *len = 0;
+    /* [DOC-0]: "finite target bitrates in [0.001, 11] bits per element" */
+    if (!(target_bpp >= 0.001 && target_bpp <= 11.0)) return -4;
+    matrix m;
+    memset(&m, 0, sizeof m);
+    int rc = load_matrix(&m, data, dtype, rows, cols);
+    if (rc) { free_matrix(&m); return rc; }
+    int64_t S = steps_per_tile > 0 ? steps_per_tile : default_steps(target_bpp);
+    double s = scale_override > 0 ? scale_override : choose_scale(&m, target_bpp, S);
+
+    /* Quantise the whole tensor at s; fit one least-squares scale per row ([DOC-RS]: "Once the
+     * scale is selected, the encoder quantizes the full tensor and fits a reconstruction scale
+     * for each row by least squares"): alpha_r = sum w y / sum y^2 over real columns, stored
+     * as fp32 (0 when sum y^2 = 0). */
+    int64_t V = rows * m.vpr;
+    uint8_t* sym9 = (uint8_t*)malloc((size_t)V * 9);
+    int16_t* raw8 = (int16_t*)malloc((size_t)V * 8 * sizeof(int16_t));
+    float* alpha = (float*)malloc((size_t)rows * sizeof(float));
+    uint64_t* cnt = (uint64_t*)calloc(ORC_NCTX * 256, sizeof(uint64_t));
+    for (int64_t r = 0; r < rows; r++) {
+        double swy = 0.0, syy = 0.0;
+        for (int64_t k = 0; k < m.vpr; k++) {
+            double y[8];
+            int c;
+            int64_t v = r * m.vpr + k;
+            quantise_vector(&m, r, k, s, y, &c);
+            vector_symbols(y, c, sym9 + 9 * v, raw8 + 8 * v);
+            for (int i = 0; i < 8; i++)
+                if (8 * k + i < cols) {
+                    swy += elem(&m, r, 8 * k + i) * y[i];
+                    syy += y[i] * y[i];
+                }
+            for (int u = 0; u <= 8; u++) cnt[256 * context_of(u, c) + sym9[9 * v + u]]++;
+        }
+        alpha[r] = syy > 0.0 ? (float)(swy / syy) : 0.0f;
+    }
+
+    /* Probability tables from the whole tensor ([DOC-LQ]: "the probability model conditions each
+     * coordinate field on the coset"). */
+    uint16_t q17[ORC_NCTX * 256];
+    for (int ctx = 0; ctx < ORC_NCTX; ctx++) orc_quantize_table(cnt + 256 * ctx, q17 + 256 * ctx);
+
+    /* Tiles. */
+    int64_t per_tile = 32 * S;
+    int64_t ntiles = (V + per_tile - 1) / per_tile;
+    uint64_t* tsize = (uint64_t*)malloc((size_t)(ntiles + 1) * sizeof(uint64_t));
+    uint64_t stream_bytes = 0;
+    for (int64_t t = 0; t < ntiles; t++) {
+        int64_t v0 = t * per_tile, nv = V - v0 < per_tile ? V - v0 : per_tile;
+        tsize[t] = orc_encode_tile(sym9 + 9 * v0, raw8 + 8 * v0, nv, q17, NULL, 0);
+        if (tsize[t] == 0) { rc = -5; goto done; }
+        stream_bytes += tsize[t];
+    }
+
+    /* Serialise. */
+    {
+        uint64_t tab_bytes = table_section_bytes(q17);
+        uint64_t off_tab = ORC_HEADER;
+        uint64_t off_alpha = off_tab + pad16(tab_bytes);
+        uint64_t off_offs = off_alpha + pad16(4u * (uint64_t)rows);
+        uint64_t off_stream = off_offs + pad16(4u * (uint64_t)(ntiles + 1));
+        uint64_t total = off_stream + stream_bytes;
+        uint8_t* b = (uint8_t*)calloc((size_t)total, 1);
+        if (!b) { rc = -2; goto done; }
+        memcpy(b, "EPK1", 4);
+        put16(b + 4, 1);
+        b[6] = (uint8_t)dtype;
+        b[7] = ORC_R;
+        put64(b + 8, (uint64_t)rows);
+        put64(b + 16, (uint64_t)cols);
+        put32(b + 24, (uint32_t)S);
+        put32(b + 28, (uint32_t)ntiles);
+        memcpy(b + 32, &s, 8);                                     /* f64, little-endian host */
+        put64(b + 40, total);
+        put64(b + 48, off_tab);
+        put64(b + 56, off_alpha);
+        put64(b + 64, off_offs);
+        put64(b + 72, off_stream);
+        uint8_t* p = b + off_tab;
+        put16(p, q17[0]);
+        put16(p + 2, q17[1]);
+        p += 4;
+        for (int ctx = 1; ctx < ORC_NCTX; ctx++) {
+            const uint16_t* q = q17 + 256 * ctx;
+            int lo = -1, hi = -1;
+            for (int sy = 0; sy < ORC_ESC; sy++)
+                if (q[sy]) { if (lo < 0) lo = sy; hi = sy; }
+            int n = lo < 0 ? 0 : hi - lo + 1;
+            put16(p, q[ORC_ESC]);
+            p[2] = (uint8_t)(lo < 0 ? 0 : lo);
+            p[3] = (uint8_t)n;
+            p += 4;
+            for (int i = 0; i < n; i++, p += 2) put16(p, q[lo + i]);
+        }
+        for (int64_t r = 0; r < rows; r++) {
+            uint32_t ab;
+            memcpy(&ab, &alpha[r], 4);
+            put32(b + off_alpha + 4 * r, ab);
+        }
+        uint64_t acc = 0;
+        for (int64_t t = 0; t <= ntiles; t++) {
+            put32(b + off_offs + 4 * t, (uint32_t)(acc / 16u));
+            if (t < ntiles) acc += tsize[t];
+        }
+        acc = 0;
+        for (int64_t t = 0; t < ntiles; t++) {
+            int64_t v0 = t * per_tile, nv = V - v0 < per_tile ? V - v0 : per_tile;
+            orc_encode_tile(sym9 + 9 * v0, raw8 + 8 * v0, nv, q17, b + off_stream + acc, tsize[t]);
+            acc += tsize[t];
+        }
+        *blob = b;
+        *len = total;
+    }
+done:
+    free(tsize);
+    free(sym9);
+    free(raw8);
+    free(alpha);
+    free(cnt);
+    free_matrix(&m);
+    return rc;
+}
+
+/* ------------------------------------------------------------------------------------------ */
+/* The decoder ([DOC-ER]: "Decoding recovers the fields, reconstructs lattice points, and       */
+/* applies the row scales ... The result has the input's shape and dtype").                    */
+/* ------------------------------------------------------------------------------------------ */
+
+typedef struct {
+    int dtype;
+    int64_t rows, cols, vpr, S, ntiles, V;
+    double s;
+    uint16_t q17[ORC_NCTX * 256];
+    const uint8_t* alpha;
+    const uint8_t* offs;
+    const uint8_t* stream;
+    uint64_t stream_bytes;
+} parsed;
+
+static int parse_blob(const uint8_t* b, uint64_t len, parsed* P)
+{
+    if (len < ORC_HEADER || memcmp(b, "EPK1", 4) != 0 || get16(b + 4) != 1 || b[7] != ORC_R) return -6;
+    P->dtype = b[6];
+    P->rows = (int64_t)get64(b + 8);
+    P->cols = (int64_t)get64(b + 16);
+    P->S = get32(b + 24);
+    P->ntiles = get32(b + 28);
+    memcpy(&P->s, b + 32, 8);
+    uint64_t total = get64(b + 40), off_tab = get64(b + 48), off_alpha = get64(b + 56);
+    uint64_t off_offs = get64(b + 64), off_stream = get64(b + 72);
+    if (total != len || P->rows <= 0 || P->cols <= 0 || P->S <= 0 || dtype_size(P->dtype) == 0) return -6;
+    P->vpr = (P->cols + 7) / 8;
+    P->V = P->rows * P->vpr;
+    if (P->ntiles != (P->V + 32 * P->S - 1) / (32 * P->S)) return -6;
+    if (off_tab < ORC_HEADER || off_tab + 4 > off_alpha || off_alpha + 4u * (uint64_t)P->rows > off_offs ||
+        off_offs + 4u * (uint64_t)(P->ntiles + 1) > off_stream || off_stream > len)
+        return -6;
+    memset(P->q17, 0, sizeof P->q17);
+    const uint8_t* p = b + off_tab;
+    P->q17[0] = (uint16_t)get16(p);
+    P->q17[1] = (uint16_t)get16(p + 2);
+    p += 4;
+    for (int ctx = 1; ctx < ORC_NCTX; ctx++) {
+        if ((uint64_t)(p + 4 - b) > off_alpha) return -6;
+        uint16_t* q = P->q17 + 256 * ctx;
+        q[ORC_ESC] = (uint16_t)get16(p);
+        int lo = p[2], n = p[3];
+        p += 4;
+        if (lo + n > ORC_ESC || (uint64_t)(p + 2 * n - b) > off_alpha) return -6;
+        for (int i = 0; i < n; i++, p += 2) q[lo + i] = (uint16_t)get16(p);
+    }
+    for (int ctx = 0; ctx < ORC_NCTX; ctx++) {
+        uint32_t sum = 0;
+        for (int sy = 0; sy < 256; sy++) sum += P->q17[256 * ctx + sy];
+        if (sum != 0 && sum != ORC_M) return -6;
+    }
+    P->alpha = b + off_alpha;
+    P->offs = b + off_offs;
+    P->stream = b + off_stream;
+    P->stream_bytes = len - off_stream;
+    if (get32(P->offs) != 0 || 16u * (uint64_t)get32(P->offs + 4 * P->ntiles) != P->stream_bytes) return -6;
+    return 0;
+}
+
+/* Decode tiles [t0, t1) to symbols.  Returns 0, or a negative code / 1 for an inconsistent tile. */
+static int decode_tiles_to_symbols(const parsed* P, int64_t t0, int64_t t1, uint8_t* sym9, int16_t* raw8)
+{
+    int64_t per_tile = 32 * P->S;
+    dtables* T = (dtables*)malloc(sizeof(dtables));
+    if (!T) return -2;
+    build_dtables(P->q17, T);
+    int out = 0;
+    for (int64_t t = t0; t < t1; t++) {
+        uint64_t a = 16u * (uint64_t)get32(P->offs + 4 * t), e = 16u * (uint64_t)get32(P->offs + 4 * (t + 1));
+        if (e < a || e > P->stream_bytes) { out = -6; break; }
+        int64_t v0 = t * per_tile, nv = P->V - v0 < per_tile ? P->V - v0 : per_tile;
+        int rc = decode_tile(P->stream + a, e - a, nv, T, sym9 + 9 * v0, raw8 + 8 * v0, NULL);
+        if (rc) { out = rc < 0 ? -7 : -8; break; }
+    }
+    free(T);
+    return out;
+}
+
+/* Field values of the vectors of tiles [t0, t1): fields[v*9] = coset, fields[v*9 + j] = f_j.
+ * The array is indexed by global vector number and has room for all V vectors. */
+int orc_decode_fields(const uint8_t* blob, uint64_t len, int64_t t0, int64_t t1, int16_t* fields)
+{
+    parsed P;
+    int rc = parse_blob(blob, len, &P);
+    if (rc) return rc;
+    if (t1 < 0 || t1 > P.ntiles) t1 = P.ntiles;
+    if (t0 < 0 || t0 > t1) return -1;
+    uint8_t* sym9 = (uint8_t*)calloc((size_t)P.V * 9, 1);
+    int16_t* raw8 = (int16_t*)calloc((size_t)P.V * 8, sizeof(int16_t));
+    rc = decode_tiles_to_symbols(&P, t0, t1, sym9, raw8);
+    if (rc == 0) {
+        int64_t v0 = t0 * 32 * P.S, v1 = t1 * 32 * P.S < P.V ? t1 * 32 * P.S : P.V;
+        for (int64_t v = v0; v < v1; v++) {
+            fields[9 * v] = sym9[9 * v];
+            for (int j = 1; j <= 8; j++) {
+                int sy = sym9[9 * v + j];
+                fields[9 * v + j] = (int16_t)(sy == ORC_ESC ? raw8[8 * v + j - 1] : sy - ORC_R);
+            }
+        }
+    }
+    free(sym9);
+    free(raw8);
+    return rc;
+}
+
+/*
+ * Decode tiles [t0, t1) (all tiles when t1 < 0) into out, a contiguous rows x cols array of
+ * dtype_out; elements of other tiles are left untouched.  Each element is the fp32 product of
+ * the row's fp32 scale and the lattice coordinate (exact in fp32), rounded to nearest-even, then
+ * rounded to the container (RNE; E4M3 saturates to +-448).
+ */
+int orc_decompress_tiles(const uint8_t* blob, uint64_t len, int64_t t0, int64_t t1, int dtype_out, void* out)
+{
+    parsed P;
+    int rc = parse_blob(blob, len, &P);
+    if (rc) return rc;
+    if (dtype_size(dtype_out) == 0) return -1;
+    if (t1 < 0 || t1 > P.ntiles) t1 = P.ntiles;
+    if (t0 < 0 || t0 > t1) return -1;
+    uint8_t* sym9 = (uint8_t*)calloc((size_t)P.V * 9, 1);
+    int16_t* raw8 = (int16_t*)calloc((size_t)P.V * 8, sizeof(int16_t));
+    rc = decode_tiles_to_symbols(&P, t0, t1, sym9, raw8);
+    if (rc == 0) {
+        int64_t v0 = t0 * 32 * P.S, v1 = t1 * 32 * P.S < P.V ? t1 * 32 * P.S : P.V;
+        for (int64_t v = v0; v < v1; v++) {
+            int64_t r = v / P.vpr, k = v % P.vpr;
+            int32_t f[8];
+            double y[8];
+            int c = sym9[9 * v];
+            for (int j = 1; j <= 8; j++) {
+                int sy = sym9[9 * v + j];
+                f[j - 1] = sy == ORC_ESC ? raw8[8 * v + j - 1] : sy - ORC_R;
+            }
+            orc_fields_to_point(c, f, y);
+            float a;
+            uint32_t ab = get32(P.alpha + 4 * r);
+            memcpy(&a, &ab, 4);
+            for (int i = 0; i < 8; i++) {
+                int64_t col = 8 * k + i;
+                if (col >= P.cols) continue;
+                store_value(out, (uint64_t)(r * P.cols + col), dtype_out, (double)a * y[i]);
+            }
+        }
+    }
+    free(sym9);
+    free(raw8);
+    return rc;
+}
+
+/* Decode the whole blob into a contiguous rows x cols array of dtype_out. */
+int orc_decompress(const uint8_t* blob, uint64_t len, int dtype_out, void* out)
+{
+    return orc_decompress_tiles(blob, len, 0, -1, dtype_out, out);
+}
+
+/* [DOC-ER]: "The actual_bpp property reports the actual stored bytes, including metadata,
+ * divided by the element count and multiplied by eight." */
+double orc_actual_bpp(const uint8_t* blob, uint64_t len)
+{
+    parsed P;
+    if (parse_blob(blob, len, &P)) return -1.0;
+    return 8.0 * (double)len / ((double)P.rows * (double)P.cols);
+}
+
+/* Header fields, for tests: rows, cols, S, n_tiles, dtype, and the shared scale. */
+int orc_blob_info(const uint8_t* blob, uint64_t len, int64_t* info5, double* scale)
+{
+    parsed P;
+    int rc = parse_blob(blob, len, &P);
+    if (rc) return rc;
+    info5[0] = P.rows;
+    info5[1] = P.cols;
+    info5[2] = P.S;
+    info5[3] = P.ntiles;
+    info5[4] = P.dtype;
+    *scale = P.s;
+    return 0;
+}
+
+void orc_free(void* p) { free(p); }
+
+/* ------------------------------------------------------------------------------------------ */
+/* Array forms of the per-vector functions, for the checks (one call per array).              */
+/* ------------------------------------------------------------------------------------------ */
+
+void orc_e8_nearest_n(const double* t, int64_t n, double* y, int32_t* coset)
+{
+    for (int64_t i = 0; i < n; i++) {
+        int c;
+        orc_e8_nearest(t + 8 * i, y + 8 * i, &c);
+        coset[i] = c;
+    }
+}
+
+void orc_point_to_fields_n(const double* y, const int32_t* coset, int64_t n, int32_t* f)
+{
+    for (int64_t i = 0; i < n; i++) orc_point_to_fields(y + 8 * i, coset[i], f + 8 * i);
+}
+
+void orc_fields_to_point_n(const int32_t* coset, const int32_t* f, int64_t n, double* y)
+{
+    for (int64_t i = 0; i < n; i++) orc_fields_to_point(coset[i], f + 8 * i, y + 8 * i);
+}
+
+void orc_dtype_to_f64_n(const void* data, int dtype, int64_t n, double* out)
+{
+    for (int64_t i = 0; i < n; i++) out[i] = orc_dtype_to_f64(load_bits(data, dtype, (uint64_t)i), dtype);
+}
+
+/* fp32 rounding of exact products a[i] * b[i] (double), returned as fp32 bit patterns. */
+void orc_round_f32_n(const double* v, int64_t n, uint32_t* out)
+{
+    for (int64_t i = 0; i < n; i++) out[i] = orc_round_f32(v[i]);
+}
