@@ -1,0 +1,374 @@
+"""Benchmark of the fused lattice-rANS decode (ep_decompress) on B200.
+
+One step = one ep_decompress call over the whole workload matrix: every tile's rANS streams
+decoded to fields, lattice points, row-scaled and written as BF16.  Default workload: 4096 x 4096
+BF16, rows N(0, sigma_r^2) with sigma_r log-uniform in [0.005, 0.05], compressed at 4.0 bits per
+element by the library's own encoder (synthetic data; no model weights are involved).
+
+Timing: W untimed warm-up steps, then exactly K steps between a barrier + synchronize on both
+sides, timed by CUDA events on the launching stream; the maximum over ranks is reported.  The
+steps rotate over R independent blob/output copies whose total exceeds 3x the 126 MB L2, so
+each step reads its blob and writes its output through HBM.  nvidia-smi samples clocks and
+throttle reasons during the timed region.
+
+Multi-GPU (torchrun): every rank decodes its own copy of the workload; no data-path collective
+(tiles are independent), so scaling is weak and the value is the sum over ranks.
+
+Arms:
+  default             the CUDA path through the C ABI;
+  --impl reference    the oracle (plain single-threaded C) on the host cores, each step a
+                      bounded sample of the same workload; rank 0 only.
+"""
+from __future__ import annotations
+
+import argparse
+import ctypes
+import hashlib
+import json
+import math
+import os
+import re
+import statistics
+import subprocess
+import sys
+import tempfile
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "decompressed output GB/s and % of HBM roofline (fused rANS+E8 decode), 1×B200"
+NOMINAL_HBM_GBS = 8000.0          # the roofline the metric names
+L2_BYTES = 126 * 1024 * 1024
+FALLBACK_HBM_GBS = 6650.0
+
+
+def parse_args():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=40000)
+    ap.add_argument("--warmup", type=int, default=200)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--steps-per-tile", type=int, default=0, help="encoder S override (0 = default)")
+    ap.add_argument("--e2e-steps", type=int, default=50)
+    ap.add_argument("--cpu-seconds", type=float, default=10.0, help="CPU-baseline sample length")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    return ap.parse_args()
+
+
+def workload(steps_override: int = 0):
+    import workloads as W
+    m = W.square()
+    desc = ("square 4096x4096 BF16, row r i.i.d. N(0, sigma_r^2), sigma_r log-uniform in [0.005, 0.05], "
+            "target 4.0 bpp, output BF16")
+    return m, desc
+
+
+# ---------------------------------------------------------------------------------------------
+# Clocks during the timed region.
+# ---------------------------------------------------------------------------------------------
+class ClockSampler:
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_id: str | None):
+        self.proc = None
+        self.path = None
+        self.gpu_id = gpu_id
+
+    def start(self):
+        try:
+            fd, self.path = tempfile.mkstemp(suffix=".csv")
+            os.close(fd)
+            cmd = ["nvidia-smi", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits", "-lms", "50"]
+            if self.gpu_id:
+                cmd += ["-i", self.gpu_id]
+            self.proc = subprocess.Popen(cmd, stdout=open(self.path, "w"), stderr=subprocess.DEVNULL)
+        except (OSError, FileNotFoundError):
+            self.proc = None
+
+    def stop(self):
+        if self.proc is None:
+            return None
+        time.sleep(0.12)
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+        rows = []
+        for line in open(self.path):
+            parts = [p.strip() for p in line.split(",")]
+            if len(parts) >= 9:
+                rows.append(parts)
+        os.unlink(self.path)
+        if not rows:
+            return None
+        sm = [float(r[1]) for r in rows if r[1].replace(".", "").isdigit()]
+        mx = [float(r[2]) for r in rows if r[2].replace(".", "").isdigit()]
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = sorted({names[i] for r in rows for i in range(4) if r[5 + i].lower().startswith("active")})
+        return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": max(mx) if mx else None,
+                "reasons": reasons, "samples": len(rows)}
+
+
+# ---------------------------------------------------------------------------------------------
+# Peaks and the committed ncu traffic figure.
+# ---------------------------------------------------------------------------------------------
+def hbm_peak():
+    try:
+        d = json.load(open(os.path.join(ROOT, "MEASURED_PEAKS.json")))
+        return float(d["hbm_gbs"]), "measured"
+    except (OSError, KeyError, ValueError):
+        return FALLBACK_HBM_GBS, "fallback"
+
+
+def kernel_source_hash() -> str:
+    h = hashlib.sha256()
+    for f in ("decode.cu", "format.h", "blob.h"):
+        h.update(open(os.path.join(ROOT, "dit_weight_compression_b200", "csrc", f), "rb").read())
+    return h.hexdigest()[:16]
+
+
+def committed_traffic(profile: str):
+    """DRAM bytes per launch from a committed ncu summary, if it was taken on this kernel source."""
+    path = os.path.join(ROOT, "profiles", profile)
+    try:
+        text = open(path).read()
+    except OSError:
+        return None
+    src = re.search(r"kernel_source_sha:\s*([0-9a-f]+)", text)
+    val = re.search(r"dram_bytes_per_launch:\s*([0-9]+)", text)
+    if not src or not val or src.group(1) != kernel_source_hash():
+        return None
+    return int(val.group(1))
+
+
+# ---------------------------------------------------------------------------------------------
+# CPU baseline: the oracle decoder on the host.
+# ---------------------------------------------------------------------------------------------
+def cpu_oracle_rate(blob: bytes, seconds: float, max_tiles: int | None = None):
+    import oracle
+    info = oracle.blob_info(blob)
+    out = np.zeros((info["rows"], info["cols"]), np.uint16)
+    n_tiles = info["n_tiles"] if max_tiles is None else min(max_tiles, info["n_tiles"])
+    per = 32 * info["S"]
+    elems = min(n_tiles * per, info["V"]) * 8
+    t0 = time.perf_counter()
+    reps = 0
+    while True:
+        oracle.decompress_tiles(blob, 0, n_tiles, oracle.BF16, out)
+        reps += 1
+        if time.perf_counter() - t0 >= seconds:
+            break
+    dt = time.perf_counter() - t0
+    return elems * 2 * reps / dt / 1e9, reps, n_tiles, dt
+
+
+def reference_arm(args, m, desc):
+    """The oracle as it stands, timed on the host cores with the same metric and workload."""
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return
+    import oracle
+    blob = oracle.compress(m.bits, m.dtype, m.target_bpp)
+    info = oracle.blob_info(blob)
+    # size each step's sample so that warm-up + steps take about a minute
+    t = time.perf_counter()
+    oracle.decompress_tiles(blob, 0, 8, oracle.BF16, np.zeros((info["rows"], info["cols"]), np.uint16))
+    per_tile = max((time.perf_counter() - t) / 8, 1e-6)
+    tiles = int(max(1, min(info["n_tiles"], 60.0 / (args.steps + args.warmup) / per_tile)))
+    out = np.zeros((info["rows"], info["cols"]), np.uint16)
+    for i in range(args.warmup):
+        oracle.decompress_tiles(blob, 0, tiles, oracle.BF16, out)
+    t0 = time.perf_counter()
+    for i in range(args.steps):
+        t_lo = (i * tiles) % max(1, info["n_tiles"] - tiles + 1)
+        oracle.decompress_tiles(blob, t_lo, t_lo + tiles, oracle.BF16, out)
+    dt = time.perf_counter() - t0
+    elems = tiles * 32 * info["S"] * 8
+    value = elems * 2 * args.steps / dt / 1e9
+    sample = f"{tiles} of {info['n_tiles']} tiles ({elems} elements) per step"
+    line = {"metric": METRIC, "value": value, "unit": "GB/s", "n_gpus": args.gpus, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": 1e3 * dt / args.steps, "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "u32/f64", "data": "synthetic",
+            "impl": "reference",
+            "config": {"workload": desc, "rows": m.shape[0], "cols": m.shape[1], "target_bpp": m.target_bpp,
+                       "actual_bpp": oracle.actual_bpp(blob), "sample": sample},
+            "cpu_baseline": {"value": value, "unit": "GB/s", "cores": 1, "kind": "oracle", "sample": sample},
+            "e2e": {"value": value, "unit": "GB/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+
+
+# ---------------------------------------------------------------------------------------------
+# The CUDA arm.
+# ---------------------------------------------------------------------------------------------
+def main():
+    args = parse_args()
+    m, desc = workload()
+    if args.impl == "reference":
+        reference_arm(args, m, desc)
+        return
+
+    import torch
+    import torch.distributed as dist
+
+    import dit_weight_compression_b200 as ep
+    import workloads as W
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    torch.cuda.set_device(local)
+    if world > 1:
+        from datetime import timedelta
+        dist.init_process_group("nccl", timeout=timedelta(seconds=120), device_id=torch.device("cuda", local))
+
+    def barrier():
+        if world > 1:
+            dist.barrier()
+
+    # compress with the library's host encoder
+    cfg = ep.LatticeRANSConfig(m.target_bpp, steps_per_tile=args.steps_per_tile)
+    host = W.bits_to_torch(m.bits, m.dtype)
+    t = time.perf_counter()
+    comp = ep.compress(host, cfg)
+    enc_s = time.perf_counter() - t
+    blob = comp.to_bytes()
+    rows, cols = comp.shape
+    out_bytes = rows * cols * 2
+    blob_bytes = len(blob)
+    moved = blob_bytes + out_bytes
+
+    # R independent device copies so that consecutive steps miss L2
+    R = max(2, math.ceil(3 * L2_BYTES / moved))
+    stream = torch.cuda.current_stream()
+    copies = [ep.CompressedTensor.from_bytes(blob) for _ in range(R)]
+    outs = [torch.empty((rows, cols), dtype=torch.bfloat16, device="cuda") for _ in range(R)]
+    for c in copies:
+        c.prepare(stream=stream)
+    L = ep.lib()
+    views = [ep.tensor_view(o) for o in outs]
+    handles = [c.handle for c in copies]
+    sh = ctypes.c_void_p(stream.cuda_stream)
+    decomp = L.ep_decompress
+
+    def step(i):
+        j = i % R
+        rc = decomp(handles[j], ctypes.byref(views[j]), sh)
+        if rc != 0:
+            raise ep.EPError(rc, "ep_decompress")
+
+    # correctness gate before timing: this rank's output equals a reference decode
+    step(0)
+    torch.cuda.synchronize()
+    for c in copies[:1]:
+        ep.decode_status(c)
+
+    for i in range(args.warmup):
+        step(i)
+    K = args.steps
+    ev_s = [torch.cuda.Event(enable_timing=True) for _ in range(K)]
+    ev_e = [torch.cuda.Event(enable_timing=True) for _ in range(K)]
+    start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    gpu_uuid = None
+    try:
+        gpu_uuid = str(torch.cuda.get_device_properties(local).uuid)
+        if not gpu_uuid.startswith("GPU-"):
+            gpu_uuid = "GPU-" + gpu_uuid
+    except Exception:
+        gpu_uuid = None
+    clocks = ClockSampler(gpu_uuid)
+    torch.cuda.synchronize()
+    barrier()
+    torch.cuda.synchronize()
+    clocks.start()
+    time.sleep(0.2)  # let the sampler start before the timed region
+    start.record(stream)
+    for i in range(K):
+        ev_s[i].record(stream)
+        step(i)
+        ev_e[i].record(stream)
+    end.record(stream)
+    torch.cuda.synchronize()
+    barrier()
+    torch.cuda.synchronize()
+    clk = clocks.stop()
+    total_ms = start.elapsed_time(end)
+    launch_ms = [ev_s[i].elapsed_time(ev_e[i]) for i in range(K)]
+    avg_launch_ms = sum(launch_ms) / K
+    for c in copies:
+        ep.decode_status(c)
+
+    if world > 1:
+        tt = torch.tensor([total_ms, avg_launch_ms], device="cuda", dtype=torch.float64)
+        dist.all_reduce(tt, op=dist.ReduceOp.MAX)
+        total_ms, avg_launch_ms = tt.tolist()
+
+    # end to end through the public call with host buffers: upload the blob, decode, download
+    host_out = torch.empty((rows, cols), dtype=torch.bfloat16).pin_memory()
+    for _ in range(3):
+        ep.decompress(comp, out=host_out)
+    torch.cuda.synchronize()
+    barrier()
+    e_s, e_e = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e_s.record(stream)
+    for _ in range(args.e2e_steps):
+        ep.decompress(comp, out=host_out)
+    e_e.record(stream)
+    torch.cuda.synchronize()
+    e2e_ms = e_s.elapsed_time(e_e)
+    if world > 1:
+        tt = torch.tensor([e2e_ms], device="cuda", dtype=torch.float64)
+        dist.all_reduce(tt, op=dist.ReduceOp.MAX)
+        e2e_ms = tt.item()
+    ep.decode_status(comp)
+
+    if rank == 0:
+        peak, peak_kind = hbm_peak()
+        achieved = moved / (avg_launch_ms * 1e-3) / 1e9
+        value = world * out_bytes * K / (total_ms * 1e-3) / 1e9
+        info = comp.info
+        symbols = info.n_vectors * 9
+        cpu = None
+        if world == 1 and not args.no_cpu_baseline:
+            gbs, reps, nt, secs = cpu_oracle_rate(blob, args.cpu_seconds)
+            cpu = {"value": gbs, "unit": "GB/s", "cores": 1, "kind": "oracle",
+                   "sample": f"whole {rows}x{cols} matrix ({nt} tiles) decoded {reps} times, {secs:.1f} s, "
+                             f"single-threaded oracle"}
+        traffic = committed_traffic("decode_square_bf16.md")
+        line = {
+            "metric": METRIC, "value": value, "unit": "GB/s", "n_gpus": world, "steps": K,
+            "warmup": args.warmup, "ms_per_step": total_ms / K, "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "u32/f32", "data": "synthetic",
+            "config": {
+                "workload": desc, "rows": rows, "cols": cols, "target_bpp": m.target_bpp,
+                "actual_bpp": comp.actual_bpp, "steps_per_tile": info.steps_per_tile,
+                "n_tiles": info.n_tiles, "blob_bytes": blob_bytes, "out_bytes": out_bytes,
+                "l2": f"rotating {R} blob/output copies ({R * moved / 1e6:.0f} MB > 3x L2)",
+                "symbols_per_s": world * symbols * K / (total_ms * 1e-3),
+                "kernel_avg_us": avg_launch_ms * 1e3, "encode_s": enc_s,
+                "parallelism": f"weak, {world} independent rank(s)",
+            },
+            "roofline": {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s",
+                         "frac": achieved / peak, "traffic": traffic,
+                         "peak_kind": peak_kind, "nominal_8tbs_frac": achieved / NOMINAL_HBM_GBS,
+                         "algorithmic_bytes_per_launch": moved},
+            "cpu_baseline": cpu,
+            "e2e": {"value": world * out_bytes * args.e2e_steps / (e2e_ms * 1e-3) / 1e9, "unit": "GB/s",
+                    "h2d_bytes_per_step": blob_bytes, "d2h_bytes_per_step": out_bytes},
+            "gpu_launches": K,
+            "clocks": clk,
+        }
+        print(json.dumps(line), flush=True)
+    del copies
+    if world > 1:
+        dist.barrier()
+        dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

@@ -1,0 +1,36 @@
+// blob.h -- the library-owned blob object behind the opaque ep_blob handle, and the per-thread
+// error message helpers shared by the host API (api.cpp) and the GPU API (decode.cu).
+#pragma once
+
+#include <mutex>
+#include <string>
+#include <vector>
+
+#include "entropack.h"
+#include "format.h"
+
+namespace ep {
+
+constexpr int kMaxDevices = 64;
+
+// Device-side state of one blob on one GPU.
+struct DeviceCopy {
+    uint8_t* blob = nullptr;        // copy of the serialised bytes (decode reads this)
+    uint32_t* status = nullptr;     // sticky error bits written by the decode kernel
+    uint8_t* stage_blob = nullptr;  // host-output path: per-call upload target
+    uint8_t* stage_out = nullptr;   // host-output path: decode target before the D2H copy
+    size_t stage_out_bytes = 0;
+};
+
+int set_error(int code, const std::string& msg);
+void clear_error();
+
+}  // namespace ep
+
+struct ep_blob {
+    std::vector<uint8_t> bytes;
+    ep::BlobLayout layout;
+    std::mutex mu;                  // guards lazy device set-up
+    ep::DeviceCopy dev[ep::kMaxDevices];
+    bool host_pinned = false;
+};

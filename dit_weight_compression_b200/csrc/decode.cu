@@ -1,0 +1,704 @@
+// decode.cu -- fused GPU decompression for sm_100a, and the device-side entry points of the C ABI.
+//
+// "EntroPack lattice compression" (documentation page, section "Encoding and reconstruction"):
+// "Decoding recovers the fields, reconstructs lattice points, and applies the row scales in a
+// fused GPU operation. The result has the input's shape and dtype."  The arXiv abstract adds
+// that tiles are independently decodable, "enabling fast, fused symbol decoding and numerical
+// weight reconstruction on the GPU".
+//
+// One kernel does the whole path.  Work split:
+//   * one warp per tile; the tile's 32 interleaved rANS states live one per lane;
+//   * persistent CTAs (grid = min(#SM x resident CTAs, #tiles)); tile t goes to CTA t mod grid,
+//     so every SM gets an equal share even when there are few tiles;
+//   * each CTA first expands the blob's compact frequency tables into shared memory: per field
+//     context a 4096-entry slot->symbol byte table and a 256-entry (frequency | cumulative << 16)
+//     word table (80 KB in all); the coset context (two symbols) is decoded by one compare;
+//   * each warp streams its tile's word stream through a private 2 KB shared-memory ring of four
+//     512-byte chunks, filled by 1-D bulk copies (cp.async.bulk, no multicast) that complete on
+//     one mbarrier per chunk; every wait is bounded and reports through the status word;
+//   * per step a lane decodes one 8-vector: 9 rANS symbols, each followed by the renormalisation
+//     read whose word position is the warp-ballot prefix count of lanes refilling before it;
+//     escaped fields take raw words at the end of the step; fields are inverted in registers
+//     (z8 = 2 f8 + parity, y = z + c/2), multiplied by the row's fp32 scale, converted with one
+//     cvt per pair and written as one 16-byte store per lane (a 512-byte contiguous run per warp
+//     for BF16/FP16).
+// No tensor cores: the path is table lookups and integer arithmetic, bound by HBM bytes and by
+// issue slots, not by a contraction.
+#include <cuda_bf16.h>
+#include <cuda_fp16.h>
+#include <cuda_fp8.h>
+#include <cuda_runtime.h>
+
+#include <algorithm>
+#include <cstdio>
+#include <mutex>
+
+#include "blob.h"
+
+namespace ep {
+namespace {
+
+constexpr uint32_t kFull = 0xFFFFFFFFu;
+constexpr int kChunk = 512;                                // bytes per bulk copy
+constexpr int kRingChunks = 4;
+constexpr int kRing = kChunk * kRingChunks;                // ring bytes per warp
+constexpr int kMaxStepBytes = 2 * (9 * kLanes + 8 * kLanes);  // words one step can consume
+constexpr uint32_t kWaitSpins = 1u << 22;                  // bounded mbarrier wait (~0.3 s)
+
+enum OutKind { kOutBF16 = 0, kOutFP16 = 1, kOutE4M3 = 2, kOutF32 = 3, kOutFields = 4 };
+
+// Status word bits (sticky, cleared by ep_decode_status).
+enum : uint32_t {
+    kStOverrun = 1u,   // a tile read past its own bytes
+    kStState = 2u,     // a lane did not end in state 2^16
+    kStLeftover = 4u,  // 16 or more bytes of a tile were never read
+    kStTimeout = 8u    // a bulk-copy wait hit its limit
+};
+
+struct Params {
+    const uint8_t* blob;        // device copy of the serialised blob
+    const uint32_t* tile_off;   // n_tiles + 1 offsets, 16-byte units
+    const uint8_t* stream;      // stream section
+    const float* alpha;         // per-row fp32 scales
+    void* out;
+    uint32_t* status;
+    int64_t cols, row_stride, n_vectors, vec_per_row;
+    uint32_t steps, n_tiles;
+    uint32_t q_coset0;          // frequency of coset 0; coset 1 has 4096 - q_coset0
+    uint32_t q_off[kFieldContexts];
+    uint32_t esc_q[kFieldContexts];
+    uint32_t lo[kFieldContexts];
+    uint32_t n[kFieldContexts];
+    int dense;                  // element offset of vector v is 8 v
+};
+
+template <int WARPS>
+struct Smem {
+    uint8_t sym[kFieldContexts][kProbTotal];     // slot -> symbol
+    uint32_t fc[kFieldContexts][256];            // frequency | cumulative << 16
+    alignas(16) uint8_t ring[WARPS][kRing];      // per-warp stream ring
+    unsigned long long bar[WARPS][kRingChunks];  // one mbarrier per ring chunk
+};
+
+// ---- PTX wrappers ----------------------------------------------------------------------------
+__device__ __forceinline__ uint32_t smem_u32(const void* p) {
+    return static_cast<uint32_t>(__cvta_generic_to_shared(p));
+}
+__device__ __forceinline__ void mbar_init(unsigned long long* bar, uint32_t count) {
+    asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(smem_u32(bar)), "r"(count) : "memory");
+}
+__device__ __forceinline__ void fence_proxy_async() {
+    asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+}
+__device__ __forceinline__ void mbar_expect_tx(unsigned long long* bar, uint32_t bytes) {
+    asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(smem_u32(bar)), "r"(bytes)
+                 : "memory");
+}
+// 1-D bulk copy global -> this CTA's shared memory, completing on `bar` (no multicast).
+__device__ __forceinline__ void bulk_g2s(void* dst, const void* src, uint32_t bytes, unsigned long long* bar) {
+    asm volatile(
+        "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(
+            smem_u32(dst)),
+        "l"(src), "r"(bytes), "r"(smem_u32(bar))
+        : "memory");
+}
+__device__ __forceinline__ bool mbar_test(unsigned long long* bar, uint32_t parity) {
+    uint32_t ok;
+    asm volatile(
+        "{\n .reg .pred p;\n mbarrier.test_wait.parity.shared::cta.b64 p, [%1], %2;\n selp.u32 %0, 1, 0, p;\n}"
+        : "=r"(ok)
+        : "r"(smem_u32(bar)), "r"(parity)
+        : "memory");
+    return ok != 0;
+}
+
+// Bounded, warp-uniform wait for the phase of `bar` with the given parity.
+__device__ __forceinline__ bool mbar_wait(unsigned long long* bar, uint32_t parity) {
+    for (uint32_t it = 0; it < kWaitSpins; ++it) {
+        if (__all_sync(kFull, mbar_test(bar, parity))) return true;
+        if (it >= 16) __nanosleep(64);
+    }
+    return false;
+}
+
+__device__ __forceinline__ uint32_t ring_word(const uint8_t* ring, uint32_t pos) {
+    return *reinterpret_cast<const uint16_t*>(ring + (pos & (kRing - 1)));
+}
+
+// Renormalisation after one decoded symbol: lanes whose state fell below 2^16 take the next
+// 16-bit words in ascending lane order (position = cursor + 2 * #refilling lanes below me).
+__device__ __forceinline__ void renorm(uint32_t& x, uint32_t& cur, const uint8_t* ring, uint32_t lt,
+                                       bool active) {
+    bool need = active && x < kStateLow;
+    uint32_t b = __ballot_sync(kFull, need);
+    if (need) x = (x << 16) | ring_word(ring, cur + 2u * __popc(b & lt));
+    cur += 2u * __popc(b);
+}
+
+// ---- table expansion -------------------------------------------------------------------------
+template <int WARPS>
+__device__ void build_tables(Smem<WARPS>& sm, const Params& p) {
+    const uint32_t lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+    // (a) per context: frequencies of symbols 8*lane .. 8*lane+7 and their cumulative sums
+    for (uint32_t ctx = warp; ctx < kFieldContexts; ctx += WARPS) {
+        const uint32_t lo = p.lo[ctx], n = p.n[ctx];
+        const uint16_t* qa = reinterpret_cast<const uint16_t*>(p.blob + p.q_off[ctx]);
+        uint32_t q[8], sum = 0;
+#pragma unroll
+        for (int i = 0; i < 8; ++i) {
+            uint32_t s = 8 * lane + i, v = 0;
+            if (s == kEscape) v = p.esc_q[ctx];
+            else if (s >= lo && s < lo + n) v = __ldg(qa + (s - lo));
+            q[i] = v;
+            sum += v;
+        }
+        uint32_t inc = sum;
+#pragma unroll
+        for (int o = 1; o < 32; o <<= 1) {
+            uint32_t t = __shfl_up_sync(kFull, inc, o);
+            if (lane >= uint32_t(o)) inc += t;
+        }
+        uint32_t c = inc - sum;
+#pragma unroll
+        for (int i = 0; i < 8; ++i) {
+            sm.fc[ctx][8 * lane + i] = q[i] | (c << 16);
+            c += q[i];
+        }
+    }
+    __syncthreads();
+    // (b) slot -> symbol, 4 slots per 32-bit store; a context is split into P parts per warp
+    constexpr int P = WARPS >= 16 ? WARPS / 16 : 1;
+    constexpr uint32_t kPerLane = kProbTotal / (32 * P);
+    for (uint32_t item = warp; item < uint32_t(kFieldContexts * P); item += WARPS) {
+        const uint32_t ctx = item / P, part = item % P;
+        const uint32_t* fc = sm.fc[ctx];
+        const uint32_t first = (part * 32 + lane) * kPerLane;
+        uint32_t* dst = reinterpret_cast<uint32_t*>(&sm.sym[ctx][first]);
+        const uint32_t total = (fc[255] >> 16) + (fc[255] & 0xFFFF);
+        if (total == 0) {  // context never used by this blob
+            for (uint32_t w = 0; w < kPerLane / 4; ++w) dst[w] = 0;
+            continue;
+        }
+        uint32_t s = 0;  // largest symbol with cum(s) <= first
+#pragma unroll
+        for (uint32_t step = 128; step; step >>= 1)
+            if ((fc[s + step] >> 16) <= first) s += step;
+        uint32_t next = s < 255 ? (fc[s + 1] >> 16) : kProbTotal;
+        for (uint32_t w = 0; w < kPerLane / 4; ++w) {
+            const uint32_t base = first + 4 * w;
+            uint32_t word;
+            if (next >= base + 4) {
+                word = s * 0x01010101u;
+            } else {
+                word = 0;
+                for (uint32_t k = 0; k < 4; ++k) {
+                    while (next <= base + k) {
+                        ++s;
+                        next = s < 255 ? (fc[s + 1] >> 16) : kProbTotal;
+                    }
+                    word |= s << (8 * k);
+                }
+            }
+            dst[w] = word;
+        }
+    }
+}
+
+// ---- output conversion -----------------------------------------------------------------------
+template <int OUT>
+__device__ __forceinline__ void store_vec(void* out, int64_t elem, const float v[8]) {
+    if constexpr (OUT == kOutBF16) {
+        uint4 u;
+        __nv_bfloat162 h0 = __floats2bfloat162_rn(v[0], v[1]), h1 = __floats2bfloat162_rn(v[2], v[3]);
+        __nv_bfloat162 h2 = __floats2bfloat162_rn(v[4], v[5]), h3 = __floats2bfloat162_rn(v[6], v[7]);
+        u.x = *reinterpret_cast<uint32_t*>(&h0);
+        u.y = *reinterpret_cast<uint32_t*>(&h1);
+        u.z = *reinterpret_cast<uint32_t*>(&h2);
+        u.w = *reinterpret_cast<uint32_t*>(&h3);
+        __stcs(reinterpret_cast<uint4*>(static_cast<__nv_bfloat16*>(out) + elem), u);
+    } else if constexpr (OUT == kOutFP16) {
+        uint4 u;
+        __half2 h0 = __floats2half2_rn(v[0], v[1]), h1 = __floats2half2_rn(v[2], v[3]);
+        __half2 h2 = __floats2half2_rn(v[4], v[5]), h3 = __floats2half2_rn(v[6], v[7]);
+        u.x = *reinterpret_cast<uint32_t*>(&h0);
+        u.y = *reinterpret_cast<uint32_t*>(&h1);
+        u.z = *reinterpret_cast<uint32_t*>(&h2);
+        u.w = *reinterpret_cast<uint32_t*>(&h3);
+        __stcs(reinterpret_cast<uint4*>(static_cast<__half*>(out) + elem), u);
+    } else if constexpr (OUT == kOutE4M3) {
+        uint32_t w[4];
+#pragma unroll
+        for (int i = 0; i < 4; ++i)
+            w[i] = __nv_cvt_float2_to_fp8x2(make_float2(v[2 * i], v[2 * i + 1]), __NV_SATFINITE, __NV_E4M3);
+        uint2 u = make_uint2(w[0] | (w[1] << 16), w[2] | (w[3] << 16));
+        __stcs(reinterpret_cast<uint2*>(static_cast<uint8_t*>(out) + elem), u);
+    } else {
+        float4* o = reinterpret_cast<float4*>(static_cast<float*>(out) + elem);
+        __stcs(o, make_float4(v[0], v[1], v[2], v[3]));
+        __stcs(o + 1, make_float4(v[4], v[5], v[6], v[7]));
+    }
+}
+
+template <int OUT>
+__device__ __forceinline__ void store_one(void* out, int64_t elem, float v) {
+    if constexpr (OUT == kOutBF16) static_cast<__nv_bfloat16*>(out)[elem] = __float2bfloat16_rn(v);
+    else if constexpr (OUT == kOutFP16) static_cast<__half*>(out)[elem] = __float2half_rn(v);
+    else if constexpr (OUT == kOutE4M3)
+        static_cast<uint8_t*>(out)[elem] = uint8_t(__nv_cvt_float_to_fp8(v, __NV_SATFINITE, __NV_E4M3));
+    else static_cast<float*>(out)[elem] = v;
+}
+
+// ---- one step: every lane decodes (at most) one 8-vector --------------------------------------
+template <int WARPS, int OUT, bool VEC, bool FULL>
+__device__ __forceinline__ void decode_step(const Smem<WARPS>& sm, const Params& p, const uint8_t* ring,
+                                            uint32_t& x, uint32_t& cur, bool active, uint32_t lt, int64_t v,
+                                            int64_t row, int64_t kcol) {
+    if (FULL) active = true;
+    // issued early, used after the symbol chain; lanes past the last vector read nothing
+    const float a = active ? __ldg(p.alpha + row) : 0.0f;
+
+    // coset (two symbols: slot < q0 -> 0)
+    const uint32_t q0 = p.q_coset0;
+    uint32_t slot = x & (kProbTotal - 1);
+    const uint32_t c = slot >= q0 ? 1u : 0u;
+    if (active) x = (c ? kProbTotal - q0 : q0) * (x >> kProbBits) + slot - (c ? q0 : 0u);
+    renorm(x, cur, ring, lt, active);
+
+    // fields f1..f8 with context (c, j)
+    const uint8_t* st = &sm.sym[8 * c][0];
+    const uint32_t* ft = &sm.fc[8 * c][0];
+    uint32_t sym[8];
+#pragma unroll
+    for (int j = 0; j < 8; ++j) {
+        slot = x & (kProbTotal - 1);
+        const uint32_t s = st[j * kProbTotal + slot];
+        const uint32_t e = ft[j * 256 + s];
+        if (active) x = (e & 0xFFFFu) * (x >> kProbBits) + slot - (e >> 16);
+        renorm(x, cur, ring, lt, active);
+        sym[j] = s;
+    }
+
+    // escaped fields: raw words after the step's renormalisation words, by field then lane
+    int32_t f[8];
+#pragma unroll
+    for (int j = 0; j < 8; ++j) f[j] = int32_t(sym[j]) - kAlphabetR;
+    uint32_t esc = 0;
+#pragma unroll
+    for (int j = 0; j < 8; ++j) esc |= (active && sym[j] == uint32_t(kEscape)) ? (1u << j) : 0u;
+    if (__any_sync(kFull, esc != 0)) {
+#pragma unroll
+        for (int j = 0; j < 8; ++j) {
+            const bool mine = (esc >> j) & 1u;
+            const uint32_t b = __ballot_sync(kFull, mine);
+            if (mine) f[j] = int16_t(ring_word(ring, cur + 2u * __popc(b & lt)));
+            cur += 2u * __popc(b);
+        }
+    }
+    if (!active) return;
+
+    if constexpr (OUT == kOutFields) {
+        int16_t* o = static_cast<int16_t*>(p.out) + 9 * v;
+        o[0] = int16_t(c);
+#pragma unroll
+        for (int j = 0; j < 8; ++j) o[1 + j] = int16_t(f[j]);
+        return;
+    } else {
+        // lattice point: z1..z7 = f1..f7, z8 = 2 f8 + (z1+..+z7 mod 2); 2y = 2z + c
+        const int32_t par = (f[0] + f[1] + f[2] + f[3] + f[4] + f[5] + f[6]) & 1;
+        f[7] = 2 * f[7] + par;
+        float val[8];
+#pragma unroll
+        for (int i = 0; i < 8; ++i) {
+            const float y = __fmul_rn(__int2float_rn(2 * f[i] + int32_t(c)), 0.5f);  // exact
+            val[i] = __fmul_rn(a, y);  // the one rounding of the reconstruction
+        }
+        if constexpr (VEC) {
+            const int64_t elem = p.dense ? 8 * v : row * p.row_stride + 8 * kcol;
+            store_vec<OUT>(p.out, elem, val);
+        } else {
+#pragma unroll
+            for (int i = 0; i < 8; ++i) {
+                const int64_t col = 8 * kcol + i;
+                if (col < p.cols) store_one<OUT>(p.out, row * p.row_stride + col, val[i]);
+            }
+        }
+    }
+}
+
+template <int WARPS, int OUT, bool VEC>
+__global__ void __launch_bounds__(WARPS * 32, (WARPS >= 32 ? 1 : 2048 / (WARPS * 32 * 2)))
+    decode_kernel(const Params p) {
+    extern __shared__ __align__(128) uint8_t smem_raw[];
+    Smem<WARPS>& sm = *reinterpret_cast<Smem<WARPS>*>(smem_raw);
+    const uint32_t lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+    const uint32_t lt = (1u << lane) - 1u;
+    unsigned long long* bar = sm.bar[warp];
+    uint8_t* ring = sm.ring[warp];
+
+    if (lane == 0) {
+        for (int i = 0; i < kRingChunks; ++i) mbar_init(&bar[i], 1);
+        fence_proxy_async();
+    }
+    __syncwarp();
+
+    const uint32_t tile_stride = gridDim.x * WARPS;
+    uint32_t tile = blockIdx.x + gridDim.x * warp;
+    uint32_t seq = 0;  // chunks this warp has issued so far: chunk g uses slot g % 4, parity (g / 4) % 2
+
+    // per-tile cursor state
+    const uint8_t* src = nullptr;
+    uint32_t bytes = 0, nch = 0, issued = 0, waited = 0, g0 = 0, x = 0;
+
+    auto issue = [&](uint32_t j) {
+        const uint32_t g = g0 + j, slot = g & (kRingChunks - 1);
+        const uint32_t nb = min(uint32_t(kChunk), bytes - j * kChunk);
+        __syncwarp();
+        if (lane == 0) {
+            fence_proxy_async();  // earlier reads of this slot come before the bulk write
+            mbar_expect_tx(&bar[slot], nb);
+            bulk_g2s(ring + slot * kChunk, src + size_t(j) * kChunk, nb, &bar[slot]);
+        }
+    };
+    auto wait = [&](uint32_t j) -> bool {
+        const uint32_t g = g0 + j;
+        return mbar_wait(&bar[g & (kRingChunks - 1)], (g >> 2) & 1u);
+    };
+    auto begin_tile = [&]() {
+        const uint64_t t0 = 16ull * __ldg(p.tile_off + tile), t1 = 16ull * __ldg(p.tile_off + tile + 1);
+        src = p.stream + t0 + kTileHeadBytes;
+        bytes = uint32_t(t1 - t0 - kTileHeadBytes);  // the host checked t1 >= t0 + 128
+        nch = (bytes + kChunk - 1) / kChunk;
+        g0 = seq;
+        seq += nch;
+        issued = waited = 0;
+        while (issued < min(nch, uint32_t(kRingChunks))) issue(issued++);
+        x = __ldg(reinterpret_cast<const uint32_t*>(p.stream + t0) + lane);
+    };
+
+    if (tile < p.n_tiles) begin_tile();  // first copies overlap the table expansion
+    build_tables<WARPS>(sm, p);
+    __syncthreads();
+
+    bool first = true;
+    for (; tile < p.n_tiles; tile += tile_stride) {
+        if (!first) begin_tile();
+        first = false;
+        const int64_t per_tile = int64_t(kLanes) * p.steps;
+        const int64_t v0 = int64_t(tile) * per_tile;
+        const int64_t vend = min(v0 + per_tile, p.n_vectors);
+        const uint32_t nsteps = uint32_t((vend - v0 + kLanes - 1) / kLanes);
+        int64_t v = v0 + lane;
+        int64_t row = v / p.vec_per_row, kcol = v - row * p.vec_per_row;
+        uint32_t cur = 0;
+        uint32_t flags = 0;
+        for (uint32_t k = 0; k < nsteps; ++k) {
+            // keep the ring full and the bytes this step may read resident
+            const uint32_t lim = min(nch, cur / kChunk + kRingChunks);
+            while (issued < lim) issue(issued++);
+            const uint32_t need = (min(bytes, cur + uint32_t(kMaxStepBytes)) + kChunk - 1) / kChunk;
+            while (waited < need) {
+                if (!wait(waited)) goto timeout;
+                ++waited;
+            }
+            if (v0 + int64_t(k + 1) * kLanes <= vend)
+                decode_step<WARPS, OUT, VEC, true>(sm, p, ring, x, cur, true, lt, v, row, kcol);
+            else
+                decode_step<WARPS, OUT, VEC, false>(sm, p, ring, x, cur, v < vend, lt, v, row, kcol);
+            if (cur > bytes) {
+                flags |= kStOverrun;
+                break;
+            }
+            v += kLanes;
+            kcol += kLanes;
+            while (kcol >= p.vec_per_row) {
+                kcol -= p.vec_per_row;
+                ++row;
+            }
+        }
+        // drain copies the decode did not need (padding) before the slots are reused
+        while (waited < issued) {
+            if (!wait(waited)) goto timeout;
+            ++waited;
+        }
+        if (!(flags & kStOverrun)) {
+            if (__any_sync(kFull, x != kStateLow)) flags |= kStState;
+            if (bytes - cur >= 16) flags |= kStLeftover;
+        }
+        if (lane == 0 && flags) atomicOr(p.status, flags);
+    }
+    return;
+
+timeout:
+    if (lane == 0) atomicOr(p.status, kStTimeout);
+    // wait (bounded again) for copies still in flight into this warp's ring before leaving
+    while (waited < issued) {
+        wait(waited);
+        ++waited;
+    }
+}
+
+// ---- host-side launch -------------------------------------------------------------------------
+constexpr int kWarps = 16;
+
+struct DevInfo {
+    bool ready = false;
+    int sms = 0;
+};
+std::mutex g_dev_mu;
+DevInfo g_dev[kMaxDevices];
+
+template <int WARPS, int OUT, bool VEC>
+int launch_one(const Params& p, cudaStream_t st, int device) {
+    auto fn = decode_kernel<WARPS, OUT, VEC>;
+    const size_t smem = sizeof(Smem<WARPS>);
+    static std::mutex mu;
+    static int per_sm[kMaxDevices] = {};
+    {
+        std::lock_guard<std::mutex> g(mu);
+        if (per_sm[device] == 0) {
+            cudaError_t e = cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, int(smem));
+            if (e != cudaSuccess) return set_error(EP_ERR_CUDA, std::string("decode kernel attribute: ") + cudaGetErrorString(e));
+            int n = 0;
+            e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, fn, WARPS * 32, smem);
+            if (e != cudaSuccess || n < 1) return set_error(EP_ERR_CUDA, "decode kernel does not fit on an SM");
+            per_sm[device] = n;
+        }
+    }
+    const uint32_t grid = uint32_t(std::min<int64_t>(int64_t(g_dev[device].sms) * per_sm[device], p.n_tiles));
+    fn<<<grid, WARPS * 32, smem, st>>>(p);
+    cudaError_t e = cudaGetLastError();
+    if (e != cudaSuccess) return set_error(EP_ERR_CUDA, std::string("decode launch: ") + cudaGetErrorString(e));
+    return EP_OK;
+}
+
+template <int OUT>
+int launch_out(const Params& p, bool vec, cudaStream_t st, int device) {
+    return vec ? launch_one<kWarps, OUT, true>(p, st, device) : launch_one<kWarps, OUT, false>(p, st, device);
+}
+
+int launch(const Params& p, int out_kind, bool vec, cudaStream_t st, int device) {
+    switch (out_kind) {
+        case kOutBF16: return launch_out<kOutBF16>(p, vec, st, device);
+        case kOutFP16: return launch_out<kOutFP16>(p, vec, st, device);
+        case kOutE4M3: return launch_out<kOutE4M3>(p, vec, st, device);
+        case kOutF32: return launch_out<kOutF32>(p, vec, st, device);
+        default: return launch_one<kWarps, kOutFields, false>(p, st, device);
+    }
+}
+
+int out_kind_of(int dtype) {
+    switch (dtype) {
+        case kBF16: return kOutBF16;
+        case kFP16: return kOutFP16;
+        case kE4M3: return kOutE4M3;
+        case kF32: return kOutF32;
+        default: return -1;
+    }
+}
+
+#define EP_CUDA(call, what)                                                                      \
+    do {                                                                                         \
+        cudaError_t e_ = (call);                                                                 \
+        if (e_ != cudaSuccess) return set_error(EP_ERR_CUDA, std::string(what) + ": " + cudaGetErrorString(e_)); \
+    } while (0)
+
+int current_device(int& dev) {
+    EP_CUDA(cudaGetDevice(&dev), "cudaGetDevice");
+    if (dev < 0 || dev >= kMaxDevices) return set_error(EP_ERR_ARG, "device ordinal out of range");
+    std::lock_guard<std::mutex> g(g_dev_mu);
+    if (!g_dev[dev].ready) {
+        EP_CUDA(cudaDeviceGetAttribute(&g_dev[dev].sms, cudaDevAttrMultiProcessorCount, dev), "SM count");
+        g_dev[dev].ready = true;
+    }
+    return EP_OK;
+}
+
+// Device copy of the blob and its status word on `dev` (allocated and filled on first use).
+int ensure_device(ep_blob* b, int dev, cudaStream_t st) {
+    std::lock_guard<std::mutex> g(b->mu);
+    DeviceCopy& d = b->dev[dev];
+    if (d.blob) return EP_OK;
+    uint8_t* blob = nullptr;
+    uint32_t* status = nullptr;
+    if (cudaMalloc(&blob, b->bytes.size()) != cudaSuccess || cudaMalloc(&status, 16) != cudaSuccess) {
+        cudaFree(blob);
+        return set_error(EP_ERR_OOM, "device copy of the blob");
+    }
+    EP_CUDA(cudaMemcpyAsync(blob, b->bytes.data(), b->bytes.size(), cudaMemcpyHostToDevice, st), "blob upload");
+    EP_CUDA(cudaMemsetAsync(status, 0, 16, st), "status clear");
+    EP_CUDA(cudaStreamSynchronize(st), "blob upload");
+    d.blob = blob;
+    d.status = status;
+    return EP_OK;
+}
+
+Params make_params(const ep_blob* b, const uint8_t* dblob, void* out, int64_t row_stride, uint32_t* status,
+                   bool vec) {
+    const BlobLayout& L = b->layout;
+    Params p;
+    p.blob = dblob;
+    p.tile_off = reinterpret_cast<const uint32_t*>(dblob + L.off_offsets);
+    p.stream = dblob + L.off_stream;
+    p.alpha = reinterpret_cast<const float*>(dblob + L.off_alpha);
+    p.out = out;
+    p.status = status;
+    p.cols = L.cols;
+    p.row_stride = row_stride;
+    p.n_vectors = L.n_vectors;
+    p.vec_per_row = L.vec_per_row;
+    p.steps = L.steps;
+    p.n_tiles = L.n_tiles;
+    p.q_coset0 = L.q_coset[0];
+    for (int c = 0; c < kFieldContexts; ++c) {
+        p.q_off[c] = L.q_offset[c];
+        p.esc_q[c] = L.esc_q[c];
+        p.lo[c] = L.lo[c];
+        p.n[c] = L.n[c];
+    }
+    p.dense = vec && row_stride == L.cols;
+    return p;
+}
+
+bool vec_ok(const BlobLayout& L, const void* out, int64_t row_stride, int dtype) {
+    const uintptr_t align = dtype == kE4M3 ? 8 : 16;
+    return L.cols % 8 == 0 && row_stride % 8 == 0 && (reinterpret_cast<uintptr_t>(out) % align) == 0;
+}
+
+}  // namespace
+}  // namespace ep
+
+using namespace ep;
+
+extern "C" int ep_blob_prepare(ep_blob* b, int device, void* stream) {
+    clear_error();
+    if (!b) return set_error(EP_ERR_ARG, "ep_blob_prepare: NULL blob");
+    int prev = 0;
+    EP_CUDA(cudaGetDevice(&prev), "cudaGetDevice");
+    EP_CUDA(cudaSetDevice(device), "cudaSetDevice");
+    int dev = 0;
+    int rc = current_device(dev);
+    if (rc == EP_OK) rc = ensure_device(b, dev, static_cast<cudaStream_t>(stream));
+    cudaSetDevice(prev);
+    return rc;
+}
+
+extern "C" int ep_decompress(const ep_blob* cb, const ep_tensor* out, void* stream) {
+    clear_error();
+    if (!cb || !out || !out->data) return set_error(EP_ERR_ARG, "ep_decompress: NULL argument");
+    ep_blob* b = const_cast<ep_blob*>(cb);
+    const BlobLayout& L = b->layout;
+    const int kind = out_kind_of(out->dtype);
+    if (kind < 0) return set_error(EP_ERR_DTYPE, "ep_decompress: unsupported output dtype");
+    if (out->rows != L.rows || out->cols != L.cols)
+        return set_error(EP_ERR_SHAPE, "ep_decompress: output shape differs from the blob's");
+    if (out->row_stride < out->cols) return set_error(EP_ERR_ARG, "ep_decompress: row_stride < cols");
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    int dev = 0;
+    int rc = current_device(dev);
+    if (rc != EP_OK) return rc;
+
+    if (out->device >= 0) {
+        if (out->device != dev)
+            return set_error(EP_ERR_ARG, "ep_decompress: output is not on the current device");
+        rc = ensure_device(b, dev, st);
+        if (rc != EP_OK) return rc;
+        const DeviceCopy& d = b->dev[dev];
+        const bool vec = vec_ok(L, out->data, out->row_stride, out->dtype);
+        Params p = make_params(b, d.blob, out->data, out->row_stride, d.status, vec);
+        return launch(p, kind, vec, st, dev);
+    }
+
+    // Host output: upload the bytes, decode into a blob-owned buffer, copy back, synchronise.
+    rc = ensure_device(b, dev, st);
+    if (rc != EP_OK) return rc;
+    const size_t es = size_t(dtype_bytes(out->dtype));
+    const size_t out_bytes = size_t(L.rows) * size_t(L.cols) * es;
+    {
+        std::lock_guard<std::mutex> g(b->mu);
+        DeviceCopy& d = b->dev[dev];
+        if (!d.stage_blob && cudaMalloc(&d.stage_blob, b->bytes.size()) != cudaSuccess)
+            return set_error(EP_ERR_OOM, "ep_decompress: staging copy of the blob");
+        if (d.stage_out_bytes < out_bytes) {
+            cudaFree(d.stage_out);
+            d.stage_out = nullptr;
+            d.stage_out_bytes = 0;
+            if (cudaMalloc(&d.stage_out, out_bytes) != cudaSuccess)
+                return set_error(EP_ERR_OOM, "ep_decompress: staging output");
+            d.stage_out_bytes = out_bytes;
+        }
+        if (!b->host_pinned) {
+            // best effort: page-locked host bytes make the per-call upload a direct DMA
+            if (cudaHostRegister(b->bytes.data(), b->bytes.size(), cudaHostRegisterDefault) == cudaSuccess)
+                b->host_pinned = true;
+            else
+                cudaGetLastError();
+        }
+    }
+    const DeviceCopy& d = b->dev[dev];
+    EP_CUDA(cudaMemcpyAsync(d.stage_blob, b->bytes.data(), b->bytes.size(), cudaMemcpyHostToDevice, st),
+            "ep_decompress: upload");
+    const bool vec = vec_ok(L, d.stage_out, L.cols, out->dtype);
+    Params p = make_params(b, d.stage_blob, d.stage_out, L.cols, d.status, vec);
+    rc = launch(p, kind, vec, st, dev);
+    if (rc != EP_OK) return rc;
+    EP_CUDA(cudaMemcpy2DAsync(out->data, size_t(out->row_stride) * es, d.stage_out, size_t(L.cols) * es,
+                              size_t(L.cols) * es, size_t(L.rows), cudaMemcpyDeviceToHost, st),
+            "ep_decompress: download");
+    EP_CUDA(cudaStreamSynchronize(st), "ep_decompress: synchronise");
+    return EP_OK;
+}
+
+extern "C" int ep_decode_fields(const ep_blob* cb, int16_t* fields, void* stream) {
+    clear_error();
+    if (!cb || !fields) return set_error(EP_ERR_ARG, "ep_decode_fields: NULL argument");
+    ep_blob* b = const_cast<ep_blob*>(cb);
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    int dev = 0;
+    int rc = current_device(dev);
+    if (rc == EP_OK) rc = ensure_device(b, dev, st);
+    if (rc != EP_OK) return rc;
+    const DeviceCopy& d = b->dev[dev];
+    Params p = make_params(b, d.blob, fields, b->layout.cols, d.status, false);
+    return launch(p, kOutFields, false, st, dev);
+}
+
+extern "C" int ep_decode_status(const ep_blob* cb, void* stream) {
+    clear_error();
+    if (!cb) return set_error(EP_ERR_ARG, "ep_decode_status: NULL blob");
+    ep_blob* b = const_cast<ep_blob*>(cb);
+    int dev = 0;
+    int rc = current_device(dev);
+    if (rc != EP_OK) return rc;
+    DeviceCopy& d = b->dev[dev];
+    if (!d.status) return EP_OK;  // never decoded on this device
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    uint32_t s = 0;
+    EP_CUDA(cudaStreamSynchronize(st), "ep_decode_status: synchronise");
+    EP_CUDA(cudaMemcpy(&s, d.status, 4, cudaMemcpyDeviceToHost), "ep_decode_status: read");
+    EP_CUDA(cudaMemset(d.status, 0, 4), "ep_decode_status: clear");
+    if (s == 0) return EP_OK;
+    std::string why = "GPU decode found a corrupt blob:";
+    if (s & kStOverrun) why += " tile read past its end;";
+    if (s & kStState) why += " final rANS state not 2^16;";
+    if (s & kStLeftover) why += " unread tile words;";
+    if (s & kStTimeout) why += " bulk-copy wait limit reached;";
+    return set_error(EP_ERR_CORRUPT, why);
+}
+
+extern "C" void ep_blob_free(ep_blob* b) {
+    if (!b) return;
+    int prev = 0;
+    cudaGetDevice(&prev);
+    for (int dv = 0; dv < kMaxDevices; ++dv) {
+        DeviceCopy& d = b->dev[dv];
+        if (!d.blob && !d.stage_blob && !d.stage_out) continue;
+        cudaSetDevice(dv);
+        cudaFree(d.blob);
+        cudaFree(d.status);
+        cudaFree(d.stage_blob);
+        cudaFree(d.stage_out);
+    }
+    if (b->host_pinned) cudaHostUnregister(b->bytes.data());
+    cudaSetDevice(prev);
+    delete b;
+}

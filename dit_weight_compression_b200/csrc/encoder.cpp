@@ -1,0 +1,546 @@
+// encoder.cpp -- host encoder of the library (ep_compress).
+//
+// Steps, as "EntroPack lattice compression" (documentation page) describes them:
+//   section "Lattice quantization and integer fields": normalise each row by its RMS, group
+//     the normalised values into 8-vectors, replace each by its nearest point of a scaled E8
+//     lattice (shared scale s), store the point as a coset bit and eight integer fields with the
+//     last coordinate compacted by the parity constraint, model each field conditioned on the
+//     coset;
+//   section "Rate selection and refinement": choose s from size estimates on sampled rows,
+//     then quantise the full tensor and fit one least-squares scale per row;
+//   section "Encoding and reconstruction": rANS-code the fields in independently decodable
+//     tiles and store tables, row scales and tile metadata with them.
+// The rANS coding step is Duda's ("Asymmetric numeral systems", 2009); the E8 nearest point is
+// the Conway-Sloane rule (1982).  Details the pages leave open are fixed as the format header
+// (format.h) and the comments below state.
+//
+// Work is split over host threads by rows, sampled rows and tiles; every reduction is over
+// integers or in a fixed order, so the bytes do not depend on the thread count.
+#include <algorithm>
+#include <atomic>
+#include <cmath>
+#include <functional>
+#include <thread>
+
+#include "format.h"
+
+namespace ep {
+
+// ---------------------------------------------------------------------------------------------
+// Parallel loop over [0, n) in contiguous blocks.
+// ---------------------------------------------------------------------------------------------
+static void parallel_for(int64_t n, int threads, const std::function<void(int64_t, int64_t, int)>& body) {
+    if (n <= 0) return;
+    int T = int(std::max<int64_t>(1, std::min<int64_t>(threads, n)));
+    if (T == 1) { body(0, n, 0); return; }
+    std::vector<std::thread> pool;
+    pool.reserve(T);
+    for (int t = 0; t < T; ++t) {
+        int64_t a = n * t / T, b = n * (t + 1) / T;
+        pool.emplace_back([=, &body] { body(a, b, t); });
+    }
+    for (auto& th : pool) th.join();
+}
+
+// ---------------------------------------------------------------------------------------------
+// Reading container elements as exact doubles.
+// ---------------------------------------------------------------------------------------------
+class ElementReader {
+public:
+    ElementReader(const void* base, int dtype, int64_t rows, int64_t cols, int64_t stride)
+        : base_(static_cast<const uint8_t*>(base)), dtype_(dtype), rows_(rows), cols_(cols), stride_(stride) {
+        if (dtype == kFP16) {
+            lut_.resize(65536);
+            for (uint32_t h = 0; h < 65536; ++h) lut_[h] = half_value(h);
+        } else if (dtype == kE4M3) {
+            lut_.resize(256);
+            for (uint32_t b = 0; b < 256; ++b) lut_[b] = e4m3_value(b);
+        }
+    }
+    // value of (r, c); columns past cols are the zero padding
+    double at(int64_t r, int64_t c) const {
+        if (c >= cols_) return 0.0;
+        size_t idx = size_t(r * stride_ + c);
+        switch (dtype_) {
+            case kBF16: {
+                uint32_t w = uint32_t(reinterpret_cast<const uint16_t*>(base_)[idx]) << 16;
+                float f;
+                std::memcpy(&f, &w, 4);
+                return f;
+            }
+            case kFP16: return lut_[reinterpret_cast<const uint16_t*>(base_)[idx]];
+            case kE4M3: return lut_[base_[idx]];
+            default: return reinterpret_cast<const float*>(base_)[idx];
+        }
+    }
+
+private:
+    static double half_value(uint32_t h) {  // IEEE binary16
+        int e = (h >> 10) & 0x1F;
+        uint32_t m = h & 0x3FF;
+        double mag = e == 0 ? std::ldexp(double(m), -24)
+                   : e == 31 ? (m ? NAN : INFINITY)
+                   : std::ldexp(double(m | 0x400), e - 25);
+        return (h & 0x8000) ? -mag : mag;
+    }
+    static double e4m3_value(uint32_t b) {  // OCP E4M3: bias 7, S.1111.111 is NaN, no inf
+        int e = (b >> 3) & 0xF;
+        uint32_t m = b & 7;
+        double mag = (e == 15 && m == 7) ? NAN
+                   : e == 0 ? std::ldexp(double(m), -9)
+                   : std::ldexp(double(m | 8), e - 10);
+        return (b & 0x80) ? -mag : mag;
+    }
+    const uint8_t* base_;
+    int dtype_;
+    int64_t rows_, cols_, stride_;
+    std::vector<double> lut_;
+};
+
+// ---------------------------------------------------------------------------------------------
+// Lattice quantisation.
+// ---------------------------------------------------------------------------------------------
+
+// Conway-Sloane nearest point of D8 = {z in Z^8 : sum even}: round every coordinate (halves away
+// from zero); on an odd sum move the coordinate that rounding disturbed most (first one on ties)
+// one step toward its value (up when it was already an integer).
+static inline void nearest_d8(const double u[8], double g[8]) {
+    long long sum = 0;
+    int worst_i = 0;
+    double worst = -1.0;
+    for (int i = 0; i < 8; ++i) {
+        g[i] = std::round(u[i]);
+        sum += (long long)g[i];
+        double miss = std::fabs(u[i] - g[i]);
+        if (miss > worst) { worst = miss; worst_i = i; }
+    }
+    if (sum % 2 != 0) g[worst_i] += (u[worst_i] < g[worst_i]) ? -1.0 : 1.0;
+}
+
+// Nearest point of E8 = D8 u (D8 + 1/2): the closer of the D8 point and the half-integer coset
+// point (the D8 rule on t - 1/2, shifted back); equal distances keep the integer coset.
+static inline int nearest_e8(const double t[8], double y[8]) {
+    double a[8], b[8], u[8];
+    nearest_d8(t, a);
+    for (int i = 0; i < 8; ++i) u[i] = t[i] - 0.5;
+    nearest_d8(u, b);
+    double da = 0.0, db = 0.0;
+    for (int i = 0; i < 8; ++i) {
+        b[i] += 0.5;
+        da += (t[i] - a[i]) * (t[i] - a[i]);
+        db += (t[i] - b[i]) * (t[i] - b[i]);
+    }
+    const double* best = db < da ? b : a;
+    for (int i = 0; i < 8; ++i) y[i] = best[i];
+    return db < da ? 1 : 0;
+}
+
+// One quantised vector: coset bit, eight fields, and the lattice point (in units of s).
+struct QVec {
+    int coset;
+    int32_t f[8];
+    double y[8];
+};
+
+class Quantiser {
+public:
+    Quantiser(const ElementReader& rd, int64_t rows, int64_t cols, const std::vector<double>& rms)
+        : rd_(rd), rows_(rows), cols_(cols), rms_(rms) {}
+
+    // vector k of row r at shared scale s; |x_hat / s| is clamped to 32764 so that every
+    // field fits an int16 raw word.
+    void quantise(int64_t r, int64_t k, double s, QVec& q) const {
+        double t[8];
+        double rr = rms_[size_t(r)];
+        for (int i = 0; i < 8; ++i) {
+            double xh = rr > 0.0 ? rd_.at(r, 8 * k + i) / rr : 0.0;
+            double v = xh / s;
+            t[i] = v > 32764.0 ? 32764.0 : (v < -32764.0 ? -32764.0 : v);
+        }
+        q.coset = nearest_e8(t, q.y);
+        // fields: z = y - c/2 in D8; f1..f7 = z1..z7; f8 = (z8 - (z1+...+z7 mod 2)) / 2
+        int32_t z[8], s7 = 0;
+        for (int i = 0; i < 8; ++i) z[i] = int32_t(q.y[i] - 0.5 * q.coset);
+        for (int i = 0; i < 7; ++i) { q.f[i] = z[i]; s7 += z[i]; }
+        int32_t par = s7 & 1;
+        q.f[7] = (z[7] - par) / 2;
+    }
+
+private:
+    const ElementReader& rd_;
+    int64_t rows_, cols_;
+    const std::vector<double>& rms_;
+};
+
+static inline int symbol_of(int32_t f) { return (f >= -kAlphabetR && f <= kAlphabetR) ? f + kAlphabetR : kEscape; }
+
+// Symbol counts of the 17 contexts: [0] the coset (symbols 0/1), [1 + 8c + j - 1] field j | c.
+struct Counts {
+    std::vector<uint64_t> c = std::vector<uint64_t>(17 * 256, 0);
+    uint64_t escapes = 0;
+    void add(const QVec& q) {
+        c[size_t(q.coset)]++;
+        for (int j = 0; j < 8; ++j) {
+            int sy = symbol_of(q.f[j]);
+            c[size_t(256 * (1 + 8 * q.coset + j) + sy)]++;
+            escapes += sy == kEscape;
+        }
+    }
+    void merge(const Counts& o) {
+        for (size_t i = 0; i < c.size(); ++i) c[i] += o.c[i];
+        escapes += o.escapes;
+    }
+};
+
+// 12-bit frequencies from counts: q = max(1, round-half-up(4096 n / N)) for used symbols, then
+// the sum is brought to 4096 -- excess taken one at a time from the largest q (> 1, lowest symbol
+// first), deficit given one at a time to the most frequent symbol (lowest symbol first).
+static void quantise_freqs(const uint64_t* n, uint16_t* q) {
+    uint64_t total = 0;
+    for (int s = 0; s < 256; ++s) total += n[s];
+    std::fill(q, q + 256, uint16_t(0));
+    if (total == 0) return;
+    int64_t sum = 0;
+    for (int s = 0; s < 256; ++s) {
+        if (!n[s]) continue;
+        uint64_t v = (2 * uint64_t(kProbTotal) * n[s] + total) / (2 * total);
+        q[s] = uint16_t(std::max<uint64_t>(v, 1));
+        sum += q[s];
+    }
+    while (sum > int64_t(kProbTotal)) {
+        int best = -1;
+        for (int s = 0; s < 256; ++s)
+            if (q[s] > 1 && (best < 0 || q[s] > q[best])) best = s;
+        --q[best];
+        --sum;
+    }
+    while (sum < int64_t(kProbTotal)) {
+        int best = -1;
+        for (int s = 0; s < 256; ++s)
+            if (n[s] && (best < 0 || n[s] > n[best])) best = s;
+        ++q[best];
+        ++sum;
+    }
+}
+
+struct Tables {
+    uint16_t q[17][256];
+    uint32_t cum[17][257];
+    void build(const Counts& cnt) {
+        for (int c = 0; c < 17; ++c) {
+            quantise_freqs(&cnt.c[size_t(256 * c)], q[c]);
+            cum[c][0] = 0;
+            for (int s = 0; s < 256; ++s) cum[c][s + 1] = cum[c][s] + q[c][s];
+        }
+    }
+    // serialised size of the table section (before padding)
+    uint64_t section_bytes() const {
+        uint64_t b = 4;
+        for (int c = 1; c < 17; ++c) {
+            int lo, cnt;
+            range(c, lo, cnt);
+            b += 4 + 2 * uint64_t(cnt);
+        }
+        return b;
+    }
+    void range(int c, int& lo, int& cnt) const {
+        int first = -1, last = -1;
+        for (int s = 0; s < kEscape; ++s)
+            if (q[c][s]) { if (first < 0) first = s; last = s; }
+        lo = first < 0 ? 0 : first;
+        cnt = first < 0 ? 0 : last - first + 1;
+    }
+};
+
+// ---------------------------------------------------------------------------------------------
+// Tiled, 32-way interleaved rANS.  Decode order of a tile: for each step, sub-steps 0 (coset)
+// and 1..8 (fields); in a sub-step, lanes whose state drops below 2^16 read the next word in
+// ascending lane order; after sub-step 8 the raw words of escaped fields, by field then lane.
+// The encoder walks that order backwards and reverses its words.
+// ---------------------------------------------------------------------------------------------
+static void encode_tile(const uint8_t* coset, const int16_t* fields, int64_t nvec, const Tables& T,
+                        std::vector<uint8_t>& out) {
+    uint32_t x[kLanes];
+    std::fill(x, x + kLanes, kStateLow);
+    std::vector<uint16_t> w;
+    w.reserve(size_t(nvec) * 5);
+    int64_t steps = (nvec + kLanes - 1) / kLanes;
+    auto put = [&](uint32_t& st, int ctx, int sym) {
+        uint32_t f = T.q[ctx][sym], c = T.cum[ctx][sym];
+        if (uint64_t(st) >= (uint64_t(f) << (32 - kProbBits))) {  // renormalise: push 16 bits out
+            w.push_back(uint16_t(st));
+            st >>= 16;
+        }
+        st = (st / f) * kProbTotal + (st % f) + c;
+    };
+    for (int64_t k = steps - 1; k >= 0; --k) {
+        int64_t first = k * kLanes;
+        int lanes = int(std::min<int64_t>(kLanes, nvec - first));
+        for (int j = 7; j >= 0; --j)
+            for (int l = lanes - 1; l >= 0; --l) {
+                int16_t f = fields[size_t(8 * (first + l) + j)];
+                if (symbol_of(f) == kEscape) w.push_back(uint16_t(f));
+            }
+        for (int j = 7; j >= 0; --j)
+            for (int l = lanes - 1; l >= 0; --l) {
+                int64_t v = first + l;
+                put(x[l], 1 + 8 * coset[v] + j, symbol_of(fields[size_t(8 * v + j)]));
+            }
+        for (int l = lanes - 1; l >= 0; --l) put(x[l], 0, coset[first + l]);
+    }
+    size_t bytes = round_up16(kTileHeadBytes + 2 * w.size());
+    out.assign(bytes, 0);
+    for (int l = 0; l < kLanes; ++l) wr32(&out[size_t(4 * l)], x[l]);
+    for (size_t i = 0; i < w.size(); ++i) wr16(&out[kTileHeadBytes + 2 * i], w[w.size() - 1 - i]);
+}
+
+// ---------------------------------------------------------------------------------------------
+// The encoder.
+// ---------------------------------------------------------------------------------------------
+static int default_steps(double target) {
+    double want = std::ceil(128.0 / target);
+    int s = 1;
+    while (double(s) < want) s *= 2;
+    return std::min(1024, std::max(16, s));
+}
+
+int encode(const EncodeInput& in, double target, const EncodeOptions& opt, std::vector<uint8_t>& blob,
+           std::string& why) {
+    const int64_t rows = in.rows, cols = in.cols, vpr = (cols + 7) / 8, V = rows * vpr;
+    const int threads = opt.threads > 0 ? opt.threads : std::max(1u, std::thread::hardware_concurrency());
+    ElementReader rd(in.bits, in.dtype, rows, cols, in.row_stride);
+
+    // RMS of every row; non-finite weights are rejected.
+    std::vector<double> rms(static_cast<size_t>(rows));
+    std::atomic<bool> finite{true};
+    parallel_for(rows, threads, [&](int64_t a, int64_t b, int) {
+        for (int64_t r = a; r < b; ++r) {
+            double acc = 0.0;
+            for (int64_t c = 0; c < cols; ++c) {
+                double v = rd.at(r, c);
+                if (!std::isfinite(v)) finite = false;
+                acc += v * v;
+            }
+            rms[size_t(r)] = std::sqrt(acc / double(cols));
+        }
+    });
+    if (!finite) { why = "input holds a non-finite value"; return -4; }
+    Quantiser Q(rd, rows, cols, rms);
+
+    const int S = opt.steps_per_tile > 0 ? opt.steps_per_tile : default_steps(target);
+    const int64_t per_tile = int64_t(kLanes) * S;
+    const int64_t n_tiles = (V + per_tile - 1) / per_tile;
+    if (n_tiles > int64_t(UINT32_MAX) - 1) { why = "too many tiles"; return -3; }
+
+    // Size estimate at scale s from min(rows, 256) rows at floor(i * rows / n): coded bits under
+    // the sample's own 12-bit tables plus 16 bits per escape, scaled to all rows, plus the exact
+    // metadata (header, tables, row scales, tile offsets) and 136 bytes per tile (32 states and
+    // the mean padding).
+    const int64_t n_sample = std::min<int64_t>(rows, 256);
+    auto estimate = [&](double s) {
+        std::vector<Counts> part(static_cast<size_t>(threads));
+        parallel_for(n_sample, threads, [&](int64_t a, int64_t b, int t) {
+            QVec q;
+            for (int64_t i = a; i < b; ++i) {
+                int64_t r = (i * rows) / n_sample;
+                for (int64_t k = 0; k < vpr; ++k) {
+                    Q.quantise(r, k, s, q);
+                    part[size_t(t)].add(q);
+                }
+            }
+        });
+        Counts all;
+        for (auto& p : part) all.merge(p);
+        Tables T;
+        T.build(all);
+        double bits = 0.0;
+        for (int c = 0; c < 17; ++c)
+            for (int sy = 0; sy < 256; ++sy) {
+                uint64_t n = all.c[size_t(256 * c + sy)];
+                if (n) bits += double(n) * -std::log2(double(T.q[c][sy]) / 4096.0);
+            }
+        double payload = (double(rows) / double(n_sample)) * (bits / 8.0 + 2.0 * double(all.escapes));
+        double meta = double(kHeaderBytes + round_up16(T.section_bytes()) + round_up16(4 * uint64_t(rows)) +
+                             round_up16(4 * uint64_t(n_tiles + 1))) +
+                      double(n_tiles) * (128.0 + 8.0);
+        return 8.0 * (meta + payload) / (double(rows) * double(cols));
+    };
+
+    // Finest scale whose estimate meets the target: bisection on log2 s over [-24, 8].
+    double s;
+    if (opt.scale > 0.0) {
+        s = opt.scale;
+    } else {
+        double lo = -24.0, hi = 8.0;
+        if (estimate(std::exp2(hi)) > target) s = std::exp2(hi);
+        else if (estimate(std::exp2(lo)) <= target) s = std::exp2(lo);
+        else {
+            for (int it = 0; it < 48; ++it) {
+                double mid = 0.5 * (lo + hi);
+                if (estimate(std::exp2(mid)) <= target) hi = mid;
+                else lo = mid;
+            }
+            s = std::exp2(hi);
+        }
+    }
+
+    // Full quantisation, least-squares row scales alpha_r = sum w y / sum y^2 (real columns).
+    std::vector<uint8_t> coset(static_cast<size_t>(V));
+    std::vector<int16_t> fields(static_cast<size_t>(V) * 8);
+    std::vector<float> alpha(static_cast<size_t>(rows));
+    std::vector<Counts> part(static_cast<size_t>(threads));
+    parallel_for(rows, threads, [&](int64_t a, int64_t b, int t) {
+        QVec q;
+        for (int64_t r = a; r < b; ++r) {
+            double swy = 0.0, syy = 0.0;
+            for (int64_t k = 0; k < vpr; ++k) {
+                Q.quantise(r, k, s, q);
+                int64_t v = r * vpr + k;
+                coset[size_t(v)] = uint8_t(q.coset);
+                for (int j = 0; j < 8; ++j) fields[size_t(8 * v + j)] = int16_t(q.f[j]);
+                for (int i = 0; i < 8; ++i)
+                    if (8 * k + i < cols) {
+                        swy += rd.at(r, 8 * k + i) * q.y[i];
+                        syy += q.y[i] * q.y[i];
+                    }
+                part[size_t(t)].add(q);
+            }
+            alpha[size_t(r)] = syy > 0.0 ? float(swy / syy) : 0.0f;
+        }
+    });
+    Counts all;
+    for (auto& p : part) all.merge(p);
+    Tables T;
+    T.build(all);
+
+    // Tiles.
+    std::vector<std::vector<uint8_t>> tiles(static_cast<size_t>(n_tiles));
+    parallel_for(n_tiles, threads, [&](int64_t a, int64_t b, int) {
+        for (int64_t t = a; t < b; ++t) {
+            int64_t v0 = t * per_tile, nv = std::min(per_tile, V - v0);
+            encode_tile(&coset[size_t(v0)], &fields[size_t(8 * v0)], nv, T, tiles[size_t(t)]);
+        }
+    });
+
+    // Serialise.
+    uint64_t tab = T.section_bytes();
+    uint64_t off_tab = kHeaderBytes, off_alpha = off_tab + round_up16(tab);
+    uint64_t off_offs = off_alpha + round_up16(4 * uint64_t(rows));
+    uint64_t off_stream = off_offs + round_up16(4 * uint64_t(n_tiles + 1));
+    uint64_t stream = 0;
+    for (auto& t : tiles) stream += t.size();
+    if (stream / 16 > UINT32_MAX) { why = "stream exceeds the 64 GiB tile-offset range"; return -3; }
+    blob.assign(size_t(off_stream + stream), 0);
+    uint8_t* p = blob.data();
+    std::memcpy(p, "EPK1", 4);
+    wr16(p + 4, kVersion);
+    p[6] = uint8_t(in.dtype);
+    p[7] = uint8_t(kAlphabetR);
+    wr64(p + 8, uint64_t(rows));
+    wr64(p + 16, uint64_t(cols));
+    wr32(p + 24, uint32_t(S));
+    wr32(p + 28, uint32_t(n_tiles));
+    std::memcpy(p + 32, &s, 8);
+    wr64(p + 40, blob.size());
+    wr64(p + 48, off_tab);
+    wr64(p + 56, off_alpha);
+    wr64(p + 64, off_offs);
+    wr64(p + 72, off_stream);
+    uint8_t* t = p + off_tab;
+    wr16(t, T.q[0][0]);
+    wr16(t + 2, T.q[0][1]);
+    t += 4;
+    for (int c = 1; c < 17; ++c) {
+        int lo, cnt;
+        T.range(c, lo, cnt);
+        wr16(t, T.q[c][kEscape]);
+        t[2] = uint8_t(lo);
+        t[3] = uint8_t(cnt);
+        t += 4;
+        for (int i = 0; i < cnt; ++i, t += 2) wr16(t, T.q[c][lo + i]);
+    }
+    for (int64_t r = 0; r < rows; ++r) {
+        uint32_t bitsf;
+        std::memcpy(&bitsf, &alpha[size_t(r)], 4);
+        wr32(p + off_alpha + 4 * r, bitsf);
+    }
+    uint64_t acc = 0;
+    for (int64_t i = 0; i <= n_tiles; ++i) {
+        wr32(p + off_offs + 4 * i, uint32_t(acc / 16));
+        if (i < n_tiles) acc += tiles[size_t(i)].size();
+    }
+    acc = 0;
+    for (auto& tb : tiles) {
+        std::memcpy(p + off_stream + acc, tb.data(), tb.size());
+        acc += tb.size();
+    }
+    return 0;
+}
+
+// ---------------------------------------------------------------------------------------------
+// Blob validation.
+// ---------------------------------------------------------------------------------------------
+bool parse_blob(const uint8_t* d, size_t n, BlobLayout& L, std::string& why) {
+    auto fail = [&](const char* m) { why = m; return false; };
+    if (n < kHeaderBytes) return fail("shorter than the 80-byte header");
+    if (std::memcmp(d, "EPK1", 4) != 0) return fail("bad magic");
+    if (rd16(d + 4) != kVersion) return fail("unknown version");
+    L.dtype = d[6];
+    if (dtype_bytes(L.dtype) == 0) return fail("unknown dtype");
+    if (d[7] != kAlphabetR) return fail("unsupported alphabet");
+    L.rows = int64_t(rd64(d + 8));
+    L.cols = int64_t(rd64(d + 16));
+    L.steps = rd32(d + 24);
+    L.n_tiles = rd32(d + 28);
+    std::memcpy(&L.scale, d + 32, 8);
+    L.total = rd64(d + 40);
+    L.off_tables = rd64(d + 48);
+    L.off_alpha = rd64(d + 56);
+    L.off_offsets = rd64(d + 64);
+    L.off_stream = rd64(d + 72);
+    if (L.total != n) return fail("stored size differs from the byte count");
+    if (L.rows <= 0 || L.cols <= 0 || L.rows > (int64_t(1) << 40) || L.cols > (int64_t(1) << 40))
+        return fail("bad shape");
+    if (L.steps == 0 || L.steps > (1u << 20)) return fail("bad steps per tile");
+    L.vec_per_row = (L.cols + 7) / 8;
+    L.n_vectors = L.rows * L.vec_per_row;
+    int64_t per = int64_t(kLanes) * L.steps;
+    if (int64_t(L.n_tiles) != (L.n_vectors + per - 1) / per) return fail("tile count does not match the shape");
+    auto aligned = [](uint64_t o) { return (o & 15) == 0; };
+    if (!aligned(L.off_tables) || !aligned(L.off_alpha) || !aligned(L.off_offsets) || !aligned(L.off_stream))
+        return fail("misaligned section");
+    if (L.off_tables < kHeaderBytes || L.off_tables + 4 > L.off_alpha ||
+        L.off_alpha + 4 * uint64_t(L.rows) > L.off_offsets ||
+        L.off_offsets + 4 * (uint64_t(L.n_tiles) + 1) > L.off_stream || L.off_stream > n)
+        return fail("sections overlap or run past the end");
+    const uint8_t* t = d + L.off_tables;
+    L.q_coset[0] = rd16(t);
+    L.q_coset[1] = rd16(t + 2);
+    if (uint32_t(L.q_coset[0]) + L.q_coset[1] != kProbTotal) return fail("coset table does not sum to 4096");
+    uint64_t pos = L.off_tables + 4;
+    for (int c = 0; c < kFieldContexts; ++c) {
+        if (pos + 4 > L.off_alpha) return fail("table section truncated");
+        L.esc_q[c] = rd16(d + pos);
+        L.lo[c] = d[pos + 2];
+        L.n[c] = d[pos + 3];
+        if (int(L.lo[c]) + L.n[c] > kEscape) return fail("table symbol range past 254");
+        L.q_offset[c] = uint32_t(pos + 4);
+        pos += 4 + 2 * uint64_t(L.n[c]);
+        if (pos > L.off_alpha) return fail("table section truncated");
+        uint32_t sum = L.esc_q[c];
+        for (int i = 0; i < L.n[c]; ++i) sum += rd16(d + L.q_offset[c] + 2 * i);
+        if (sum != 0 && sum != kProbTotal) return fail("field table does not sum to 4096");
+    }
+    const uint8_t* off = d + L.off_offsets;
+    uint64_t stream = n - L.off_stream, prev = 0;
+    if (rd32(off) != 0) return fail("first tile offset is not 0");
+    for (uint64_t i = 1; i <= L.n_tiles; ++i) {
+        uint64_t o = uint64_t(rd32(off + 4 * i)) * 16;
+        if (o < prev + kTileHeadBytes) return fail("tile shorter than its 128-byte state block");
+        prev = o;
+    }
+    if (prev != stream) return fail("tile offsets do not end at the stream end");
+    return true;
+}
+
+}  // namespace ep

@@ -1,0 +1,160 @@
+/*
+ * entropack.h -- C ABI of the B200 lattice-rANS weight codec.
+ *
+ * The codec follows the EntroPack method: rows are normalised by their RMS and split into
+ * 8-vectors, each vector is replaced by its nearest point of a scaled E8 lattice, the point is
+ * stored as a coset bit plus eight integer fields, the fields are rANS-coded in independently
+ * decodable tiles, and decoding rebuilds the weights on the GPU in one fused kernel.  Sources,
+ * by page title and section: "EntroPack: Fast and Accurate Entropy-Coded Weight Compression at
+ * Arbitrary Bitrates" (arXiv abstract); "EntroPack lattice compression" (documentation page
+ * Principles / Lattice-rANS), sections "Lattice quantization and integer fields", "Rate
+ * selection and refinement", "Encoding and reconstruction" and "Usage".
+ *
+ * Conventions (all calls):
+ *   - Every int-returning call returns EP_OK (0) or a negative ep_status; a message describing
+ *     the last failure on the calling thread is available from ep_last_error().
+ *   - Pointers are plain host or device addresses; sizes are element or byte counts as stated.
+ *     The header needs no CUDA include: a CUDA stream is passed as `void*` (a cudaStream_t;
+ *     NULL means the legacy default stream).
+ *   - Tensors are owned by the caller; blobs are owned by the library and released with
+ *     ep_blob_free().
+ */
+#ifndef ENTROPACK_H
+#define ENTROPACK_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* Element containers.  Decompression keeps the input's dtype by default ("EntroPack lattice
+ * compression", opening paragraph: "Decompression retains the input dtype"); the abstract lists
+ * BF16, FP16 and FP8 containers.  FP32 is accepted as an extra container. */
+typedef enum {
+    EP_BF16 = 1,
+    EP_FP16 = 2,
+    EP_FP8_E4M3 = 3,  /* OCP E4M3 (bias 7, no infinities); outputs saturate to +-448 */
+    EP_F32 = 4
+} ep_dtype;
+
+typedef enum {
+    EP_OK = 0,
+    EP_ERR_ARG = -1,      /* NULL pointer, bad stride, unknown device                       */
+    EP_ERR_DTYPE = -2,    /* unsupported container                                           */
+    EP_ERR_SHAPE = -3,    /* empty tensor, or output shape differs from the blob's          */
+    EP_ERR_RANGE = -4,    /* target bpp outside [0.001, 11] or not finite; non-finite weight */
+    EP_ERR_CORRUPT = -5,  /* blob bytes fail validation, or the GPU decode found them broken */
+    EP_ERR_CUDA = -6,     /* a CUDA runtime call failed (message in ep_last_error)           */
+    EP_ERR_OOM = -7       /* host or device allocation failed                                */
+} ep_status;
+
+/* A 2-D tensor view.  Element (r, c) lives at data + (r * row_stride + c) * element size. */
+typedef struct {
+    void* data;
+    int device;          /* -1: host memory; >= 0: CUDA device ordinal                          */
+    int dtype;           /* ep_dtype                                                            */
+    int64_t rows;
+    int64_t cols;
+    int64_t row_stride;  /* elements between consecutive rows, >= cols                         */
+} ep_tensor;
+
+/* Optional encoder settings (ep_compress uses all defaults). */
+typedef struct {
+    int steps_per_tile;  /* S: tile = 32*S vectors; 0 = clamp(next_pow2(ceil(128/bpp)), 16, 1024) */
+    int num_threads;     /* host encoder threads; 0 = all hardware threads                       */
+    double scale;        /* > 0: use this lattice scale instead of searching for one             */
+} ep_options;
+
+typedef struct ep_blob ep_blob;
+
+/* Header fields of a blob. */
+typedef struct {
+    int64_t rows, cols;
+    int dtype;           /* input container recorded at compression */
+    int steps_per_tile;  /* S */
+    int64_t n_tiles;
+    int64_t n_vectors;   /* rows * ceil(cols / 8) */
+    double scale;        /* the shared lattice scale s chosen by the rate search */
+    uint64_t bytes;      /* stored bytes, including all metadata */
+} ep_blob_info;
+
+/*
+ * Compress a 2-D tensor to a target rate ("EntroPack lattice compression": opening paragraph --
+ * "finite target bitrates in [0.001, 11] bits per element, including non-integer values";
+ * sections "Lattice quantization and integer fields" and "Rate selection and refinement").
+ *   in          tensor to compress, host or device memory, any ep_dtype; rows, cols >= 1.
+ *               Device tensors are copied to the host first (the encoder runs on the host).
+ *   target_bpp  requested stored bits per element, finite, in [0.001, 11].
+ *   out         receives a new blob (free with ep_blob_free).
+ * Synchronous.  Errors: EP_ERR_ARG, EP_ERR_DTYPE, EP_ERR_SHAPE (empty), EP_ERR_RANGE,
+ * EP_ERR_CUDA, EP_ERR_OOM.  Deterministic: the same input and settings give the same bytes.
+ */
+int ep_compress(const ep_tensor* in, double target_bpp, ep_blob** out);
+
+/* ep_compress with explicit encoder settings (opt may be NULL for the defaults). */
+int ep_compress_ex(const ep_tensor* in, double target_bpp, const ep_options* opt, ep_blob** out);
+
+/*
+ * Decompress into `out` ("EntroPack lattice compression", section "Encoding and
+ * reconstruction": "Decoding recovers the fields, reconstructs lattice points, and applies the
+ * row scales in a fused GPU operation. The result has the input's shape and dtype").
+ *   b       blob.
+ *   out     rows x cols equal to the blob's; dtype any ep_dtype (the blob's own by convention).
+ *           Device output (out->device >= 0, must be the calling thread's current device): one
+ *           kernel launch on `stream`, asynchronous.  The first call on a device copies the
+ *           blob to that device (it allocates and synchronises once; do that before any stream
+ *           capture).  Later calls allocate nothing and do not synchronise.
+ *           Host output (out->device == -1): end-to-end path on the current device -- copies the
+ *           blob bytes host->device, decodes into a blob-owned device buffer, copies the result
+ *           device->host into out->data, and synchronises `stream` before returning.
+ *   stream  cudaStream_t as void*.
+ * Errors found on the GPU (corrupt tiles) are not returned here: read them with
+ * ep_decode_status().  Returns EP_ERR_ARG, EP_ERR_SHAPE, EP_ERR_DTYPE, EP_ERR_CUDA, EP_ERR_OOM.
+ * Not thread-safe for concurrent first calls on the same blob and device.
+ */
+int ep_decompress(const ep_blob* b, const ep_tensor* out, void* stream);
+
+/* Stored bits per element: 8 * (stored bytes including metadata) / (rows * cols)
+ * ("EntroPack lattice compression", section "Encoding and reconstruction": "The actual_bpp
+ * property reports the actual stored bytes, including metadata, divided by the element count
+ * and multiplied by eight").  Returns -1.0 for a NULL blob. */
+double ep_actual_bpp(const ep_blob* b);
+
+/* Header fields of the blob. */
+int ep_get_info(const ep_blob* b, ep_blob_info* info);
+
+/* A view of the serialised bytes, valid until ep_blob_free(b). */
+int ep_blob_to_bytes(const ep_blob* b, const uint8_t** data, size_t* n);
+
+/* Copy and validate serialised bytes (header, sections, tables, tile offsets) into a new blob.
+ * Returns EP_ERR_CORRUPT with a reason when the bytes are not a valid blob. */
+int ep_blob_from_bytes(const uint8_t* data, size_t n, ep_blob** out);
+
+/* Copy the blob to `device` now (otherwise the first ep_decompress does it), on `stream`,
+ * and wait for the copy.  Lets a caller keep allocation out of a timed or captured region. */
+int ep_blob_prepare(ep_blob* b, int device, void* stream);
+
+/* Synchronise `stream`, then read and clear the blob's device status word on the current
+ * device.  Returns EP_OK when every decode since the last call found consistent tiles, else
+ * EP_ERR_CORRUPT with the failing checks in ep_last_error() (tile overrun, final rANS state
+ * not 2^16, unused words, bad tile extent, bulk-copy wait limit). */
+int ep_decode_status(const ep_blob* b, void* stream);
+
+/* Test hook: decode the fields of every vector into device memory `fields` (int16, n_vectors
+ * x 9: column 0 the coset bit, columns 1..8 the fields f1..f8), asynchronously on `stream`.
+ * Same kernel as ep_decompress up to the field inversion. */
+int ep_decode_fields(const ep_blob* b, int16_t* fields, void* stream);
+
+/* Release a blob, its host bytes and any device copies (synchronises those devices). */
+void ep_blob_free(ep_blob* b);
+
+/* Message for the last failure on the calling thread ("" if none). */
+const char* ep_last_error(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* ENTROPACK_H */

@@ -933,10 +933,11 @@ static int parse_blob(const uint8_t* b, uint64_t len, parsed* P)
     return 0;
 }
 
-/* Decode tiles [t0, t1) to symbols.  Returns 0, or a negative code / 1 for an inconsistent tile. */
+/* Decode tiles [t0, t1) to symbols.  sym9 / raw8 hold the vectors of those tiles only (vector
+ * t0 * 32S is element 0).  Returns 0, or a negative code for an inconsistent tile. */
 static int decode_tiles_to_symbols(const parsed* P, int64_t t0, int64_t t1, uint8_t* sym9, int16_t* raw8)
 {
-    int64_t per_tile = 32 * P->S;
+    int64_t per_tile = 32 * P->S, base = t0 * per_tile;
     dtables* T = (dtables*)malloc(sizeof(dtables));
     if (!T) return -2;
     build_dtables(P->q17, T);
@@ -945,7 +946,7 @@ static int decode_tiles_to_symbols(const parsed* P, int64_t t0, int64_t t1, uint
         uint64_t a = 16u * (uint64_t)get32(P->offs + 4 * t), e = 16u * (uint64_t)get32(P->offs + 4 * (t + 1));
         if (e < a || e > P->stream_bytes) { out = -6; break; }
         int64_t v0 = t * per_tile, nv = P->V - v0 < per_tile ? P->V - v0 : per_tile;
-        int rc = decode_tile(P->stream + a, e - a, nv, T, sym9 + 9 * v0, raw8 + 8 * v0, NULL);
+        int rc = decode_tile(P->stream + a, e - a, nv, T, sym9 + 9 * (v0 - base), raw8 + 8 * (v0 - base), NULL);
         if (rc) { out = rc < 0 ? -7 : -8; break; }
     }
     free(T);
@@ -961,16 +962,17 @@ int orc_decode_fields(const uint8_t* blob, uint64_t len, int64_t t0, int64_t t1,
     if (rc) return rc;
     if (t1 < 0 || t1 > P.ntiles) t1 = P.ntiles;
     if (t0 < 0 || t0 > t1) return -1;
-    uint8_t* sym9 = (uint8_t*)calloc((size_t)P.V * 9, 1);
-    int16_t* raw8 = (int16_t*)calloc((size_t)P.V * 8, sizeof(int16_t));
+    int64_t v0 = t0 * 32 * P.S, v1 = t1 * 32 * P.S < P.V ? t1 * 32 * P.S : P.V;
+    uint8_t* sym9 = (uint8_t*)calloc((size_t)(v1 - v0) * 9 + 9, 1);
+    int16_t* raw8 = (int16_t*)calloc((size_t)(v1 - v0) * 8 + 8, sizeof(int16_t));
     rc = decode_tiles_to_symbols(&P, t0, t1, sym9, raw8);
     if (rc == 0) {
-        int64_t v0 = t0 * 32 * P.S, v1 = t1 * 32 * P.S < P.V ? t1 * 32 * P.S : P.V;
         for (int64_t v = v0; v < v1; v++) {
-            fields[9 * v] = sym9[9 * v];
+            const uint8_t* sy9 = sym9 + 9 * (v - v0);
+            fields[9 * v] = sy9[0];
             for (int j = 1; j <= 8; j++) {
-                int sy = sym9[9 * v + j];
-                fields[9 * v + j] = (int16_t)(sy == ORC_ESC ? raw8[8 * v + j - 1] : sy - ORC_R);
+                int sy = sy9[j];
+                fields[9 * v + j] = (int16_t)(sy == ORC_ESC ? raw8[8 * (v - v0) + j - 1] : sy - ORC_R);
             }
         }
     }
@@ -993,19 +995,20 @@ int orc_decompress_tiles(const uint8_t* blob, uint64_t len, int64_t t0, int64_t 
     if (dtype_size(dtype_out) == 0) return -1;
     if (t1 < 0 || t1 > P.ntiles) t1 = P.ntiles;
     if (t0 < 0 || t0 > t1) return -1;
-    uint8_t* sym9 = (uint8_t*)calloc((size_t)P.V * 9, 1);
-    int16_t* raw8 = (int16_t*)calloc((size_t)P.V * 8, sizeof(int16_t));
+    int64_t v0 = t0 * 32 * P.S, v1 = t1 * 32 * P.S < P.V ? t1 * 32 * P.S : P.V;
+    uint8_t* sym9 = (uint8_t*)calloc((size_t)(v1 - v0) * 9 + 9, 1);
+    int16_t* raw8 = (int16_t*)calloc((size_t)(v1 - v0) * 8 + 8, sizeof(int16_t));
     rc = decode_tiles_to_symbols(&P, t0, t1, sym9, raw8);
     if (rc == 0) {
-        int64_t v0 = t0 * 32 * P.S, v1 = t1 * 32 * P.S < P.V ? t1 * 32 * P.S : P.V;
         for (int64_t v = v0; v < v1; v++) {
             int64_t r = v / P.vpr, k = v % P.vpr;
             int32_t f[8];
             double y[8];
-            int c = sym9[9 * v];
+            const uint8_t* sy9 = sym9 + 9 * (v - v0);
+            int c = sy9[0];
             for (int j = 1; j <= 8; j++) {
-                int sy = sym9[9 * v + j];
-                f[j - 1] = sy == ORC_ESC ? raw8[8 * v + j - 1] : sy - ORC_R;
+                int sy = sy9[j];
+                f[j - 1] = sy == ORC_ESC ? raw8[8 * (v - v0) + j - 1] : sy - ORC_R;
             }
             orc_fields_to_point(c, f, y);
             float a;

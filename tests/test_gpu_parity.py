@@ -1,0 +1,276 @@
+"""GPU parity: the CUDA decode against the oracle, through the C ABI.
+
+Bars (per element):
+  * fields (coset bit, f1..f8) bit-exact;
+  * restored values within 1 ulp of the output container -- both sides compute the same IEEE
+    sequence (fp32 product of the fp32 row scale and the exact lattice coordinate, then one
+    round-to-nearest-even into the container), so the checks below require 0 ulp;
+  * relative L2 error against the input equal to the oracle's to 1e-6.
+Both cross directions: the GPU decodes oracle-encoded blobs, and (host suite) the oracle decodes
+library-encoded blobs.  Full-size workloads compare every element where the oracle finishes in
+seconds and sampled tiles (first, last, and seeded random ones) elsewhere.
+"""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+import workloads as W
+
+pytestmark = pytest.mark.gpu
+
+TORCH = {W.BF16: torch.bfloat16, W.FP16: torch.float16, W.E4M3: torch.float8_e4m3fn, W.F32: torch.float32}
+NP = {W.BF16: np.uint16, W.FP16: np.uint16, W.E4M3: np.uint8, W.F32: np.uint32}
+
+
+@pytest.fixture(scope="module")
+def ep():
+    if not torch.cuda.is_available():
+        pytest.skip("no CUDA device")
+    from dit_weight_compression_b200 import build
+    build.build()
+    import dit_weight_compression_b200 as ep
+    return ep
+
+
+def _bits(t: torch.Tensor, dtype: int) -> np.ndarray:
+    v = {1: torch.int16, 2: torch.int16, 3: torch.uint8, 4: torch.int32}[dtype]
+    return t.contiguous().view(v).cpu().numpy().view(NP[dtype])
+
+
+def _ulp(a: np.ndarray, b: np.ndarray, dtype: int) -> np.ndarray:
+    """Distance in units in the last place between two arrays of container bit patterns."""
+    nb = {1: 16, 2: 16, 3: 8, 4: 32}[dtype]
+    def key(x):
+        x = x.astype(np.int64)
+        sign = 1 << (nb - 1)
+        return np.where(x & sign, -(x & (sign - 1)), x)
+    return np.abs(key(a) - key(b))
+
+
+def _rel_l2(bits, dtype, ref):
+    x = oracle.dtype_to_f64(bits, dtype)
+    return np.linalg.norm(x - ref) / np.linalg.norm(ref)
+
+
+def _gpu_decode(ep, c, dtype=None, **kw):
+    out = ep.decompress(c, dtype=TORCH[dtype] if dtype else None, **kw)
+    torch.cuda.synchronize()
+    ep.decode_status(c)
+    return out
+
+
+def _check_full(ep, blob: bytes, m: W.Matrix, out_dtypes=None):
+    """Every field and every element against the oracle."""
+    c = ep.CompressedTensor.from_bytes(blob)
+    f_gpu = ep.decode_fields(c).cpu().numpy()
+    ep.decode_status(c)
+    assert np.array_equal(f_gpu, oracle.decode_fields(blob))
+    ref = oracle.dtype_to_f64(m.bits, m.dtype)
+    for dt in out_dtypes or [m.dtype]:
+        g = _bits(_gpu_decode(ep, c, dt), dt)
+        o = oracle.decompress(blob, dt)
+        assert g.shape == o.shape
+        assert _ulp(g, o, dt).max() <= 1
+        assert np.array_equal(g, o)
+        if dt != W.E4M3:
+            assert abs(_rel_l2(g, dt, ref) - _rel_l2(o, dt, ref)) <= 1e-6
+    return c
+
+
+def _tiles_sample(n_tiles, k=6, seed=0):
+    g = np.random.Generator(np.random.PCG64(seed))
+    pick = {0, n_tiles - 1} | set(g.integers(0, n_tiles, k).tolist())
+    return sorted(pick)
+
+
+def _check_sampled(ep, c, m: W.Matrix, out_dtypes=None, seed=0):
+    """Sampled tiles of a full-size blob against the oracle (the oracle decodes a tile at a time)."""
+    blob = c.to_bytes()
+    info = oracle.blob_info(blob)
+    tiles = _tiles_sample(info["n_tiles"], seed=seed)
+    per = 32 * info["S"]
+    vpr = (info["cols"] + 7) // 8
+    f_gpu = ep.decode_fields(c).cpu().numpy()
+    ep.decode_status(c)
+    for dt in out_dtypes or [m.dtype]:
+        g = _bits(_gpu_decode(ep, c, dt), dt)
+        o = np.zeros_like(g)
+        for t in tiles:
+            oracle.decompress_tiles(blob, t, t + 1, dt, o)
+        for t in tiles:
+            v0, v1 = t * per, min((t + 1) * per, info["V"])
+            r0, r1 = v0 // vpr, (v1 - 1) // vpr + 1
+            # whole rows fully inside the tile compare directly; partial rows by element mask
+            mask = np.zeros(g.shape, bool)
+            vv = np.arange(v0, v1)
+            rr, kk = vv // vpr, vv % vpr
+            for i in range(8):
+                col = 8 * kk + i
+                ok = col < info["cols"]
+                mask[rr[ok], col[ok]] = True
+            assert np.array_equal(g[mask], o[mask]), (t, dt)
+            del r0, r1
+    fo = np.zeros_like(f_gpu)
+    for t in tiles:
+        v0, v1 = t * per, min((t + 1) * per, info["V"])
+        fo[v0:v1] = oracle.decode_fields(blob, t, t + 1)[v0:v1]
+        assert np.array_equal(f_gpu[v0:v1], fo[v0:v1])
+
+
+# ---------------------------------------------------------------------------------------------
+# GPU decodes oracle-encoded blobs (cross direction 1), every element.
+# ---------------------------------------------------------------------------------------------
+
+def test_small_oracle_blob_all_containers(ep):
+    m = W.small()
+    blob = oracle.compress(m.bits, m.dtype, m.target_bpp)
+    _check_full(ep, blob, m, [W.BF16, W.FP16, W.E4M3, W.F32])
+
+
+def test_square_full_size_oracle_blob(ep):
+    m = W.square()
+    blob = oracle.compress(m.bits, m.dtype, m.target_bpp)
+    _check_full(ep, blob, m)
+
+
+@pytest.mark.parametrize("S", [1, 2, 3, 16, 33, 1024])
+def test_steps_per_tile_and_partial_tiles(ep, S):
+    m = W.square(rows=97, cols=1000)
+    blob = oracle.compress(m.bits, m.dtype, 4.0, steps_per_tile=S)
+    _check_full(ep, blob, m, [W.BF16, W.F32])
+
+
+@pytest.mark.parametrize("shape", [(1, 1), (1, 8), (3, 13), (7, 9), (33, 7), (5, 1000), (17, 4100)])
+def test_ragged_shapes(ep, shape):
+    g = np.random.Generator(np.random.PCG64(shape[0] * 1000 + shape[1]))
+    m = W.Matrix(W.to_bf16_bits(g.normal(0, 0.02, shape)), W.BF16, 3.0)
+    blob = oracle.compress(m.bits, m.dtype, m.target_bpp)
+    _check_full(ep, blob, m, [W.BF16, W.FP16, W.E4M3, W.F32])
+
+
+@pytest.mark.parametrize("rate", [0.5, 2.0, 11.0])
+def test_rate_extremes_oracle_blob(ep, rate):
+    m = W.sweep(rate, rows=128, cols=1376)
+    blob = oracle.compress(m.bits, m.dtype, rate)
+    _check_full(ep, blob, m)
+
+
+def test_degenerate_tables(ep):
+    # constant rows: lone symbols (q = 4096) in most contexts; a zero row; FP16 input
+    g = np.random.Generator(np.random.PCG64(5))
+    x = g.normal(0, 0.05, (64, 1)) * np.ones((1, 1024))
+    x[3] = 0.0
+    m = W.Matrix(W.to_fp16_bits(x), W.FP16, 4.0)
+    blob = oracle.compress(m.bits, m.dtype, m.target_bpp)
+    _check_full(ep, blob, m)
+    z = W.Matrix(W.to_bf16_bits(np.zeros((40, 64))), W.BF16, 1.0)
+    blob = oracle.compress(z.bits, z.dtype, z.target_bpp)
+    _check_full(ep, blob, z)
+
+
+# ---------------------------------------------------------------------------------------------
+# Library-encoded blobs at full workload sizes (the oracle decodes sampled tiles).
+# ---------------------------------------------------------------------------------------------
+
+def test_dit_set_full_size(ep):
+    for j in range(len(W.DIT_SHAPES)):
+        m = W.dit(j)
+        c = ep.compress(W.bits_to_torch(m.bits, m.dtype), m.target_bpp)
+        _check_sampled(ep, c, m, seed=j)
+
+
+@pytest.mark.parametrize("rate", W.SWEEP_RATES)
+def test_sweep_full_size(ep, rate):
+    m = W.sweep(rate)
+    c = ep.compress(W.bits_to_torch(m.bits, m.dtype), rate)
+    _check_sampled(ep, c, m, seed=int(rate * 10))
+
+
+def test_large_layer_full_size_bf16_and_fp8(ep):
+    m = W.large(0)
+    c = ep.compress(W.bits_to_torch(m.bits, m.dtype), m.target_bpp)
+    _check_sampled(ep, c, m, [W.BF16, W.E4M3])
+    # whole-tensor property at full size: the GPU's rel-L2 matches the blob's lattice error
+    out = _gpu_decode(ep, c)
+    x = W.bits_to_torch(m.bits, m.dtype).cuda().float()
+    rel = ((out.float() - x).norm() / x.norm()).item()
+    assert 0.01 < rel < 0.12, rel
+
+
+# ---------------------------------------------------------------------------------------------
+# Output layouts, streams, the end-to-end host path, and corruption reporting.
+# ---------------------------------------------------------------------------------------------
+
+def test_strided_and_misaligned_outputs(ep):
+    m = W.square(rows=64, cols=512)
+    blob = oracle.compress(m.bits, m.dtype, 4.0)
+    c = ep.CompressedTensor.from_bytes(blob)
+    ref = oracle.decompress(blob, W.BF16)
+    big = torch.zeros((64, 520), dtype=torch.bfloat16, device="cuda")
+    ep.decompress(c, out=big[:, :512])                      # row stride 520 (vector stores)
+    big2 = torch.zeros((64, 515), dtype=torch.bfloat16, device="cuda")
+    ep.decompress(c, out=big2[:, 1:513])                    # misaligned: element stores
+    torch.cuda.synchronize()
+    ep.decode_status(c)
+    assert np.array_equal(_bits(big[:, :512], W.BF16), ref)
+    assert np.array_equal(_bits(big2[:, 1:513], W.BF16), ref)
+    assert torch.count_nonzero(big[:, 512:]) == 0 and torch.count_nonzero(big2[:, 0]) == 0
+
+
+def test_host_output_path_matches_device_path(ep):
+    m = W.square(rows=256, cols=1024)
+    c = ep.compress(W.bits_to_torch(m.bits, m.dtype), 4.0)
+    dev = _bits(_gpu_decode(ep, c), W.BF16)
+    host = torch.empty((256, 1024), dtype=torch.bfloat16).pin_memory()
+    ep.decompress(c, out=host)
+    assert np.array_equal(_bits(host, W.BF16), dev)
+    ep.decode_status(c)
+
+
+def test_side_stream(ep):
+    m = W.small()
+    c = ep.compress(W.bits_to_torch(m.bits, m.dtype), m.target_bpp)
+    s = torch.cuda.Stream()
+    c.prepare(stream=s)
+    with torch.cuda.stream(s):
+        out = ep.decompress(c, stream=s)
+    s.synchronize()
+    assert np.array_equal(_bits(out, W.BF16), oracle.decompress(c.to_bytes()))
+
+
+def test_corrupt_stream_reported_not_hung(ep):
+    """Flip bits inside tile payloads (the blob still passes host validation): the kernel must
+    finish, flag the status word, and leave the context usable."""
+    m = W.square(rows=128, cols=1024)
+    b = bytearray(ep.compress(W.bits_to_torch(m.bits, m.dtype), 4.0).to_bytes())
+    off_stream = int.from_bytes(b[72:80], "little")
+    for pos in (off_stream + 200, off_stream + 3000, len(b) - 40):
+        b[pos] ^= 0x5A
+    c = ep.CompressedTensor.from_bytes(bytes(b))
+    out = ep.decompress(c)
+    torch.cuda.synchronize()
+    with pytest.raises(ep.EPError) as e:
+        ep.decode_status(c)
+    assert e.value.code == -5
+    # the context still works and the status word was cleared
+    good = ep.compress(W.bits_to_torch(m.bits, m.dtype), 4.0)
+    ep.decompress(good)
+    ep.decode_status(good)
+    del out
+
+
+def test_rel_l2_matches_oracle_usage_example(ep):
+    """The pages' usage example: 256 x 256 BF16 N(0, 0.02^2) at 3.5 bpp; restored shape and
+    dtype equal the input's; stored rate and relative L2 error as the oracle reports them."""
+    m = W.small()
+    t = W.bits_to_torch(m.bits, m.dtype).cuda()
+    cfg = ep.LatticeRANSConfig(target_bpp=3.5)
+    comp = ep.compress(t, cfg)
+    restored = ep.decompress(comp, cfg)
+    assert restored.shape == t.shape and restored.dtype == t.dtype
+    rel = ((restored.float() - t.float()).norm() / t.float().norm()).item()
+    blob = comp.to_bytes()
+    rel_o = _rel_l2(oracle.decompress(blob), W.BF16, oracle.dtype_to_f64(m.bits, m.dtype))
+    assert abs(rel - rel_o) <= 1e-6
+    assert comp.actual_bpp == oracle.actual_bpp(blob)
