@@ -345,9 +345,10 @@ __global__ void __launch_bounds__(WARPS * 32, (WARPS >= 32 ? 1 : 2048 / (WARPS *
     uint32_t tile = blockIdx.x + gridDim.x * warp;
     uint32_t seq = 0;  // chunks this warp has issued so far: chunk g uses slot g % 4, parity (g / 4) % 2
 
-    // per-tile cursor state
+    // per-tile cursor state; chunk j of a tile lives in ring slot (g0 + j) % 4, so the tile's
+    // byte 0 sits at ring offset rofs = (g0 % 4) * 512 and ring positions are rofs + offset
     const uint8_t* src = nullptr;
-    uint32_t bytes = 0, nch = 0, issued = 0, waited = 0, g0 = 0, x = 0;
+    uint32_t bytes = 0, nch = 0, issued = 0, waited = 0, g0 = 0, rofs = 0, x = 0;
 
     auto issue = [&](uint32_t j) {
         const uint32_t g = g0 + j, slot = g & (kRingChunks - 1);
@@ -370,6 +371,7 @@ __global__ void __launch_bounds__(WARPS * 32, (WARPS >= 32 ? 1 : 2048 / (WARPS *
         nch = (bytes + kChunk - 1) / kChunk;
         g0 = seq;
         seq += nch;
+        rofs = (g0 & (kRingChunks - 1)) * kChunk;
         issued = waited = 0;
         while (issued < min(nch, uint32_t(kRingChunks))) issue(issued++);
         x = __ldg(reinterpret_cast<const uint32_t*>(p.stream + t0) + lane);
@@ -389,13 +391,14 @@ __global__ void __launch_bounds__(WARPS * 32, (WARPS >= 32 ? 1 : 2048 / (WARPS *
         const uint32_t nsteps = uint32_t((vend - v0 + kLanes - 1) / kLanes);
         int64_t v = v0 + lane;
         int64_t row = v / p.vec_per_row, kcol = v - row * p.vec_per_row;
-        uint32_t cur = 0;
+        uint32_t cur = rofs;  // ring position of the next unread byte
         uint32_t flags = 0;
         for (uint32_t k = 0; k < nsteps; ++k) {
             // keep the ring full and the bytes this step may read resident
-            const uint32_t lim = min(nch, cur / kChunk + kRingChunks);
+            const uint32_t done = cur - rofs;  // bytes of this tile consumed so far
+            const uint32_t lim = min(nch, done / kChunk + kRingChunks);
             while (issued < lim) issue(issued++);
-            const uint32_t need = (min(bytes, cur + uint32_t(kMaxStepBytes)) + kChunk - 1) / kChunk;
+            const uint32_t need = (min(bytes, done + uint32_t(kMaxStepBytes)) + kChunk - 1) / kChunk;
             while (waited < need) {
                 if (!wait(waited)) goto timeout;
                 ++waited;
@@ -404,7 +407,7 @@ __global__ void __launch_bounds__(WARPS * 32, (WARPS >= 32 ? 1 : 2048 / (WARPS *
                 decode_step<WARPS, OUT, VEC, true>(sm, p, ring, x, cur, true, lt, v, row, kcol);
             else
                 decode_step<WARPS, OUT, VEC, false>(sm, p, ring, x, cur, v < vend, lt, v, row, kcol);
-            if (cur > bytes) {
+            if (cur - rofs > bytes) {
                 flags |= kStOverrun;
                 break;
             }
@@ -422,7 +425,7 @@ __global__ void __launch_bounds__(WARPS * 32, (WARPS >= 32 ? 1 : 2048 / (WARPS *
         }
         if (!(flags & kStOverrun)) {
             if (__any_sync(kFull, x != kStateLow)) flags |= kStState;
-            if (bytes - cur >= 16) flags |= kStLeftover;
+            if (bytes - (cur - rofs) >= 16) flags |= kStLeftover;
         }
         if (lane == 0 && flags) atomicOr(p.status, flags);
     }

@@ -73,7 +73,7 @@ def _check_full(ep, blob: bytes, m: W.Matrix, out_dtypes=None):
         assert g.shape == o.shape
         assert _ulp(g, o, dt).max() <= 1
         assert np.array_equal(g, o)
-        if dt != W.E4M3:
+        if dt != W.E4M3 and np.linalg.norm(ref) > 0:   # (an all-zero input has no relative error)
             assert abs(_rel_l2(g, dt, ref) - _rel_l2(o, dt, ref)) <= 1e-6
     return c
 
@@ -100,8 +100,6 @@ def _check_sampled(ep, c, m: W.Matrix, out_dtypes=None, seed=0):
             oracle.decompress_tiles(blob, t, t + 1, dt, o)
         for t in tiles:
             v0, v1 = t * per, min((t + 1) * per, info["V"])
-            r0, r1 = v0 // vpr, (v1 - 1) // vpr + 1
-            # whole rows fully inside the tile compare directly; partial rows by element mask
             mask = np.zeros(g.shape, bool)
             vv = np.arange(v0, v1)
             rr, kk = vv // vpr, vv % vpr
@@ -110,7 +108,6 @@ def _check_sampled(ep, c, m: W.Matrix, out_dtypes=None, seed=0):
                 ok = col < info["cols"]
                 mask[rr[ok], col[ok]] = True
             assert np.array_equal(g[mask], o[mask]), (t, dt)
-            del r0, r1
     fo = np.zeros_like(f_gpu)
     for t in tiles:
         v0, v1 = t * per, min((t + 1) * per, info["V"])
@@ -139,6 +136,16 @@ def test_steps_per_tile_and_partial_tiles(ep, S):
     m = W.square(rows=97, cols=1000)
     blob = oracle.compress(m.bits, m.dtype, 4.0, steps_per_tile=S)
     _check_full(ep, blob, m, [W.BF16, W.F32])
+
+
+@pytest.mark.parametrize("S,rate", [(1, 11.0), (2, 4.0), (1, 0.5)])
+def test_many_tiles_per_warp(ep, S, rate):
+    """More tiles than resident warps (148 SMs x 32 warps), so warps decode several tiles in a
+    row and a tile's first chunk lands in any of the four ring slots."""
+    m = W.sweep(rate, rows=2400, cols=1024)
+    blob = oracle.compress(m.bits, m.dtype, rate, steps_per_tile=S)
+    assert oracle.blob_info(blob)["n_tiles"] > 148 * 32
+    _check_full(ep, blob, m)
 
 
 @pytest.mark.parametrize("shape", [(1, 1), (1, 8), (3, 13), (7, 9), (33, 7), (5, 1000), (17, 4100)])
