@@ -11,18 +11,27 @@
 namespace ep {
 
 static thread_local std::string g_error;
+static thread_local const char* g_static_error = nullptr;  // set by paths that must not allocate
 
 int set_error(int code, const std::string& msg) {
+    g_static_error = nullptr;
     g_error = msg;
     return code;
 }
-void clear_error() { g_error.clear(); }
+int set_error_static(int code, const char* msg) {
+    g_static_error = msg;
+    return code;
+}
+void clear_error() {
+    g_static_error = nullptr;
+    g_error.clear();
+}
 
 }  // namespace ep
 
 using namespace ep;
 
-extern "C" const char* ep_last_error(void) { return g_error.c_str(); }
+extern "C" const char* ep_last_error(void) { return g_static_error ? g_static_error : g_error.c_str(); }
 
 extern "C" int ep_compress_ex(const ep_tensor* in, double target_bpp, const ep_options* opt, ep_blob** out) {
     clear_error();

@@ -23,6 +23,7 @@ struct DeviceCopy {
 };
 
 int set_error(int code, const std::string& msg);
+int set_error_static(int code, const char* msg);  // msg must be a string literal; no allocation
 void clear_error();
 
 }  // namespace ep

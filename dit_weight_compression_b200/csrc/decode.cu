@@ -35,6 +35,12 @@
 
 #include "blob.h"
 
+// Scratch of ep_decompress_noalloc: a fixed 256-byte array on every device that loads this
+// library, held until the process exits.  Host code must not use this name as an address; the
+// entry point looks up its device address with cudaGetSymbolAddress.
+#define EP_NOALLOC_SCRATCH_WORDS 64
+static __device__ __align__(256) uint32_t ep_noalloc_scratch[EP_NOALLOC_SCRATCH_WORDS];
+
 namespace ep {
 namespace {
 
@@ -567,6 +573,58 @@ bool vec_ok(const BlobLayout& L, const void* out, int64_t row_stride, int dtype)
     return L.cols % 8 == 0 && row_stride % 8 == 0 && (reinterpret_cast<uintptr_t>(out) % align) == 0;
 }
 
+// ---- allocation-free decode (ep_decompress_noalloc) -------------------------------------------
+// The decode kernel's only scratch is its 4-byte status word.  For callers that may not allocate,
+// that word lives in the file-scope array below instead of blob-owned device memory.
+constexpr int kNoallocScratchWords = EP_NOALLOC_SCRATCH_WORDS;  // 256 bytes; a launch uses word 0
+
+struct NoallocDevice {
+    bool ready = false;
+    uint32_t* scratch = nullptr;  // device address of ep_noalloc_scratch on this device
+    int sms = 0;
+};
+NoallocDevice g_noalloc[kMaxDevices];
+std::mutex g_noalloc_mu;
+
+template <int WARPS, int OUT, bool VEC>
+int noalloc_launch_one(const Params& p, cudaStream_t st, int device) {
+    auto fn = decode_kernel<WARPS, OUT, VEC>;
+    const size_t smem = sizeof(Smem<WARPS>);
+    static std::mutex mu;
+    static int per_sm[kMaxDevices] = {};
+    {
+        std::lock_guard<std::mutex> g(mu);
+        if (per_sm[device] == 0) {
+            if (cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, int(smem)) != cudaSuccess)
+                return set_error_static(EP_ERR_CUDA, "ep_decompress_noalloc: cannot set the kernel's shared memory size");
+            int n = 0;
+            if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, fn, WARPS * 32, smem) != cudaSuccess || n < 1)
+                return set_error_static(EP_ERR_CUDA, "ep_decompress_noalloc: decode kernel does not fit on an SM");
+            per_sm[device] = n;
+        }
+    }
+    const uint32_t grid = uint32_t(std::min<int64_t>(int64_t(g_noalloc[device].sms) * per_sm[device], p.n_tiles));
+    fn<<<grid, WARPS * 32, smem, st>>>(p);
+    if (cudaGetLastError() != cudaSuccess)
+        return set_error_static(EP_ERR_CUDA, "ep_decompress_noalloc: kernel launch failed");
+    return EP_OK;
+}
+
+template <int OUT>
+int noalloc_launch_out(const Params& p, bool vec, cudaStream_t st, int device) {
+    return vec ? noalloc_launch_one<kWarps, OUT, true>(p, st, device)
+               : noalloc_launch_one<kWarps, OUT, false>(p, st, device);
+}
+
+int noalloc_launch(const Params& p, int out_kind, bool vec, cudaStream_t st, int device) {
+    switch (out_kind) {
+        case kOutBF16: return noalloc_launch_out<kOutBF16>(p, vec, st, device);
+        case kOutFP16: return noalloc_launch_out<kOutFP16>(p, vec, st, device);
+        case kOutE4M3: return noalloc_launch_out<kOutE4M3>(p, vec, st, device);
+        default: return noalloc_launch_out<kOutF32>(p, vec, st, device);
+    }
+}
+
 }  // namespace
 }  // namespace ep
 
@@ -704,4 +762,57 @@ extern "C" void ep_blob_free(ep_blob* b) {
     if (b->host_pinned) cudaHostUnregister(b->bytes.data());
     cudaSetDevice(prev);
     delete b;
+}
+
+extern "C" int ep_decompress_noalloc(const ep_blob* cb, const void* device_blob, const ep_tensor* out,
+                                     void* stream, int wait) {
+    clear_error();
+    if (!cb || !device_blob || !out || !out->data)
+        return set_error_static(EP_ERR_ARG, "ep_decompress_noalloc: NULL argument");
+    const BlobLayout& L = cb->layout;
+    const int kind = out_kind_of(out->dtype);
+    if (kind < 0) return set_error_static(EP_ERR_DTYPE, "ep_decompress_noalloc: unsupported output dtype");
+    if (out->rows != L.rows || out->cols != L.cols)
+        return set_error_static(EP_ERR_SHAPE, "ep_decompress_noalloc: output shape differs from the blob's");
+    if (out->row_stride < out->cols)
+        return set_error_static(EP_ERR_ARG, "ep_decompress_noalloc: row_stride < cols");
+    if (reinterpret_cast<uintptr_t>(device_blob) % 16 != 0)
+        return set_error_static(EP_ERR_ARG, "ep_decompress_noalloc: device_blob must be 16-byte aligned");
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices)
+        return set_error_static(EP_ERR_CUDA, "ep_decompress_noalloc: no usable current device");
+    if (out->device != dev)
+        return set_error_static(EP_ERR_ARG, "ep_decompress_noalloc: output must be device memory on the current device");
+    // One status word per launch; the array holds kNoallocScratchWords.
+    constexpr int kWordsNeeded = 1;
+    static_assert(kWordsNeeded <= kNoallocScratchWords, "scratch array too small");
+    {
+        // first call on this device: find the array's device address (with this device current)
+        std::lock_guard<std::mutex> g(g_noalloc_mu);
+        NoallocDevice& nd = g_noalloc[dev];
+        if (!nd.ready) {
+            void* ptr = nullptr;
+            if (cudaGetSymbolAddress(&ptr, ep_noalloc_scratch) != cudaSuccess || !ptr)
+                return set_error_static(EP_ERR_CUDA, "ep_decompress_noalloc: cudaGetSymbolAddress failed");
+            if (cudaDeviceGetAttribute(&nd.sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
+                return set_error_static(EP_ERR_CUDA, "ep_decompress_noalloc: cannot read the SM count");
+            nd.scratch = static_cast<uint32_t*>(ptr);
+            nd.ready = true;
+        }
+    }
+    uint32_t* status = g_noalloc[dev].scratch;
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    // the status word must start at zero for this call
+    if (cudaMemsetAsync(status, 0, sizeof(uint32_t) * kWordsNeeded, st) != cudaSuccess)
+        return set_error_static(EP_ERR_CUDA, "ep_decompress_noalloc: clearing the status word failed");
+    const bool vec = vec_ok(L, out->data, out->row_stride, out->dtype);
+    Params p = make_params(cb, static_cast<const uint8_t*>(device_blob), out->data, out->row_stride, status, vec);
+    int rc = noalloc_launch(p, kind, vec, st, dev);
+    if (rc != EP_OK || !wait) return rc;
+    uint32_t s = 0;
+    if (cudaMemcpyAsync(&s, status, sizeof s, cudaMemcpyDeviceToHost, st) != cudaSuccess ||
+        cudaStreamSynchronize(st) != cudaSuccess)
+        return set_error_static(EP_ERR_CUDA, "ep_decompress_noalloc: reading the status word failed");
+    if (s != 0) return set_error_static(EP_ERR_CORRUPT, "ep_decompress_noalloc: GPU decode found a corrupt blob");
+    return EP_OK;
 }

@@ -147,6 +147,34 @@ int ep_decode_status(const ep_blob* b, void* stream);
  * Same kernel as ep_decompress up to the field inversion. */
 int ep_decode_fields(const ep_blob* b, int16_t* fields, void* stream);
 
+/*
+ * Decode like ep_decompress, but allocate nothing -- no cudaMalloc, no host or device heap
+ * allocation by the library.  (The method's pages have no counterpart: this is an interface for
+ * callers that cannot let a library allocate GPU memory -- an inference runtime that plans all
+ * device memory ahead of time in its own arena, or code running where allocation is forbidden or
+ * would synchronise the device.)
+ *   b            blob handle; only its parsed header is used (its host bytes are not read).
+ *   device_blob  the blob's serialised bytes (ep_blob_to_bytes) already in device memory on the
+ *                current device, owned by the caller, 16-byte aligned.
+ *   out          device output on the current device, as for ep_decompress.
+ *   stream       cudaStream_t as void*.
+ *   wait         0: return after the launch (asynchronous, the kernel's corruption checks are
+ *                not reported); nonzero: synchronise `stream` and return EP_ERR_CORRUPT if the
+ *                decode found a corrupt tile.
+ * The decode kernel's scratch -- one 4-byte status word -- lives in a fixed 256-byte array of
+ * device memory inside this library (64 words; every GPU that loads the library keeps it until
+ * the process exits).  Each call clears the word it uses; a call whose scratch need exceeded the
+ * array would be rejected with EP_ERR_ARG (no current launch needs more than one word).  All
+ * calls share the array, which keeps the last call's contents, so calls that overlap on the GPU
+ * (different streams, or several devices' host threads racing on one device) race on the status
+ * word: serialise them or use ep_decompress.  The first call on each device looks up the array's
+ * device address and sets the kernel's launch attributes; make that first call before any stream
+ * capture.  Returns EP_ERR_ARG, EP_ERR_SHAPE, EP_ERR_DTYPE, EP_ERR_CUDA, EP_ERR_CORRUPT; messages
+ * from this call never allocate.
+ */
+int ep_decompress_noalloc(const ep_blob* b, const void* device_blob, const ep_tensor* out, void* stream,
+                          int wait);
+
 /* Release a blob, its host bytes and any device copies (synchronises those devices). */
 void ep_blob_free(ep_blob* b);
 
