@@ -1,35 +1,40 @@
 // decode.cu -- fused GPU decompression for sm_100a, and the device-side entry points of the C ABI.
 //
 // "EntroPack lattice compression" (documentation page, section "Encoding and reconstruction"):
-// "Decoding recovers the fields, reconstructs lattice points, and applies the row scales in a
-// fused GPU operation. The result has the input's shape and dtype."  The arXiv abstract adds
-// that tiles are independently decodable, "enabling fast, fused symbol decoding and numerical
-// weight reconstruction on the GPU".
+// decoding recovers the fields, reconstructs lattice points and applies the row scales in one
+// fused GPU operation, and the result has the input's shape and dtype.  The arXiv abstract adds
+// that tiles are independently decodable, which is what lets the GPU decode them in parallel.
 //
 // One kernel does the whole path.  Work split:
 //   * one warp per tile; the tile's 32 interleaved rANS states live one per lane;
-//   * persistent CTAs (grid = min(#SM x resident CTAs, #tiles)); tile t goes to CTA t mod grid,
-//     so every SM gets an equal share even when there are few tiles;
-//   * each CTA first expands the blob's compact frequency tables into shared memory: per field
-//     context a 4096-entry slot->symbol byte table and a 256-entry (frequency | cumulative << 16)
-//     word table (80 KB in all); the coset context (two symbols) is decoded by one compare;
-//   * each warp streams its tile's word stream through a private 2 KB shared-memory ring of four
-//     512-byte chunks, filled by 1-D bulk copies (cp.async.bulk, no multicast) that complete on
-//     one mbarrier per chunk; every wait is bounded and reports through the status word;
-//   * per step a lane decodes one 8-vector: 9 rANS symbols, each followed by the renormalisation
-//     read whose word position is the warp-ballot prefix count of lanes refilling before it;
-//     escaped fields take raw words at the end of the step; fields are inverted in registers
-//     (z8 = 2 f8 + parity, y = z + c/2), multiplied by the row's fp32 scale, converted with one
-//     cvt per pair and written as one 16-byte store per lane (a 512-byte contiguous run per warp
-//     for BF16/FP16).
+//   * one persistent CTA of 32 warps per SM (grid = min(#SM, #tiles)); tile t goes to CTA
+//     t mod grid, so every SM gets an equal share even when there are few tiles;
+//   * decode tables: per field context a 4096-entry slot->symbol byte table and a 256-entry
+//     frequency / cumulative-frequency table pair of u16, 80 KB in all.  They are expanded once per blob
+//     and device by a small kernel into a block next to the device copy; every CTA stages that
+//     block into shared memory with bulk copies, overlapped with the fetch of its first tiles.
+//     (The allocation-free entry point expands them inside each CTA instead.)  The coset
+//     context, two symbols, is decoded by one compare;
+//   * each warp streams its tile's words through a private shared-memory ring of four 512-byte
+//     chunks filled by 1-D bulk copies (cp.async.bulk, no multicast) that complete on one
+//     mbarrier per chunk; the 1088 bytes after the ring (the most one step can read) mirror its
+//     start, so a step reads one linear window with no wrap-around arithmetic; every wait is
+//     bounded and reports through the status word;
+//   * per step a lane decodes one 8-vector: 9 rANS symbols, each followed by the
+//     renormalisation read whose word position is the warp-ballot prefix count of lanes
+//     refilling before it; escaped fields take raw words at the end of the step; fields are
+//     inverted in registers (z8 = 2 f8 + parity, y = z + c/2), multiplied by the row's fp32
+//     scale, converted one pair per cvt and written as one 16-byte store per lane (a 512-byte
+//     contiguous run per warp for BF16/FP16).
 // No tensor cores: the path is table lookups and integer arithmetic, bound by HBM bytes and by
-// issue slots, not by a contraction.
+// the latency and issue slots of that arithmetic, not by a contraction.
 #include <cuda_bf16.h>
 #include <cuda_fp16.h>
 #include <cuda_fp8.h>
 #include <cuda_runtime.h>
 
 #include <algorithm>
+#include <cstddef>
 #include <cstdio>
 #include <mutex>
 
@@ -45,11 +50,14 @@ namespace ep {
 namespace {
 
 constexpr uint32_t kFull = 0xFFFFFFFFu;
-constexpr int kChunk = 512;                                // bytes per bulk copy
+constexpr int kChunk = 512;                                   // bytes per bulk copy
 constexpr int kRingChunks = 4;
-constexpr int kRing = kChunk * kRingChunks;                // ring bytes per warp
-constexpr int kMaxStepBytes = 2 * (9 * kLanes + 8 * kLanes);  // words one step can consume
-constexpr uint32_t kWaitSpins = 1u << 22;                  // bounded mbarrier wait (~0.3 s)
+constexpr int kRing = kChunk * kRingChunks;                   // ring bytes per warp
+constexpr int kMaxStepBytes = 2 * (9 * kLanes + 8 * kLanes);  // bytes one step can consume (1088)
+constexpr int kMirror = kMaxStepBytes;                        // mirror of the ring's first bytes
+constexpr uint32_t kWaitSpins = 1u << 22;                     // bounded mbarrier wait (~0.3 s)
+constexpr uint32_t kTableBytes = kFieldContexts * (kProbTotal + 256 * 4);  // 81920
+constexpr uint32_t kTablePiece = 16384;                       // bytes per table bulk copy
 
 enum OutKind { kOutBF16 = 0, kOutFP16 = 1, kOutE4M3 = 2, kOutF32 = 3, kOutFields = 4 };
 
@@ -63,6 +71,7 @@ enum : uint32_t {
 
 struct Params {
     const uint8_t* blob;        // device copy of the serialised blob
+    const uint8_t* tables;      // expanded decode tables (kTableBytes), or null: expand in-kernel
     const uint32_t* tile_off;   // n_tiles + 1 offsets, 16-byte units
     const uint8_t* stream;      // stream section
     const float* alpha;         // per-row fp32 scales
@@ -80,11 +89,13 @@ struct Params {
 
 template <int WARPS>
 struct Smem {
-    uint8_t sym[kFieldContexts][kProbTotal];     // slot -> symbol
-    uint32_t fc[kFieldContexts][256];            // frequency | cumulative << 16
-    alignas(16) uint8_t ring[WARPS][kRing];      // per-warp stream ring
-    unsigned long long bar[WARPS][kRingChunks];  // one mbarrier per ring chunk
+    uint8_t sym[kFieldContexts][kProbTotal];        // slot -> symbol               } the 80 KB
+    uint16_t fc[kFieldContexts][2][256];            // [0] frequency, [1] cumulative } table block
+    alignas(16) uint8_t ring[WARPS][kRing + kMirror];  // per-warp stream ring (+ mirror)
+    unsigned long long bar[WARPS][kRingChunks];     // one mbarrier per ring chunk
+    unsigned long long tbar;                        // the table block's bulk copies
 };
+static_assert(offsetof(Smem<32>, ring) == kTableBytes, "table block must be contiguous");
 
 // ---- PTX wrappers ----------------------------------------------------------------------------
 __device__ __forceinline__ uint32_t smem_u32(const void* p) {
@@ -127,18 +138,36 @@ __device__ __forceinline__ bool mbar_wait(unsigned long long* bar, uint32_t pari
     return false;
 }
 
-__device__ __forceinline__ uint32_t ring_word(const uint8_t* ring, uint32_t pos) {
-    return *reinterpret_cast<const uint16_t*>(ring + (pos & (kRing - 1)));
+// Shared-memory loads at 32-bit shared-window addresses (plus a constant byte offset).
+template <int OFF = 0>
+__device__ __forceinline__ uint32_t lds_u8(uint32_t a) {
+    uint32_t v;
+    asm volatile("ld.shared.u8 %0, [%1+%2];" : "=r"(v) : "r"(a), "n"(OFF));
+    return v;
+}
+template <int OFF = 0>
+__device__ __forceinline__ uint32_t lds_u16(uint32_t a) {
+    uint32_t v;
+    asm volatile("ld.shared.u16 %0, [%1+%2];" : "=r"(v) : "r"(a), "n"(OFF));
+    return v;
+}
+template <int OFF = 0>
+__device__ __forceinline__ uint32_t lds_u32(uint32_t a) {
+    uint32_t v;
+    asm volatile("ld.shared.u32 %0, [%1+%2];" : "=r"(v) : "r"(a), "n"(OFF));
+    return v;
 }
 
 // Renormalisation after one decoded symbol: lanes whose state fell below 2^16 take the next
 // 16-bit words in ascending lane order (position = cursor + 2 * #refilling lanes below me).
-__device__ __forceinline__ void renorm(uint32_t& x, uint32_t& cur, const uint8_t* ring, uint32_t lt,
-                                       bool active) {
-    bool need = active && x < kStateLow;
-    uint32_t b = __ballot_sync(kFull, need);
-    if (need) x = (x << 16) | ring_word(ring, cur + 2u * __popc(b & lt));
-    cur += 2u * __popc(b);
+// `pos` is the shared address of the next unread word; within one step it only grows, and the
+// ring's mirror keeps every address of the step inside the ring allocation.
+__device__ __forceinline__ void renorm(uint32_t& x, uint32_t& pos, uint32_t lt, bool active) {
+    const bool need = active && x < kStateLow;
+    const uint32_t b = __ballot_sync(kFull, need);
+    const uint32_t w = lds_u16(pos + 2u * __popc(b & lt));
+    if (need) x = x * 65536u + w;
+    pos += 2u * __popc(b);
 }
 
 // ---- table expansion -------------------------------------------------------------------------
@@ -167,43 +196,42 @@ __device__ void build_tables(Smem<WARPS>& sm, const Params& p) {
         uint32_t c = inc - sum;
 #pragma unroll
         for (int i = 0; i < 8; ++i) {
-            sm.fc[ctx][8 * lane + i] = q[i] | (c << 16);
+            sm.fc[ctx][0][8 * lane + i] = uint16_t(q[i]);
+            sm.fc[ctx][1][8 * lane + i] = uint16_t(c);  // < 4096 for every used symbol
             c += q[i];
         }
     }
     __syncthreads();
-    // (b) slot -> symbol, 4 slots per 32-bit store; a context is split into P parts per warp
+    // (b) slot -> symbol, 4 slots per 32-bit store.  Lane l of a warp writes words it*32 + l
+    // (it = 0, 1, ...), so the 32 stores of one instruction hit 32 different banks; each lane
+    // walks its symbol forward as its slots grow.  A context is split into P parts over warps.
     constexpr int P = WARPS >= 16 ? WARPS / 16 : 1;
-    constexpr uint32_t kPerLane = kProbTotal / (32 * P);
+    constexpr uint32_t kWordsPerPart = kProbTotal / 4 / P;
     for (uint32_t item = warp; item < uint32_t(kFieldContexts * P); item += WARPS) {
         const uint32_t ctx = item / P, part = item % P;
-        const uint32_t* fc = sm.fc[ctx];
-        const uint32_t first = (part * 32 + lane) * kPerLane;
-        uint32_t* dst = reinterpret_cast<uint32_t*>(&sm.sym[ctx][first]);
-        const uint32_t total = (fc[255] >> 16) + (fc[255] & 0xFFFF);
+        const uint16_t* cum = sm.fc[ctx][1];
+        uint32_t* dst = reinterpret_cast<uint32_t*>(&sm.sym[ctx][0]) + part * kWordsPerPart;
+        const uint32_t total = uint32_t(cum[255]) + sm.fc[ctx][0][255];
         if (total == 0) {  // context never used by this blob
-            for (uint32_t w = 0; w < kPerLane / 4; ++w) dst[w] = 0;
+            for (uint32_t w = lane; w < kWordsPerPart; w += 32) dst[w] = 0;
             continue;
         }
+        const uint32_t first = 4 * (part * kWordsPerPart + lane);
         uint32_t s = 0;  // largest symbol with cum(s) <= first
 #pragma unroll
         for (uint32_t step = 128; step; step >>= 1)
-            if ((fc[s + step] >> 16) <= first) s += step;
-        uint32_t next = s < 255 ? (fc[s + 1] >> 16) : kProbTotal;
-        for (uint32_t w = 0; w < kPerLane / 4; ++w) {
-            const uint32_t base = first + 4 * w;
-            uint32_t word;
-            if (next >= base + 4) {
-                word = s * 0x01010101u;
-            } else {
-                word = 0;
-                for (uint32_t k = 0; k < 4; ++k) {
-                    while (next <= base + k) {
-                        ++s;
-                        next = s < 255 ? (fc[s + 1] >> 16) : kProbTotal;
-                    }
-                    word |= s << (8 * k);
+            if (cum[s + step] <= first) s += step;
+        uint32_t next = s < 255 ? cum[s + 1] : kProbTotal;
+        for (uint32_t w = lane; w < kWordsPerPart; w += 32) {
+            const uint32_t base = 4 * (part * kWordsPerPart + w);
+            uint32_t word = 0;
+#pragma unroll
+            for (uint32_t k = 0; k < 4; ++k) {
+                while (next <= base + k) {
+                    ++s;
+                    next = s < 255 ? cum[s + 1] : kProbTotal;
                 }
+                word |= s << (8 * k);
             }
             dst[w] = word;
         }
@@ -255,10 +283,12 @@ __device__ __forceinline__ void store_one(void* out, int64_t elem, float v) {
 }
 
 // ---- one step: every lane decodes (at most) one 8-vector --------------------------------------
-template <int WARPS, int OUT, bool VEC, bool FULL>
-__device__ __forceinline__ void decode_step(const Smem<WARPS>& sm, const Params& p, const uint8_t* ring,
-                                            uint32_t& x, uint32_t& cur, bool active, uint32_t lt, int64_t v,
-                                            int64_t row, int64_t kcol) {
+// `pos` is the shared address of the step's first unread word; on return it points past the
+// words the step consumed.
+template <int OUT, bool VEC, bool FULL>
+__device__ __forceinline__ void decode_step(const Params& p, uint32_t sym0, uint32_t fc0, uint32_t& pos,
+                                            uint32_t& x, bool active, uint32_t lt, int64_t v, int64_t row,
+                                            int64_t kcol) {
     if (FULL) active = true;
     // issued early, used after the symbol chain; lanes past the last vector read nothing
     const float a = active ? __ldg(p.alpha + row) : 0.0f;
@@ -267,37 +297,41 @@ __device__ __forceinline__ void decode_step(const Smem<WARPS>& sm, const Params&
     const uint32_t q0 = p.q_coset0;
     uint32_t slot = x & (kProbTotal - 1);
     const uint32_t c = slot >= q0 ? 1u : 0u;
-    if (active) x = (c ? kProbTotal - q0 : q0) * (x >> kProbBits) + slot - (c ? q0 : 0u);
-    renorm(x, cur, ring, lt, active);
+    if (active) x = (c ? kProbTotal - q0 : q0) * (x >> kProbBits) + (slot - (c ? q0 : 0u));
+    renorm(x, pos, lt, active);
 
-    // fields f1..f8 with context (c, j)
-    const uint8_t* st = &sm.sym[8 * c][0];
-    const uint32_t* ft = &sm.fc[8 * c][0];
+    // fields f1..f8 with context (c, j): tables of coset c start 8 contexts further on
+    const uint32_t st = sym0 + c * (8u * kProbTotal);
+    const uint32_t ft = fc0 + c * (8u * 1024u);
     uint32_t sym[8];
-#pragma unroll
-    for (int j = 0; j < 8; ++j) {
-        slot = x & (kProbTotal - 1);
-        const uint32_t s = st[j * kProbTotal + slot];
-        const uint32_t e = ft[j * 256 + s];
-        if (active) x = (e & 0xFFFFu) * (x >> kProbBits) + slot - (e >> 16);
-        renorm(x, cur, ring, lt, active);
-        sym[j] = s;
+    uint32_t top = 0;
+#define EP_FIELD(j)                                                                    \
+    {                                                                                  \
+        slot = x & (kProbTotal - 1);                                                   \
+        const uint32_t s = lds_u8<(j) * kProbTotal>(st + slot);                        \
+        const uint32_t fa = ft + 2u * s;                                               \
+        const uint32_t q = lds_u16<(j) * 1024>(fa);                                    \
+        const uint32_t cm = lds_u16<(j) * 1024 + 512>(fa);                             \
+        if (active) x = q * (x >> kProbBits) + (slot - cm);                            \
+        renorm(x, pos, lt, active);                                                    \
+        sym[j] = s;                                                                    \
+        top = max(top, s);                                                             \
     }
+    EP_FIELD(0) EP_FIELD(1) EP_FIELD(2) EP_FIELD(3) EP_FIELD(4) EP_FIELD(5) EP_FIELD(6) EP_FIELD(7)
+#undef EP_FIELD
 
     // escaped fields: raw words after the step's renormalisation words, by field then lane
     int32_t f[8];
 #pragma unroll
     for (int j = 0; j < 8; ++j) f[j] = int32_t(sym[j]) - kAlphabetR;
-    uint32_t esc = 0;
-#pragma unroll
-    for (int j = 0; j < 8; ++j) esc |= (active && sym[j] == uint32_t(kEscape)) ? (1u << j) : 0u;
-    if (__any_sync(kFull, esc != 0)) {
+    if (__any_sync(kFull, active && top == uint32_t(kEscape))) {
 #pragma unroll
         for (int j = 0; j < 8; ++j) {
-            const bool mine = (esc >> j) & 1u;
+            const bool mine = active && sym[j] == uint32_t(kEscape);
             const uint32_t b = __ballot_sync(kFull, mine);
-            if (mine) f[j] = int16_t(ring_word(ring, cur + 2u * __popc(b & lt)));
-            cur += 2u * __popc(b);
+            const uint32_t w = lds_u16(pos + 2u * __popc(b & lt));
+            if (mine) f[j] = int16_t(w);
+            pos += 2u * __popc(b);
         }
     }
     if (!active) return;
@@ -331,21 +365,31 @@ __device__ __forceinline__ void decode_step(const Smem<WARPS>& sm, const Params&
     }
 }
 
-template <int WARPS, int OUT, bool VEC>
-__global__ void __launch_bounds__(WARPS * 32, (WARPS >= 32 ? 1 : 2048 / (WARPS * 32 * 2)))
-    decode_kernel(const Params p) {
+// BUILD = false: stage the pre-expanded table block from p.tables; true: expand it in each CTA.
+template <int WARPS, int OUT, bool VEC, bool BUILD>
+__global__ void __launch_bounds__(WARPS * 32, 1) decode_kernel(const Params p) {
     extern __shared__ __align__(128) uint8_t smem_raw[];
     Smem<WARPS>& sm = *reinterpret_cast<Smem<WARPS>*>(smem_raw);
     const uint32_t lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
     const uint32_t lt = (1u << lane) - 1u;
     unsigned long long* bar = sm.bar[warp];
     uint8_t* ring = sm.ring[warp];
+    const uint32_t ring_a = smem_u32(ring);
 
     if (lane == 0) {
         for (int i = 0; i < kRingChunks; ++i) mbar_init(&bar[i], 1);
+        if (!BUILD && warp == 0) mbar_init(&sm.tbar, 1);
         fence_proxy_async();
     }
     __syncwarp();
+    if (!BUILD) {
+        __syncthreads();  // tbar initialised before anyone waits on it
+        if (threadIdx.x == 0) {
+            mbar_expect_tx(&sm.tbar, kTableBytes);
+            for (uint32_t o = 0; o < kTableBytes; o += kTablePiece)
+                bulk_g2s(smem_raw + o, p.tables + o, kTablePiece, &sm.tbar);
+        }
+    }
 
     const uint32_t tile_stride = gridDim.x * WARPS;
     uint32_t tile = blockIdx.x + gridDim.x * warp;
@@ -359,11 +403,15 @@ __global__ void __launch_bounds__(WARPS * 32, (WARPS >= 32 ? 1 : 2048 / (WARPS *
     auto issue = [&](uint32_t j) {
         const uint32_t g = g0 + j, slot = g & (kRingChunks - 1);
         const uint32_t nb = min(uint32_t(kChunk), bytes - j * kChunk);
+        // ring bytes [0, kMirror) are repeated at [kRing, kRing + kMirror)
+        const uint32_t lo = slot * kChunk;
+        const uint32_t mirror = lo < uint32_t(kMirror) ? min(uint32_t(kMirror) - lo, nb) : 0u;
         __syncwarp();
         if (lane == 0) {
             fence_proxy_async();  // earlier reads of this slot come before the bulk write
-            mbar_expect_tx(&bar[slot], nb);
-            bulk_g2s(ring + slot * kChunk, src + size_t(j) * kChunk, nb, &bar[slot]);
+            mbar_expect_tx(&bar[slot], nb + mirror);
+            bulk_g2s(ring + lo, src + size_t(j) * kChunk, nb, &bar[slot]);
+            if (mirror) bulk_g2s(ring + kRing + lo, src + size_t(j) * kChunk, mirror, &bar[slot]);
         }
     };
     auto wait = [&](uint32_t j) -> bool {
@@ -383,57 +431,68 @@ __global__ void __launch_bounds__(WARPS * 32, (WARPS >= 32 ? 1 : 2048 / (WARPS *
         x = __ldg(reinterpret_cast<const uint32_t*>(p.stream + t0) + lane);
     };
 
-    if (tile < p.n_tiles) begin_tile();  // first copies overlap the table expansion
-    build_tables<WARPS>(sm, p);
-    __syncthreads();
+    if (tile < p.n_tiles) begin_tile();  // the first tile's fetch overlaps the table staging
+    if (BUILD) {
+        build_tables<WARPS>(sm, p);
+        __syncthreads();
+    } else if (!mbar_wait(&sm.tbar, 0)) {
+        if (lane == 0) atomicOr(p.status, kStTimeout);
+        goto timeout;
+    }
 
-    bool first = true;
-    for (; tile < p.n_tiles; tile += tile_stride) {
-        if (!first) begin_tile();
-        first = false;
-        const int64_t per_tile = int64_t(kLanes) * p.steps;
-        const int64_t v0 = int64_t(tile) * per_tile;
-        const int64_t vend = min(v0 + per_tile, p.n_vectors);
-        const uint32_t nsteps = uint32_t((vend - v0 + kLanes - 1) / kLanes);
-        int64_t v = v0 + lane;
-        int64_t row = v / p.vec_per_row, kcol = v - row * p.vec_per_row;
-        uint32_t cur = rofs;  // ring position of the next unread byte
-        uint32_t flags = 0;
-        for (uint32_t k = 0; k < nsteps; ++k) {
-            // keep the ring full and the bytes this step may read resident
-            const uint32_t done = cur - rofs;  // bytes of this tile consumed so far
-            const uint32_t lim = min(nch, done / kChunk + kRingChunks);
-            while (issued < lim) issue(issued++);
-            const uint32_t need = (min(bytes, done + uint32_t(kMaxStepBytes)) + kChunk - 1) / kChunk;
-            while (waited < need) {
+    {
+        const uint32_t sym0 = smem_u32(&sm.sym[0][0]), fc0 = smem_u32(&sm.fc[0][0][0]);
+        bool first = true;
+        for (; tile < p.n_tiles; tile += tile_stride) {
+            if (!first) begin_tile();
+            first = false;
+            const int64_t per_tile = int64_t(kLanes) * p.steps;
+            const int64_t v0 = int64_t(tile) * per_tile;
+            const int64_t vend = min(v0 + per_tile, p.n_vectors);
+            const uint32_t nsteps = uint32_t((vend - v0 + kLanes - 1) / kLanes);
+            int64_t v = v0 + lane;
+            int64_t row = v / p.vec_per_row, kcol = v - row * p.vec_per_row;
+            uint32_t cur = rofs;  // ring position of the next unread byte
+            uint32_t flags = 0;
+            for (uint32_t k = 0; k < nsteps; ++k) {
+                // keep the ring full and the bytes this step may read resident
+                const uint32_t done = cur - rofs;  // bytes of this tile consumed so far
+                const uint32_t lim = min(nch, done / kChunk + kRingChunks);
+                while (issued < lim) issue(issued++);
+                const uint32_t need = (min(bytes, done + uint32_t(kMaxStepBytes)) + kChunk - 1) / kChunk;
+                while (waited < need) {
+                    if (!wait(waited)) goto timeout;
+                    ++waited;
+                }
+                const uint32_t pos0 = ring_a + (cur & (kRing - 1));
+                uint32_t pos = pos0;
+                if (v0 + int64_t(k + 1) * kLanes <= vend)
+                    decode_step<OUT, VEC, true>(p, sym0, fc0, pos, x, true, lt, v, row, kcol);
+                else
+                    decode_step<OUT, VEC, false>(p, sym0, fc0, pos, x, v < vend, lt, v, row, kcol);
+                cur += pos - pos0;
+                if (cur - rofs > bytes) {
+                    flags |= kStOverrun;
+                    break;
+                }
+                v += kLanes;
+                kcol += kLanes;
+                while (kcol >= p.vec_per_row) {
+                    kcol -= p.vec_per_row;
+                    ++row;
+                }
+            }
+            // drain copies the decode did not need (padding) before the slots are reused
+            while (waited < issued) {
                 if (!wait(waited)) goto timeout;
                 ++waited;
             }
-            if (v0 + int64_t(k + 1) * kLanes <= vend)
-                decode_step<WARPS, OUT, VEC, true>(sm, p, ring, x, cur, true, lt, v, row, kcol);
-            else
-                decode_step<WARPS, OUT, VEC, false>(sm, p, ring, x, cur, v < vend, lt, v, row, kcol);
-            if (cur - rofs > bytes) {
-                flags |= kStOverrun;
-                break;
+            if (!(flags & kStOverrun)) {
+                if (__any_sync(kFull, x != kStateLow)) flags |= kStState;
+                if (bytes - (cur - rofs) >= 16) flags |= kStLeftover;
             }
-            v += kLanes;
-            kcol += kLanes;
-            while (kcol >= p.vec_per_row) {
-                kcol -= p.vec_per_row;
-                ++row;
-            }
+            if (lane == 0 && flags) atomicOr(p.status, flags);
         }
-        // drain copies the decode did not need (padding) before the slots are reused
-        while (waited < issued) {
-            if (!wait(waited)) goto timeout;
-            ++waited;
-        }
-        if (!(flags & kStOverrun)) {
-            if (__any_sync(kFull, x != kStateLow)) flags |= kStState;
-            if (bytes - (cur - rofs) >= 16) flags |= kStLeftover;
-        }
-        if (lane == 0 && flags) atomicOr(p.status, flags);
     }
     return;
 
@@ -446,8 +505,20 @@ timeout:
     }
 }
 
+// Expands the blob's compact frequency tables into the 80 KB decode-table block (one CTA).
+template <int WARPS>
+__global__ void __launch_bounds__(WARPS * 32, 1) expand_tables_kernel(const Params p, uint8_t* tables) {
+    extern __shared__ __align__(128) uint8_t smem_raw[];
+    Smem<WARPS>& sm = *reinterpret_cast<Smem<WARPS>*>(smem_raw);
+    build_tables<WARPS>(sm, p);
+    __syncthreads();
+    const uint4* s = reinterpret_cast<const uint4*>(smem_raw);
+    uint4* d = reinterpret_cast<uint4*>(tables);
+    for (uint32_t i = threadIdx.x; i < kTableBytes / 16; i += blockDim.x) d[i] = s[i];
+}
+
 // ---- host-side launch -------------------------------------------------------------------------
-constexpr int kWarps = 16;
+constexpr int kWarps = 32;
 
 struct DevInfo {
     bool ready = false;
@@ -458,7 +529,7 @@ DevInfo g_dev[kMaxDevices];
 
 template <int WARPS, int OUT, bool VEC>
 int launch_one(const Params& p, cudaStream_t st, int device) {
-    auto fn = decode_kernel<WARPS, OUT, VEC>;
+    auto fn = decode_kernel<WARPS, OUT, VEC, false>;
     const size_t smem = sizeof(Smem<WARPS>);
     static std::mutex mu;
     static int per_sm[kMaxDevices] = {};
@@ -522,30 +593,12 @@ int current_device(int& dev) {
     return EP_OK;
 }
 
-// Device copy of the blob and its status word on `dev` (allocated and filled on first use).
-int ensure_device(ep_blob* b, int dev, cudaStream_t st) {
-    std::lock_guard<std::mutex> g(b->mu);
-    DeviceCopy& d = b->dev[dev];
-    if (d.blob) return EP_OK;
-    uint8_t* blob = nullptr;
-    uint32_t* status = nullptr;
-    if (cudaMalloc(&blob, b->bytes.size()) != cudaSuccess || cudaMalloc(&status, 16) != cudaSuccess) {
-        cudaFree(blob);
-        return set_error(EP_ERR_OOM, "device copy of the blob");
-    }
-    EP_CUDA(cudaMemcpyAsync(blob, b->bytes.data(), b->bytes.size(), cudaMemcpyHostToDevice, st), "blob upload");
-    EP_CUDA(cudaMemsetAsync(status, 0, 16, st), "status clear");
-    EP_CUDA(cudaStreamSynchronize(st), "blob upload");
-    d.blob = blob;
-    d.status = status;
-    return EP_OK;
-}
-
-Params make_params(const ep_blob* b, const uint8_t* dblob, void* out, int64_t row_stride, uint32_t* status,
-                   bool vec) {
+Params make_params(const ep_blob* b, const uint8_t* dblob, const uint8_t* tables, void* out, int64_t row_stride,
+                   uint32_t* status, bool vec) {
     const BlobLayout& L = b->layout;
     Params p;
     p.blob = dblob;
+    p.tables = tables;
     p.tile_off = reinterpret_cast<const uint32_t*>(dblob + L.off_offsets);
     p.stream = dblob + L.off_stream;
     p.alpha = reinterpret_cast<const float*>(dblob + L.off_alpha);
@@ -568,6 +621,36 @@ Params make_params(const ep_blob* b, const uint8_t* dblob, void* out, int64_t ro
     return p;
 }
 
+// Device copy of the blob and its status word on `dev` (allocated and filled on first use).
+int ensure_device(ep_blob* b, int dev, cudaStream_t st) {
+    std::lock_guard<std::mutex> g(b->mu);
+    DeviceCopy& d = b->dev[dev];
+    if (d.blob) return EP_OK;
+    uint8_t* blob = nullptr;
+    uint8_t* tables = nullptr;
+    uint32_t* status = nullptr;
+    if (cudaMalloc(&blob, b->bytes.size()) != cudaSuccess || cudaMalloc(&tables, kTableBytes) != cudaSuccess ||
+        cudaMalloc(&status, 16) != cudaSuccess) {
+        cudaFree(blob);
+        cudaFree(tables);
+        return set_error(EP_ERR_OOM, "device copy of the blob");
+    }
+    EP_CUDA(cudaMemcpyAsync(blob, b->bytes.data(), b->bytes.size(), cudaMemcpyHostToDevice, st), "blob upload");
+    EP_CUDA(cudaMemsetAsync(status, 0, 16, st), "status clear");
+    // expand the compact frequency tables once for this device copy
+    Params p = make_params(b, blob, nullptr, nullptr, b->layout.cols, status, false);
+    auto fn = expand_tables_kernel<kWarps>;
+    EP_CUDA(cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, int(kTableBytes)),
+            "table expansion attribute");
+    fn<<<1, kWarps * 32, kTableBytes, st>>>(p, tables);
+    EP_CUDA(cudaGetLastError(), "table expansion launch");
+    EP_CUDA(cudaStreamSynchronize(st), "blob upload");
+    d.blob = blob;
+    d.tables = tables;
+    d.status = status;
+    return EP_OK;
+}
+
 bool vec_ok(const BlobLayout& L, const void* out, int64_t row_stride, int dtype) {
     const uintptr_t align = dtype == kE4M3 ? 8 : 16;
     return L.cols % 8 == 0 && row_stride % 8 == 0 && (reinterpret_cast<uintptr_t>(out) % align) == 0;
@@ -588,7 +671,7 @@ std::mutex g_noalloc_mu;
 
 template <int WARPS, int OUT, bool VEC>
 int noalloc_launch_one(const Params& p, cudaStream_t st, int device) {
-    auto fn = decode_kernel<WARPS, OUT, VEC>;
+    auto fn = decode_kernel<WARPS, OUT, VEC, true>;
     const size_t smem = sizeof(Smem<WARPS>);
     static std::mutex mu;
     static int per_sm[kMaxDevices] = {};
@@ -665,7 +748,7 @@ extern "C" int ep_decompress(const ep_blob* cb, const ep_tensor* out, void* stre
         if (rc != EP_OK) return rc;
         const DeviceCopy& d = b->dev[dev];
         const bool vec = vec_ok(L, out->data, out->row_stride, out->dtype);
-        Params p = make_params(b, d.blob, out->data, out->row_stride, d.status, vec);
+        Params p = make_params(b, d.blob, d.tables, out->data, out->row_stride, d.status, vec);
         return launch(p, kind, vec, st, dev);
     }
 
@@ -699,7 +782,7 @@ extern "C" int ep_decompress(const ep_blob* cb, const ep_tensor* out, void* stre
     EP_CUDA(cudaMemcpyAsync(d.stage_blob, b->bytes.data(), b->bytes.size(), cudaMemcpyHostToDevice, st),
             "ep_decompress: upload");
     const bool vec = vec_ok(L, d.stage_out, L.cols, out->dtype);
-    Params p = make_params(b, d.stage_blob, d.stage_out, L.cols, d.status, vec);
+    Params p = make_params(b, d.stage_blob, d.tables, d.stage_out, L.cols, d.status, vec);
     rc = launch(p, kind, vec, st, dev);
     if (rc != EP_OK) return rc;
     EP_CUDA(cudaMemcpy2DAsync(out->data, size_t(out->row_stride) * es, d.stage_out, size_t(L.cols) * es,
@@ -719,7 +802,7 @@ extern "C" int ep_decode_fields(const ep_blob* cb, int16_t* fields, void* stream
     if (rc == EP_OK) rc = ensure_device(b, dev, st);
     if (rc != EP_OK) return rc;
     const DeviceCopy& d = b->dev[dev];
-    Params p = make_params(b, d.blob, fields, b->layout.cols, d.status, false);
+    Params p = make_params(b, d.blob, d.tables, fields, b->layout.cols, d.status, false);
     return launch(p, kOutFields, false, st, dev);
 }
 
@@ -755,6 +838,7 @@ extern "C" void ep_blob_free(ep_blob* b) {
         if (!d.blob && !d.stage_blob && !d.stage_out) continue;
         cudaSetDevice(dv);
         cudaFree(d.blob);
+        cudaFree(d.tables);
         cudaFree(d.status);
         cudaFree(d.stage_blob);
         cudaFree(d.stage_out);
@@ -806,7 +890,8 @@ extern "C" int ep_decompress_noalloc(const ep_blob* cb, const void* device_blob,
     if (cudaMemsetAsync(status, 0, sizeof(uint32_t) * kWordsNeeded, st) != cudaSuccess)
         return set_error_static(EP_ERR_CUDA, "ep_decompress_noalloc: clearing the status word failed");
     const bool vec = vec_ok(L, out->data, out->row_stride, out->dtype);
-    Params p = make_params(cb, static_cast<const uint8_t*>(device_blob), out->data, out->row_stride, status, vec);
+    Params p = make_params(cb, static_cast<const uint8_t*>(device_blob), nullptr, out->data, out->row_stride,
+                           status, vec);
     int rc = noalloc_launch(p, kind, vec, st, dev);
     if (rc != EP_OK || !wait) return rc;
     uint32_t s = 0;
