@@ -71,7 +71,7 @@ extern "C" int ep_compress_ex(const ep_tensor* in, double target_bpp, const ep_o
 
     EncodeOptions o;
     if (opt) {
-        if (opt->steps_per_tile < 0 || opt->steps_per_tile > (1 << 20) || opt->num_threads < 0 ||
+        if (opt->steps_per_tile < 0 || opt->steps_per_tile > 1024 || opt->num_threads < 0 ||
             !(opt->scale >= 0.0) || !std::isfinite(opt->scale))
             return set_error(EP_ERR_ARG, "ep_compress: bad options");
         o.steps_per_tile = opt->steps_per_tile;

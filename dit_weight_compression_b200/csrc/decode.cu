@@ -10,22 +10,22 @@
 //   * one persistent CTA of 32 warps per SM (grid = min(#SM, #tiles)); tile t goes to CTA
 //     t mod grid, so every SM gets an equal share even when there are few tiles;
 //   * decode tables: per field context a 4096-entry slot->symbol byte table and a 256-entry
-//     frequency / cumulative-frequency table pair of u16, 80 KB in all.  They are expanded once per blob
-//     and device by a small kernel into a block next to the device copy; every CTA stages that
-//     block into shared memory with bulk copies, overlapped with the fetch of its first tiles.
-//     (The allocation-free entry point expands them inside each CTA instead.)  The coset
+//     frequency / cumulative-frequency table pair of u16, 80 KB in all.  They are expanded once per
+//     blob and device by a small kernel into a block next to the device copy; every CTA stages
+//     that block into shared memory with bulk copies, overlapped with the fetch of its first
+//     tiles.  (The allocation-free entry point expands them inside each CTA instead.)  The coset
 //     context, two symbols, is decoded by one compare;
-//   * each warp streams its tile's words through a private shared-memory ring of four 512-byte
-//     chunks filled by 1-D bulk copies (cp.async.bulk, no multicast) that complete on one
-//     mbarrier per chunk; the 1088 bytes after the ring (the most one step can read) mirror its
-//     start, so a step reads one linear window with no wrap-around arithmetic; every wait is
-//     bounded and reports through the status word;
-//   * per step a lane decodes one 8-vector: 9 rANS symbols, each followed by the
-//     renormalisation read whose word position is the warp-ballot prefix count of lanes
-//     refilling before it; escaped fields take raw words at the end of the step; fields are
-//     inverted in registers (z8 = 2 f8 + parity, y = z + c/2), multiplied by the row's fp32
-//     scale, converted one pair per cvt and written as one 16-byte store per lane (a 512-byte
-//     contiguous run per warp for BF16/FP16).
+//   * words: every lane reads its own word stream.  Lanes 2p and 2p+1 share region p of the tile
+//     (one forward from the region start, one backward from its end); a warp-shuffle prefix sum
+//     over the 16 region counts gives every lane its start.  The tile is prefetched into L2 by
+//     a bulk prefetch; each lane keeps two 8-byte chunks of its stream in registers, loads the
+//     next chunk four words ahead, and has its next word ready before it needs it, so a
+//     renormalisation costs one compare and one byte permute on the dependent chain;
+//   * per step a lane decodes one 8-vector: 9 rANS symbols (each followed by its conditional
+//     refill), then the raw words of its escaped fields; fields are inverted in registers
+//     (z8 = 2 f8 + parity, y = z + c/2), multiplied by the row's fp32 scale, converted one pair
+//     per cvt and written as one 16-byte store per lane (a 512-byte contiguous run per warp for
+//     BF16/FP16).
 // No tensor cores: the path is table lookups and integer arithmetic, bound by HBM bytes and by
 // the latency and issue slots of that arithmetic, not by a contraction.
 #include <cuda_bf16.h>
@@ -50,11 +50,6 @@ namespace ep {
 namespace {
 
 constexpr uint32_t kFull = 0xFFFFFFFFu;
-constexpr int kChunk = 512;                                   // bytes per bulk copy
-constexpr int kRingChunks = 4;
-constexpr int kRing = kChunk * kRingChunks;                   // ring bytes per warp
-constexpr int kMaxStepBytes = 2 * (9 * kLanes + 8 * kLanes);  // bytes one step can consume (1088)
-constexpr int kMirror = kMaxStepBytes;                        // mirror of the ring's first bytes
 constexpr uint32_t kWaitSpins = 1u << 22;                     // bounded mbarrier wait (~0.3 s)
 constexpr uint32_t kTableBytes = kFieldContexts * (kProbTotal + 256 * 4);  // 81920
 constexpr uint32_t kTablePiece = 16384;                       // bytes per table bulk copy
@@ -63,9 +58,9 @@ enum OutKind { kOutBF16 = 0, kOutFP16 = 1, kOutE4M3 = 2, kOutF32 = 3, kOutFields
 
 // Status word bits (sticky, cleared by ep_decode_status).
 enum : uint32_t {
-    kStOverrun = 1u,   // a tile read past its own bytes
+    kStOverrun = 1u,   // a lane read past its region, or the regions overrun the tile
     kStState = 2u,     // a lane did not end in state 2^16
-    kStLeftover = 4u,  // 16 or more bytes of a tile were never read
+    kStLeftover = 4u,  // a region's two lanes did not meet, or 16+ bytes follow the regions
     kStTimeout = 8u    // a bulk-copy wait hit its limit
 };
 
@@ -87,15 +82,26 @@ struct Params {
     int dense;                  // element offset of vector v is 8 v
 };
 
+constexpr uint32_t kSmemOptin = 232448;  // 227 KB: the largest dynamic shared memory of one CTA
+constexpr uint32_t kBufSlack = 48;        // bytes after a tile buffer that a step may over-read
+
+// Per-warp tile buffer size for a CTA of WARPS warps: what the 227 KB leave after the tables.
+template <int WARPS>
+struct Geo {
+    static constexpr uint32_t kBuf =
+        ((kSmemOptin - kTableBytes - 64 - WARPS * (kBufSlack + 8) - 8) / WARPS) & ~15u;
+};
+
 template <int WARPS>
 struct Smem {
-    uint8_t sym[kFieldContexts][kProbTotal];        // slot -> symbol               } the 80 KB
-    uint16_t fc[kFieldContexts][2][256];            // [0] frequency, [1] cumulative } table block
-    alignas(16) uint8_t ring[WARPS][kRing + kMirror];  // per-warp stream ring (+ mirror)
-    unsigned long long bar[WARPS][kRingChunks];     // one mbarrier per ring chunk
-    unsigned long long tbar;                        // the table block's bulk copies
+    uint8_t sym[kFieldContexts][kProbTotal];                    // slot -> symbol    } 80 KB table
+    uint16_t fc[kFieldContexts][2][256];                        // [0] freq, [1] cum } block
+    alignas(16) uint8_t tbuf[WARPS][Geo<WARPS>::kBuf + kBufSlack];  // one staged tile per warp
+    unsigned long long bar[WARPS];                              // tile staging, one per warp
+    unsigned long long tbar;                                    // the table block's bulk copies
 };
-static_assert(offsetof(Smem<32>, ring) == kTableBytes, "table block must be contiguous");
+static_assert(offsetof(Smem<32>, tbuf) == kTableBytes, "table block must be contiguous");
+static_assert(sizeof(Smem<32>) <= kSmemOptin && sizeof(Smem<16>) <= kSmemOptin, "shared memory budget");
 
 // ---- PTX wrappers ----------------------------------------------------------------------------
 __device__ __forceinline__ uint32_t smem_u32(const void* p) {
@@ -158,16 +164,50 @@ __device__ __forceinline__ uint32_t lds_u32(uint32_t a) {
     return v;
 }
 
-// Renormalisation after one decoded symbol: lanes whose state fell below 2^16 take the next
-// 16-bit words in ascending lane order (position = cursor + 2 * #refilling lanes below me).
-// `pos` is the shared address of the next unread word; within one step it only grows, and the
-// ring's mirror keeps every address of the step inside the ring allocation.
-__device__ __forceinline__ void renorm(uint32_t& x, uint32_t& pos, uint32_t lt, bool active) {
+// Prefetch `bytes` (a multiple of 16) at a 16-byte aligned global address into L2.
+__device__ __forceinline__ void prefetch_l2(const void* p, uint32_t bytes) {
+    asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(p), "r"(bytes) : "memory");
+}
+
+// A lane's word stream, read from the warp's shared-memory copy of the tile.  `wp` is the
+// shared address of the lane's next word and `wn` that word, loaded right after the previous
+// one was used -- well before it is needed, so a refill costs a compare and a byte permute on
+// the dependent chain.  Predicated loads keep the warp converged.
+struct SmemReader {
+    uint32_t wp, wn, nread;
+    int32_t wd;  // +2 (lane 2p, forward) or -2 (lane 2p+1, backward)
+    __device__ __forceinline__ void consume_if(bool take) {
+        nread += take ? 1u : 0u;
+        wp += take ? uint32_t(wd) : 0u;
+        asm volatile("{\n .reg .pred p;\n setp.ne.u32 p, %1, 0;\n @p ld.shared.u16 %0, [%2];\n}"
+                     : "+r"(wn)
+                     : "r"(uint32_t(take)), "r"(wp));
+    }
+};
+
+// The same for a tile too large for the buffer: words come from global memory, every address
+// clamped into the tile.
+struct GlobalReader {
+    const uint8_t* tile;
+    int32_t off, hi, wd;  // byte offset of the next word; last legal word offset; +-2
+    uint32_t wn, nread;
+    __device__ __forceinline__ void consume_if(bool take) {
+        nread += take ? 1u : 0u;
+        off += take ? wd : 0;
+        const uint8_t* src = tile + min(max(off, 0), hi);
+        asm volatile("{\n .reg .pred p;\n setp.ne.u32 p, %1, 0;\n @p ld.global.nc.u16 %0, [%2];\n}"
+                     : "+r"(wn)
+                     : "r"(uint32_t(take)), "l"(src));
+    }
+};
+
+// Renormalisation after one decoded symbol: a lane whose state fell below 2^16 shifts in its
+// next word (x * 2^16 + w, i.e. the byte permutation {w.lo, w.hi, x.lo, x.hi}).
+template <class Reader>
+__device__ __forceinline__ void renorm(uint32_t& x, Reader& rd, bool active) {
     const bool need = active && x < kStateLow;
-    const uint32_t b = __ballot_sync(kFull, need);
-    const uint32_t w = lds_u16(pos + 2u * __popc(b & lt));
-    if (need) x = x * 65536u + w;
-    pos += 2u * __popc(b);
+    x = need ? __byte_perm(rd.wn, x, 0x5410) : x;
+    rd.consume_if(need);
 }
 
 // ---- table expansion -------------------------------------------------------------------------
@@ -283,12 +323,9 @@ __device__ __forceinline__ void store_one(void* out, int64_t elem, float v) {
 }
 
 // ---- one step: every lane decodes (at most) one 8-vector --------------------------------------
-// `pos` is the shared address of the step's first unread word; on return it points past the
-// words the step consumed.
-template <int OUT, bool VEC, bool FULL>
-__device__ __forceinline__ void decode_step(const Params& p, uint32_t sym0, uint32_t fc0, uint32_t& pos,
-                                            uint32_t& x, bool active, uint32_t lt, int64_t v, int64_t row,
-                                            int64_t kcol) {
+template <int OUT, bool VEC, bool FULL, class Reader>
+__device__ __forceinline__ void decode_step(const Params& p, uint32_t sym0, uint32_t fc0, Reader& rd,
+                                            uint32_t& x, bool active, int64_t v, int64_t row, int64_t kcol) {
     if (FULL) active = true;
     // issued early, used after the symbol chain; lanes past the last vector read nothing
     const float a = active ? __ldg(p.alpha + row) : 0.0f;
@@ -298,7 +335,7 @@ __device__ __forceinline__ void decode_step(const Params& p, uint32_t sym0, uint
     uint32_t slot = x & (kProbTotal - 1);
     const uint32_t c = slot >= q0 ? 1u : 0u;
     if (active) x = (c ? kProbTotal - q0 : q0) * (x >> kProbBits) + (slot - (c ? q0 : 0u));
-    renorm(x, pos, lt, active);
+    renorm(x, rd, active);
 
     // fields f1..f8 with context (c, j): tables of coset c start 8 contexts further on
     const uint32_t st = sym0 + c * (8u * kProbTotal);
@@ -313,14 +350,14 @@ __device__ __forceinline__ void decode_step(const Params& p, uint32_t sym0, uint
         const uint32_t q = lds_u16<(j) * 1024>(fa);                                    \
         const uint32_t cm = lds_u16<(j) * 1024 + 512>(fa);                             \
         if (active) x = q * (x >> kProbBits) + (slot - cm);                            \
-        renorm(x, pos, lt, active);                                                    \
+        renorm(x, rd, active);                                                         \
         sym[j] = s;                                                                    \
         top = max(top, s);                                                             \
     }
     EP_FIELD(0) EP_FIELD(1) EP_FIELD(2) EP_FIELD(3) EP_FIELD(4) EP_FIELD(5) EP_FIELD(6) EP_FIELD(7)
 #undef EP_FIELD
 
-    // escaped fields: raw words after the step's renormalisation words, by field then lane
+    // escaped fields: the lane's raw words after its renormalisation words, by field
     int32_t f[8];
 #pragma unroll
     for (int j = 0; j < 8; ++j) f[j] = int32_t(sym[j]) - kAlphabetR;
@@ -328,10 +365,8 @@ __device__ __forceinline__ void decode_step(const Params& p, uint32_t sym0, uint
 #pragma unroll
         for (int j = 0; j < 8; ++j) {
             const bool mine = active && sym[j] == uint32_t(kEscape);
-            const uint32_t b = __ballot_sync(kFull, mine);
-            const uint32_t w = lds_u16(pos + 2u * __popc(b & lt));
-            if (mine) f[j] = int16_t(w);
-            pos += 2u * __popc(b);
+            f[j] = mine ? int32_t(int16_t(rd.wn)) : f[j];
+            rd.consume_if(mine);
         }
     }
     if (!active) return;
@@ -365,144 +400,170 @@ __device__ __forceinline__ void decode_step(const Params& p, uint32_t sym0, uint
     }
 }
 
+// Decode the steps of one tile with a given word reader; returns the status flags of the tile.
+template <int OUT, bool VEC, class Reader, class Guard>
+__device__ __forceinline__ uint32_t decode_tile_steps(const Params& p, uint32_t sym0, uint32_t fc0, Reader& rd,
+                                                      uint32_t& x, uint32_t tile, uint32_t lane, Guard in_range) {
+    const int64_t per_tile = int64_t(kLanes) * p.steps;
+    const int64_t v0 = int64_t(tile) * per_tile;
+    const int64_t vend = min(v0 + per_tile, p.n_vectors);
+    const uint32_t nsteps = uint32_t((vend - v0 + kLanes - 1) / kLanes);
+    int64_t v = v0 + lane;
+    int64_t row = v / p.vec_per_row, kcol = v - row * p.vec_per_row;
+    for (uint32_t k = 0; k < nsteps; ++k) {
+        if (!__all_sync(kFull, in_range(rd))) return kStOverrun;  // a corrupt tile ran away
+        if (v0 + int64_t(k + 1) * kLanes <= vend)
+            decode_step<OUT, VEC, true>(p, sym0, fc0, rd, x, true, v, row, kcol);
+        else
+            decode_step<OUT, VEC, false>(p, sym0, fc0, rd, x, v < vend, v, row, kcol);
+        v += kLanes;
+        kcol += kLanes;
+        while (kcol >= p.vec_per_row) {
+            kcol -= p.vec_per_row;
+            ++row;
+        }
+    }
+    return 0;
+}
+
 // BUILD = false: stage the pre-expanded table block from p.tables; true: expand it in each CTA.
 template <int WARPS, int OUT, bool VEC, bool BUILD>
 __global__ void __launch_bounds__(WARPS * 32, 1) decode_kernel(const Params p) {
     extern __shared__ __align__(128) uint8_t smem_raw[];
     Smem<WARPS>& sm = *reinterpret_cast<Smem<WARPS>*>(smem_raw);
+    constexpr uint32_t kBuf = Geo<WARPS>::kBuf;
     const uint32_t lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-    const uint32_t lt = (1u << lane) - 1u;
-    unsigned long long* bar = sm.bar[warp];
-    uint8_t* ring = sm.ring[warp];
-    const uint32_t ring_a = smem_u32(ring);
+    const bool fwd = (lane & 1) == 0;  // lanes 2p read forward, lanes 2p+1 backward
+    uint8_t* buf = sm.tbuf[warp];
+    const uint32_t buf_a = smem_u32(buf);
 
-    if (lane == 0) {
-        for (int i = 0; i < kRingChunks; ++i) mbar_init(&bar[i], 1);
-        if (!BUILD && warp == 0) mbar_init(&sm.tbar, 1);
+    if (threadIdx.x == 0) {
+        if (!BUILD) mbar_init(&sm.tbar, 1);
+        for (int w = 0; w < WARPS; ++w) mbar_init(&sm.bar[w], 1);
         fence_proxy_async();
     }
-    __syncwarp();
-    if (!BUILD) {
-        __syncthreads();  // tbar initialised before anyone waits on it
-        if (threadIdx.x == 0) {
-            mbar_expect_tx(&sm.tbar, kTableBytes);
-            for (uint32_t o = 0; o < kTableBytes; o += kTablePiece)
-                bulk_g2s(smem_raw + o, p.tables + o, kTablePiece, &sm.tbar);
-        }
+    __syncthreads();  // barriers initialised before anyone uses them
+    if (!BUILD && threadIdx.x == 0) {
+        mbar_expect_tx(&sm.tbar, kTableBytes);
+        for (uint32_t o = 0; o < kTableBytes; o += kTablePiece)
+            bulk_g2s(smem_raw + o, p.tables + o, kTablePiece, &sm.tbar);
     }
 
     const uint32_t tile_stride = gridDim.x * WARPS;
     uint32_t tile = blockIdx.x + gridDim.x * warp;
-    uint32_t seq = 0;  // chunks this warp has issued so far: chunk g uses slot g % 4, parity (g / 4) % 2
+    uint32_t staged = 0;  // tiles this warp has staged: its barrier's phase parity
 
-    // per-tile cursor state; chunk j of a tile lives in ring slot (g0 + j) % 4, so the tile's
-    // byte 0 sits at ring offset rofs = (g0 % 4) * 512 and ring positions are rofs + offset
-    const uint8_t* src = nullptr;
-    uint32_t bytes = 0, nch = 0, issued = 0, waited = 0, g0 = 0, rofs = 0, x = 0;
-
-    auto issue = [&](uint32_t j) {
-        const uint32_t g = g0 + j, slot = g & (kRingChunks - 1);
-        const uint32_t nb = min(uint32_t(kChunk), bytes - j * kChunk);
-        // ring bytes [0, kMirror) are repeated at [kRing, kRing + kMirror)
-        const uint32_t lo = slot * kChunk;
-        const uint32_t mirror = lo < uint32_t(kMirror) ? min(uint32_t(kMirror) - lo, nb) : 0u;
+    // Stage a tile that fits the buffer (one bulk copy), and ask L2 for the warp's next tile.
+    auto stage = [&](uint32_t t, uint64_t t0, uint32_t tbytes) {
         __syncwarp();
         if (lane == 0) {
-            fence_proxy_async();  // earlier reads of this slot come before the bulk write
-            mbar_expect_tx(&bar[slot], nb + mirror);
-            bulk_g2s(ring + lo, src + size_t(j) * kChunk, nb, &bar[slot]);
-            if (mirror) bulk_g2s(ring + kRing + lo, src + size_t(j) * kChunk, mirror, &bar[slot]);
+            fence_proxy_async();  // the previous tile's reads of the buffer come first
+            mbar_expect_tx(&sm.bar[warp], tbytes);
+            bulk_g2s(buf, p.stream + t0, tbytes, &sm.bar[warp]);
+            const uint32_t nt = t + tile_stride;
+            if (nt < p.n_tiles) {
+                const uint64_t n0 = 16ull * __ldg(p.tile_off + nt), n1 = 16ull * __ldg(p.tile_off + nt + 1);
+                prefetch_l2(p.stream + n0, uint32_t(min(n1 - n0, uint64_t(kBuf))));
+            }
         }
     };
-    auto wait = [&](uint32_t j) -> bool {
-        const uint32_t g = g0 + j;
-        return mbar_wait(&bar[g & (kRingChunks - 1)], (g >> 2) & 1u);
-    };
-    auto begin_tile = [&]() {
-        const uint64_t t0 = 16ull * __ldg(p.tile_off + tile), t1 = 16ull * __ldg(p.tile_off + tile + 1);
-        src = p.stream + t0 + kTileHeadBytes;
-        bytes = uint32_t(t1 - t0 - kTileHeadBytes);  // the host checked t1 >= t0 + 128
-        nch = (bytes + kChunk - 1) / kChunk;
-        g0 = seq;
-        seq += nch;
-        rofs = (g0 & (kRingChunks - 1)) * kChunk;
-        issued = waited = 0;
-        while (issued < min(nch, uint32_t(kRingChunks))) issue(issued++);
-        x = __ldg(reinterpret_cast<const uint32_t*>(p.stream + t0) + lane);
-    };
 
-    if (tile < p.n_tiles) begin_tile();  // the first tile's fetch overlaps the table staging
+    uint64_t t0 = 0;
+    uint32_t tbytes = 0;
+    if (tile < p.n_tiles) {  // the first tile's fetch overlaps the table staging
+        t0 = 16ull * __ldg(p.tile_off + tile);
+        tbytes = uint32_t(16ull * __ldg(p.tile_off + tile + 1) - t0);  // the host checked >= 160
+        if (tbytes <= kBuf) stage(tile, t0, tbytes);
+    }
     if (BUILD) {
         build_tables<WARPS>(sm, p);
         __syncthreads();
     } else if (!mbar_wait(&sm.tbar, 0)) {
         if (lane == 0) atomicOr(p.status, kStTimeout);
-        goto timeout;
+        goto drain;
     }
 
     {
         const uint32_t sym0 = smem_u32(&sm.sym[0][0]), fc0 = smem_u32(&sm.fc[0][0][0]);
         bool first = true;
         for (; tile < p.n_tiles; tile += tile_stride) {
-            if (!first) begin_tile();
+            if (!first) {
+                t0 = 16ull * __ldg(p.tile_off + tile);
+                tbytes = uint32_t(16ull * __ldg(p.tile_off + tile + 1) - t0);
+                if (tbytes <= kBuf) stage(tile, t0, tbytes);
+            }
             first = false;
-            const int64_t per_tile = int64_t(kLanes) * p.steps;
-            const int64_t v0 = int64_t(tile) * per_tile;
-            const int64_t vend = min(v0 + per_tile, p.n_vectors);
-            const uint32_t nsteps = uint32_t((vend - v0 + kLanes - 1) / kLanes);
-            int64_t v = v0 + lane;
-            int64_t row = v / p.vec_per_row, kcol = v - row * p.vec_per_row;
-            uint32_t cur = rofs;  // ring position of the next unread byte
-            uint32_t flags = 0;
-            for (uint32_t k = 0; k < nsteps; ++k) {
-                // keep the ring full and the bytes this step may read resident
-                const uint32_t done = cur - rofs;  // bytes of this tile consumed so far
-                const uint32_t lim = min(nch, done / kChunk + kRingChunks);
-                while (issued < lim) issue(issued++);
-                const uint32_t need = (min(bytes, done + uint32_t(kMaxStepBytes)) + kChunk - 1) / kChunk;
-                while (waited < need) {
-                    if (!wait(waited)) goto timeout;
-                    ++waited;
+            const bool in_smem = tbytes <= kBuf;
+            const uint8_t* tg = p.stream + t0;
+            if (in_smem) {
+                if (!mbar_wait(&sm.bar[warp], staged & 1u)) {
+                    if (lane == 0) atomicOr(p.status, kStTimeout);
+                    return;  // nothing else is in flight into this warp's buffer
                 }
-                const uint32_t pos0 = ring_a + (cur & (kRing - 1));
-                uint32_t pos = pos0;
-                if (v0 + int64_t(k + 1) * kLanes <= vend)
-                    decode_step<OUT, VEC, true>(p, sym0, fc0, pos, x, true, lt, v, row, kcol);
-                else
-                    decode_step<OUT, VEC, false>(p, sym0, fc0, pos, x, v < vend, lt, v, row, kcol);
-                cur += pos - pos0;
-                if (cur - rofs > bytes) {
-                    flags |= kStOverrun;
-                    break;
-                }
-                v += kLanes;
-                kcol += kLanes;
-                while (kcol >= p.vec_per_row) {
-                    kcol -= p.vec_per_row;
-                    ++row;
-                }
+                ++staged;
             }
-            // drain copies the decode did not need (padding) before the slots are reused
-            while (waited < issued) {
-                if (!wait(waited)) goto timeout;
-                ++waited;
+            // tile header: this lane's state; a warp-shuffle prefix sum over the 16 region
+            // word counts gives each lane its region
+            uint32_t x, cnt;
+            if (in_smem) {
+                x = lds_u32(buf_a + 4 * lane);
+                cnt = lane < uint32_t(kPairs) ? lds_u16(buf_a + 4 * kLanes + 2 * lane) : 0u;
+            } else {
+                x = __ldg(reinterpret_cast<const uint32_t*>(tg) + lane);
+                cnt = lane < uint32_t(kPairs) ? __ldg(reinterpret_cast<const uint16_t*>(tg + 4 * kLanes) + lane) : 0u;
             }
+            uint32_t inc = cnt;
+#pragma unroll
+            for (int o = 1; o < kPairs; o <<= 1) {
+                const uint32_t t = __shfl_up_sync(kFull, inc, o);
+                if (lane >= uint32_t(o)) inc += t;
+            }
+            const uint32_t start = __shfl_sync(kFull, inc - cnt, lane >> 1);
+            const uint32_t n_region = __shfl_sync(kFull, cnt, lane >> 1);
+            const uint32_t total_words = __shfl_sync(kFull, inc, kPairs - 1);
+            const int32_t w0 = fwd ? int32_t(start) : int32_t(start + n_region) - 1;  // first word
+            const int32_t o0 = int32_t(kTileHeadBytes) + 2 * w0;                     // byte offset
+            uint32_t flags, nread;
+            if (in_smem) {
+                SmemReader rd;
+                rd.wd = fwd ? 2 : -2;
+                rd.wp = buf_a + uint32_t(min(max(o0, 0), int32_t(tbytes) - 2));
+                rd.wn = lds_u16(rd.wp);
+                rd.nread = 0;
+                const uint32_t lo = buf_a, hi = buf_a + kBuf;
+                flags = decode_tile_steps<OUT, VEC>(p, sym0, fc0, rd, x, tile, lane,
+                                                    [=](const SmemReader& r) { return r.wp >= lo && r.wp <= hi; });
+                nread = rd.nread;
+            } else {
+                GlobalReader rd;
+                rd.tile = tg;
+                rd.wd = fwd ? 2 : -2;
+                rd.hi = int32_t(tbytes) - 2;
+                rd.off = o0;
+                rd.wn = __ldg(reinterpret_cast<const uint16_t*>(tg + min(max(o0, 0), rd.hi)));
+                rd.nread = 0;
+                flags = decode_tile_steps<OUT, VEC>(p, sym0, fc0, rd, x, tile, lane,
+                                                    [](const GlobalReader&) { return true; });
+                nread = rd.nread;
+            }
+            // integrity: every state back at 2^16; in every region the two lanes read exactly
+            // its words; the regions fill the tile up to < 16 bytes of padding
             if (!(flags & kStOverrun)) {
                 if (__any_sync(kFull, x != kStateLow)) flags |= kStState;
-                if (bytes - (cur - rofs) >= 16) flags |= kStLeftover;
+                const uint32_t pair_read = nread + __shfl_xor_sync(kFull, nread, 1);
+                if (__any_sync(kFull, pair_read != n_region)) flags |= kStLeftover;
+                const uint32_t used = uint32_t(kTileHeadBytes) + 2u * total_words;
+                if (used > tbytes) flags |= kStOverrun;
+                else if (tbytes - used >= 16) flags |= kStLeftover;
             }
             if (lane == 0 && flags) atomicOr(p.status, flags);
         }
     }
     return;
 
-timeout:
-    if (lane == 0) atomicOr(p.status, kStTimeout);
-    // wait (bounded again) for copies still in flight into this warp's ring before leaving
-    while (waited < issued) {
-        wait(waited);
-        ++waited;
-    }
+drain:
+    // the table wait failed: wait (bounded) for the first tile's copy before leaving
+    if (tile < p.n_tiles && tbytes <= kBuf) mbar_wait(&sm.bar[warp], 0);
 }
 
 // Expands the blob's compact frequency tables into the 80 KB decode-table block (one CTA).
@@ -518,7 +579,9 @@ __global__ void __launch_bounds__(WARPS * 32, 1) expand_tables_kernel(const Para
 }
 
 // ---- host-side launch -------------------------------------------------------------------------
-constexpr int kWarps = 32;
+// 32 warps per CTA when every tile fits a 4.5 KB buffer (more tiles in flight per SM), else 16
+// warps with 9 KB buffers; a tile larger than that is read from global memory.
+constexpr int kWarpsWide = 32, kWarpsNarrow = 16;
 
 struct DevInfo {
     bool ready = false;
@@ -552,17 +615,22 @@ int launch_one(const Params& p, cudaStream_t st, int device) {
 }
 
 template <int OUT>
-int launch_out(const Params& p, bool vec, cudaStream_t st, int device) {
-    return vec ? launch_one<kWarps, OUT, true>(p, st, device) : launch_one<kWarps, OUT, false>(p, st, device);
+int launch_out(const Params& p, bool vec, bool wide, cudaStream_t st, int device) {
+    if (wide)
+        return vec ? launch_one<kWarpsWide, OUT, true>(p, st, device) : launch_one<kWarpsWide, OUT, false>(p, st, device);
+    return vec ? launch_one<kWarpsNarrow, OUT, true>(p, st, device) : launch_one<kWarpsNarrow, OUT, false>(p, st, device);
 }
 
-int launch(const Params& p, int out_kind, bool vec, cudaStream_t st, int device) {
+int launch(const Params& p, int out_kind, bool vec, uint64_t max_tile, cudaStream_t st, int device) {
+    const bool wide = max_tile <= Geo<kWarpsWide>::kBuf;
     switch (out_kind) {
-        case kOutBF16: return launch_out<kOutBF16>(p, vec, st, device);
-        case kOutFP16: return launch_out<kOutFP16>(p, vec, st, device);
-        case kOutE4M3: return launch_out<kOutE4M3>(p, vec, st, device);
-        case kOutF32: return launch_out<kOutF32>(p, vec, st, device);
-        default: return launch_one<kWarps, kOutFields, false>(p, st, device);
+        case kOutBF16: return launch_out<kOutBF16>(p, vec, wide, st, device);
+        case kOutFP16: return launch_out<kOutFP16>(p, vec, wide, st, device);
+        case kOutE4M3: return launch_out<kOutE4M3>(p, vec, wide, st, device);
+        case kOutF32: return launch_out<kOutF32>(p, vec, wide, st, device);
+        default:
+            return wide ? launch_one<kWarpsWide, kOutFields, false>(p, st, device)
+                        : launch_one<kWarpsNarrow, kOutFields, false>(p, st, device);
     }
 }
 
@@ -639,10 +707,10 @@ int ensure_device(ep_blob* b, int dev, cudaStream_t st) {
     EP_CUDA(cudaMemsetAsync(status, 0, 16, st), "status clear");
     // expand the compact frequency tables once for this device copy
     Params p = make_params(b, blob, nullptr, nullptr, b->layout.cols, status, false);
-    auto fn = expand_tables_kernel<kWarps>;
+    auto fn = expand_tables_kernel<kWarpsWide>;
     EP_CUDA(cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, int(kTableBytes)),
             "table expansion attribute");
-    fn<<<1, kWarps * 32, kTableBytes, st>>>(p, tables);
+    fn<<<1, kWarpsWide * 32, kTableBytes, st>>>(p, tables);
     EP_CUDA(cudaGetLastError(), "table expansion launch");
     EP_CUDA(cudaStreamSynchronize(st), "blob upload");
     d.blob = blob;
@@ -695,8 +763,8 @@ int noalloc_launch_one(const Params& p, cudaStream_t st, int device) {
 
 template <int OUT>
 int noalloc_launch_out(const Params& p, bool vec, cudaStream_t st, int device) {
-    return vec ? noalloc_launch_one<kWarps, OUT, true>(p, st, device)
-               : noalloc_launch_one<kWarps, OUT, false>(p, st, device);
+    return vec ? noalloc_launch_one<kWarpsNarrow, OUT, true>(p, st, device)
+               : noalloc_launch_one<kWarpsNarrow, OUT, false>(p, st, device);
 }
 
 int noalloc_launch(const Params& p, int out_kind, bool vec, cudaStream_t st, int device) {
@@ -749,7 +817,7 @@ extern "C" int ep_decompress(const ep_blob* cb, const ep_tensor* out, void* stre
         const DeviceCopy& d = b->dev[dev];
         const bool vec = vec_ok(L, out->data, out->row_stride, out->dtype);
         Params p = make_params(b, d.blob, d.tables, out->data, out->row_stride, d.status, vec);
-        return launch(p, kind, vec, st, dev);
+        return launch(p, kind, vec, L.max_tile_bytes, st, dev);
     }
 
     // Host output: upload the bytes, decode into a blob-owned buffer, copy back, synchronise.
@@ -783,7 +851,7 @@ extern "C" int ep_decompress(const ep_blob* cb, const ep_tensor* out, void* stre
             "ep_decompress: upload");
     const bool vec = vec_ok(L, d.stage_out, L.cols, out->dtype);
     Params p = make_params(b, d.stage_blob, d.tables, d.stage_out, L.cols, d.status, vec);
-    rc = launch(p, kind, vec, st, dev);
+    rc = launch(p, kind, vec, L.max_tile_bytes, st, dev);
     if (rc != EP_OK) return rc;
     EP_CUDA(cudaMemcpy2DAsync(out->data, size_t(out->row_stride) * es, d.stage_out, size_t(L.cols) * es,
                               size_t(L.cols) * es, size_t(L.rows), cudaMemcpyDeviceToHost, st),
@@ -803,7 +871,7 @@ extern "C" int ep_decode_fields(const ep_blob* cb, int16_t* fields, void* stream
     if (rc != EP_OK) return rc;
     const DeviceCopy& d = b->dev[dev];
     Params p = make_params(b, d.blob, d.tables, fields, b->layout.cols, d.status, false);
-    return launch(p, kOutFields, false, st, dev);
+    return launch(p, kOutFields, false, b->layout.max_tile_bytes, st, dev);
 }
 
 extern "C" int ep_decode_status(const ep_blob* cb, void* stream) {

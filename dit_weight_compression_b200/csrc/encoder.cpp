@@ -253,19 +253,19 @@ struct Tables {
 };
 
 // ---------------------------------------------------------------------------------------------
-// Tiled, 32-way interleaved rANS.  Decode order of a tile: for each step, sub-steps 0 (coset)
-// and 1..8 (fields); in a sub-step, lanes whose state drops below 2^16 read the next word in
-// ascending lane order; after sub-step 8 the raw words of escaped fields, by field then lane.
-// The encoder walks that order backwards and reverses its words.
+// Tiled, 32-way interleaved rANS.  Lane l of a tile owns vectors l, 32 + l, 64 + l, ... and one
+// 32-bit state.  A lane reads its own words: for each step, after each of its 9 decodes (coset,
+// f1..f8) one word if the state fell below 2^16, then the raw words of its escaped fields in
+// field order.  Lanes 2p and 2p+1 share region p: lane 2p reads forward from the region start,
+// lane 2p+1 backward from the region end.  Tile: 32 u32 states, 16 u16 region word counts, the
+// regions, zero padding to 16 bytes.  Each lane is encoded in reverse reading order.
 // ---------------------------------------------------------------------------------------------
 static void encode_tile(const uint8_t* coset, const int16_t* fields, int64_t nvec, const Tables& T,
                         std::vector<uint8_t>& out) {
     uint32_t x[kLanes];
-    std::fill(x, x + kLanes, kStateLow);
-    std::vector<uint16_t> w;
-    w.reserve(size_t(nvec) * 5);
-    int64_t steps = (nvec + kLanes - 1) / kLanes;
-    auto put = [&](uint32_t& st, int ctx, int sym) {
+    std::vector<uint16_t> lw[kLanes];  // emission order (reverse of reading order)
+    const int64_t steps = (nvec + kLanes - 1) / kLanes;
+    auto put = [&](uint32_t& st, std::vector<uint16_t>& w, int ctx, int sym) {
         uint32_t f = T.q[ctx][sym], c = T.cum[ctx][sym];
         if (uint64_t(st) >= (uint64_t(f) << (32 - kProbBits))) {  // renormalise: push 16 bits out
             w.push_back(uint16_t(st));
@@ -273,25 +273,33 @@ static void encode_tile(const uint8_t* coset, const int16_t* fields, int64_t nve
         }
         st = (st / f) * kProbTotal + (st % f) + c;
     };
-    for (int64_t k = steps - 1; k >= 0; --k) {
-        int64_t first = k * kLanes;
-        int lanes = int(std::min<int64_t>(kLanes, nvec - first));
-        for (int j = 7; j >= 0; --j)
-            for (int l = lanes - 1; l >= 0; --l) {
-                int16_t f = fields[size_t(8 * (first + l) + j)];
-                if (symbol_of(f) == kEscape) w.push_back(uint16_t(f));
-            }
-        for (int j = 7; j >= 0; --j)
-            for (int l = lanes - 1; l >= 0; --l) {
-                int64_t v = first + l;
-                put(x[l], 1 + 8 * coset[v] + j, symbol_of(fields[size_t(8 * v + j)]));
-            }
-        for (int l = lanes - 1; l >= 0; --l) put(x[l], 0, coset[first + l]);
+    for (int l = 0; l < kLanes; ++l) {
+        x[l] = kStateLow;
+        lw[l].reserve(size_t(steps) * 5);
+        for (int64_t k = steps - 1; k >= 0; --k) {
+            const int64_t v = k * kLanes + l;
+            if (v >= nvec) continue;
+            const int16_t* f = &fields[size_t(8 * v)];
+            for (int j = 7; j >= 0; --j)
+                if (symbol_of(f[j]) == kEscape) lw[l].push_back(uint16_t(f[j]));
+            for (int j = 7; j >= 0; --j) put(x[l], lw[l], 1 + 8 * coset[v] + j, symbol_of(f[j]));
+            put(x[l], lw[l], 0, coset[v]);
+        }
     }
-    size_t bytes = round_up16(kTileHeadBytes + 2 * w.size());
-    out.assign(bytes, 0);
+    size_t words = 0;
+    for (auto& w : lw) words += w.size();
+    out.assign(round_up16(kTileHeadBytes + 2 * words), 0);
     for (int l = 0; l < kLanes; ++l) wr32(&out[size_t(4 * l)], x[l]);
-    for (size_t i = 0; i < w.size(); ++i) wr16(&out[kTileHeadBytes + 2 * i], w[w.size() - 1 - i]);
+    size_t r = kTileHeadBytes;  // byte offset of the current region
+    for (int p = 0; p < kPairs; ++p) {
+        const auto& fw = lw[2 * p];
+        const auto& bw = lw[2 * p + 1];
+        const size_t n = fw.size() + bw.size();
+        wr16(&out[size_t(4 * kLanes + 2 * p)], uint32_t(n));
+        for (size_t i = 0; i < fw.size(); ++i) wr16(&out[r + 2 * i], fw[fw.size() - 1 - i]);
+        for (size_t i = 0; i < bw.size(); ++i) wr16(&out[r + 2 * (n - 1 - i)], bw[bw.size() - 1 - i]);
+        r += 2 * n;
+    }
 }
 
 // ---------------------------------------------------------------------------------------------
@@ -334,8 +342,8 @@ int encode(const EncodeInput& in, double target, const EncodeOptions& opt, std::
 
     // Size estimate at scale s from min(rows, 256) rows at floor(i * rows / n): coded bits under
     // the sample's own 12-bit tables plus 16 bits per escape, scaled to all rows, plus the exact
-    // metadata (header, tables, row scales, tile offsets) and 136 bytes per tile (32 states and
-    // the mean padding).
+    // metadata (header, tables, row scales, tile offsets) and 168 bytes per tile (32 states, 16
+    // region counts and the mean padding).
     const int64_t n_sample = std::min<int64_t>(rows, 256);
     auto estimate = [&](double s) {
         std::vector<Counts> part(static_cast<size_t>(threads));
@@ -362,7 +370,7 @@ int encode(const EncodeInput& in, double target, const EncodeOptions& opt, std::
         double payload = (double(rows) / double(n_sample)) * (bits / 8.0 + 2.0 * double(all.escapes));
         double meta = double(kHeaderBytes + round_up16(T.section_bytes()) + round_up16(4 * uint64_t(rows)) +
                              round_up16(4 * uint64_t(n_tiles + 1))) +
-                      double(n_tiles) * (128.0 + 8.0);
+                      double(n_tiles) * (160.0 + 8.0);
         return 8.0 * (meta + payload) / (double(rows) * double(cols));
     };
 
@@ -413,7 +421,7 @@ int encode(const EncodeInput& in, double target, const EncodeOptions& opt, std::
     Tables T;
     T.build(all);
 
-    // Tiles.
+    // Tiles.  (A region's word count is a u16: at most 2 * 17 * S words, fine for S <= 1024.)
     std::vector<std::vector<uint8_t>> tiles(static_cast<size_t>(n_tiles));
     parallel_for(n_tiles, threads, [&](int64_t a, int64_t b, int) {
         for (int64_t t = a; t < b; ++t) {
@@ -501,7 +509,7 @@ bool parse_blob(const uint8_t* d, size_t n, BlobLayout& L, std::string& why) {
     if (L.total != n) return fail("stored size differs from the byte count");
     if (L.rows <= 0 || L.cols <= 0 || L.rows > (int64_t(1) << 40) || L.cols > (int64_t(1) << 40))
         return fail("bad shape");
-    if (L.steps == 0 || L.steps > (1u << 20)) return fail("bad steps per tile");
+    if (L.steps == 0 || L.steps > 1024) return fail("bad steps per tile");
     L.vec_per_row = (L.cols + 7) / 8;
     L.n_vectors = L.rows * L.vec_per_row;
     int64_t per = int64_t(kLanes) * L.steps;
@@ -536,7 +544,8 @@ bool parse_blob(const uint8_t* d, size_t n, BlobLayout& L, std::string& why) {
     if (rd32(off) != 0) return fail("first tile offset is not 0");
     for (uint64_t i = 1; i <= L.n_tiles; ++i) {
         uint64_t o = uint64_t(rd32(off + 4 * i)) * 16;
-        if (o < prev + kTileHeadBytes) return fail("tile shorter than its 128-byte state block");
+        if (o < prev + kTileHeadBytes) return fail("tile shorter than its 160-byte header");
+        L.max_tile_bytes = std::max<uint64_t>(L.max_tile_bytes, o - prev);
         prev = o;
     }
     if (prev != stream) return fail("tile offsets do not end at the stream end");

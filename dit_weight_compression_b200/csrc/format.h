@@ -12,8 +12,9 @@
 //                      u16 q(escape), u8 lo, u8 n, u16 q[lo .. lo + n - 1]
 //   row scales:        f32 per row
 //   tile offsets:      u32[n_tiles + 1], in 16-byte units from the stream start
-//   stream:            per tile: 32 u32 initial rANS states (lane order), u16 words in decode
-//                      order, zero padding to a multiple of 16 bytes
+//   stream:            per tile: 32 u32 initial rANS states (lane order), 16 u16 region word
+//                      counts, the regions (lane 2p's words forward from the region start, lane
+//                      2p+1's backward from its end), zero padding to a multiple of 16 bytes
 //
 // Symbols: field value f with |f| <= 127 is the symbol f + 127; any other value is the escape
 // symbol 255 followed by the raw int16 word.  Frequencies of every used context sum to 4096.
@@ -33,9 +34,10 @@ constexpr uint32_t kProbBits = 12;
 constexpr uint32_t kProbTotal = 1u << kProbBits;  // 4096
 constexpr uint32_t kStateLow = 1u << 16;          // rANS lower bound, 16-bit renormalisation
 constexpr int kLanes = 32;                        // interleaved states per tile
+constexpr int kPairs = kLanes / 2;                // lanes 2p, 2p+1 share word region p
 constexpr int kFieldContexts = 16;                // (coset c, field j) -> 8c + j - 1
 constexpr size_t kHeaderBytes = 80;
-constexpr size_t kTileHeadBytes = 4 * kLanes;     // 32 x u32 states
+constexpr size_t kTileHeadBytes = 4 * kLanes + 2 * kPairs;  // 32 u32 states + 16 u16 counts
 constexpr double kTargetMin = 0.001, kTargetMax = 11.0;
 
 enum Dtype : int { kBF16 = 1, kFP16 = 2, kE4M3 = 3, kF32 = 4 };
@@ -56,6 +58,7 @@ struct BlobLayout {
     int dtype = 0;
     int64_t rows = 0, cols = 0, vec_per_row = 0, n_vectors = 0;
     uint32_t steps = 0, n_tiles = 0;
+    uint64_t max_tile_bytes = 0;  // largest tile (selects the decoder's shared-memory layout)
     double scale = 0.0;
     uint64_t total = 0, off_tables = 0, off_alpha = 0, off_offsets = 0, off_stream = 0;
     uint16_t q_coset[2] = {0, 0};

@@ -62,7 +62,7 @@ typedef struct {
 
 /* Optional encoder settings (ep_compress uses all defaults). */
 typedef struct {
-    int steps_per_tile;  /* S: tile = 32*S vectors; 0 = clamp(next_pow2(ceil(128/bpp)), 16, 1024) */
+    int steps_per_tile;  /* S in [1, 1024]: tile = 32*S vectors; 0 = clamp(next_pow2(ceil(128/bpp)), 16, 1024) */
     int num_threads;     /* host encoder threads; 0 = all hardware threads                       */
     double scale;        /* > 0: use this lattice scale instead of searching for one             */
 } ep_options;

@@ -382,17 +382,23 @@ static void cumulate(const uint16_t q[256], uint32_t cum[257])
 static int context_of(int u, int c) { return u == 0 ? 0 : 1 + 8 * c + (u - 1); }
 
 /* ------------------------------------------------------------------------------------------ */
-/* Tiled, 32-way interleaved rANS [ANS] with the word order of the format ([DOC-ER]: "encoded   */
+/* Tiled, 32-way interleaved rANS [ANS] with the word layout of the format ([DOC-ER]: "encoded  */
 /* with rANS in independently decodable tiles").                                               */
 /*                                                                                            */
 /* One tile holds up to 32*S consecutive vectors; lane l at step k owns vector 32k + l of the  */
-/* tile.  Each vector is 9 symbols: the coset (context 0) and f1..f8 (context 1 + 8c + j - 1).  */
-/* Decode order: for each step k, for each sub-step u = 0..8, lanes 0..31 in turn decode their */
-/* symbol and, if the 32-bit state fell below 2^16, read the next 16-bit word; after sub-step 8 */
-/* the raw words of escaped fields follow, ordered by field j = 1..8, then lane.               */
-/* Tile bytes: 32 little-endian u32 initial states (lane order), the u16 words in decode order, */
-/* zero padding to a multiple of 16 bytes.  Every lane ends in state 2^16.                     */
+/* tile and has its own 32-bit rANS state.  Each vector is 9 symbols: the coset (context 0) and */
+/* f1..f8 (context 1 + 8c + j - 1).  A lane's words, in the order it reads them: for each step, */
+/* for each sub-step u = 0..8, after decoding its symbol, one 16-bit word if the state fell    */
+/* below 2^16; after sub-step 8 the raw words of its escaped fields, by field.                 */
+/* reading: lanes 2p and 2p+1 share region p: lane 2p's words run forward from the region's    */
+/* start, lane 2p+1's run backward from its end.                                                */
+/* Tile bytes: 32 little-endian u32 initial states (lane order); 16 u16 word counts of the      */
+/* regions (pairs); the regions in pair order; zero padding to a multiple of 16 bytes.  Every  */
+/* lane ends in state 2^16, and in every region the two lanes' words meet exactly.             */
 /* ------------------------------------------------------------------------------------------ */
+
+#define ORC_PAIRS (ORC_LANES / 2)
+#define ORC_TILE_HEAD (4 * ORC_LANES + 2 * ORC_PAIRS)   /* 160 bytes: states + region counts */
 
 typedef struct {
     uint16_t* w;
@@ -402,7 +408,7 @@ typedef struct {
 static int push_word(wordbuf* b, uint32_t v)
 {
     if (b->n == b->cap) {
-        uint64_t nc = b->cap ? 2 * b->cap : 1024;
+        uint64_t nc = b->cap ? 2 * b->cap : 64;
         uint16_t* nw = (uint16_t*)realloc(b->w, nc * sizeof(uint16_t));
         if (!nw) return -1;
         b->w = nw;
@@ -420,7 +426,8 @@ static int push_word(wordbuf* b, uint32_t v)
  *
  * rANS encode of symbol s with frequency q and cumulative cum [ANS]: while x >= q * 2^20,
  * emit the low 16 bits of x and shift them out; then x <- floor(x / q) * 4096 + (x mod q) + cum.
- * The encoder runs in reverse decode order and the emitted words are reversed at the end.
+ * Each lane is encoded on its own, in reverse of its reading order, and its words are reversed
+ * at the end.
  */
 uint64_t orc_encode_tile(const uint8_t* sym9, const int16_t* raw8, int64_t nvec,
                          const uint16_t* q17, uint8_t* out, uint64_t cap)
@@ -428,42 +435,57 @@ uint64_t orc_encode_tile(const uint8_t* sym9, const int16_t* raw8, int64_t nvec,
     uint32_t cum[ORC_NCTX][257];
     for (int c = 0; c < ORC_NCTX; c++) cumulate(q17 + 256 * c, cum[c]);
     uint32_t x[ORC_LANES];
-    for (int l = 0; l < ORC_LANES; l++) x[l] = ORC_L;
-    wordbuf wb = {0, 0, 0};
+    wordbuf wb[ORC_LANES];
+    memset(wb, 0, sizeof wb);
     int64_t nsteps = (nvec + ORC_LANES - 1) / ORC_LANES;
-    for (int64_t k = nsteps - 1; k >= 0; k--) {
-        for (int j = 8; j >= 1; j--)
-            for (int l = ORC_LANES - 1; l >= 0; l--) {
-                int64_t v = k * ORC_LANES + l;
-                if (v < nvec && sym9[v * 9 + j] == ORC_ESC)
-                    if (push_word(&wb, (uint16_t)raw8[v * 8 + (j - 1)])) goto fail;
-            }
-        for (int u = 8; u >= 0; u--)
-            for (int l = ORC_LANES - 1; l >= 0; l--) {
-                int64_t v = k * ORC_LANES + l;
-                if (v >= nvec) continue;
+    uint64_t bytes = 0;
+    for (int l = 0; l < ORC_LANES; l++) {
+        x[l] = ORC_L;
+        for (int64_t k = nsteps - 1; k >= 0; k--) {
+            int64_t v = k * ORC_LANES + l;
+            if (v >= nvec) continue;
+            for (int j = 8; j >= 1; j--)
+                if (sym9[v * 9 + j] == ORC_ESC)
+                    if (push_word(&wb[l], (uint16_t)raw8[v * 8 + (j - 1)])) goto fail;
+            for (int u = 8; u >= 0; u--) {
                 int s = sym9[v * 9 + u];
                 int ctx = context_of(u, sym9[v * 9]);
                 uint32_t q = q17[256 * ctx + s];
                 if (q == 0) goto fail;
                 if ((uint64_t)x[l] >= ((uint64_t)q << 20)) {
-                    if (push_word(&wb, x[l] & 0xFFFFu)) goto fail;
+                    if (push_word(&wb[l], x[l] & 0xFFFFu)) goto fail;
                     x[l] >>= 16;
                 }
                 x[l] = (x[l] / q) * ORC_M + (x[l] % q) + cum[ctx][s];
             }
+        }
     }
-    uint64_t bytes = pad16(4u * ORC_LANES + 2u * wb.n);
-    if (out && cap >= bytes) {
-        memset(out, 0, bytes);
-        for (int l = 0; l < ORC_LANES; l++) put32(out + 4 * l, x[l]);
-        for (uint64_t i = 0; i < wb.n; i++)                      /* reversed emission order */
-            put16(out + 4 * ORC_LANES + 2 * i, wb.w[wb.n - 1 - i]);
+    {
+        uint64_t words = 0;
+        for (int l = 0; l < ORC_LANES; l++) words += wb[l].n;
+        for (int p = 0; p < ORC_PAIRS; p++)
+            if (wb[2 * p].n + wb[2 * p + 1].n > 0xFFFFu) goto fail;
+        bytes = pad16(ORC_TILE_HEAD + 2u * words);
+        if (out && cap >= bytes) {
+            memset(out, 0, bytes);
+            for (int l = 0; l < ORC_LANES; l++) put32(out + 4 * l, x[l]);
+            uint8_t* r = out + ORC_TILE_HEAD;
+            for (int p = 0; p < ORC_PAIRS; p++) {
+                const wordbuf* e = &wb[2 * p];       /* forward lane */
+                const wordbuf* o = &wb[2 * p + 1];   /* backward lane */
+                uint64_t n = e->n + o->n;
+                put16(out + 4 * ORC_LANES + 2 * p, (uint32_t)n);
+                /* reading order is the reverse of emission order */
+                for (uint64_t i = 0; i < e->n; i++) put16(r + 2 * i, e->w[e->n - 1 - i]);
+                for (uint64_t i = 0; i < o->n; i++) put16(r + 2 * (n - 1 - i), o->w[o->n - 1 - i]);
+                r += 2 * n;
+            }
+        }
     }
-    free(wb.w);
+    for (int l = 0; l < ORC_LANES; l++) free(wb[l].w);
     return bytes;
 fail:
-    free(wb.w);
+    for (int l = 0; l < ORC_LANES; l++) free(wb[l].w);
     return 0;
 }
 
@@ -489,49 +511,62 @@ static void build_dtables(const uint16_t* q17, dtables* T)
  * Decode one tile of nvec vectors with prepared tables.  Writes sym9 / raw8 as orc_encode_tile
  * reads them and the 32 final states.  rANS decode [ANS]: slot = x mod 4096, s = the symbol with
  * cum[s] <= slot < cum[s+1], x <- q_s * floor(x / 4096) + slot - cum[s]; if x < 2^16,
- * x <- x * 2^16 + next word.  Returns 0 when the tile is consistent (every state back at 2^16 and
- * every word used, up to the zero padding), 1 when it is not, -1 when the words ran out.
+ * x <- x * 2^16 + the lane's next word.  Returns 0 when the tile is consistent (every state back
+ * at 2^16, the two lanes of every region meeting exactly, only padding after the last region),
+ * 1 when it is not, -1 when a lane's words ran outside the tile.
  */
 static int decode_tile(const uint8_t* tile, uint64_t nbytes, int64_t nvec, const dtables* T,
                        uint8_t* sym9, int16_t* raw8, uint32_t* final_states)
 {
-    if (nbytes < 4u * ORC_LANES) return -1;
-    uint32_t x[ORC_LANES];
-    for (int l = 0; l < ORC_LANES; l++) x[l] = get32(tile + 4 * l);
-    const uint8_t* words = tile + 4 * ORC_LANES;
-    uint64_t nwords = (nbytes - 4u * ORC_LANES) / 2u, pos = 0;
-    int64_t nsteps = (nvec + ORC_LANES - 1) / ORC_LANES;
-    for (int64_t k = 0; k < nsteps; k++) {
-        for (int u = 0; u <= 8; u++)
-            for (int l = 0; l < ORC_LANES; l++) {
-                int64_t v = k * ORC_LANES + l;
-                if (v >= nvec) continue;
-                int ctx = context_of(u, u == 0 ? 0 : sym9[v * 9]);
-                uint32_t slot = x[l] & (ORC_M - 1);
-                int s = T->slot_sym[ctx][slot];
-                uint32_t q = T->q17[256 * ctx + s];
-                x[l] = q * (x[l] >> 12) + slot - T->cum[ctx][s];
-                sym9[v * 9 + u] = (uint8_t)s;
-                if (x[l] < ORC_L) {
-                    if (pos >= nwords) return -1;
-                    x[l] = (x[l] << 16) | get16(words + 2 * pos++);
-                }
-            }
-        for (int j = 1; j <= 8; j++)
-            for (int l = 0; l < ORC_LANES; l++) {
-                int64_t v = k * ORC_LANES + l;
-                if (v < nvec && sym9[v * 9 + j] == ORC_ESC) {
-                    if (pos >= nwords) return -1;
-                    raw8[v * 8 + (j - 1)] = (int16_t)get16(words + 2 * pos++);
-                }
-            }
+    if (nbytes < ORC_TILE_HEAD) return -1;
+    int64_t nwords = (int64_t)(nbytes - ORC_TILE_HEAD) / 2;
+    const uint8_t* words = tile + ORC_TILE_HEAD;
+    int64_t start[ORC_PAIRS], count[ORC_PAIRS], total = 0;
+    for (int p = 0; p < ORC_PAIRS; p++) {
+        count[p] = get16(tile + 4 * ORC_LANES + 2 * p);
+        start[p] = total;
+        total += count[p];
     }
+    if (total > nwords) return -1;
+    int64_t nsteps = (nvec + ORC_LANES - 1) / ORC_LANES;
+    int64_t used[ORC_LANES];
     int bad = 0;
     for (int l = 0; l < ORC_LANES; l++) {
-        if (final_states) final_states[l] = x[l];
-        if (x[l] != ORC_L) bad = 1;
+        int p = l / 2, fwd = (l % 2) == 0;
+        uint32_t x = get32(tile + 4 * l);
+        int64_t n = 0;   /* words this lane has read */
+        for (int64_t k = 0; k < nsteps; k++) {
+            int64_t v = k * ORC_LANES + l;
+            if (v >= nvec) continue;
+            for (int u = 0; u <= 8; u++) {
+                int ctx = context_of(u, u == 0 ? 0 : sym9[v * 9]);
+                uint32_t slot = x & (ORC_M - 1);
+                int s = T->slot_sym[ctx][slot];
+                uint32_t q = T->q17[256 * ctx + s];
+                x = q * (x >> 12) + slot - T->cum[ctx][s];
+                sym9[v * 9 + u] = (uint8_t)s;
+                if (x < ORC_L) {
+                    int64_t w = fwd ? start[p] + n : start[p] + count[p] - 1 - n;
+                    if (n >= count[p]) return -1;
+                    x = (x << 16) | get16(words + 2 * w);
+                    n++;
+                }
+            }
+            for (int j = 1; j <= 8; j++)
+                if (sym9[v * 9 + j] == ORC_ESC) {
+                    int64_t w = fwd ? start[p] + n : start[p] + count[p] - 1 - n;
+                    if (n >= count[p]) return -1;
+                    raw8[v * 8 + (j - 1)] = (int16_t)get16(words + 2 * w);
+                    n++;
+                }
+        }
+        used[l] = n;
+        if (final_states) final_states[l] = x;
+        if (x != ORC_L) bad = 1;
     }
-    if (nbytes - 4u * ORC_LANES - 2u * pos >= 16u) bad = 1;
+    for (int p = 0; p < ORC_PAIRS; p++)
+        if (used[2 * p] + used[2 * p + 1] != count[p]) bad = 1;
+    if (nbytes - ORC_TILE_HEAD - 2u * (uint64_t)total >= 16u) bad = 1;
     return bad;
 }
 
@@ -634,7 +669,7 @@ static uint64_t table_section_bytes(const uint16_t* q17)
  * reading: n_s = min(rows, 256) rows at floor(i * rows / n_s); tables are quantised from the
  * sample's counts; coded size = sum over contexts and symbols of n * -log2(q / 4096) bits plus
  * 16 bits per escape, scaled by rows / n_s; metadata = exact header, table, row-scale and
- * tile-offset bytes, plus 128 state bytes and 8 padding bytes per tile.
+ * tile-offset bytes, plus 160 header bytes (states, region counts) and 8 padding bytes per tile.
  * With full_sample != 0 every row is used (n_s = rows).
  */
 static double estimate_bpp(const matrix* m, double s, int64_t S, int full_sample)
@@ -668,7 +703,7 @@ static double estimate_bpp(const matrix* m, double s, int64_t S, int full_sample
     int64_t ntiles = (V + 32 * S - 1) / (32 * S);
     double meta = (double)(ORC_HEADER + pad16(table_section_bytes(q17)) + pad16(4u * (uint64_t)m->rows) +
                            pad16(4u * (uint64_t)(ntiles + 1))) +
-                  (double)ntiles * (128.0 + 8.0);
+                  (double)ntiles * (160.0 + 8.0);
     free(cnt);
     return 8.0 * (meta + payload) / ((double)m->rows * (double)m->cols);
 }
@@ -756,6 +791,7 @@ int orc_compress(const void* data, int dtype, int64_t rows, int64_t cols, double
     memset(&m, 0, sizeof m);
     int rc = load_matrix(&m, data, dtype, rows, cols);
     if (rc) { free_matrix(&m); return rc; }
+    if (steps_per_tile > 1024) { free_matrix(&m); return -4; }   /* region counts are u16 */
     int64_t S = steps_per_tile > 0 ? steps_per_tile : default_steps(target_bpp);
     double s = scale_override > 0 ? scale_override : choose_scale(&m, target_bpp, S);
 

@@ -198,21 +198,24 @@ def test_rans_closed_form_one_bit_symbols():
     """Two steps, 32 lanes, every field one bit (q = 2048 for f = 0 and f = 1), coset free
     (q = 4096).  Encoding x <- floor(x/2048)*4096 + (x mod 2048) + 2048*b from x = 2^16 gives,
     after n bits b_1..b_n (first encoded first), x = 2^(16+n) + 2048 * sum_i b_i 2^(n-i) while
-    x < 2^31.  The encoder meets its 16 bits in reverse decode order: step 1 f8..f1, then step 0
+    x < 2^31.  A lane meets its 16 bits in reverse reading order: step 1 f8..f1, then step 0
     f8..f1; before the 16th (step 0, f1) x = 2^31 + 2048*B15 >= 2^31, so it emits the low 16 bits
     2048*(B15 mod 32) and keeps 2^15 + (B15 >> 5); encoding f1 then gives the initial state
     2^16 + 2048*f1 + (B15 >> 5).  B15 mod 32 = 16 f6 + 8 f5 + 4 f4 + 2 f3 + f2 (step 0), and
-    B15 >> 5 = 4*(128 f8 + 64 f7 + ... + f1 of step 1) + 2 f8 + f7 (step 0).  Every lane refills
-    at step 0 sub-step 1, so the tile holds 32 states and then one word per lane in lane order."""
+    B15 >> 5 = 4*(128 f8 + 64 f7 + ... + f1 of step 1) + 2 f8 + f7 (step 0).  Every lane has
+    exactly one word, so each region holds 2 words: lane 2p's (read forward from the region
+    start) then lane 2p+1's (read backward from the region end) -- lane order overall."""
     q17 = _tables({127: 2048, 128: 2048})
     bits = RNG.integers(0, 2, (64, 8))                              # vector v = 32k + lane
     sym9 = np.zeros((64, 9), np.uint8)
     sym9[:, 1:] = 127 + bits
     raw8 = np.zeros((64, 8), np.int16)
     tile = oracle.encode_tile(sym9, raw8, q17)
-    assert len(tile) == 128 + 64
+    assert len(tile) == 160 + 64
     states = np.frombuffer(tile[:128], "<u4")
-    words = np.frombuffer(tile[128:], "<u2")
+    counts = np.frombuffer(tile[128:160], "<u2")
+    words = np.frombuffer(tile[160:], "<u2")
+    assert np.all(counts == 2)
     for lane in range(32):
         f0 = bits[lane]            # step 0: f1..f8 at indices 0..7
         f1 = bits[32 + lane]       # step 1
@@ -226,8 +229,9 @@ def test_rans_closed_form_one_bit_symbols():
 
 
 def test_rans_all_escape_closed_form():
-    """Coset free, every field the escape symbol with q = 4096: no state ever changes, so the
-    tile is 32 states of 2^16 followed by the raw values in order step, field, lane."""
+    """Coset free, every field the escape symbol with q = 4096: no state ever changes, so each
+    lane's words are its raw values in step, field order; region p holds lane 2p's words forward
+    and lane 2p+1's words backward from the region end."""
     q17 = _tables({255: 4096})
     nvec = 70                                                       # 3 steps, the last partial
     sym9 = np.zeros((nvec, 9), np.uint8)
@@ -236,31 +240,34 @@ def test_rans_all_escape_closed_form():
     tile = oracle.encode_tile(sym9, raw8, q17)
     states = np.frombuffer(tile[:128], "<u4")
     assert np.all(states == 65536)
-    expect = []
-    for k in range(3):
-        for j in range(8):
-            for lane in range(32):
-                v = 32 * k + lane
-                if v < nvec:
-                    expect.append(raw8[v, j])
-    expect = np.array(expect, np.int16).view(np.uint16)
-    words = np.frombuffer(tile[128:128 + 2 * len(expect)], "<u2")
+    lane_words = []
+    for lane in range(32):
+        w = [raw8[32 * k + lane, j] for k in range(3) if 32 * k + lane < nvec for j in range(8)]
+        lane_words.append(np.array(w, np.int16).view(np.uint16))
+    expect, counts = [], []
+    for p in range(16):
+        e, o = lane_words[2 * p], lane_words[2 * p + 1]
+        expect += list(e) + list(o[::-1])
+        counts.append(len(e) + len(o))
+    expect = np.array(expect, np.uint16)
+    assert np.array_equal(np.frombuffer(tile[128:160], "<u2"), np.array(counts))
+    words = np.frombuffer(tile[160:160 + 2 * len(expect)], "<u2")
     assert np.array_equal(words, expect)
-    assert len(tile) == (128 + 2 * len(expect) + 15) // 16 * 16
-    assert all(b == 0 for b in tile[128 + 2 * len(expect):])
+    assert len(tile) == (160 + 2 * len(expect) + 15) // 16 * 16
+    assert all(b == 0 for b in tile[160 + 2 * len(expect):])
     rc, s9, r8, st = oracle.decode_tile(tile, nvec, q17)
     assert rc == 0 and np.array_equal(s9, sym9) and np.array_equal(r8, raw8)
 
 
 def test_rans_lone_symbols_closed_form():
     """Every context holds one symbol with q = 4096: coding it costs nothing, so the tile is
-    exactly the 32 states, all 2^16."""
+    exactly the 32 states, all 2^16, and 16 zero region counts."""
     q17 = _tables({127: 4096})
     for nvec in (1, 31, 32, 33, 1000):
         sym9 = np.full((nvec, 9), 127, np.uint8)
         sym9[:, 0] = 0
         tile = oracle.encode_tile(sym9, np.zeros((nvec, 8), np.int16), q17)
-        assert tile == np.full(32, 65536, "<u4").tobytes()
+        assert tile == np.full(32, 65536, "<u4").tobytes() + bytes(32)
         rc, s9, _, _ = oracle.decode_tile(tile, nvec, q17)
         assert rc == 0 and np.array_equal(s9, sym9)
 
@@ -312,6 +319,11 @@ def test_rans_corruption_detected():
     tile[5] ^= 0x10                                                  # flip a bit of lane 1's state
     rc, *_ = oracle.decode_tile(bytes(tile), 2048, q17)
     assert rc != 0
+    tile[5] ^= 0x10
+    tile[130] ^= 0x01                                                # a region count off by one
+    rc, *_ = oracle.decode_tile(bytes(tile), 2048, q17)
+    assert rc != 0
+    tile[130] ^= 0x01
     rc, *_ = oracle.decode_tile(bytes(tile[:-32]), 2048, q17)       # truncated
     assert rc != 0
 
@@ -329,9 +341,9 @@ def test_rans_size_near_cross_entropy():
     info = -np.log2(q / 4096.0).sum() + 16.0 * (sym9[:, 1:] == 255).sum()
     states = np.frombuffer(tile[:128], "<u4").astype(np.float64)
     held = np.log2(states / 65536.0).sum()                          # bits parked in the states
-    words_bits = 8.0 * (len(tile) - 128)
+    words_bits = 16.0 * int(np.frombuffer(tile[128:160], "<u2").astype(np.int64).sum())
     assert words_bits + held >= info - 1e-6
-    assert words_bits + held <= info + 32 * 1.0 + 8 * 16
+    assert words_bits + held <= info + 32 * 1.0
 
 
 # ---------------------------------------------------------------------------------------------
