@@ -35,6 +35,7 @@
 
 #include <algorithm>
 #include <cstddef>
+#include <type_traits>
 #include <cstdio>
 #include <mutex>
 
@@ -80,6 +81,7 @@ struct Params {
     uint32_t lo[kFieldContexts];
     uint32_t n[kFieldContexts];
     int dense;                  // element offset of vector v is 8 v
+    int tiny_alpha;             // some |alpha| < 2^-125, where alpha / 2 would round
 };
 
 constexpr uint32_t kSmemOptin = 232448;  // 227 KB: the largest dynamic shared memory of one CTA
@@ -174,15 +176,15 @@ __device__ __forceinline__ void prefetch_l2(const void* p, uint32_t bytes) {
 // one was used -- well before it is needed, so a refill costs a compare and a byte permute on
 // the dependent chain.  Predicated loads keep the warp converged.
 struct SmemReader {
-    uint32_t wp, wn, nread;
+    uint32_t wp, wn;
     int32_t wd;  // +2 (lane 2p, forward) or -2 (lane 2p+1, backward)
     __device__ __forceinline__ void consume_if(bool take) {
-        nread += take ? 1u : 0u;
-        wp += take ? uint32_t(wd) : 0u;
-        asm volatile("{\n .reg .pred p;\n setp.ne.u32 p, %1, 0;\n @p ld.shared.u16 %0, [%2];\n}"
-                     : "+r"(wn)
-                     : "r"(uint32_t(take)), "r"(wp));
+        asm volatile("{\n .reg .pred p;\n setp.ne.u32 p, %2, 0;\n @p add.u32 %1, %1, %3;\n @p ld.shared.u16 %0, [%1];\n}"
+                     : "+r"(wn), "+r"(wp)
+                     : "r"(uint32_t(take)), "r"(wd));
     }
+    // words consumed since `wp` was `wp0`
+    __device__ __forceinline__ uint32_t consumed(uint32_t wp0) const { return uint32_t(int32_t(wp - wp0) / wd); }
 };
 
 // The same for a tile too large for the buffer: words come from global memory, every address
@@ -190,24 +192,39 @@ struct SmemReader {
 struct GlobalReader {
     const uint8_t* tile;
     int32_t off, hi, wd;  // byte offset of the next word; last legal word offset; +-2
-    uint32_t wn, nread;
+    uint32_t wn;
     __device__ __forceinline__ void consume_if(bool take) {
-        nread += take ? 1u : 0u;
         off += take ? wd : 0;
         const uint8_t* src = tile + min(max(off, 0), hi);
         asm volatile("{\n .reg .pred p;\n setp.ne.u32 p, %1, 0;\n @p ld.global.nc.u16 %0, [%2];\n}"
                      : "+r"(wn)
                      : "r"(uint32_t(take)), "l"(src));
     }
+    __device__ __forceinline__ uint32_t consumed(int32_t off0) const { return uint32_t((off - off0) / wd); }
 };
 
 // Renormalisation after one decoded symbol: a lane whose state fell below 2^16 shifts in its
-// next word (x * 2^16 + w, i.e. the byte permutation {w.lo, w.hi, x.lo, x.hi}).
+// next word (x * 2^16 + w, i.e. the byte permutation {w.lo, w.hi, x.lo, x.hi}) and loads the
+// word after it.
 template <class Reader>
 __device__ __forceinline__ void renorm(uint32_t& x, Reader& rd, bool active) {
     const bool need = active && x < kStateLow;
     x = need ? __byte_perm(rd.wn, x, 0x5410) : x;
     rd.consume_if(need);
+}
+// The same for full steps from shared memory, as one predicated block: compare, permute,
+// advance, load -- no materialised predicate or select.
+__device__ __forceinline__ void renorm(uint32_t& x, SmemReader& rd) {
+    asm volatile(
+        "{\n .reg .pred p;\n setp.lt.u32 p, %0, 65536;\n @p prmt.b32 %0, %1, %0, 0x5410;\n"
+        " @p add.u32 %2, %2, %3;\n @p ld.shared.u16 %1, [%2];\n}"
+        : "+r"(x), "+r"(rd.wn), "+r"(rd.wp)
+        : "r"(rd.wd));
+}
+template <bool FULL, class Reader>
+__device__ __forceinline__ void renorm_step(uint32_t& x, Reader& rd, bool active) {
+    if constexpr (FULL && std::is_same<Reader, SmemReader>::value) renorm(x, rd);
+    else renorm(x, rd, active);
 }
 
 // ---- table expansion -------------------------------------------------------------------------
@@ -329,13 +346,14 @@ __device__ __forceinline__ void decode_step(const Params& p, uint32_t sym0, uint
     if (FULL) active = true;
     // issued early, used after the symbol chain; lanes past the last vector read nothing
     const float a = active ? __ldg(p.alpha + row) : 0.0f;
+    const float ah = __fmul_rn(a, 0.5f);  // exact unless |a| < 2^-125 (p.tiny_alpha)
 
     // coset (two symbols: slot < q0 -> 0)
     const uint32_t q0 = p.q_coset0;
     uint32_t slot = x & (kProbTotal - 1);
     const uint32_t c = slot >= q0 ? 1u : 0u;
     if (active) x = (c ? kProbTotal - q0 : q0) * (x >> kProbBits) + (slot - (c ? q0 : 0u));
-    renorm(x, rd, active);
+    renorm_step<FULL>(x, rd, active);
 
     // fields f1..f8 with context (c, j): tables of coset c start 8 contexts further on
     const uint32_t st = sym0 + c * (8u * kProbTotal);
@@ -350,7 +368,7 @@ __device__ __forceinline__ void decode_step(const Params& p, uint32_t sym0, uint
         const uint32_t q = lds_u16<(j) * 1024>(fa);                                    \
         const uint32_t cm = lds_u16<(j) * 1024 + 512>(fa);                             \
         if (active) x = q * (x >> kProbBits) + (slot - cm);                            \
-        renorm(x, rd, active);                                                         \
+        renorm_step<FULL>(x, rd, active);                                              \
         sym[j] = s;                                                                    \
         top = max(top, s);                                                             \
     }
@@ -382,10 +400,16 @@ __device__ __forceinline__ void decode_step(const Params& p, uint32_t sym0, uint
         const int32_t par = (f[0] + f[1] + f[2] + f[3] + f[4] + f[5] + f[6]) & 1;
         f[7] = 2 * f[7] + par;
         float val[8];
+        if (!p.tiny_alpha) {
+            // a * y = (a/2) * (2z + c) exactly, so one product rounds once
 #pragma unroll
-        for (int i = 0; i < 8; ++i) {
-            const float y = __fmul_rn(__int2float_rn(2 * f[i] + int32_t(c)), 0.5f);  // exact
-            val[i] = __fmul_rn(a, y);  // the one rounding of the reconstruction
+            for (int i = 0; i < 8; ++i) val[i] = __fmul_rn(ah, __int2float_rn(2 * f[i] + int32_t(c)));
+        } else {
+#pragma unroll
+            for (int i = 0; i < 8; ++i) {
+                const float y = __fmul_rn(__int2float_rn(2 * f[i] + int32_t(c)), 0.5f);  // exact
+                val[i] = __fmul_rn(a, y);  // the one rounding of the reconstruction
+            }
         }
         if constexpr (VEC) {
             const int64_t elem = p.dense ? 8 * v : row * p.row_stride + 8 * kcol;
@@ -435,6 +459,10 @@ __global__ void __launch_bounds__(WARPS * 32, 1) decode_kernel(const Params p) {
     const uint32_t lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
     const bool fwd = (lane & 1) == 0;  // lanes 2p read forward, lanes 2p+1 backward
     uint8_t* buf = sm.tbuf[warp];
+    // Launched as a programmatic dependent of the previous decode on the stream, this kernel may
+    // start while that one drains: its prologue (barriers, table and first-tile staging) only
+    // reads the blob, and it waits for the previous grid before its first global write.
+    asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
     const uint32_t buf_a = smem_u32(buf);
 
     if (threadIdx.x == 0) {
@@ -483,6 +511,7 @@ __global__ void __launch_bounds__(WARPS * 32, 1) decode_kernel(const Params p) {
         goto drain;
     }
 
+    asm volatile("griddepcontrol.wait;" ::: "memory");  // no-op unless launched as a dependent
     {
         const uint32_t sym0 = smem_u32(&sm.sym[0][0]), fc0 = smem_u32(&sm.fc[0][0][0]);
         bool first = true;
@@ -527,13 +556,14 @@ __global__ void __launch_bounds__(WARPS * 32, 1) decode_kernel(const Params p) {
             if (in_smem) {
                 SmemReader rd;
                 rd.wd = fwd ? 2 : -2;
+                // (clamped: a corrupt count must not move the first load outside the buffer; for a
+                // valid tile only a lane with no words is affected, and it reads nothing)
                 rd.wp = buf_a + uint32_t(min(max(o0, 0), int32_t(tbytes) - 2));
                 rd.wn = lds_u16(rd.wp);
-                rd.nread = 0;
-                const uint32_t lo = buf_a, hi = buf_a + kBuf;
+                const uint32_t wp0 = rd.wp, lo = buf_a, hi = buf_a + kBuf;
                 flags = decode_tile_steps<OUT, VEC>(p, sym0, fc0, rd, x, tile, lane,
                                                     [=](const SmemReader& r) { return r.wp >= lo && r.wp <= hi; });
-                nread = rd.nread;
+                nread = rd.consumed(wp0);
             } else {
                 GlobalReader rd;
                 rd.tile = tg;
@@ -541,10 +571,9 @@ __global__ void __launch_bounds__(WARPS * 32, 1) decode_kernel(const Params p) {
                 rd.hi = int32_t(tbytes) - 2;
                 rd.off = o0;
                 rd.wn = __ldg(reinterpret_cast<const uint16_t*>(tg + min(max(o0, 0), rd.hi)));
-                rd.nread = 0;
                 flags = decode_tile_steps<OUT, VEC>(p, sym0, fc0, rd, x, tile, lane,
                                                     [](const GlobalReader&) { return true; });
-                nread = rd.nread;
+                nread = rd.consumed(o0);
             }
             // integrity: every state back at 2^16; in every region the two lanes read exactly
             // its words; the regions fill the tile up to < 16 bytes of padding
@@ -591,7 +620,7 @@ std::mutex g_dev_mu;
 DevInfo g_dev[kMaxDevices];
 
 template <int WARPS, int OUT, bool VEC>
-int launch_one(const Params& p, cudaStream_t st, int device) {
+int launch_one(const Params& p, cudaStream_t st, int device, bool dependent) {
     auto fn = decode_kernel<WARPS, OUT, VEC, false>;
     const size_t smem = sizeof(Smem<WARPS>);
     static std::mutex mu;
@@ -608,29 +637,44 @@ int launch_one(const Params& p, cudaStream_t st, int device) {
         }
     }
     const uint32_t grid = uint32_t(std::min<int64_t>(int64_t(g_dev[device].sms) * per_sm[device], p.n_tiles));
-    fn<<<grid, WARPS * 32, smem, st>>>(p);
-    cudaError_t e = cudaGetLastError();
+    // A dependent launch may begin while the previous kernel on the stream drains (the kernel
+    // waits for it before writing); used only when the previous work is another decode.
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(grid);
+    cfg.blockDim = dim3(WARPS * 32);
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = st;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = dependent ? 1 : 0;
+    cudaError_t e = cudaLaunchKernelEx(&cfg, fn, p);
+    if (e == cudaSuccess) e = cudaGetLastError();
     if (e != cudaSuccess) return set_error(EP_ERR_CUDA, std::string("decode launch: ") + cudaGetErrorString(e));
     return EP_OK;
 }
 
 template <int OUT>
-int launch_out(const Params& p, bool vec, bool wide, cudaStream_t st, int device) {
+int launch_out(const Params& p, bool vec, bool wide, cudaStream_t st, int device, bool dep) {
     if (wide)
-        return vec ? launch_one<kWarpsWide, OUT, true>(p, st, device) : launch_one<kWarpsWide, OUT, false>(p, st, device);
-    return vec ? launch_one<kWarpsNarrow, OUT, true>(p, st, device) : launch_one<kWarpsNarrow, OUT, false>(p, st, device);
+        return vec ? launch_one<kWarpsWide, OUT, true>(p, st, device, dep)
+                   : launch_one<kWarpsWide, OUT, false>(p, st, device, dep);
+    return vec ? launch_one<kWarpsNarrow, OUT, true>(p, st, device, dep)
+               : launch_one<kWarpsNarrow, OUT, false>(p, st, device, dep);
 }
 
-int launch(const Params& p, int out_kind, bool vec, uint64_t max_tile, cudaStream_t st, int device) {
+int launch(const Params& p, int out_kind, bool vec, uint64_t max_tile, cudaStream_t st, int device,
+           bool dependent) {
     const bool wide = max_tile <= Geo<kWarpsWide>::kBuf;
     switch (out_kind) {
-        case kOutBF16: return launch_out<kOutBF16>(p, vec, wide, st, device);
-        case kOutFP16: return launch_out<kOutFP16>(p, vec, wide, st, device);
-        case kOutE4M3: return launch_out<kOutE4M3>(p, vec, wide, st, device);
-        case kOutF32: return launch_out<kOutF32>(p, vec, wide, st, device);
+        case kOutBF16: return launch_out<kOutBF16>(p, vec, wide, st, device, dependent);
+        case kOutFP16: return launch_out<kOutFP16>(p, vec, wide, st, device, dependent);
+        case kOutE4M3: return launch_out<kOutE4M3>(p, vec, wide, st, device, dependent);
+        case kOutF32: return launch_out<kOutF32>(p, vec, wide, st, device, dependent);
         default:
-            return wide ? launch_one<kWarpsWide, kOutFields, false>(p, st, device)
-                        : launch_one<kWarpsNarrow, kOutFields, false>(p, st, device);
+            return wide ? launch_one<kWarpsWide, kOutFields, false>(p, st, device, false)
+                        : launch_one<kWarpsNarrow, kOutFields, false>(p, st, device, false);
     }
 }
 
@@ -686,6 +730,7 @@ Params make_params(const ep_blob* b, const uint8_t* dblob, const uint8_t* tables
         p.n[c] = L.n[c];
     }
     p.dense = vec && row_stride == L.cols;
+    p.tiny_alpha = L.tiny_alpha;
     return p;
 }
 
@@ -817,7 +862,7 @@ extern "C" int ep_decompress(const ep_blob* cb, const ep_tensor* out, void* stre
         const DeviceCopy& d = b->dev[dev];
         const bool vec = vec_ok(L, out->data, out->row_stride, out->dtype);
         Params p = make_params(b, d.blob, d.tables, out->data, out->row_stride, d.status, vec);
-        return launch(p, kind, vec, L.max_tile_bytes, st, dev);
+        return launch(p, kind, vec, L.max_tile_bytes, st, dev, true);
     }
 
     // Host output: upload the bytes, decode into a blob-owned buffer, copy back, synchronise.
@@ -851,7 +896,7 @@ extern "C" int ep_decompress(const ep_blob* cb, const ep_tensor* out, void* stre
             "ep_decompress: upload");
     const bool vec = vec_ok(L, d.stage_out, L.cols, out->dtype);
     Params p = make_params(b, d.stage_blob, d.tables, d.stage_out, L.cols, d.status, vec);
-    rc = launch(p, kind, vec, L.max_tile_bytes, st, dev);
+    rc = launch(p, kind, vec, L.max_tile_bytes, st, dev, false);
     if (rc != EP_OK) return rc;
     EP_CUDA(cudaMemcpy2DAsync(out->data, size_t(out->row_stride) * es, d.stage_out, size_t(L.cols) * es,
                               size_t(L.cols) * es, size_t(L.rows), cudaMemcpyDeviceToHost, st),
@@ -871,7 +916,7 @@ extern "C" int ep_decode_fields(const ep_blob* cb, int16_t* fields, void* stream
     if (rc != EP_OK) return rc;
     const DeviceCopy& d = b->dev[dev];
     Params p = make_params(b, d.blob, d.tables, fields, b->layout.cols, d.status, false);
-    return launch(p, kOutFields, false, b->layout.max_tile_bytes, st, dev);
+    return launch(p, kOutFields, false, b->layout.max_tile_bytes, st, dev, false);
 }
 
 extern "C" int ep_decode_status(const ep_blob* cb, void* stream) {

@@ -176,6 +176,17 @@ def test_degenerate_tables(ep):
     _check_full(ep, blob, z)
 
 
+def test_tiny_row_scales(ep):
+    """Rows around 2^-135 (FP32 subnormals) give row scales below 2^-125, where halving the
+    scale would round: the kernel must take its exact two-multiply path."""
+    g = np.random.Generator(np.random.PCG64(11))
+    x = g.normal(0, 1, (64, 256)) * 2.0 ** -135
+    x[::2] *= 2.0 ** 100                                           # half the rows ordinary
+    m = W.Matrix(np.ascontiguousarray(x, np.float32).view(np.uint32), W.F32, 4.0)
+    blob = oracle.compress(m.bits, m.dtype, m.target_bpp)
+    _check_full(ep, blob, m, [W.F32, W.BF16])
+
+
 # ---------------------------------------------------------------------------------------------
 # Library-encoded blobs at full workload sizes (the oracle decodes sampled tiles).
 # ---------------------------------------------------------------------------------------------
