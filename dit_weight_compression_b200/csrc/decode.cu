@@ -375,17 +375,24 @@ __device__ __forceinline__ void decode_step(const Params& p, uint32_t sym0, uint
     EP_FIELD(0) EP_FIELD(1) EP_FIELD(2) EP_FIELD(3) EP_FIELD(4) EP_FIELD(5) EP_FIELD(6) EP_FIELD(7)
 #undef EP_FIELD
 
-    // escaped fields: the lane's raw words after its renormalisation words, by field
-    int32_t f[8];
-#pragma unroll
-    for (int j = 0; j < 8; ++j) f[j] = int32_t(sym[j]) - kAlphabetR;
+    // t[j] = 2 z_j + c, the doubled lattice coordinate (z1..z7 = f1..f7, z8 = 2 f8 + parity of
+    // z1..z7), carried as the bits of the float 1.5 * 2^23 + t, which reads back exactly as
+    // 12582912 + t for |t| < 2^22.  Without escapes f_j = s_j - 127, so t comes straight from the
+    // symbols: 2 s_j - 254 + c, and for the last coordinate 4 s_8 - 508 + 2 par + c with
+    // par = (s_1 + ... + s_7 + 1) mod 2 (7 * 127 is odd).
+    constexpr int32_t kMagic = 0x4B400000;  // bits of 12582912.0f = 1.5 * 2^23
+    int32_t t[8];
+    bool fields_from_symbols = true;
+    int32_t f[8];  // only for the escape path and the fields output
     if (__any_sync(kFull, active && top == uint32_t(kEscape))) {
+        // escaped fields: the lane's raw words after its renormalisation words, by field
 #pragma unroll
         for (int j = 0; j < 8; ++j) {
             const bool mine = active && sym[j] == uint32_t(kEscape);
-            f[j] = mine ? int32_t(int16_t(rd.wn)) : f[j];
+            f[j] = mine ? int32_t(int16_t(rd.wn)) : int32_t(sym[j]) - kAlphabetR;
             rd.consume_if(mine);
         }
+        fields_from_symbols = false;
     }
     if (!active) return;
 
@@ -393,21 +400,30 @@ __device__ __forceinline__ void decode_step(const Params& p, uint32_t sym0, uint
         int16_t* o = static_cast<int16_t*>(p.out) + 9 * v;
         o[0] = int16_t(c);
 #pragma unroll
-        for (int j = 0; j < 8; ++j) o[1 + j] = int16_t(f[j]);
+        for (int j = 0; j < 8; ++j) o[1 + j] = int16_t(fields_from_symbols ? int32_t(sym[j]) - kAlphabetR : f[j]);
         return;
     } else {
-        // lattice point: z1..z7 = f1..f7, z8 = 2 f8 + (z1+..+z7 mod 2); 2y = 2z + c
-        const int32_t par = (f[0] + f[1] + f[2] + f[3] + f[4] + f[5] + f[6]) & 1;
-        f[7] = 2 * f[7] + par;
+        if (fields_from_symbols) {
+            const int32_t kc = kMagic - 2 * kAlphabetR + int32_t(c);
+            const int32_t par = int32_t(sym[0] + sym[1] + sym[2] + sym[3] + sym[4] + sym[5] + sym[6] + 1u) & 1;
+#pragma unroll
+            for (int j = 0; j < 7; ++j) t[j] = 2 * int32_t(sym[j]) + kc;
+            t[7] = 4 * int32_t(sym[7]) + 2 * par + (kc - 2 * kAlphabetR);
+        } else {
+            const int32_t par = (f[0] + f[1] + f[2] + f[3] + f[4] + f[5] + f[6]) & 1;
+            f[7] = 2 * f[7] + par;
+#pragma unroll
+            for (int j = 0; j < 8; ++j) t[j] = kMagic + 2 * f[j] + int32_t(c);
+        }
         float val[8];
         if (!p.tiny_alpha) {
             // a * y = (a/2) * (2z + c) exactly, so one product rounds once
 #pragma unroll
-            for (int i = 0; i < 8; ++i) val[i] = __fmul_rn(ah, __int2float_rn(2 * f[i] + int32_t(c)));
+            for (int i = 0; i < 8; ++i) val[i] = __fmul_rn(ah, __fsub_rn(__int_as_float(t[i]), 12582912.0f));
         } else {
 #pragma unroll
             for (int i = 0; i < 8; ++i) {
-                const float y = __fmul_rn(__int2float_rn(2 * f[i] + int32_t(c)), 0.5f);  // exact
+                const float y = __fmul_rn(__fsub_rn(__int_as_float(t[i]), 12582912.0f), 0.5f);  // exact
                 val[i] = __fmul_rn(a, y);  // the one rounding of the reconstruction
             }
         }
@@ -672,9 +688,8 @@ int launch(const Params& p, int out_kind, bool vec, uint64_t max_tile, cudaStrea
         case kOutFP16: return launch_out<kOutFP16>(p, vec, wide, st, device, dependent);
         case kOutE4M3: return launch_out<kOutE4M3>(p, vec, wide, st, device, dependent);
         case kOutF32: return launch_out<kOutF32>(p, vec, wide, st, device, dependent);
-        default:
-            return wide ? launch_one<kWarpsWide, kOutFields, false>(p, st, device, false)
-                        : launch_one<kWarpsNarrow, kOutFields, false>(p, st, device, false);
+        default:  // the fields test hook: the 16-warp kernel has the registers it needs
+            return launch_one<kWarpsNarrow, kOutFields, false>(p, st, device, false);
     }
 }
 
