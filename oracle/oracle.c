@@ -47,8 +47,9 @@ enum { ORC_BF16 = 1, ORC_FP16 = 2, ORC_E4M3 = 3, ORC_F32 = 4 };
 
 #define ORC_R 127          /* reading: field alphabet [-R, R] coded directly, R = 127     */
 #define ORC_ESC 255        /* symbol that announces a raw 16-bit field value               */
-#define ORC_M 4096u        /* frequency totals are 12-bit: every table sums to 4096       */
+#define ORC_M 1024u        /* reading: frequency totals are 10-bit, every table sums to M  */
 #define ORC_L 65536u       /* rANS lower bound 2^16, 32-bit state, 16-bit renormalisation */
+#define ORC_VERSION 2      /* blob format version (2: 10-bit frequency totals)            */
 #define ORC_LANES 32       /* interleaved rANS states per tile                            */
 #define ORC_NCTX 17        /* context 0: coset; 1 + 8c + (j-1): field j given coset c     */
 #define ORC_HEADER 80      /* bytes in the fixed header                                   */
@@ -332,13 +333,13 @@ void orc_fields_to_point(int coset, const int32_t f[8], double y[8])
 static int field_symbol(int32_t f) { return (f >= -ORC_R && f <= ORC_R) ? f + ORC_R : ORC_ESC; }
 
 /* ------------------------------------------------------------------------------------------ */
-/* Probability tables with 12-bit totals.                                                     */
+/* Probability tables with 10-bit totals (M = 1024).                                          */
 /* ------------------------------------------------------------------------------------------ */
 
 /*
- * Quantise symbol counts n[0..255] to frequencies q[] summing to 4096.
- * reading: q_s = max(1, round_half_up(4096 n_s / N)) for n_s > 0, else 0; then, while the sum
- * exceeds 4096, decrement the largest q (> 1; lowest symbol on ties); while it is below 4096,
+ * Quantise symbol counts n[0..255] to frequencies q[] summing to M.
+ * reading: q_s = max(1, round_half_up(M n_s / N)) for n_s > 0, else 0; then, while the sum
+ * exceeds M, decrement the largest q (> 1; lowest symbol on ties); while it is below M,
  * increment the symbol with the largest count (lowest symbol on ties).  N = 0 gives all zeros.
  */
 void orc_quantize_table(const uint64_t n[256], uint16_t q[256])
@@ -424,8 +425,9 @@ static int push_word(wordbuf* b, uint32_t v)
  * (17 x 256 frequencies).  Returns the tile size in bytes (written to out when out != NULL and
  * cap is large enough), or 0 on failure.
  *
- * rANS encode of symbol s with frequency q and cumulative cum [ANS]: while x >= q * 2^20,
- * emit the low 16 bits of x and shift them out; then x <- floor(x / q) * 4096 + (x mod q) + cum.
+ * rANS encode of symbol s with frequency q and cumulative cum [ANS]: while x >= q * (L / M) * 2^16
+ * (= q * 2^22), emit the low 16 bits of x and shift them out; then
+ * x <- floor(x / q) * M + (x mod q) + cum.
  * Each lane is encoded on its own, in reverse of its reading order, and its words are reversed
  * at the end.
  */
@@ -452,7 +454,7 @@ uint64_t orc_encode_tile(const uint8_t* sym9, const int16_t* raw8, int64_t nvec,
                 int ctx = context_of(u, sym9[v * 9]);
                 uint32_t q = q17[256 * ctx + s];
                 if (q == 0) goto fail;
-                if ((uint64_t)x[l] >= ((uint64_t)q << 20)) {
+                if ((uint64_t)x[l] >= (uint64_t)q * (ORC_L / ORC_M) * 65536u) {
                     if (push_word(&wb[l], x[l] & 0xFFFFu)) goto fail;
                     x[l] >>= 16;
                 }
@@ -509,8 +511,8 @@ static void build_dtables(const uint16_t* q17, dtables* T)
 
 /*
  * Decode one tile of nvec vectors with prepared tables.  Writes sym9 / raw8 as orc_encode_tile
- * reads them and the 32 final states.  rANS decode [ANS]: slot = x mod 4096, s = the symbol with
- * cum[s] <= slot < cum[s+1], x <- q_s * floor(x / 4096) + slot - cum[s]; if x < 2^16,
+ * reads them and the 32 final states.  rANS decode [ANS]: slot = x mod M, s = the symbol with
+ * cum[s] <= slot < cum[s+1], x <- q_s * floor(x / M) + slot - cum[s]; if x < 2^16,
  * x <- x * 2^16 + the lane's next word.  Returns 0 when the tile is consistent (every state back
  * at 2^16, the two lanes of every region meeting exactly, only padding after the last region),
  * 1 when it is not, -1 when a lane's words ran outside the tile.
@@ -543,7 +545,7 @@ static int decode_tile(const uint8_t* tile, uint64_t nbytes, int64_t nvec, const
                 uint32_t slot = x & (ORC_M - 1);
                 int s = T->slot_sym[ctx][slot];
                 uint32_t q = T->q17[256 * ctx + s];
-                x = q * (x >> 12) + slot - T->cum[ctx][s];
+                x = q * (x / ORC_M) + slot - T->cum[ctx][s];
                 sym9[v * 9 + u] = (uint8_t)s;
                 if (x < ORC_L) {
                     int64_t w = fwd ? start[p] + n : start[p] + count[p] - 1 - n;
@@ -667,7 +669,7 @@ static uint64_t table_section_bytes(const uint16_t* q17)
  * Estimated blob size in bits per element at scale s from the sampled rows ([DOC-RS]: "For each
  * candidate scale, it estimates the coded field size and the metadata needed for decoding").
  * reading: n_s = min(rows, 256) rows at floor(i * rows / n_s); tables are quantised from the
- * sample's counts; coded size = sum over contexts and symbols of n * -log2(q / 4096) bits plus
+ * sample's counts; coded size = sum over contexts and symbols of n * -log2(q / M) bits plus
  * 16 bits per escape, scaled by rows / n_s; metadata = exact header, table, row-scale and
  * tile-offset bytes, plus 160 header bytes (states, region counts) and 8 padding bytes per tile.
  * With full_sample != 0 every row is used (n_s = rows).
@@ -697,7 +699,7 @@ static double estimate_bpp(const matrix* m, double s, int64_t S, int full_sample
     double bits = 0.0;
     for (int ctx = 0; ctx < ORC_NCTX; ctx++)
         for (int sy = 0; sy < 256; sy++)
-            if (cnt[256 * ctx + sy]) bits += (double)cnt[256 * ctx + sy] * -log2((double)q17[256 * ctx + sy] / 4096.0);
+            if (cnt[256 * ctx + sy]) bits += (double)cnt[256 * ctx + sy] * -log2((double)q17[256 * ctx + sy] / (double)ORC_M);
     double payload = ((double)m->rows / (double)ns) * (bits / 8.0 + 2.0 * (double)nesc);
     int64_t V = m->rows * m->vpr;
     int64_t ntiles = (V + 32 * S - 1) / (32 * S);
@@ -771,7 +773,7 @@ double orc_estimate_bpp(const void* data, int dtype, int64_t rows, int64_t cols,
  *
  * Blob layout (little-endian, every section 16-byte aligned; [DOC-ER]: "the representation also
  * stores the probability tables, row scales, and tile metadata"):
- *   header (80 bytes): "EPK1", u16 version 1, u8 dtype, u8 R, u64 rows, u64 cols, u32 S,
+ *   header (80 bytes): "EPK1", u16 version 2, u8 dtype, u8 R, u64 rows, u64 cols, u32 S,
  *     u32 n_tiles, f64 s, u64 total bytes, u64 offsets of the table, row-scale, tile-offset
  *     and stream sections;
  *   tables: u16 q(coset 0), u16 q(coset 1); then for c = 0,1 and j = 1..8: u16 q(escape),
@@ -850,7 +852,7 @@ int orc_compress(const void* data, int dtype, int64_t rows, int64_t cols, double
         uint8_t* b = (uint8_t*)calloc((size_t)total, 1);
         if (!b) { rc = -2; goto done; }
         memcpy(b, "EPK1", 4);
-        put16(b + 4, 1);
+        put16(b + 4, ORC_VERSION);
         b[6] = (uint8_t)dtype;
         b[7] = ORC_R;
         put64(b + 8, (uint64_t)rows);
@@ -926,7 +928,7 @@ typedef struct {
 
 static int parse_blob(const uint8_t* b, uint64_t len, parsed* P)
 {
-    if (len < ORC_HEADER || memcmp(b, "EPK1", 4) != 0 || get16(b + 4) != 1 || b[7] != ORC_R) return -6;
+    if (len < ORC_HEADER || memcmp(b, "EPK1", 4) != 0 || get16(b + 4) != ORC_VERSION || b[7] != ORC_R) return -6;
     P->dtype = b[6];
     P->rows = (int64_t)get64(b + 8);
     P->cols = (int64_t)get64(b + 16);

@@ -142,8 +142,10 @@ def test_fields_enumerated_box():
 
 
 # ---------------------------------------------------------------------------------------------
-# 12-bit frequency tables.
+# 10-bit frequency tables (every table sums to M = 1024).
 # ---------------------------------------------------------------------------------------------
+
+M = 1024
 
 def _q(counts):
     a = np.zeros(256, np.uint64)
@@ -153,17 +155,17 @@ def _q(counts):
 
 
 def test_table_hand_cases():
-    q = _q({0: 1, 1: 1}); assert (q[0], q[1]) == (2048, 2048)
-    q = _q({5: 3, 9: 1}); assert (q[5], q[9]) == (3072, 1024)
-    q = _q({200: 17}); assert q[200] == 4096 and q.sum() == 4096
-    # 4096/3 = 1365.33 -> 1365 each, sum 4095 -> +1 to the largest count, lowest symbol first
-    q = _q({1: 1, 2: 1, 3: 1}); assert (q[1], q[2], q[3]) == (1366, 1365, 1365)
+    q = _q({0: 1, 1: 1}); assert (q[0], q[1]) == (512, 512)
+    q = _q({5: 3, 9: 1}); assert (q[5], q[9]) == (768, 256)
+    q = _q({200: 17}); assert q[200] == 1024 and q.sum() == 1024
+    # 1024/3 = 341.33 -> 341 each, sum 1023 -> +1 to the largest count, lowest symbol first
+    q = _q({1: 1, 2: 1, 3: 1}); assert (q[1], q[2], q[3]) == (342, 341, 341)
     # a rare symbol keeps frequency 1; the big one gives back the excess
-    q = _q({0: 1_000_000, 255: 1}); assert (q[0], q[255]) == (4095, 1)
+    q = _q({0: 1_000_000, 255: 1}); assert (q[0], q[255]) == (1023, 1)
     counts = {s: 1 for s in range(200)}
     counts[250] = 1_000_000
     q = _q(counts)
-    assert all(q[s] == 1 for s in range(200)) and q[250] == 4096 - 200
+    assert all(q[s] == 1 for s in range(200)) and q[250] == 1024 - 200
     assert _q({}).sum() == 0
 
 
@@ -174,17 +176,22 @@ def test_table_invariants():
         sel = RNG.choice(256, k, replace=False)
         n[sel] = RNG.integers(1, 10 ** RNG.integers(1, 7), k)
         q = oracle.quantize_table(n)
-        assert int(q.sum()) == 4096
+        assert int(q.sum()) == M
         assert np.array_equal(q > 0, n > 0)
-        ideal = 4096.0 * n / n.sum()
-        assert np.all(np.abs(q - ideal) <= np.maximum(2.0, 0.02 * ideal) + k / 4)
+        ideal = M * n / n.sum()
+        # Rounding moves each symbol at most 1/2 from its share (less than 1 for the r symbols
+        # raised to 1), so the excess or deficit the repair loop removes is at most k/2 + r/2,
+        # and it can all land on one symbol.
+        r = int(((ideal < 0.5) & (n > 0)).sum())
+        assert np.all(np.abs(q - ideal) <= 1.0 + k / 2 + r / 2)
+        assert np.abs(q - ideal).sum() <= 2.0 * (k / 2 + r / 2) + 1e-9
 
 
 # ---------------------------------------------------------------------------------------------
 # rANS tiles.
 # ---------------------------------------------------------------------------------------------
 
-def _tables(field_q: dict, coset_q=(4096, 0)):
+def _tables(field_q: dict, coset_q=(M, 0)):
     """17 x 256 tables: context 0 the coset, contexts 1..16 all equal to field_q."""
     q17 = np.zeros((17, 256), np.uint16)
     q17[0, 0], q17[0, 1] = coset_q
@@ -195,17 +202,18 @@ def _tables(field_q: dict, coset_q=(4096, 0)):
 
 
 def test_rans_closed_form_one_bit_symbols():
-    """Two steps, 32 lanes, every field one bit (q = 2048 for f = 0 and f = 1), coset free
-    (q = 4096).  Encoding x <- floor(x/2048)*4096 + (x mod 2048) + 2048*b from x = 2^16 gives,
-    after n bits b_1..b_n (first encoded first), x = 2^(16+n) + 2048 * sum_i b_i 2^(n-i) while
-    x < 2^31.  A lane meets its 16 bits in reverse reading order: step 1 f8..f1, then step 0
-    f8..f1; before the 16th (step 0, f1) x = 2^31 + 2048*B15 >= 2^31, so it emits the low 16 bits
-    2048*(B15 mod 32) and keeps 2^15 + (B15 >> 5); encoding f1 then gives the initial state
-    2^16 + 2048*f1 + (B15 >> 5).  B15 mod 32 = 16 f6 + 8 f5 + 4 f4 + 2 f3 + f2 (step 0), and
-    B15 >> 5 = 4*(128 f8 + 64 f7 + ... + f1 of step 1) + 2 f8 + f7 (step 0).  Every lane has
-    exactly one word, so each region holds 2 words: lane 2p's (read forward from the region
-    start) then lane 2p+1's (read backward from the region end) -- lane order overall."""
-    q17 = _tables({127: 2048, 128: 2048})
+    """Two steps, 32 lanes, every field one bit (q = 512 for f = 0 and f = 1), coset free
+    (q = 1024).  Encoding x <- floor(x/512)*1024 + (x mod 512) + 512*b from x = 2^16 gives,
+    after n bits b_1..b_n (first encoded first), x = 2^(16+n) + 512 * sum_i b_i 2^(n-i) while
+    x < 2^31 (the renormalisation bound q * (L/M) * 2^16 = 2^31).  A lane meets its 16 bits in
+    reverse reading order: step 1 f8..f1, then step 0 f8..f1; before the 16th (step 0, f1)
+    x = 2^31 + 512*B15 >= 2^31, so it emits the low 16 bits 512*(B15 mod 128) and keeps
+    2^15 + (B15 >> 7); encoding f1 then gives the initial state 2^16 + 512*f1 + (B15 >> 7).
+    B15 mod 128 = 64 f8 + 32 f7 + ... + 2 f3 + f2 (step 0), and B15 >> 7 = 128 f8 + 64 f7 + ...
+    + f1 of step 1.  Every lane has exactly one word, so each region holds 2 words: lane 2p's
+    (read forward from the region start) then lane 2p+1's (read backward from the region end)
+    -- lane order overall."""
+    q17 = _tables({127: 512, 128: 512})
     bits = RNG.integers(0, 2, (64, 8))                              # vector v = 32k + lane
     sym9 = np.zeros((64, 9), np.uint8)
     sym9[:, 1:] = 127 + bits
@@ -220,19 +228,18 @@ def test_rans_closed_form_one_bit_symbols():
         f0 = bits[lane]            # step 0: f1..f8 at indices 0..7
         f1 = bits[32 + lane]       # step 1
         step1 = sum(int(f1[j]) << j for j in range(8))             # 128 f8 + ... + f1
-        hi = 4 * step1 + 2 * int(f0[7]) + int(f0[6])
-        assert states[lane] == 65536 + 2048 * int(f0[0]) + hi
-        low5 = 16 * f0[5] + 8 * f0[4] + 4 * f0[3] + 2 * f0[2] + f0[1]
-        assert words[lane] == 2048 * low5
+        assert states[lane] == 65536 + 512 * int(f0[0]) + step1
+        low7 = sum(int(f0[j]) << (j - 1) for j in range(1, 8))       # 64 f8 + ... + f2
+        assert words[lane] == 512 * low7
     rc, s9, r8, st = oracle.decode_tile(tile, 64, q17)
     assert rc == 0 and np.array_equal(s9, sym9) and np.all(st == 65536)
 
 
 def test_rans_all_escape_closed_form():
-    """Coset free, every field the escape symbol with q = 4096: no state ever changes, so each
+    """Coset free, every field the escape symbol with q = M: no state ever changes, so each
     lane's words are its raw values in step, field order; region p holds lane 2p's words forward
     and lane 2p+1's words backward from the region end."""
-    q17 = _tables({255: 4096})
+    q17 = _tables({255: M})
     nvec = 70                                                       # 3 steps, the last partial
     sym9 = np.zeros((nvec, 9), np.uint8)
     sym9[:, 1:] = 255
@@ -260,9 +267,9 @@ def test_rans_all_escape_closed_form():
 
 
 def test_rans_lone_symbols_closed_form():
-    """Every context holds one symbol with q = 4096: coding it costs nothing, so the tile is
+    """Every context holds one symbol with q = M: coding it costs nothing, so the tile is
     exactly the 32 states, all 2^16, and 16 zero region counts."""
-    q17 = _tables({127: 4096})
+    q17 = _tables({127: M})
     for nvec in (1, 31, 32, 33, 1000):
         sym9 = np.full((nvec, 9), 127, np.uint8)
         sym9[:, 0] = 0
@@ -287,12 +294,12 @@ def _random_tables(nsym_max=40):
 
 def _draw(q17, nvec):
     sym9 = np.zeros((nvec, 9), np.uint8)
-    p0 = q17[0, :2] / 4096.0
+    p0 = q17[0, :2] / M
     sym9[:, 0] = RNG.choice(2, nvec, p=p0)
     for u in range(1, 9):
         for c in (0, 1):
             m = sym9[:, 0] == c
-            p = q17[1 + 8 * c + u - 1] / 4096.0
+            p = q17[1 + 8 * c + u - 1] / M
             sym9[m, u] = RNG.choice(256, int(m.sum()), p=p)
     raw8 = RNG.integers(-32768, 32768, (nvec, 8)).astype(np.int16)
     return sym9, raw8
@@ -330,7 +337,7 @@ def test_rans_corruption_detected():
 
 def test_rans_size_near_cross_entropy():
     """Coded words carry the symbols' information: 16 * words + the information held by the
-    final states (at most 16 bits per lane above 2^16) is the sum of -log2(q/4096)."""
+    final states (at most 16 bits per lane above 2^16) is the sum of -log2(q/M)."""
     q17 = _random_tables(30)
     nvec = 32 * 256
     sym9, raw8 = _draw(q17, nvec)
@@ -338,7 +345,7 @@ def test_rans_size_near_cross_entropy():
     ctx = np.zeros((nvec, 9), np.int64)
     ctx[:, 1:] = 1 + 8 * sym9[:, :1] + np.arange(8)[None, :]
     q = q17[ctx, sym9].astype(np.float64)
-    info = -np.log2(q / 4096.0).sum() + 16.0 * (sym9[:, 1:] == 255).sum()
+    info = -np.log2(q / M).sum() + 16.0 * (sym9[:, 1:] == 255).sum()
     states = np.frombuffer(tile[:128], "<u4").astype(np.float64)
     held = np.log2(states / 65536.0).sum()                          # bits parked in the states
     words_bits = 16.0 * int(np.frombuffer(tile[128:160], "<u2").astype(np.int64).sum())
