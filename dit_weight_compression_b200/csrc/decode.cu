@@ -9,18 +9,19 @@
 //   * one warp per tile; the tile's 32 interleaved rANS states live one per lane;
 //   * one persistent CTA of 32 warps per SM (grid = min(#SM, #tiles)); tile t goes to CTA
 //     t mod grid, so every SM gets an equal share even when there are few tiles;
-//   * decode tables: per field context a 4096-entry slot->symbol byte table and a 256-entry
-//     frequency / cumulative-frequency table pair of u16, 80 KB in all.  They are expanded once per
-//     blob and device by a small kernel into a block next to the device copy; every CTA stages
-//     that block into shared memory with bulk copies, overlapped with the fetch of its first
-//     tiles.  (The allocation-free entry point expands them inside each CTA instead.)  The coset
-//     context, two symbols, is decoded by one compare;
+//   * decode table: per field context one packed 32-bit entry per slot of the 1024-slot range,
+//     {slot - cum(s), 2 s, escape flag, q(s)}, 64 KB in all, so one shared-memory load per symbol
+//     gives everything the state update needs.  It is expanded once per blob and device by a
+//     small kernel into a block next to the device copy; every CTA stages that block into shared
+//     memory with bulk copies, overlapped with the fetch of its first tiles.  (The
+//     allocation-free entry point expands it inside each CTA instead.)  The coset context, two
+//     symbols, is decoded by one compare;
 //   * words: every lane reads its own word stream.  Lanes 2p and 2p+1 share region p of the tile
 //     (one forward from the region start, one backward from its end); a warp-shuffle prefix sum
-//     over the 16 region counts gives every lane its start.  The tile is prefetched into L2 by
-//     a bulk prefetch; each lane keeps two 8-byte chunks of its stream in registers, loads the
-//     next chunk four words ahead, and has its next word ready before it needs it, so a
-//     renormalisation costs one compare and one byte permute on the dependent chain;
+//     over the 16 region counts gives every lane its start.  The whole tile is staged into a
+//     per-warp shared-memory buffer by one bulk copy (the next tile is prefetched into L2); each
+//     lane has its next word loaded before it needs it, so a renormalisation costs one compare
+//     and one byte permute on the dependent chain;
 //   * per step a lane decodes one 8-vector: 9 rANS symbols (each followed by its conditional
 //     refill), then the raw words of its escaped fields; fields are inverted in registers
 //     (z8 = 2 f8 + parity, y = z + c/2), multiplied by the row's fp32 scale, converted one pair
@@ -52,8 +53,24 @@ namespace {
 
 constexpr uint32_t kFull = 0xFFFFFFFFu;
 constexpr uint32_t kWaitSpins = 1u << 22;                     // bounded mbarrier wait (~0.3 s)
-constexpr uint32_t kTableBytes = kFieldContexts * (kProbTotal + 256 * 4);  // 81920
+constexpr uint32_t kSlotMask = kProbTotal - 1;
+constexpr uint32_t kCtxBytes = 4 * kProbTotal;                // one context's packed table: 4 KB
+constexpr uint32_t kTableBytes = kFieldContexts * kCtxBytes;  // 65536
 constexpr uint32_t kTablePiece = 16384;                       // bytes per table bulk copy
+
+// Packed decode-table entry of slot u in context (c, j), symbol s = the one with
+// cum(s) <= u < cum(s) + q(s):
+//   bits  0..9   u - cum(s)           (< q(s) <= 1024)
+//   bits 10..18  2 s                  (bit 10 is zero)
+//   bit  19      s is the escape symbol
+//   bits 21..31  q(s)                 (<= 1024)
+// so the state update x <- q (x >> 10) + u - cum(s) takes two field extractions, and the
+// reconstruction takes 2 s out with one shift and mask.
+constexpr uint32_t kEntryBiasMask = 0x3FFu;
+constexpr uint32_t kEntrySymShift = 10;
+constexpr uint32_t kEntryEsc = 1u << 19;
+constexpr uint32_t kEntryQShift = 21;
+static_assert(kProbBits == 10, "the packed entry holds 10-bit slots");
 
 enum OutKind { kOutBF16 = 0, kOutFP16 = 1, kOutE4M3 = 2, kOutF32 = 3, kOutFields = 4 };
 
@@ -67,27 +84,27 @@ enum : uint32_t {
 
 struct Params {
     const uint8_t* blob;        // device copy of the serialised blob
-    const uint8_t* tables;      // expanded decode tables (kTableBytes), or null: expand in-kernel
+    const uint8_t* tables;      // expanded decode table (kTableBytes), or null: expand in-kernel
     const uint32_t* tile_off;   // n_tiles + 1 offsets, 16-byte units
     const uint8_t* stream;      // stream section
     const float* alpha;         // per-row fp32 scales
     void* out;
     uint32_t* status;
-    int64_t cols, row_stride, n_vectors, vec_per_row;
+    int64_t rows, cols, row_stride, n_vectors;
+    uint32_t vec_per_row;       // < 2^31 (checked when the blob is parsed)
     uint32_t steps, n_tiles;
-    uint32_t q_coset0;          // frequency of coset 0; coset 1 has 4096 - q_coset0
+    uint32_t q_coset0;          // frequency of coset 0; coset 1 has M - q_coset0
     uint32_t q_off[kFieldContexts];
     uint32_t esc_q[kFieldContexts];
     uint32_t lo[kFieldContexts];
     uint32_t n[kFieldContexts];
-    int dense;                  // element offset of vector v is 8 v
     int tiny_alpha;             // some |alpha| < 2^-125, where alpha / 2 would round
 };
 
 constexpr uint32_t kSmemOptin = 232448;  // 227 KB: the largest dynamic shared memory of one CTA
 constexpr uint32_t kBufSlack = 48;        // bytes after a tile buffer that a step may over-read
 
-// Per-warp tile buffer size for a CTA of WARPS warps: what the 227 KB leave after the tables.
+// Per-warp tile buffer size for a CTA of WARPS warps: what the 227 KB leave after the table.
 template <int WARPS>
 struct Geo {
     static constexpr uint32_t kBuf =
@@ -96,14 +113,20 @@ struct Geo {
 
 template <int WARPS>
 struct Smem {
-    uint8_t sym[kFieldContexts][kProbTotal];                    // slot -> symbol    } 80 KB table
-    uint16_t fc[kFieldContexts][2][256];                        // [0] freq, [1] cum } block
+    uint32_t tab[kFieldContexts][kProbTotal];                       // packed decode table, 64 KB
     alignas(16) uint8_t tbuf[WARPS][Geo<WARPS>::kBuf + kBufSlack];  // one staged tile per warp
-    unsigned long long bar[WARPS];                              // tile staging, one per warp
-    unsigned long long tbar;                                    // the table block's bulk copies
+    unsigned long long bar[WARPS];                                  // tile staging, one per warp
+    unsigned long long tbar;                                        // the table's bulk copies
 };
 static_assert(offsetof(Smem<32>, tbuf) == kTableBytes, "table block must be contiguous");
 static_assert(sizeof(Smem<32>) <= kSmemOptin && sizeof(Smem<16>) <= kSmemOptin, "shared memory budget");
+
+// Scratch of the table expansion: frequencies and cumulative frequencies of every context.
+struct BuildScratch {
+    uint16_t q[kFieldContexts][256];
+    uint16_t cum[kFieldContexts][257];
+};
+static_assert(sizeof(BuildScratch) <= 16 * Geo<32>::kBuf, "expansion scratch fits the tile buffers");
 
 // ---- PTX wrappers ----------------------------------------------------------------------------
 __device__ __forceinline__ uint32_t smem_u32(const void* p) {
@@ -147,12 +170,6 @@ __device__ __forceinline__ bool mbar_wait(unsigned long long* bar, uint32_t pari
 }
 
 // Shared-memory loads at 32-bit shared-window addresses (plus a constant byte offset).
-template <int OFF = 0>
-__device__ __forceinline__ uint32_t lds_u8(uint32_t a) {
-    uint32_t v;
-    asm volatile("ld.shared.u8 %0, [%1+%2];" : "=r"(v) : "r"(a), "n"(OFF));
-    return v;
-}
 template <int OFF = 0>
 __device__ __forceinline__ uint32_t lds_u16(uint32_t a) {
     uint32_t v;
@@ -228,8 +245,10 @@ __device__ __forceinline__ void renorm_step(uint32_t& x, Reader& rd, bool active
 }
 
 // ---- table expansion -------------------------------------------------------------------------
+// Fills tab[16][1024] from the blob's compact frequency tables.  `scr` is shared-memory scratch
+// (BuildScratch) that the caller does not use meanwhile.
 template <int WARPS>
-__device__ void build_tables(Smem<WARPS>& sm, const Params& p) {
+__device__ void build_tables(uint32_t (*tab)[kProbTotal], BuildScratch& scr, const Params& p) {
     const uint32_t lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
     // (a) per context: frequencies of symbols 8*lane .. 8*lane+7 and their cumulative sums
     for (uint32_t ctx = warp; ctx < kFieldContexts; ctx += WARPS) {
@@ -253,51 +272,54 @@ __device__ void build_tables(Smem<WARPS>& sm, const Params& p) {
         uint32_t c = inc - sum;
 #pragma unroll
         for (int i = 0; i < 8; ++i) {
-            sm.fc[ctx][0][8 * lane + i] = uint16_t(q[i]);
-            sm.fc[ctx][1][8 * lane + i] = uint16_t(c);  // < 4096 for every used symbol
+            scr.q[ctx][8 * lane + i] = uint16_t(q[i]);
+            scr.cum[ctx][8 * lane + i] = uint16_t(c);  // <= M for a valid table
             c += q[i];
         }
+        if (lane == 31) scr.cum[ctx][256] = uint16_t(min(c, 0xFFFFu));
     }
     __syncthreads();
-    // (b) slot -> symbol, 4 slots per 32-bit store.  Lane l of a warp writes words it*32 + l
-    // (it = 0, 1, ...), so the 32 stores of one instruction hit 32 different banks; each lane
-    // walks its symbol forward as its slots grow.  A context is split into P parts over warps.
+    // (b) slot -> packed entry.  Lane l of a warp writes slots it*32 + l of its part (one
+    // 128-byte run per store instruction); each lane walks its symbol forward as its slots grow.
     constexpr int P = WARPS >= 16 ? WARPS / 16 : 1;
-    constexpr uint32_t kWordsPerPart = kProbTotal / 4 / P;
+    constexpr uint32_t kSlotsPerPart = kProbTotal / P;
     for (uint32_t item = warp; item < uint32_t(kFieldContexts * P); item += WARPS) {
         const uint32_t ctx = item / P, part = item % P;
-        const uint16_t* cum = sm.fc[ctx][1];
-        uint32_t* dst = reinterpret_cast<uint32_t*>(&sm.sym[ctx][0]) + part * kWordsPerPart;
-        const uint32_t total = uint32_t(cum[255]) + sm.fc[ctx][0][255];
-        if (total == 0) {  // context never used by this blob
-            for (uint32_t w = lane; w < kWordsPerPart; w += 32) dst[w] = 0;
+        const uint16_t* cum = scr.cum[ctx];
+        const uint16_t* qs = scr.q[ctx];
+        uint32_t* dst = tab[ctx] + part * kSlotsPerPart;
+        if (cum[256] != kProbTotal) {  // context never used by this blob (the host checked the rest)
+            for (uint32_t w = lane; w < kSlotsPerPart; w += 32) dst[w] = 0;
             continue;
         }
-        const uint32_t first = 4 * (part * kWordsPerPart + lane);
+        const uint32_t first = part * kSlotsPerPart + lane;
         uint32_t s = 0;  // largest symbol with cum(s) <= first
 #pragma unroll
         for (uint32_t step = 128; step; step >>= 1)
             if (cum[s + step] <= first) s += step;
-        uint32_t next = s < 255 ? cum[s + 1] : kProbTotal;
-        for (uint32_t w = lane; w < kWordsPerPart; w += 32) {
-            const uint32_t base = 4 * (part * kWordsPerPart + w);
-            uint32_t word = 0;
-#pragma unroll
-            for (uint32_t k = 0; k < 4; ++k) {
-                while (next <= base + k) {
-                    ++s;
-                    next = s < 255 ? cum[s + 1] : kProbTotal;
-                }
-                word |= s << (8 * k);
+        uint32_t c0 = cum[s], next = cum[s + 1];
+        for (uint32_t w = lane; w < kSlotsPerPart; w += 32) {
+            const uint32_t slot = part * kSlotsPerPart + w;
+            while (next <= slot) {
+                ++s;
+                c0 = next;
+                next = cum[s + 1];
             }
-            dst[w] = word;
+            dst[w] = (slot - c0) | (s << (kEntrySymShift + 1)) | (s == uint32_t(kEscape) ? kEntryEsc : 0u) |
+                     (uint32_t(qs[s]) << kEntryQShift);
         }
     }
 }
 
 // ---- output conversion -----------------------------------------------------------------------
 template <int OUT>
-__device__ __forceinline__ void store_vec(void* out, int64_t elem, const float v[8]) {
+struct OutElem {
+    static constexpr int kBytes = OUT == kOutE4M3 ? 1 : (OUT == kOutF32 ? 4 : 2);
+};
+
+// Eight values to eight consecutive elements at `dst` (aligned to the vector's size).
+template <int OUT>
+__device__ __forceinline__ void store_vec(uint8_t* dst, const float v[8]) {
     if constexpr (OUT == kOutBF16) {
         uint4 u;
         __nv_bfloat162 h0 = __floats2bfloat162_rn(v[0], v[1]), h1 = __floats2bfloat162_rn(v[2], v[3]);
@@ -306,7 +328,7 @@ __device__ __forceinline__ void store_vec(void* out, int64_t elem, const float v
         u.y = *reinterpret_cast<uint32_t*>(&h1);
         u.z = *reinterpret_cast<uint32_t*>(&h2);
         u.w = *reinterpret_cast<uint32_t*>(&h3);
-        __stcs(reinterpret_cast<uint4*>(static_cast<__nv_bfloat16*>(out) + elem), u);
+        __stcs(reinterpret_cast<uint4*>(dst), u);
     } else if constexpr (OUT == kOutFP16) {
         uint4 u;
         __half2 h0 = __floats2half2_rn(v[0], v[1]), h1 = __floats2half2_rn(v[2], v[3]);
@@ -315,153 +337,193 @@ __device__ __forceinline__ void store_vec(void* out, int64_t elem, const float v
         u.y = *reinterpret_cast<uint32_t*>(&h1);
         u.z = *reinterpret_cast<uint32_t*>(&h2);
         u.w = *reinterpret_cast<uint32_t*>(&h3);
-        __stcs(reinterpret_cast<uint4*>(static_cast<__half*>(out) + elem), u);
+        __stcs(reinterpret_cast<uint4*>(dst), u);
     } else if constexpr (OUT == kOutE4M3) {
         uint32_t w[4];
 #pragma unroll
         for (int i = 0; i < 4; ++i)
             w[i] = __nv_cvt_float2_to_fp8x2(make_float2(v[2 * i], v[2 * i + 1]), __NV_SATFINITE, __NV_E4M3);
-        uint2 u = make_uint2(w[0] | (w[1] << 16), w[2] | (w[3] << 16));
-        __stcs(reinterpret_cast<uint2*>(static_cast<uint8_t*>(out) + elem), u);
+        __stcs(reinterpret_cast<uint2*>(dst), make_uint2(w[0] | (w[1] << 16), w[2] | (w[3] << 16)));
     } else {
-        float4* o = reinterpret_cast<float4*>(static_cast<float*>(out) + elem);
+        float4* o = reinterpret_cast<float4*>(dst);
         __stcs(o, make_float4(v[0], v[1], v[2], v[3]));
         __stcs(o + 1, make_float4(v[4], v[5], v[6], v[7]));
     }
 }
 
 template <int OUT>
-__device__ __forceinline__ void store_one(void* out, int64_t elem, float v) {
-    if constexpr (OUT == kOutBF16) static_cast<__nv_bfloat16*>(out)[elem] = __float2bfloat16_rn(v);
-    else if constexpr (OUT == kOutFP16) static_cast<__half*>(out)[elem] = __float2half_rn(v);
-    else if constexpr (OUT == kOutE4M3)
-        static_cast<uint8_t*>(out)[elem] = uint8_t(__nv_cvt_float_to_fp8(v, __NV_SATFINITE, __NV_E4M3));
-    else static_cast<float*>(out)[elem] = v;
+__device__ __forceinline__ void store_one(uint8_t* dst, float v) {
+    if constexpr (OUT == kOutBF16) *reinterpret_cast<__nv_bfloat16*>(dst) = __float2bfloat16_rn(v);
+    else if constexpr (OUT == kOutFP16) *reinterpret_cast<__half*>(dst) = __float2half_rn(v);
+    else if constexpr (OUT == kOutE4M3) *dst = uint8_t(__nv_cvt_float_to_fp8(v, __NV_SATFINITE, __NV_E4M3));
+    else *reinterpret_cast<float*>(dst) = v;
 }
 
 // ---- one step: every lane decodes (at most) one 8-vector --------------------------------------
-template <int OUT, bool VEC, bool FULL, class Reader>
-__device__ __forceinline__ void decode_step(const Params& p, uint32_t sym0, uint32_t fc0, Reader& rd,
-                                            uint32_t& x, bool active, int64_t v, int64_t row, int64_t kcol) {
-    if (FULL) active = true;
-    // issued early, used after the symbol chain; lanes past the last vector read nothing
-    const float a = active ? __ldg(p.alpha + row) : 0.0f;
-    const float ah = __fmul_rn(a, 0.5f);  // exact unless |a| < 2^-125 (p.tiny_alpha)
+// Where a lane's current vector goes: vector kcol of row `row`, whose first element is at optr.
+struct Pos {
+    uint8_t* optr;
+    int64_t row;
+    uint32_t kcol;
+    float a, ah;  // the row's scale, and scale / 2
+};
 
+template <int OUT>
+__device__ __forceinline__ Pos first_pos(const Params& p, int64_t v) {
+    Pos s;
+    if constexpr (OUT == kOutFields) {
+        s.optr = static_cast<uint8_t*>(p.out) + 18 * v;  // 9 int16 per vector
+        s.row = 0;
+        s.kcol = 0;
+        s.a = s.ah = 0.0f;
+    } else {
+        s.row = v / p.vec_per_row;
+        s.kcol = uint32_t(v - s.row * p.vec_per_row);
+        s.optr = static_cast<uint8_t*>(p.out) + (s.row * p.row_stride + 8 * int64_t(s.kcol)) * OutElem<OUT>::kBytes;
+        s.a = v < p.n_vectors ? __ldg(p.alpha + s.row) : 0.0f;
+        s.ah = __fmul_rn(s.a, 0.5f);
+    }
+    return s;
+}
+
+// The lane's next vector is 32 further on; the row scale is reloaded only when the row changes.
+template <int OUT>
+__device__ __forceinline__ void advance(const Params& p, Pos& s) {
+    if constexpr (OUT == kOutFields) {
+        s.optr += 32 * 18;
+    } else {
+        constexpr int es = OutElem<OUT>::kBytes;
+        s.kcol += 32;
+        s.optr += 32 * 8 * es;
+        if (s.kcol >= p.vec_per_row) {
+            const int64_t wrap = (p.row_stride - 8 * int64_t(p.vec_per_row)) * es;
+            do {
+                s.kcol -= p.vec_per_row;
+                ++s.row;
+                s.optr += wrap;
+            } while (s.kcol >= p.vec_per_row);
+            s.a = s.row < p.rows ? __ldg(p.alpha + s.row) : 0.0f;
+            s.ah = __fmul_rn(s.a, 0.5f);
+        }
+    }
+}
+
+template <int OUT, bool VEC, bool FULL, class Reader>
+__device__ __forceinline__ void decode_step(const Params& p, uint32_t tab, Reader& rd, uint32_t& x, bool active,
+                                            const Pos& pos) {
+    if (FULL) active = true;
     // coset (two symbols: slot < q0 -> 0)
     const uint32_t q0 = p.q_coset0;
-    uint32_t slot = x & (kProbTotal - 1);
-    const uint32_t c = slot >= q0 ? 1u : 0u;
-    if (active) x = (c ? kProbTotal - q0 : q0) * (x >> kProbBits) + (slot - (c ? q0 : 0u));
+    const uint32_t cslot = x & kSlotMask;
+    const bool c1 = cslot >= q0;
+    if (active) x = (c1 ? kProbTotal - q0 : q0) * (x >> kProbBits) + (cslot - (c1 ? q0 : 0u));
     renorm_step<FULL>(x, rd, active);
 
-    // fields f1..f8 with context (c, j): tables of coset c start 8 contexts further on
-    const uint32_t st = sym0 + c * (8u * kProbTotal);
-    const uint32_t ft = fc0 + c * (8u * 1024u);
-    uint32_t sym[8];
-    uint32_t top = 0;
+    // fields f1..f8 with context (c, j): the 8 tables of coset 1 follow those of coset 0.  A lane
+    // past the last vector still loads (from its masked slot, inside the table) but keeps x.
+    const uint32_t c = c1 ? 1u : 0u;
+    const uint32_t tb = tab + (c1 ? 8u * kCtxBytes : 0u);
+    uint32_t e[8], acc = 0;
 #define EP_FIELD(j)                                                                    \
     {                                                                                  \
-        slot = x & (kProbTotal - 1);                                                   \
-        const uint32_t s = lds_u8<(j) * kProbTotal>(st + slot);                        \
-        const uint32_t fa = ft + 2u * s;                                               \
-        const uint32_t q = lds_u16<(j) * 1024>(fa);                                    \
-        const uint32_t cm = lds_u16<(j) * 1024 + 512>(fa);                             \
-        if (active) x = q * (x >> kProbBits) + (slot - cm);                            \
+        const uint32_t ent = lds_u32<(j) * kCtxBytes>(tb + ((x & kSlotMask) << 2));    \
+        if (active) x = (ent >> kEntryQShift) * (x >> kProbBits) + (ent & kEntryBiasMask); \
         renorm_step<FULL>(x, rd, active);                                              \
-        sym[j] = s;                                                                    \
-        top = max(top, s);                                                             \
+        e[j] = ent;                                                                    \
+        acc |= ent;                                                                    \
     }
     EP_FIELD(0) EP_FIELD(1) EP_FIELD(2) EP_FIELD(3) EP_FIELD(4) EP_FIELD(5) EP_FIELD(6) EP_FIELD(7)
 #undef EP_FIELD
 
-    // t[j] = 2 z_j + c, the doubled lattice coordinate (z1..z7 = f1..f7, z8 = 2 f8 + parity of
-    // z1..z7), carried as the bits of the float 1.5 * 2^23 + t, which reads back exactly as
-    // 12582912 + t for |t| < 2^22.  Without escapes f_j = s_j - 127, so t comes straight from the
-    // symbols: 2 s_j - 254 + c, and for the last coordinate 4 s_8 - 508 + 2 par + c with
-    // par = (s_1 + ... + s_7 + 1) mod 2 (7 * 127 is odd).
-    constexpr int32_t kMagic = 0x4B400000;  // bits of 12582912.0f = 1.5 * 2^23
-    int32_t t[8];
-    bool fields_from_symbols = true;
+    bool from_symbols = true;
     int32_t f[8];  // only for the escape path and the fields output
-    if (__any_sync(kFull, active && top == uint32_t(kEscape))) {
+    if (__any_sync(kFull, active && (acc & kEntryEsc))) {
         // escaped fields: the lane's raw words after its renormalisation words, by field
 #pragma unroll
         for (int j = 0; j < 8; ++j) {
-            const bool mine = active && sym[j] == uint32_t(kEscape);
-            f[j] = mine ? int32_t(int16_t(rd.wn)) : int32_t(sym[j]) - kAlphabetR;
+            const bool mine = active && (e[j] & kEntryEsc);
+            f[j] = mine ? int32_t(int16_t(rd.wn)) : int32_t((e[j] >> (kEntrySymShift + 1)) & 255u) - kAlphabetR;
             rd.consume_if(mine);
         }
-        fields_from_symbols = false;
+        from_symbols = false;
     }
     if (!active) return;
 
     if constexpr (OUT == kOutFields) {
-        int16_t* o = static_cast<int16_t*>(p.out) + 9 * v;
+        int16_t* o = reinterpret_cast<int16_t*>(pos.optr);
         o[0] = int16_t(c);
 #pragma unroll
-        for (int j = 0; j < 8; ++j) o[1 + j] = int16_t(fields_from_symbols ? int32_t(sym[j]) - kAlphabetR : f[j]);
+        for (int j = 0; j < 8; ++j)
+            o[1 + j] = int16_t(from_symbols ? int32_t((e[j] >> (kEntrySymShift + 1)) & 255u) - kAlphabetR : f[j]);
         return;
     } else {
-        if (fields_from_symbols) {
-            const int32_t kc = kMagic - 2 * kAlphabetR + int32_t(c);
-            const int32_t par = int32_t(sym[0] + sym[1] + sym[2] + sym[3] + sym[4] + sym[5] + sym[6] + 1u) & 1;
+        // t[j] = 2 z_j + c, the doubled lattice coordinate (z1..z7 = f1..f7, z8 = 2 f8 + parity of
+        // z1..z7), carried as the bits of the float 1.5 * 2^23 + 254 + t, which holds every
+        // integer up to 2^22 away exactly; subtracting 1.5 * 2^23 + 254 then gives t exactly.
+        // Without escapes f_j = s_j - 127, so 254 + t_j = 2 s_j + c comes straight out of the
+        // table entry, and 254 + t_8 = 4 s_8 + 2 par + c - 254 with par = (s_1 + ... + s_7 + 1)
+        // mod 2 (7 * 127 is odd): bit 1 of 2 s_j is the low bit of s_j.
+        constexpr uint32_t kMagic = 0x4B400000u;  // bits of 1.5 * 2^23
+        constexpr float kBias = 12583166.0f;      // 1.5 * 2^23 + 254
+        uint32_t t[8];
+        if (from_symbols) {
+            const uint32_t km = kMagic | c;
 #pragma unroll
-            for (int j = 0; j < 7; ++j) t[j] = 2 * int32_t(sym[j]) + kc;
-            t[7] = 4 * int32_t(sym[7]) + 2 * par + (kc - 2 * kAlphabetR);
+            for (int j = 0; j < 7; ++j) t[j] = ((e[j] >> kEntrySymShift) & 0x1FEu) | km;
+            const uint32_t par2 = ~(t[0] ^ t[1] ^ t[2] ^ t[3] ^ t[4] ^ t[5] ^ t[6]) & 2u;
+            t[7] = (((e[7] >> (kEntrySymShift - 1)) & 0x3FCu) | par2) + (km - 254u);
         } else {
             const int32_t par = (f[0] + f[1] + f[2] + f[3] + f[4] + f[5] + f[6]) & 1;
             f[7] = 2 * f[7] + par;
 #pragma unroll
-            for (int j = 0; j < 8; ++j) t[j] = kMagic + 2 * f[j] + int32_t(c);
+            for (int j = 0; j < 8; ++j) t[j] = uint32_t(int32_t(kMagic + 254u + c) + 2 * f[j]);
         }
         float val[8];
         if (!p.tiny_alpha) {
             // a * y = (a/2) * (2z + c) exactly, so one product rounds once
+            const float2 nb = make_float2(-kBias, -kBias), ah2 = make_float2(pos.ah, pos.ah);
 #pragma unroll
-            for (int i = 0; i < 8; ++i) val[i] = __fmul_rn(ah, __fsub_rn(__int_as_float(t[i]), 12582912.0f));
+            for (int i = 0; i < 4; ++i) {
+                const float2 d = __fadd2_rn(make_float2(__uint_as_float(t[2 * i]), __uint_as_float(t[2 * i + 1])), nb);
+                const float2 r = __fmul2_rn(d, ah2);
+                val[2 * i] = r.x;
+                val[2 * i + 1] = r.y;
+            }
         } else {
 #pragma unroll
             for (int i = 0; i < 8; ++i) {
-                const float y = __fmul_rn(__fsub_rn(__int_as_float(t[i]), 12582912.0f), 0.5f);  // exact
-                val[i] = __fmul_rn(a, y);  // the one rounding of the reconstruction
+                const float y = __fmul_rn(__fsub_rn(__uint_as_float(t[i]), kBias), 0.5f);  // exact
+                val[i] = __fmul_rn(pos.a, y);  // the one rounding of the reconstruction
             }
         }
         if constexpr (VEC) {
-            const int64_t elem = p.dense ? 8 * v : row * p.row_stride + 8 * kcol;
-            store_vec<OUT>(p.out, elem, val);
+            store_vec<OUT>(pos.optr, val);
         } else {
+            constexpr int es = OutElem<OUT>::kBytes;
 #pragma unroll
-            for (int i = 0; i < 8; ++i) {
-                const int64_t col = 8 * kcol + i;
-                if (col < p.cols) store_one<OUT>(p.out, row * p.row_stride + col, val[i]);
-            }
+            for (int i = 0; i < 8; ++i)
+                if (8 * int64_t(pos.kcol) + i < p.cols) store_one<OUT>(pos.optr + i * es, val[i]);
         }
     }
 }
 
 // Decode the steps of one tile with a given word reader; returns the status flags of the tile.
 template <int OUT, bool VEC, class Reader, class Guard>
-__device__ __forceinline__ uint32_t decode_tile_steps(const Params& p, uint32_t sym0, uint32_t fc0, Reader& rd,
-                                                      uint32_t& x, uint32_t tile, uint32_t lane, Guard in_range) {
+__device__ __forceinline__ uint32_t decode_tile_steps(const Params& p, uint32_t tab, Reader& rd, uint32_t& x,
+                                                      uint32_t tile, uint32_t lane, Guard in_range) {
     const int64_t per_tile = int64_t(kLanes) * p.steps;
     const int64_t v0 = int64_t(tile) * per_tile;
-    const int64_t vend = min(v0 + per_tile, p.n_vectors);
-    const uint32_t nsteps = uint32_t((vend - v0 + kLanes - 1) / kLanes);
-    int64_t v = v0 + lane;
-    int64_t row = v / p.vec_per_row, kcol = v - row * p.vec_per_row;
-    for (uint32_t k = 0; k < nsteps; ++k) {
+    const uint32_t nv = uint32_t(min(per_tile, p.n_vectors - v0));
+    const uint32_t nfull = nv / kLanes, rem = nv % kLanes;
+    Pos pos = first_pos<OUT>(p, v0 + lane);
+    for (uint32_t k = 0; k < nfull; ++k) {
         if (!__all_sync(kFull, in_range(rd))) return kStOverrun;  // a corrupt tile ran away
-        if (v0 + int64_t(k + 1) * kLanes <= vend)
-            decode_step<OUT, VEC, true>(p, sym0, fc0, rd, x, true, v, row, kcol);
-        else
-            decode_step<OUT, VEC, false>(p, sym0, fc0, rd, x, v < vend, v, row, kcol);
-        v += kLanes;
-        kcol += kLanes;
-        while (kcol >= p.vec_per_row) {
-            kcol -= p.vec_per_row;
-            ++row;
-        }
+        decode_step<OUT, VEC, true>(p, tab, rd, x, true, pos);
+        advance<OUT>(p, pos);
+    }
+    if (rem) {
+        if (!__all_sync(kFull, in_range(rd))) return kStOverrun;
+        decode_step<OUT, VEC, false>(p, tab, rd, x, lane < rem, pos);
     }
     return 0;
 }
@@ -514,22 +576,23 @@ __global__ void __launch_bounds__(WARPS * 32, 1) decode_kernel(const Params p) {
 
     uint64_t t0 = 0;
     uint32_t tbytes = 0;
+    if (BUILD) {  // expand the table first: its scratch lies in the tile buffers
+        build_tables<WARPS>(sm.tab, *reinterpret_cast<BuildScratch*>(&sm.tbuf[0][0]), p);
+        __syncthreads();
+    }
     if (tile < p.n_tiles) {  // the first tile's fetch overlaps the table staging
         t0 = 16ull * __ldg(p.tile_off + tile);
         tbytes = uint32_t(16ull * __ldg(p.tile_off + tile + 1) - t0);  // the host checked >= 160
         if (tbytes <= kBuf) stage(tile, t0, tbytes);
     }
-    if (BUILD) {
-        build_tables<WARPS>(sm, p);
-        __syncthreads();
-    } else if (!mbar_wait(&sm.tbar, 0)) {
+    if (!BUILD && !mbar_wait(&sm.tbar, 0)) {
         if (lane == 0) atomicOr(p.status, kStTimeout);
         goto drain;
     }
 
     asm volatile("griddepcontrol.wait;" ::: "memory");  // no-op unless launched as a dependent
     {
-        const uint32_t sym0 = smem_u32(&sm.sym[0][0]), fc0 = smem_u32(&sm.fc[0][0][0]);
+        const uint32_t tab = smem_u32(&sm.tab[0][0]);
         bool first = true;
         for (; tile < p.n_tiles; tile += tile_stride) {
             if (!first) {
@@ -577,8 +640,8 @@ __global__ void __launch_bounds__(WARPS * 32, 1) decode_kernel(const Params p) {
                 rd.wp = buf_a + uint32_t(min(max(o0, 0), int32_t(tbytes) - 2));
                 rd.wn = lds_u16(rd.wp);
                 const uint32_t wp0 = rd.wp, lo = buf_a, hi = buf_a + kBuf;
-                flags = decode_tile_steps<OUT, VEC>(p, sym0, fc0, rd, x, tile, lane,
-                                                    [=](const SmemReader& r) { return r.wp >= lo && r.wp <= hi; });
+                flags = decode_tile_steps<OUT, VEC>(p, tab, rd, x, tile, lane,
+                                                    [=](const SmemReader& r) { return r.wp - lo <= hi - lo; });
                 nread = rd.consumed(wp0);
             } else {
                 GlobalReader rd;
@@ -587,7 +650,7 @@ __global__ void __launch_bounds__(WARPS * 32, 1) decode_kernel(const Params p) {
                 rd.hi = int32_t(tbytes) - 2;
                 rd.off = o0;
                 rd.wn = __ldg(reinterpret_cast<const uint16_t*>(tg + min(max(o0, 0), rd.hi)));
-                flags = decode_tile_steps<OUT, VEC>(p, sym0, fc0, rd, x, tile, lane,
+                flags = decode_tile_steps<OUT, VEC>(p, tab, rd, x, tile, lane,
                                                     [](const GlobalReader&) { return true; });
                 nread = rd.consumed(o0);
             }
@@ -611,12 +674,17 @@ drain:
     if (tile < p.n_tiles && tbytes <= kBuf) mbar_wait(&sm.bar[warp], 0);
 }
 
-// Expands the blob's compact frequency tables into the 80 KB decode-table block (one CTA).
+// Expands the blob's compact frequency tables into the 64 KB packed decode table (one CTA).
+struct ExpandSmem {
+    uint32_t tab[kFieldContexts][kProbTotal];
+    BuildScratch scratch;
+};
+
 template <int WARPS>
 __global__ void __launch_bounds__(WARPS * 32, 1) expand_tables_kernel(const Params p, uint8_t* tables) {
     extern __shared__ __align__(128) uint8_t smem_raw[];
-    Smem<WARPS>& sm = *reinterpret_cast<Smem<WARPS>*>(smem_raw);
-    build_tables<WARPS>(sm, p);
+    ExpandSmem& sm = *reinterpret_cast<ExpandSmem*>(smem_raw);
+    build_tables<WARPS>(sm.tab, sm.scratch, p);
     __syncthreads();
     const uint4* s = reinterpret_cast<const uint4*>(smem_raw);
     uint4* d = reinterpret_cast<uint4*>(tables);
@@ -624,8 +692,8 @@ __global__ void __launch_bounds__(WARPS * 32, 1) expand_tables_kernel(const Para
 }
 
 // ---- host-side launch -------------------------------------------------------------------------
-// 32 warps per CTA when every tile fits a 4.5 KB buffer (more tiles in flight per SM), else 16
-// warps with 9 KB buffers; a tile larger than that is read from global memory.
+// 32 warps per CTA when every tile fits a 5 KB buffer (more tiles in flight per SM), else 16
+// warps with 10 KB buffers; a tile larger than that is read from global memory.
 constexpr int kWarpsWide = 32, kWarpsNarrow = 16;
 
 struct DevInfo {
@@ -731,10 +799,11 @@ Params make_params(const ep_blob* b, const uint8_t* dblob, const uint8_t* tables
     p.alpha = reinterpret_cast<const float*>(dblob + L.off_alpha);
     p.out = out;
     p.status = status;
+    p.rows = L.rows;
     p.cols = L.cols;
     p.row_stride = row_stride;
     p.n_vectors = L.n_vectors;
-    p.vec_per_row = L.vec_per_row;
+    p.vec_per_row = uint32_t(L.vec_per_row);
     p.steps = L.steps;
     p.n_tiles = L.n_tiles;
     p.q_coset0 = L.q_coset[0];
@@ -744,7 +813,6 @@ Params make_params(const ep_blob* b, const uint8_t* dblob, const uint8_t* tables
         p.lo[c] = L.lo[c];
         p.n[c] = L.n[c];
     }
-    p.dense = vec && row_stride == L.cols;
     p.tiny_alpha = L.tiny_alpha;
     return p;
 }
@@ -768,9 +836,9 @@ int ensure_device(ep_blob* b, int dev, cudaStream_t st) {
     // expand the compact frequency tables once for this device copy
     Params p = make_params(b, blob, nullptr, nullptr, b->layout.cols, status, false);
     auto fn = expand_tables_kernel<kWarpsWide>;
-    EP_CUDA(cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, int(kTableBytes)),
+    EP_CUDA(cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, int(sizeof(ExpandSmem))),
             "table expansion attribute");
-    fn<<<1, kWarpsWide * 32, kTableBytes, st>>>(p, tables);
+    fn<<<1, kWarpsWide * 32, sizeof(ExpandSmem), st>>>(p, tables);
     EP_CUDA(cudaGetLastError(), "table expansion launch");
     EP_CUDA(cudaStreamSynchronize(st), "blob upload");
     d.blob = blob;

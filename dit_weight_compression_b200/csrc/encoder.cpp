@@ -192,8 +192,8 @@ struct Counts {
     }
 };
 
-// 12-bit frequencies from counts: q = max(1, round-half-up(4096 n / N)) for used symbols, then
-// the sum is brought to 4096 -- excess taken one at a time from the largest q (> 1, lowest symbol
+// 10-bit frequencies from counts: q = max(1, round-half-up(M n / N)) for used symbols, then
+// the sum is brought to M -- excess taken one at a time from the largest q (> 1, lowest symbol
 // first), deficit given one at a time to the most frequent symbol (lowest symbol first).
 static void quantise_freqs(const uint64_t* n, uint16_t* q) {
     uint64_t total = 0;
@@ -365,7 +365,7 @@ int encode(const EncodeInput& in, double target, const EncodeOptions& opt, std::
         for (int c = 0; c < 17; ++c)
             for (int sy = 0; sy < 256; ++sy) {
                 uint64_t n = all.c[size_t(256 * c + sy)];
-                if (n) bits += double(n) * -std::log2(double(T.q[c][sy]) / 4096.0);
+                if (n) bits += double(n) * -std::log2(double(T.q[c][sy]) / double(kProbTotal));
             }
         double payload = (double(rows) / double(n_sample)) * (bits / 8.0 + 2.0 * double(all.escapes));
         double meta = double(kHeaderBytes + round_up16(T.section_bytes()) + round_up16(4 * uint64_t(rows)) +
@@ -507,8 +507,8 @@ bool parse_blob(const uint8_t* d, size_t n, BlobLayout& L, std::string& why) {
     L.off_offsets = rd64(d + 64);
     L.off_stream = rd64(d + 72);
     if (L.total != n) return fail("stored size differs from the byte count");
-    if (L.rows <= 0 || L.cols <= 0 || L.rows > (int64_t(1) << 40) || L.cols > (int64_t(1) << 40))
-        return fail("bad shape");
+    if (L.rows <= 0 || L.cols <= 0 || L.rows > (int64_t(1) << 40) || L.cols > (int64_t(1) << 33))
+        return fail("bad shape");  // (the decoder keeps a row's vector index in 32 bits)
     if (L.steps == 0 || L.steps > 1024) return fail("bad steps per tile");
     L.vec_per_row = (L.cols + 7) / 8;
     L.n_vectors = L.rows * L.vec_per_row;
@@ -524,7 +524,7 @@ bool parse_blob(const uint8_t* d, size_t n, BlobLayout& L, std::string& why) {
     const uint8_t* t = d + L.off_tables;
     L.q_coset[0] = rd16(t);
     L.q_coset[1] = rd16(t + 2);
-    if (uint32_t(L.q_coset[0]) + L.q_coset[1] != kProbTotal) return fail("coset table does not sum to 4096");
+    if (uint32_t(L.q_coset[0]) + L.q_coset[1] != kProbTotal) return fail("coset table does not sum to 1024");
     uint64_t pos = L.off_tables + 4;
     for (int c = 0; c < kFieldContexts; ++c) {
         if (pos + 4 > L.off_alpha) return fail("table section truncated");
@@ -537,7 +537,7 @@ bool parse_blob(const uint8_t* d, size_t n, BlobLayout& L, std::string& why) {
         if (pos > L.off_alpha) return fail("table section truncated");
         uint32_t sum = L.esc_q[c];
         for (int i = 0; i < L.n[c]; ++i) sum += rd16(d + L.q_offset[c] + 2 * i);
-        if (sum != 0 && sum != kProbTotal) return fail("field table does not sum to 4096");
+        if (sum != 0 && sum != kProbTotal) return fail("field table does not sum to 1024");
     }
     for (int64_t r = 0; r < L.rows; ++r) {
         uint32_t ab = rd32(d + L.off_alpha + 4 * r);

@@ -5,7 +5,7 @@
 // and reconstruction") lists: "the probability tables, row scales, and tile metadata" next to
 // the rANS-coded fields.  Byte layout (little-endian, every section 16-byte aligned):
 //
-//   header, 80 bytes:  "EPK1" | u16 version = 1 | u8 dtype | u8 R = 127 | u64 rows | u64 cols |
+//   header, 80 bytes:  "EPK1" | u16 version = 2 | u8 dtype | u8 R = 127 | u64 rows | u64 cols |
 //                      u32 S | u32 n_tiles | f64 s | u64 total bytes | u64 table offset |
 //                      u64 row-scale offset | u64 tile-offset offset | u64 stream offset
 //   tables:            u16 q(coset 0), u16 q(coset 1); then for c = 0, 1 and j = 1..8:
@@ -17,7 +17,8 @@
 //                      2p+1's backward from its end), zero padding to a multiple of 16 bytes
 //
 // Symbols: field value f with |f| <= 127 is the symbol f + 127; any other value is the escape
-// symbol 255 followed by the raw int16 word.  Frequencies of every used context sum to 4096.
+// symbol 255 followed by the raw int16 word.  Frequencies of every used context sum to
+// M = 1024 (version 2; 10-bit totals).
 #pragma once
 
 #include <cstdint>
@@ -27,11 +28,11 @@
 
 namespace ep {
 
-constexpr uint32_t kVersion = 1;
+constexpr uint32_t kVersion = 2;
 constexpr int kAlphabetR = 127;
 constexpr int kEscape = 255;
-constexpr uint32_t kProbBits = 12;
-constexpr uint32_t kProbTotal = 1u << kProbBits;  // 4096
+constexpr uint32_t kProbBits = 10;
+constexpr uint32_t kProbTotal = 1u << kProbBits;  // M = 1024
 constexpr uint32_t kStateLow = 1u << 16;          // rANS lower bound, 16-bit renormalisation
 constexpr int kLanes = 32;                        // interleaved states per tile
 constexpr int kPairs = kLanes / 2;                // lanes 2p, 2p+1 share word region p

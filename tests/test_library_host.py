@@ -123,16 +123,16 @@ def test_corrupt_blobs_rejected(ep):
     bad = [
         b[:79],                                            # truncated header
         _corrupt(b, 0, b"EPK2"),                           # magic
-        _corrupt(b, 4, b"\x02\x00"),                       # version
+        _corrupt(b, 4, b"\x01\x00"),                       # version (1: 12-bit totals)
         _corrupt(b, 6, b"\x09"),                           # dtype
         _corrupt(b, 7, b"\x7e"),                           # alphabet
         b[:-16],                                           # size mismatch
         _corrupt(b, 24, (1).to_bytes(4, "little")),        # S inconsistent with n_tiles
         _corrupt(b, 48, (81).to_bytes(8, "little")),       # misaligned table section
-        _corrupt(b, 80, (4095).to_bytes(2, "little")),     # coset table does not sum to 4096
+        _corrupt(b, 80, (1023).to_bytes(2, "little")),     # coset table does not sum to 1024
     ]
     off_offs = int.from_bytes(b[64:72], "little")
-    bad.append(_corrupt(b, off_offs + 4, (3).to_bytes(4, "little")))   # tile shorter than 128 B
+    bad.append(_corrupt(b, off_offs + 4, (3).to_bytes(4, "little")))   # tile shorter than its header
     for i, x in enumerate(bad):
         with pytest.raises(ep.EPError) as e:
             ep.CompressedTensor.from_bytes(x)
