@@ -98,11 +98,10 @@ struct Params {
     uint32_t esc_q[kFieldContexts];
     uint32_t lo[kFieldContexts];
     uint32_t n[kFieldContexts];
-    int tiny_alpha;             // some |alpha| < 2^-125, where alpha / 2 would round
 };
 
 constexpr uint32_t kSmemOptin = 232448;  // 227 KB: the largest dynamic shared memory of one CTA
-constexpr uint32_t kBufSlack = 48;        // bytes after a tile buffer that a step may over-read
+constexpr uint32_t kBufSlack = 80;        // bytes after a tile buffer that two steps may over-read
 
 // Per-warp tile buffer size for a CTA of WARPS warps: what the 227 KB leave after the table.
 template <int WARPS>
@@ -360,12 +359,13 @@ __device__ __forceinline__ void store_one(uint8_t* dst, float v) {
 }
 
 // ---- one step: every lane decodes (at most) one 8-vector --------------------------------------
-// Where a lane's current vector goes: vector kcol of row `row`, whose first element is at optr.
+// Where a lane's current vector goes: vector kcol of row `row`, whose first element is at optr,
+// and that row's scale.
 struct Pos {
     uint8_t* optr;
     int64_t row;
     uint32_t kcol;
-    float a, ah;  // the row's scale, and scale / 2
+    float a;
 };
 
 template <int OUT>
@@ -375,40 +375,46 @@ __device__ __forceinline__ Pos first_pos(const Params& p, int64_t v) {
         s.optr = static_cast<uint8_t*>(p.out) + 18 * v;  // 9 int16 per vector
         s.row = 0;
         s.kcol = 0;
-        s.a = s.ah = 0.0f;
+        s.a = 0.0f;
     } else {
         s.row = v / p.vec_per_row;
         s.kcol = uint32_t(v - s.row * p.vec_per_row);
         s.optr = static_cast<uint8_t*>(p.out) + (s.row * p.row_stride + 8 * int64_t(s.kcol)) * OutElem<OUT>::kBytes;
         s.a = v < p.n_vectors ? __ldg(p.alpha + s.row) : 0.0f;
-        s.ah = __fmul_rn(s.a, 0.5f);
     }
     return s;
 }
 
 // The lane's next vector is 32 further on; the row scale is reloaded only when the row changes.
-template <int OUT>
+// WIDE: rows hold at least 32 vectors, so a step crosses at most one row end (no branch).
+template <int OUT, bool WIDE>
 __device__ __forceinline__ void advance(const Params& p, Pos& s) {
     if constexpr (OUT == kOutFields) {
         s.optr += 32 * 18;
     } else {
         constexpr int es = OutElem<OUT>::kBytes;
+        const int64_t wrap = (p.row_stride - 8 * int64_t(p.vec_per_row)) * es;
         s.kcol += 32;
         s.optr += 32 * 8 * es;
-        if (s.kcol >= p.vec_per_row) {
-            const int64_t wrap = (p.row_stride - 8 * int64_t(p.vec_per_row)) * es;
+        if constexpr (WIDE) {
+            const bool w = s.kcol >= p.vec_per_row;
+            s.kcol -= w ? p.vec_per_row : 0u;
+            s.row += w ? 1 : 0;
+            s.optr += w ? wrap : 0;
+            if (w && s.row < p.rows) s.a = __ldg(p.alpha + s.row);
+        } else if (s.kcol >= p.vec_per_row) {
             do {
                 s.kcol -= p.vec_per_row;
                 ++s.row;
                 s.optr += wrap;
             } while (s.kcol >= p.vec_per_row);
             s.a = s.row < p.rows ? __ldg(p.alpha + s.row) : 0.0f;
-            s.ah = __fmul_rn(s.a, 0.5f);
         }
     }
 }
 
-template <int OUT, bool VEC, bool FULL, class Reader>
+// ESC: the blob's tables give the escape symbol a frequency, so a field may be a raw word.
+template <int OUT, bool VEC, bool ESC, bool FULL, class Reader>
 __device__ __forceinline__ void decode_step(const Params& p, uint32_t tab, Reader& rd, uint32_t& x, bool active,
                                             const Pos& pos) {
     if (FULL) active = true;
@@ -430,14 +436,14 @@ __device__ __forceinline__ void decode_step(const Params& p, uint32_t tab, Reade
         if (active) x = (ent >> kEntryQShift) * (x >> kProbBits) + (ent & kEntryBiasMask); \
         renorm_step<FULL>(x, rd, active);                                              \
         e[j] = ent;                                                                    \
-        acc |= ent;                                                                    \
+        if (ESC) acc |= ent;                                                           \
     }
     EP_FIELD(0) EP_FIELD(1) EP_FIELD(2) EP_FIELD(3) EP_FIELD(4) EP_FIELD(5) EP_FIELD(6) EP_FIELD(7)
 #undef EP_FIELD
 
     bool from_symbols = true;
     int32_t f[8];  // only for the escape path and the fields output
-    if (__any_sync(kFull, active && (acc & kEntryEsc))) {
+    if (ESC && __any_sync(kFull, active && (acc & kEntryEsc))) {
         // escaped fields: the lane's raw words after its renormalisation words, by field
 #pragma unroll
         for (int j = 0; j < 8; ++j) {
@@ -458,13 +464,12 @@ __device__ __forceinline__ void decode_step(const Params& p, uint32_t tab, Reade
         return;
     } else {
         // t[j] = 2 z_j + c, the doubled lattice coordinate (z1..z7 = f1..f7, z8 = 2 f8 + parity of
-        // z1..z7), carried as the bits of the float 1.5 * 2^23 + 254 + t, which holds every
-        // integer up to 2^22 away exactly; subtracting 1.5 * 2^23 + 254 then gives t exactly.
-        // Without escapes f_j = s_j - 127, so 254 + t_j = 2 s_j + c comes straight out of the
-        // table entry, and 254 + t_8 = 4 s_8 + 2 par + c - 254 with par = (s_1 + ... + s_7 + 1)
-        // mod 2 (7 * 127 is odd): bit 1 of 2 s_j is the low bit of s_j.
-        constexpr uint32_t kMagic = 0x4B400000u;  // bits of 1.5 * 2^23
-        constexpr float kBias = 12583166.0f;      // 1.5 * 2^23 + 254
+        // z1..z7), carried as the bits of the float T = 1.5 * 2^23 + 254 + t, which holds every
+        // integer up to 2^22 away exactly.  Without escapes f_j = s_j - 127, so 254 + t_j = 2 s_j + c
+        // comes straight out of the table entry, and 254 + t_8 = 4 s_8 + 2 par + c - 254 with
+        // par = (s_1 + ... + s_7 + 1) mod 2 (7 * 127 is odd): bit 1 of 2 s_j is the low bit of s_j.
+        constexpr uint32_t kMagic = 0x4B400000u;     // bits of 1.5 * 2^23
+        constexpr float kHalfBias = 6291583.0f;      // (1.5 * 2^23 + 254) / 2
         uint32_t t[8];
         if (from_symbols) {
             const uint32_t km = kMagic | c;
@@ -478,23 +483,17 @@ __device__ __forceinline__ void decode_step(const Params& p, uint32_t tab, Reade
 #pragma unroll
             for (int j = 0; j < 8; ++j) t[j] = uint32_t(int32_t(kMagic + 254u + c) + 2 * f[j]);
         }
+        // y = T / 2 - kHalfBias = z + c/2 in one fused multiply-add: T / 2 is exact and so is
+        // the difference (a multiple of 1/2 below 2^17), so y is exact; a * y then rounds once.
         float val[8];
-        if (!p.tiny_alpha) {
-            // a * y = (a/2) * (2z + c) exactly, so one product rounds once
-            const float2 nb = make_float2(-kBias, -kBias), ah2 = make_float2(pos.ah, pos.ah);
+        const float2 half = make_float2(0.5f, 0.5f), nb = make_float2(-kHalfBias, -kHalfBias);
+        const float2 a2 = make_float2(pos.a, pos.a);
 #pragma unroll
-            for (int i = 0; i < 4; ++i) {
-                const float2 d = __fadd2_rn(make_float2(__uint_as_float(t[2 * i]), __uint_as_float(t[2 * i + 1])), nb);
-                const float2 r = __fmul2_rn(d, ah2);
-                val[2 * i] = r.x;
-                val[2 * i + 1] = r.y;
-            }
-        } else {
-#pragma unroll
-            for (int i = 0; i < 8; ++i) {
-                const float y = __fmul_rn(__fsub_rn(__uint_as_float(t[i]), kBias), 0.5f);  // exact
-                val[i] = __fmul_rn(pos.a, y);  // the one rounding of the reconstruction
-            }
+        for (int i = 0; i < 4; ++i) {
+            const float2 y = __ffma2_rn(make_float2(__uint_as_float(t[2 * i]), __uint_as_float(t[2 * i + 1])), half, nb);
+            const float2 r = __fmul2_rn(y, a2);
+            val[2 * i] = r.x;
+            val[2 * i + 1] = r.y;
         }
         if constexpr (VEC) {
             store_vec<OUT>(pos.optr, val);
@@ -507,8 +506,29 @@ __device__ __forceinline__ void decode_step(const Params& p, uint32_t tab, Reade
     }
 }
 
+// Decode the full steps of a tile, two between runaway checks (the tile buffer's slack covers
+// what two steps may read past a checked position).
+template <int OUT, bool VEC, bool ESC, bool WIDE, class Reader, class Guard>
+__device__ __forceinline__ uint32_t full_steps(const Params& p, uint32_t tab, Reader& rd, uint32_t& x, Pos& pos,
+                                               uint32_t nfull, Guard in_range) {
+    uint32_t k = 0;
+    for (; k + 2 <= nfull; k += 2) {
+        if (!__all_sync(kFull, in_range(rd))) return kStOverrun;  // a corrupt tile ran away
+        decode_step<OUT, VEC, ESC, true>(p, tab, rd, x, true, pos);
+        advance<OUT, WIDE>(p, pos);
+        decode_step<OUT, VEC, ESC, true>(p, tab, rd, x, true, pos);
+        advance<OUT, WIDE>(p, pos);
+    }
+    if (k < nfull) {
+        if (!__all_sync(kFull, in_range(rd))) return kStOverrun;
+        decode_step<OUT, VEC, ESC, true>(p, tab, rd, x, true, pos);
+        advance<OUT, WIDE>(p, pos);
+    }
+    return 0;
+}
+
 // Decode the steps of one tile with a given word reader; returns the status flags of the tile.
-template <int OUT, bool VEC, class Reader, class Guard>
+template <int OUT, bool VEC, bool ESC, class Reader, class Guard>
 __device__ __forceinline__ uint32_t decode_tile_steps(const Params& p, uint32_t tab, Reader& rd, uint32_t& x,
                                                       uint32_t tile, uint32_t lane, Guard in_range) {
     const int64_t per_tile = int64_t(kLanes) * p.steps;
@@ -516,20 +536,19 @@ __device__ __forceinline__ uint32_t decode_tile_steps(const Params& p, uint32_t 
     const uint32_t nv = uint32_t(min(per_tile, p.n_vectors - v0));
     const uint32_t nfull = nv / kLanes, rem = nv % kLanes;
     Pos pos = first_pos<OUT>(p, v0 + lane);
-    for (uint32_t k = 0; k < nfull; ++k) {
-        if (!__all_sync(kFull, in_range(rd))) return kStOverrun;  // a corrupt tile ran away
-        decode_step<OUT, VEC, true>(p, tab, rd, x, true, pos);
-        advance<OUT>(p, pos);
-    }
+    const uint32_t st = p.vec_per_row >= uint32_t(kLanes)
+                            ? full_steps<OUT, VEC, ESC, true>(p, tab, rd, x, pos, nfull, in_range)
+                            : full_steps<OUT, VEC, ESC, false>(p, tab, rd, x, pos, nfull, in_range);
+    if (st) return st;
     if (rem) {
         if (!__all_sync(kFull, in_range(rd))) return kStOverrun;
-        decode_step<OUT, VEC, false>(p, tab, rd, x, lane < rem, pos);
+        decode_step<OUT, VEC, ESC, false>(p, tab, rd, x, lane < rem, pos);
     }
     return 0;
 }
 
 // BUILD = false: stage the pre-expanded table block from p.tables; true: expand it in each CTA.
-template <int WARPS, int OUT, bool VEC, bool BUILD>
+template <int WARPS, int OUT, bool VEC, bool BUILD, bool ESC>
 __global__ void __launch_bounds__(WARPS * 32, 1) decode_kernel(const Params p) {
     extern __shared__ __align__(128) uint8_t smem_raw[];
     Smem<WARPS>& sm = *reinterpret_cast<Smem<WARPS>*>(smem_raw);
@@ -640,8 +659,8 @@ __global__ void __launch_bounds__(WARPS * 32, 1) decode_kernel(const Params p) {
                 rd.wp = buf_a + uint32_t(min(max(o0, 0), int32_t(tbytes) - 2));
                 rd.wn = lds_u16(rd.wp);
                 const uint32_t wp0 = rd.wp, lo = buf_a, hi = buf_a + kBuf;
-                flags = decode_tile_steps<OUT, VEC>(p, tab, rd, x, tile, lane,
-                                                    [=](const SmemReader& r) { return r.wp - lo <= hi - lo; });
+                flags = decode_tile_steps<OUT, VEC, ESC>(p, tab, rd, x, tile, lane,
+                                                         [=](const SmemReader& r) { return r.wp - lo <= hi - lo; });
                 nread = rd.consumed(wp0);
             } else {
                 GlobalReader rd;
@@ -650,8 +669,8 @@ __global__ void __launch_bounds__(WARPS * 32, 1) decode_kernel(const Params p) {
                 rd.hi = int32_t(tbytes) - 2;
                 rd.off = o0;
                 rd.wn = __ldg(reinterpret_cast<const uint16_t*>(tg + min(max(o0, 0), rd.hi)));
-                flags = decode_tile_steps<OUT, VEC>(p, tab, rd, x, tile, lane,
-                                                    [](const GlobalReader&) { return true; });
+                flags = decode_tile_steps<OUT, VEC, ESC>(p, tab, rd, x, tile, lane,
+                                                         [](const GlobalReader&) { return true; });
                 nread = rd.consumed(o0);
             }
             // integrity: every state back at 2^16; in every region the two lanes read exactly
@@ -703,9 +722,9 @@ struct DevInfo {
 std::mutex g_dev_mu;
 DevInfo g_dev[kMaxDevices];
 
-template <int WARPS, int OUT, bool VEC>
+template <int WARPS, int OUT, bool VEC, bool ESC>
 int launch_one(const Params& p, cudaStream_t st, int device, bool dependent) {
-    auto fn = decode_kernel<WARPS, OUT, VEC, false>;
+    auto fn = decode_kernel<WARPS, OUT, VEC, false, ESC>;
     const size_t smem = sizeof(Smem<WARPS>);
     static std::mutex mu;
     static int per_sm[kMaxDevices] = {};
@@ -739,25 +758,32 @@ int launch_one(const Params& p, cudaStream_t st, int device, bool dependent) {
     return EP_OK;
 }
 
-template <int OUT>
+template <int OUT, bool ESC>
 int launch_out(const Params& p, bool vec, bool wide, cudaStream_t st, int device, bool dep) {
     if (wide)
-        return vec ? launch_one<kWarpsWide, OUT, true>(p, st, device, dep)
-                   : launch_one<kWarpsWide, OUT, false>(p, st, device, dep);
-    return vec ? launch_one<kWarpsNarrow, OUT, true>(p, st, device, dep)
-               : launch_one<kWarpsNarrow, OUT, false>(p, st, device, dep);
+        return vec ? launch_one<kWarpsWide, OUT, true, ESC>(p, st, device, dep)
+                   : launch_one<kWarpsWide, OUT, false, ESC>(p, st, device, dep);
+    return vec ? launch_one<kWarpsNarrow, OUT, true, ESC>(p, st, device, dep)
+               : launch_one<kWarpsNarrow, OUT, false, ESC>(p, st, device, dep);
 }
 
-int launch(const Params& p, int out_kind, bool vec, uint64_t max_tile, cudaStream_t st, int device,
+template <int OUT>
+int launch_out(const Params& p, bool vec, bool wide, bool esc, cudaStream_t st, int device, bool dep) {
+    return esc ? launch_out<OUT, true>(p, vec, wide, st, device, dep)
+               : launch_out<OUT, false>(p, vec, wide, st, device, dep);
+}
+
+// esc: the blob's tables give the escape symbol a frequency (else the escape-free kernel runs).
+int launch(const Params& p, int out_kind, bool vec, uint64_t max_tile, bool esc, cudaStream_t st, int device,
            bool dependent) {
     const bool wide = max_tile <= Geo<kWarpsWide>::kBuf;
     switch (out_kind) {
-        case kOutBF16: return launch_out<kOutBF16>(p, vec, wide, st, device, dependent);
-        case kOutFP16: return launch_out<kOutFP16>(p, vec, wide, st, device, dependent);
-        case kOutE4M3: return launch_out<kOutE4M3>(p, vec, wide, st, device, dependent);
-        case kOutF32: return launch_out<kOutF32>(p, vec, wide, st, device, dependent);
+        case kOutBF16: return launch_out<kOutBF16>(p, vec, wide, esc, st, device, dependent);
+        case kOutFP16: return launch_out<kOutFP16>(p, vec, wide, esc, st, device, dependent);
+        case kOutE4M3: return launch_out<kOutE4M3>(p, vec, wide, esc, st, device, dependent);
+        case kOutF32: return launch_out<kOutF32>(p, vec, wide, esc, st, device, dependent);
         default:  // the fields test hook: the 16-warp kernel has the registers it needs
-            return launch_one<kWarpsNarrow, kOutFields, false>(p, st, device, false);
+            return launch_one<kWarpsNarrow, kOutFields, false, true>(p, st, device, false);
     }
 }
 
@@ -813,7 +839,6 @@ Params make_params(const ep_blob* b, const uint8_t* dblob, const uint8_t* tables
         p.lo[c] = L.lo[c];
         p.n[c] = L.n[c];
     }
-    p.tiny_alpha = L.tiny_alpha;
     return p;
 }
 
@@ -865,9 +890,9 @@ struct NoallocDevice {
 NoallocDevice g_noalloc[kMaxDevices];
 std::mutex g_noalloc_mu;
 
-template <int WARPS, int OUT, bool VEC>
+template <int WARPS, int OUT, bool VEC, bool ESC>
 int noalloc_launch_one(const Params& p, cudaStream_t st, int device) {
-    auto fn = decode_kernel<WARPS, OUT, VEC, true>;
+    auto fn = decode_kernel<WARPS, OUT, VEC, true, ESC>;
     const size_t smem = sizeof(Smem<WARPS>);
     static std::mutex mu;
     static int per_sm[kMaxDevices] = {};
@@ -890,17 +915,20 @@ int noalloc_launch_one(const Params& p, cudaStream_t st, int device) {
 }
 
 template <int OUT>
-int noalloc_launch_out(const Params& p, bool vec, cudaStream_t st, int device) {
-    return vec ? noalloc_launch_one<kWarpsNarrow, OUT, true>(p, st, device)
-               : noalloc_launch_one<kWarpsNarrow, OUT, false>(p, st, device);
+int noalloc_launch_out(const Params& p, bool vec, bool esc, cudaStream_t st, int device) {
+    if (esc)
+        return vec ? noalloc_launch_one<kWarpsNarrow, OUT, true, true>(p, st, device)
+                   : noalloc_launch_one<kWarpsNarrow, OUT, false, true>(p, st, device);
+    return vec ? noalloc_launch_one<kWarpsNarrow, OUT, true, false>(p, st, device)
+               : noalloc_launch_one<kWarpsNarrow, OUT, false, false>(p, st, device);
 }
 
-int noalloc_launch(const Params& p, int out_kind, bool vec, cudaStream_t st, int device) {
+int noalloc_launch(const Params& p, int out_kind, bool vec, bool esc, cudaStream_t st, int device) {
     switch (out_kind) {
-        case kOutBF16: return noalloc_launch_out<kOutBF16>(p, vec, st, device);
-        case kOutFP16: return noalloc_launch_out<kOutFP16>(p, vec, st, device);
-        case kOutE4M3: return noalloc_launch_out<kOutE4M3>(p, vec, st, device);
-        default: return noalloc_launch_out<kOutF32>(p, vec, st, device);
+        case kOutBF16: return noalloc_launch_out<kOutBF16>(p, vec, esc, st, device);
+        case kOutFP16: return noalloc_launch_out<kOutFP16>(p, vec, esc, st, device);
+        case kOutE4M3: return noalloc_launch_out<kOutE4M3>(p, vec, esc, st, device);
+        default: return noalloc_launch_out<kOutF32>(p, vec, esc, st, device);
     }
 }
 
@@ -945,7 +973,7 @@ extern "C" int ep_decompress(const ep_blob* cb, const ep_tensor* out, void* stre
         const DeviceCopy& d = b->dev[dev];
         const bool vec = vec_ok(L, out->data, out->row_stride, out->dtype);
         Params p = make_params(b, d.blob, d.tables, out->data, out->row_stride, d.status, vec);
-        return launch(p, kind, vec, L.max_tile_bytes, st, dev, true);
+        return launch(p, kind, vec, L.max_tile_bytes, L.has_escape, st, dev, true);
     }
 
     // Host output: upload the bytes, decode into a blob-owned buffer, copy back, synchronise.
@@ -979,7 +1007,7 @@ extern "C" int ep_decompress(const ep_blob* cb, const ep_tensor* out, void* stre
             "ep_decompress: upload");
     const bool vec = vec_ok(L, d.stage_out, L.cols, out->dtype);
     Params p = make_params(b, d.stage_blob, d.tables, d.stage_out, L.cols, d.status, vec);
-    rc = launch(p, kind, vec, L.max_tile_bytes, st, dev, false);
+    rc = launch(p, kind, vec, L.max_tile_bytes, L.has_escape, st, dev, false);
     if (rc != EP_OK) return rc;
     EP_CUDA(cudaMemcpy2DAsync(out->data, size_t(out->row_stride) * es, d.stage_out, size_t(L.cols) * es,
                               size_t(L.cols) * es, size_t(L.rows), cudaMemcpyDeviceToHost, st),
@@ -999,7 +1027,7 @@ extern "C" int ep_decode_fields(const ep_blob* cb, int16_t* fields, void* stream
     if (rc != EP_OK) return rc;
     const DeviceCopy& d = b->dev[dev];
     Params p = make_params(b, d.blob, d.tables, fields, b->layout.cols, d.status, false);
-    return launch(p, kOutFields, false, b->layout.max_tile_bytes, st, dev, false);
+    return launch(p, kOutFields, false, b->layout.max_tile_bytes, true, st, dev, false);
 }
 
 extern "C" int ep_decode_status(const ep_blob* cb, void* stream) {
@@ -1088,7 +1116,7 @@ extern "C" int ep_decompress_noalloc(const ep_blob* cb, const void* device_blob,
     const bool vec = vec_ok(L, out->data, out->row_stride, out->dtype);
     Params p = make_params(cb, static_cast<const uint8_t*>(device_blob), nullptr, out->data, out->row_stride,
                            status, vec);
-    int rc = noalloc_launch(p, kind, vec, st, dev);
+    int rc = noalloc_launch(p, kind, vec, L.has_escape, st, dev);
     if (rc != EP_OK || !wait) return rc;
     uint32_t s = 0;
     if (cudaMemcpyAsync(&s, status, sizeof s, cudaMemcpyDeviceToHost, st) != cudaSuccess ||

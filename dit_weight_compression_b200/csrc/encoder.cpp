@@ -539,12 +539,8 @@ bool parse_blob(const uint8_t* d, size_t n, BlobLayout& L, std::string& why) {
         for (int i = 0; i < L.n[c]; ++i) sum += rd16(d + L.q_offset[c] + 2 * i);
         if (sum != 0 && sum != kProbTotal) return fail("field table does not sum to 1024");
     }
-    for (int64_t r = 0; r < L.rows; ++r) {
-        uint32_t ab = rd32(d + L.off_alpha + 4 * r);
-        float a;
-        std::memcpy(&a, &ab, 4);
-        if (a != 0.0f && std::fabs(a) < 0x1p-125f) L.tiny_alpha = 1;
-    }
+    for (int c = 0; c < kFieldContexts; ++c)
+        if (L.esc_q[c]) L.has_escape = 1;
     const uint8_t* off = d + L.off_offsets;
     uint64_t stream = n - L.off_stream, prev = 0;
     if (rd32(off) != 0) return fail("first tile offset is not 0");

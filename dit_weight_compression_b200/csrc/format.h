@@ -60,7 +60,7 @@ struct BlobLayout {
     int64_t rows = 0, cols = 0, vec_per_row = 0, n_vectors = 0;
     uint32_t steps = 0, n_tiles = 0;
     uint64_t max_tile_bytes = 0;  // largest tile (selects the decoder's shared-memory layout)
-    int tiny_alpha = 0;           // a row scale with 0 < |alpha| < 2^-125 (alpha / 2 would round)
+    int has_escape = 0;           // some field context gives the escape symbol a frequency
     double scale = 0.0;
     uint64_t total = 0, off_tables = 0, off_alpha = 0, off_offsets = 0, off_stream = 0;
     uint16_t q_coset[2] = {0, 0};
