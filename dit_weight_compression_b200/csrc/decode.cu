@@ -101,13 +101,14 @@ struct Params {
 };
 
 constexpr uint32_t kSmemOptin = 232448;  // 227 KB: the largest dynamic shared memory of one CTA
+constexpr uint32_t kAlignSlack = 4096;    // the table starts on a 4 KB boundary of the shared window
 constexpr uint32_t kBufSlack = 80;        // bytes after a tile buffer that two steps may over-read
 
 // Per-warp tile buffer size for a CTA of WARPS warps: what the 227 KB leave after the table.
 template <int WARPS>
 struct Geo {
     static constexpr uint32_t kBuf =
-        ((kSmemOptin - kTableBytes - 64 - WARPS * (kBufSlack + 8) - 8) / WARPS) & ~15u;
+        ((kSmemOptin - kAlignSlack - kTableBytes - 64 - WARPS * (kBufSlack + 8) - 8) / WARPS) & ~15u;
 };
 
 template <int WARPS>
@@ -118,7 +119,8 @@ struct Smem {
     unsigned long long tbar;                                        // the table's bulk copies
 };
 static_assert(offsetof(Smem<32>, tbuf) == kTableBytes, "table block must be contiguous");
-static_assert(sizeof(Smem<32>) <= kSmemOptin && sizeof(Smem<16>) <= kSmemOptin, "shared memory budget");
+static_assert(sizeof(Smem<32>) + kAlignSlack <= kSmemOptin && sizeof(Smem<16>) + kAlignSlack <= kSmemOptin,
+              "shared memory budget");
 
 // Scratch of the table expansion: frequencies and cumulative frequencies of every context.
 struct BuildScratch {
@@ -432,7 +434,7 @@ __device__ __forceinline__ void decode_step(const Params& p, uint32_t tab, Reade
     uint32_t e[8], acc = 0;
 #define EP_FIELD(j)                                                                    \
     {                                                                                  \
-        const uint32_t ent = lds_u32<(j) * kCtxBytes>(tb + ((x & kSlotMask) << 2));    \
+        const uint32_t ent = lds_u32<(j) * kCtxBytes>(((x << 2) & (kSlotMask << 2)) | tb); \
         if (active) x = (ent >> kEntryQShift) * (x >> kProbBits) + (ent & kEntryBiasMask); \
         renorm_step<FULL>(x, rd, active);                                              \
         e[j] = ent;                                                                    \
@@ -547,11 +549,20 @@ __device__ __forceinline__ uint32_t decode_tile_steps(const Params& p, uint32_t 
     return 0;
 }
 
+// The CTA's layout inside its dynamic shared memory: shifted so that the table (and so every
+// context's 4 KB sub-table) starts on a 4 KB boundary of the shared window, which makes a
+// table address one OR of the slot into the sub-table's base.
+template <int WARPS>
+__device__ __forceinline__ Smem<WARPS>& smem_layout(uint8_t* raw) {
+    const uint32_t pad = (kAlignSlack - (smem_u32(raw) & (kAlignSlack - 1))) & (kAlignSlack - 1);
+    return *reinterpret_cast<Smem<WARPS>*>(raw + pad);
+}
+
 // BUILD = false: stage the pre-expanded table block from p.tables; true: expand it in each CTA.
 template <int WARPS, int OUT, bool VEC, bool BUILD, bool ESC>
 __global__ void __launch_bounds__(WARPS * 32, 1) decode_kernel(const Params p) {
     extern __shared__ __align__(128) uint8_t smem_raw[];
-    Smem<WARPS>& sm = *reinterpret_cast<Smem<WARPS>*>(smem_raw);
+    Smem<WARPS>& sm = smem_layout<WARPS>(smem_raw);
     constexpr uint32_t kBuf = Geo<WARPS>::kBuf;
     const uint32_t lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
     const bool fwd = (lane & 1) == 0;  // lanes 2p read forward, lanes 2p+1 backward
@@ -571,7 +582,7 @@ __global__ void __launch_bounds__(WARPS * 32, 1) decode_kernel(const Params p) {
     if (!BUILD && threadIdx.x == 0) {
         mbar_expect_tx(&sm.tbar, kTableBytes);
         for (uint32_t o = 0; o < kTableBytes; o += kTablePiece)
-            bulk_g2s(smem_raw + o, p.tables + o, kTablePiece, &sm.tbar);
+            bulk_g2s(reinterpret_cast<uint8_t*>(&sm.tab[0][0]) + o, p.tables + o, kTablePiece, &sm.tbar);
     }
 
     const uint32_t tile_stride = gridDim.x * WARPS;
@@ -711,8 +722,8 @@ __global__ void __launch_bounds__(WARPS * 32, 1) expand_tables_kernel(const Para
 }
 
 // ---- host-side launch -------------------------------------------------------------------------
-// 32 warps per CTA when every tile fits a 5 KB buffer (more tiles in flight per SM), else 16
-// warps with 10 KB buffers; a tile larger than that is read from global memory.
+// CTA widths: 32 warps with 4992-byte tile buffers, or 16 warps with 10080-byte buffers; a tile
+// larger than its warp's buffer is read from global memory.
 constexpr int kWarpsWide = 32, kWarpsNarrow = 16;
 
 struct DevInfo {
@@ -725,7 +736,7 @@ DevInfo g_dev[kMaxDevices];
 template <int WARPS, int OUT, bool VEC, bool ESC>
 int launch_one(const Params& p, cudaStream_t st, int device, bool dependent) {
     auto fn = decode_kernel<WARPS, OUT, VEC, false, ESC>;
-    const size_t smem = sizeof(Smem<WARPS>);
+    const size_t smem = sizeof(Smem<WARPS>) + kAlignSlack;
     static std::mutex mu;
     static int per_sm[kMaxDevices] = {};
     {
@@ -776,7 +787,9 @@ int launch_out(const Params& p, bool vec, bool wide, bool esc, cudaStream_t st, 
 // esc: the blob's tables give the escape symbol a frequency (else the escape-free kernel runs).
 int launch(const Params& p, int out_kind, bool vec, uint64_t max_tile, bool esc, cudaStream_t st, int device,
            bool dependent) {
-    const bool wide = max_tile <= Geo<kWarpsWide>::kBuf;
+    // 32 warps only when there are more tiles than 16 warps per SM can hold at once (the 16-warp
+    // kernel has twice the registers per thread) and every tile fits the smaller buffer
+    const bool wide = max_tile <= Geo<kWarpsWide>::kBuf && p.n_tiles > uint32_t(kWarpsNarrow) * g_dev[device].sms;
     switch (out_kind) {
         case kOutBF16: return launch_out<kOutBF16>(p, vec, wide, esc, st, device, dependent);
         case kOutFP16: return launch_out<kOutFP16>(p, vec, wide, esc, st, device, dependent);
@@ -893,7 +906,7 @@ std::mutex g_noalloc_mu;
 template <int WARPS, int OUT, bool VEC, bool ESC>
 int noalloc_launch_one(const Params& p, cudaStream_t st, int device) {
     auto fn = decode_kernel<WARPS, OUT, VEC, true, ESC>;
-    const size_t smem = sizeof(Smem<WARPS>);
+    const size_t smem = sizeof(Smem<WARPS>) + kAlignSlack;
     static std::mutex mu;
     static int per_sm[kMaxDevices] = {};
     {
