@@ -415,6 +415,14 @@ __device__ __forceinline__ void advance(const Params& p, Pos& s) {
     }
 }
 
+// How a lane's output position moves from step to step.
+//   kWalkRows32: rows hold a multiple of 32 vectors (and every vector is one aligned store), so the
+//                32 lanes of a warp change rows at the same step: the steps of a tile run row by
+//                row, with nothing but the output pointer moving inside a row;
+//   kWalkWide:   rows of at least 32 vectors: a step crosses at most one row end;
+//   kWalkNarrow: shorter rows.
+enum Walk { kWalkRows32 = 0, kWalkWide = 1, kWalkNarrow = 2 };
+
 // ESC: the blob's tables give the escape symbol a frequency, so a field may be a raw word.
 template <int OUT, bool VEC, bool ESC, bool FULL, class Reader>
 __device__ __forceinline__ void decode_step(const Params& p, uint32_t tab, Reader& rd, uint32_t& x, bool active,
@@ -508,25 +516,57 @@ __device__ __forceinline__ void decode_step(const Params& p, uint32_t tab, Reade
     }
 }
 
-// Decode the full steps of a tile, two between runaway checks (the tile buffer's slack covers
-// what two steps may read past a checked position).
-template <int OUT, bool VEC, bool ESC, bool WIDE, class Reader, class Guard>
-__device__ __forceinline__ uint32_t full_steps(const Params& p, uint32_t tab, Reader& rd, uint32_t& x, Pos& pos,
-                                               uint32_t nfull, Guard in_range) {
+// Decode `n` full steps, two between runaway checks (the tile buffer's slack covers what two
+// steps may read past a checked position), moving the output position by `walk` after each.
+template <int OUT, bool VEC, bool ESC, class Reader, class Guard, class Step>
+__device__ __forceinline__ uint32_t full_run(const Params& p, uint32_t tab, Reader& rd, uint32_t& x, Pos& pos,
+                                             uint32_t n, Guard in_range, Step walk) {
     uint32_t k = 0;
-    for (; k + 2 <= nfull; k += 2) {
+    for (; k + 2 <= n; k += 2) {
         if (!__all_sync(kFull, in_range(rd))) return kStOverrun;  // a corrupt tile ran away
         decode_step<OUT, VEC, ESC, true>(p, tab, rd, x, true, pos);
-        advance<OUT, WIDE>(p, pos);
+        walk(pos);
         decode_step<OUT, VEC, ESC, true>(p, tab, rd, x, true, pos);
-        advance<OUT, WIDE>(p, pos);
+        walk(pos);
     }
-    if (k < nfull) {
+    if (k < n) {
         if (!__all_sync(kFull, in_range(rd))) return kStOverrun;
         decode_step<OUT, VEC, ESC, true>(p, tab, rd, x, true, pos);
-        advance<OUT, WIDE>(p, pos);
+        walk(pos);
     }
     return 0;
+}
+
+template <int OUT, bool VEC, bool ESC, int WALK, class Reader, class Guard>
+__device__ __forceinline__ uint32_t full_steps(const Params& p, uint32_t tab, Reader& rd, uint32_t& x, Pos& pos,
+                                               uint32_t nfull, Guard in_range) {
+    if constexpr (OUT == kOutFields) {
+        return full_run<OUT, VEC, ESC>(p, tab, rd, x, pos, nfull, in_range, [](Pos& s) { s.optr += 32 * 18; });
+    } else if constexpr (WALK == kWalkRows32) {
+        constexpr int es = OutElem<OUT>::kBytes;
+        const uint32_t per_row = p.vec_per_row / kLanes;
+        const int64_t wrap = (p.row_stride - 8 * int64_t(p.vec_per_row)) * es;
+        uint32_t left = (p.vec_per_row - pos.kcol + kLanes - 1) / kLanes;  // the same for all 32 lanes
+        for (uint32_t k = 0; k < nfull;) {
+            const uint32_t n = min(left, nfull - k);
+            const float a_next = pos.row + 1 < p.rows ? __ldg(p.alpha + pos.row + 1) : 0.0f;
+            const uint32_t st =
+                full_run<OUT, VEC, ESC>(p, tab, rd, x, pos, n, in_range, [](Pos& s) { s.optr += 32 * 8 * es; });
+            if (st) return st;
+            k += n;
+            left -= n;
+            if (left == 0) {  // the warp moves to the next row
+                left = per_row;
+                pos.optr += wrap;
+                ++pos.row;
+                pos.a = a_next;
+            }
+        }
+        return 0;
+    } else {
+        return full_run<OUT, VEC, ESC>(p, tab, rd, x, pos, nfull, in_range,
+                                       [&p](Pos& s) { advance<OUT, WALK == kWalkWide>(p, s); });
+    }
 }
 
 // Decode the steps of one tile with a given word reader; returns the status flags of the tile.
@@ -538,9 +578,14 @@ __device__ __forceinline__ uint32_t decode_tile_steps(const Params& p, uint32_t 
     const uint32_t nv = uint32_t(min(per_tile, p.n_vectors - v0));
     const uint32_t nfull = nv / kLanes, rem = nv % kLanes;
     Pos pos = first_pos<OUT>(p, v0 + lane);
-    const uint32_t st = p.vec_per_row >= uint32_t(kLanes)
-                            ? full_steps<OUT, VEC, ESC, true>(p, tab, rd, x, pos, nfull, in_range)
-                            : full_steps<OUT, VEC, ESC, false>(p, tab, rd, x, pos, nfull, in_range);
+    uint32_t st;
+    if (VEC && OUT != kOutFields && p.vec_per_row % kLanes == 0)
+        st = full_steps<OUT, VEC, ESC, (VEC && OUT != kOutFields) ? kWalkRows32 : kWalkWide>(p, tab, rd, x, pos, nfull,
+                                                                                            in_range);
+    else if (p.vec_per_row >= uint32_t(kLanes))
+        st = full_steps<OUT, VEC, ESC, kWalkWide>(p, tab, rd, x, pos, nfull, in_range);
+    else
+        st = full_steps<OUT, VEC, ESC, kWalkNarrow>(p, tab, rd, x, pos, nfull, in_range);
     if (st) return st;
     if (rem) {
         if (!__all_sync(kFull, in_range(rd))) return kStOverrun;
