@@ -53,6 +53,7 @@ SIGNATURES = {
     "ep_compress": (_I, [ctypes.POINTER(EpTensor), _D, ctypes.POINTER(_P)]),
     "ep_compress_ex": (_I, [ctypes.POINTER(EpTensor), _D, ctypes.POINTER(EpOptions), ctypes.POINTER(_P)]),
     "ep_decompress": (_I, [_P, ctypes.POINTER(EpTensor), _P]),
+    "ep_decompress_group": (_I, [ctypes.POINTER(_P), ctypes.POINTER(EpTensor), _I, _P]),
     "ep_actual_bpp": (_D, [_P]),
     "ep_get_info": (_I, [_P, ctypes.POINTER(EpBlobInfo)]),
     "ep_blob_to_bytes": (_I, [_P, ctypes.POINTER(_P), ctypes.POINTER(_SZ)]),
@@ -216,6 +217,30 @@ def decompress(compressed: CompressedTensor, config=None, *, out: torch.Tensor |
     return out
 
 
+def decompress_group(compressed: list, *, outs: list | None = None, dtype: torch.dtype | None = None,
+                     device=None, stream=None) -> list:
+    """Decode several blobs (e.g. one block's linear layers) with ep_decompress_group: one kernel
+    launch per 32 blobs, results bit-identical to decompress().  Outputs are CUDA tensors of one
+    dtype (the first blob's unless `dtype` or `outs` say otherwise), written asynchronously."""
+    n = len(compressed)
+    if outs is None:
+        dev = torch.device("cuda", torch.cuda.current_device()) if device is None else torch.device(device)
+        dt = dtype or (compressed[0].dtype if n else torch.bfloat16)
+        outs = [torch.empty(c.shape, dtype=dt, device=dev) for c in compressed]
+    if len(outs) != n:
+        raise ValueError("decompress_group: one output per blob")
+    if n == 0:
+        return outs
+    handles = (_P * n)(*[c.handle.value for c in compressed])
+    views = (EpTensor * n)(*[tensor_view(o) for o in outs])
+    if outs[0].is_cuda:
+        with torch.cuda.device(outs[0].device):
+            _check(lib().ep_decompress_group(handles, views, n, _stream_handle(stream)), "ep_decompress_group")
+    else:  # rejected by the library (device outputs only)
+        _check(lib().ep_decompress_group(handles, views, n, _stream_handle(stream)), "ep_decompress_group")
+    return outs
+
+
 def decode_status(compressed: CompressedTensor, stream=None) -> None:
     """Raise EPError if any decode of this blob on the current device found corrupt tiles."""
     _check(lib().ep_decode_status(compressed.handle, _stream_handle(stream)), "ep_decode_status")
@@ -229,5 +254,5 @@ def decode_fields(compressed: CompressedTensor, stream=None) -> torch.Tensor:
     return out
 
 
-__all__ = ["LatticeRANSConfig", "CompressedTensor", "compress", "decompress", "decode_status",
+__all__ = ["LatticeRANSConfig", "CompressedTensor", "compress", "decompress", "decompress_group", "decode_status",
            "decode_fields", "EPError", "lib", "BF16", "FP16", "FP8_E4M3", "F32"]

@@ -39,6 +39,7 @@
 #include <type_traits>
 #include <cstdio>
 #include <mutex>
+#include <vector>
 
 #include "blob.h"
 
@@ -82,8 +83,9 @@ enum : uint32_t {
     kStTimeout = 8u    // a bulk-copy wait hit its limit
 };
 
+// What the decode of one blob needs (small: a grouped launch passes up to kMaxGroup of them as
+// its kernel parameter).
 struct Params {
-    const uint8_t* blob;        // device copy of the serialised blob
     const uint8_t* tables;      // expanded decode table (kTableBytes), or null: expand in-kernel
     const uint32_t* tile_off;   // n_tiles + 1 offsets, 16-byte units
     const uint8_t* stream;      // stream section
@@ -94,6 +96,11 @@ struct Params {
     uint32_t vec_per_row;       // < 2^31 (checked when the blob is parsed)
     uint32_t steps, n_tiles;
     uint32_t q_coset0;          // frequency of coset 0; coset 1 has M - q_coset0
+};
+
+// Where the blob keeps the compact frequency tables the decode table is expanded from.
+struct TableSrc {
+    const uint8_t* blob;        // device copy of the serialised blob
     uint32_t q_off[kFieldContexts];
     uint32_t esc_q[kFieldContexts];
     uint32_t lo[kFieldContexts];
@@ -249,7 +256,7 @@ __device__ __forceinline__ void renorm_step(uint32_t& x, Reader& rd, bool active
 // Fills tab[16][1024] from the blob's compact frequency tables.  `scr` is shared-memory scratch
 // (BuildScratch) that the caller does not use meanwhile.
 template <int WARPS>
-__device__ void build_tables(uint32_t (*tab)[kProbTotal], BuildScratch& scr, const Params& p) {
+__device__ void build_tables(uint32_t (*tab)[kProbTotal], BuildScratch& scr, const TableSrc& p) {
     const uint32_t lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
     // (a) per context: frequencies of symbols 8*lane .. 8*lane+7 and their cumulative sums
     for (uint32_t ctx = warp; ctx < kFieldContexts; ctx += WARPS) {
@@ -603,10 +610,11 @@ __device__ __forceinline__ Smem<WARPS>& smem_layout(uint8_t* raw) {
     return *reinterpret_cast<Smem<WARPS>*>(raw + pad);
 }
 
-// BUILD = false: stage the pre-expanded table block from p.tables; true: expand it in each CTA.
+// The work of CTA `cta` of the `ncta` CTAs that decode one blob.
+// BUILD = false: stage the pre-expanded table from p.tables; true: expand it from `ts` in each CTA.
 template <int WARPS, int OUT, bool VEC, bool BUILD, bool ESC>
-__global__ void __launch_bounds__(WARPS * 32, 1) decode_kernel(const Params p) {
-    extern __shared__ __align__(128) uint8_t smem_raw[];
+__device__ __forceinline__ void decode_ctas(const Params& p, const TableSrc* ts, uint8_t* smem_raw, uint32_t cta,
+                                            uint32_t ncta) {
     Smem<WARPS>& sm = smem_layout<WARPS>(smem_raw);
     constexpr uint32_t kBuf = Geo<WARPS>::kBuf;
     const uint32_t lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
@@ -630,8 +638,8 @@ __global__ void __launch_bounds__(WARPS * 32, 1) decode_kernel(const Params p) {
             bulk_g2s(reinterpret_cast<uint8_t*>(&sm.tab[0][0]) + o, p.tables + o, kTablePiece, &sm.tbar);
     }
 
-    const uint32_t tile_stride = gridDim.x * WARPS;
-    uint32_t tile = blockIdx.x + gridDim.x * warp;
+    const uint32_t tile_stride = ncta * WARPS;
+    uint32_t tile = cta + ncta * warp;
     uint32_t staged = 0;  // tiles this warp has staged: its barrier's phase parity
 
     // Stage a tile that fits the buffer (one bulk copy), and ask L2 for the warp's next tile.
@@ -652,7 +660,7 @@ __global__ void __launch_bounds__(WARPS * 32, 1) decode_kernel(const Params p) {
     uint64_t t0 = 0;
     uint32_t tbytes = 0;
     if (BUILD) {  // expand the table first: its scratch lies in the tile buffers
-        build_tables<WARPS>(sm.tab, *reinterpret_cast<BuildScratch*>(&sm.tbuf[0][0]), p);
+        build_tables<WARPS>(sm.tab, *reinterpret_cast<BuildScratch*>(&sm.tbuf[0][0]), *ts);
         __syncthreads();
     }
     if (tile < p.n_tiles) {  // the first tile's fetch overlaps the table staging
@@ -749,6 +757,45 @@ drain:
     if (tile < p.n_tiles && tbytes <= kBuf) mbar_wait(&sm.bar[warp], 0);
 }
 
+// One blob over the whole grid.
+template <int WARPS, int OUT, bool VEC, bool BUILD, bool ESC>
+__global__ void __launch_bounds__(WARPS * 32, 1) decode_kernel(const __grid_constant__ Params p,
+                                                               const __grid_constant__ TableSrc ts) {
+    extern __shared__ __align__(128) uint8_t smem_raw[];
+    decode_ctas<WARPS, OUT, VEC, BUILD, ESC>(p, &ts, smem_raw, blockIdx.x, gridDim.x);
+}
+
+// A set of blobs in one launch: blob m owns CTAs [cta0, cta0 + ncta) and stages only its own
+// table.  Every blob picks its store and escape variant.
+constexpr int kMaxGroup = 32;
+struct GroupEntry {
+    Params p;
+    uint32_t cta0, ncta;
+    uint32_t vec, esc;
+};
+struct GroupParams {
+    uint32_t n;
+    GroupEntry e[kMaxGroup];
+};
+static_assert(sizeof(GroupParams) <= 4000, "a group must fit the kernel parameter space");
+
+template <int WARPS, int OUT>
+__global__ void __launch_bounds__(WARPS * 32, 1) group_kernel(const __grid_constant__ GroupParams g) {
+    extern __shared__ __align__(128) uint8_t smem_raw[];
+    uint32_t m = 0;
+    while (m + 1 < g.n && blockIdx.x >= g.e[m + 1].cta0) ++m;
+    const GroupEntry& e = g.e[m];
+    if (blockIdx.x >= e.cta0 + e.ncta) return;  // a CTA beyond the last blob's share
+    const uint32_t cta = blockIdx.x - e.cta0;
+    if (e.vec) {
+        if (e.esc) decode_ctas<WARPS, OUT, true, false, true>(e.p, nullptr, smem_raw, cta, e.ncta);
+        else decode_ctas<WARPS, OUT, true, false, false>(e.p, nullptr, smem_raw, cta, e.ncta);
+    } else {
+        if (e.esc) decode_ctas<WARPS, OUT, false, false, true>(e.p, nullptr, smem_raw, cta, e.ncta);
+        else decode_ctas<WARPS, OUT, false, false, false>(e.p, nullptr, smem_raw, cta, e.ncta);
+    }
+}
+
 // Expands the blob's compact frequency tables into the 64 KB packed decode table (one CTA).
 struct ExpandSmem {
     uint32_t tab[kFieldContexts][kProbTotal];
@@ -756,7 +803,8 @@ struct ExpandSmem {
 };
 
 template <int WARPS>
-__global__ void __launch_bounds__(WARPS * 32, 1) expand_tables_kernel(const Params p, uint8_t* tables) {
+__global__ void __launch_bounds__(WARPS * 32, 1) expand_tables_kernel(const __grid_constant__ TableSrc p,
+                                                                       uint8_t* tables) {
     extern __shared__ __align__(128) uint8_t smem_raw[];
     ExpandSmem& sm = *reinterpret_cast<ExpandSmem*>(smem_raw);
     build_tables<WARPS>(sm.tab, sm.scratch, p);
@@ -808,7 +856,8 @@ int launch_one(const Params& p, cudaStream_t st, int device, bool dependent) {
     attr[0].val.programmaticStreamSerializationAllowed = 1;
     cfg.attrs = attr;
     cfg.numAttrs = dependent ? 1 : 0;
-    cudaError_t e = cudaLaunchKernelEx(&cfg, fn, p);
+    const TableSrc none = {};  // the table is pre-expanded
+    cudaError_t e = cudaLaunchKernelEx(&cfg, fn, p, none);
     if (e == cudaSuccess) e = cudaGetLastError();
     if (e != cudaSuccess) return set_error(EP_ERR_CUDA, std::string("decode launch: ") + cudaGetErrorString(e));
     return EP_OK;
@@ -845,6 +894,60 @@ int launch(const Params& p, int out_kind, bool vec, uint64_t max_tile, bool esc,
     }
 }
 
+// ---- grouped launch (ep_decompress_group) ----------------------------------------------------
+template <int WARPS, int OUT>
+int group_launch_one(const GroupParams& g, uint32_t grid, cudaStream_t st, int device) {
+    auto fn = group_kernel<WARPS, OUT>;
+    const size_t smem = sizeof(Smem<WARPS>) + kAlignSlack;
+    static std::mutex mu;
+    static bool ready[kMaxDevices] = {};
+    {
+        std::lock_guard<std::mutex> lk(mu);
+        if (!ready[device]) {
+            cudaError_t e = cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, int(smem));
+            if (e != cudaSuccess)
+                return set_error(EP_ERR_CUDA, std::string("group kernel attribute: ") + cudaGetErrorString(e));
+            ready[device] = true;
+        }
+    }
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(grid);
+    cfg.blockDim = dim3(WARPS * 32);
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = st;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    cudaError_t e = cudaLaunchKernelEx(&cfg, fn, g);
+    if (e == cudaSuccess) e = cudaGetLastError();
+    if (e != cudaSuccess) return set_error(EP_ERR_CUDA, std::string("group launch: ") + cudaGetErrorString(e));
+    return EP_OK;
+}
+
+template <int OUT>
+int group_launch_out(const GroupParams& g, uint32_t grid, bool wide, cudaStream_t st, int device) {
+    return wide ? group_launch_one<kWarpsWide, OUT>(g, grid, st, device)
+                : group_launch_one<kWarpsNarrow, OUT>(g, grid, st, device);
+}
+
+// Share `ctas` CTAs among blobs with tiles[i] tiles: every blob gets one, then each further CTA
+// goes to the blob with the most tiles per CTA (lowest index on ties), never more CTAs than tiles.
+std::vector<uint32_t> share_ctas(const std::vector<uint32_t>& tiles, uint32_t ctas) {
+    std::vector<uint32_t> g(tiles.size(), 1);
+    for (uint32_t left = ctas > tiles.size() ? ctas - uint32_t(tiles.size()) : 0; left; --left) {
+        int best = -1;
+        for (size_t i = 0; i < tiles.size(); ++i) {
+            if (g[i] >= tiles[i]) continue;
+            if (best < 0 || uint64_t(tiles[i]) * g[best] > uint64_t(tiles[best]) * g[i]) best = int(i);
+        }
+        if (best < 0) break;
+        ++g[best];
+    }
+    return g;
+}
+
 int out_kind_of(int dtype) {
     switch (dtype) {
         case kBF16: return kOutBF16;
@@ -876,7 +979,6 @@ Params make_params(const ep_blob* b, const uint8_t* dblob, const uint8_t* tables
                    uint32_t* status, bool vec) {
     const BlobLayout& L = b->layout;
     Params p;
-    p.blob = dblob;
     p.tables = tables;
     p.tile_off = reinterpret_cast<const uint32_t*>(dblob + L.off_offsets);
     p.stream = dblob + L.off_stream;
@@ -891,13 +993,20 @@ Params make_params(const ep_blob* b, const uint8_t* dblob, const uint8_t* tables
     p.steps = L.steps;
     p.n_tiles = L.n_tiles;
     p.q_coset0 = L.q_coset[0];
-    for (int c = 0; c < kFieldContexts; ++c) {
-        p.q_off[c] = L.q_offset[c];
-        p.esc_q[c] = L.esc_q[c];
-        p.lo[c] = L.lo[c];
-        p.n[c] = L.n[c];
-    }
     return p;
+}
+
+TableSrc make_tablesrc(const ep_blob* b, const uint8_t* dblob) {
+    const BlobLayout& L = b->layout;
+    TableSrc t;
+    t.blob = dblob;
+    for (int c = 0; c < kFieldContexts; ++c) {
+        t.q_off[c] = L.q_offset[c];
+        t.esc_q[c] = L.esc_q[c];
+        t.lo[c] = L.lo[c];
+        t.n[c] = L.n[c];
+    }
+    return t;
 }
 
 // Device copy of the blob and its status word on `dev` (allocated and filled on first use).
@@ -917,11 +1026,11 @@ int ensure_device(ep_blob* b, int dev, cudaStream_t st) {
     EP_CUDA(cudaMemcpyAsync(blob, b->bytes.data(), b->bytes.size(), cudaMemcpyHostToDevice, st), "blob upload");
     EP_CUDA(cudaMemsetAsync(status, 0, 16, st), "status clear");
     // expand the compact frequency tables once for this device copy
-    Params p = make_params(b, blob, nullptr, nullptr, b->layout.cols, status, false);
+    const TableSrc ts = make_tablesrc(b, blob);
     auto fn = expand_tables_kernel<kWarpsWide>;
     EP_CUDA(cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, int(sizeof(ExpandSmem))),
             "table expansion attribute");
-    fn<<<1, kWarpsWide * 32, sizeof(ExpandSmem), st>>>(p, tables);
+    fn<<<1, kWarpsWide * 32, sizeof(ExpandSmem), st>>>(ts, tables);
     EP_CUDA(cudaGetLastError(), "table expansion launch");
     EP_CUDA(cudaStreamSynchronize(st), "blob upload");
     d.blob = blob;
@@ -949,7 +1058,7 @@ NoallocDevice g_noalloc[kMaxDevices];
 std::mutex g_noalloc_mu;
 
 template <int WARPS, int OUT, bool VEC, bool ESC>
-int noalloc_launch_one(const Params& p, cudaStream_t st, int device) {
+int noalloc_launch_one(const Params& p, const TableSrc& ts, cudaStream_t st, int device) {
     auto fn = decode_kernel<WARPS, OUT, VEC, true, ESC>;
     const size_t smem = sizeof(Smem<WARPS>) + kAlignSlack;
     static std::mutex mu;
@@ -966,27 +1075,28 @@ int noalloc_launch_one(const Params& p, cudaStream_t st, int device) {
         }
     }
     const uint32_t grid = uint32_t(std::min<int64_t>(int64_t(g_noalloc[device].sms) * per_sm[device], p.n_tiles));
-    fn<<<grid, WARPS * 32, smem, st>>>(p);
+    fn<<<grid, WARPS * 32, smem, st>>>(p, ts);
     if (cudaGetLastError() != cudaSuccess)
         return set_error_static(EP_ERR_CUDA, "ep_decompress_noalloc: kernel launch failed");
     return EP_OK;
 }
 
 template <int OUT>
-int noalloc_launch_out(const Params& p, bool vec, bool esc, cudaStream_t st, int device) {
+int noalloc_launch_out(const Params& p, const TableSrc& ts, bool vec, bool esc, cudaStream_t st, int device) {
     if (esc)
-        return vec ? noalloc_launch_one<kWarpsNarrow, OUT, true, true>(p, st, device)
-                   : noalloc_launch_one<kWarpsNarrow, OUT, false, true>(p, st, device);
-    return vec ? noalloc_launch_one<kWarpsNarrow, OUT, true, false>(p, st, device)
-               : noalloc_launch_one<kWarpsNarrow, OUT, false, false>(p, st, device);
+        return vec ? noalloc_launch_one<kWarpsNarrow, OUT, true, true>(p, ts, st, device)
+                   : noalloc_launch_one<kWarpsNarrow, OUT, false, true>(p, ts, st, device);
+    return vec ? noalloc_launch_one<kWarpsNarrow, OUT, true, false>(p, ts, st, device)
+               : noalloc_launch_one<kWarpsNarrow, OUT, false, false>(p, ts, st, device);
 }
 
-int noalloc_launch(const Params& p, int out_kind, bool vec, bool esc, cudaStream_t st, int device) {
+int noalloc_launch(const Params& p, const TableSrc& ts, int out_kind, bool vec, bool esc, cudaStream_t st,
+                   int device) {
     switch (out_kind) {
-        case kOutBF16: return noalloc_launch_out<kOutBF16>(p, vec, esc, st, device);
-        case kOutFP16: return noalloc_launch_out<kOutFP16>(p, vec, esc, st, device);
-        case kOutE4M3: return noalloc_launch_out<kOutE4M3>(p, vec, esc, st, device);
-        default: return noalloc_launch_out<kOutF32>(p, vec, esc, st, device);
+        case kOutBF16: return noalloc_launch_out<kOutBF16>(p, ts, vec, esc, st, device);
+        case kOutFP16: return noalloc_launch_out<kOutFP16>(p, ts, vec, esc, st, device);
+        case kOutE4M3: return noalloc_launch_out<kOutE4M3>(p, ts, vec, esc, st, device);
+        default: return noalloc_launch_out<kOutF32>(p, ts, vec, esc, st, device);
     }
 }
 
@@ -1071,6 +1181,73 @@ extern "C" int ep_decompress(const ep_blob* cb, const ep_tensor* out, void* stre
                               size_t(L.cols) * es, size_t(L.rows), cudaMemcpyDeviceToHost, st),
             "ep_decompress: download");
     EP_CUDA(cudaStreamSynchronize(st), "ep_decompress: synchronise");
+    return EP_OK;
+}
+
+extern "C" int ep_decompress_group(const ep_blob* const* blobs, const ep_tensor* outs, int n, void* stream) {
+    clear_error();
+    if (n == 0) return EP_OK;
+    if (n < 0 || !blobs || !outs) return set_error(EP_ERR_ARG, "ep_decompress_group: NULL argument or n < 0");
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    int dev = 0;
+    int rc = current_device(dev);
+    if (rc != EP_OK) return rc;
+    const int dtype = outs[0].dtype;
+    const int kind = out_kind_of(dtype);
+    if (kind < 0) return set_error(EP_ERR_DTYPE, "ep_decompress_group: unsupported output dtype");
+    for (int i = 0; i < n; ++i) {  // validate everything before launching anything
+        const ep_tensor& o = outs[i];
+        if (!blobs[i] || !o.data) return set_error(EP_ERR_ARG, "ep_decompress_group: NULL blob or output");
+        if (o.dtype != dtype) return set_error(EP_ERR_DTYPE, "ep_decompress_group: outputs differ in dtype");
+        if (o.device != dev)
+            return set_error(EP_ERR_ARG, "ep_decompress_group: outputs must be on the current device");
+        const BlobLayout& L = blobs[i]->layout;
+        if (o.rows != L.rows || o.cols != L.cols)
+            return set_error(EP_ERR_SHAPE, "ep_decompress_group: an output's shape differs from its blob's");
+        if (o.row_stride < o.cols) return set_error(EP_ERR_ARG, "ep_decompress_group: row_stride < cols");
+    }
+    for (int i = 0; i < n; ++i) {
+        rc = ensure_device(const_cast<ep_blob*>(blobs[i]), dev, st);
+        if (rc != EP_OK) return rc;
+    }
+    const int sms = g_dev[dev].sms;
+    const int chunk = std::max(1, std::min(kMaxGroup, sms));
+    for (int c0 = 0; c0 < n; c0 += chunk) {
+        const int cn = std::min(chunk, n - c0);
+        std::vector<uint32_t> tiles(static_cast<size_t>(cn));
+        uint64_t total = 0, max_tile = 0;
+        for (int i = 0; i < cn; ++i) {
+            const BlobLayout& L = blobs[c0 + i]->layout;
+            tiles[size_t(i)] = L.n_tiles;
+            total += L.n_tiles;
+            max_tile = std::max<uint64_t>(max_tile, L.max_tile_bytes);
+        }
+        const std::vector<uint32_t> g = share_ctas(tiles, uint32_t(sms));
+        GroupParams gp = {};
+        gp.n = uint32_t(cn);
+        uint32_t cta = 0;
+        for (int i = 0; i < cn; ++i) {
+            const ep_blob* b = blobs[c0 + i];
+            const ep_tensor& o = outs[c0 + i];
+            const DeviceCopy& d = b->dev[dev];
+            const bool vec = vec_ok(b->layout, o.data, o.row_stride, dtype);
+            GroupEntry& e = gp.e[i];
+            e.p = make_params(b, d.blob, d.tables, o.data, o.row_stride, d.status, vec);
+            e.cta0 = cta;
+            e.ncta = g[size_t(i)];
+            e.vec = vec ? 1u : 0u;
+            e.esc = b->layout.has_escape ? 1u : 0u;
+            cta += e.ncta;
+        }
+        const bool wide = max_tile <= Geo<kWarpsWide>::kBuf && total > uint64_t(kWarpsNarrow) * uint64_t(cta);
+        switch (kind) {
+            case kOutBF16: rc = group_launch_out<kOutBF16>(gp, cta, wide, st, dev); break;
+            case kOutFP16: rc = group_launch_out<kOutFP16>(gp, cta, wide, st, dev); break;
+            case kOutE4M3: rc = group_launch_out<kOutE4M3>(gp, cta, wide, st, dev); break;
+            default: rc = group_launch_out<kOutF32>(gp, cta, wide, st, dev); break;
+        }
+        if (rc != EP_OK) return rc;
+    }
     return EP_OK;
 }
 
@@ -1174,7 +1351,8 @@ extern "C" int ep_decompress_noalloc(const ep_blob* cb, const void* device_blob,
     const bool vec = vec_ok(L, out->data, out->row_stride, out->dtype);
     Params p = make_params(cb, static_cast<const uint8_t*>(device_blob), nullptr, out->data, out->row_stride,
                            status, vec);
-    int rc = noalloc_launch(p, kind, vec, L.has_escape, st, dev);
+    const TableSrc ts = make_tablesrc(cb, static_cast<const uint8_t*>(device_blob));
+    int rc = noalloc_launch(p, ts, kind, vec, L.has_escape, st, dev);
     if (rc != EP_OK || !wait) return rc;
     uint32_t s = 0;
     if (cudaMemcpyAsync(&s, status, sizeof s, cudaMemcpyDeviceToHost, st) != cudaSuccess ||

@@ -116,6 +116,26 @@ int ep_compress_ex(const ep_tensor* in, double target_bpp, const ep_options* opt
  */
 int ep_decompress(const ep_blob* b, const ep_tensor* out, void* stream);
 
+/*
+ * Decompress a set of blobs -- for example the linear layers of one transformer block, decoded
+ * just before they are used -- in as few kernel launches as possible: one per 32 blobs.  Each
+ * blob is decoded exactly as ep_decompress would decode it (same arithmetic, bit-identical
+ * results); the launch divides the GPU among the blobs in proportion to their tiles, so small
+ * matrices that would each leave most SMs idle share the GPU instead.  (The pages motivate it:
+ * the abstract names diffusion denoising and transformer prefill, where a whole block's weights
+ * are decoded online; the documentation's "Encoding and reconstruction" makes every tile
+ * independently decodable, which is what lets tiles of different blobs run side by side.)
+ *   blobs   n blob handles.
+ *   outs    n device tensors on the current device, outs[i] shaped like blobs[i]; all n with the
+ *           same dtype.  Host outputs are not accepted.
+ *   n       number of blobs; n == 0 does nothing.
+ *   stream  cudaStream_t as void*; asynchronous like ep_decompress on device outputs.
+ * The first call for a blob on a device copies it there (allocates and synchronises once).
+ * Corrupt tiles are reported per blob by ep_decode_status().  Returns EP_ERR_ARG, EP_ERR_SHAPE,
+ * EP_ERR_DTYPE, EP_ERR_CUDA, EP_ERR_OOM; nothing is launched when an argument is invalid.
+ */
+int ep_decompress_group(const ep_blob* const* blobs, const ep_tensor* outs, int n, void* stream);
+
 /* Stored bits per element: 8 * (stored bytes including metadata) / (rows * cols)
  * ("EntroPack lattice compression", section "Encoding and reconstruction": "The actual_bpp
  * property reports the actual stored bytes, including metadata, divided by the element count
