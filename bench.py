@@ -55,15 +55,36 @@ def parse_args():
     ap.add_argument("--e2e-steps", type=int, default=50)
     ap.add_argument("--cpu-seconds", type=float, default=10.0, help="CPU-baseline sample length")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--cpu-cores", type=int, default=0,
+                    help="also time the oracle tile-parallel on this many host cores (0 = all, 1 = skip)")
+    ap.add_argument("--workload", default="square",
+                    help="square (default) | small | dit-set | sweep:<bpp> | large")
+    ap.add_argument("--decode", choices=["grouped", "single"], default="grouped",
+                    help="for a set of matrices: one ep_decompress_group call per step, or one "
+                         "ep_decompress call per matrix")
     return ap.parse_args()
 
 
-def workload(steps_override: int = 0):
+def workload(name: str = "square"):
+    """The matrices one step decodes, and a description."""
     import workloads as W
-    m = W.square()
-    desc = ("square 4096x4096 BF16, row r i.i.d. N(0, sigma_r^2), sigma_r log-uniform in [0.005, 0.05], "
-            "target 4.0 bpp, output BF16")
-    return m, desc
+    if name == "square":
+        return [W.square()], ("square 4096x4096 BF16, row r i.i.d. N(0, sigma_r^2), sigma_r log-uniform in "
+                              "[0.005, 0.05], target 4.0 bpp, output BF16")
+    if name == "small":
+        return [W.small()], "small 256x256 BF16 N(0, 0.02^2), target 3.5 bpp, output BF16"
+    if name == "dit-set":
+        return ([W.dit(j) for j in range(len(W.DIT_SHAPES))],
+                "dit-set: a DiT block's linear layers (4 x 3072x3072, 3072x8192, 8192x3072) BF16, Student-t(5) "
+                "x 0.02/sqrt(5/3) with 1% of rows x10, target 2.5 bpp, output BF16")
+    if name.startswith("sweep:"):
+        rate = float(name.split(":", 1)[1])
+        return [W.sweep(rate)], f"sweep 4096x11008 FP16 N(0, 0.02^2), target {rate} bpp, output FP16"
+    if name == "large":
+        return ([W.large(j) for j in range(4)],
+                "large: 4 x 28672x8192 BF16, N(0, 0.015^2) x per-column scale log-uniform in [0.5, 2], "
+                "target 4.0 bpp, output BF16")
+    raise SystemExit(f"unknown workload {name!r}")
 
 
 # ---------------------------------------------------------------------------------------------
@@ -187,6 +208,56 @@ def cpu_oracle_rate(blob: bytes, seconds: float, max_tiles: int | None = None):
     return elems * 2 * reps / dt / 1e9, reps, n_tiles, dt
 
 
+_POOL_BLOB = None
+
+
+def _pool_init(blob: bytes):
+    global _POOL_BLOB
+    _POOL_BLOB = blob
+
+
+def _pool_decode(job):
+    """One worker's share: decode tiles [t0, t1) repeatedly for about `seconds`."""
+    import oracle
+    t0, t1, seconds = job
+    info = oracle.blob_info(_POOL_BLOB)
+    out = np.zeros((info["rows"], info["cols"]), np.uint16)
+    per = 32 * info["S"]
+    elems = (min(t1 * per, info["V"]) - t0 * per) * 8
+    start = time.perf_counter()
+    reps = 0
+    while True:
+        oracle.decompress_tiles(_POOL_BLOB, t0, t1, oracle.BF16, out)
+        reps += 1
+        if time.perf_counter() - start >= seconds:
+            break
+    return elems * reps, time.perf_counter() - start
+
+
+def cpu_oracle_rate_parallel(blob: bytes, seconds: float, cores: int):
+    """The same oracle decode, tile-parallel: `cores` processes (spawned, so no CUDA state is
+    inherited), each on a contiguous tile range.  GB/s of output over the slowest worker."""
+    import multiprocessing as mp
+    import oracle
+    info = oracle.blob_info(blob)
+    n = info["n_tiles"]
+    cores = max(1, min(cores, n))
+    bounds = [n * i // cores for i in range(cores + 1)]
+    jobs = [(bounds[i], bounds[i + 1], seconds) for i in range(cores)]
+    with mp.get_context("spawn").Pool(cores, initializer=_pool_init, initargs=(blob,)) as pool:
+        res = pool.map(_pool_decode, jobs)
+    elems = sum(r[0] for r in res)
+    dt = max(r[1] for r in res)
+    return elems * 2 / dt / 1e9, cores, dt
+
+
+def host_cores() -> int:
+    try:
+        return len(os.sched_getaffinity(0))
+    except AttributeError:
+        return os.cpu_count() or 1
+
+
 def reference_arm(args, m, desc):
     """The oracle as it stands, timed on the host cores with the same metric and workload."""
     rank = int(os.environ.get("RANK", "0"))
@@ -227,9 +298,9 @@ def reference_arm(args, m, desc):
 # ---------------------------------------------------------------------------------------------
 def main():
     args = parse_args()
-    m, desc = workload()
+    mats, desc = workload(args.workload)
     if args.impl == "reference":
-        reference_arm(args, m, desc)
+        reference_arm(args, mats[0], desc)
         return
 
     import torch
@@ -251,40 +322,51 @@ def main():
             dist.barrier()
 
     # compress with the library's host encoder
-    cfg = ep.LatticeRANSConfig(m.target_bpp, steps_per_tile=args.steps_per_tile)
-    host = W.bits_to_torch(m.bits, m.dtype)
+    cfg = ep.LatticeRANSConfig(mats[0].target_bpp, steps_per_tile=args.steps_per_tile)
     t = time.perf_counter()
-    comp = ep.compress(host, cfg)
+    comps = [ep.compress(W.bits_to_torch(m.bits, m.dtype), cfg) for m in mats]
     enc_s = time.perf_counter() - t
-    blob = comp.to_bytes()
-    rows, cols = comp.shape
-    out_bytes = rows * cols * 2
-    blob_bytes = len(blob)
+    blobs = [c.to_bytes() for c in comps]
+    n = len(comps)
+    out_dt = comps[0].dtype
+    es = torch.empty((), dtype=out_dt).element_size()
+    out_bytes = sum(c.shape[0] * c.shape[1] * es for c in comps)
+    blob_bytes = sum(len(b) for b in blobs)
     moved = blob_bytes + out_bytes
+    grouped = n > 1 and args.decode == "grouped"
 
-    # R independent device copies so that consecutive steps miss L2
+    # R independent device copies of the whole set so that consecutive steps miss L2
     R = max(2, math.ceil(3 * L2_BYTES / moved))
     stream = torch.cuda.current_stream()
-    copies = [ep.CompressedTensor.from_bytes(blob) for _ in range(R)]
-    outs = [torch.empty((rows, cols), dtype=torch.bfloat16, device="cuda") for _ in range(R)]
-    for c in copies:
-        c.prepare(stream=stream)
+    copies = [[ep.CompressedTensor.from_bytes(b) for b in blobs] for _ in range(R)]
+    outs = [[torch.empty(c.shape, dtype=out_dt, device="cuda") for c in comps] for _ in range(R)]
+    for cs in copies:
+        for c in cs:
+            c.prepare(stream=stream)
     L = ep.lib()
-    views = [ep.tensor_view(o) for o in outs]
-    handles = [c.handle for c in copies]
+    views = [[ep.tensor_view(o) for o in os_] for os_ in outs]
+    handles = [[c.handle for c in cs] for cs in copies]
+    g_handles = [(ctypes.c_void_p * n)(*[h.value for h in hs]) for hs in handles]
+    g_views = [(ep.EpTensor * n)(*vs) for vs in views]
     sh = ctypes.c_void_p(stream.cuda_stream)
-    decomp = L.ep_decompress
+    launches_per_step = math.ceil(n / 32) if grouped else n
 
     def step(i):
         j = i % R
-        rc = decomp(handles[j], ctypes.byref(views[j]), sh)
-        if rc != 0:
-            raise ep.EPError(rc, "ep_decompress")
+        if grouped:
+            rc = L.ep_decompress_group(g_handles[j], g_views[j], n, sh)
+            if rc != 0:
+                raise ep.EPError(rc, "ep_decompress_group")
+            return
+        for h, v in zip(handles[j], views[j]):
+            rc = L.ep_decompress(h, ctypes.byref(v), sh)
+            if rc != 0:
+                raise ep.EPError(rc, "ep_decompress")
 
-    # correctness gate before timing: this rank's output equals a reference decode
+    # a first step, checked by the kernels' own integrity checks
     step(0)
     torch.cuda.synchronize()
-    for c in copies[:1]:
+    for c in copies[0]:
         ep.decode_status(c)
 
     for i in range(args.warmup):
@@ -304,9 +386,9 @@ def main():
     torch.cuda.synchronize()
     clocks.start()
     time.sleep(0.2)  # let the sampler start before the timed region
-    # One decode kernel per step, launched back to back on one stream (each may overlap the
-    # previous one's drain, see the kernel); the average launch duration is the timed region
-    # over K, which also counts any gap between launches.
+    # Decode kernels launched back to back on one stream (each may overlap the previous one's
+    # drain, see the kernel); the average step is the timed region over K, which also counts
+    # any gap between launches.
     start.record(stream)
     for i in range(K):
         step(i)
@@ -316,62 +398,85 @@ def main():
     torch.cuda.synchronize()
     clk = clocks.stop()
     total_ms = start.elapsed_time(end)
-    avg_launch_ms = total_ms / K
-    for c in copies:
-        ep.decode_status(c)
+    avg_step_ms = total_ms / K
+    for cs in copies:
+        for c in cs:
+            ep.decode_status(c)
 
-    total_ms, avg_launch_ms = max_over_ranks([total_ms, avg_launch_ms], world)
+    total_ms, avg_step_ms = max_over_ranks([total_ms, avg_step_ms], world)
 
-    # end to end through the public call with host buffers: upload the blob, decode, download
-    host_out = torch.empty((rows, cols), dtype=torch.bfloat16).pin_memory()
+    # end to end through the public call with host buffers: upload each blob, decode, download
+    host_outs = [torch.empty(c.shape, dtype=out_dt).pin_memory() for c in comps]
+
+    def e2e_step():
+        for c, ho in zip(comps, host_outs):
+            ep.decompress(c, out=ho)
+
     for _ in range(3):
-        ep.decompress(comp, out=host_out)
+        e2e_step()
     torch.cuda.synchronize()
     barrier()
     e_s, e_e = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     e_s.record(stream)
     for _ in range(args.e2e_steps):
-        ep.decompress(comp, out=host_out)
+        e2e_step()
     e_e.record(stream)
     torch.cuda.synchronize()
     e2e_ms = e_s.elapsed_time(e_e)
     (e2e_ms,) = max_over_ranks([e2e_ms], world)
-    ep.decode_status(comp)
+    for c in comps:
+        ep.decode_status(c)
 
     if rank == 0:
         peak, peak_kind = hbm_peak()
-        achieved = moved / (avg_launch_ms * 1e-3) / 1e9
+        achieved = moved / (avg_step_ms * 1e-3) / 1e9   # algorithmic bytes over the step's device time
         value = job_throughput(world, out_bytes, K, total_ms)
-        info = comp.info
-        symbols = info.n_vectors * 9
+        symbols = sum(c.info.n_vectors for c in comps) * 9
         cpu = None
         if world == 1 and not args.no_cpu_baseline:
-            gbs, reps, nt, secs = cpu_oracle_rate(blob, args.cpu_seconds)
+            gbs, reps, nt, secs = cpu_oracle_rate(blobs[0], args.cpu_seconds)
+            r0, c0 = comps[0].shape
+            what = "matrix" if n == 1 else f"first matrix of the {n}"
             cpu = {"value": gbs, "unit": "GB/s", "cores": 1, "kind": "oracle",
-                   "sample": f"whole {rows}x{cols} matrix ({nt} tiles) decoded {reps} times, {secs:.1f} s, "
+                   "sample": f"whole {r0}x{c0} {what} ({nt} tiles) decoded {reps} times, {secs:.1f} s, "
                              f"single-threaded oracle"}
-        traffic = committed_traffic("decode_square_bf16.md")
+            if args.cpu_cores != 1:
+                want = host_cores() if args.cpu_cores <= 0 else args.cpu_cores
+                pg, used, psecs = cpu_oracle_rate_parallel(blobs[0], args.cpu_seconds, want)
+                cpu["all_cores"] = {"value": pg, "unit": "GB/s", "cores": used, "kind": "oracle",
+                                    "sample": f"the same {what}, tile-parallel over {used} processes, "
+                                              f"{psecs:.1f} s"}
+        traffic = committed_traffic("decode_square_bf16.md") if args.workload == "square" else None
+        info = comps[0].info
+        config = {
+            "workload": desc, "matrices": n,
+            "shapes": [list(c.shape) for c in comps],
+            "target_bpp": mats[0].target_bpp,
+            "actual_bpp": 8.0 * blob_bytes / sum(c.shape[0] * c.shape[1] for c in comps),
+            "steps_per_tile": sorted({c.info.steps_per_tile for c in comps}),
+            "n_tiles": sum(c.info.n_tiles for c in comps), "blob_bytes": blob_bytes, "out_bytes": out_bytes,
+            "l2": f"rotating {R} blob/output copies ({R * moved / 1e6:.0f} MB > 3x L2)",
+            "symbols_per_s": world * symbols * K / (total_ms * 1e-3),
+            "step_avg_us": avg_step_ms * 1e3, "encode_s": enc_s,
+            "decode": ("ep_decompress_group, one launch per step" if grouped else
+                       f"ep_decompress, {n} launch(es) per step"),
+            "parallelism": f"weak, {world} independent rank(s)",
+        }
+        if n == 1:
+            config.update(rows=info.rows, cols=info.cols, kernel_avg_us=avg_step_ms * 1e3)
         line = {
             "metric": METRIC, "value": value, "unit": "GB/s", "n_gpus": world, "steps": K,
             "warmup": args.warmup, "ms_per_step": total_ms / K, "higher_is_better": True,
             "scaling": "weak", "vs_baseline": None, "dtype": "u32/f32", "data": "synthetic",
-            "config": {
-                "workload": desc, "rows": rows, "cols": cols, "target_bpp": m.target_bpp,
-                "actual_bpp": comp.actual_bpp, "steps_per_tile": info.steps_per_tile,
-                "n_tiles": info.n_tiles, "blob_bytes": blob_bytes, "out_bytes": out_bytes,
-                "l2": f"rotating {R} blob/output copies ({R * moved / 1e6:.0f} MB > 3x L2)",
-                "symbols_per_s": world * symbols * K / (total_ms * 1e-3),
-                "kernel_avg_us": avg_launch_ms * 1e3, "encode_s": enc_s,
-                "parallelism": f"weak, {world} independent rank(s)",
-            },
+            "config": config,
             "roofline": {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s",
                          "frac": achieved / peak, "traffic": traffic,
                          "peak_kind": peak_kind, "nominal_8tbs_frac": achieved / NOMINAL_HBM_GBS,
-                         "algorithmic_bytes_per_launch": moved},
+                         "algorithmic_bytes_per_launch" if launches_per_step == 1 else "algorithmic_bytes_per_step": moved},
             "cpu_baseline": cpu,
             "e2e": {"value": job_throughput(world, out_bytes, args.e2e_steps, e2e_ms), "unit": "GB/s",
                     "h2d_bytes_per_step": blob_bytes, "d2h_bytes_per_step": out_bytes},
-            "gpu_launches": K,
+            "gpu_launches": K * launches_per_step,
             "clocks": clk,
         }
         print(json.dumps(line), flush=True)
