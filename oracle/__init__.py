@@ -5,7 +5,7 @@ precision of the encoder, the blob format and the decoder.  Only the test suite,
 and the CPU-baseline leg of the benchmark may import this package; the product package never
 does, and the two share no code.
 
-Dtype codes follow the blob header: 1 = BF16, 2 = FP16, 3 = FP8 E4M3, 4 = FP32.
+Dtype codes follow the blob header: 1 = BF16, 2 = FP16, 3 = FP8 E4M3, 4 = FP32, 5 = INT8.
 """
 from __future__ import annotations
 
@@ -19,9 +19,9 @@ _HERE = os.path.dirname(os.path.abspath(__file__))
 _SRC = os.path.join(_HERE, "oracle.c")
 _LIB = os.path.join(_HERE, "liboracle.so")
 
-BF16, FP16, E4M3, F32 = 1, 2, 3, 4
-ITEMSIZE = {BF16: 2, FP16: 2, E4M3: 1, F32: 4}
-NPTYPE = {BF16: np.uint16, FP16: np.uint16, E4M3: np.uint8, F32: np.uint32}
+BF16, FP16, E4M3, F32, INT8 = 1, 2, 3, 4, 5
+ITEMSIZE = {BF16: 2, FP16: 2, E4M3: 1, F32: 4, INT8: 1}
+NPTYPE = {BF16: np.uint16, FP16: np.uint16, E4M3: np.uint8, F32: np.uint32, INT8: np.uint8}
 
 
 def build() -> str:

@@ -43,7 +43,7 @@
 /* Constants of the format.                                                                    */
 /* ------------------------------------------------------------------------------------------ */
 
-enum { ORC_BF16 = 1, ORC_FP16 = 2, ORC_E4M3 = 3, ORC_F32 = 4 };
+enum { ORC_BF16 = 1, ORC_FP16 = 2, ORC_E4M3 = 3, ORC_F32 = 4, ORC_INT8 = 5 };
 
 #define ORC_R 127          /* reading: field alphabet [-R, R] coded directly, R = 127     */
 #define ORC_ESC 255        /* symbol that announces a raw 16-bit field value               */
@@ -75,7 +75,7 @@ static uint64_t pad16(uint64_t n) { return (n + 15u) / 16u * 16u; }
 
 /* ------------------------------------------------------------------------------------------ */
 /* Number formats: reading each container exactly, and rounding to it.                        */
-/* [DOC-0]: the tensor is restored in the input's dtype; [ABS] lists BF16, FP16 and FP8.       */
+/* [DOC-0]: the tensor is restored in the input's dtype; [ABS] lists BF16, FP16, FP8 and INT8. */
 /* ------------------------------------------------------------------------------------------ */
 
 /* Exact value of one stored element of the given dtype. */
@@ -108,6 +108,7 @@ double orc_dtype_to_f64(uint32_t bits, int dtype)
         else v = ldexp((double)(8 + m), e - 10);
         return s ? -v : v;
     }
+    if (dtype == ORC_INT8) return (double)(int8_t)(uint8_t)bits;   /* two's complement */
     return NAN;
 }
 
@@ -201,13 +202,29 @@ uint32_t orc_f32_to_e4m3(uint32_t fbits)
     return sign | ((uint32_t)(lead + 7) << 3) | mant;
 }
 
-/* Array form of the three conversions (used by the exhaustive conversion checks). */
+/* fp32 bit pattern -> INT8.  reading: the integer container takes the nearest integer, ties to
+ * even (the rounding the float containers use), saturating to [-128, 127] as E4M3 saturates;
+ * NaN, which no reconstruction produces, gives 0.  rint() rounds half-to-even in the default
+ * rounding mode. */
+uint32_t orc_f32_to_i8(uint32_t fbits)
+{
+    float f;
+    memcpy(&f, &fbits, 4);
+    if (isnan(f)) return 0;
+    double r = rint((double)f);
+    if (r > 127.0) r = 127.0;
+    if (r < -128.0) r = -128.0;
+    return (uint32_t)(uint8_t)(int8_t)r;
+}
+
+/* Array form of the conversions (used by the exhaustive conversion checks). */
 void orc_cvt_f32_array(const uint32_t* in, uint64_t n, int dtype_out, void* out)
 {
     for (uint64_t i = 0; i < n; i++) {
         if (dtype_out == ORC_BF16) ((uint16_t*)out)[i] = (uint16_t)orc_f32_to_bf16(in[i]);
         else if (dtype_out == ORC_FP16) ((uint16_t*)out)[i] = (uint16_t)orc_f32_to_f16(in[i]);
         else if (dtype_out == ORC_E4M3) ((uint8_t*)out)[i] = (uint8_t)orc_f32_to_e4m3(in[i]);
+        else if (dtype_out == ORC_INT8) ((uint8_t*)out)[i] = (uint8_t)orc_f32_to_i8(in[i]);
         else ((uint32_t*)out)[i] = in[i];
     }
 }
@@ -220,17 +237,19 @@ static void store_value(void* out, uint64_t idx, int dtype_out, double w)
     if (dtype_out == ORC_BF16) ((uint16_t*)out)[idx] = (uint16_t)orc_f32_to_bf16(fb);
     else if (dtype_out == ORC_FP16) ((uint16_t*)out)[idx] = (uint16_t)orc_f32_to_f16(fb);
     else if (dtype_out == ORC_E4M3) ((uint8_t*)out)[idx] = (uint8_t)orc_f32_to_e4m3(fb);
+    else if (dtype_out == ORC_INT8) ((uint8_t*)out)[idx] = (uint8_t)orc_f32_to_i8(fb);
     else ((uint32_t*)out)[idx] = fb;
 }
 
 static int dtype_size(int dtype)
 {
-    return dtype == ORC_E4M3 ? 1 : dtype == ORC_F32 ? 4 : (dtype == ORC_BF16 || dtype == ORC_FP16) ? 2 : 0;
+    return (dtype == ORC_E4M3 || dtype == ORC_INT8) ? 1 : dtype == ORC_F32 ? 4
+           : (dtype == ORC_BF16 || dtype == ORC_FP16) ? 2 : 0;
 }
 
 static uint32_t load_bits(const void* data, int dtype, uint64_t i)
 {
-    if (dtype == ORC_E4M3) return ((const uint8_t*)data)[i];
+    if (dtype == ORC_E4M3 || dtype == ORC_INT8) return ((const uint8_t*)data)[i];
     if (dtype == ORC_F32) return ((const uint32_t*)data)[i];
     return ((const uint16_t*)data)[i];
 }

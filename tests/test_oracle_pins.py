@@ -19,7 +19,8 @@ Pin map (oracle function -> test):
                              test_rans_size_near_cross_entropy
   orc_dtype_to_f64        -> test_dtype_decode_vs_numpy_torch
   orc_f32_to_bf16/f16/
-  e4m3, orc_round_f32     -> test_conversions_vs_library
+  e4m3/i8, orc_round_f32  -> test_conversions_vs_library
+  INT8 store and read     -> test_int8_container_round_trip
   orc_compress (RMS, LS,
   scale search, tiling)   -> test_end_to_end_fields_vs_independent_quantiser, test_rms_scale_invariance,
                              test_least_squares_orthogonality, test_constant_rows_exact,
@@ -388,6 +389,20 @@ def test_conversions_vs_library():
     big = fin & (np.abs(f) >= 464.0)
     assert np.all((got8[big] & 0x7F) == 0x7E)
     assert np.array_equal(got8[big] >> 7, (p[big] >> 31).astype(np.uint8))
+    # INT8: numpy's rint (nearest, ties to even) clipped to [-128, 127]; ties and the saturation
+    # edges are drawn explicitly as well
+    ties = np.concatenate([np.arange(-300, 301, dtype=np.float64) + 0.5, [127.49, 127.5, -128.5, -128.51]])
+    pi = np.concatenate([p, ties.astype(np.float32).view(np.uint32)])
+    fi = pi.view(np.float32)
+    got_i = oracle.cvt_f32(pi, oracle.INT8).view(np.int8)
+    fin_i = np.isfinite(fi)
+    ref_i = np.clip(np.rint(fi[fin_i].astype(np.float64)), -128, 127).astype(np.int8)
+    assert np.array_equal(got_i[fin_i], ref_i)
+    inf = np.isinf(fi)
+    assert np.array_equal(got_i[inf], np.where(fi[inf] > 0, 127, -128).astype(np.int8))
+    assert np.all(got_i[np.isnan(fi)] == 0)
+    assert list(oracle.cvt_f32(np.array([0.5, 1.5, 2.5, -0.5, -1.5], np.float32).view(np.uint32),
+                               oracle.INT8).view(np.int8)) == [0, 2, 2, 0, -2]
     # fp32 rounding of exact doubles: numpy's float64 -> float32 cast
     v = np.concatenate([RNG.normal(0, 1, 100_000) * 10.0 ** RNG.integers(-30, 30, 100_000),
                         (RNG.normal(0, 1, 1000).astype(np.float32).astype(np.float64)
@@ -411,6 +426,8 @@ def test_dtype_decode_vs_numpy_torch():
     assert np.array_equal(np.isnan(got), np.isnan(e))
     assert np.array_equal(got[~np.isnan(e)], e[~np.isnan(e)])
     assert got[0x7E] == 448.0 and got[0x01] == 2.0 ** -9
+    got = oracle.dtype_to_f64(p8, oracle.INT8)
+    assert np.array_equal(got, p8.view(np.int8).astype(np.float64))
 
 
 # ---------------------------------------------------------------------------------------------
@@ -610,3 +627,18 @@ def test_ragged_shapes_roundtrip(shape):
     f = oracle.decode_fields(blob)
     y = oracle.fields_to_point(f[:, 0], f[:, 1:])
     assert y.shape[0] == shape[0] * ((shape[1] + 7) // 8)
+
+
+def test_int8_container_round_trip():
+    """The integer container ([abstract]: INT8 among the weight containers): an INT8 input is read
+    as exact integers and restored as INT8, each element the fp32 reconstruction rounded to the
+    nearest integer (ties to even) and saturated -- numpy's rint and clip of the FP32 decode."""
+    m = W.int8(rows=64, cols=256)
+    blob = oracle.compress(m.bits, m.dtype, m.target_bpp)
+    assert oracle.blob_info(blob)["dtype"] == oracle.INT8
+    o8 = oracle.decompress(blob)
+    o32 = oracle.decompress(blob, oracle.F32).view(np.float32).astype(np.float64)
+    assert o8.dtype == np.uint8
+    assert np.array_equal(o8.view(np.int8), np.clip(np.rint(o32), -128, 127).astype(np.int8))
+    x = m.bits.view(np.int8).astype(np.float64)
+    assert np.linalg.norm(o8.view(np.int8) - x) / np.linalg.norm(x) < 0.3

@@ -21,6 +21,9 @@ available; shapes follow DiT / transformer linear layers):
 4. ``sweep``   4096 x 11008 FP16, i.i.d. N(0, 0.02^2), targets 0.5, 2.0, 3.5, 6.0, 11.0.
 5. ``large``   four 28672 x 8192 BF16, N(0, 0.015^2) times per-column scales log-uniform in
                [0.5, 2], target 4.0; decoded to BF16 and to FP8 E4M3.
+6. ``int8``    1024 x 4096 INT8 (the integer container): rows N(0, sigma_r^2), sigma_r
+               log-uniform in [0.005, 0.05], each row scaled by 127 / its absmax and rounded to
+               the nearest integer, target 3.0.
 """
 from __future__ import annotations
 
@@ -28,14 +31,14 @@ from dataclasses import dataclass
 
 import numpy as np
 
-BF16, FP16, E4M3, F32 = 1, 2, 3, 4
-DTYPE_NAME = {BF16: "bf16", FP16: "fp16", E4M3: "fp8_e4m3", F32: "fp32"}
+BF16, FP16, E4M3, F32, INT8 = 1, 2, 3, 4, 5
+DTYPE_NAME = {BF16: "bf16", FP16: "fp16", E4M3: "fp8_e4m3", F32: "fp32", INT8: "int8"}
 
 
 @dataclass(frozen=True)
 class Matrix:
     bits: np.ndarray     # rows x cols array of container bit patterns (uint16 / uint8 / uint32)
-    dtype: int           # container code: 1 BF16, 2 FP16, 3 E4M3, 4 FP32
+    dtype: int           # container code: 1 BF16, 2 FP16, 3 E4M3, 4 FP32, 5 INT8
     target_bpp: float
 
     @property
@@ -61,6 +64,8 @@ def _store(x: np.ndarray, dtype: int) -> np.ndarray:
         return to_fp16_bits(x)
     if dtype == F32:
         return np.ascontiguousarray(x, np.float32).view(np.uint32)
+    if dtype == INT8:  # nearest integer (ties to even), saturated
+        return np.clip(np.rint(x), -128, 127).astype(np.int8).view(np.uint8)
     raise ValueError(dtype)
 
 
@@ -107,6 +112,16 @@ def large(j: int, rows: int = 28672, cols: int = 8192) -> Matrix:
     return Matrix(_store(x, BF16), BF16, 4.0)
 
 
+def int8(rows: int = 1024, cols: int = 4096, target_bpp: float = 3.0) -> Matrix:
+    """Integer weights as an INT8 checkpoint stores them: rows N(0, sigma_r^2) with sigma_r
+    log-uniform in [0.005, 0.05], each row divided by its own absmax / 127 and rounded."""
+    g = _rng(6)
+    sigma = np.exp(g.uniform(np.log(0.005), np.log(0.05), size=(rows, 1)))
+    x = g.standard_normal((rows, cols)) * sigma
+    x = x / (np.abs(x).max(axis=1, keepdims=True) / 127.0)
+    return Matrix(_store(x, INT8), INT8, target_bpp)
+
+
 def bits_to_torch(bits: np.ndarray, dtype: int):
     """A torch CPU tensor of the container dtype sharing the bit patterns."""
     import torch
@@ -119,4 +134,6 @@ def bits_to_torch(bits: np.ndarray, dtype: int):
         return t.view(torch.float8_e4m3fn)
     if dtype == F32:
         return t.view(torch.float32)
+    if dtype == INT8:
+        return t.view(torch.int8)
     raise ValueError(dtype)
