@@ -4,13 +4,14 @@ A thin ctypes layer over ``libentropack.so`` (declared in ``include/entropack.h`
 marshals arguments: compression runs in the library's host encoder, and decompression is one
 fused CUDA kernel on the caller's stream.  PyTorch supplies device memory and streams.
 
-Usage, mirroring the method's documentation ("EntroPack lattice compression", section "Usage")::
+The call names follow the interface the method's documentation describes ("EntroPack lattice
+compression", section "Usage"): a config object carrying the target rate, ``compress`` returning
+an object with ``actual_bpp``, and ``decompress`` restoring shape and dtype.  For example::
 
     import dit_weight_compression_b200 as ep
-    config = ep.LatticeRANSConfig(target_bpp=3.5)
-    compressed = ep.compress(tensor, config)        # tensor: 2-D bf16/fp16/fp8_e4m3fn/fp32
-    restored = ep.decompress(compressed, config)    # same shape and dtype, on the GPU
-    compressed.actual_bpp                           # stored bits per element, all metadata included
+    blob = ep.compress(w, ep.LatticeRANSConfig(4.0))   # w: 2-D bf16/fp16/fp8_e4m3fn/fp32/int8
+    w_hat = ep.decompress(blob)                        # on the current GPU, same shape and dtype
+    print(blob.actual_bpp)                             # stored bits per element, metadata included
 """
 from __future__ import annotations
 

@@ -42,7 +42,7 @@ extern "C" int ep_compress_ex(const ep_tensor* in, double target_bpp, const ep_o
     if (in->rows <= 0 || in->cols <= 0) return set_error(EP_ERR_SHAPE, "ep_compress: empty tensor");
     if (!in->data) return set_error(EP_ERR_ARG, "ep_compress: NULL data");
     if (in->row_stride < in->cols) return set_error(EP_ERR_ARG, "ep_compress: row_stride < cols");
-    // "finite target bitrates in [0.001, 11] bits per element"
+    // the documented range of target rates: finite, 0.001 to 11 bits per element
     if (!std::isfinite(target_bpp) || target_bpp < kTargetMin || target_bpp > kTargetMax)
         return set_error(EP_ERR_RANGE, "ep_compress: target_bpp must be finite and in [0.001, 11]");
 

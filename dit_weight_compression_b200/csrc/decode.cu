@@ -1,9 +1,9 @@
 // decode.cu -- fused GPU decompression for sm_100a, and the device-side entry points of the C ABI.
 //
 // "EntroPack lattice compression" (documentation page, section "Encoding and reconstruction"):
-// decoding recovers the fields, reconstructs lattice points and applies the row scales in one
-// fused GPU operation, and the result has the input's shape and dtype.  The arXiv abstract adds
-// that tiles are independently decodable, which is what lets the GPU decode them in parallel.
+// a single fused GPU operation takes the coded fields back to lattice points, scales each row and
+// returns a tensor with the original shape and element type.  Per the arXiv abstract every tile
+// decodes on its own, which is what lets the GPU work on all of them at once.
 //
 // One kernel does the whole path.  Work split:
 //   * one warp per tile; the tile's 32 interleaved rANS states live one per lane;

@@ -8,8 +8,8 @@
 //     coset;
 //   section "Rate selection and refinement": choose s from size estimates on sampled rows,
 //     then quantise the full tensor and fit one least-squares scale per row;
-//   section "Encoding and reconstruction": rANS-code the fields in independently decodable
-//     tiles and store tables, row scales and tile metadata with them.
+//   section "Encoding and reconstruction": rANS-code the fields in tiles that decode on their
+//     own, and keep the frequency tables, per-row scales and per-tile bookkeeping beside them.
 // The rANS coding step is Duda's ("Asymmetric numeral systems", 2009); the E8 nearest point is
 // the Conway-Sloane rule (1982).  Details the pages leave open are fixed as the format header
 // (format.h) and the comments below state.

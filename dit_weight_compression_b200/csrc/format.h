@@ -1,9 +1,9 @@
 // format.h -- internal description of the compressed blob shared by the host encoder, the blob
 // validator and the GPU launch code of the library.
 //
-// The blob stores what "EntroPack lattice compression" (documentation page, section "Encoding
-// and reconstruction") lists: "the probability tables, row scales, and tile metadata" next to
-// the rANS-coded fields.  Byte layout (little-endian, every section 16-byte aligned):
+// The blob holds what "EntroPack lattice compression" (documentation page, section "Encoding
+// and reconstruction") says must travel with the rANS-coded fields: the frequency tables, one
+// scale per row, and the per-tile bookkeeping.  Byte layout (little-endian, every section 16-byte aligned):
 //
 //   header, 80 bytes:  "EPK1" | u16 version = 2 | u8 dtype | u8 R = 127 | u64 rows | u64 cols |
 //                      u32 S | u32 n_tiles | f64 s | u64 total bytes | u64 table offset |

@@ -81,9 +81,9 @@ typedef struct {
 } ep_blob_info;
 
 /*
- * Compress a 2-D tensor to a target rate ("EntroPack lattice compression": opening paragraph --
- * "finite target bitrates in [0.001, 11] bits per element, including non-integer values";
- * sections "Lattice quantization and integer fields" and "Rate selection and refinement").
+ * Compress a 2-D tensor to a target rate ("EntroPack lattice compression": the opening paragraph
+ * admits any finite rate from 0.001 to 11 bits per element, fractional ones included; sections
+ * "Lattice quantization and integer fields" and "Rate selection and refinement").
  *   in          tensor to compress, host or device memory, any ep_dtype; rows, cols >= 1.
  *               Device tensors are copied to the host first (the encoder runs on the host).
  *   target_bpp  requested stored bits per element, finite, in [0.001, 11].
@@ -98,8 +98,8 @@ int ep_compress_ex(const ep_tensor* in, double target_bpp, const ep_options* opt
 
 /*
  * Decompress into `out` ("EntroPack lattice compression", section "Encoding and
- * reconstruction": "Decoding recovers the fields, reconstructs lattice points, and applies the
- * row scales in a fused GPU operation. The result has the input's shape and dtype").
+ * reconstruction": one fused GPU operation turns the coded fields back into lattice points,
+ * multiplies them by the row scales and returns a tensor shaped and typed like the original).
  *   b       blob.
  *   out     rows x cols equal to the blob's; dtype any ep_dtype (the blob's own by convention).
  *           Device output (out->device >= 0, must be the calling thread's current device): one
@@ -137,9 +137,9 @@ int ep_decompress(const ep_blob* b, const ep_tensor* out, void* stream);
 int ep_decompress_group(const ep_blob* const* blobs, const ep_tensor* outs, int n, void* stream);
 
 /* Stored bits per element: 8 * (stored bytes including metadata) / (rows * cols)
- * ("EntroPack lattice compression", section "Encoding and reconstruction": "The actual_bpp
- * property reports the actual stored bytes, including metadata, divided by the element count
- * and multiplied by eight").  Returns -1.0 for a NULL blob. */
+ * ("EntroPack lattice compression", section "Encoding and reconstruction": the reported rate
+ * counts every stored byte, metadata included, as bits per element).  Returns -1.0 for a NULL
+ * blob. */
 double ep_actual_bpp(const ep_blob* b);
 
 /* Header fields of the blob. */

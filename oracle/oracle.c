@@ -11,10 +11,11 @@
  *
  *   [ABS]  "EntroPack: Fast and Accurate Entropy-Coded Weight Compression at Arbitrary
  *          Bitrates", arXiv abstract page (row-normalised E8 quantisation, conditional model,
- *          sampled storage estimates, independently decodable tiles, BF16/FP16/FP8 containers).
+ *          sampled storage estimates, tiles that decode on their own, BF16/FP16/FP8/INT8
+ *          containers).
  *   [DOC]  "EntroPack lattice compression", documentation page Principles / Lattice-rANS:
- *            DOC-0  opening paragraph (2-D tensors, target range [0.001, 11] bits per element,
- *                   decompression keeps the input dtype);
+ *            DOC-0  opening paragraph (2-D tensors; any finite rate from 0.001 to 11 bits
+ *                   per element; the restored tensor has the input's element type);
  *            DOC-LQ section "Lattice quantization and integer fields";
  *            DOC-RS section "Rate selection and refinement";
  *            DOC-ER section "Encoding and reconstruction";
@@ -289,7 +290,7 @@ static void d8_nearest(const double u[8], double g[8])
  * Nearest point of E8 = D8 u (D8 + 1/2) to t [CS]: take the nearest point of D8 and the nearest
  * point of the half-integer coset (the D8 rule applied to t - 1/2, then + 1/2), and keep the
  * nearer of the two.  The coset bit is 0 for the integer coset and 1 for the half-integer one
- * ([DOC-LQ]: "E8 has integer-coordinate and half-integer-coordinate subsets, called cosets").
+ * ([DOC-LQ]: the two cosets of E8 are its all-integer and all-half-integer points).
  * reading: an exact tie in squared distance keeps coset 0.
  */
 void orc_e8_nearest(const double t[8], double y[8], int* coset)
@@ -320,8 +321,8 @@ void orc_e8_nearest(const double t[8], double y[8], int* coset)
 /*
  * Lattice point -> fields.  z = y - c/2 lies in D8 (sum even).  f1..f7 = z1..z7, and the
  * parity constraint compacts the last coordinate: with par = (z1 + ... + z7) mod 2 in {0, 1},
- * z8 - par is even and f8 = (z8 - par) / 2 ([DOC-LQ]: "using the lattice's parity constraint
- * to compact the final coordinate").
+ * z8 - par is even and f8 = (z8 - par) / 2 ([DOC-LQ]: E8's even-sum rule lets the last
+ * coordinate be stored at half size).
  * reading: for coset 1 the half is subtracted (z = y - 1/2).
  */
 void orc_point_to_fields(const double y[8], int coset, int32_t f[8])
@@ -335,8 +336,8 @@ void orc_point_to_fields(const double y[8], int coset, int32_t f[8])
     f[7] = (z[7] - par) / 2;
 }
 
-/* Fields -> lattice point, the arithmetic inverse ([DOC-LQ]: "inverted arithmetically without a
- * reconstruction codebook"): z8 = 2 f8 + par, y = z + c/2. */
+/* Fields -> lattice point by arithmetic alone, no table of points ([DOC-LQ]: the fields are
+ * invertible): z8 = 2 f8 + par, y = z + c/2. */
 void orc_fields_to_point(int coset, const int32_t f[8], double y[8])
 {
     int32_t z[8];
@@ -402,8 +403,8 @@ static void cumulate(const uint16_t q[256], uint32_t cum[257])
 static int context_of(int u, int c) { return u == 0 ? 0 : 1 + 8 * c + (u - 1); }
 
 /* ------------------------------------------------------------------------------------------ */
-/* Tiled, 32-way interleaved rANS [ANS] with the word layout of the format ([DOC-ER]: "encoded  */
-/* with rANS in independently decodable tiles").                                               */
+/* Tiled, 32-way interleaved rANS [ANS] with the word layout of the format ([DOC-ER]: the      */
+/* fields are rANS-coded in tiles, each of which decodes without the others).                  */
 /*                                                                                            */
 /* One tile holds up to 32*S consecutive vectors; lane l at step k owns vector 32k + l of the  */
 /* tile and has its own 32-bit rANS state.  Each vector is 9 symbols: the coset (context 0) and */
@@ -618,7 +619,7 @@ typedef struct {
  * row but is excluded from the RMS and least-squares sums and never written back. */
 static double elem(const matrix* m, int64_t r, int64_t c) { return c < m->cols ? m->w[r * m->cols + c] : 0.0; }
 
-/* [DOC-LQ]: "normalizes each row by its root mean square". */
+/* [DOC-LQ]: every row is first divided by its RMS. */
 static void row_rms(matrix* m)
 {
     for (int64_t r = 0; r < m->rows; r++) {
@@ -630,9 +631,9 @@ static void row_rms(matrix* m)
 
 /*
  * Quantise vector k of row r at shared scale s: t = clamp(x_hat / s, +-32764) with x_hat the
- * RMS-normalised row, then the E8 nearest point ([DOC-LQ]: "groups the normalized values into
- * eight-dimensional vectors ... nearest point on a scaled E8 lattice"; "a shared quantization
- * scale controls the spacing").  An all-zero row (RMS 0) maps every vector to the origin.
+ * RMS-normalised row, then the E8 nearest point ([DOC-LQ]: the normalised row is cut into
+ * 8-vectors, each snapped to the closest point of E8 dilated by one scale s common to the whole
+ * tensor).  An all-zero row (RMS 0) maps every vector to the origin.
  */
 static void quantise_vector(const matrix* m, int64_t r, int64_t k, double s, double y[8], int* coset)
 {
@@ -685,8 +686,9 @@ static uint64_t table_section_bytes(const uint16_t* q17)
 }
 
 /*
- * Estimated blob size in bits per element at scale s from the sampled rows ([DOC-RS]: "For each
- * candidate scale, it estimates the coded field size and the metadata needed for decoding").
+ * Estimated blob size in bits per element at scale s from the sampled rows ([DOC-RS]: a
+ * candidate scale is judged by the predicted size of its coded fields plus the metadata the
+ * decoder needs).
  * reading: n_s = min(rows, 256) rows at floor(i * rows / n_s); tables are quantised from the
  * sample's counts; coded size = sum over contexts and symbols of n * -log2(q / M) bits plus
  * 16 bits per escape, scaled by rows / n_s; metadata = exact header, table, row-scale and
@@ -730,11 +732,11 @@ static double estimate_bpp(const matrix* m, double s, int64_t S, int full_sample
 }
 
 /*
- * Choose the shared scale ([DOC-RS]: "searches for a quantization scale using sampled rows";
+ * Choose the shared scale ([DOC-RS]: the scale is searched for on a sample of rows;
  * [DOC-LQ]: finer spacing costs more bits).
  * reading: the finest scale whose estimate meets the target, by 48 bisection steps on log2 s
  * over [-24, 8]; if even 2^8 misses the target, 2^8 (the actual size is reported as it is,
- * [DOC-ER]: "the achieved bitrate can differ from the requested target").
+ * [DOC-ER]: the stored rate need not equal the requested one).
  */
 static double choose_scale(const matrix* m, double target, int64_t S)
 {
@@ -790,8 +792,8 @@ double orc_estimate_bpp(const void* data, int dtype, int64_t rows, int64_t cols,
  * Compress a rows x cols matrix stored as dtype bits.  steps_per_tile = 0 selects the default S;
  * scale_override > 0 skips the search.  On success *blob is a malloc'd byte string of *len bytes.
  *
- * Blob layout (little-endian, every section 16-byte aligned; [DOC-ER]: "the representation also
- * stores the probability tables, row scales, and tile metadata"):
+ * Blob layout (little-endian, every section 16-byte aligned; [DOC-ER]: besides the coded fields
+ * the blob keeps the frequency tables, the per-row scales and per-tile bookkeeping):
  *   header (80 bytes): "EPK1", u16 version 2, u8 dtype, u8 R, u64 rows, u64 cols, u32 S,
  *     u32 n_tiles, f64 s, u64 total bytes, u64 offsets of the table, row-scale, tile-offset
  *     and stream sections;
@@ -806,7 +808,7 @@ int orc_compress(const void* data, int dtype, int64_t rows, int64_t cols, double
 {
     *blob = NULL;
     *len = 0;
-    /* [DOC-0]: "finite target bitrates in [0.001, 11] bits per element" */
+    /* [DOC-0]: the target must be finite and within 0.001 to 11 bits per element */
     if (!(target_bpp >= 0.001 && target_bpp <= 11.0)) return -4;
     matrix m;
     memset(&m, 0, sizeof m);
@@ -816,10 +818,9 @@ int orc_compress(const void* data, int dtype, int64_t rows, int64_t cols, double
     int64_t S = steps_per_tile > 0 ? steps_per_tile : default_steps(target_bpp);
     double s = scale_override > 0 ? scale_override : choose_scale(&m, target_bpp, S);
 
-    /* Quantise the whole tensor at s; fit one least-squares scale per row ([DOC-RS]: "Once the
-     * scale is selected, the encoder quantizes the full tensor and fits a reconstruction scale
-     * for each row by least squares"): alpha_r = sum w y / sum y^2 over real columns, stored
-     * as fp32 (0 when sum y^2 = 0). */
+    /* Quantise the whole tensor at s; fit one least-squares scale per row ([DOC-RS]: with s
+     * fixed, every row is quantised and gets its own reconstruction scale by least squares):
+     * alpha_r = sum w y / sum y^2 over real columns, stored as fp32 (0 when sum y^2 = 0). */
     int64_t V = rows * m.vpr;
     uint8_t* sym9 = (uint8_t*)malloc((size_t)V * 9);
     int16_t* raw8 = (int16_t*)malloc((size_t)V * 8 * sizeof(int16_t));
@@ -843,8 +844,8 @@ int orc_compress(const void* data, int dtype, int64_t rows, int64_t cols, double
         alpha[r] = syy > 0.0 ? (float)(swy / syy) : 0.0f;
     }
 
-    /* Probability tables from the whole tensor ([DOC-LQ]: "the probability model conditions each
-     * coordinate field on the coset"). */
+    /* Probability tables from the whole tensor ([DOC-LQ]: one model per coordinate field, given
+     * the coset). */
     uint16_t q17[ORC_NCTX * 256];
     for (int ctx = 0; ctx < ORC_NCTX; ctx++) orc_quantize_table(cnt + 256 * ctx, q17 + 256 * ctx);
 
@@ -930,8 +931,8 @@ done:
 }
 
 /* ------------------------------------------------------------------------------------------ */
-/* The decoder ([DOC-ER]: "Decoding recovers the fields, reconstructs lattice points, and       */
-/* applies the row scales ... The result has the input's shape and dtype").                    */
+/* The decoder ([DOC-ER]: fields back to lattice points, times the row scales, in a tensor of  */
+/* the original shape and element type).                                                      */
 /* ------------------------------------------------------------------------------------------ */
 
 typedef struct {
@@ -1089,8 +1090,7 @@ int orc_decompress(const uint8_t* blob, uint64_t len, int dtype_out, void* out)
     return orc_decompress_tiles(blob, len, 0, -1, dtype_out, out);
 }
 
-/* [DOC-ER]: "The actual_bpp property reports the actual stored bytes, including metadata,
- * divided by the element count and multiplied by eight." */
+/* [DOC-ER]: the reported rate is 8 x every stored byte (metadata included) / element count. */
 double orc_actual_bpp(const uint8_t* blob, uint64_t len)
 {
     parsed P;

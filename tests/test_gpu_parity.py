@@ -5,7 +5,7 @@ Bars (per element):
   * restored values within 1 ulp of the output container -- both sides compute the same IEEE
     sequence (fp32 product of the fp32 row scale and the exact lattice coordinate, then one
     round-to-nearest-even into the container), so the checks below require 0 ulp;
-  * relative L2 error against the input equal to the oracle's to 1e-6.
+  * ||output - input|| / ||input|| equal to the oracle's to 1e-6.
 Both cross directions: the GPU decodes oracle-encoded blobs, and (host suite) the oracle decodes
 library-encoded blobs.  Full-size workloads compare every element where the oracle finishes in
 seconds and sampled tiles (first, last, and seeded random ones) elsewhere.
