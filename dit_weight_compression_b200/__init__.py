@@ -24,9 +24,9 @@ import torch
 _PKG = os.path.dirname(os.path.abspath(__file__))
 LIB_PATH = os.path.join(_PKG, "libentropack.so")
 
-BF16, FP16, FP8_E4M3, F32 = 1, 2, 3, 4
+BF16, FP16, FP8_E4M3, F32, INT8 = 1, 2, 3, 4, 5
 _TORCH_TO_EP = {torch.bfloat16: BF16, torch.float16: FP16, torch.float8_e4m3fn: FP8_E4M3,
-                torch.float32: F32}
+                torch.float32: F32, torch.int8: INT8}
 _EP_TO_TORCH = {v: k for k, v in _TORCH_TO_EP.items()}
 
 ERRORS = {-1: "EP_ERR_ARG", -2: "EP_ERR_DTYPE", -3: "EP_ERR_SHAPE", -4: "EP_ERR_RANGE",
@@ -256,4 +256,4 @@ def decode_fields(compressed: CompressedTensor, stream=None) -> torch.Tensor:
 
 
 __all__ = ["LatticeRANSConfig", "CompressedTensor", "compress", "decompress", "decompress_group", "decode_status",
-           "decode_fields", "EPError", "lib", "BF16", "FP16", "FP8_E4M3", "F32"]
+           "decode_fields", "EPError", "lib", "BF16", "FP16", "FP8_E4M3", "F32", "INT8"]

@@ -73,7 +73,7 @@ constexpr uint32_t kEntryEsc = 1u << 19;
 constexpr uint32_t kEntryQShift = 21;
 static_assert(kProbBits == 10, "the packed entry holds 10-bit slots");
 
-enum OutKind { kOutBF16 = 0, kOutFP16 = 1, kOutE4M3 = 2, kOutF32 = 3, kOutFields = 4 };
+enum OutKind { kOutBF16 = 0, kOutFP16 = 1, kOutE4M3 = 2, kOutF32 = 3, kOutFields = 4, kOutI8 = 5 };
 
 // Status word bits (sticky, cleared by ep_decode_status).
 enum : uint32_t {
@@ -322,7 +322,7 @@ __device__ void build_tables(uint32_t (*tab)[kProbTotal], BuildScratch& scr, con
 // ---- output conversion -----------------------------------------------------------------------
 template <int OUT>
 struct OutElem {
-    static constexpr int kBytes = OUT == kOutE4M3 ? 1 : (OUT == kOutF32 ? 4 : 2);
+    static constexpr int kBytes = (OUT == kOutE4M3 || OUT == kOutI8) ? 1 : (OUT == kOutF32 ? 4 : 2);
 };
 
 // Eight values to eight consecutive elements at `dst` (aligned to the vector's size).
@@ -346,6 +346,14 @@ __device__ __forceinline__ void store_vec(uint8_t* dst, const float v[8]) {
         u.z = *reinterpret_cast<uint32_t*>(&h2);
         u.w = *reinterpret_cast<uint32_t*>(&h3);
         __stcs(reinterpret_cast<uint4*>(dst), u);
+    } else if constexpr (OUT == kOutI8) {
+        // nearest integer, ties to even, saturated to [-128, 127]; bytes packed in order
+        int32_t q[8];
+#pragma unroll
+        for (int i = 0; i < 8; ++i) q[i] = max(-128, min(127, __float2int_rn(v[i])));
+        const uint32_t lo = __byte_perm(__byte_perm(q[0], q[1], 0x0040), __byte_perm(q[2], q[3], 0x0040), 0x5410);
+        const uint32_t hi = __byte_perm(__byte_perm(q[4], q[5], 0x0040), __byte_perm(q[6], q[7], 0x0040), 0x5410);
+        __stcs(reinterpret_cast<uint2*>(dst), make_uint2(lo, hi));
     } else if constexpr (OUT == kOutE4M3) {
         uint32_t w[4];
 #pragma unroll
@@ -364,6 +372,7 @@ __device__ __forceinline__ void store_one(uint8_t* dst, float v) {
     if constexpr (OUT == kOutBF16) *reinterpret_cast<__nv_bfloat16*>(dst) = __float2bfloat16_rn(v);
     else if constexpr (OUT == kOutFP16) *reinterpret_cast<__half*>(dst) = __float2half_rn(v);
     else if constexpr (OUT == kOutE4M3) *dst = uint8_t(__nv_cvt_float_to_fp8(v, __NV_SATFINITE, __NV_E4M3));
+    else if constexpr (OUT == kOutI8) *dst = uint8_t(max(-128, min(127, __float2int_rn(v))));
     else *reinterpret_cast<float*>(dst) = v;
 }
 
@@ -889,6 +898,7 @@ int launch(const Params& p, int out_kind, bool vec, uint64_t max_tile, bool esc,
         case kOutFP16: return launch_out<kOutFP16>(p, vec, wide, esc, st, device, dependent);
         case kOutE4M3: return launch_out<kOutE4M3>(p, vec, wide, esc, st, device, dependent);
         case kOutF32: return launch_out<kOutF32>(p, vec, wide, esc, st, device, dependent);
+        case kOutI8: return launch_out<kOutI8>(p, vec, wide, esc, st, device, dependent);
         default:  // the fields test hook: the 16-warp kernel has the registers it needs
             return launch_one<kWarpsNarrow, kOutFields, false, true>(p, st, device, false);
     }
@@ -954,6 +964,7 @@ int out_kind_of(int dtype) {
         case kFP16: return kOutFP16;
         case kE4M3: return kOutE4M3;
         case kF32: return kOutF32;
+        case kI8: return kOutI8;
         default: return -1;
     }
 }
@@ -1040,7 +1051,7 @@ int ensure_device(ep_blob* b, int dev, cudaStream_t st) {
 }
 
 bool vec_ok(const BlobLayout& L, const void* out, int64_t row_stride, int dtype) {
-    const uintptr_t align = dtype == kE4M3 ? 8 : 16;
+    const uintptr_t align = (dtype == kE4M3 || dtype == kI8) ? 8 : 16;
     return L.cols % 8 == 0 && row_stride % 8 == 0 && (reinterpret_cast<uintptr_t>(out) % align) == 0;
 }
 
@@ -1096,6 +1107,7 @@ int noalloc_launch(const Params& p, const TableSrc& ts, int out_kind, bool vec, 
         case kOutBF16: return noalloc_launch_out<kOutBF16>(p, ts, vec, esc, st, device);
         case kOutFP16: return noalloc_launch_out<kOutFP16>(p, ts, vec, esc, st, device);
         case kOutE4M3: return noalloc_launch_out<kOutE4M3>(p, ts, vec, esc, st, device);
+        case kOutI8: return noalloc_launch_out<kOutI8>(p, ts, vec, esc, st, device);
         default: return noalloc_launch_out<kOutF32>(p, ts, vec, esc, st, device);
     }
 }
@@ -1244,6 +1256,7 @@ extern "C" int ep_decompress_group(const ep_blob* const* blobs, const ep_tensor*
             case kOutBF16: rc = group_launch_out<kOutBF16>(gp, cta, wide, st, dev); break;
             case kOutFP16: rc = group_launch_out<kOutFP16>(gp, cta, wide, st, dev); break;
             case kOutE4M3: rc = group_launch_out<kOutE4M3>(gp, cta, wide, st, dev); break;
+            case kOutI8: rc = group_launch_out<kOutI8>(gp, cta, wide, st, dev); break;
             default: rc = group_launch_out<kOutF32>(gp, cta, wide, st, dev); break;
         }
         if (rc != EP_OK) return rc;

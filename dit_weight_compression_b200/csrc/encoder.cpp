@@ -70,6 +70,7 @@ public:
             }
             case kFP16: return lut_[reinterpret_cast<const uint16_t*>(base_)[idx]];
             case kE4M3: return lut_[base_[idx]];
+            case kI8: return double(int8_t(base_[idx]));  // two's complement integer
             default: return reinterpret_cast<const float*>(base_)[idx];
         }
     }

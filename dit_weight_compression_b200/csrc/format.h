@@ -41,12 +41,12 @@ constexpr size_t kHeaderBytes = 80;
 constexpr size_t kTileHeadBytes = 4 * kLanes + 2 * kPairs;  // 32 u32 states + 16 u16 counts
 constexpr double kTargetMin = 0.001, kTargetMax = 11.0;
 
-enum Dtype : int { kBF16 = 1, kFP16 = 2, kE4M3 = 3, kF32 = 4 };
+enum Dtype : int { kBF16 = 1, kFP16 = 2, kE4M3 = 3, kF32 = 4, kI8 = 5 };
 
 inline int dtype_bytes(int dt) {
     switch (dt) {
         case kBF16: case kFP16: return 2;
-        case kE4M3: return 1;
+        case kE4M3: case kI8: return 1;
         case kF32: return 4;
         default: return 0;
     }

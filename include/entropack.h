@@ -29,14 +29,16 @@
 extern "C" {
 #endif
 
-/* Element containers.  Decompression keeps the input's dtype by default ("EntroPack lattice
- * compression", opening paragraph: "Decompression retains the input dtype"); the abstract lists
- * BF16, FP16 and FP8 containers.  FP32 is accepted as an extra container. */
+/* Element containers.  By default a tensor is restored in the element type it was compressed
+ * from ("EntroPack lattice compression", opening paragraph); the abstract names BF16, FP16, FP8
+ * and INT8 containers.  FP32 is accepted as an extra container. */
 typedef enum {
     EP_BF16 = 1,
     EP_FP16 = 2,
     EP_FP8_E4M3 = 3,  /* OCP E4M3 (bias 7, no infinities); outputs saturate to +-448 */
-    EP_F32 = 4
+    EP_F32 = 4,
+    EP_INT8 = 5       /* two's complement integers; outputs round to nearest (ties to even) and
+                         saturate to [-128, 127] */
 } ep_dtype;
 
 typedef enum {

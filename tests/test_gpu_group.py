@@ -14,8 +14,9 @@ import workloads as W
 
 pytestmark = pytest.mark.gpu
 
-TORCH = {W.BF16: torch.bfloat16, W.FP16: torch.float16, W.E4M3: torch.float8_e4m3fn, W.F32: torch.float32}
-NP = {W.BF16: np.uint16, W.FP16: np.uint16, W.E4M3: np.uint8, W.F32: np.uint32}
+TORCH = {W.BF16: torch.bfloat16, W.FP16: torch.float16, W.E4M3: torch.float8_e4m3fn, W.F32: torch.float32,
+         W.INT8: torch.int8}
+NP = {W.BF16: np.uint16, W.FP16: np.uint16, W.E4M3: np.uint8, W.F32: np.uint32, W.INT8: np.uint8}
 
 
 @pytest.fixture(scope="module")
@@ -29,7 +30,7 @@ def ep():
 
 
 def _bits(t: torch.Tensor, dtype: int) -> np.ndarray:
-    v = {1: torch.int16, 2: torch.int16, 3: torch.uint8, 4: torch.int32}[dtype]
+    v = {1: torch.int16, 2: torch.int16, 3: torch.uint8, 4: torch.int32, 5: torch.uint8}[dtype]
     return t.contiguous().view(v).cpu().numpy().view(NP[dtype])
 
 
@@ -79,7 +80,7 @@ def _mixed_set(ep):
     return out
 
 
-@pytest.mark.parametrize("dtype", [W.BF16, W.FP16, W.E4M3, W.F32])
+@pytest.mark.parametrize("dtype", [W.BF16, W.FP16, W.E4M3, W.F32, W.INT8])
 def test_group_mixed_set_vs_oracle(ep, dtype):
     mixed = _mixed_set(ep)
     comps = [c for _, c, _ in mixed]

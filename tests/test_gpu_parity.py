@@ -19,8 +19,9 @@ import workloads as W
 
 pytestmark = pytest.mark.gpu
 
-TORCH = {W.BF16: torch.bfloat16, W.FP16: torch.float16, W.E4M3: torch.float8_e4m3fn, W.F32: torch.float32}
-NP = {W.BF16: np.uint16, W.FP16: np.uint16, W.E4M3: np.uint8, W.F32: np.uint32}
+TORCH = {W.BF16: torch.bfloat16, W.FP16: torch.float16, W.E4M3: torch.float8_e4m3fn, W.F32: torch.float32,
+         W.INT8: torch.int8}
+NP = {W.BF16: np.uint16, W.FP16: np.uint16, W.E4M3: np.uint8, W.F32: np.uint32, W.INT8: np.uint8}
 
 
 @pytest.fixture(scope="module")
@@ -34,12 +35,14 @@ def ep():
 
 
 def _bits(t: torch.Tensor, dtype: int) -> np.ndarray:
-    v = {1: torch.int16, 2: torch.int16, 3: torch.uint8, 4: torch.int32}[dtype]
+    v = {1: torch.int16, 2: torch.int16, 3: torch.uint8, 4: torch.int32, 5: torch.uint8}[dtype]
     return t.contiguous().view(v).cpu().numpy().view(NP[dtype])
 
 
 def _ulp(a: np.ndarray, b: np.ndarray, dtype: int) -> np.ndarray:
     """Distance in units in the last place between two arrays of container bit patterns."""
+    if dtype == W.INT8:
+        return np.abs(a.view(np.int8).astype(np.int64) - b.view(np.int8).astype(np.int64))
     nb = {1: 16, 2: 16, 3: 8, 4: 32}[dtype]
     def key(x):
         x = x.astype(np.int64)
@@ -122,7 +125,17 @@ def _check_sampled(ep, c, m: W.Matrix, out_dtypes=None, seed=0):
 def test_small_oracle_blob_all_containers(ep):
     m = W.small()
     blob = oracle.compress(m.bits, m.dtype, m.target_bpp)
-    _check_full(ep, blob, m, [W.BF16, W.FP16, W.E4M3, W.F32])
+    _check_full(ep, blob, m, [W.BF16, W.FP16, W.E4M3, W.F32, W.INT8])
+
+
+def test_int8_container_oracle_blob(ep):
+    """An INT8 input (rows scaled to their absmax) restored as INT8 -- nearest integer, ties to
+    even, saturated -- and, from the same blob, as BF16 and FP32."""
+    m = W.int8()
+    blob = oracle.compress(m.bits, m.dtype, m.target_bpp)
+    assert oracle.blob_info(blob)["dtype"] == W.INT8
+    c = _check_full(ep, blob, m, [W.INT8, W.BF16, W.F32])
+    assert c.dtype == torch.int8
 
 
 def test_square_full_size_oracle_blob(ep):
@@ -153,7 +166,7 @@ def test_ragged_shapes(ep, shape):
     g = np.random.Generator(np.random.PCG64(shape[0] * 1000 + shape[1]))
     m = W.Matrix(W.to_bf16_bits(g.normal(0, 0.02, shape)), W.BF16, 3.0)
     blob = oracle.compress(m.bits, m.dtype, m.target_bpp)
-    _check_full(ep, blob, m, [W.BF16, W.FP16, W.E4M3, W.F32])
+    _check_full(ep, blob, m, [W.BF16, W.FP16, W.E4M3, W.F32, W.INT8])
 
 
 @pytest.mark.parametrize("rate", [0.5, 2.0, 11.0])

@@ -51,6 +51,7 @@ CASES = [
     ("sweep0.5", lambda: W.sweep(0.5, rows=128, cols=1376)),
     ("sweep11", lambda: W.sweep(11.0, rows=64, cols=1376)),
     ("large", lambda: W.large(0, rows=256, cols=1024)),
+    ("int8", lambda: W.int8(rows=256, cols=1024)),
 ]
 
 
@@ -63,10 +64,12 @@ def test_library_blob_equals_oracle_blob(ep, name, make):
 
 
 @pytest.mark.parametrize("shape", [(1, 1), (3, 13), (7, 9), (33, 7), (5, 1000), (2, 4096)])
-@pytest.mark.parametrize("dtype", [W.BF16, W.FP16, W.E4M3, W.F32])
+@pytest.mark.parametrize("dtype", [W.BF16, W.FP16, W.E4M3, W.F32, W.INT8])
 def test_ragged_and_containers_equal_oracle(ep, shape, dtype):
     g = np.random.Generator(np.random.PCG64(shape[0] * 7919 + shape[1] * 31 + dtype))
     x = g.normal(0, 0.05, shape)
+    if dtype == W.INT8:
+        x = x * 1000.0                                  # integers spread over the int8 range
     if dtype == W.E4M3:
         bits = torch.from_numpy(x).to(torch.float8_e4m3fn).view(torch.uint8).numpy()
     else:
