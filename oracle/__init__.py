@@ -44,6 +44,7 @@ def lib() -> ctypes.CDLL:
         P, I64, U64, D, I = ctypes.c_void_p, ctypes.c_int64, ctypes.c_uint64, ctypes.c_double, ctypes.c_int
         sig = {
             "orc_compress": (I, [P, I, I64, I64, D, I64, D, ctypes.POINTER(P), ctypes.POINTER(U64)]),
+            "orc_compress_ex": (I, [P, I, I64, I64, D, I64, D, I, ctypes.POINTER(P), ctypes.POINTER(U64)]),
             "orc_decompress": (I, [P, U64, I, P]),
             "orc_decompress_tiles": (I, [P, U64, I64, I64, I, P]),
             "orc_decode_fields": (I, [P, U64, I64, I64, P]),
@@ -80,14 +81,16 @@ def _buf(b: bytes):
 # ---- codec -------------------------------------------------------------------------------------
 
 def compress(bits: np.ndarray, dtype: int, target_bpp: float, steps_per_tile: int = 0,
-             scale: float = 0.0) -> bytes:
-    """Encode a 2-D array of dtype bit patterns; returns the blob bytes."""
+             scale: float = 0.0, rd_refine: bool = False) -> bytes:
+    """Encode a 2-D array of dtype bit patterns; returns the blob bytes.  rd_refine turns on the
+    per-row rate-distortion refinement (off by default)."""
     bits = np.ascontiguousarray(bits)
     assert bits.ndim == 2 and bits.dtype == NPTYPE[dtype]
     out = ctypes.c_void_p()
     n = ctypes.c_uint64()
-    rc = lib().orc_compress(_ptr(bits), dtype, bits.shape[0], bits.shape[1], float(target_bpp),
-                            int(steps_per_tile), float(scale), ctypes.byref(out), ctypes.byref(n))
+    rc = lib().orc_compress_ex(_ptr(bits), dtype, bits.shape[0], bits.shape[1], float(target_bpp),
+                               int(steps_per_tile), float(scale), int(bool(rd_refine)), ctypes.byref(out),
+                               ctypes.byref(n))
     if rc != 0:
         raise ValueError(f"oracle compress failed: {rc}")
     data = ctypes.string_at(out, n.value)

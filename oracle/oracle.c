@@ -788,6 +788,149 @@ double orc_estimate_bpp(const void* data, int dtype, int64_t rows, int64_t cols,
     return b;
 }
 
+/* ------------------------------------------------------------------------------------------ */
+/* Per-row rate-distortion refinement ([DOC-RS]: optional and off by default; several           */
+/* resolutions are compared for every row and handed out under the estimated storage budget,    */
+/* alternating the choice with updates of the shared probability model).                        */
+/*                                                                                            */
+/* reading: the candidates of row r are s_r = s * 2^(k/2) for k in {0, -1, 1, -2, 2} (in this   */
+/* order, which breaks ties), s the searched shared scale.  For each candidate:                 */
+/*   D = sum over real columns of (w - alpha * y)^2, alpha the row's fp32 least-squares scale   */
+/*       at that resolution (what the decoder multiplies by), in fp64;                          */
+/*   R = sum over the row's symbols of -log2(q / M) under the current tables (log2 M for a      */
+/*       symbol they do not hold) plus 16 bits per escape.                                      */
+/* A round picks k_r = argmin D + lambda R for every row, with lambda = 2^u the smallest, by 64 */
+/* bisection steps on u over [-100, 40], whose total R meets the budget                        */
+/* target * rows * cols - 8 * (metadata bytes, counted as the size estimate counts them); 0 if  */
+/* even the finest choices meet it.  The tables are then rebuilt from the chosen quantisations. */
+/* Three rounds, starting from tables of k = 0 everywhere.  The decode format is unchanged: a   */
+/* row's resolution is absorbed by its least-squares scale.                                     */
+/* ------------------------------------------------------------------------------------------ */
+
+#define RD_NK 5
+#define RD_ROUNDS 3
+static const int rd_k[RD_NK] = {0, -1, 1, -2, 2};
+
+static double rd_resolution(double s, int ki) { return s * exp2(0.5 * rd_k[ki]); }
+
+/* Quantise row r at scale sr: its symbols (vpr x 9) and escape count; returns D. */
+static double rd_row(const matrix* m, int64_t r, double sr, uint8_t* sym, uint64_t* nesc)
+{
+    double swy = 0.0, syy = 0.0;
+    double* ys = (double*)malloc((size_t)m->vpr * 8 * sizeof(double));
+    *nesc = 0;
+    for (int64_t k = 0; k < m->vpr; k++) {
+        int c;
+        int16_t raw[8];
+        quantise_vector(m, r, k, sr, ys + 8 * k, &c);
+        vector_symbols(ys + 8 * k, c, sym + 9 * k, raw);
+        for (int j = 1; j <= 8; j++) *nesc += sym[9 * k + j] == ORC_ESC;
+        for (int i = 0; i < 8; i++)
+            if (8 * k + i < m->cols) {
+                swy += elem(m, r, 8 * k + i) * ys[8 * k + i];
+                syy += ys[8 * k + i] * ys[8 * k + i];
+            }
+    }
+    float a = syy > 0.0 ? (float)(swy / syy) : 0.0f;
+    double d = 0.0;
+    for (int64_t k = 0; k < m->vpr; k++)
+        for (int i = 0; i < 8; i++)
+            if (8 * k + i < m->cols) {
+                double e = elem(m, r, 8 * k + i) - (double)a * ys[8 * k + i];
+                d += e * e;
+            }
+    free(ys);
+    return d;
+}
+
+/* Symbol counts of the rows at their chosen candidates. */
+static void rd_counts(const matrix* m, const uint8_t* sym, const int* kr, uint64_t* cnt)
+{
+    memset(cnt, 0, ORC_NCTX * 256 * sizeof(uint64_t));
+    for (int64_t r = 0; r < m->rows; r++) {
+        const uint8_t* sr = sym + ((size_t)r * RD_NK + (size_t)kr[r]) * (size_t)m->vpr * 9;
+        for (int64_t k = 0; k < m->vpr; k++)
+            for (int u = 0; u <= 8; u++) cnt[256 * context_of(u, sr[9 * k]) + sr[9 * k + u]]++;
+    }
+}
+
+/* Row choices k_r (indexes into rd_k) for the given lambda; returns the total rate. */
+static double rd_choose(const matrix* m, const double* D, const double* R, double lambda, int* kr)
+{
+    double total = 0.0;
+    for (int64_t r = 0; r < m->rows; r++) {
+        int best = 0;
+        double bc = D[r * RD_NK] + lambda * R[r * RD_NK];
+        for (int ki = 1; ki < RD_NK; ki++) {
+            double c = D[r * RD_NK + ki] + lambda * R[r * RD_NK + ki];
+            if (c < bc) { bc = c; best = ki; }
+        }
+        kr[r] = best;
+        total += R[r * RD_NK + best];
+    }
+    return total;
+}
+
+/* The refinement: fills kr[rows] with each row's candidate index.  Returns 0 or -2 (memory). */
+static int rd_allocate(const matrix* m, double s, double target, int64_t S, int* kr)
+{
+    const size_t per = (size_t)m->vpr * 9;
+    uint8_t* sym = (uint8_t*)malloc((size_t)m->rows * RD_NK * per);
+    uint64_t* nesc = (uint64_t*)malloc((size_t)m->rows * RD_NK * sizeof(uint64_t));
+    double* D = (double*)malloc((size_t)m->rows * RD_NK * sizeof(double));
+    double* R = (double*)malloc((size_t)m->rows * RD_NK * sizeof(double));
+    uint64_t* cnt = (uint64_t*)malloc(ORC_NCTX * 256 * sizeof(uint64_t));
+    int rc = 0;
+    if (!sym || !nesc || !D || !R || !cnt) { rc = -2; goto out; }
+    for (int64_t r = 0; r < m->rows; r++)
+        for (int ki = 0; ki < RD_NK; ki++)
+            D[r * RD_NK + ki] = rd_row(m, r, rd_resolution(s, ki), sym + ((size_t)r * RD_NK + ki) * per,
+                                       &nesc[r * RD_NK + ki]);
+    for (int64_t r = 0; r < m->rows; r++) kr[r] = 0;
+    {
+        int64_t V = m->rows * m->vpr;
+        int64_t ntiles = (V + 32 * S - 1) / (32 * S);
+        for (int round = 0; round < RD_ROUNDS; round++) {
+            uint16_t q17[ORC_NCTX * 256];
+            double cost[ORC_NCTX * 256];
+            rd_counts(m, sym, kr, cnt);
+            for (int ctx = 0; ctx < ORC_NCTX; ctx++) orc_quantize_table(cnt + 256 * ctx, q17 + 256 * ctx);
+            for (int i = 0; i < ORC_NCTX * 256; i++)
+                cost[i] = q17[i] ? -log2((double)q17[i] / (double)ORC_M) : log2((double)ORC_M);
+            for (int64_t r = 0; r < m->rows; r++)
+                for (int ki = 0; ki < RD_NK; ki++) {
+                    const uint8_t* sr = sym + ((size_t)r * RD_NK + ki) * per;
+                    double bits = 16.0 * (double)nesc[r * RD_NK + ki];
+                    for (int64_t k = 0; k < m->vpr; k++)
+                        for (int u = 0; u <= 8; u++) bits += cost[256 * context_of(u, sr[9 * k]) + sr[9 * k + u]];
+                    R[r * RD_NK + ki] = bits;
+                }
+            double meta = (double)(ORC_HEADER + pad16(table_section_bytes(q17)) + pad16(4u * (uint64_t)m->rows) +
+                                   pad16(4u * (uint64_t)(ntiles + 1))) +
+                          (double)ntiles * (160.0 + 8.0);
+            double budget = target * (double)m->rows * (double)m->cols - 8.0 * meta;
+            if (rd_choose(m, D, R, 0.0, kr) > budget) {
+                double lo = -100.0, hi = 40.0;
+                if (rd_choose(m, D, R, exp2(hi), kr) <= budget) {
+                    for (int it = 0; it < 64; it++) {
+                        double mid = 0.5 * (lo + hi);
+                        if (rd_choose(m, D, R, exp2(mid), kr) <= budget) hi = mid;
+                        else lo = mid;
+                    }
+                }
+                rd_choose(m, D, R, exp2(hi), kr);
+            }
+        }
+    }
+out:
+    free(sym);
+    free(nesc);
+    free(D);
+    free(R);
+    free(cnt);
+    return rc;
+}
+
 /*
  * Compress a rows x cols matrix stored as dtype bits.  steps_per_tile = 0 selects the default S;
  * scale_override > 0 skips the search.  On success *blob is a malloc'd byte string of *len bytes.
@@ -803,8 +946,9 @@ double orc_estimate_bpp(const void* data, int dtype, int64_t rows, int64_t cols,
  *   tile offsets: u32[n_tiles + 1], in 16-byte units from the stream section start;
  *   stream: the tiles.
  */
-int orc_compress(const void* data, int dtype, int64_t rows, int64_t cols, double target_bpp,
-                 int64_t steps_per_tile, double scale_override, uint8_t** blob, uint64_t* len)
+int orc_compress_ex(const void* data, int dtype, int64_t rows, int64_t cols, double target_bpp,
+                    int64_t steps_per_tile, double scale_override, int rd_refine, uint8_t** blob,
+                    uint64_t* len)
 {
     *blob = NULL;
     *len = 0;
@@ -817,6 +961,11 @@ int orc_compress(const void* data, int dtype, int64_t rows, int64_t cols, double
     if (steps_per_tile > 1024) { free_matrix(&m); return -4; }   /* region counts are u16 */
     int64_t S = steps_per_tile > 0 ? steps_per_tile : default_steps(target_bpp);
     double s = scale_override > 0 ? scale_override : choose_scale(&m, target_bpp, S);
+    int* kr = NULL;                      /* per-row candidate of the refinement, when enabled */
+    if (rd_refine) {
+        kr = (int*)malloc((size_t)rows * sizeof(int));
+        if (!kr || rd_allocate(&m, s, target_bpp, S, kr)) { free(kr); free_matrix(&m); return -2; }
+    }
 
     /* Quantise the whole tensor at s; fit one least-squares scale per row ([DOC-RS]: with s
      * fixed, every row is quantised and gets its own reconstruction scale by least squares):
@@ -832,7 +981,7 @@ int orc_compress(const void* data, int dtype, int64_t rows, int64_t cols, double
             double y[8];
             int c;
             int64_t v = r * m.vpr + k;
-            quantise_vector(&m, r, k, s, y, &c);
+            quantise_vector(&m, r, k, kr ? rd_resolution(s, kr[r]) : s, y, &c);
             vector_symbols(y, c, sym9 + 9 * v, raw8 + 8 * v);
             for (int i = 0; i < 8; i++)
                 if (8 * k + i < cols) {
@@ -921,6 +1070,7 @@ int orc_compress(const void* data, int dtype, int64_t rows, int64_t cols, double
         *len = total;
     }
 done:
+    free(kr);
     free(tsize);
     free(sym9);
     free(raw8);
@@ -928,6 +1078,13 @@ done:
     free(cnt);
     free_matrix(&m);
     return rc;
+}
+
+/* orc_compress_ex with the refinement off (the default). */
+int orc_compress(const void* data, int dtype, int64_t rows, int64_t cols, double target_bpp,
+                 int64_t steps_per_tile, double scale_override, uint8_t** blob, uint64_t* len)
+{
+    return orc_compress_ex(data, dtype, rows, cols, target_bpp, steps_per_tile, scale_override, 0, blob, len);
 }
 
 /* ------------------------------------------------------------------------------------------ */
