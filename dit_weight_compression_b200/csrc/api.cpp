@@ -77,6 +77,7 @@ extern "C" int ep_compress_ex(const ep_tensor* in, double target_bpp, const ep_o
         o.steps_per_tile = opt->steps_per_tile;
         o.threads = opt->num_threads;
         o.scale = opt->scale;
+        o.rd_refine = opt->rd_refine != 0;
     }
     ep_blob* b = new (std::nothrow) ep_blob();
     if (!b) return set_error(EP_ERR_OOM, "ep_compress: blob");

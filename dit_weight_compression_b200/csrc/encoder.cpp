@@ -306,6 +306,130 @@ static void encode_tile(const uint8_t* coset, const int16_t* fields, int64_t nve
 // ---------------------------------------------------------------------------------------------
 // The encoder.
 // ---------------------------------------------------------------------------------------------
+// ---------------------------------------------------------------------------------------------
+// Per-row rate-distortion refinement ("EntroPack lattice compression", section "Rate selection
+// and refinement": optional, off by default; several resolutions are compared per row and handed
+// out under the estimated storage budget, alternating with updates of the shared tables).
+// Candidates s * 2^(k/2) for k in {0, -1, 1, -2, 2} (this order breaks ties).  Per candidate:
+// D = sum over real columns of (w - alpha y)^2 with alpha the row's fp32 least-squares scale, and
+// R = the row's code length under the current tables (log2 M bits for a symbol they do not hold)
+// plus 16 bits per escape.  A round picks argmin D + lambda R per row, lambda = 2^u the smallest
+// (64 bisection steps on u over [-100, 40]) whose total R meets target * N - 8 * metadata bytes;
+// then the tables are rebuilt from the chosen rows.  Three rounds from tables of k = 0.
+// ---------------------------------------------------------------------------------------------
+constexpr int kRdCandidates = 5, kRdRounds = 3;
+constexpr int kRdK[kRdCandidates] = {0, -1, 1, -2, 2};
+
+static double rd_resolution(double s, int ki) { return s * std::exp2(0.5 * kRdK[ki]); }
+
+static std::vector<int> rd_allocate(const ElementReader& rd, const Quantiser& Q, int64_t rows, int64_t cols,
+                                    int64_t vpr, double s, double target, int64_t n_tiles, int threads) {
+    const size_t per = size_t(vpr) * 9, R5 = size_t(kRdCandidates);
+    std::vector<uint8_t> sym(size_t(rows) * R5 * per);
+    std::vector<uint64_t> nesc(size_t(rows) * R5);
+    std::vector<double> D(size_t(rows) * R5), R(size_t(rows) * R5);
+    parallel_for(rows, threads, [&](int64_t a, int64_t b, int) {
+        QVec q;
+        std::vector<double> ys(size_t(vpr) * 8);
+        for (int64_t r = a; r < b; ++r)
+            for (int ki = 0; ki < kRdCandidates; ++ki) {
+                const size_t idx = size_t(r) * R5 + size_t(ki);
+                uint8_t* sy = &sym[idx * per];
+                uint64_t ne = 0;
+                double swy = 0.0, syy = 0.0;
+                for (int64_t k = 0; k < vpr; ++k) {
+                    Q.quantise(r, k, rd_resolution(s, ki), q);
+                    sy[9 * k] = uint8_t(q.coset);
+                    for (int j = 0; j < 8; ++j) {
+                        sy[9 * k + 1 + j] = uint8_t(symbol_of(q.f[j]));
+                        ne += sy[9 * k + 1 + j] == kEscape;
+                    }
+                    for (int i = 0; i < 8; ++i) {
+                        ys[size_t(8 * k + i)] = q.y[i];
+                        if (8 * k + i < cols) {
+                            swy += rd.at(r, 8 * k + i) * q.y[i];
+                            syy += q.y[i] * q.y[i];
+                        }
+                    }
+                }
+                const float al = syy > 0.0 ? float(swy / syy) : 0.0f;
+                double d = 0.0;
+                for (int64_t k = 0; k < vpr; ++k)
+                    for (int i = 0; i < 8; ++i)
+                        if (8 * k + i < cols) {
+                            double e = rd.at(r, 8 * k + i) - double(al) * ys[size_t(8 * k + i)];
+                            d += e * e;
+                        }
+                D[idx] = d;
+                nesc[idx] = ne;
+            }
+    });
+    std::vector<int> kr(static_cast<size_t>(rows), 0);
+    auto choose = [&](double lambda) {
+        double total = 0.0;
+        for (int64_t r = 0; r < rows; ++r) {
+            const size_t b0 = size_t(r) * R5;
+            int best = 0;
+            double bc = D[b0] + lambda * R[b0];
+            for (int ki = 1; ki < kRdCandidates; ++ki) {
+                double c = D[b0 + size_t(ki)] + lambda * R[b0 + size_t(ki)];
+                if (c < bc) { bc = c; best = ki; }
+            }
+            kr[size_t(r)] = best;
+            total += R[b0 + size_t(best)];
+        }
+        return total;
+    };
+    for (int round = 0; round < kRdRounds; ++round) {
+        Counts all;
+        for (int64_t r = 0; r < rows; ++r) {
+            const uint8_t* sy = &sym[(size_t(r) * R5 + size_t(kr[size_t(r)])) * per];
+            for (int64_t k = 0; k < vpr; ++k) {
+                const int c = sy[9 * k];
+                all.c[size_t(c)]++;
+                for (int j = 0; j < 8; ++j) all.c[size_t(256 * (1 + 8 * c + j) + sy[9 * k + 1 + j])]++;
+            }
+        }
+        Tables T;
+        T.build(all);
+        double cost[17 * 256];
+        for (int c = 0; c < 17; ++c)
+            for (int sy = 0; sy < 256; ++sy)
+                cost[256 * c + sy] = T.q[c][sy] ? -std::log2(double(T.q[c][sy]) / double(kProbTotal))
+                                                : std::log2(double(kProbTotal));
+        parallel_for(rows, threads, [&](int64_t a, int64_t b, int) {
+            for (int64_t r = a; r < b; ++r)
+                for (int ki = 0; ki < kRdCandidates; ++ki) {
+                    const size_t idx = size_t(r) * R5 + size_t(ki);
+                    const uint8_t* sy = &sym[idx * per];
+                    double bits = 16.0 * double(nesc[idx]);
+                    for (int64_t k = 0; k < vpr; ++k) {
+                        const int c = sy[9 * k];
+                        bits += cost[sy[9 * k]];
+                        for (int j = 0; j < 8; ++j) bits += cost[256 * (1 + 8 * c + j) + sy[9 * k + 1 + j]];
+                    }
+                    R[idx] = bits;
+                }
+        });
+        const double meta = double(kHeaderBytes + round_up16(T.section_bytes()) + round_up16(4 * uint64_t(rows)) +
+                                   round_up16(4 * uint64_t(n_tiles + 1))) +
+                            double(n_tiles) * (160.0 + 8.0);
+        const double budget = target * double(rows) * double(cols) - 8.0 * meta;
+        if (choose(0.0) > budget) {
+            double lo = -100.0, hi = 40.0;
+            if (choose(std::exp2(hi)) <= budget) {
+                for (int it = 0; it < 64; ++it) {
+                    double mid = 0.5 * (lo + hi);
+                    if (choose(std::exp2(mid)) <= budget) hi = mid;
+                    else lo = mid;
+                }
+            }
+            choose(std::exp2(hi));
+        }
+    }
+    return kr;
+}
+
 static int default_steps(double target) {
     double want = std::ceil(128.0 / target);
     int s = 1;
@@ -342,7 +466,7 @@ int encode(const EncodeInput& in, double target, const EncodeOptions& opt, std::
     if (n_tiles > int64_t(UINT32_MAX) - 1) { why = "too many tiles"; return -3; }
 
     // Size estimate at scale s from min(rows, 256) rows at floor(i * rows / n): coded bits under
-    // the sample's own 12-bit tables plus 16 bits per escape, scaled to all rows, plus the exact
+    // the sample's own 10-bit tables plus 16 bits per escape, scaled to all rows, plus the exact
     // metadata (header, tables, row scales, tile offsets) and 168 bytes per tile (32 states, 16
     // region counts and the mean padding).
     const int64_t n_sample = std::min<int64_t>(rows, 256);
@@ -393,6 +517,10 @@ int encode(const EncodeInput& in, double target, const EncodeOptions& opt, std::
         }
     }
 
+    // Optional per-row resolutions (the rate-distortion refinement).
+    std::vector<int> kr;
+    if (opt.rd_refine) kr = rd_allocate(rd, Q, rows, cols, vpr, s, target, n_tiles, threads);
+
     // Full quantisation, least-squares row scales alpha_r = sum w y / sum y^2 (real columns).
     std::vector<uint8_t> coset(static_cast<size_t>(V));
     std::vector<int16_t> fields(static_cast<size_t>(V) * 8);
@@ -402,8 +530,9 @@ int encode(const EncodeInput& in, double target, const EncodeOptions& opt, std::
         QVec q;
         for (int64_t r = a; r < b; ++r) {
             double swy = 0.0, syy = 0.0;
+            const double sr = kr.empty() ? s : rd_resolution(s, kr[size_t(r)]);
             for (int64_t k = 0; k < vpr; ++k) {
-                Q.quantise(r, k, s, q);
+                Q.quantise(r, k, sr, q);
                 int64_t v = r * vpr + k;
                 coset[size_t(v)] = uint8_t(q.coset);
                 for (int j = 0; j < 8; ++j) fields[size_t(8 * v + j)] = int16_t(q.f[j]);

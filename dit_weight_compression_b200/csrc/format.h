@@ -93,6 +93,7 @@ struct EncodeOptions {
     int steps_per_tile = 0;  // S; 0 = default rule
     int threads = 0;         // 0 = all hardware threads
     double scale = 0.0;      // > 0: skip the scale search
+    bool rd_refine = false;  // per-row rate-distortion refinement
 };
 // Returns 0, -3 (shape/size limits) or -4 (non-finite input); `why` explains a failure.
 int encode(const EncodeInput& in, double target, const EncodeOptions& opt, std::vector<uint8_t>& blob,

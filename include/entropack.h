@@ -67,6 +67,11 @@ typedef struct {
     int steps_per_tile;  /* S in [1, 1024]: tile = 32*S vectors; 0 = clamp(next_pow2(ceil(128/bpp)), 16, 1024) */
     int num_threads;     /* host encoder threads; 0 = all hardware threads                       */
     double scale;        /* > 0: use this lattice scale instead of searching for one             */
+    int rd_refine;       /* nonzero: per-row rate-distortion refinement ("Rate selection and
+                            refinement": optional, off by default) -- every row picks one of five
+                            resolutions s * 2^(k/2), k in {0, -1, 1, -2, 2}, by a Lagrangian
+                            choice under the storage budget, in three rounds that rebuild the
+                            probability tables; the decode format does not change           */
 } ep_options;
 
 typedef struct ep_blob ep_blob;

@@ -128,6 +128,14 @@ def test_small_oracle_blob_all_containers(ep):
     _check_full(ep, blob, m, [W.BF16, W.FP16, W.E4M3, W.F32, W.INT8])
 
 
+def test_rd_refined_oracle_blob(ep):
+    """A blob made with the per-row rate-distortion refinement (rows at different resolutions,
+    the decode format unchanged) decodes as the oracle decodes it."""
+    m = W.square(rows=512, cols=1024)
+    blob = oracle.compress(m.bits, m.dtype, m.target_bpp, rd_refine=True)
+    _check_full(ep, blob, m, [W.BF16, W.F32])
+
+
 def test_int8_container_oracle_blob(ep):
     """An INT8 input (rows scaled to their absmax) restored as INT8 -- nearest integer, ties to
     even, saturated -- and, from the same blob, as BF16 and FP32."""

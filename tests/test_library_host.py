@@ -63,6 +63,19 @@ def test_library_blob_equals_oracle_blob(ep, name, make):
     assert lb == ob
 
 
+@pytest.mark.parametrize("name,make", [CASES[1], CASES[2], CASES[4], ("ragged", lambda: W.small(rows=37, cols=203))],
+                         ids=["square", "dit", "sweep11", "ragged"])
+def test_rd_refined_blob_equals_oracle_blob(ep, name, make):
+    """The optional per-row rate-distortion refinement: library and oracle blobs byte-identical,
+    and the thread count does not change the bytes."""
+    m = make()
+    ob = oracle.compress(m.bits, m.dtype, m.target_bpp, rd_refine=True)
+    for threads in (1, 5):
+        cfg = ep.LatticeRANSConfig(m.target_bpp, num_threads=threads, rd_refine=True)
+        lb = ep.compress(W.bits_to_torch(m.bits, m.dtype), cfg).to_bytes()
+        assert lb == ob
+
+
 @pytest.mark.parametrize("shape", [(1, 1), (3, 13), (7, 9), (33, 7), (5, 1000), (2, 4096)])
 @pytest.mark.parametrize("dtype", [W.BF16, W.FP16, W.E4M3, W.F32, W.INT8])
 def test_ragged_and_containers_equal_oracle(ep, shape, dtype):
