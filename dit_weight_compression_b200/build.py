@@ -16,7 +16,7 @@ ROOT = os.path.dirname(PKG)
 CSRC = os.path.join(PKG, "csrc")
 LIB = os.path.join(PKG, "libentropack.so")
 SOURCES = ["api.cpp", "encoder.cpp", "decode.cu"]
-HEADERS = ["format.h", "blob.h"]
+HEADERS = ["format.h", "blob.h", "tables.h"]
 
 
 def nvcc() -> str:

@@ -23,6 +23,7 @@
 #include <thread>
 
 #include "format.h"
+#include "tables.h"
 
 namespace ep {
 
@@ -171,86 +172,6 @@ private:
     const ElementReader& rd_;
     int64_t rows_, cols_;
     const std::vector<double>& rms_;
-};
-
-static inline int symbol_of(int32_t f) { return (f >= -kAlphabetR && f <= kAlphabetR) ? f + kAlphabetR : kEscape; }
-
-// Symbol counts of the 17 contexts: [0] the coset (symbols 0/1), [1 + 8c + j - 1] field j | c.
-struct Counts {
-    std::vector<uint64_t> c = std::vector<uint64_t>(17 * 256, 0);
-    uint64_t escapes = 0;
-    void add(const QVec& q) {
-        c[size_t(q.coset)]++;
-        for (int j = 0; j < 8; ++j) {
-            int sy = symbol_of(q.f[j]);
-            c[size_t(256 * (1 + 8 * q.coset + j) + sy)]++;
-            escapes += sy == kEscape;
-        }
-    }
-    void merge(const Counts& o) {
-        for (size_t i = 0; i < c.size(); ++i) c[i] += o.c[i];
-        escapes += o.escapes;
-    }
-};
-
-// 10-bit frequencies from counts: q = max(1, round-half-up(M n / N)) for used symbols, then
-// the sum is brought to M -- excess taken one at a time from the largest q (> 1, lowest symbol
-// first), deficit given one at a time to the most frequent symbol (lowest symbol first).
-static void quantise_freqs(const uint64_t* n, uint16_t* q) {
-    uint64_t total = 0;
-    for (int s = 0; s < 256; ++s) total += n[s];
-    std::fill(q, q + 256, uint16_t(0));
-    if (total == 0) return;
-    int64_t sum = 0;
-    for (int s = 0; s < 256; ++s) {
-        if (!n[s]) continue;
-        uint64_t v = (2 * uint64_t(kProbTotal) * n[s] + total) / (2 * total);
-        q[s] = uint16_t(std::max<uint64_t>(v, 1));
-        sum += q[s];
-    }
-    while (sum > int64_t(kProbTotal)) {
-        int best = -1;
-        for (int s = 0; s < 256; ++s)
-            if (q[s] > 1 && (best < 0 || q[s] > q[best])) best = s;
-        --q[best];
-        --sum;
-    }
-    while (sum < int64_t(kProbTotal)) {
-        int best = -1;
-        for (int s = 0; s < 256; ++s)
-            if (n[s] && (best < 0 || n[s] > n[best])) best = s;
-        ++q[best];
-        ++sum;
-    }
-}
-
-struct Tables {
-    uint16_t q[17][256];
-    uint32_t cum[17][257];
-    void build(const Counts& cnt) {
-        for (int c = 0; c < 17; ++c) {
-            quantise_freqs(&cnt.c[size_t(256 * c)], q[c]);
-            cum[c][0] = 0;
-            for (int s = 0; s < 256; ++s) cum[c][s + 1] = cum[c][s] + q[c][s];
-        }
-    }
-    // serialised size of the table section (before padding)
-    uint64_t section_bytes() const {
-        uint64_t b = 4;
-        for (int c = 1; c < 17; ++c) {
-            int lo, cnt;
-            range(c, lo, cnt);
-            b += 4 + 2 * uint64_t(cnt);
-        }
-        return b;
-    }
-    void range(int c, int& lo, int& cnt) const {
-        int first = -1, last = -1;
-        for (int s = 0; s < kEscape; ++s)
-            if (q[c][s]) { if (first < 0) first = s; last = s; }
-        lo = first < 0 ? 0 : first;
-        cnt = first < 0 ? 0 : last - first + 1;
-    }
 };
 
 // ---------------------------------------------------------------------------------------------
@@ -430,11 +351,59 @@ static std::vector<int> rd_allocate(const ElementReader& rd, const Quantiser& Q,
     return kr;
 }
 
-static int default_steps(double target) {
-    double want = std::ceil(128.0 / target);
-    int s = 1;
-    while (double(s) < want) s *= 2;
-    return std::min(1024, std::max(16, s));
+
+bool assemble_blob(int dtype, int64_t rows, int64_t cols, int S, double s, const Tables& T,
+                   const std::vector<float>& alpha, const std::vector<uint64_t>& tile_bytes,
+                   std::vector<uint8_t>& blob, uint64_t* off_stream_out, std::string& why) {
+    const int64_t n_tiles = int64_t(tile_bytes.size());
+    uint64_t tab = T.section_bytes();
+    uint64_t off_tab = kHeaderBytes, off_alpha = off_tab + round_up16(tab);
+    uint64_t off_offs = off_alpha + round_up16(4 * uint64_t(rows));
+    uint64_t off_stream = off_offs + round_up16(4 * uint64_t(n_tiles + 1));
+    uint64_t stream = 0;
+    for (uint64_t t : tile_bytes) stream += t;
+    if (stream / 16 > UINT32_MAX) { why = "stream exceeds the 64 GiB tile-offset range"; return false; }
+    blob.assign(size_t(off_stream + stream), 0);
+    uint8_t* p = blob.data();
+    std::memcpy(p, "EPK1", 4);
+    wr16(p + 4, kVersion);
+    p[6] = uint8_t(dtype);
+    p[7] = uint8_t(kAlphabetR);
+    wr64(p + 8, uint64_t(rows));
+    wr64(p + 16, uint64_t(cols));
+    wr32(p + 24, uint32_t(S));
+    wr32(p + 28, uint32_t(n_tiles));
+    std::memcpy(p + 32, &s, 8);
+    wr64(p + 40, blob.size());
+    wr64(p + 48, off_tab);
+    wr64(p + 56, off_alpha);
+    wr64(p + 64, off_offs);
+    wr64(p + 72, off_stream);
+    uint8_t* t = p + off_tab;
+    wr16(t, T.q[0][0]);
+    wr16(t + 2, T.q[0][1]);
+    t += 4;
+    for (int c = 1; c < 17; ++c) {
+        int lo, cnt;
+        T.range(c, lo, cnt);
+        wr16(t, T.q[c][kEscape]);
+        t[2] = uint8_t(lo);
+        t[3] = uint8_t(cnt);
+        t += 4;
+        for (int i = 0; i < cnt; ++i, t += 2) wr16(t, T.q[c][lo + i]);
+    }
+    for (int64_t r = 0; r < rows; ++r) {
+        uint32_t bitsf;
+        std::memcpy(&bitsf, &alpha[size_t(r)], 4);
+        wr32(p + off_alpha + 4 * r, bitsf);
+    }
+    uint64_t acc = 0;
+    for (int64_t i = 0; i <= n_tiles; ++i) {
+        wr32(p + off_offs + 4 * i, uint32_t(acc / 16));
+        if (i < n_tiles) acc += tile_bytes[size_t(i)];
+    }
+    *off_stream_out = off_stream;
+    return true;
 }
 
 int encode(const EncodeInput& in, double target, const EncodeOptions& opt, std::vector<uint8_t>& blob,
@@ -465,10 +434,7 @@ int encode(const EncodeInput& in, double target, const EncodeOptions& opt, std::
     const int64_t n_tiles = (V + per_tile - 1) / per_tile;
     if (n_tiles > int64_t(UINT32_MAX) - 1) { why = "too many tiles"; return -3; }
 
-    // Size estimate at scale s from min(rows, 256) rows at floor(i * rows / n): coded bits under
-    // the sample's own 10-bit tables plus 16 bits per escape, scaled to all rows, plus the exact
-    // metadata (header, tables, row scales, tile offsets) and 168 bytes per tile (32 states, 16
-    // region counts and the mean padding).
+    // Size estimate at scale s from min(rows, 256) rows at floor(i * rows / n) (tables.h).
     const int64_t n_sample = std::min<int64_t>(rows, 256);
     auto estimate = [&](double s) {
         std::vector<Counts> part(static_cast<size_t>(threads));
@@ -478,25 +444,13 @@ int encode(const EncodeInput& in, double target, const EncodeOptions& opt, std::
                 int64_t r = (i * rows) / n_sample;
                 for (int64_t k = 0; k < vpr; ++k) {
                     Q.quantise(r, k, s, q);
-                    part[size_t(t)].add(q);
+                    part[size_t(t)].add(q.coset, q.f);
                 }
             }
         });
         Counts all;
         for (auto& p : part) all.merge(p);
-        Tables T;
-        T.build(all);
-        double bits = 0.0;
-        for (int c = 0; c < 17; ++c)
-            for (int sy = 0; sy < 256; ++sy) {
-                uint64_t n = all.c[size_t(256 * c + sy)];
-                if (n) bits += double(n) * -std::log2(double(T.q[c][sy]) / double(kProbTotal));
-            }
-        double payload = (double(rows) / double(n_sample)) * (bits / 8.0 + 2.0 * double(all.escapes));
-        double meta = double(kHeaderBytes + round_up16(T.section_bytes()) + round_up16(4 * uint64_t(rows)) +
-                             round_up16(4 * uint64_t(n_tiles + 1))) +
-                      double(n_tiles) * (160.0 + 8.0);
-        return 8.0 * (meta + payload) / (double(rows) * double(cols));
+        return estimate_from_counts(all, rows, cols, n_sample, n_tiles);
     };
 
     // Finest scale whose estimate meets the target: bisection on log2 s over [-24, 8].
@@ -541,7 +495,7 @@ int encode(const EncodeInput& in, double target, const EncodeOptions& opt, std::
                         swy += rd.at(r, 8 * k + i) * q.y[i];
                         syy += q.y[i] * q.y[i];
                     }
-                part[size_t(t)].add(q);
+                part[size_t(t)].add(q.coset, q.f);
             }
             alpha[size_t(r)] = syy > 0.0 ? float(swy / syy) : 0.0f;
         }
@@ -561,55 +515,13 @@ int encode(const EncodeInput& in, double target, const EncodeOptions& opt, std::
     });
 
     // Serialise.
-    uint64_t tab = T.section_bytes();
-    uint64_t off_tab = kHeaderBytes, off_alpha = off_tab + round_up16(tab);
-    uint64_t off_offs = off_alpha + round_up16(4 * uint64_t(rows));
-    uint64_t off_stream = off_offs + round_up16(4 * uint64_t(n_tiles + 1));
-    uint64_t stream = 0;
-    for (auto& t : tiles) stream += t.size();
-    if (stream / 16 > UINT32_MAX) { why = "stream exceeds the 64 GiB tile-offset range"; return -3; }
-    blob.assign(size_t(off_stream + stream), 0);
-    uint8_t* p = blob.data();
-    std::memcpy(p, "EPK1", 4);
-    wr16(p + 4, kVersion);
-    p[6] = uint8_t(in.dtype);
-    p[7] = uint8_t(kAlphabetR);
-    wr64(p + 8, uint64_t(rows));
-    wr64(p + 16, uint64_t(cols));
-    wr32(p + 24, uint32_t(S));
-    wr32(p + 28, uint32_t(n_tiles));
-    std::memcpy(p + 32, &s, 8);
-    wr64(p + 40, blob.size());
-    wr64(p + 48, off_tab);
-    wr64(p + 56, off_alpha);
-    wr64(p + 64, off_offs);
-    wr64(p + 72, off_stream);
-    uint8_t* t = p + off_tab;
-    wr16(t, T.q[0][0]);
-    wr16(t + 2, T.q[0][1]);
-    t += 4;
-    for (int c = 1; c < 17; ++c) {
-        int lo, cnt;
-        T.range(c, lo, cnt);
-        wr16(t, T.q[c][kEscape]);
-        t[2] = uint8_t(lo);
-        t[3] = uint8_t(cnt);
-        t += 4;
-        for (int i = 0; i < cnt; ++i, t += 2) wr16(t, T.q[c][lo + i]);
-    }
-    for (int64_t r = 0; r < rows; ++r) {
-        uint32_t bitsf;
-        std::memcpy(&bitsf, &alpha[size_t(r)], 4);
-        wr32(p + off_alpha + 4 * r, bitsf);
-    }
+    std::vector<uint64_t> sizes(static_cast<size_t>(n_tiles));
+    for (int64_t i = 0; i < n_tiles; ++i) sizes[size_t(i)] = tiles[size_t(i)].size();
+    uint64_t off_stream = 0;
+    if (!assemble_blob(in.dtype, rows, cols, S, s, T, alpha, sizes, blob, &off_stream, why)) return -3;
     uint64_t acc = 0;
-    for (int64_t i = 0; i <= n_tiles; ++i) {
-        wr32(p + off_offs + 4 * i, uint32_t(acc / 16));
-        if (i < n_tiles) acc += tiles[size_t(i)].size();
-    }
-    acc = 0;
     for (auto& tb : tiles) {
-        std::memcpy(p + off_stream + acc, tb.data(), tb.size());
+        std::memcpy(blob.data() + off_stream + acc, tb.data(), tb.size());
         acc += tb.size();
     }
     return 0;

@@ -1,0 +1,132 @@
+// tables.h -- pieces both encoders (host threads, GPU) share: symbols, symbol counts, the 10-bit
+// frequency tables built from them, the default tile length, the sampled size estimate and the
+// blob serialiser.  One definition, so the two encoders cannot drift apart.
+#pragma once
+
+#include <algorithm>
+#include <cmath>
+#include <cstdint>
+#include <string>
+#include <vector>
+
+#include "format.h"
+
+namespace ep {
+
+// Field value -> symbol: f + 127 for |f| <= 127, else the escape symbol.
+inline int symbol_of(int32_t f) { return (f >= -kAlphabetR && f <= kAlphabetR) ? f + kAlphabetR : kEscape; }
+
+// Symbol counts of the 17 contexts: [0] the coset (symbols 0/1), [1 + 8c + j - 1] field j | c.
+struct Counts {
+    std::vector<uint64_t> c = std::vector<uint64_t>(17 * 256, 0);
+    uint64_t escapes = 0;
+    void add(int coset, const int32_t f[8]) {
+        c[size_t(coset)]++;
+        for (int j = 0; j < 8; ++j) {
+            int sy = symbol_of(f[j]);
+            c[size_t(256 * (1 + 8 * coset + j) + sy)]++;
+            escapes += sy == kEscape;
+        }
+    }
+    void merge(const Counts& o) {
+        for (size_t i = 0; i < c.size(); ++i) c[i] += o.c[i];
+        escapes += o.escapes;
+    }
+};
+
+// 10-bit frequencies from counts: q = max(1, round-half-up(M n / N)) for used symbols, then
+// the sum is brought to M -- excess taken one at a time from the largest q (> 1, lowest symbol
+// first), deficit given one at a time to the most frequent symbol (lowest symbol first).
+inline void quantise_freqs(const uint64_t* n, uint16_t* q) {
+    uint64_t total = 0;
+    for (int s = 0; s < 256; ++s) total += n[s];
+    std::fill(q, q + 256, uint16_t(0));
+    if (total == 0) return;
+    int64_t sum = 0;
+    for (int s = 0; s < 256; ++s) {
+        if (!n[s]) continue;
+        uint64_t v = (2 * uint64_t(kProbTotal) * n[s] + total) / (2 * total);
+        q[s] = uint16_t(std::max<uint64_t>(v, 1));
+        sum += q[s];
+    }
+    while (sum > int64_t(kProbTotal)) {
+        int best = -1;
+        for (int s = 0; s < 256; ++s)
+            if (q[s] > 1 && (best < 0 || q[s] > q[best])) best = s;
+        --q[best];
+        --sum;
+    }
+    while (sum < int64_t(kProbTotal)) {
+        int best = -1;
+        for (int s = 0; s < 256; ++s)
+            if (n[s] && (best < 0 || n[s] > n[best])) best = s;
+        ++q[best];
+        ++sum;
+    }
+}
+
+struct Tables {
+    uint16_t q[17][256];
+    uint32_t cum[17][257];
+    void build(const Counts& cnt) {
+        for (int c = 0; c < 17; ++c) {
+            quantise_freqs(&cnt.c[size_t(256 * c)], q[c]);
+            cum[c][0] = 0;
+            for (int s = 0; s < 256; ++s) cum[c][s + 1] = cum[c][s] + q[c][s];
+        }
+    }
+    // serialised size of the table section (before padding)
+    uint64_t section_bytes() const {
+        uint64_t b = 4;
+        for (int c = 1; c < 17; ++c) {
+            int lo, cnt;
+            range(c, lo, cnt);
+            b += 4 + 2 * uint64_t(cnt);
+        }
+        return b;
+    }
+    void range(int c, int& lo, int& cnt) const {
+        int first = -1, last = -1;
+        for (int s = 0; s < kEscape; ++s)
+            if (q[c][s]) { if (first < 0) first = s; last = s; }
+        lo = first < 0 ? 0 : first;
+        cnt = first < 0 ? 0 : last - first + 1;
+    }
+};
+
+// Default tile length: S = clamp(next_pow2(ceil(128 / target)), 16, 1024).
+inline int default_steps(double target) {
+    double want = std::ceil(128.0 / target);
+    int s = 1;
+    while (double(s) < want) s *= 2;
+    return std::min(1024, std::max(16, s));
+}
+
+// Estimated bits per element from the symbol counts of n_sample sampled rows (of `rows`): coded
+// bits under the sample's own tables plus 16 bits per escape, scaled to all rows, plus the exact
+// metadata (header, tables, row scales, tile offsets) and 168 bytes per tile (32 states, 16
+// region counts and the mean padding).
+inline double estimate_from_counts(const Counts& all, int64_t rows, int64_t cols, int64_t n_sample, int64_t n_tiles) {
+    Tables T;
+    T.build(all);
+    double bits = 0.0;
+    for (int c = 0; c < 17; ++c)
+        for (int sy = 0; sy < 256; ++sy) {
+            uint64_t n = all.c[size_t(256 * c + sy)];
+            if (n) bits += double(n) * -std::log2(double(T.q[c][sy]) / double(kProbTotal));
+        }
+    double payload = (double(rows) / double(n_sample)) * (bits / 8.0 + 2.0 * double(all.escapes));
+    double meta = double(kHeaderBytes + round_up16(T.section_bytes()) + round_up16(4 * uint64_t(rows)) +
+                         round_up16(4 * uint64_t(n_tiles + 1))) +
+                  double(n_tiles) * (160.0 + 8.0);
+    return 8.0 * (meta + payload) / (double(rows) * double(cols));
+}
+
+// Write the blob: header, table section, row scales, tile offsets (from the tile byte sizes) and
+// room for the stream.  The stream's bytes are left zero; its offset is returned in *off_stream.
+// Returns false (with `why`) when the stream would exceed the tile-offset range.
+bool assemble_blob(int dtype, int64_t rows, int64_t cols, int S, double s, const Tables& T,
+                   const std::vector<float>& alpha, const std::vector<uint64_t>& tile_bytes,
+                   std::vector<uint8_t>& blob, uint64_t* off_stream, std::string& why);
+
+}  // namespace ep
