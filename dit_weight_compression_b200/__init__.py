@@ -42,7 +42,8 @@ class EpTensor(ctypes.Structure):
 
 
 class EpOptions(ctypes.Structure):
-    _fields_ = [("steps_per_tile", _I), ("num_threads", _I), ("scale", _D), ("rd_refine", _I)]
+    _fields_ = [("steps_per_tile", _I), ("num_threads", _I), ("scale", _D), ("rd_refine", _I),
+                ("host_encoder", _I)]
 
 
 class EpBlobInfo(ctypes.Structure):
@@ -129,6 +130,7 @@ class LatticeRANSConfig:
     steps_per_tile: int = 0     # rANS steps per tile (tile = 32 x S vectors); 0 = default rule
     num_threads: int = 0        # host encoder threads; 0 = all
     rd_refine: bool = False     # per-row rate-distortion refinement (slower encode; off by default)
+    host_encoder: bool = False  # encode CUDA tensors on the host instead of on their GPU
 
     def __post_init__(self):
         t = float(self.target_bpp)
@@ -193,7 +195,8 @@ def compress(tensor: torch.Tensor, config, *, scale: float = 0.0) -> CompressedT
     if t.stride(1) != 1 and t.shape[1] > 1:
         t = t.contiguous()
     view = tensor_view(t)
-    opts = EpOptions(cfg.steps_per_tile, cfg.num_threads, float(scale), int(bool(cfg.rd_refine)))
+    opts = EpOptions(cfg.steps_per_tile, cfg.num_threads, float(scale), int(bool(cfg.rd_refine)),
+                     int(bool(cfg.host_encoder)))
     h = ctypes.c_void_p()
     _check(lib().ep_compress_ex(ctypes.byref(view), cfg.target_bpp, ctypes.byref(opts), ctypes.byref(h)),
            "ep_compress")

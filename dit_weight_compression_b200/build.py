@@ -15,7 +15,7 @@ PKG = os.path.dirname(os.path.abspath(__file__))
 ROOT = os.path.dirname(PKG)
 CSRC = os.path.join(PKG, "csrc")
 LIB = os.path.join(PKG, "libentropack.so")
-SOURCES = ["api.cpp", "encoder.cpp", "decode.cu"]
+SOURCES = ["api.cpp", "encoder.cpp", "decode.cu", "encode_gpu.cu"]
 HEADERS = ["format.h", "blob.h", "tables.h"]
 
 

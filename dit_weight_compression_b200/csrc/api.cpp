@@ -46,11 +46,25 @@ extern "C" int ep_compress_ex(const ep_tensor* in, double target_bpp, const ep_o
     if (!std::isfinite(target_bpp) || target_bpp < kTargetMin || target_bpp > kTargetMax)
         return set_error(EP_ERR_RANGE, "ep_compress: target_bpp must be finite and in [0.001, 11]");
 
-    // The encoder runs on the host: bring device tensors over first.
+    EncodeOptions o;
+    bool host_encoder = false;
+    if (opt) {
+        if (opt->steps_per_tile < 0 || opt->steps_per_tile > 1024 || opt->num_threads < 0 ||
+            !(opt->scale >= 0.0) || !std::isfinite(opt->scale))
+            return set_error(EP_ERR_ARG, "ep_compress: bad options");
+        o.steps_per_tile = opt->steps_per_tile;
+        o.threads = opt->num_threads;
+        o.scale = opt->scale;
+        o.rd_refine = opt->rd_refine != 0;
+        host_encoder = opt->host_encoder != 0;
+    }
+    // A device tensor is encoded on its GPU (same bytes), unless the refinement or the caller asks
+    // for the host encoder; then it is copied to the host first.
+    const bool on_gpu = in->device >= 0 && !o.rd_refine && !host_encoder;
     std::vector<uint8_t> host_copy;
     const void* src = in->data;
     int64_t stride = in->row_stride;
-    if (in->device >= 0) {
+    if (in->device >= 0 && !on_gpu) {
         size_t row_bytes = size_t(in->cols) * es;
         try {
             host_copy.resize(row_bytes * size_t(in->rows));
@@ -69,29 +83,32 @@ extern "C" int ep_compress_ex(const ep_tensor* in, double target_bpp, const ep_o
         stride = in->cols;
     }
 
-    EncodeOptions o;
-    if (opt) {
-        if (opt->steps_per_tile < 0 || opt->steps_per_tile > 1024 || opt->num_threads < 0 ||
-            !(opt->scale >= 0.0) || !std::isfinite(opt->scale))
-            return set_error(EP_ERR_ARG, "ep_compress: bad options");
-        o.steps_per_tile = opt->steps_per_tile;
-        o.threads = opt->num_threads;
-        o.scale = opt->scale;
-        o.rd_refine = opt->rd_refine != 0;
-    }
     ep_blob* b = new (std::nothrow) ep_blob();
     if (!b) return set_error(EP_ERR_OOM, "ep_compress: blob");
     std::string why;
     int rc;
     try {
-        rc = encode(EncodeInput{src, in->dtype, in->rows, in->cols, stride}, target_bpp, o, b->bytes, why);
+        const EncodeInput ei{src, in->dtype, in->rows, in->cols, stride};
+        if (on_gpu) {
+            int prev = 0;
+            cudaGetDevice(&prev);
+            if (cudaSetDevice(in->device) != cudaSuccess) {
+                delete b;
+                return set_error(EP_ERR_ARG, "ep_compress: cannot use the tensor's device");
+            }
+            rc = encode_gpu(ei, target_bpp, o, b->bytes, why);
+            cudaSetDevice(prev);
+        } else {
+            rc = encode(ei, target_bpp, o, b->bytes, why);
+        }
     } catch (const std::bad_alloc&) {
         delete b;
         return set_error(EP_ERR_OOM, "ep_compress: out of host memory");
     }
     if (rc != 0) {
         delete b;
-        return set_error(rc == -4 ? EP_ERR_RANGE : EP_ERR_SHAPE, "ep_compress: " + why);
+        const int code = rc == -4 ? EP_ERR_RANGE : rc == -6 ? EP_ERR_CUDA : rc == -7 ? EP_ERR_OOM : EP_ERR_SHAPE;
+        return set_error(code, "ep_compress: " + why);
     }
     if (!parse_blob(b->bytes.data(), b->bytes.size(), b->layout, why)) {
         delete b;

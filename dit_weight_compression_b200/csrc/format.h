@@ -26,6 +26,13 @@
 #include <string>
 #include <vector>
 
+// Functions the device code of the library shares with its host code.
+#ifdef __CUDACC__
+#define EP_HD __host__ __device__
+#else
+#define EP_HD
+#endif
+
 namespace ep {
 
 constexpr uint32_t kVersion = 2;
@@ -52,7 +59,7 @@ inline int dtype_bytes(int dt) {
     }
 }
 
-inline uint64_t round_up16(uint64_t n) { return (n + 15) & ~uint64_t(15); }
+EP_HD inline uint64_t round_up16(uint64_t n) { return (n + 15) & ~uint64_t(15); }
 
 // Parsed, validated header of a blob plus the decoded frequency tables.
 struct BlobLayout {
@@ -98,5 +105,9 @@ struct EncodeOptions {
 // Returns 0, -3 (shape/size limits) or -4 (non-finite input); `why` explains a failure.
 int encode(const EncodeInput& in, double target, const EncodeOptions& opt, std::vector<uint8_t>& blob,
            std::string& why);
+// The same encoder with its parallel work on the GPU, for a device tensor (in.bits on the current
+// device); the same bytes.  Also -6 (a CUDA call failed) and -7 (device memory).  No refinement.
+int encode_gpu(const EncodeInput& in, double target, const EncodeOptions& opt, std::vector<uint8_t>& blob,
+               std::string& why);
 
 }  // namespace ep

@@ -14,7 +14,7 @@
 namespace ep {
 
 // Field value -> symbol: f + 127 for |f| <= 127, else the escape symbol.
-inline int symbol_of(int32_t f) { return (f >= -kAlphabetR && f <= kAlphabetR) ? f + kAlphabetR : kEscape; }
+EP_HD inline int symbol_of(int32_t f) { return (f >= -kAlphabetR && f <= kAlphabetR) ? f + kAlphabetR : kEscape; }
 
 // Symbol counts of the 17 contexts: [0] the coset (symbols 0/1), [1 + 8c + j - 1] field j | c.
 struct Counts {

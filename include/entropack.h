@@ -72,6 +72,9 @@ typedef struct {
                             resolutions s * 2^(k/2), k in {0, -1, 1, -2, 2}, by a Lagrangian
                             choice under the storage budget, in three rounds that rebuild the
                             probability tables; the decode format does not change           */
+    int host_encoder;    /* nonzero: encode a device tensor on the host (it is copied there first);
+                            by default a device tensor is encoded on its GPU -- the same bytes --
+                            except with rd_refine, which runs on the host                    */
 } ep_options;
 
 typedef struct ep_blob ep_blob;
