@@ -58,6 +58,7 @@ def lib() -> ctypes.CDLL:
             "orc_round_f32_n": (None, [P, I64, P]),
             "orc_cvt_f32_array": (None, [P, U64, I, P]),
             "orc_quantize_table": (None, [P, P]),
+            "orc_build_tables16": (None, [P, P]),
             "orc_encode_tile": (U64, [P, P, I64, P, P, U64]),
             "orc_decode_tile": (I, [P, U64, I64, P, P, P, P]),
             "orc_estimate_bpp": (D, [P, I, I64, I64, D, I64, I]),
@@ -204,24 +205,33 @@ def quantize_table(counts: np.ndarray) -> np.ndarray:
     return q
 
 
-def encode_tile(sym9: np.ndarray, raw8: np.ndarray, q17: np.ndarray) -> bytes:
+def build_tables16(counts: np.ndarray) -> np.ndarray:
+    """The 16 context tables (16 x 256) from symbol counts (16 x 256): contexts 0 and 8 quantised
+    together as the joint (coset, f1) table, the others one by one."""
+    counts = np.ascontiguousarray(counts, np.uint64).reshape(16, 256)
+    q = np.zeros((16, 256), np.uint16)
+    lib().orc_build_tables16(_ptr(counts), _ptr(q))
+    return q
+
+
+def encode_tile(sym9: np.ndarray, raw8: np.ndarray, q16: np.ndarray) -> bytes:
     sym9 = np.ascontiguousarray(sym9, np.uint8).reshape(-1, 9)
     raw8 = np.ascontiguousarray(raw8, np.int16).reshape(-1, 8)
-    q17 = np.ascontiguousarray(q17, np.uint16).reshape(17, 256)
-    n = lib().orc_encode_tile(_ptr(sym9), _ptr(raw8), len(sym9), _ptr(q17), None, 0)
+    q16 = np.ascontiguousarray(q16, np.uint16).reshape(16, 256)
+    n = lib().orc_encode_tile(_ptr(sym9), _ptr(raw8), len(sym9), _ptr(q16), None, 0)
     if n == 0:
         raise ValueError("oracle encode_tile failed")
     out = np.zeros(n, np.uint8)
-    lib().orc_encode_tile(_ptr(sym9), _ptr(raw8), len(sym9), _ptr(q17), _ptr(out), n)
+    lib().orc_encode_tile(_ptr(sym9), _ptr(raw8), len(sym9), _ptr(q16), _ptr(out), n)
     return out.tobytes()
 
 
-def decode_tile(tile: bytes, nvec: int, q17: np.ndarray):
+def decode_tile(tile: bytes, nvec: int, q16: np.ndarray):
     """Returns (rc, sym9, raw8, final_states); raw8 is meaningful only where sym9 is the escape."""
-    q17 = np.ascontiguousarray(q17, np.uint16).reshape(17, 256)
+    q16 = np.ascontiguousarray(q16, np.uint16).reshape(16, 256)
     sym9 = np.zeros((nvec, 9), np.uint8)
     raw8 = np.zeros((nvec, 8), np.int16)
     st = np.zeros(32, np.uint32)
-    rc = lib().orc_decode_tile(_buf(tile), len(tile), nvec, _ptr(q17), _ptr(sym9), _ptr(raw8),
+    rc = lib().orc_decode_tile(_buf(tile), len(tile), nvec, _ptr(q16), _ptr(sym9), _ptr(raw8),
                                _ptr(st))
     return rc, sym9, raw8, st

@@ -50,9 +50,9 @@ enum { ORC_BF16 = 1, ORC_FP16 = 2, ORC_E4M3 = 3, ORC_F32 = 4, ORC_INT8 = 5 };
 #define ORC_ESC 255        /* symbol that announces a raw 16-bit field value               */
 #define ORC_M 1024u        /* reading: frequency totals are 10-bit, every table sums to M  */
 #define ORC_L 65536u       /* rANS lower bound 2^16, 32-bit state, 16-bit renormalisation */
-#define ORC_VERSION 2      /* blob format version (2: 10-bit frequency totals)            */
+#define ORC_VERSION 3      /* blob format version (3: coset coded jointly with f1)        */
 #define ORC_LANES 32       /* interleaved rANS states per tile                            */
-#define ORC_NCTX 17        /* context 0: coset; 1 + 8c + (j-1): field j given coset c     */
+#define ORC_NCTX 16        /* field j given coset c: 8c + (j-1); 0 and 8 = joint (c, f1)  */
 #define ORC_HEADER 80      /* bytes in the fixed header                                   */
 #define ORC_CLAMP 32764.0  /* reading: |t| clamp, keeps every field inside int16          */
 
@@ -362,14 +362,14 @@ static int field_symbol(int32_t f) { return (f >= -ORC_R && f <= ORC_R) ? f + OR
  * exceeds M, decrement the largest q (> 1; lowest symbol on ties); while it is below M,
  * increment the symbol with the largest count (lowest symbol on ties).  N = 0 gives all zeros.
  */
-void orc_quantize_table(const uint64_t n[256], uint16_t q[256])
+static void quantize_n(const uint64_t* n, int nb, uint16_t* q)
 {
     uint64_t N = 0;
-    for (int s = 0; s < 256; s++) N += n[s];
-    for (int s = 0; s < 256; s++) q[s] = 0;
+    for (int s = 0; s < nb; s++) N += n[s];
+    for (int s = 0; s < nb; s++) q[s] = 0;
     if (N == 0) return;
     long sum = 0;
-    for (int s = 0; s < 256; s++) {
+    for (int s = 0; s < nb; s++) {
         if (n[s] == 0) continue;
         uint64_t v = (2u * ORC_M * n[s] + N) / (2u * N);      /* round half up */
         if (v < 1) v = 1;
@@ -378,19 +378,45 @@ void orc_quantize_table(const uint64_t n[256], uint16_t q[256])
     }
     while (sum > (long)ORC_M) {
         int best = -1;
-        for (int s = 0; s < 256; s++)
+        for (int s = 0; s < nb; s++)
             if (q[s] > 1 && (best < 0 || q[s] > q[best])) best = s;
         q[best]--;
         sum--;
     }
     while (sum < (long)ORC_M) {
         int best = -1;
-        for (int s = 0; s < 256; s++)
+        for (int s = 0; s < nb; s++)
             if (n[s] > 0 && (best < 0 || n[s] > n[best])) best = s;
         q[best]++;
         sum++;
     }
 }
+
+void orc_quantize_table(const uint64_t n[256], uint16_t q[256]) { quantize_n(n, 256, q); }
+
+/*
+ * The 16 context tables from symbol counts cnt[16 x 256].  reading: the coset and the first field
+ * are one symbol ([DOC-LQ]: every field is modelled given the coset; coding the pair (c, f1) as
+ * one symbol of the joint distribution P(c) P(f1 | c) keeps that model and spends one rANS step
+ * where two would do): contexts 0 and 8 are the two coset halves of one 512-symbol table,
+ * quantised together to sum to M (coset-major order, so ties go to coset 0 first); every other
+ * context (c, j >= 2) is quantised on its own.
+ */
+static void build_tables16(const uint64_t* cnt, uint16_t* q16)
+{
+    uint64_t nj[512];
+    uint16_t qj[512];
+    memcpy(nj, cnt, 256 * sizeof(uint64_t));
+    memcpy(nj + 256, cnt + 256 * 8, 256 * sizeof(uint64_t));
+    quantize_n(nj, 512, qj);
+    memcpy(q16, qj, 256 * sizeof(uint16_t));
+    memcpy(q16 + 256 * 8, qj + 256, 256 * sizeof(uint16_t));
+    for (int ctx = 1; ctx < ORC_NCTX; ctx++)
+        if (ctx != 8) orc_quantize_table(cnt + 256 * ctx, q16 + 256 * ctx);
+}
+
+/* Exposed for the table checks. */
+void orc_build_tables16(const uint64_t* cnt, uint16_t* q16) { build_tables16(cnt, q16); }
 
 /* Cumulative frequencies: cum[s] = q[0] + ... + q[s-1]. */
 static void cumulate(const uint16_t q[256], uint32_t cum[257])
@@ -399,18 +425,29 @@ static void cumulate(const uint16_t q[256], uint32_t cum[257])
     for (int s = 0; s < 256; s++) cum[s + 1] = cum[s] + q[s];
 }
 
-/* Context index of sub-step u (0 = coset, 1..8 = field u) of a vector with coset c. */
-static int context_of(int u, int c) { return u == 0 ? 0 : 1 + 8 * c + (u - 1); }
+/* Context of field j (1..8) of a vector with coset c. */
+static int context_of(int j, int c) { return 8 * c + (j - 1); }
+
+/* Frequency and cumulative frequency of symbol s of field j given coset c.  For j = 1 the two
+ * coset halves (contexts 0 and 8) are one distribution over (c, s): coset 1's slots follow all
+ * of coset 0's. */
+static void freq_cum(const uint16_t* q16, const uint32_t cum[ORC_NCTX][257], int j, int c, int s,
+                     uint32_t* q, uint32_t* cm)
+{
+    int ctx = context_of(j, c);
+    *q = q16[256 * ctx + s];
+    *cm = cum[ctx][s] + ((j == 1 && c == 1) ? cum[0][256] : 0u);
+}
 
 /* ------------------------------------------------------------------------------------------ */
 /* Tiled, 32-way interleaved rANS [ANS] with the word layout of the format ([DOC-ER]: the      */
 /* fields are rANS-coded in tiles, each of which decodes without the others).                  */
 /*                                                                                            */
 /* One tile holds up to 32*S consecutive vectors; lane l at step k owns vector 32k + l of the  */
-/* tile and has its own 32-bit rANS state.  Each vector is 9 symbols: the coset (context 0) and */
-/* f1..f8 (context 1 + 8c + j - 1).  A lane's words, in the order it reads them: for each step, */
-/* for each sub-step u = 0..8, after decoding its symbol, one 16-bit word if the state fell    */
-/* below 2^16; after sub-step 8 the raw words of its escaped fields, by field.                 */
+/* tile and has its own 32-bit rANS state.  Each vector is 8 symbols: (coset, f1) jointly, then */
+/* f2..f8 (context 8c + j - 1).  A lane's words, in the order it reads them: for each step, for */
+/* each of the 8 symbols, after decoding it, one 16-bit word if the state fell below 2^16;     */
+/* after the last the raw words of its escaped fields, by field.                               */
 /* reading: lanes 2p and 2p+1 share region p: lane 2p's words run forward from the region's    */
 /* start, lane 2p+1's run backward from its end.                                                */
 /* Tile bytes: 32 little-endian u32 initial states (lane order); 16 u16 word counts of the      */
@@ -440,10 +477,11 @@ static int push_word(wordbuf* b, uint32_t v)
 }
 
 /*
- * Encode one tile.  sym9[v*9 + u] is the symbol of sub-step u of vector v, raw8[v*8 + j-1] the raw
- * value of field j (used when its symbol is the escape).  q17 holds the 17 context tables
- * (17 x 256 frequencies).  Returns the tile size in bytes (written to out when out != NULL and
- * cap is large enough), or 0 on failure.
+ * Encode one tile.  sym9[v*9] is the coset of vector v and sym9[v*9 + j] the symbol of its field j,
+ * raw8[v*8 + j-1] the raw value of field j (used when its symbol is the escape).  q16 holds the 16
+ * context tables (16 x 256 frequencies; contexts 0 and 8 the joint (coset, f1) table).  Returns
+ * the tile size in bytes (written to out when out != NULL and cap is large enough), or 0 on
+ * failure.
  *
  * rANS encode of symbol s with frequency q and cumulative cum [ANS]: while x >= q * (L / M) * 2^16
  * (= q * 2^22), emit the low 16 bits of x and shift them out; then
@@ -452,10 +490,10 @@ static int push_word(wordbuf* b, uint32_t v)
  * at the end.
  */
 uint64_t orc_encode_tile(const uint8_t* sym9, const int16_t* raw8, int64_t nvec,
-                         const uint16_t* q17, uint8_t* out, uint64_t cap)
+                         const uint16_t* q16, uint8_t* out, uint64_t cap)
 {
     uint32_t cum[ORC_NCTX][257];
-    for (int c = 0; c < ORC_NCTX; c++) cumulate(q17 + 256 * c, cum[c]);
+    for (int c = 0; c < ORC_NCTX; c++) cumulate(q16 + 256 * c, cum[c]);
     uint32_t x[ORC_LANES];
     wordbuf wb[ORC_LANES];
     memset(wb, 0, sizeof wb);
@@ -469,16 +507,15 @@ uint64_t orc_encode_tile(const uint8_t* sym9, const int16_t* raw8, int64_t nvec,
             for (int j = 8; j >= 1; j--)
                 if (sym9[v * 9 + j] == ORC_ESC)
                     if (push_word(&wb[l], (uint16_t)raw8[v * 8 + (j - 1)])) goto fail;
-            for (int u = 8; u >= 0; u--) {
-                int s = sym9[v * 9 + u];
-                int ctx = context_of(u, sym9[v * 9]);
-                uint32_t q = q17[256 * ctx + s];
+            for (int j = 8; j >= 1; j--) {      /* j = 1 codes the coset too */
+                uint32_t q, cm;
+                freq_cum(q16, cum, j, sym9[v * 9], sym9[v * 9 + j], &q, &cm);
                 if (q == 0) goto fail;
                 if ((uint64_t)x[l] >= (uint64_t)q * (ORC_L / ORC_M) * 65536u) {
                     if (push_word(&wb[l], x[l] & 0xFFFFu)) goto fail;
                     x[l] >>= 16;
                 }
-                x[l] = (x[l] / q) * ORC_M + (x[l] % q) + cum[ctx][s];
+                x[l] = (x[l] / q) * ORC_M + (x[l] % q) + cm;
             }
         }
     }
@@ -511,18 +548,19 @@ fail:
     return 0;
 }
 
-/* Decoding tables of the 17 contexts: cumulative frequencies and the symbol of every slot. */
+/* Decoding tables of the 16 contexts: cumulative frequencies and the symbol of every slot (for
+ * the two halves of the joint table, slots relative to each half's start). */
 typedef struct {
-    const uint16_t* q17;
+    const uint16_t* q16;
     uint32_t cum[ORC_NCTX][257];
     uint8_t slot_sym[ORC_NCTX][ORC_M];
 } dtables;
 
-static void build_dtables(const uint16_t* q17, dtables* T)
+static void build_dtables(const uint16_t* q16, dtables* T)
 {
-    T->q17 = q17;
+    T->q16 = q16;
     for (int c = 0; c < ORC_NCTX; c++) {
-        cumulate(q17 + 256 * c, T->cum[c]);
+        cumulate(q16 + 256 * c, T->cum[c]);
         memset(T->slot_sym[c], 0, ORC_M);
         for (int s = 0; s < 256; s++)
             for (uint32_t i = T->cum[c][s]; i < T->cum[c][s + 1] && i < ORC_M; i++) T->slot_sym[c][i] = (uint8_t)s;
@@ -560,13 +598,22 @@ static int decode_tile(const uint8_t* tile, uint64_t nbytes, int64_t nvec, const
         for (int64_t k = 0; k < nsteps; k++) {
             int64_t v = k * ORC_LANES + l;
             if (v >= nvec) continue;
-            for (int u = 0; u <= 8; u++) {
-                int ctx = context_of(u, u == 0 ? 0 : sym9[v * 9]);
+            for (int j = 1; j <= 8; j++) {
                 uint32_t slot = x & (ORC_M - 1);
-                int s = T->slot_sym[ctx][slot];
-                uint32_t q = T->q17[256 * ctx + s];
-                x = q * (x / ORC_M) + slot - T->cum[ctx][s];
-                sym9[v * 9 + u] = (uint8_t)s;
+                int c, s;
+                if (j == 1) {                    /* (coset, f1): coset 1's slots follow coset 0's */
+                    uint32_t tot0 = T->cum[0][256];
+                    c = slot < tot0 ? 0 : 1;
+                    s = T->slot_sym[context_of(1, c)][c ? slot - tot0 : slot];
+                    sym9[v * 9] = (uint8_t)c;
+                } else {
+                    c = sym9[v * 9];
+                    s = T->slot_sym[context_of(j, c)][slot];
+                }
+                uint32_t q, cm;
+                freq_cum(T->q16, T->cum, j, c, s, &q, &cm);
+                x = q * (x / ORC_M) + slot - cm;
+                sym9[v * 9 + j] = (uint8_t)s;
                 if (x < ORC_L) {
                     int64_t w = fwd ? start[p] + n : start[p] + count[p] - 1 - n;
                     if (n >= count[p]) return -1;
@@ -592,13 +639,13 @@ static int decode_tile(const uint8_t* tile, uint64_t nbytes, int64_t nvec, const
     return bad;
 }
 
-/* Decode one tile given the 17 x 256 frequency tables (exposed for the rANS checks). */
-int orc_decode_tile(const uint8_t* tile, uint64_t nbytes, int64_t nvec, const uint16_t* q17,
+/* Decode one tile given the 16 x 256 frequency tables (exposed for the rANS checks). */
+int orc_decode_tile(const uint8_t* tile, uint64_t nbytes, int64_t nvec, const uint16_t* q16,
                     uint8_t* sym9, int16_t* raw8, uint32_t* final_states)
 {
     dtables* T = (dtables*)malloc(sizeof(dtables));
     if (!T) return -2;
-    build_dtables(q17, T);
+    build_dtables(q16, T);
     int rc = decode_tile(tile, nbytes, nvec, T, sym9, raw8, final_states);
     free(T);
     return rc;
@@ -671,12 +718,12 @@ static int64_t default_steps(double target)
     return s;
 }
 
-/* Bytes of the serialised table section for the given 17 tables (unpadded). */
-static uint64_t table_section_bytes(const uint16_t* q17)
+/* Bytes of the serialised table section for the given 16 tables (unpadded). */
+static uint64_t table_section_bytes(const uint16_t* q16)
 {
-    uint64_t bytes = 4;                                   /* coset q0, q1 */
-    for (int ctx = 1; ctx < ORC_NCTX; ctx++) {
-        const uint16_t* q = q17 + 256 * ctx;
+    uint64_t bytes = 0;
+    for (int ctx = 0; ctx < ORC_NCTX; ctx++) {
+        const uint16_t* q = q16 + 256 * ctx;
         int lo = -1, hi = -1;
         for (int s = 0; s < ORC_ESC; s++)
             if (q[s]) { if (lo < 0) lo = s; hi = s; }
@@ -709,22 +756,22 @@ static double estimate_bpp(const matrix* m, double s, int64_t S, int full_sample
             int16_t raw[8];
             quantise_vector(m, r, k, s, y, &c);
             vector_symbols(y, c, sym, raw);
-            for (int u = 0; u <= 8; u++) {
+            for (int u = 1; u <= 8; u++) {
                 cnt[256 * context_of(u, c) + sym[u]]++;
                 if (u > 0 && sym[u] == ORC_ESC) nesc++;
             }
         }
     }
-    uint16_t q17[ORC_NCTX * 256];
-    for (int ctx = 0; ctx < ORC_NCTX; ctx++) orc_quantize_table(cnt + 256 * ctx, q17 + 256 * ctx);
+    uint16_t q16[ORC_NCTX * 256];
+    build_tables16(cnt, q16);
     double bits = 0.0;
     for (int ctx = 0; ctx < ORC_NCTX; ctx++)
         for (int sy = 0; sy < 256; sy++)
-            if (cnt[256 * ctx + sy]) bits += (double)cnt[256 * ctx + sy] * -log2((double)q17[256 * ctx + sy] / (double)ORC_M);
+            if (cnt[256 * ctx + sy]) bits += (double)cnt[256 * ctx + sy] * -log2((double)q16[256 * ctx + sy] / (double)ORC_M);
     double payload = ((double)m->rows / (double)ns) * (bits / 8.0 + 2.0 * (double)nesc);
     int64_t V = m->rows * m->vpr;
     int64_t ntiles = (V + 32 * S - 1) / (32 * S);
-    double meta = (double)(ORC_HEADER + pad16(table_section_bytes(q17)) + pad16(4u * (uint64_t)m->rows) +
+    double meta = (double)(ORC_HEADER + pad16(table_section_bytes(q16)) + pad16(4u * (uint64_t)m->rows) +
                            pad16(4u * (uint64_t)(ntiles + 1))) +
                   (double)ntiles * (160.0 + 8.0);
     free(cnt);
@@ -850,7 +897,7 @@ static void rd_counts(const matrix* m, const uint8_t* sym, const int* kr, uint64
     for (int64_t r = 0; r < m->rows; r++) {
         const uint8_t* sr = sym + ((size_t)r * RD_NK + (size_t)kr[r]) * (size_t)m->vpr * 9;
         for (int64_t k = 0; k < m->vpr; k++)
-            for (int u = 0; u <= 8; u++) cnt[256 * context_of(u, sr[9 * k]) + sr[9 * k + u]]++;
+            for (int u = 1; u <= 8; u++) cnt[256 * context_of(u, sr[9 * k]) + sr[9 * k + u]]++;
     }
 }
 
@@ -891,21 +938,21 @@ static int rd_allocate(const matrix* m, double s, double target, int64_t S, int*
         int64_t V = m->rows * m->vpr;
         int64_t ntiles = (V + 32 * S - 1) / (32 * S);
         for (int round = 0; round < RD_ROUNDS; round++) {
-            uint16_t q17[ORC_NCTX * 256];
+            uint16_t q16[ORC_NCTX * 256];
             double cost[ORC_NCTX * 256];
             rd_counts(m, sym, kr, cnt);
-            for (int ctx = 0; ctx < ORC_NCTX; ctx++) orc_quantize_table(cnt + 256 * ctx, q17 + 256 * ctx);
+            build_tables16(cnt, q16);
             for (int i = 0; i < ORC_NCTX * 256; i++)
-                cost[i] = q17[i] ? -log2((double)q17[i] / (double)ORC_M) : log2((double)ORC_M);
+                cost[i] = q16[i] ? -log2((double)q16[i] / (double)ORC_M) : log2((double)ORC_M);
             for (int64_t r = 0; r < m->rows; r++)
                 for (int ki = 0; ki < RD_NK; ki++) {
                     const uint8_t* sr = sym + ((size_t)r * RD_NK + ki) * per;
                     double bits = 16.0 * (double)nesc[r * RD_NK + ki];
                     for (int64_t k = 0; k < m->vpr; k++)
-                        for (int u = 0; u <= 8; u++) bits += cost[256 * context_of(u, sr[9 * k]) + sr[9 * k + u]];
+                        for (int u = 1; u <= 8; u++) bits += cost[256 * context_of(u, sr[9 * k]) + sr[9 * k + u]];
                     R[r * RD_NK + ki] = bits;
                 }
-            double meta = (double)(ORC_HEADER + pad16(table_section_bytes(q17)) + pad16(4u * (uint64_t)m->rows) +
+            double meta = (double)(ORC_HEADER + pad16(table_section_bytes(q16)) + pad16(4u * (uint64_t)m->rows) +
                                    pad16(4u * (uint64_t)(ntiles + 1))) +
                           (double)ntiles * (160.0 + 8.0);
             double budget = target * (double)m->rows * (double)m->cols - 8.0 * meta;
@@ -940,8 +987,8 @@ out:
  *   header (80 bytes): "EPK1", u16 version 2, u8 dtype, u8 R, u64 rows, u64 cols, u32 S,
  *     u32 n_tiles, f64 s, u64 total bytes, u64 offsets of the table, row-scale, tile-offset
  *     and stream sections;
- *   tables: u16 q(coset 0), u16 q(coset 1); then for c = 0,1 and j = 1..8: u16 q(escape),
- *     u8 lo, u8 n, u16 q[lo .. lo+n-1] (symbols 0..254);
+ *   tables: for c = 0,1 and j = 1..8: u16 q(escape), u8 lo, u8 n, u16 q[lo .. lo+n-1]
+ *     (symbols 0..254); the two j = 1 tables are the coset halves of the joint (c, f1) table;
  *   row scales: f32 per row;
  *   tile offsets: u32[n_tiles + 1], in 16-byte units from the stream section start;
  *   stream: the tiles.
@@ -988,15 +1035,15 @@ int orc_compress_ex(const void* data, int dtype, int64_t rows, int64_t cols, dou
                     swy += elem(&m, r, 8 * k + i) * y[i];
                     syy += y[i] * y[i];
                 }
-            for (int u = 0; u <= 8; u++) cnt[256 * context_of(u, c) + sym9[9 * v + u]]++;
+            for (int u = 1; u <= 8; u++) cnt[256 * context_of(u, c) + sym9[9 * v + u]]++;
         }
         alpha[r] = syy > 0.0 ? (float)(swy / syy) : 0.0f;
     }
 
     /* Probability tables from the whole tensor ([DOC-LQ]: one model per coordinate field, given
      * the coset). */
-    uint16_t q17[ORC_NCTX * 256];
-    for (int ctx = 0; ctx < ORC_NCTX; ctx++) orc_quantize_table(cnt + 256 * ctx, q17 + 256 * ctx);
+    uint16_t q16[ORC_NCTX * 256];
+    build_tables16(cnt, q16);
 
     /* Tiles. */
     int64_t per_tile = 32 * S;
@@ -1005,14 +1052,14 @@ int orc_compress_ex(const void* data, int dtype, int64_t rows, int64_t cols, dou
     uint64_t stream_bytes = 0;
     for (int64_t t = 0; t < ntiles; t++) {
         int64_t v0 = t * per_tile, nv = V - v0 < per_tile ? V - v0 : per_tile;
-        tsize[t] = orc_encode_tile(sym9 + 9 * v0, raw8 + 8 * v0, nv, q17, NULL, 0);
+        tsize[t] = orc_encode_tile(sym9 + 9 * v0, raw8 + 8 * v0, nv, q16, NULL, 0);
         if (tsize[t] == 0) { rc = -5; goto done; }
         stream_bytes += tsize[t];
     }
 
     /* Serialise. */
     {
-        uint64_t tab_bytes = table_section_bytes(q17);
+        uint64_t tab_bytes = table_section_bytes(q16);
         uint64_t off_tab = ORC_HEADER;
         uint64_t off_alpha = off_tab + pad16(tab_bytes);
         uint64_t off_offs = off_alpha + pad16(4u * (uint64_t)rows);
@@ -1035,11 +1082,8 @@ int orc_compress_ex(const void* data, int dtype, int64_t rows, int64_t cols, dou
         put64(b + 64, off_offs);
         put64(b + 72, off_stream);
         uint8_t* p = b + off_tab;
-        put16(p, q17[0]);
-        put16(p + 2, q17[1]);
-        p += 4;
-        for (int ctx = 1; ctx < ORC_NCTX; ctx++) {
-            const uint16_t* q = q17 + 256 * ctx;
+        for (int ctx = 0; ctx < ORC_NCTX; ctx++) {
+            const uint16_t* q = q16 + 256 * ctx;
             int lo = -1, hi = -1;
             for (int sy = 0; sy < ORC_ESC; sy++)
                 if (q[sy]) { if (lo < 0) lo = sy; hi = sy; }
@@ -1063,7 +1107,7 @@ int orc_compress_ex(const void* data, int dtype, int64_t rows, int64_t cols, dou
         acc = 0;
         for (int64_t t = 0; t < ntiles; t++) {
             int64_t v0 = t * per_tile, nv = V - v0 < per_tile ? V - v0 : per_tile;
-            orc_encode_tile(sym9 + 9 * v0, raw8 + 8 * v0, nv, q17, b + off_stream + acc, tsize[t]);
+            orc_encode_tile(sym9 + 9 * v0, raw8 + 8 * v0, nv, q16, b + off_stream + acc, tsize[t]);
             acc += tsize[t];
         }
         *blob = b;
@@ -1096,7 +1140,7 @@ typedef struct {
     int dtype;
     int64_t rows, cols, vpr, S, ntiles, V;
     double s;
-    uint16_t q17[ORC_NCTX * 256];
+    uint16_t q16[ORC_NCTX * 256];
     const uint8_t* alpha;
     const uint8_t* offs;
     const uint8_t* stream;
@@ -1118,28 +1162,28 @@ static int parse_blob(const uint8_t* b, uint64_t len, parsed* P)
     P->vpr = (P->cols + 7) / 8;
     P->V = P->rows * P->vpr;
     if (P->ntiles != (P->V + 32 * P->S - 1) / (32 * P->S)) return -6;
-    if (off_tab < ORC_HEADER || off_tab + 4 > off_alpha || off_alpha + 4u * (uint64_t)P->rows > off_offs ||
+    if (off_tab < ORC_HEADER || off_tab > off_alpha || off_alpha + 4u * (uint64_t)P->rows > off_offs ||
         off_offs + 4u * (uint64_t)(P->ntiles + 1) > off_stream || off_stream > len)
         return -6;
-    memset(P->q17, 0, sizeof P->q17);
+    memset(P->q16, 0, sizeof P->q16);
     const uint8_t* p = b + off_tab;
-    P->q17[0] = (uint16_t)get16(p);
-    P->q17[1] = (uint16_t)get16(p + 2);
-    p += 4;
-    for (int ctx = 1; ctx < ORC_NCTX; ctx++) {
+    for (int ctx = 0; ctx < ORC_NCTX; ctx++) {
         if ((uint64_t)(p + 4 - b) > off_alpha) return -6;
-        uint16_t* q = P->q17 + 256 * ctx;
+        uint16_t* q = P->q16 + 256 * ctx;
         q[ORC_ESC] = (uint16_t)get16(p);
         int lo = p[2], n = p[3];
         p += 4;
         if (lo + n > ORC_ESC || (uint64_t)(p + 2 * n - b) > off_alpha) return -6;
         for (int i = 0; i < n; i++, p += 2) q[lo + i] = (uint16_t)get16(p);
     }
+    uint32_t sums[ORC_NCTX];
     for (int ctx = 0; ctx < ORC_NCTX; ctx++) {
-        uint32_t sum = 0;
-        for (int sy = 0; sy < 256; sy++) sum += P->q17[256 * ctx + sy];
-        if (sum != 0 && sum != ORC_M) return -6;
+        sums[ctx] = 0;
+        for (int sy = 0; sy < 256; sy++) sums[ctx] += P->q16[256 * ctx + sy];
     }
+    if (sums[0] + sums[8] != ORC_M) return -6;                 /* the joint (coset, f1) table */
+    for (int ctx = 0; ctx < ORC_NCTX; ctx++)
+        if (ctx != 0 && ctx != 8 && sums[ctx] != 0 && sums[ctx] != ORC_M) return -6;
     P->alpha = b + off_alpha;
     P->offs = b + off_offs;
     P->stream = b + off_stream;
@@ -1155,7 +1199,7 @@ static int decode_tiles_to_symbols(const parsed* P, int64_t t0, int64_t t1, uint
     int64_t per_tile = 32 * P->S, base = t0 * per_tile;
     dtables* T = (dtables*)malloc(sizeof(dtables));
     if (!T) return -2;
-    build_dtables(P->q17, T);
+    build_dtables(P->q16, T);
     int out = 0;
     for (int64_t t = t0; t < t1; t++) {
         uint64_t a = 16u * (uint64_t)get32(P->offs + 4 * t), e = 16u * (uint64_t)get32(P->offs + 4 * (t + 1));

@@ -191,18 +191,49 @@ def test_table_invariants():
         assert np.abs(q - ideal).sum() <= 2.0 * (k / 2 + r / 2) + 1e-9
 
 
+def test_joint_coset_f1_table():
+    """Contexts 0 and 8 (field 1 given coset 0 / 1) are one table over the 512 pairs (c, f1):
+    the same quantisation rule on the concatenated counts, coset 0 first on ties."""
+    counts = np.zeros((16, 256), np.uint64)
+    counts[0, 5], counts[8, 5] = 3, 1                   # 3 : 1 over the pair -> 768 : 256
+    counts[1, [0, 1]] = 1                               # a context on its own -> 512 : 512
+    q = oracle.build_tables16(counts)
+    assert (q[0, 5], q[8, 5]) == (768, 256) and (q[1, 0], q[1, 1]) == (512, 512)
+    assert q[2:8].sum() == 0 and q[9:].sum() == 0       # empty contexts stay empty
+    counts = np.zeros((16, 256), np.uint64)
+    counts[0, 7], counts[8, 7] = 1, 1                   # 1024 / 3 -> 341 each, sum 1023: the
+    counts[0, 8] = 1                                    # first largest count (coset 0, 7) gets +1
+    q = oracle.build_tables16(counts)
+    assert (q[0, 7], q[0, 8], q[8, 7]) == (342, 341, 341)
+    for _ in range(50):
+        c = np.zeros((16, 256), np.uint64)
+        for ctx in range(16):
+            k = RNG.integers(0, 60)
+            c[ctx, RNG.choice(256, k, replace=False)] = RNG.integers(1, 10 ** 4, k)
+        if c[0].sum() + c[8].sum() == 0:
+            c[0, 127] = 1
+        q = oracle.build_tables16(c)
+        assert int(q[0].sum()) + int(q[8].sum()) == M
+        assert np.array_equal(q[[0, 8]] > 0, c[[0, 8]] > 0)
+        for ctx in set(range(16)) - {0, 8}:
+            assert int(q[ctx].sum()) in (0, M) and np.array_equal(q[ctx], oracle.quantize_table(c[ctx]))
+
+
 # ---------------------------------------------------------------------------------------------
 # rANS tiles.
 # ---------------------------------------------------------------------------------------------
 
-def _tables(field_q: dict, coset_q=(M, 0)):
-    """17 x 256 tables: context 0 the coset, contexts 1..16 all equal to field_q."""
-    q17 = np.zeros((17, 256), np.uint16)
-    q17[0, 0], q17[0, 1] = coset_q
-    for ctx in range(1, 17):
+def _tables(field_q: dict):
+    """16 x 256 tables for vectors that are all in coset 0: the joint (coset, f1) table is field_q
+    on its coset-0 half (context 0) and empty on its coset-1 half (context 8); every other
+    context equals field_q."""
+    q16 = np.zeros((16, 256), np.uint16)
+    for ctx in range(16):
+        if ctx == 8:
+            continue
         for s, q in field_q.items():
-            q17[ctx, s] = q
-    return q17
+            q16[ctx, s] = q
+    return q16
 
 
 def test_rans_closed_form_one_bit_symbols():
@@ -217,12 +248,12 @@ def test_rans_closed_form_one_bit_symbols():
     + f1 of step 1.  Every lane has exactly one word, so each region holds 2 words: lane 2p's
     (read forward from the region start) then lane 2p+1's (read backward from the region end)
     -- lane order overall."""
-    q17 = _tables({127: 512, 128: 512})
+    q16 = _tables({127: 512, 128: 512})
     bits = RNG.integers(0, 2, (64, 8))                              # vector v = 32k + lane
     sym9 = np.zeros((64, 9), np.uint8)
     sym9[:, 1:] = 127 + bits
     raw8 = np.zeros((64, 8), np.int16)
-    tile = oracle.encode_tile(sym9, raw8, q17)
+    tile = oracle.encode_tile(sym9, raw8, q16)
     assert len(tile) == 160 + 64
     states = np.frombuffer(tile[:128], "<u4")
     counts = np.frombuffer(tile[128:160], "<u2")
@@ -235,7 +266,7 @@ def test_rans_closed_form_one_bit_symbols():
         assert states[lane] == 65536 + 512 * int(f0[0]) + step1
         low7 = sum(int(f0[j]) << (j - 1) for j in range(1, 8))       # 64 f8 + ... + f2
         assert words[lane] == 512 * low7
-    rc, s9, r8, st = oracle.decode_tile(tile, 64, q17)
+    rc, s9, r8, st = oracle.decode_tile(tile, 64, q16)
     assert rc == 0 and np.array_equal(s9, sym9) and np.all(st == 65536)
 
 
@@ -243,12 +274,12 @@ def test_rans_all_escape_closed_form():
     """Coset free, every field the escape symbol with q = M: no state ever changes, so each
     lane's words are its raw values in step, field order; region p holds lane 2p's words forward
     and lane 2p+1's words backward from the region end."""
-    q17 = _tables({255: M})
+    q16 = _tables({255: M})
     nvec = 70                                                       # 3 steps, the last partial
     sym9 = np.zeros((nvec, 9), np.uint8)
     sym9[:, 1:] = 255
     raw8 = RNG.integers(-32768, 32768, (nvec, 8)).astype(np.int16)
-    tile = oracle.encode_tile(sym9, raw8, q17)
+    tile = oracle.encode_tile(sym9, raw8, q16)
     states = np.frombuffer(tile[:128], "<u4")
     assert np.all(states == 65536)
     lane_words = []
@@ -266,44 +297,42 @@ def test_rans_all_escape_closed_form():
     assert np.array_equal(words, expect)
     assert len(tile) == (160 + 2 * len(expect) + 15) // 16 * 16
     assert all(b == 0 for b in tile[160 + 2 * len(expect):])
-    rc, s9, r8, st = oracle.decode_tile(tile, nvec, q17)
+    rc, s9, r8, st = oracle.decode_tile(tile, nvec, q16)
     assert rc == 0 and np.array_equal(s9, sym9) and np.array_equal(r8, raw8)
 
 
 def test_rans_lone_symbols_closed_form():
     """Every context holds one symbol with q = M: coding it costs nothing, so the tile is
     exactly the 32 states, all 2^16, and 16 zero region counts."""
-    q17 = _tables({127: M})
+    q16 = _tables({127: M})
     for nvec in (1, 31, 32, 33, 1000):
         sym9 = np.full((nvec, 9), 127, np.uint8)
         sym9[:, 0] = 0
-        tile = oracle.encode_tile(sym9, np.zeros((nvec, 8), np.int16), q17)
+        tile = oracle.encode_tile(sym9, np.zeros((nvec, 8), np.int16), q16)
         assert tile == np.full(32, 65536, "<u4").tobytes() + bytes(32)
-        rc, s9, _, _ = oracle.decode_tile(tile, nvec, q17)
+        rc, s9, _, _ = oracle.decode_tile(tile, nvec, q16)
         assert rc == 0 and np.array_equal(s9, sym9)
 
 
 def _random_tables(nsym_max=40):
-    q17 = np.zeros((17, 256), np.uint16)
-    counts = np.zeros((17, 256), np.uint64)
-    counts[0, :2] = RNG.integers(1, 100, 2)
-    for ctx in range(1, 17):
+    counts = np.zeros((16, 256), np.uint64)
+    for ctx in range(16):
         k = RNG.integers(1, nsym_max)
         sel = RNG.choice(256, k, replace=False)
         counts[ctx, sel] = RNG.integers(1, 1000, k) ** 2
-    for ctx in range(17):
-        q17[ctx] = oracle.quantize_table(counts[ctx])
-    return q17
+    return oracle.build_tables16(counts)
 
 
-def _draw(q17, nvec):
+def _draw(q16, nvec):
+    """Vectors drawn from the tables: (coset, f1) from the joint table, then f2..f8 given c."""
     sym9 = np.zeros((nvec, 9), np.uint8)
-    p0 = q17[0, :2] / M
-    sym9[:, 0] = RNG.choice(2, nvec, p=p0)
-    for u in range(1, 9):
+    joint = np.concatenate([q16[0], q16[8]]).astype(np.float64)
+    jt = RNG.choice(512, nvec, p=joint / joint.sum())
+    sym9[:, 0], sym9[:, 1] = jt // 256, jt % 256
+    for u in range(2, 9):
         for c in (0, 1):
             m = sym9[:, 0] == c
-            p = q17[1 + 8 * c + u - 1] / M
+            p = q16[8 * c + u - 1] / M
             sym9[m, u] = RNG.choice(256, int(m.sum()), p=p)
     raw8 = RNG.integers(-32768, 32768, (nvec, 8)).astype(np.int16)
     return sym9, raw8
@@ -311,11 +340,11 @@ def _draw(q17, nvec):
 
 def test_rans_roundtrip_random():
     for nvec in (1, 5, 32, 33, 63, 64, 65, 1000, 32 * 64):
-        q17 = _random_tables()
-        sym9, raw8 = _draw(q17, nvec)
-        tile = oracle.encode_tile(sym9, raw8, q17)
+        q16 = _random_tables()
+        sym9, raw8 = _draw(q16, nvec)
+        tile = oracle.encode_tile(sym9, raw8, q16)
         assert len(tile) % 16 == 0
-        rc, s9, r8, st = oracle.decode_tile(tile, nvec, q17)
+        rc, s9, r8, st = oracle.decode_tile(tile, nvec, q16)
         assert rc == 0
         assert np.array_equal(s9, sym9)
         esc = sym9[:, 1:] == 255
@@ -324,37 +353,38 @@ def test_rans_roundtrip_random():
 
 
 def test_rans_corruption_detected():
-    q17 = _random_tables()
-    sym9, raw8 = _draw(q17, 2048)
-    tile = bytearray(oracle.encode_tile(sym9, raw8, q17))
+    q16 = _random_tables()
+    sym9, raw8 = _draw(q16, 2048)
+    tile = bytearray(oracle.encode_tile(sym9, raw8, q16))
     tile[5] ^= 0x10                                                  # flip a bit of lane 1's state
-    rc, *_ = oracle.decode_tile(bytes(tile), 2048, q17)
+    rc, *_ = oracle.decode_tile(bytes(tile), 2048, q16)
     assert rc != 0
     tile[5] ^= 0x10
     tile[130] ^= 0x01                                                # a region count off by one
-    rc, *_ = oracle.decode_tile(bytes(tile), 2048, q17)
+    rc, *_ = oracle.decode_tile(bytes(tile), 2048, q16)
     assert rc != 0
     tile[130] ^= 0x01
-    rc, *_ = oracle.decode_tile(bytes(tile[:-32]), 2048, q17)       # truncated
+    rc, *_ = oracle.decode_tile(bytes(tile[:-32]), 2048, q16)       # truncated
     assert rc != 0
 
 
 def test_rans_size_near_cross_entropy():
     """Coded words carry the symbols' information: 16 * words + the information held by the
     final states (at most 16 bits per lane above 2^16) is the sum of -log2(q/M)."""
-    q17 = _random_tables(30)
+    q16 = _random_tables(30)
     nvec = 32 * 256
-    sym9, raw8 = _draw(q17, nvec)
-    tile = oracle.encode_tile(sym9, raw8, q17)
-    ctx = np.zeros((nvec, 9), np.int64)
-    ctx[:, 1:] = 1 + 8 * sym9[:, :1] + np.arange(8)[None, :]
-    q = q17[ctx, sym9].astype(np.float64)
+    sym9, raw8 = _draw(q16, nvec)
+    tile = oracle.encode_tile(sym9, raw8, q16)
+    ctx = 8 * sym9[:, :1].astype(np.int64) + np.arange(8)[None, :]          # field j: 8c + j - 1
+    q = q16[ctx, sym9[:, 1:]].astype(np.float64)                             # j = 1: joint (c, f1)
     info = -np.log2(q / M).sum() + 16.0 * (sym9[:, 1:] == 255).sum()
     states = np.frombuffer(tile[:128], "<u4").astype(np.float64)
     held = np.log2(states / 65536.0).sum()                          # bits parked in the states
     words_bits = 16.0 * int(np.frombuffer(tile[128:160], "<u2").astype(np.int64).sum())
-    assert words_bits + held >= info - 1e-6
-    assert words_bits + held <= info + 32 * 1.0
+    # Each encode step stores log2(M / q) bits up to its floor(x / q) rounding (a fraction of a
+    # bit over the whole tile here), and each lane's final state holds its last partial word:
+    # within one bit per lane.  A wrong frequency or context would be off by kilobits.
+    assert abs(words_bits + held - info) <= 32 * 1.0
 
 
 # ---------------------------------------------------------------------------------------------
