@@ -56,20 +56,24 @@ constexpr uint32_t kFull = 0xFFFFFFFFu;
 constexpr uint32_t kWaitSpins = 1u << 22;                     // bounded mbarrier wait (~0.3 s)
 constexpr uint32_t kSlotMask = kProbTotal - 1;
 constexpr uint32_t kCtxBytes = 4 * kProbTotal;                // one context's packed table: 4 KB
-constexpr uint32_t kTableBytes = kFieldContexts * kCtxBytes;  // 65536
-constexpr uint32_t kTablePiece = 16384;                       // bytes per table bulk copy
+// Decode tables: [0] the joint (coset, f1) symbol; [1 + 7c + (j - 2)] field j = 2..8 given coset c.
+constexpr int kDecodeTables = 15;
+constexpr uint32_t kTableBytes = kDecodeTables * kCtxBytes;   // 61440
+constexpr uint32_t kTablePiece = kTableBytes / 4;             // bytes per table bulk copy (15 KB)
 
-// Packed decode-table entry of slot u in context (c, j), symbol s = the one with
-// cum(s) <= u < cum(s) + q(s):
+// Packed decode-table entry of slot u, symbol s = the one with cum(s) <= u < cum(s) + q(s) (for
+// the joint table the symbol is the pair (c, s) and cum runs over coset 0's symbols first):
 //   bits  0..9   u - cum(s)           (< q(s) <= 1024)
 //   bits 10..18  2 s                  (bit 10 is zero)
 //   bit  19      s is the escape symbol
+//   bit  20      the coset c          (joint table only)
 //   bits 21..31  q(s)                 (<= 1024)
 // so the state update x <- q (x >> 10) + u - cum(s) takes two field extractions, and the
 // reconstruction takes 2 s out with one shift and mask.
 constexpr uint32_t kEntryBiasMask = 0x3FFu;
 constexpr uint32_t kEntrySymShift = 10;
 constexpr uint32_t kEntryEsc = 1u << 19;
+constexpr uint32_t kEntryCosetShift = 20;
 constexpr uint32_t kEntryQShift = 21;
 static_assert(kProbBits == 10, "the packed entry holds 10-bit slots");
 
@@ -95,7 +99,6 @@ struct Params {
     int64_t rows, cols, row_stride, n_vectors;
     uint32_t vec_per_row;       // < 2^31 (checked when the blob is parsed)
     uint32_t steps, n_tiles;
-    uint32_t q_coset0;          // frequency of coset 0; coset 1 has M - q_coset0
 };
 
 // Where the blob keeps the compact frequency tables the decode table is expanded from.
@@ -120,7 +123,7 @@ struct Geo {
 
 template <int WARPS>
 struct Smem {
-    uint32_t tab[kFieldContexts][kProbTotal];                       // packed decode table, 64 KB
+    uint32_t tab[kDecodeTables][kProbTotal];                        // packed decode tables, 60 KB
     alignas(16) uint8_t tbuf[WARPS][Geo<WARPS>::kBuf + kBufSlack];  // one staged tile per warp
     unsigned long long bar[WARPS];                                  // tile staging, one per warp
     unsigned long long tbar;                                        // the table's bulk copies
@@ -253,8 +256,23 @@ __device__ __forceinline__ void renorm_step(uint32_t& x, Reader& rd, bool active
 }
 
 // ---- table expansion -------------------------------------------------------------------------
-// Fills tab[16][1024] from the blob's compact frequency tables.  `scr` is shared-memory scratch
-// (BuildScratch) that the caller does not use meanwhile.
+// Largest symbol s with cum[s] <= slot: the symbol of that slot (its frequency is not zero).
+__device__ __forceinline__ uint32_t slot_symbol(const uint16_t* cum, uint32_t slot) {
+    uint32_t s = 0;
+#pragma unroll
+    for (uint32_t step = 128; step; step >>= 1)
+        if (cum[s + step] <= slot) s += step;
+    return s;
+}
+
+__device__ __forceinline__ uint32_t pack_entry(uint32_t bias, uint32_t s, uint32_t q, uint32_t coset) {
+    return bias | (s << (kEntrySymShift + 1)) | (s == uint32_t(kEscape) ? kEntryEsc : 0u) |
+           (coset << kEntryCosetShift) | (q << kEntryQShift);
+}
+
+// Fills tab[15][1024] from the blob's compact frequency tables (16 contexts; 0 and 8 together are
+// the joint (coset, f1) table).  `scr` is shared-memory scratch (BuildScratch) that the caller does
+// not use meanwhile.
 template <int WARPS>
 __device__ void build_tables(uint32_t (*tab)[kProbTotal], BuildScratch& scr, const TableSrc& p) {
     const uint32_t lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
@@ -289,32 +307,42 @@ __device__ void build_tables(uint32_t (*tab)[kProbTotal], BuildScratch& scr, con
     __syncthreads();
     // (b) slot -> packed entry.  Lane l of a warp writes slots it*32 + l of its part (one
     // 128-byte run per store instruction); each lane walks its symbol forward as its slots grow.
-    constexpr int P = WARPS >= 16 ? WARPS / 16 : 1;
+    constexpr int P = WARPS >= 15 ? WARPS / 15 : 1;
     constexpr uint32_t kSlotsPerPart = kProbTotal / P;
-    for (uint32_t item = warp; item < uint32_t(kFieldContexts * P); item += WARPS) {
-        const uint32_t ctx = item / P, part = item % P;
+    static_assert(kProbTotal % P == 0, "parts split the slots evenly");
+    for (uint32_t item = warp; item < uint32_t(kDecodeTables * P); item += WARPS) {
+        const uint32_t ti = item / P, part = item % P;
+        uint32_t* dst = tab[ti] + part * kSlotsPerPart;
+        if (ti == 0) {  // the joint table: coset 0's slots, then coset 1's
+            const uint32_t split = scr.cum[0][256];
+            for (uint32_t w = lane; w < kSlotsPerPart; w += 32) {
+                const uint32_t slot = part * kSlotsPerPart + w;
+                const uint32_t c = slot < split ? 0u : 1u;
+                const uint32_t local = slot - (c ? split : 0u);
+                const uint16_t* cum = scr.cum[8 * c];
+                const uint32_t sy = slot_symbol(cum, local);
+                dst[w] = pack_entry(local - cum[sy], sy, scr.q[8 * c][sy], c);
+            }
+            continue;
+        }
+        const uint32_t ctx = 8 * ((ti - 1) / 7) + 1 + (ti - 1) % 7;  // field j = 2..8 given coset c
         const uint16_t* cum = scr.cum[ctx];
         const uint16_t* qs = scr.q[ctx];
-        uint32_t* dst = tab[ctx] + part * kSlotsPerPart;
         if (cum[256] != kProbTotal) {  // context never used by this blob (the host checked the rest)
             for (uint32_t w = lane; w < kSlotsPerPart; w += 32) dst[w] = 0;
             continue;
         }
         const uint32_t first = part * kSlotsPerPart + lane;
-        uint32_t s = 0;  // largest symbol with cum(s) <= first
-#pragma unroll
-        for (uint32_t step = 128; step; step >>= 1)
-            if (cum[s + step] <= first) s += step;
-        uint32_t c0 = cum[s], next = cum[s + 1];
+        uint32_t sy = slot_symbol(cum, first);
+        uint32_t c0 = cum[sy], next = cum[sy + 1];
         for (uint32_t w = lane; w < kSlotsPerPart; w += 32) {
             const uint32_t slot = part * kSlotsPerPart + w;
             while (next <= slot) {
-                ++s;
+                ++sy;
                 c0 = next;
-                next = cum[s + 1];
+                next = cum[sy + 1];
             }
-            dst[w] = (slot - c0) | (s << (kEntrySymShift + 1)) | (s == uint32_t(kEscape) ? kEntryEsc : 0u) |
-                     (uint32_t(qs[s]) << kEntryQShift);
+            dst[w] = pack_entry(slot - c0, sy, qs[sy], 0u);
         }
     }
 }
@@ -444,27 +472,24 @@ template <int OUT, bool VEC, bool ESC, bool FULL, class Reader>
 __device__ __forceinline__ void decode_step(const Params& p, uint32_t tab, Reader& rd, uint32_t& x, bool active,
                                             const Pos& pos) {
     if (FULL) active = true;
-    // coset (two symbols: slot < q0 -> 0)
-    const uint32_t q0 = p.q_coset0;
-    const uint32_t cslot = x & kSlotMask;
-    const bool c1 = cslot >= q0;
-    if (active) x = (c1 ? kProbTotal - q0 : q0) * (x >> kProbBits) + (cslot - (c1 ? q0 : 0u));
-    renorm_step<FULL>(x, rd, active);
-
-    // fields f1..f8 with context (c, j): the 8 tables of coset 1 follow those of coset 0.  A lane
-    // past the last vector still loads (from its masked slot, inside the table) but keeps x.
-    const uint32_t c = c1 ? 1u : 0u;
-    const uint32_t tb = tab + (c1 ? 8u * kCtxBytes : 0u);
+    // (coset, f1) as one symbol of the joint table, then f2..f8 from the 7 tables of that coset.
+    // A lane past the last vector still loads (from its masked slot, inside the table) but keeps x.
     uint32_t e[8], acc = 0;
+    e[0] = lds_u32<0>(((x << 2) & (kSlotMask << 2)) | tab);
+    if (active) x = (e[0] >> kEntryQShift) * (x >> kProbBits) + (e[0] & kEntryBiasMask);
+    renorm_step<FULL>(x, rd, active);
+    if (ESC) acc = e[0];
+    const uint32_t c = (e[0] >> kEntryCosetShift) & 1u;
+    const uint32_t tb = tab + kCtxBytes + c * (7u * kCtxBytes);  // 4 KB aligned
 #define EP_FIELD(j)                                                                    \
     {                                                                                  \
-        const uint32_t ent = lds_u32<(j) * kCtxBytes>(((x << 2) & (kSlotMask << 2)) | tb); \
+        const uint32_t ent = lds_u32<((j) - 1) * kCtxBytes>(((x << 2) & (kSlotMask << 2)) | tb); \
         if (active) x = (ent >> kEntryQShift) * (x >> kProbBits) + (ent & kEntryBiasMask); \
         renorm_step<FULL>(x, rd, active);                                              \
         e[j] = ent;                                                                    \
         if (ESC) acc |= ent;                                                           \
     }
-    EP_FIELD(0) EP_FIELD(1) EP_FIELD(2) EP_FIELD(3) EP_FIELD(4) EP_FIELD(5) EP_FIELD(6) EP_FIELD(7)
+    EP_FIELD(1) EP_FIELD(2) EP_FIELD(3) EP_FIELD(4) EP_FIELD(5) EP_FIELD(6) EP_FIELD(7)
 #undef EP_FIELD
 
     bool from_symbols = true;
@@ -807,7 +832,7 @@ __global__ void __launch_bounds__(WARPS * 32, 1) group_kernel(const __grid_const
 
 // Expands the blob's compact frequency tables into the 64 KB packed decode table (one CTA).
 struct ExpandSmem {
-    uint32_t tab[kFieldContexts][kProbTotal];
+    uint32_t tab[kDecodeTables][kProbTotal];
     BuildScratch scratch;
 };
 
@@ -1003,7 +1028,6 @@ Params make_params(const ep_blob* b, const uint8_t* dblob, const uint8_t* tables
     p.vec_per_row = uint32_t(L.vec_per_row);
     p.steps = L.steps;
     p.n_tiles = L.n_tiles;
-    p.q_coset0 = L.q_coset[0];
     return p;
 }
 

@@ -133,14 +133,15 @@ __global__ void __launch_bounds__(kRowWarps * 32) rms_kernel(const In in, double
 }
 
 // ---- lattice quantisation: one thread per vector -----------------------------------------------
-// Rows: all (n_sample == 0) or the sampled rows floor(i * rows / n_sample).  Symbol counts go to
-// counts[17 * 256] and escapes; cosets and fields are written when coset != null.
+// Rows: all (n_sample == 0) or the sampled rows floor(i * rows / n_sample).  Symbol counts of the
+// 16 contexts (field j given coset c at 8c + j - 1) go to counts[16 * 256] and escapes; cosets and
+// fields are written when coset != null.
 __global__ void __launch_bounds__(256) quant_kernel(const In in, const double* rms, double s, int64_t n_sample,
                                                     unsigned long long* counts, unsigned long long* escapes,
                                                     uint8_t* coset_out, int16_t* fields_out) {
-    __shared__ uint32_t hist[17 * 256];
+    __shared__ uint32_t hist[16 * 256];
     __shared__ uint32_t esc;
-    for (int i = threadIdx.x; i < 17 * 256; i += blockDim.x) hist[i] = 0;
+    for (int i = threadIdx.x; i < 16 * 256; i += blockDim.x) hist[i] = 0;
     if (threadIdx.x == 0) esc = 0;
     __syncthreads();
     const int64_t nrows = n_sample ? n_sample : in.rows;
@@ -163,12 +164,11 @@ __global__ void __launch_bounds__(256) quant_kernel(const In in, const double* r
 #pragma unroll
         for (int e = 0; e < 7; ++e) { f[e] = z[e]; s7 += z[e]; }
         f[7] = (z[7] - (s7 & 1)) / 2;
-        atomicAdd(&hist[c], 1u);
         uint32_t ne = 0;
 #pragma unroll
         for (int j = 0; j < 8; ++j) {
             const int sy = symbol_of(f[j]);
-            atomicAdd(&hist[256 * (1 + 8 * c + j) + sy], 1u);
+            atomicAdd(&hist[256 * (8 * c + j) + sy], 1u);
             ne += sy == kEscape;
         }
         if (ne) atomicAdd(&esc, ne);
@@ -184,7 +184,7 @@ __global__ void __launch_bounds__(256) quant_kernel(const In in, const double* r
         }
     }
     __syncthreads();
-    for (int i = threadIdx.x; i < 17 * 256; i += blockDim.x)
+    for (int i = threadIdx.x; i < 16 * 256; i += blockDim.x)
         if (hist[i]) atomicAdd(&counts[i], (unsigned long long)hist[i]);
     if (threadIdx.x == 0 && esc) atomicAdd(escapes, (unsigned long long)esc);
 }
@@ -241,8 +241,8 @@ struct TileArgs {
     const int16_t* fields;
     int64_t n_vectors;
     uint32_t steps, n_tiles;
-    const uint16_t* q;          // [17][256]
-    const uint32_t* cum;        // [17][257]
+    const uint16_t* q;          // [16][256]
+    const uint32_t* cum;        // [16][257]
     uint32_t* lane_words;       // [n_tiles][32]: words of each lane (counting pass output)
     uint64_t* tile_bytes;       // [n_tiles] (counting pass output)
     const uint64_t* tile_off;   // [n_tiles] byte offsets in the stream (writing pass input)
@@ -254,10 +254,10 @@ constexpr int kTileWarps = 4;
 // WRITE = false: count every lane's words and the tile's size.  WRITE = true: write the tile.
 template <bool WRITE>
 __global__ void __launch_bounds__(kTileWarps * 32) tiles_kernel(const TileArgs a) {
-    __shared__ uint16_t q[17][256];
-    __shared__ uint32_t cum[17][257];
-    for (int i = threadIdx.x; i < 17 * 256; i += blockDim.x) q[i / 256][i % 256] = a.q[i];
-    for (int i = threadIdx.x; i < 17 * 257; i += blockDim.x) cum[i / 257][i % 257] = a.cum[i];
+    __shared__ uint16_t q[16][256];
+    __shared__ uint32_t cum[16][257];
+    for (int i = threadIdx.x; i < 16 * 256; i += blockDim.x) q[i / 256][i % 256] = a.q[i];
+    for (int i = threadIdx.x; i < 16 * 257; i += blockDim.x) cum[i / 257][i % 257] = a.cum[i];
     __syncthreads();
     const int lane = threadIdx.x & 31;
     const uint32_t tile = blockIdx.x * kTileWarps + (threadIdx.x >> 5);
@@ -299,8 +299,7 @@ __global__ void __launch_bounds__(kTileWarps * 32) tiles_kernel(const TileArgs a
         ++emitted;
     };
     uint32_t x = kStateLow;
-    auto put = [&](int ctx, int sym) {
-        const uint32_t f = q[ctx][sym], c = cum[ctx][sym];
+    auto code = [&](uint32_t f, uint32_t c) {
         if (uint64_t(x) >= (uint64_t(f) << (32 - kProbBits))) {  // renormalise: push 16 bits out
             emit(x & 0xFFFFu);
             x >>= 16;
@@ -314,8 +313,9 @@ __global__ void __launch_bounds__(kTileWarps * 32) tiles_kernel(const TileArgs a
         const int c = a.coset[v];
         for (int j = 7; j >= 0; --j)
             if (symbol_of(f[j]) == kEscape) emit(uint16_t(f[j]));
-        for (int j = 7; j >= 0; --j) put(1 + 8 * c + j, symbol_of(f[j]));
-        put(0, c);
+        for (int j = 7; j >= 1; --j) code(q[8 * c + j][symbol_of(f[j])], cum[8 * c + j][symbol_of(f[j])]);
+        const int s1 = symbol_of(f[0]);  // (coset, f1): coset 1's slots follow coset 0's
+        code(q[8 * c][s1], cum[8 * c][s1] + (c ? cum[0][256] : 0u));
     }
     if (!WRITE) {
         a.lane_words[size_t(tile) * kLanes + lane] = emitted;
@@ -373,7 +373,7 @@ int encode_gpu(const EncodeInput& in, double target, const EncodeOptions& opt, s
     In d{static_cast<const uint8_t*>(in.bits), in.dtype, dtype_bytes(in.dtype), rows, cols, in.row_stride, vpr};
     double* rms = buf.alloc<double>(size_t(rows));
     uint32_t* bad = buf.alloc<uint32_t>(1);
-    unsigned long long* counts = buf.alloc<unsigned long long>(17 * 256 + 1);
+    unsigned long long* counts = buf.alloc<unsigned long long>(16 * 256 + 1);
     uint8_t* coset = buf.alloc<uint8_t>(size_t(V));
     int16_t* fields = buf.alloc<int16_t>(size_t(V) * 8);
     float* alpha_d = buf.alloc<float>(size_t(rows));
@@ -389,18 +389,18 @@ int encode_gpu(const EncodeInput& in, double target, const EncodeOptions& opt, s
     if (bad_h) { why = "input holds a non-finite value"; return -4; }
 
     // counts of one quantisation pass (all rows or the sample) as host Counts
-    std::vector<unsigned long long> ch(17 * 256 + 1);
+    std::vector<unsigned long long> ch(16 * 256 + 1);
     auto quantise = [&](double s, int64_t n_sample, bool store, Counts& out) -> int {
-        EPG(cudaMemsetAsync(counts, 0, sizeof(unsigned long long) * (17 * 256 + 1), st), "encode: clear");
+        EPG(cudaMemsetAsync(counts, 0, sizeof(unsigned long long) * (16 * 256 + 1), st), "encode: clear");
         const int64_t work = (n_sample ? n_sample : rows) * vpr;
-        quant_kernel<<<unsigned((work + 255) / 256), 256, 0, st>>>(d, rms, s, n_sample, counts, counts + 17 * 256,
+        quant_kernel<<<unsigned((work + 255) / 256), 256, 0, st>>>(d, rms, s, n_sample, counts, counts + 16 * 256,
                                                                     store ? coset : nullptr, store ? fields : nullptr);
         EPG(cudaGetLastError(), "encode: quantise");
         EPG(cudaMemcpyAsync(ch.data(), counts, sizeof(unsigned long long) * ch.size(), cudaMemcpyDeviceToHost, st),
             "encode: read back");
         EPG(cudaStreamSynchronize(st), "encode: quantise");
-        for (int i = 0; i < 17 * 256; ++i) out.c[size_t(i)] = ch[size_t(i)];
-        out.escapes = ch[17 * 256];
+        for (int i = 0; i < 16 * 256; ++i) out.c[size_t(i)] = ch[size_t(i)];
+        out.escapes = ch[16 * 256];
         return 0;
     };
 
@@ -444,8 +444,8 @@ int encode_gpu(const EncodeInput& in, double target, const EncodeOptions& opt, s
     EPG(cudaMemcpyAsync(alpha.data(), alpha_d, 4 * size_t(rows), cudaMemcpyDeviceToHost, st), "encode: read back");
 
     // Tiles: count, lay out, write.
-    uint16_t* q_d = buf.alloc<uint16_t>(17 * 256);
-    uint32_t* cum_d = buf.alloc<uint32_t>(17 * 257);
+    uint16_t* q_d = buf.alloc<uint16_t>(16 * 256);
+    uint32_t* cum_d = buf.alloc<uint32_t>(16 * 257);
     uint32_t* lane_words = buf.alloc<uint32_t>(size_t(n_tiles) * kLanes);
     uint64_t* tbytes_d = buf.alloc<uint64_t>(size_t(n_tiles));
     uint64_t* toff_d = buf.alloc<uint64_t>(size_t(n_tiles));

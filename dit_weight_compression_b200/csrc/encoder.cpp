@@ -187,13 +187,18 @@ static void encode_tile(const uint8_t* coset, const int16_t* fields, int64_t nve
     uint32_t x[kLanes];
     std::vector<uint16_t> lw[kLanes];  // emission order (reverse of reading order)
     const int64_t steps = (nvec + kLanes - 1) / kLanes;
-    auto put = [&](uint32_t& st, std::vector<uint16_t>& w, int ctx, int sym) {
-        uint32_t f = T.q[ctx][sym], c = T.cum[ctx][sym];
+    auto code = [&](uint32_t& st, std::vector<uint16_t>& w, uint32_t f, uint32_t c) {
         if (uint64_t(st) >= (uint64_t(f) << (32 - kProbBits))) {  // renormalise: push 16 bits out
             w.push_back(uint16_t(st));
             st >>= 16;
         }
         st = (st / f) * kProbTotal + (st % f) + c;
+    };
+    auto put = [&](uint32_t& st, std::vector<uint16_t>& w, int ctx, int sym) {
+        code(st, w, T.q[ctx][sym], T.cum[ctx][sym]);
+    };
+    auto put_joint = [&](uint32_t& st, std::vector<uint16_t>& w, int coset, int sym) {
+        code(st, w, T.q[8 * coset][sym], T.joint_cum(coset, sym));
     };
     for (int l = 0; l < kLanes; ++l) {
         x[l] = kStateLow;
@@ -204,8 +209,8 @@ static void encode_tile(const uint8_t* coset, const int16_t* fields, int64_t nve
             const int16_t* f = &fields[size_t(8 * v)];
             for (int j = 7; j >= 0; --j)
                 if (symbol_of(f[j]) == kEscape) lw[l].push_back(uint16_t(f[j]));
-            for (int j = 7; j >= 0; --j) put(x[l], lw[l], 1 + 8 * coset[v] + j, symbol_of(f[j]));
-            put(x[l], lw[l], 0, coset[v]);
+            for (int j = 7; j >= 1; --j) put(x[l], lw[l], 8 * coset[v] + j, symbol_of(f[j]));
+            put_joint(x[l], lw[l], coset[v], symbol_of(f[0]));  // (coset, f1): one symbol
         }
     }
     size_t words = 0;
@@ -307,14 +312,13 @@ static std::vector<int> rd_allocate(const ElementReader& rd, const Quantiser& Q,
             const uint8_t* sy = &sym[(size_t(r) * R5 + size_t(kr[size_t(r)])) * per];
             for (int64_t k = 0; k < vpr; ++k) {
                 const int c = sy[9 * k];
-                all.c[size_t(c)]++;
-                for (int j = 0; j < 8; ++j) all.c[size_t(256 * (1 + 8 * c + j) + sy[9 * k + 1 + j])]++;
+                for (int j = 0; j < 8; ++j) all.c[size_t(256 * (8 * c + j) + sy[9 * k + 1 + j])]++;
             }
         }
         Tables T;
         T.build(all);
-        double cost[17 * 256];
-        for (int c = 0; c < 17; ++c)
+        double cost[16 * 256];
+        for (int c = 0; c < 16; ++c)
             for (int sy = 0; sy < 256; ++sy)
                 cost[256 * c + sy] = T.q[c][sy] ? -std::log2(double(T.q[c][sy]) / double(kProbTotal))
                                                 : std::log2(double(kProbTotal));
@@ -326,8 +330,7 @@ static std::vector<int> rd_allocate(const ElementReader& rd, const Quantiser& Q,
                     double bits = 16.0 * double(nesc[idx]);
                     for (int64_t k = 0; k < vpr; ++k) {
                         const int c = sy[9 * k];
-                        bits += cost[sy[9 * k]];
-                        for (int j = 0; j < 8; ++j) bits += cost[256 * (1 + 8 * c + j) + sy[9 * k + 1 + j]];
+                        for (int j = 0; j < 8; ++j) bits += cost[256 * (8 * c + j) + sy[9 * k + 1 + j]];
                     }
                     R[idx] = bits;
                 }
@@ -380,10 +383,7 @@ bool assemble_blob(int dtype, int64_t rows, int64_t cols, int S, double s, const
     wr64(p + 64, off_offs);
     wr64(p + 72, off_stream);
     uint8_t* t = p + off_tab;
-    wr16(t, T.q[0][0]);
-    wr16(t + 2, T.q[0][1]);
-    t += 4;
-    for (int c = 1; c < 17; ++c) {
+    for (int c = 0; c < 16; ++c) {
         int lo, cnt;
         T.range(c, lo, cnt);
         wr16(t, T.q[c][kEscape]);
@@ -559,15 +559,12 @@ bool parse_blob(const uint8_t* d, size_t n, BlobLayout& L, std::string& why) {
     auto aligned = [](uint64_t o) { return (o & 15) == 0; };
     if (!aligned(L.off_tables) || !aligned(L.off_alpha) || !aligned(L.off_offsets) || !aligned(L.off_stream))
         return fail("misaligned section");
-    if (L.off_tables < kHeaderBytes || L.off_tables + 4 > L.off_alpha ||
+    if (L.off_tables < kHeaderBytes || L.off_tables > L.off_alpha ||
         L.off_alpha + 4 * uint64_t(L.rows) > L.off_offsets ||
         L.off_offsets + 4 * (uint64_t(L.n_tiles) + 1) > L.off_stream || L.off_stream > n)
         return fail("sections overlap or run past the end");
-    const uint8_t* t = d + L.off_tables;
-    L.q_coset[0] = rd16(t);
-    L.q_coset[1] = rd16(t + 2);
-    if (uint32_t(L.q_coset[0]) + L.q_coset[1] != kProbTotal) return fail("coset table does not sum to 1024");
-    uint64_t pos = L.off_tables + 4;
+    uint64_t pos = L.off_tables;
+    uint32_t sums[kFieldContexts];
     for (int c = 0; c < kFieldContexts; ++c) {
         if (pos + 4 > L.off_alpha) return fail("table section truncated");
         L.esc_q[c] = rd16(d + pos);
@@ -579,8 +576,11 @@ bool parse_blob(const uint8_t* d, size_t n, BlobLayout& L, std::string& why) {
         if (pos > L.off_alpha) return fail("table section truncated");
         uint32_t sum = L.esc_q[c];
         for (int i = 0; i < L.n[c]; ++i) sum += rd16(d + L.q_offset[c] + 2 * i);
-        if (sum != 0 && sum != kProbTotal) return fail("field table does not sum to 1024");
+        sums[c] = sum;
+        if (c != 0 && c != 8 && sum != 0 && sum != kProbTotal) return fail("field table does not sum to 1024");
     }
+    L.joint_split = sums[0];  // coset-0 half of the joint (coset, f1) table
+    if (sums[0] + sums[8] != kProbTotal) return fail("joint (coset, f1) table does not sum to 1024");
     for (int c = 0; c < kFieldContexts; ++c)
         if (L.esc_q[c]) L.has_escape = 1;
     const uint8_t* off = d + L.off_offsets;

@@ -5,11 +5,12 @@
 // and reconstruction") says must travel with the rANS-coded fields: the frequency tables, one
 // scale per row, and the per-tile bookkeeping.  Byte layout (little-endian, every section 16-byte aligned):
 //
-//   header, 80 bytes:  "EPK1" | u16 version = 2 | u8 dtype | u8 R = 127 | u64 rows | u64 cols |
+//   header, 80 bytes:  "EPK1" | u16 version = 3 | u8 dtype | u8 R = 127 | u64 rows | u64 cols |
 //                      u32 S | u32 n_tiles | f64 s | u64 total bytes | u64 table offset |
 //                      u64 row-scale offset | u64 tile-offset offset | u64 stream offset
-//   tables:            u16 q(coset 0), u16 q(coset 1); then for c = 0, 1 and j = 1..8:
-//                      u16 q(escape), u8 lo, u8 n, u16 q[lo .. lo + n - 1]
+//   tables:            for c = 0, 1 and j = 1..8: u16 q(escape), u8 lo, u8 n,
+//                      u16 q[lo .. lo + n - 1]; the two j = 1 tables are the coset halves of
+//                      one table over the pairs (coset, f1), summing to M together
 //   row scales:        f32 per row
 //   tile offsets:      u32[n_tiles + 1], in 16-byte units from the stream start
 //   stream:            per tile: 32 u32 initial rANS states (lane order), 16 u16 region word
@@ -17,8 +18,8 @@
 //                      2p+1's backward from its end), zero padding to a multiple of 16 bytes
 //
 // Symbols: field value f with |f| <= 127 is the symbol f + 127; any other value is the escape
-// symbol 255 followed by the raw int16 word.  Frequencies of every used context sum to
-// M = 1024 (version 2; 10-bit totals).
+// symbol 255 followed by the raw int16 word.  A vector is 8 rANS symbols: (coset, f1), then
+// f2..f8 given the coset.  Frequencies of every used context sum to M = 1024 (10-bit totals).
 #pragma once
 
 #include <cstdint>
@@ -35,7 +36,7 @@
 
 namespace ep {
 
-constexpr uint32_t kVersion = 2;
+constexpr uint32_t kVersion = 3;
 constexpr int kAlphabetR = 127;
 constexpr int kEscape = 255;
 constexpr uint32_t kProbBits = 10;
@@ -43,7 +44,8 @@ constexpr uint32_t kProbTotal = 1u << kProbBits;  // M = 1024
 constexpr uint32_t kStateLow = 1u << 16;          // rANS lower bound, 16-bit renormalisation
 constexpr int kLanes = 32;                        // interleaved states per tile
 constexpr int kPairs = kLanes / 2;                // lanes 2p, 2p+1 share word region p
-constexpr int kFieldContexts = 16;                // (coset c, field j) -> 8c + j - 1
+constexpr int kFieldContexts = 16;                // (coset c, field j) -> 8c + j - 1; 0 and 8
+                                                  // together: the joint (coset, f1) table
 constexpr size_t kHeaderBytes = 80;
 constexpr size_t kTileHeadBytes = 4 * kLanes + 2 * kPairs;  // 32 u32 states + 16 u16 counts
 constexpr double kTargetMin = 0.001, kTargetMax = 11.0;
@@ -70,7 +72,7 @@ struct BlobLayout {
     int has_escape = 0;           // some field context gives the escape symbol a frequency
     double scale = 0.0;
     uint64_t total = 0, off_tables = 0, off_alpha = 0, off_offsets = 0, off_stream = 0;
-    uint16_t q_coset[2] = {0, 0};
+    uint32_t joint_split = 0;     // slots of coset 0 in the joint (coset, f1) table
     // field contexts: escape frequency, symbol range, byte offset of q[] inside the blob
     uint16_t esc_q[kFieldContexts] = {};
     uint8_t lo[kFieldContexts] = {}, n[kFieldContexts] = {};

@@ -16,15 +16,15 @@ namespace ep {
 // Field value -> symbol: f + 127 for |f| <= 127, else the escape symbol.
 EP_HD inline int symbol_of(int32_t f) { return (f >= -kAlphabetR && f <= kAlphabetR) ? f + kAlphabetR : kEscape; }
 
-// Symbol counts of the 17 contexts: [0] the coset (symbols 0/1), [1 + 8c + j - 1] field j | c.
+// Symbol counts of the 16 contexts, field j (1..8) given coset c at 8c + j - 1.  Contexts 0 and 8
+// (field 1) are the two coset halves of the joint (coset, f1) symbol.
 struct Counts {
-    std::vector<uint64_t> c = std::vector<uint64_t>(17 * 256, 0);
+    std::vector<uint64_t> c = std::vector<uint64_t>(16 * 256, 0);
     uint64_t escapes = 0;
     void add(int coset, const int32_t f[8]) {
-        c[size_t(coset)]++;
         for (int j = 0; j < 8; ++j) {
             int sy = symbol_of(f[j]);
-            c[size_t(256 * (1 + 8 * coset + j) + sy)]++;
+            c[size_t(256 * (8 * coset + j) + sy)]++;
             escapes += sy == kEscape;
         }
     }
@@ -37,13 +37,13 @@ struct Counts {
 // 10-bit frequencies from counts: q = max(1, round-half-up(M n / N)) for used symbols, then
 // the sum is brought to M -- excess taken one at a time from the largest q (> 1, lowest symbol
 // first), deficit given one at a time to the most frequent symbol (lowest symbol first).
-inline void quantise_freqs(const uint64_t* n, uint16_t* q) {
+inline void quantise_freqs(const uint64_t* n, uint16_t* q, int nb = 256) {
     uint64_t total = 0;
-    for (int s = 0; s < 256; ++s) total += n[s];
-    std::fill(q, q + 256, uint16_t(0));
+    for (int s = 0; s < nb; ++s) total += n[s];
+    std::fill(q, q + nb, uint16_t(0));
     if (total == 0) return;
     int64_t sum = 0;
-    for (int s = 0; s < 256; ++s) {
+    for (int s = 0; s < nb; ++s) {
         if (!n[s]) continue;
         uint64_t v = (2 * uint64_t(kProbTotal) * n[s] + total) / (2 * total);
         q[s] = uint16_t(std::max<uint64_t>(v, 1));
@@ -51,34 +51,47 @@ inline void quantise_freqs(const uint64_t* n, uint16_t* q) {
     }
     while (sum > int64_t(kProbTotal)) {
         int best = -1;
-        for (int s = 0; s < 256; ++s)
+        for (int s = 0; s < nb; ++s)
             if (q[s] > 1 && (best < 0 || q[s] > q[best])) best = s;
         --q[best];
         --sum;
     }
     while (sum < int64_t(kProbTotal)) {
         int best = -1;
-        for (int s = 0; s < 256; ++s)
+        for (int s = 0; s < nb; ++s)
             if (n[s] && (best < 0 || n[s] > n[best])) best = s;
         ++q[best];
         ++sum;
     }
 }
 
+// The 16 context tables.  Contexts 0 and 8 are quantised together as one 512-symbol table over
+// the pairs (coset, f1) (coset-major, so ties go to coset 0 first), the others one by one.  The
+// joint symbol (c, s) has frequency q[8c][s] and cumulative frequency joint_cum(c, s): coset 1's
+// slots follow all of coset 0's.
 struct Tables {
-    uint16_t q[17][256];
-    uint32_t cum[17][257];
+    uint16_t q[16][256];
+    uint32_t cum[16][257];
     void build(const Counts& cnt) {
-        for (int c = 0; c < 17; ++c) {
-            quantise_freqs(&cnt.c[size_t(256 * c)], q[c]);
+        uint64_t nj[512];
+        uint16_t qj[512];
+        std::copy(&cnt.c[0], &cnt.c[0] + 256, nj);
+        std::copy(&cnt.c[256 * 8], &cnt.c[256 * 8] + 256, nj + 256);
+        quantise_freqs(nj, qj, 512);
+        std::copy(qj, qj + 256, q[0]);
+        std::copy(qj + 256, qj + 512, q[8]);
+        for (int c = 1; c < 16; ++c)
+            if (c != 8) quantise_freqs(&cnt.c[size_t(256 * c)], q[c]);
+        for (int c = 0; c < 16; ++c) {
             cum[c][0] = 0;
             for (int s = 0; s < 256; ++s) cum[c][s + 1] = cum[c][s] + q[c][s];
         }
     }
+    uint32_t joint_cum(int coset, int s) const { return cum[8 * coset][s] + (coset ? cum[0][256] : 0u); }
     // serialised size of the table section (before padding)
     uint64_t section_bytes() const {
-        uint64_t b = 4;
-        for (int c = 1; c < 17; ++c) {
+        uint64_t b = 0;
+        for (int c = 0; c < 16; ++c) {
             int lo, cnt;
             range(c, lo, cnt);
             b += 4 + 2 * uint64_t(cnt);
@@ -110,7 +123,7 @@ inline double estimate_from_counts(const Counts& all, int64_t rows, int64_t cols
     Tables T;
     T.build(all);
     double bits = 0.0;
-    for (int c = 0; c < 17; ++c)
+    for (int c = 0; c < 16; ++c)
         for (int sy = 0; sy < 256; ++sy) {
             uint64_t n = all.c[size_t(256 * c + sy)];
             if (n) bits += double(n) * -std::log2(double(T.q[c][sy]) / double(kProbTotal));

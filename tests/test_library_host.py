@@ -145,7 +145,7 @@ def test_corrupt_blobs_rejected(ep):
         b[:-16],                                           # size mismatch
         _corrupt(b, 24, (1).to_bytes(4, "little")),        # S inconsistent with n_tiles
         _corrupt(b, 48, (81).to_bytes(8, "little")),       # misaligned table section
-        _corrupt(b, 80, (1023).to_bytes(2, "little")),     # coset table does not sum to 1024
+        _corrupt(b, 80, (1023).to_bytes(2, "little")),     # joint (coset, f1) table off 1024
     ]
     off_offs = int.from_bytes(b[64:72], "little")
     bad.append(_corrupt(b, off_offs + 4, (3).to_bytes(4, "little")))   # tile shorter than its header
