@@ -103,7 +103,7 @@ struct In {
 };
 
 // ---- row RMS: 32 rows per warp, column order ---------------------------------------------------
-constexpr int kRowWarps = 4;  // warps per block of the row kernels
+constexpr int kRowWarps = 1;  // warps per block of the row kernels (32 rows per block)
 
 __global__ void __launch_bounds__(kRowWarps * 32) rms_kernel(const In in, double* rms, uint32_t* bad) {
     __shared__ double sq[kRowWarps][32][33];
@@ -114,14 +114,14 @@ __global__ void __launch_bounds__(kRowWarps * 32) rms_kernel(const In in, double
     bool finite = true;
     for (int64_t c0 = 0; c0 < in.cols; c0 += 32) {
         const int64_t c = c0 + lane;
+        double v[32];
+#pragma unroll
+        for (int i = 0; i < 32; ++i)  // all loads first, so their latencies overlap
+            v[i] = (r0 + i < in.rows && c < in.cols) ? load_elem(in.base, in.dtype, (r0 + i) * in.stride + c) : 0.0;
+#pragma unroll
         for (int i = 0; i < 32; ++i) {
-            double sqv = 0.0;
-            if (r0 + i < in.rows && c < in.cols) {
-                const double v = load_elem(in.base, in.dtype, (r0 + i) * in.stride + c);
-                finite = finite && isfinite(v);
-                sqv = __dmul_rn(v, v);
-            }
-            sq[w][i][lane] = sqv;
+            finite = finite && isfinite(v[i]);
+            sq[w][i][lane] = __dmul_rn(v[i], v[i]);
         }
         __syncwarp();
         const int n = int(in.cols - c0 < 32 ? in.cols - c0 : 32);
@@ -190,19 +190,9 @@ __global__ void __launch_bounds__(256) quant_kernel(const In in, const double* r
 }
 
 // ---- row least-squares scales: alpha_r = sum w y / sum y^2 over real columns, column order ----
-__device__ __forceinline__ double lattice_coord(const uint8_t* coset, const int16_t* fields, int64_t v, int e) {
-    const int16_t* f = fields + 8 * v;
-    int32_t z;
-    if (e < 7) {
-        z = f[e];
-    } else {
-        int32_t s7 = 0;
-        for (int j = 0; j < 7; ++j) s7 += f[j];
-        z = 2 * int32_t(f[7]) + (s7 & 1);
-    }
-    return double(z) + 0.5 * coset[v];  // exact: a half-integer far below 2^52
-}
-
+// Per 32-column chunk of 32 rows (128 vectors), each lane takes 4 vectors: it reads the vector's
+// coset and fields once, rebuilds its 8 lattice coordinates (y = z + c/2, z8 = 2 f8 + parity) and
+// stages w y and y^2 for every real column; then every lane adds its row's terms in column order.
 __global__ void __launch_bounds__(kRowWarps * 32) alpha_kernel(const In in, const uint8_t* coset,
                                                                const int16_t* fields, float* alpha) {
     extern __shared__ double sh[];  // [kRowWarps][2][32][33]
@@ -213,16 +203,37 @@ __global__ void __launch_bounds__(kRowWarps * 32) alpha_kernel(const In in, cons
     if (r0 >= in.rows) return;
     double swy = 0.0, syy = 0.0;
     for (int64_t c0 = 0; c0 < in.cols; c0 += 32) {
-        const int64_t c = c0 + lane;
-        for (int i = 0; i < 32; ++i) {
-            double a = 0.0, b = 0.0;
-            if (r0 + i < in.rows && c < in.cols) {
-                const double y = lattice_coord(coset, fields, (r0 + i) * in.vpr + c / 8, int(c % 8));
-                a = __dmul_rn(load_elem(in.base, in.dtype, (r0 + i) * in.stride + c), y);
-                b = __dmul_rn(y, y);
+#pragma unroll
+        for (int m = 0; m < 4; ++m) {
+            const int q = m * 32 + lane, i = q >> 2, vk = q & 3;
+            const int64_t r = r0 + i, col0 = c0 + 8 * vk;
+            double a[8], b[8];
+#pragma unroll
+            for (int e = 0; e < 8; ++e) a[e] = b[e] = 0.0;
+            if (r < in.rows && col0 < in.cols) {
+                const int64_t v = r * in.vpr + col0 / 8;
+                const int4 pk = reinterpret_cast<const int4*>(fields)[v];
+                const int32_t f[8] = {int16_t(pk.x & 0xFFFF), int16_t(uint32_t(pk.x) >> 16),
+                                      int16_t(pk.y & 0xFFFF), int16_t(uint32_t(pk.y) >> 16),
+                                      int16_t(pk.z & 0xFFFF), int16_t(uint32_t(pk.z) >> 16),
+                                      int16_t(pk.w & 0xFFFF), int16_t(uint32_t(pk.w) >> 16)};
+                const double half = 0.5 * coset[v];
+                const int32_t s7 = f[0] + f[1] + f[2] + f[3] + f[4] + f[5] + f[6];
+#pragma unroll
+                for (int e = 0; e < 8; ++e) {
+                    if (col0 + e < in.cols) {
+                        const int32_t z = e < 7 ? f[e] : 2 * f[7] + (s7 & 1);
+                        const double y = double(z) + half;  // exact: a half-integer
+                        a[e] = __dmul_rn(load_elem(in.base, in.dtype, r * in.stride + col0 + e), y);
+                        b[e] = __dmul_rn(y, y);
+                    }
+                }
             }
-            wy[i][lane] = a;
-            yy[i][lane] = b;
+#pragma unroll
+            for (int e = 0; e < 8; ++e) {
+                wy[i][8 * vk + e] = a[e];
+                yy[i][8 * vk + e] = b[e];
+            }
         }
         __syncwarp();
         const int n = int(in.cols - c0 < 32 ? in.cols - c0 : 32);
@@ -332,16 +343,19 @@ __global__ void __launch_bounds__(kTileWarps * 32) tiles_kernel(const TileArgs a
     }
 }
 
-// Device buffers of one encode, freed on every exit path.
+// Device buffers of one encode, from the device's stream-ordered pool (freed memory is reused by
+// the next encode without a device-wide synchronisation), released on every exit path.
 struct DevBuf {
+    cudaStream_t st;
     std::vector<void*> ptrs;
+    explicit DevBuf(cudaStream_t s) : st(s) {}
     ~DevBuf() {
-        for (void* p : ptrs) cudaFree(p);
+        for (void* p : ptrs) cudaFreeAsync(p, st);
     }
     template <class T>
     T* alloc(size_t n) {
         void* p = nullptr;
-        if (cudaMalloc(&p, std::max<size_t>(n, 1) * sizeof(T)) != cudaSuccess) return nullptr;
+        if (cudaMallocAsync(&p, std::max<size_t>(n, 1) * sizeof(T), st) != cudaSuccess) return nullptr;
         ptrs.push_back(p);
         return static_cast<T*>(p);
     }
@@ -359,7 +373,7 @@ int encode_gpu(const EncodeInput& in, double target, const EncodeOptions& opt, s
     const int64_t n_tiles = (V + per_tile - 1) / per_tile;
     if (n_tiles > int64_t(UINT32_MAX) - 1) { why = "too many tiles"; return -3; }
     cudaStream_t st = cudaStreamPerThread;
-    DevBuf buf;
+    DevBuf buf(st);
     auto cuda_fail = [&](cudaError_t e, const char* what) {
         why = std::string(what) + ": " + cudaGetErrorString(e);
         return -6;
