@@ -9,21 +9,22 @@
 //   * one warp per tile; the tile's 32 interleaved rANS states live one per lane;
 //   * one persistent CTA of 32 warps per SM (grid = min(#SM, #tiles)); tile t goes to CTA
 //     t mod grid, so every SM gets an equal share even when there are few tiles;
-//   * decode table: per field context one packed 32-bit entry per slot of the 1024-slot range,
-//     {slot - cum(s), 2 s, escape flag, q(s)}, 64 KB in all, so one shared-memory load per symbol
-//     gives everything the state update needs.  It is expanded once per blob and device by a
-//     small kernel into a block next to the device copy; every CTA stages that block into shared
-//     memory with bulk copies, overlapped with the fetch of its first tiles.  (The
-//     allocation-free entry point expands it inside each CTA instead.)  The coset context, two
-//     symbols, is decoded by one compare;
+//   * decode tables: one packed 32-bit entry per slot of the 1024-slot range, {slot - cum(s), 2 s,
+//     escape flag, coset bit, q(s)}, for the joint (coset, f1) symbol and for f2..f8 given each
+//     coset -- 15 tables, 60 KB -- so one shared-memory load per symbol gives everything the
+//     state update needs.  They are expanded once per blob and device by a small kernel into a
+//     block next to the device copy; every CTA stages that block into shared memory with bulk
+//     copies, overlapped with the fetch of its first tiles.  (The allocation-free entry point
+//     expands them inside each CTA instead.);
 //   * words: every lane reads its own word stream.  Lanes 2p and 2p+1 share region p of the tile
 //     (one forward from the region start, one backward from its end); a warp-shuffle prefix sum
 //     over the 16 region counts gives every lane its start.  The whole tile is staged into a
 //     per-warp shared-memory buffer by one bulk copy (the next tile is prefetched into L2); each
 //     lane has its next word loaded before it needs it, so a renormalisation costs one compare
 //     and one byte permute on the dependent chain;
-//   * per step a lane decodes one 8-vector: 9 rANS symbols (each followed by its conditional
-//     refill), then the raw words of its escaped fields; fields are inverted in registers
+//   * per step a lane decodes one 8-vector: 8 rANS symbols, (coset, f1) then f2..f8 (each
+//     followed by its conditional refill), then the raw words of its escaped fields; fields are
+//     inverted in registers
 //     (z8 = 2 f8 + parity, y = z + c/2), multiplied by the row's fp32 scale, converted one pair
 //     per cvt and written as one 16-byte store per lane (a 512-byte contiguous run per warp for
 //     BF16/FP16).

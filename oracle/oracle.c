@@ -695,7 +695,8 @@ static void quantise_vector(const matrix* m, int64_t r, int64_t k, double s, dou
     orc_e8_nearest(t, y, coset);
 }
 
-/* The nine symbols of a quantised vector and the raw values of escaped fields. */
+/* A quantised vector's coset and field symbols (9 values; the coset is coded with f1) and the raw
+ * values of escaped fields. */
 static void vector_symbols(const double y[8], int coset, uint8_t sym[9], int16_t raw[8])
 {
     int32_t f[8];
