@@ -27,7 +27,8 @@
 //     inverted in registers
 //     (z8 = 2 f8 + parity, y = z + c/2), multiplied by the row's fp32 scale, converted one pair
 //     per cvt and written as one 16-byte store per lane (a 512-byte contiguous run per warp for
-//     BF16/FP16).
+//     BF16/FP16).  Steps are software-pipelined: step k + 1's symbols are decoded before step k
+//     is written, so the writes fill the stalls of the rANS chain.
 // No tensor cores: the path is table lookups and integer arithmetic, bound by HBM bytes and by
 // the latency and issue slots of that arithmetic, not by a contraction.
 #include <cuda_bf16.h>
@@ -65,12 +66,13 @@ constexpr uint32_t kTablePiece = kTableBytes / 4;             // bytes per table
 // Packed decode-table entry of slot u, symbol s = the one with cum(s) <= u < cum(s) + q(s) (for
 // the joint table the symbol is the pair (c, s) and cum runs over coset 0's symbols first):
 //   bits  0..9   u - cum(s)           (< q(s) <= 1024)
-//   bits 10..18  2 s                  (bit 10 is zero)
+//   bits 10..18  s at bit 10 for fields 1..7 (bit 18 zero), s at bit 11 for field 8 (bit 10 zero)
 //   bit  19      s is the escape symbol
 //   bit  20      the coset c          (joint table only)
 //   bits 21..31  q(s)                 (<= 1024)
-// so the state update x <- q (x >> 10) + u - cum(s) takes two field extractions, and the
-// reconstruction takes 2 s out with one shift and mask.
+// so the state update x <- q (x >> 10) + u - cum(s) takes two field extractions, and one mask
+// puts s (or 2 s for field 8, whose lattice coordinate is 2 f8 + parity) in place as mantissa
+// bits of the float the reconstruction starts from.
 constexpr uint32_t kEntryBiasMask = 0x3FFu;
 constexpr uint32_t kEntrySymShift = 10;
 constexpr uint32_t kEntryEsc = 1u << 19;
@@ -194,6 +196,13 @@ __device__ __forceinline__ uint32_t lds_u32(uint32_t a) {
     asm volatile("ld.shared.u32 %0, [%1+%2];" : "=r"(v) : "r"(a), "n"(OFF));
     return v;
 }
+// Shared address of slot (x mod M) of a 4 KB-aligned table at `base`: a mask and a multiply-add,
+// which keeps one of the two steps off the integer ALU pipe.
+__device__ __forceinline__ uint32_t slot_addr(uint32_t x, uint32_t base) {
+    uint32_t a;
+    asm("{\n .reg .b32 t;\n and.b32 t, %1, 1023;\n mad.lo.u32 %0, t, 4, %2;\n}" : "=r"(a) : "r"(x), "r"(base));
+    return a;
+}
 
 // Prefetch `bytes` (a multiple of 16) at a 16-byte aligned global address into L2.
 __device__ __forceinline__ void prefetch_l2(const void* p, uint32_t bytes) {
@@ -202,7 +211,7 @@ __device__ __forceinline__ void prefetch_l2(const void* p, uint32_t bytes) {
 
 // A lane's word stream, read from the warp's shared-memory copy of the tile.  `wp` is the
 // shared address of the lane's next word and `wn` that word, loaded right after the previous
-// one was used -- well before it is needed, so a refill costs a compare and a byte permute on
+// one was used -- well before it is needed, so a refill costs a compare and a multiply-add on
 // the dependent chain.  Predicated loads keep the warp converged.
 struct SmemReader {
     uint32_t wp, wn;
@@ -233,19 +242,19 @@ struct GlobalReader {
 };
 
 // Renormalisation after one decoded symbol: a lane whose state fell below 2^16 shifts in its
-// next word (x * 2^16 + w, i.e. the byte permutation {w.lo, w.hi, x.lo, x.hi}) and loads the
-// word after it.
+// next word (x * 2^16 + w) and loads the word after it.
 template <class Reader>
 __device__ __forceinline__ void renorm(uint32_t& x, Reader& rd, bool active) {
     const bool need = active && x < kStateLow;
     x = need ? __byte_perm(rd.wn, x, 0x5410) : x;
     rd.consume_if(need);
 }
-// The same for full steps from shared memory, as one predicated block: compare, permute,
-// advance, load -- no materialised predicate or select.
+// The same for full steps from shared memory, as one predicated block: compare, multiply-add
+// (on the FMA pipe, which the rest of the step leaves idle), advance, load -- no materialised
+// predicate or select.
 __device__ __forceinline__ void renorm(uint32_t& x, SmemReader& rd) {
     asm volatile(
-        "{\n .reg .pred p;\n setp.lt.u32 p, %0, 65536;\n @p prmt.b32 %0, %1, %0, 0x5410;\n"
+        "{\n .reg .pred p;\n setp.lt.u32 p, %0, 65536;\n @p mad.lo.u32 %0, %0, 65536, %1;\n"
         " @p add.u32 %2, %2, %3;\n @p ld.shared.u16 %1, [%2];\n}"
         : "+r"(x), "+r"(rd.wn), "+r"(rd.wp)
         : "r"(rd.wd));
@@ -266,8 +275,8 @@ __device__ __forceinline__ uint32_t slot_symbol(const uint16_t* cum, uint32_t sl
     return s;
 }
 
-__device__ __forceinline__ uint32_t pack_entry(uint32_t bias, uint32_t s, uint32_t q, uint32_t coset) {
-    return bias | (s << (kEntrySymShift + 1)) | (s == uint32_t(kEscape) ? kEntryEsc : 0u) |
+__device__ __forceinline__ uint32_t pack_entry(uint32_t bias, uint32_t s, uint32_t q, uint32_t coset, uint32_t sh) {
+    return bias | (s << sh) | (s == uint32_t(kEscape) ? kEntryEsc : 0u) |
            (coset << kEntryCosetShift) | (q << kEntryQShift);
 }
 
@@ -322,13 +331,14 @@ __device__ void build_tables(uint32_t (*tab)[kProbTotal], BuildScratch& scr, con
                 const uint32_t local = slot - (c ? split : 0u);
                 const uint16_t* cum = scr.cum[8 * c];
                 const uint32_t sy = slot_symbol(cum, local);
-                dst[w] = pack_entry(local - cum[sy], sy, scr.q[8 * c][sy], c);
+                dst[w] = pack_entry(local - cum[sy], sy, scr.q[8 * c][sy], c, kEntrySymShift);
             }
             continue;
         }
         const uint32_t ctx = 8 * ((ti - 1) / 7) + 1 + (ti - 1) % 7;  // field j = 2..8 given coset c
         const uint16_t* cum = scr.cum[ctx];
         const uint16_t* qs = scr.q[ctx];
+        const uint32_t sh = (ti - 1) % 7 == 6 ? kEntrySymShift + 1 : kEntrySymShift;  // field 8: 2 s
         if (cum[256] != kProbTotal) {  // context never used by this blob (the host checked the rest)
             for (uint32_t w = lane; w < kSlotsPerPart; w += 32) dst[w] = 0;
             continue;
@@ -343,7 +353,7 @@ __device__ void build_tables(uint32_t (*tab)[kProbTotal], BuildScratch& scr, con
                 c0 = next;
                 next = cum[sy + 1];
             }
-            dst[w] = pack_entry(slot - c0, sy, qs[sy], 0u);
+            dst[w] = pack_entry(slot - c0, sy, qs[sy], 0u, sh);
         }
     }
 }
@@ -468,23 +478,33 @@ __device__ __forceinline__ void advance(const Params& p, Pos& s) {
 //   kWalkNarrow: shorter rows.
 enum Walk { kWalkRows32 = 0, kWalkWide = 1, kWalkNarrow = 2 };
 
+// The decoded symbols of one step, held between the rANS chain and the writes so that a step's
+// reconstruction can overlap the next step's chain.
+struct StepSyms {
+    uint32_t e[8];
+    int32_t f[8];  // only for the escape path and the fields output
+    uint32_t c;
+    bool from_symbols;
+};
+
 // ESC: the blob's tables give the escape symbol a frequency, so a field may be a raw word.
-template <int OUT, bool VEC, bool ESC, bool FULL, class Reader>
-__device__ __forceinline__ void decode_step(const Params& p, uint32_t tab, Reader& rd, uint32_t& x, bool active,
-                                            const Pos& pos) {
+template <bool ESC, bool FULL, class Reader>
+__device__ __forceinline__ void step_symbols(uint32_t tab, Reader& rd, uint32_t& x, bool active, StepSyms& s) {
     if (FULL) active = true;
     // (coset, f1) as one symbol of the joint table, then f2..f8 from the 7 tables of that coset.
     // A lane past the last vector still loads (from its masked slot, inside the table) but keeps x.
-    uint32_t e[8], acc = 0;
-    e[0] = lds_u32<0>(((x << 2) & (kSlotMask << 2)) | tab);
+    uint32_t* e = s.e;
+    uint32_t acc = 0;
+    e[0] = lds_u32<0>(slot_addr(x, tab));
     if (active) x = (e[0] >> kEntryQShift) * (x >> kProbBits) + (e[0] & kEntryBiasMask);
     renorm_step<FULL>(x, rd, active);
     if (ESC) acc = e[0];
     const uint32_t c = (e[0] >> kEntryCosetShift) & 1u;
+    s.c = c;
     const uint32_t tb = tab + kCtxBytes + c * (7u * kCtxBytes);  // 4 KB aligned
 #define EP_FIELD(j)                                                                    \
     {                                                                                  \
-        const uint32_t ent = lds_u32<((j) - 1) * kCtxBytes>(((x << 2) & (kSlotMask << 2)) | tb); \
+        const uint32_t ent = lds_u32<((j) - 1) * kCtxBytes>(slot_addr(x, tb)); \
         if (active) x = (ent >> kEntryQShift) * (x >> kProbBits) + (ent & kEntryBiasMask); \
         renorm_step<FULL>(x, rd, active);                                              \
         e[j] = ent;                                                                    \
@@ -493,59 +513,83 @@ __device__ __forceinline__ void decode_step(const Params& p, uint32_t tab, Reade
     EP_FIELD(1) EP_FIELD(2) EP_FIELD(3) EP_FIELD(4) EP_FIELD(5) EP_FIELD(6) EP_FIELD(7)
 #undef EP_FIELD
 
-    bool from_symbols = true;
-    int32_t f[8];  // only for the escape path and the fields output
+    s.from_symbols = true;
+    if constexpr (ESC) {
+#pragma unroll
+        for (int j = 0; j < 8; ++j) s.f[j] = 0;
+    }
     if (ESC && __any_sync(kFull, active && (acc & kEntryEsc))) {
         // escaped fields: the lane's raw words after its renormalisation words, by field
 #pragma unroll
         for (int j = 0; j < 8; ++j) {
             const bool mine = active && (e[j] & kEntryEsc);
-            f[j] = mine ? int32_t(int16_t(rd.wn)) : int32_t((e[j] >> (kEntrySymShift + 1)) & 255u) - kAlphabetR;
+            s.f[j] = mine ? int32_t(int16_t(rd.wn)) : int32_t((e[j] >> (kEntrySymShift + (j == 7))) & 255u) - kAlphabetR;
             rd.consume_if(mine);
         }
-        from_symbols = false;
+        s.from_symbols = false;
     }
-    if (!active) return;
+}
 
+template <int OUT, bool VEC, bool ESC>
+__device__ __forceinline__ void step_emit(const Params& p, const StepSyms& s, const Pos& pos) {
+    const uint32_t* e = s.e;
+    const uint32_t c = s.c;
+    const bool from_symbols = !ESC || s.from_symbols;
+    int32_t f[8];
+#pragma unroll
+    for (int j = 0; j < 8; ++j) f[j] = s.f[j];
     if constexpr (OUT == kOutFields) {
         int16_t* o = reinterpret_cast<int16_t*>(pos.optr);
         o[0] = int16_t(c);
 #pragma unroll
         for (int j = 0; j < 8; ++j)
-            o[1 + j] = int16_t(from_symbols ? int32_t((e[j] >> (kEntrySymShift + 1)) & 255u) - kAlphabetR : f[j]);
+            o[1 + j] = int16_t(from_symbols ? int32_t((e[j] >> (kEntrySymShift + (j == 7))) & 255u) - kAlphabetR : f[j]);
         return;
     } else {
-        // t[j] = 2 z_j + c, the doubled lattice coordinate (z1..z7 = f1..f7, z8 = 2 f8 + parity of
-        // z1..z7), carried as the bits of the float T = 1.5 * 2^23 + 254 + t, which holds every
-        // integer up to 2^22 away exactly.  Without escapes f_j = s_j - 127, so 254 + t_j = 2 s_j + c
-        // comes straight out of the table entry, and 254 + t_8 = 4 s_8 + 2 par + c - 254 with
-        // par = (s_1 + ... + s_7 + 1) mod 2 (7 * 127 is odd): bit 1 of 2 s_j is the low bit of s_j.
+        // y_j = z_j + c/2, the lattice coordinate (z1..z7 = f1..f7, z8 = 2 f8 + parity of z1..z7),
+        // comes from a float T_j built from integer bits: T_j = 1.5 * 2^23 + (an integer below
+        // 2^22), so one fused multiply-add y = T k - b is exact (T k is a power-of-two scaling and
+        // the difference is a small multiple of 1/2); a * y then rounds once.
         constexpr uint32_t kMagic = 0x4B400000u;     // bits of 1.5 * 2^23
-        constexpr float kHalfBias = 6291583.0f;      // (1.5 * 2^23 + 254) / 2
-        uint32_t t[8];
-        if (from_symbols) {
-            const uint32_t km = kMagic | c;
+        float val[8];
+        const float2 a2 = make_float2(pos.a, pos.a);
+        // y = T k - b for the pairs (T_1, T_2), (T_3, T_4), (T_5, T_6), (T_7, T_8), then a * y
+        auto scale = [&](const uint32_t (&t)[8], float2 k012, float2 b012, float2 k3, float2 b3) {
 #pragma unroll
-            for (int j = 0; j < 7; ++j) t[j] = ((e[j] >> kEntrySymShift) & 0x1FEu) | km;
-            const uint32_t par2 = ~(t[0] ^ t[1] ^ t[2] ^ t[3] ^ t[4] ^ t[5] ^ t[6]) & 2u;
-            t[7] = (((e[7] >> (kEntrySymShift - 1)) & 0x3FCu) | par2) + (km - 254u);
+            for (int i = 0; i < 4; ++i) {
+                const float2 y = __ffma2_rn(make_float2(__uint_as_float(t[2 * i]), __uint_as_float(t[2 * i + 1])),
+                                            i < 3 ? k012 : k3, i < 3 ? b012 : b3);
+                const float2 r = __fmul2_rn(y, a2);
+                val[2 * i] = r.x;
+                val[2 * i + 1] = r.y;
+            }
+        };
+        if (from_symbols) {
+            // Without escapes f_j = s_j - 127.  s_j sits in bits 10..17 of a field-1..7 entry and
+            // s_8 in bits 11..18 of a field-8 entry, so one mask and OR give
+            //   T_j = 1.5 * 2^23 + 1024 s_j + 512 c:               T_j / 1024 - 12415 = s_j - 127 + c/2,
+            //   T_8 = 1.5 * 2^23 + 2048 s_8 + 1024 par + 512 c:    T_8 / 1024 - 12542 = z_8 + c/2,
+            // with par = (s_1 + ... + s_7 + 1) mod 2 (7 * 127 is odd), the complement of bit 10
+            // of t_1 ^ ... ^ t_7.
+            uint32_t t[8];
+            const uint32_t km = kMagic | (c << 9);
+#pragma unroll
+            for (int j = 0; j < 7; ++j) t[j] = (e[j] & (0xFFu << kEntrySymShift)) | km;
+            const uint32_t px = t[0] ^ t[1] ^ t[2] ^ t[3] ^ t[4] ^ t[5] ^ t[6];
+            t[7] = ((e[7] & (0xFFu << (kEntrySymShift + 1))) | km) | (~px & 0x400u);
+            const float2 k = make_float2(1.0f / 1024, 1.0f / 1024), b = make_float2(-12415.0f, -12415.0f);
+            scale(t, k, b, k, make_float2(-12415.0f, -12542.0f));
         } else {
+            // a raw field may be as large as 2^15: T_j = 1.5 * 2^23 + 254 + c + 2 z_j, and
+            // T_j / 2 - (1.5 * 2^23 + 254) / 2 = z_j + c/2
+            constexpr float kHalfBias = 6291583.0f;      // (1.5 * 2^23 + 254) / 2
+            uint32_t t[8];
             const int32_t par = (f[0] + f[1] + f[2] + f[3] + f[4] + f[5] + f[6]) & 1;
             f[7] = 2 * f[7] + par;
 #pragma unroll
             for (int j = 0; j < 8; ++j) t[j] = uint32_t(int32_t(kMagic + 254u + c) + 2 * f[j]);
-        }
-        // y = T / 2 - kHalfBias = z + c/2 in one fused multiply-add: T / 2 is exact and so is
-        // the difference (a multiple of 1/2 below 2^17), so y is exact; a * y then rounds once.
-        float val[8];
-        const float2 half = make_float2(0.5f, 0.5f), nb = make_float2(-kHalfBias, -kHalfBias);
-        const float2 a2 = make_float2(pos.a, pos.a);
-#pragma unroll
-        for (int i = 0; i < 4; ++i) {
-            const float2 y = __ffma2_rn(make_float2(__uint_as_float(t[2 * i]), __uint_as_float(t[2 * i + 1])), half, nb);
-            const float2 r = __fmul2_rn(y, a2);
-            val[2 * i] = r.x;
-            val[2 * i + 1] = r.y;
+            const float2 k = make_float2(0.5f, 0.5f), b = make_float2(-kHalfBias, -kHalfBias);
+            scale(t, k, b, k, b);
         }
         if constexpr (VEC) {
             store_vec<OUT>(pos.optr, val);
@@ -558,25 +602,66 @@ __device__ __forceinline__ void decode_step(const Params& p, uint32_t tab, Reade
     }
 }
 
+
+template <int OUT, bool VEC, bool ESC, bool FULL, class Reader>
+__device__ __forceinline__ void decode_step(const Params& p, uint32_t tab, Reader& rd, uint32_t& x, bool active,
+                                            const Pos& pos) {
+    if (FULL) active = true;
+    StepSyms s;
+    step_symbols<ESC, FULL>(tab, rd, x, active, s);
+    if (!active) return;
+    step_emit<OUT, VEC, ESC>(p, s, pos);
+}
+
 // Decode `n` full steps, two between runaway checks (the tile buffer's slack covers what two
 // steps may read past a checked position), moving the output position by `walk` after each.
+// Escape-free blobs are software-pipelined: the symbols of step k + 1 are decoded before step k
+// is written (blobs with escapes keep one step at a time, whose raw-field path would otherwise
+// hold two steps' fields in registers).
 template <int OUT, bool VEC, bool ESC, class Reader, class Guard, class Step>
 __device__ __forceinline__ uint32_t full_run(const Params& p, uint32_t tab, Reader& rd, uint32_t& x, Pos& pos,
                                              uint32_t n, Guard in_range, Step walk) {
-    uint32_t k = 0;
+    if constexpr (ESC) {
+        uint32_t k = 0;
+        for (; k + 2 <= n; k += 2) {
+            if (!__all_sync(kFull, in_range(rd))) return kStOverrun;  // a corrupt tile ran away
+            decode_step<OUT, VEC, ESC, true>(p, tab, rd, x, true, pos);
+            walk(pos);
+            decode_step<OUT, VEC, ESC, true>(p, tab, rd, x, true, pos);
+            walk(pos);
+        }
+        if (k < n) {
+            if (!__all_sync(kFull, in_range(rd))) return kStOverrun;
+            decode_step<OUT, VEC, ESC, true>(p, tab, rd, x, true, pos);
+            walk(pos);
+        }
+        return 0;
+    } else {
+    if (n == 0) return 0;
+    StepSyms a, b;
+    if (!__all_sync(kFull, in_range(rd))) return kStOverrun;
+    step_symbols<ESC, true>(tab, rd, x, true, a);
+    uint32_t k = 1;
     for (; k + 2 <= n; k += 2) {
         if (!__all_sync(kFull, in_range(rd))) return kStOverrun;  // a corrupt tile ran away
-        decode_step<OUT, VEC, ESC, true>(p, tab, rd, x, true, pos);
+        step_symbols<ESC, true>(tab, rd, x, true, b);
+        step_emit<OUT, VEC, ESC>(p, a, pos);
         walk(pos);
-        decode_step<OUT, VEC, ESC, true>(p, tab, rd, x, true, pos);
+        step_symbols<ESC, true>(tab, rd, x, true, a);
+        step_emit<OUT, VEC, ESC>(p, b, pos);
         walk(pos);
     }
     if (k < n) {
         if (!__all_sync(kFull, in_range(rd))) return kStOverrun;
-        decode_step<OUT, VEC, ESC, true>(p, tab, rd, x, true, pos);
+        step_symbols<ESC, true>(tab, rd, x, true, b);
+        step_emit<OUT, VEC, ESC>(p, a, pos);
         walk(pos);
+        a = b;
     }
+    step_emit<OUT, VEC, ESC>(p, a, pos);
+    walk(pos);
     return 0;
+    }
 }
 
 template <int OUT, bool VEC, bool ESC, int WALK, class Reader, class Guard>
