@@ -514,7 +514,7 @@ __device__ __forceinline__ void step_symbols(uint32_t tab, Reader& rd, uint32_t&
 #undef EP_FIELD
 
     s.from_symbols = true;
-    if constexpr (ESC) {
+    if constexpr (ESC) {  // defined on both paths (an undefined join costs the kernel its registers)
 #pragma unroll
         for (int j = 0; j < 8; ++j) s.f[j] = 0;
     }
@@ -674,6 +674,22 @@ __device__ __forceinline__ uint32_t full_steps(const Params& p, uint32_t tab, Re
         const uint32_t per_row = p.vec_per_row / kLanes;
         const int64_t wrap = (p.row_stride - 8 * int64_t(p.vec_per_row)) * es;
         uint32_t left = (p.vec_per_row - pos.kcol + kLanes - 1) / kLanes;  // the same for all 32 lanes
+        if (per_row < 8) {
+            // short rows: one run over the whole tile (the step pipeline does not restart at every
+            // row), the row change a warp-uniform branch in the walk
+            float a_next = pos.row + 1 < p.rows ? __ldg(p.alpha + pos.row + 1) : 0.0f;
+            return full_run<OUT, VEC, ESC>(p, tab, rd, x, pos, nfull, in_range, [&](Pos& s) {
+                s.optr += 32 * 8 * es;
+                if (--left == 0) {
+                    left = per_row;
+                    s.optr += wrap;
+                    ++s.row;
+                    s.a = a_next;
+                    a_next = s.row + 1 < p.rows ? __ldg(p.alpha + s.row + 1) : 0.0f;
+                }
+            });
+        }
+        // rows of 8 steps or more: one run per row, nothing but the output pointer moving inside it
         for (uint32_t k = 0; k < nfull;) {
             const uint32_t n = min(left, nfull - k);
             const float a_next = pos.row + 1 < p.rows ? __ldg(p.alpha + pos.row + 1) : 0.0f;
@@ -697,14 +713,15 @@ __device__ __forceinline__ uint32_t full_steps(const Params& p, uint32_t tab, Re
 }
 
 // Decode the steps of one tile with a given word reader; returns the status flags of the tile.
+// `pos` is the lane's first vector of the tile (first_pos), found by the caller before the tile's
+// words arrived.
 template <int OUT, bool VEC, bool ESC, class Reader, class Guard>
 __device__ __forceinline__ uint32_t decode_tile_steps(const Params& p, uint32_t tab, Reader& rd, uint32_t& x,
-                                                      uint32_t tile, uint32_t lane, Guard in_range) {
+                                                      uint32_t tile, uint32_t lane, Pos pos, Guard in_range) {
     const int64_t per_tile = int64_t(kLanes) * p.steps;
     const int64_t v0 = int64_t(tile) * per_tile;
     const uint32_t nv = uint32_t(min(per_tile, p.n_vectors - v0));
     const uint32_t nfull = nv / kLanes, rem = nv % kLanes;
-    Pos pos = first_pos<OUT>(p, v0 + lane);
     uint32_t st;
     if (VEC && OUT != kOutFields && p.vec_per_row % kLanes == 0)
         st = full_steps<OUT, VEC, ESC, (VEC && OUT != kOutFields) ? kWalkRows32 : kWalkWide>(p, tab, rd, x, pos, nfull,
@@ -804,6 +821,8 @@ __device__ __forceinline__ void decode_ctas(const Params& p, const TableSrc* ts,
                 if (tbytes <= kBuf) stage(tile, t0, tbytes);
             }
             first = false;
+            // the lane's output position and row scale: their global loads overlap the staging
+            const Pos pos = first_pos<OUT>(p, int64_t(tile) * kLanes * p.steps + lane);
             const bool in_smem = tbytes <= kBuf;
             const uint8_t* tg = p.stream + t0;
             if (in_smem) {
@@ -843,7 +862,7 @@ __device__ __forceinline__ void decode_ctas(const Params& p, const TableSrc* ts,
                 rd.wp = buf_a + uint32_t(min(max(o0, 0), int32_t(tbytes) - 2));
                 rd.wn = lds_u16(rd.wp);
                 const uint32_t wp0 = rd.wp, lo = buf_a, hi = buf_a + kBuf;
-                flags = decode_tile_steps<OUT, VEC, ESC>(p, tab, rd, x, tile, lane,
+                flags = decode_tile_steps<OUT, VEC, ESC>(p, tab, rd, x, tile, lane, pos,
                                                          [=](const SmemReader& r) { return r.wp - lo <= hi - lo; });
                 nread = rd.consumed(wp0);
             } else {
@@ -853,7 +872,7 @@ __device__ __forceinline__ void decode_ctas(const Params& p, const TableSrc* ts,
                 rd.hi = int32_t(tbytes) - 2;
                 rd.off = o0;
                 rd.wn = __ldg(reinterpret_cast<const uint16_t*>(tg + min(max(o0, 0), rd.hi)));
-                flags = decode_tile_steps<OUT, VEC, ESC>(p, tab, rd, x, tile, lane,
+                flags = decode_tile_steps<OUT, VEC, ESC>(p, tab, rd, x, tile, lane, pos,
                                                          [](const GlobalReader&) { return true; });
                 nread = rd.consumed(o0);
             }
