@@ -56,7 +56,6 @@ namespace {
 
 constexpr uint32_t kFull = 0xFFFFFFFFu;
 constexpr uint32_t kWaitSpins = 1u << 22;                     // bounded mbarrier wait (~0.3 s)
-constexpr uint32_t kSlotMask = kProbTotal - 1;
 constexpr uint32_t kCtxBytes = 4 * kProbTotal;                // one context's packed table: 4 KB
 // Decode tables: [0] the joint (coset, f1) symbol; [1 + 7c + (j - 2)] field j = 2..8 given coset c.
 constexpr int kDecodeTables = 15;
