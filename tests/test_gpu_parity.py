@@ -159,10 +159,21 @@ def test_steps_per_tile_and_partial_tiles(ep, S):
     _check_full(ep, blob, m, [W.BF16, W.F32])
 
 
+@pytest.mark.parametrize("cols,S", [(256, 5), (512, 3), (768, 3), (768, 16), (1280, 5), (1536, 100), (1792, 7)])
+def test_short_rows_tiles_starting_mid_row(ep, cols, S):
+    """Rows of 1 to 7 steps (a multiple of 32 vectors per row, so a warp's lanes change rows
+    together) with tile lengths that are not multiples of the row length: tiles start and end
+    inside rows, the row change falls anywhere in a tile's run of steps, the last tile is
+    partial."""
+    m = W.square(rows=41, cols=cols)
+    blob = oracle.compress(m.bits, m.dtype, 4.0, steps_per_tile=S)
+    _check_full(ep, blob, m, [W.BF16, W.FP16, W.E4M3])
+
+
 @pytest.mark.parametrize("S,rate", [(1, 11.0), (2, 4.0), (1, 0.5)])
 def test_many_tiles_per_warp(ep, S, rate):
-    """More tiles than resident warps (148 SMs x 32 warps), so warps decode several tiles in a
-    row and a tile's first chunk lands in any of the four ring slots."""
+    """More tiles than resident warps (148 SMs x 32 warps), so warps decode several tiles one
+    after another, each staged into the buffer the previous one used."""
     m = W.sweep(rate, rows=2400, cols=1024)
     blob = oracle.compress(m.bits, m.dtype, rate, steps_per_tile=S)
     assert oracle.blob_info(blob)["n_tiles"] > 148 * 32
