@@ -9,8 +9,8 @@
 //   * one warp per tile; the tile's 32 interleaved rANS states live one per lane;
 //   * one persistent CTA of 32 warps per SM (grid = min(#SM, #tiles)); tile t goes to CTA
 //     t mod grid, so every SM gets an equal share even when there are few tiles;
-//   * decode tables: one packed 32-bit entry per slot of the 1024-slot range, {slot - cum(s), 2 s,
-//     escape flag, coset bit, q(s)}, for the joint (coset, f1) symbol and for f2..f8 given each
+//   * decode tables: one packed 32-bit entry per slot of the 1024-slot range, {slot - cum(s), s
+//     (2 s for f8), escape flag, coset bit, q(s)}, for the joint (coset, f1) symbol and for f2..f8 given each
 //     coset -- 15 tables, 60 KB -- so one shared-memory load per symbol gives everything the
 //     state update needs.  They are expanded once per blob and device by a small kernel into a
 //     block next to the device copy; every CTA stages that block into shared memory with bulk
