@@ -6,10 +6,12 @@ BF16, rows N(0, sigma_r^2) with sigma_r log-uniform in [0.005, 0.05], compressed
 element by the library's own encoder (synthetic data; no model weights are involved).
 
 Timing: W untimed warm-up steps, then exactly K steps between a barrier + synchronize on both
-sides, timed by CUDA events on the launching stream; the maximum over ranks is reported.  The
-steps rotate over R independent blob/output copies whose total exceeds 3x the 126 MB L2, so
-each step reads its blob and writes its output through HBM.  nvidia-smi samples clocks and
-throttle reasons during the timed region.
+sides, timed by CUDA events on the launching stream; the maximum over ranks is reported.  The K
+launches are queued behind a short device-side delay recorded before the start event, so the
+timed region holds K back-to-back decodes and no host launch cost.  The steps rotate over R
+independent blob/output copies whose total exceeds 3x the 126 MB L2, so each step reads its blob
+and writes its output through HBM.  nvidia-smi samples clocks and throttle reasons from the
+warm-up through the timed region.
 
 Multi-GPU (torchrun): every rank decodes its own copy of the workload; no data-path collective
 (tiles are independent), so scaling is weak and the value is the sum over ranks.
@@ -27,7 +29,6 @@ import hashlib
 import json
 import math
 import os
-import re
 import statistics
 import subprocess
 import sys
@@ -59,6 +60,9 @@ def parse_args():
                     help="also time the oracle tile-parallel on this many host cores (0 = all, 1 = skip)")
     ap.add_argument("--workload", default="square",
                     help="square (default) | small | dit-set | sweep:<bpp> | large")
+    ap.add_argument("--out-dtype", default="",
+                    help="output container(s), comma-separated, decoded back to back every step: "
+                         "bf16, fp16, e4m3, f32, int8 (default: the input's)")
     ap.add_argument("--decode", choices=["grouped", "single"], default="grouped",
                     help="for a set of matrices: one ep_decompress_group call per step, or one "
                          "ep_decompress call per matrix")
@@ -147,25 +151,31 @@ def hbm_peak():
         return FALLBACK_HBM_GBS, "fallback"
 
 
+KERNEL_SOURCES = ("decode_device.cuh", "decode_launch.h", "format.h")
+TRAFFIC_FILE = os.path.join(ROOT, "profiles", "decode_traffic.json")
+
+
 def kernel_source_hash() -> str:
+    """Hash of the decode kernel's sources: a DRAM traffic figure is valid only for this code."""
     h = hashlib.sha256()
-    for f in ("decode.cu", "format.h", "blob.h"):
+    for f in KERNEL_SOURCES:
         h.update(open(os.path.join(ROOT, "dit_weight_compression_b200", "csrc", f), "rb").read())
     return h.hexdigest()[:16]
 
 
-def committed_traffic(profile: str):
-    """DRAM bytes per launch from a committed ncu summary, if it was taken on this kernel source."""
-    path = os.path.join(ROOT, "profiles", profile)
+def measured_traffic(key: str):
+    """DRAM bytes (read + write) per decode launch from the ncu capture of consecutive launches
+    summarised in profiles/decode_traffic.json, if it was taken on this kernel source; else None."""
     try:
-        text = open(path).read()
-    except OSError:
+        d = json.load(open(TRAFFIC_FILE))
+    except (OSError, ValueError):
         return None
-    src = re.search(r"kernel_source_sha:\s*([0-9a-f]+)", text)
-    val = re.search(r"dram_bytes_per_launch:\s*([0-9]+)", text)
-    if not src or not val or src.group(1) != kernel_source_hash():
+    if d.get("kernel_source_sha") != kernel_source_hash():
         return None
-    return int(val.group(1))
+    w = d.get("workloads", {}).get(key)
+    if not w:
+        return None
+    return int(w["dram_bytes_read_per_launch"]) + int(w["dram_bytes_write_per_launch"])
 
 
 # ---------------------------------------------------------------------------------------------
@@ -296,6 +306,31 @@ def reference_arm(args, m, desc):
 # ---------------------------------------------------------------------------------------------
 # The CUDA arm.
 # ---------------------------------------------------------------------------------------------
+OUT_DTYPES = {"bf16": "bfloat16", "fp16": "float16", "e4m3": "float8_e4m3fn", "f32": "float32",
+              "int8": "int8"}
+
+
+def out_containers(arg: str, default):
+    """The torch dtypes each step decodes into, in order (the input's own by default)."""
+    import torch
+    if not arg:
+        return [default]
+    out = []
+    for name in arg.split(","):
+        name = name.strip().lower()
+        if name not in OUT_DTYPES:
+            raise SystemExit(f"unknown output container {name!r} (one of {', '.join(OUT_DTYPES)})")
+        out.append(getattr(torch, OUT_DTYPES[name]))
+    return out
+
+
+def queue_delay_cycles(launches: int) -> int:
+    """Length of the device-side delay queued before the timed region: long enough for the host
+    to enqueue the first launches behind it (about 10 us each through ctypes), so host launch
+    cost and idle gaps stay out of the timed region."""
+    return int(max(1e-3, min(launches, 2048) * 10e-6) * 2.0e9)
+
+
 def main():
     args = parse_args()
     mats, desc = workload(args.workload)
@@ -338,40 +373,42 @@ def main():
         raise SystemExit("GPU encoder blob differs from the host encoder's")
     del gcomps, dev_in
     n = len(comps)
-    out_dt = comps[0].dtype
-    es = torch.empty((), dtype=out_dt).element_size()
-    out_bytes = sum(c.shape[0] * c.shape[1] * es for c in comps)
+    out_dts = out_containers(args.out_dtype, comps[0].dtype)
+    nd = len(out_dts)
+    out_bytes = sum(c.shape[0] * c.shape[1] * torch.empty((), dtype=dt).element_size()
+                    for c in comps for dt in out_dts)
     blob_bytes = sum(len(b) for b in blobs)
-    moved = blob_bytes + out_bytes
+    moved = nd * blob_bytes + out_bytes          # every decode reads its blob once
     grouped = n > 1 and args.decode == "grouped"
 
     # R independent device copies of the whole set so that consecutive steps miss L2
     R = max(2, math.ceil(3 * L2_BYTES / moved))
     stream = torch.cuda.current_stream()
     copies = [[ep.CompressedTensor.from_bytes(b) for b in blobs] for _ in range(R)]
-    outs = [[torch.empty(c.shape, dtype=out_dt, device="cuda") for c in comps] for _ in range(R)]
+    outs = [[[torch.empty(c.shape, dtype=dt, device="cuda") for c in comps] for dt in out_dts] for _ in range(R)]
     for cs in copies:
         for c in cs:
             c.prepare(stream=stream)
     L = ep.lib()
-    views = [[ep.tensor_view(o) for o in os_] for os_ in outs]
+    views = [[[ep.tensor_view(o) for o in od] for od in os_] for os_ in outs]
     handles = [[c.handle for c in cs] for cs in copies]
     g_handles = [(ctypes.c_void_p * n)(*[h.value for h in hs]) for hs in handles]
-    g_views = [(ep.EpTensor * n)(*vs) for vs in views]
+    g_views = [[(ep.EpTensor * n)(*vs) for vs in vd] for vd in views]
     sh = ctypes.c_void_p(stream.cuda_stream)
-    launches_per_step = math.ceil(n / 32) if grouped else n
+    launches_per_step = nd * (math.ceil(n / 32) if grouped else n)
 
     def step(i):
         j = i % R
-        if grouped:
-            rc = L.ep_decompress_group(g_handles[j], g_views[j], n, sh)
-            if rc != 0:
-                raise ep.EPError(rc, "ep_decompress_group")
-            return
-        for h, v in zip(handles[j], views[j]):
-            rc = L.ep_decompress(h, ctypes.byref(v), sh)
-            if rc != 0:
-                raise ep.EPError(rc, "ep_decompress")
+        for d in range(nd):
+            if grouped:
+                rc = L.ep_decompress_group(g_handles[j], g_views[j][d], n, sh)
+                if rc != 0:
+                    raise ep.EPError(rc, "ep_decompress_group")
+                continue
+            for h, v in zip(handles[j], views[j][d]):
+                rc = L.ep_decompress(h, ctypes.byref(v), sh)
+                if rc != 0:
+                    raise ep.EPError(rc, "ep_decompress")
 
     # a first step, checked by the kernels' own integrity checks
     step(0)
@@ -379,10 +416,6 @@ def main():
     for c in copies[0]:
         ep.decode_status(c)
 
-    for i in range(args.warmup):
-        step(i)
-    K = args.steps
-    start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     gpu_uuid = None
     try:
         gpu_uuid = str(torch.cuda.get_device_properties(local).uuid)
@@ -391,22 +424,26 @@ def main():
     except Exception:
         gpu_uuid = None
     clocks = ClockSampler(gpu_uuid)
+    clocks.start()  # samples warm-up and timed region alike: the GPU is never idle in between
+    for i in range(args.warmup):
+        step(i)
+    K = args.steps
+    start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     torch.cuda.synchronize()
     barrier()
     torch.cuda.synchronize()
-    clocks.start()
-    time.sleep(0.2)  # let the sampler start before the timed region
-    # Decode kernels launched back to back on one stream (each may overlap the previous one's
-    # drain, see the kernel); the average step is the timed region over K, which also counts
-    # any gap between launches.
+    # The K launches queue up behind a device-side delay recorded before the start event, so the
+    # timed region holds exactly K back-to-back decodes (each may overlap the previous one's drain,
+    # see the kernel) and neither host launch cost nor a gap after the barrier.
+    torch.cuda._sleep(queue_delay_cycles(K * launches_per_step))
     start.record(stream)
     for i in range(K):
-        step(i)
+        step(args.warmup + i)
     end.record(stream)
     torch.cuda.synchronize()
+    clk = clocks.stop()
     barrier()
     torch.cuda.synchronize()
-    clk = clocks.stop()
     total_ms = start.elapsed_time(end)
     avg_step_ms = total_ms / K
     for cs in copies:
@@ -416,11 +453,12 @@ def main():
     total_ms, avg_step_ms = max_over_ranks([total_ms, avg_step_ms], world)
 
     # end to end through the public call with host buffers: upload each blob, decode, download
-    host_outs = [torch.empty(c.shape, dtype=out_dt).pin_memory() for c in comps]
+    host_outs = [[torch.empty(c.shape, dtype=dt).pin_memory() for c in comps] for dt in out_dts]
 
     def e2e_step():
-        for c, ho in zip(comps, host_outs):
-            ep.decompress(c, out=ho)
+        for ho in host_outs:
+            for c, o in zip(comps, ho):
+                ep.decompress(c, out=o)
 
     for _ in range(3):
         e2e_step()
@@ -441,7 +479,7 @@ def main():
         peak, peak_kind = hbm_peak()
         achieved = moved / (avg_step_ms * 1e-3) / 1e9   # algorithmic bytes over the step's device time
         value = job_throughput(world, out_bytes, K, total_ms)
-        symbols = sum(c.info.n_vectors for c in comps) * 9
+        symbols = nd * sum(c.info.n_vectors for c in comps) * 8   # a vector is 8 rANS symbols
         cpu = None
         if world == 1 and not args.no_cpu_baseline:
             gbs, reps, nt, secs = cpu_oracle_rate(blobs[0], args.cpu_seconds)
@@ -449,30 +487,37 @@ def main():
             what = "matrix" if n == 1 else f"first matrix of the {n}"
             cpu = {"value": gbs, "unit": "GB/s", "cores": 1, "kind": "oracle",
                    "sample": f"whole {r0}x{c0} {what} ({nt} tiles) decoded {reps} times, {secs:.1f} s, "
-                             f"single-threaded oracle"}
+                             f"single-threaded oracle, BF16 output"}
             if args.cpu_cores != 1:
                 want = host_cores() if args.cpu_cores <= 0 else args.cpu_cores
                 pg, used, psecs = cpu_oracle_rate_parallel(blobs[0], args.cpu_seconds, want)
                 cpu["all_cores"] = {"value": pg, "unit": "GB/s", "cores": used, "kind": "oracle",
                                     "sample": f"the same {what}, tile-parallel over {used} processes, "
                                               f"{psecs:.1f} s"}
-        traffic = committed_traffic("decode_square_bf16.md") if args.workload == "square" else None
+        traffic = None
+        if launches_per_step == 1:
+            traffic = measured_traffic(f"{args.workload}:{str(out_dts[0]).replace('torch.', '')}")
         info = comps[0].info
+        dt_names = [str(dt).replace("torch.", "") for dt in out_dts]
         config = {
-            "workload": desc, "matrices": n,
+            "workload": desc if not args.out_dtype else f"{desc.rsplit(', output', 1)[0]}, output "
+                                                        f"{' then '.join(dt_names)}",
+            "matrices": n,
             "shapes": [list(c.shape) for c in comps],
             "target_bpp": mats[0].target_bpp,
             "actual_bpp": 8.0 * blob_bytes / sum(c.shape[0] * c.shape[1] for c in comps),
             "steps_per_tile": sorted({c.info.steps_per_tile for c in comps}),
             "n_tiles": sum(c.info.n_tiles for c in comps), "blob_bytes": blob_bytes, "out_bytes": out_bytes,
+            "out_containers": dt_names,
             "l2": f"rotating {R} blob/output copies ({R * moved / 1e6:.0f} MB > 3x L2)",
-            "symbols_per_s": world * symbols * K / (total_ms * 1e-3),
+            "rans_symbols_per_s": world * symbols * K / (total_ms * 1e-3),
             "step_avg_us": avg_step_ms * 1e3, "encode_s": enc_s, "encode_gpu_s": enc_gpu_s,
-            "decode": ("ep_decompress_group, one launch per step" if grouped else
-                       f"ep_decompress, {n} launch(es) per step"),
+            "decode": ("ep_decompress_group, one launch per container per step" if grouped else
+                       f"ep_decompress, {launches_per_step} launch(es) per step"),
+            "timing": "K launches queued behind a device-side delay; CUDA events around exactly K steps",
             "parallelism": f"weak, {world} independent rank(s)",
         }
-        if n == 1:
+        if n == 1 and nd == 1:
             config.update(rows=info.rows, cols=info.cols, kernel_avg_us=avg_step_ms * 1e3)
         line = {
             "metric": METRIC, "value": value, "unit": "GB/s", "n_gpus": world, "steps": K,
@@ -485,7 +530,7 @@ def main():
                          "algorithmic_bytes_per_launch" if launches_per_step == 1 else "algorithmic_bytes_per_step": moved},
             "cpu_baseline": cpu,
             "e2e": {"value": job_throughput(world, out_bytes, args.e2e_steps, e2e_ms), "unit": "GB/s",
-                    "h2d_bytes_per_step": blob_bytes, "d2h_bytes_per_step": out_bytes},
+                    "h2d_bytes_per_step": nd * blob_bytes, "d2h_bytes_per_step": out_bytes},
             "gpu_launches": K * launches_per_step,
             "clocks": clk,
         }

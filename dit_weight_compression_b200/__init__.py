@@ -63,7 +63,8 @@ SIGNATURES = {
     "ep_blob_prepare": (_I, [_P, _I, _P]),
     "ep_decode_status": (_I, [_P, _P]),
     "ep_decode_fields": (_I, [_P, _P, _P]),
-    "ep_decompress_noalloc": (_I, [_P, _P, ctypes.POINTER(EpTensor), _P, _I]),
+    "ep_decompress_noalloc": (_I, [_P, _P, _SZ, ctypes.POINTER(EpTensor), _P, _I]),
+    "ep_decode_wait_probe": (_I, [_P, ctypes.c_uint32, _P]),
     "ep_blob_free": (None, [_P]),
     "ep_last_error": (ctypes.c_char_p, []),
 }

@@ -176,9 +176,9 @@ private:
 
 // ---------------------------------------------------------------------------------------------
 // Tiled, 32-way interleaved rANS.  Lane l of a tile owns vectors l, 32 + l, 64 + l, ... and one
-// 32-bit state.  A lane reads its own words: for each step, after each of its 9 decodes (coset,
-// f1..f8) one word if the state fell below 2^16, then the raw words of its escaped fields in
-// field order.  Lanes 2p and 2p+1 share region p: lane 2p reads forward from the region start,
+// 32-bit state.  A lane reads its own words: for each step, after each of its 8 decodes ((coset,
+// f1) as one symbol, then f2..f8) one word if the state fell below 2^16, then the raw words of its
+// escaped fields in field order.  Lanes 2p and 2p+1 share region p: lane 2p reads forward from the region start,
 // lane 2p+1 backward from the region end.  Tile: 32 u32 states, 16 u16 region word counts, the
 // regions, zero padding to 16 bytes.  Each lane is encoded in reverse reading order.
 // ---------------------------------------------------------------------------------------------

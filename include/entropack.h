@@ -183,14 +183,21 @@ int ep_decode_fields(const ep_blob* b, int16_t* fields, void* stream);
  * callers that cannot let a library allocate GPU memory -- an inference runtime that plans all
  * device memory ahead of time in its own arena, or code running where allocation is forbidden or
  * would synchronise the device.)
- *   b            blob handle; only its parsed header is used (its host bytes are not read).
- *   device_blob  the blob's serialised bytes (ep_blob_to_bytes) already in device memory on the
- *                current device, owned by the caller, 16-byte aligned.
- *   out          device output on the current device, as for ep_decompress.
- *   stream       cudaStream_t as void*.
- *   wait         0: return after the launch (asynchronous, the kernel's corruption checks are
- *                not reported); nonzero: synchronise `stream` and return EP_ERR_CORRUPT if the
- *                decode found a corrupt tile.
+ *   b                  blob handle; only its parsed header is used (its host bytes are not read).
+ *   device_blob        the blob's serialised bytes (exactly those of ep_blob_to_bytes(b)) already
+ *                      in device memory on the current device, owned by the caller, 16-byte
+ *                      aligned.
+ *   device_blob_bytes  size of the caller's device buffer; EP_ERR_ARG if it is smaller than the
+ *                      blob.  The kernel reads nothing beyond the blob's size, and it checks
+ *                      every tile's extent against the stream section before reading it, so a
+ *                      stale or different copy is reported as corrupt rather than read outside
+ *                      the buffer.
+ *   out                device output on the current device, as for ep_decompress.
+ *   stream             cudaStream_t as void*.
+ *   wait               0: return after the launch (asynchronous; the kernel's corruption checks
+ *                      are not reported, and ep_decode_status does not see them -- it reads the
+ *                      blob's own status word, not this path's); nonzero: synchronise `stream`
+ *                      and return EP_ERR_CORRUPT if the decode found a corrupt tile.
  * The decode kernel's scratch -- one 4-byte status word -- lives in a fixed 256-byte array of
  * device memory inside this library (64 words; every GPU that loads the library keeps it until
  * the process exits).  Each call clears the word it uses; a call whose scratch need exceeded the
@@ -202,8 +209,16 @@ int ep_decode_fields(const ep_blob* b, int16_t* fields, void* stream);
  * capture.  Returns EP_ERR_ARG, EP_ERR_SHAPE, EP_ERR_DTYPE, EP_ERR_CUDA, EP_ERR_CORRUPT; messages
  * from this call never allocate.
  */
-int ep_decompress_noalloc(const ep_blob* b, const void* device_blob, const ep_tensor* out, void* stream,
-                          int wait);
+int ep_decompress_noalloc(const ep_blob* b, const void* device_blob, size_t device_blob_bytes, const ep_tensor* out,
+                          void* stream, int wait);
+
+/* Test hook for the bounded waits (the method's pages have no counterpart).  Launches the decode
+ * kernel on the blob's device copy with every CTA waiting, for at most `wait_spins` polls, on a
+ * shared-memory barrier that expects 16 bytes no copy delivers; the wait gives up, the CTA
+ * records "bulk-copy wait limit reached" in the blob's status word, waits for its real copies and
+ * leaves.  Nothing is decoded or written.  ep_decode_status then returns EP_ERR_CORRUPT, and the
+ * context stays usable.  Returns EP_ERR_ARG (NULL blob, zero limit), EP_ERR_CUDA, EP_ERR_OOM. */
+int ep_decode_wait_probe(const ep_blob* b, uint32_t wait_spins, void* stream);
 
 /* Release a blob, its host bytes and any device copies (synchronises those devices). */
 void ep_blob_free(ep_blob* b);

@@ -985,7 +985,7 @@ out:
  *
  * Blob layout (little-endian, every section 16-byte aligned; [DOC-ER]: besides the coded fields
  * the blob keeps the frequency tables, the per-row scales and per-tile bookkeeping):
- *   header (80 bytes): "EPK1", u16 version 2, u8 dtype, u8 R, u64 rows, u64 cols, u32 S,
+ *   header (80 bytes): "EPK1", u16 version 3, u8 dtype, u8 R, u64 rows, u64 cols, u32 S,
  *     u32 n_tiles, f64 s, u64 total bytes, u64 offsets of the table, row-scale, tile-offset
  *     and stream sections;
  *   tables: for c = 0,1 and j = 1..8: u16 q(escape), u8 lo, u8 n, u16 q[lo .. lo+n-1]

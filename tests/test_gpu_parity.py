@@ -10,6 +10,8 @@ Both cross directions: the GPU decodes oracle-encoded blobs, and (host suite) th
 library-encoded blobs.  Full-size workloads compare every element where the oracle finishes in
 seconds and sampled tiles (first, last, and seeded random ones) elsewhere.
 """
+import ctypes
+
 import numpy as np
 import pytest
 import torch
@@ -209,8 +211,9 @@ def test_degenerate_tables(ep):
 
 
 def test_tiny_row_scales(ep):
-    """Rows around 2^-135 (FP32 subnormals) give row scales below 2^-125, where halving the
-    scale would round: the kernel must take its exact two-multiply path."""
+    """Rows around 2^-135 (FP32 subnormals) give row scales below 2^-125, where any rewriting of
+    alpha * y that scales alpha first (halving it, say) would round: the kernel's exact lattice
+    coordinate times alpha, rounded once, must still equal the oracle's."""
     g = np.random.Generator(np.random.PCG64(11))
     x = g.normal(0, 1, (64, 256)) * 2.0 ** -135
     x[::2] *= 2.0 ** 100                                           # half the rows ordinary
@@ -308,6 +311,24 @@ def test_corrupt_stream_reported_not_hung(ep):
     ep.decompress(good)
     ep.decode_status(good)
     del out
+
+
+def test_bounded_wait_gives_up_and_reports(ep):
+    """A bulk-copy wait that can never complete (the barrier expects bytes no copy delivers) gives
+    up after its short limit: the kernel ends, the status word reports the wait limit, and the
+    context stays usable -- nothing faults or hangs."""
+    m = W.small()
+    c = ep.compress(W.bits_to_torch(m.bits, m.dtype), m.target_bpp)
+    ref = _gpu_decode(ep, c)                  # also makes the blob's device copy
+    L = ep.lib()
+    rc = L.ep_decode_wait_probe(c.handle, 2000, ctypes.c_void_p(torch.cuda.current_stream().cuda_stream))
+    assert rc == 0, L.ep_last_error()
+    torch.cuda.synchronize()
+    with pytest.raises(ep.EPError) as e:
+        ep.decode_status(c)
+    assert e.value.code == -5 and "wait limit" in str(e.value)
+    again = _gpu_decode(ep, c)                # status cleared, decode still correct
+    assert np.array_equal(_bits(again, W.BF16), _bits(ref, W.BF16))
 
 
 def test_rel_l2_matches_oracle_usage_example(ep):

@@ -7,11 +7,14 @@ in device memory (their allocation, not the library's) and keeps the decode kern
 in a fixed array inside the library instead of allocating one.
 
 This file checks that entry point against the ordinary ep_decompress on the same blob, bit for
-bit (the tolerance the parity tests use), on two calls in a row, and that the two calls leave
-the device's free memory unchanged.  It is named so that pytest collects it after every other
-test file.
+bit (the tolerance the parity tests use), on two calls in a row, for every kernel variant it can
+launch: vector and element stores, blobs with and without escape symbols, and each output
+container.  It also checks that the two calls leave the device's free memory unchanged, that a
+corrupt tile is reported and the next clean call is not, and that a device buffer shorter than
+the blob is refused.  It is named so that pytest collects it after every other test file.
 """
 import ctypes
+import struct
 
 import numpy as np
 import pytest
@@ -20,6 +23,9 @@ import torch
 import workloads as W
 
 pytestmark = pytest.mark.gpu
+
+TORCH = {W.BF16: torch.bfloat16, W.FP16: torch.float16, W.E4M3: torch.float8_e4m3fn, W.F32: torch.float32,
+         W.INT8: torch.int8}
 
 
 @pytest.fixture(scope="module")
@@ -32,39 +38,93 @@ def ep():
     return ep
 
 
-def _bits(t):
-    return t.contiguous().view(torch.int16).cpu().numpy()
+def _bytes(t):
+    return t.contiguous().view(torch.uint8).cpu().numpy()
 
 
-def test_noalloc_matches_decompress_twice(ep):
-    m = W.square(rows=1024, cols=2048)
-    comp = ep.compress(W.bits_to_torch(m.bits, m.dtype), m.target_bpp)
+def _noalloc(ep, comp, dev_blob, out, wait=1, nbytes=None):
+    L = ep.lib()
+    view = ep.tensor_view(out)
+    n = dev_blob.numel() if nbytes is None else nbytes
+    s = ctypes.c_void_p(torch.cuda.current_stream().cuda_stream)
+    return L.ep_decompress_noalloc(comp.handle, ctypes.c_void_p(dev_blob.data_ptr()), n, ctypes.byref(view), s,
+                                   wait)
 
-    # reference: the ordinary entry point (it allocates its own device copy of the blob)
-    ref = ep.decompress(comp)
+
+def _two_calls_match(ep, comp, out_dtype, make_out):
+    """Two allocation-free decodes in a row equal ep_decompress, with free memory unchanged."""
+    ref = make_out()
+    ep.decompress(comp, out=ref)
     torch.cuda.synchronize()
     ep.decode_status(comp)
-
-    # the caller owns the device copy of the bytes
-    blob = comp.to_bytes()
-    dev_blob = torch.frombuffer(bytearray(blob), dtype=torch.uint8).cuda()
+    dev_blob = torch.frombuffer(bytearray(comp.to_bytes()), dtype=torch.uint8).cuda()
     assert dev_blob.data_ptr() % 16 == 0
-    stream = torch.cuda.current_stream()
-    L = ep.lib()
-
-    outs = [torch.full(comp.shape, float("nan"), dtype=torch.bfloat16, device="cuda") for _ in range(2)]
-    views = [ep.tensor_view(o) for o in outs]
+    outs = [make_out() for _ in range(2)]
+    for o in outs:
+        o.view(torch.uint8).fill_(0x7F)
     torch.cuda.synchronize()
     free_before, _ = torch.cuda.mem_get_info()
-    for i in range(2):
-        rc = L.ep_decompress_noalloc(comp.handle, ctypes.c_void_p(dev_blob.data_ptr()),
-                                     ctypes.byref(views[i]), ctypes.c_void_p(stream.cuda_stream), 1)
-        assert rc == 0, L.ep_last_error()
+    for o in outs:
+        rc = _noalloc(ep, comp, dev_blob, o)
+        assert rc == 0, ep.lib().ep_last_error()
     torch.cuda.synchronize()
     free_after, _ = torch.cuda.mem_get_info()
     for o in outs:
-        assert np.array_equal(_bits(o), _bits(ref))
+        assert np.array_equal(_bytes(o), _bytes(ref)), out_dtype
     assert free_after == free_before
+
+
+def test_noalloc_matches_decompress_twice(ep):
+    """BF16, vector stores, an escape-free blob."""
+    m = W.square(rows=1024, cols=2048)
+    comp = ep.compress(W.bits_to_torch(m.bits, m.dtype), m.target_bpp)
+    _two_calls_match(ep, comp, W.BF16, lambda: torch.empty(comp.shape, dtype=torch.bfloat16, device="cuda"))
+
+
+@pytest.mark.parametrize("dtype", [W.FP16, W.E4M3, W.F32, W.INT8])
+def test_noalloc_escapes_every_container(ep, dtype):
+    """An 11-bpp blob (most fields are escapes, so the escape kernel runs) in every container."""
+    m = W.sweep(11.0, rows=96, cols=704)
+    comp = ep.compress(W.bits_to_torch(m.bits, m.dtype), m.target_bpp)
+    _two_calls_match(ep, comp, dtype, lambda: torch.empty(comp.shape, dtype=TORCH[dtype], device="cuda"))
+
+
+@pytest.mark.parametrize("dtype", [W.BF16, W.E4M3])
+def test_noalloc_element_stores(ep, dtype):
+    """Outputs the vector stores cannot take: ragged columns, and a misaligned output pointer."""
+    m = W.small(rows=37, cols=203)
+    comp = ep.compress(W.bits_to_torch(m.bits, m.dtype), m.target_bpp)
+    _two_calls_match(ep, comp, dtype, lambda: torch.empty(comp.shape, dtype=TORCH[dtype], device="cuda"))
+    m2 = W.small(rows=40, cols=256)
+    comp2 = ep.compress(W.bits_to_torch(m2.bits, m2.dtype), m2.target_bpp)
+
+    def shifted():
+        base = torch.empty(40 * 256 + 1, dtype=TORCH[dtype], device="cuda")
+        return base[1:].view(40, 256)   # one element off the vector alignment
+
+    _two_calls_match(ep, comp2, dtype, shifted)
+
+
+def test_noalloc_corrupt_tile_then_clean_call(ep):
+    """Flipped payload bytes inside one tile (offsets and headers intact) give EP_ERR_CORRUPT; the
+    next call on intact bytes returns 0, because each call clears the shared status word."""
+    m = W.square(rows=256, cols=1024)
+    comp = ep.compress(W.bits_to_torch(m.bits, m.dtype), m.target_bpp)
+    blob = comp.to_bytes()
+    off_offsets, off_stream = struct.unpack_from("<QQ", blob, 64)   # header: tile-offset, stream offsets
+    off = off_stream + 16 * struct.unpack_from("<I", blob, off_offsets + 4)[0]   # start of tile 1
+    bad = bytearray(blob)
+    for k in range(off + 200, off + 260):      # inside tile 1's regions, past its 160-byte header
+        bad[k] ^= 0x5A
+    out = torch.empty(comp.shape, dtype=torch.bfloat16, device="cuda")
+    dev_bad = torch.frombuffer(bad, dtype=torch.uint8).cuda()
+    dev_good = torch.frombuffer(bytearray(blob), dtype=torch.uint8).cuda()
+    assert _noalloc(ep, comp, dev_bad, out) == -5
+    assert b"corrupt" in ep.lib().ep_last_error()
+    assert _noalloc(ep, comp, dev_good, out) == 0
+    ref = ep.decompress(comp)
+    torch.cuda.synchronize()
+    assert np.array_equal(_bytes(out), _bytes(ref))
 
 
 def test_noalloc_rejects_bad_arguments(ep):
@@ -75,15 +135,19 @@ def test_noalloc_rejects_bad_arguments(ep):
     view = ep.tensor_view(out)
     L = ep.lib()
     s = ctypes.c_void_p(torch.cuda.current_stream().cuda_stream)
+    n = dev_blob.numel()
     # misaligned device bytes
-    rc = L.ep_decompress_noalloc(comp.handle, ctypes.c_void_p(dev_blob.data_ptr() + 8), ctypes.byref(view), s, 1)
+    rc = L.ep_decompress_noalloc(comp.handle, ctypes.c_void_p(dev_blob.data_ptr() + 8), n, ctypes.byref(view), s, 1)
     assert rc == -1 and b"aligned" in L.ep_last_error()
+    # a device buffer shorter than the blob
+    assert _noalloc(ep, comp, dev_blob, out, nbytes=n - 16) == -1
+    assert b"smaller" in L.ep_last_error()
     # host output is not accepted
     host = torch.empty(comp.shape, dtype=torch.bfloat16)
     hv = ep.tensor_view(host)
-    rc = L.ep_decompress_noalloc(comp.handle, ctypes.c_void_p(dev_blob.data_ptr()), ctypes.byref(hv), s, 1)
+    rc = L.ep_decompress_noalloc(comp.handle, ctypes.c_void_p(dev_blob.data_ptr()), n, ctypes.byref(hv), s, 1)
     assert rc == -1
     # wrong shape
     bad = ep.EpTensor(out.data_ptr(), out.device.index, 1, 255, 256, 256)
-    rc = L.ep_decompress_noalloc(comp.handle, ctypes.c_void_p(dev_blob.data_ptr()), ctypes.byref(bad), s, 1)
+    rc = L.ep_decompress_noalloc(comp.handle, ctypes.c_void_p(dev_blob.data_ptr()), n, ctypes.byref(bad), s, 1)
     assert rc == -3
