@@ -48,12 +48,13 @@ enum { ORC_BF16 = 1, ORC_FP16 = 2, ORC_E4M3 = 3, ORC_F32 = 4, ORC_INT8 = 5 };
 
 #define ORC_R 127          /* reading: field alphabet [-R, R] coded directly, R = 127     */
 #define ORC_ESC 255        /* symbol that announces a raw 16-bit field value               */
-#define ORC_M 1024u        /* reading: frequency totals are 10-bit, every table sums to M  */
+#define ORC_PB_DEFAULT 12  /* frequency totals: 12-bit (M = 4096), the fixed format choice */
+#define ORC_M_MAX 4096u    /* largest total M = 2^prob_bits; prob_bits is 12 or 10         */
 #define ORC_L 65536u       /* rANS lower bound 2^16, 32-bit state, 16-bit renormalisation */
-#define ORC_VERSION 3      /* blob format version (3: coset coded jointly with f1)        */
+#define ORC_VERSION 4      /* blob format version (4: totals in the header, row maxima)   */
 #define ORC_LANES 32       /* interleaved rANS states per tile                            */
 #define ORC_NCTX 16        /* field j given coset c: 8c + (j-1); 0 and 8 = joint (c, f1)  */
-#define ORC_HEADER 80      /* bytes in the fixed header                                   */
+#define ORC_HEADER 96      /* bytes in the fixed header                                   */
 #define ORC_CLAMP 32764.0  /* reading: |t| clamp, keeps every field inside int16          */
 
 /* ------------------------------------------------------------------------------------------ */
@@ -353,16 +354,16 @@ void orc_fields_to_point(int coset, const int32_t f[8], double y[8])
 static int field_symbol(int32_t f) { return (f >= -ORC_R && f <= ORC_R) ? f + ORC_R : ORC_ESC; }
 
 /* ------------------------------------------------------------------------------------------ */
-/* Probability tables with 10-bit totals (M = 1024).                                          */
+/* Probability tables with totals M = 2^prob_bits: 4096 (12-bit, the fixed choice) or 1024.    */
 /* ------------------------------------------------------------------------------------------ */
 
 /*
- * Quantise symbol counts n[0..255] to frequencies q[] summing to M.
+ * Quantise symbol counts n[0..nb-1] to frequencies q[] summing to M.
  * reading: q_s = max(1, round_half_up(M n_s / N)) for n_s > 0, else 0; then, while the sum
  * exceeds M, decrement the largest q (> 1; lowest symbol on ties); while it is below M,
  * increment the symbol with the largest count (lowest symbol on ties).  N = 0 gives all zeros.
  */
-static void quantize_n(const uint64_t* n, int nb, uint16_t* q)
+static void quantize_n(const uint64_t* n, int nb, uint16_t* q, uint32_t M)
 {
     uint64_t N = 0;
     for (int s = 0; s < nb; s++) N += n[s];
@@ -371,19 +372,19 @@ static void quantize_n(const uint64_t* n, int nb, uint16_t* q)
     long sum = 0;
     for (int s = 0; s < nb; s++) {
         if (n[s] == 0) continue;
-        uint64_t v = (2u * ORC_M * n[s] + N) / (2u * N);      /* round half up */
+        uint64_t v = (2u * (uint64_t)M * n[s] + N) / (2u * N);  /* round half up */
         if (v < 1) v = 1;
         q[s] = (uint16_t)v;
         sum += (long)v;
     }
-    while (sum > (long)ORC_M) {
+    while (sum > (long)M) {
         int best = -1;
         for (int s = 0; s < nb; s++)
             if (q[s] > 1 && (best < 0 || q[s] > q[best])) best = s;
         q[best]--;
         sum--;
     }
-    while (sum < (long)ORC_M) {
+    while (sum < (long)M) {
         int best = -1;
         for (int s = 0; s < nb; s++)
             if (n[s] > 0 && (best < 0 || n[s] > n[best])) best = s;
@@ -392,7 +393,10 @@ static void quantize_n(const uint64_t* n, int nb, uint16_t* q)
     }
 }
 
-void orc_quantize_table(const uint64_t n[256], uint16_t q[256]) { quantize_n(n, 256, q); }
+void orc_quantize_table(const uint64_t n[256], uint16_t q[256], int prob_bits)
+{
+    quantize_n(n, 256, q, 1u << prob_bits);
+}
 
 /*
  * The 16 context tables from symbol counts cnt[16 x 256].  reading: the coset and the first field
@@ -402,21 +406,21 @@ void orc_quantize_table(const uint64_t n[256], uint16_t q[256]) { quantize_n(n, 
  * quantised together to sum to M (coset-major order, so ties go to coset 0 first); every other
  * context (c, j >= 2) is quantised on its own.
  */
-static void build_tables16(const uint64_t* cnt, uint16_t* q16)
+static void build_tables16(const uint64_t* cnt, uint16_t* q16, int prob_bits)
 {
     uint64_t nj[512];
     uint16_t qj[512];
     memcpy(nj, cnt, 256 * sizeof(uint64_t));
     memcpy(nj + 256, cnt + 256 * 8, 256 * sizeof(uint64_t));
-    quantize_n(nj, 512, qj);
+    quantize_n(nj, 512, qj, 1u << prob_bits);
     memcpy(q16, qj, 256 * sizeof(uint16_t));
     memcpy(q16 + 256 * 8, qj + 256, 256 * sizeof(uint16_t));
     for (int ctx = 1; ctx < ORC_NCTX; ctx++)
-        if (ctx != 8) orc_quantize_table(cnt + 256 * ctx, q16 + 256 * ctx);
+        if (ctx != 8) orc_quantize_table(cnt + 256 * ctx, q16 + 256 * ctx, prob_bits);
 }
 
 /* Exposed for the table checks. */
-void orc_build_tables16(const uint64_t* cnt, uint16_t* q16) { build_tables16(cnt, q16); }
+void orc_build_tables16(const uint64_t* cnt, uint16_t* q16, int prob_bits) { build_tables16(cnt, q16, prob_bits); }
 
 /* Cumulative frequencies: cum[s] = q[0] + ... + q[s-1]. */
 static void cumulate(const uint16_t q[256], uint32_t cum[257])
@@ -479,19 +483,20 @@ static int push_word(wordbuf* b, uint32_t v)
 /*
  * Encode one tile.  sym9[v*9] is the coset of vector v and sym9[v*9 + j] the symbol of its field j,
  * raw8[v*8 + j-1] the raw value of field j (used when its symbol is the escape).  q16 holds the 16
- * context tables (16 x 256 frequencies; contexts 0 and 8 the joint (coset, f1) table).  Returns
- * the tile size in bytes (written to out when out != NULL and cap is large enough), or 0 on
- * failure.
+ * context tables (16 x 256 frequencies summing to M = 2^prob_bits; contexts 0 and 8 the joint
+ * (coset, f1) table).  Returns the tile size in bytes (written to out when out != NULL and cap is
+ * large enough), or 0 on failure.
  *
  * rANS encode of symbol s with frequency q and cumulative cum [ANS]: while x >= q * (L / M) * 2^16
- * (= q * 2^22), emit the low 16 bits of x and shift them out; then
+ * (= q * 2^(32 - prob_bits)), emit the low 16 bits of x and shift them out; then
  * x <- floor(x / q) * M + (x mod q) + cum.
  * Each lane is encoded on its own, in reverse of its reading order, and its words are reversed
  * at the end.
  */
 uint64_t orc_encode_tile(const uint8_t* sym9, const int16_t* raw8, int64_t nvec,
-                         const uint16_t* q16, uint8_t* out, uint64_t cap)
+                         const uint16_t* q16, int prob_bits, uint8_t* out, uint64_t cap)
 {
+    const uint32_t M = 1u << prob_bits;
     uint32_t cum[ORC_NCTX][257];
     for (int c = 0; c < ORC_NCTX; c++) cumulate(q16 + 256 * c, cum[c]);
     uint32_t x[ORC_LANES];
@@ -511,11 +516,11 @@ uint64_t orc_encode_tile(const uint8_t* sym9, const int16_t* raw8, int64_t nvec,
                 uint32_t q, cm;
                 freq_cum(q16, cum, j, sym9[v * 9], sym9[v * 9 + j], &q, &cm);
                 if (q == 0) goto fail;
-                if ((uint64_t)x[l] >= (uint64_t)q * (ORC_L / ORC_M) * 65536u) {
+                if ((uint64_t)x[l] >= (uint64_t)q * (ORC_L / M) * 65536u) {
                     if (push_word(&wb[l], x[l] & 0xFFFFu)) goto fail;
                     x[l] >>= 16;
                 }
-                x[l] = (x[l] / q) * ORC_M + (x[l] % q) + cm;
+                x[l] = (x[l] / q) * M + (x[l] % q) + cm;
             }
         }
     }
@@ -548,22 +553,26 @@ fail:
     return 0;
 }
 
-/* Decoding tables of the 16 contexts: cumulative frequencies and the symbol of every slot (for
- * the two halves of the joint table, slots relative to each half's start). */
+/* Decoding tables of the 16 contexts: the total M, cumulative frequencies and the symbol of every
+ * slot (for the two halves of the joint table, slots relative to each half's start). */
 typedef struct {
     const uint16_t* q16;
+    uint32_t M;
+    int prob_bits;
     uint32_t cum[ORC_NCTX][257];
-    uint8_t slot_sym[ORC_NCTX][ORC_M];
+    uint8_t slot_sym[ORC_NCTX][ORC_M_MAX];
 } dtables;
 
-static void build_dtables(const uint16_t* q16, dtables* T)
+static void build_dtables(const uint16_t* q16, int prob_bits, dtables* T)
 {
     T->q16 = q16;
+    T->prob_bits = prob_bits;
+    T->M = 1u << prob_bits;
     for (int c = 0; c < ORC_NCTX; c++) {
         cumulate(q16 + 256 * c, T->cum[c]);
-        memset(T->slot_sym[c], 0, ORC_M);
+        memset(T->slot_sym[c], 0, ORC_M_MAX);
         for (int s = 0; s < 256; s++)
-            for (uint32_t i = T->cum[c][s]; i < T->cum[c][s + 1] && i < ORC_M; i++) T->slot_sym[c][i] = (uint8_t)s;
+            for (uint32_t i = T->cum[c][s]; i < T->cum[c][s + 1] && i < T->M; i++) T->slot_sym[c][i] = (uint8_t)s;
     }
 }
 
@@ -599,7 +608,7 @@ static int decode_tile(const uint8_t* tile, uint64_t nbytes, int64_t nvec, const
             int64_t v = k * ORC_LANES + l;
             if (v >= nvec) continue;
             for (int j = 1; j <= 8; j++) {
-                uint32_t slot = x & (ORC_M - 1);
+                uint32_t slot = x & (T->M - 1);
                 int c, s;
                 if (j == 1) {                    /* (coset, f1): coset 1's slots follow coset 0's */
                     uint32_t tot0 = T->cum[0][256];
@@ -612,7 +621,7 @@ static int decode_tile(const uint8_t* tile, uint64_t nbytes, int64_t nvec, const
                 }
                 uint32_t q, cm;
                 freq_cum(T->q16, T->cum, j, c, s, &q, &cm);
-                x = q * (x / ORC_M) + slot - cm;
+                x = q * (x / T->M) + slot - cm;
                 sym9[v * 9 + j] = (uint8_t)s;
                 if (x < ORC_L) {
                     int64_t w = fwd ? start[p] + n : start[p] + count[p] - 1 - n;
@@ -640,12 +649,12 @@ static int decode_tile(const uint8_t* tile, uint64_t nbytes, int64_t nvec, const
 }
 
 /* Decode one tile given the 16 x 256 frequency tables (exposed for the rANS checks). */
-int orc_decode_tile(const uint8_t* tile, uint64_t nbytes, int64_t nvec, const uint16_t* q16,
+int orc_decode_tile(const uint8_t* tile, uint64_t nbytes, int64_t nvec, const uint16_t* q16, int prob_bits,
                     uint8_t* sym9, int16_t* raw8, uint32_t* final_states)
 {
     dtables* T = (dtables*)malloc(sizeof(dtables));
     if (!T) return -2;
-    build_dtables(q16, T);
+    build_dtables(q16, prob_bits, T);
     int rc = decode_tile(tile, nbytes, nvec, T, sym9, raw8, final_states);
     free(T);
     return rc;
@@ -733,17 +742,26 @@ static uint64_t table_section_bytes(const uint16_t* q16)
     return bytes;
 }
 
+/* Metadata bytes of a blob with these tables: the exact header, table, row-scale, row-maximum and
+ * tile-offset sections, plus per tile its 160 header bytes (states, region counts) and 8 bytes,
+ * the mean padding. */
+static double metadata_bytes(const uint16_t* q16, int64_t rows, int64_t ntiles)
+{
+    return (double)(ORC_HEADER + pad16(table_section_bytes(q16)) + pad16(4u * (uint64_t)rows) +
+                    pad16(2u * (uint64_t)rows) + pad16(4u * (uint64_t)(ntiles + 1))) +
+           (double)ntiles * (160.0 + 8.0);
+}
+
 /*
  * Estimated blob size in bits per element at scale s from the sampled rows ([DOC-RS]: a
  * candidate scale is judged by the predicted size of its coded fields plus the metadata the
  * decoder needs).
  * reading: n_s = min(rows, 256) rows at floor(i * rows / n_s); tables are quantised from the
  * sample's counts; coded size = sum over contexts and symbols of n * -log2(q / M) bits plus
- * 16 bits per escape, scaled by rows / n_s; metadata = exact header, table, row-scale and
- * tile-offset bytes, plus 160 header bytes (states, region counts) and 8 padding bytes per tile.
+ * 16 bits per escape, scaled by rows / n_s; metadata as metadata_bytes counts it.
  * With full_sample != 0 every row is used (n_s = rows).
  */
-static double estimate_bpp(const matrix* m, double s, int64_t S, int full_sample)
+static double estimate_bpp(const matrix* m, double s, int64_t S, int full_sample, int prob_bits)
 {
     int64_t ns = full_sample ? m->rows : (m->rows < 256 ? m->rows : 256);
     uint64_t* cnt = (uint64_t*)calloc(ORC_NCTX * 256, sizeof(uint64_t));
@@ -764,17 +782,16 @@ static double estimate_bpp(const matrix* m, double s, int64_t S, int full_sample
         }
     }
     uint16_t q16[ORC_NCTX * 256];
-    build_tables16(cnt, q16);
+    build_tables16(cnt, q16, prob_bits);
+    const double M = (double)(1u << prob_bits);
     double bits = 0.0;
     for (int ctx = 0; ctx < ORC_NCTX; ctx++)
         for (int sy = 0; sy < 256; sy++)
-            if (cnt[256 * ctx + sy]) bits += (double)cnt[256 * ctx + sy] * -log2((double)q16[256 * ctx + sy] / (double)ORC_M);
+            if (cnt[256 * ctx + sy]) bits += (double)cnt[256 * ctx + sy] * -log2((double)q16[256 * ctx + sy] / M);
     double payload = ((double)m->rows / (double)ns) * (bits / 8.0 + 2.0 * (double)nesc);
     int64_t V = m->rows * m->vpr;
     int64_t ntiles = (V + 32 * S - 1) / (32 * S);
-    double meta = (double)(ORC_HEADER + pad16(table_section_bytes(q16)) + pad16(4u * (uint64_t)m->rows) +
-                           pad16(4u * (uint64_t)(ntiles + 1))) +
-                  (double)ntiles * (160.0 + 8.0);
+    double meta = metadata_bytes(q16, m->rows, ntiles);
     free(cnt);
     return 8.0 * (meta + payload) / ((double)m->rows * (double)m->cols);
 }
@@ -786,14 +803,14 @@ static double estimate_bpp(const matrix* m, double s, int64_t S, int full_sample
  * over [-24, 8]; if even 2^8 misses the target, 2^8 (the actual size is reported as it is,
  * [DOC-ER]: the stored rate need not equal the requested one).
  */
-static double choose_scale(const matrix* m, double target, int64_t S)
+static double choose_scale(const matrix* m, double target, int64_t S, int prob_bits)
 {
     double lo = -24.0, hi = 8.0;
-    if (estimate_bpp(m, exp2(hi), S, 0) > target) return exp2(hi);
-    if (estimate_bpp(m, exp2(lo), S, 0) <= target) return exp2(lo);
+    if (estimate_bpp(m, exp2(hi), S, 0, prob_bits) > target) return exp2(hi);
+    if (estimate_bpp(m, exp2(lo), S, 0, prob_bits) <= target) return exp2(lo);
     for (int it = 0; it < 48; it++) {
         double mid = 0.5 * (lo + hi);
-        if (estimate_bpp(m, exp2(mid), S, 0) <= target) hi = mid;
+        if (estimate_bpp(m, exp2(mid), S, 0, prob_bits) <= target) hi = mid;
         else lo = mid;
     }
     return exp2(hi);
@@ -826,12 +843,14 @@ static void free_matrix(matrix* m)
 
 /* Estimated bits per element at a given scale (exposed for the size-estimate check). */
 double orc_estimate_bpp(const void* data, int dtype, int64_t rows, int64_t cols, double scale,
-                        int64_t S, int full_sample)
+                        int64_t S, int full_sample, int prob_bits)
 {
+    if (prob_bits == 0) prob_bits = ORC_PB_DEFAULT;
+    if (prob_bits != 10 && prob_bits != 12) return -1.0;
     matrix m;
     memset(&m, 0, sizeof m);
     if (load_matrix(&m, data, dtype, rows, cols)) { free_matrix(&m); return -1.0; }
-    double b = estimate_bpp(&m, scale, S, full_sample);
+    double b = estimate_bpp(&m, scale, S, full_sample, prob_bits);
     free_matrix(&m);
     return b;
 }
@@ -920,8 +939,9 @@ static double rd_choose(const matrix* m, const double* D, const double* R, doubl
 }
 
 /* The refinement: fills kr[rows] with each row's candidate index.  Returns 0 or -2 (memory). */
-static int rd_allocate(const matrix* m, double s, double target, int64_t S, int* kr)
+static int rd_allocate(const matrix* m, double s, double target, int64_t S, int prob_bits, int* kr)
 {
+    const double M = (double)(1u << prob_bits);
     const size_t per = (size_t)m->vpr * 9;
     uint8_t* sym = (uint8_t*)malloc((size_t)m->rows * RD_NK * per);
     uint64_t* nesc = (uint64_t*)malloc((size_t)m->rows * RD_NK * sizeof(uint64_t));
@@ -942,9 +962,9 @@ static int rd_allocate(const matrix* m, double s, double target, int64_t S, int*
             uint16_t q16[ORC_NCTX * 256];
             double cost[ORC_NCTX * 256];
             rd_counts(m, sym, kr, cnt);
-            build_tables16(cnt, q16);
+            build_tables16(cnt, q16, prob_bits);
             for (int i = 0; i < ORC_NCTX * 256; i++)
-                cost[i] = q16[i] ? -log2((double)q16[i] / (double)ORC_M) : log2((double)ORC_M);
+                cost[i] = q16[i] ? -log2((double)q16[i] / M) : log2(M);
             for (int64_t r = 0; r < m->rows; r++)
                 for (int ki = 0; ki < RD_NK; ki++) {
                     const uint8_t* sr = sym + ((size_t)r * RD_NK + ki) * per;
@@ -953,9 +973,7 @@ static int rd_allocate(const matrix* m, double s, double target, int64_t S, int*
                         for (int u = 1; u <= 8; u++) bits += cost[256 * context_of(u, sr[9 * k]) + sr[9 * k + u]];
                     R[r * RD_NK + ki] = bits;
                 }
-            double meta = (double)(ORC_HEADER + pad16(table_section_bytes(q16)) + pad16(4u * (uint64_t)m->rows) +
-                                   pad16(4u * (uint64_t)(ntiles + 1))) +
-                          (double)ntiles * (160.0 + 8.0);
+            double meta = metadata_bytes(q16, m->rows, ntiles);
             double budget = target * (double)m->rows * (double)m->cols - 8.0 * meta;
             if (rd_choose(m, D, R, 0.0, kr) > budget) {
                 double lo = -100.0, hi = 40.0;
@@ -981,47 +999,54 @@ out:
 
 /*
  * Compress a rows x cols matrix stored as dtype bits.  steps_per_tile = 0 selects the default S;
- * scale_override > 0 skips the search.  On success *blob is a malloc'd byte string of *len bytes.
+ * scale_override > 0 skips the search; prob_bits is 12 or 10 (0 selects 12).  On success *blob is
+ * a malloc'd byte string of *len bytes.
  *
  * Blob layout (little-endian, every section 16-byte aligned; [DOC-ER]: besides the coded fields
  * the blob keeps the frequency tables, the per-row scales and per-tile bookkeeping):
- *   header (80 bytes): "EPK1", u16 version 3, u8 dtype, u8 R, u64 rows, u64 cols, u32 S,
+ *   header (96 bytes): "EPK1", u16 version 4, u8 dtype, u8 R, u64 rows, u64 cols, u32 S,
  *     u32 n_tiles, f64 s, u64 total bytes, u64 offsets of the table, row-scale, tile-offset
- *     and stream sections;
+ *     and stream sections, u64 offset of the row-maximum section, u8 prob_bits, 7 zero bytes;
  *   tables: for c = 0,1 and j = 1..8: u16 q(escape), u8 lo, u8 n, u16 q[lo .. lo+n-1]
  *     (symbols 0..254); the two j = 1 tables are the coset halves of the joint (c, f1) table;
  *   row scales: f32 per row;
+ *   row maxima: u16 per row, the largest |2 y| over the row's real columns (2 y is an integer:
+ *     the lattice coordinates are integers or half-integers, |y| <= 32764.5);
  *   tile offsets: u32[n_tiles + 1], in 16-byte units from the stream section start;
  *   stream: the tiles.
  */
 int orc_compress_ex(const void* data, int dtype, int64_t rows, int64_t cols, double target_bpp,
-                    int64_t steps_per_tile, double scale_override, int rd_refine, uint8_t** blob,
+                    int64_t steps_per_tile, double scale_override, int rd_refine, int prob_bits, uint8_t** blob,
                     uint64_t* len)
 {
     *blob = NULL;
     *len = 0;
     /* [DOC-0]: the target must be finite and within 0.001 to 11 bits per element */
     if (!(target_bpp >= 0.001 && target_bpp <= 11.0)) return -4;
+    if (prob_bits == 0) prob_bits = ORC_PB_DEFAULT;
+    if (prob_bits != 10 && prob_bits != 12) return -4;
     matrix m;
     memset(&m, 0, sizeof m);
     int rc = load_matrix(&m, data, dtype, rows, cols);
     if (rc) { free_matrix(&m); return rc; }
     if (steps_per_tile > 1024) { free_matrix(&m); return -4; }   /* region counts are u16 */
     int64_t S = steps_per_tile > 0 ? steps_per_tile : default_steps(target_bpp);
-    double s = scale_override > 0 ? scale_override : choose_scale(&m, target_bpp, S);
+    double s = scale_override > 0 ? scale_override : choose_scale(&m, target_bpp, S, prob_bits);
     int* kr = NULL;                      /* per-row candidate of the refinement, when enabled */
     if (rd_refine) {
         kr = (int*)malloc((size_t)rows * sizeof(int));
-        if (!kr || rd_allocate(&m, s, target_bpp, S, kr)) { free(kr); free_matrix(&m); return -2; }
+        if (!kr || rd_allocate(&m, s, target_bpp, S, prob_bits, kr)) { free(kr); free_matrix(&m); return -2; }
     }
 
     /* Quantise the whole tensor at s; fit one least-squares scale per row ([DOC-RS]: with s
      * fixed, every row is quantised and gets its own reconstruction scale by least squares):
-     * alpha_r = sum w y / sum y^2 over real columns, stored as fp32 (0 when sum y^2 = 0). */
+     * alpha_r = sum w y / sum y^2 over real columns, stored as fp32 (0 when sum y^2 = 0); and
+     * keep each row's largest |2 y| over its real columns. */
     int64_t V = rows * m.vpr;
     uint8_t* sym9 = (uint8_t*)malloc((size_t)V * 9);
     int16_t* raw8 = (int16_t*)malloc((size_t)V * 8 * sizeof(int16_t));
     float* alpha = (float*)malloc((size_t)rows * sizeof(float));
+    uint32_t* rowmax = (uint32_t*)calloc((size_t)rows, sizeof(uint32_t));
     uint64_t* cnt = (uint64_t*)calloc(ORC_NCTX * 256, sizeof(uint64_t));
     for (int64_t r = 0; r < rows; r++) {
         double swy = 0.0, syy = 0.0;
@@ -1035,6 +1060,8 @@ int orc_compress_ex(const void* data, int dtype, int64_t rows, int64_t cols, dou
                 if (8 * k + i < cols) {
                     swy += elem(&m, r, 8 * k + i) * y[i];
                     syy += y[i] * y[i];
+                    uint32_t a2 = (uint32_t)fabs(2.0 * y[i]);
+                    if (a2 > rowmax[r]) rowmax[r] = a2;
                 }
             for (int u = 1; u <= 8; u++) cnt[256 * context_of(u, c) + sym9[9 * v + u]]++;
         }
@@ -1044,7 +1071,7 @@ int orc_compress_ex(const void* data, int dtype, int64_t rows, int64_t cols, dou
     /* Probability tables from the whole tensor ([DOC-LQ]: one model per coordinate field, given
      * the coset). */
     uint16_t q16[ORC_NCTX * 256];
-    build_tables16(cnt, q16);
+    build_tables16(cnt, q16, prob_bits);
 
     /* Tiles. */
     int64_t per_tile = 32 * S;
@@ -1053,7 +1080,7 @@ int orc_compress_ex(const void* data, int dtype, int64_t rows, int64_t cols, dou
     uint64_t stream_bytes = 0;
     for (int64_t t = 0; t < ntiles; t++) {
         int64_t v0 = t * per_tile, nv = V - v0 < per_tile ? V - v0 : per_tile;
-        tsize[t] = orc_encode_tile(sym9 + 9 * v0, raw8 + 8 * v0, nv, q16, NULL, 0);
+        tsize[t] = orc_encode_tile(sym9 + 9 * v0, raw8 + 8 * v0, nv, q16, prob_bits, NULL, 0);
         if (tsize[t] == 0) { rc = -5; goto done; }
         stream_bytes += tsize[t];
     }
@@ -1063,7 +1090,8 @@ int orc_compress_ex(const void* data, int dtype, int64_t rows, int64_t cols, dou
         uint64_t tab_bytes = table_section_bytes(q16);
         uint64_t off_tab = ORC_HEADER;
         uint64_t off_alpha = off_tab + pad16(tab_bytes);
-        uint64_t off_offs = off_alpha + pad16(4u * (uint64_t)rows);
+        uint64_t off_rmax = off_alpha + pad16(4u * (uint64_t)rows);
+        uint64_t off_offs = off_rmax + pad16(2u * (uint64_t)rows);
         uint64_t off_stream = off_offs + pad16(4u * (uint64_t)(ntiles + 1));
         uint64_t total = off_stream + stream_bytes;
         uint8_t* b = (uint8_t*)calloc((size_t)total, 1);
@@ -1082,6 +1110,8 @@ int orc_compress_ex(const void* data, int dtype, int64_t rows, int64_t cols, dou
         put64(b + 56, off_alpha);
         put64(b + 64, off_offs);
         put64(b + 72, off_stream);
+        put64(b + 80, off_rmax);
+        b[88] = (uint8_t)prob_bits;
         uint8_t* p = b + off_tab;
         for (int ctx = 0; ctx < ORC_NCTX; ctx++) {
             const uint16_t* q = q16 + 256 * ctx;
@@ -1099,6 +1129,7 @@ int orc_compress_ex(const void* data, int dtype, int64_t rows, int64_t cols, dou
             uint32_t ab;
             memcpy(&ab, &alpha[r], 4);
             put32(b + off_alpha + 4 * r, ab);
+            put16(b + off_rmax + 2 * r, rowmax[r]);
         }
         uint64_t acc = 0;
         for (int64_t t = 0; t <= ntiles; t++) {
@@ -1108,7 +1139,7 @@ int orc_compress_ex(const void* data, int dtype, int64_t rows, int64_t cols, dou
         acc = 0;
         for (int64_t t = 0; t < ntiles; t++) {
             int64_t v0 = t * per_tile, nv = V - v0 < per_tile ? V - v0 : per_tile;
-            orc_encode_tile(sym9 + 9 * v0, raw8 + 8 * v0, nv, q16, b + off_stream + acc, tsize[t]);
+            orc_encode_tile(sym9 + 9 * v0, raw8 + 8 * v0, nv, q16, prob_bits, b + off_stream + acc, tsize[t]);
             acc += tsize[t];
         }
         *blob = b;
@@ -1120,16 +1151,17 @@ done:
     free(sym9);
     free(raw8);
     free(alpha);
+    free(rowmax);
     free(cnt);
     free_matrix(&m);
     return rc;
 }
 
-/* orc_compress_ex with the refinement off (the default). */
+/* orc_compress_ex with the refinement off (the default) and 12-bit totals. */
 int orc_compress(const void* data, int dtype, int64_t rows, int64_t cols, double target_bpp,
                  int64_t steps_per_tile, double scale_override, uint8_t** blob, uint64_t* len)
 {
-    return orc_compress_ex(data, dtype, rows, cols, target_bpp, steps_per_tile, scale_override, 0, blob, len);
+    return orc_compress_ex(data, dtype, rows, cols, target_bpp, steps_per_tile, scale_override, 0, 0, blob, len);
 }
 
 /* ------------------------------------------------------------------------------------------ */
@@ -1138,33 +1170,38 @@ int orc_compress(const void* data, int dtype, int64_t rows, int64_t cols, double
 /* ------------------------------------------------------------------------------------------ */
 
 typedef struct {
-    int dtype;
+    int dtype, prob_bits;
     int64_t rows, cols, vpr, S, ntiles, V;
     double s;
     uint16_t q16[ORC_NCTX * 256];
     const uint8_t* alpha;
+    const uint8_t* rowmax;
     const uint8_t* offs;
     const uint8_t* stream;
-    uint64_t stream_bytes;
+    uint64_t off_offs, off_stream, stream_bytes;
 } parsed;
 
 static int parse_blob(const uint8_t* b, uint64_t len, parsed* P)
 {
     if (len < ORC_HEADER || memcmp(b, "EPK1", 4) != 0 || get16(b + 4) != ORC_VERSION || b[7] != ORC_R) return -6;
     P->dtype = b[6];
+    P->prob_bits = b[88];
+    if (P->prob_bits != 10 && P->prob_bits != 12) return -6;
+    const uint32_t M = 1u << P->prob_bits;
     P->rows = (int64_t)get64(b + 8);
     P->cols = (int64_t)get64(b + 16);
     P->S = get32(b + 24);
     P->ntiles = get32(b + 28);
     memcpy(&P->s, b + 32, 8);
     uint64_t total = get64(b + 40), off_tab = get64(b + 48), off_alpha = get64(b + 56);
-    uint64_t off_offs = get64(b + 64), off_stream = get64(b + 72);
+    uint64_t off_offs = get64(b + 64), off_stream = get64(b + 72), off_rmax = get64(b + 80);
     if (total != len || P->rows <= 0 || P->cols <= 0 || P->S <= 0 || dtype_size(P->dtype) == 0) return -6;
     P->vpr = (P->cols + 7) / 8;
     P->V = P->rows * P->vpr;
     if (P->ntiles != (P->V + 32 * P->S - 1) / (32 * P->S)) return -6;
-    if (off_tab < ORC_HEADER || off_tab > off_alpha || off_alpha + 4u * (uint64_t)P->rows > off_offs ||
-        off_offs + 4u * (uint64_t)(P->ntiles + 1) > off_stream || off_stream > len)
+    if (off_tab < ORC_HEADER || off_tab > off_alpha || off_alpha + 4u * (uint64_t)P->rows > off_rmax ||
+        off_rmax + 2u * (uint64_t)P->rows > off_offs || off_offs + 4u * (uint64_t)(P->ntiles + 1) > off_stream ||
+        off_stream > len)
         return -6;
     memset(P->q16, 0, sizeof P->q16);
     const uint8_t* p = b + off_tab;
@@ -1182,12 +1219,15 @@ static int parse_blob(const uint8_t* b, uint64_t len, parsed* P)
         sums[ctx] = 0;
         for (int sy = 0; sy < 256; sy++) sums[ctx] += P->q16[256 * ctx + sy];
     }
-    if (sums[0] + sums[8] != ORC_M) return -6;                 /* the joint (coset, f1) table */
+    if (sums[0] + sums[8] != M) return -6;                     /* the joint (coset, f1) table */
     for (int ctx = 0; ctx < ORC_NCTX; ctx++)
-        if (ctx != 0 && ctx != 8 && sums[ctx] != 0 && sums[ctx] != ORC_M) return -6;
+        if (ctx != 0 && ctx != 8 && sums[ctx] != 0 && sums[ctx] != M) return -6;
     P->alpha = b + off_alpha;
+    P->rowmax = b + off_rmax;
     P->offs = b + off_offs;
     P->stream = b + off_stream;
+    P->off_offs = off_offs;
+    P->off_stream = off_stream;
     P->stream_bytes = len - off_stream;
     if (get32(P->offs) != 0 || 16u * (uint64_t)get32(P->offs + 4 * P->ntiles) != P->stream_bytes) return -6;
     return 0;
@@ -1200,7 +1240,7 @@ static int decode_tiles_to_symbols(const parsed* P, int64_t t0, int64_t t1, uint
     int64_t per_tile = 32 * P->S, base = t0 * per_tile;
     dtables* T = (dtables*)malloc(sizeof(dtables));
     if (!T) return -2;
-    build_dtables(P->q16, T);
+    build_dtables(P->q16, P->prob_bits, T);
     int out = 0;
     for (int64_t t = t0; t < t1; t++) {
         uint64_t a = 16u * (uint64_t)get32(P->offs + 4 * t), e = 16u * (uint64_t)get32(P->offs + 4 * (t + 1));
@@ -1292,6 +1332,78 @@ int orc_decompress(const uint8_t* blob, uint64_t len, int dtype_out, void* out)
     return orc_decompress_tiles(blob, len, 0, -1, dtype_out, out);
 }
 
+/*
+ * FP8 container with a per-row scale ([ABS]: FP8 is one of the containers, and the storage rate
+ * is set apart from the numerical precision of the restored weights).
+ * reading: the E4M3 payload of row r holds the row normalised to the format's range and sigma_r
+ * carries the scale, sigma_r * payload ~ alpha_r * y:
+ *   m_r     = the row's largest |2 y| (the blob's row-maximum section),
+ *   g_r     = RNE_fp32(896 / m_r), negated when alpha_r < 0; 0 when m_r = 0 or alpha_r = 0,
+ *   payload = E4M3(RNE_fp32(y * g_r)), round to nearest even, saturating (|y * g_r| <= 448),
+ *   sigma_r = RNE_fp32(|alpha_r| * m_r / 896), i.e. rowmax |alpha_r * y| / 448.
+ * Both quotients are rounded once from their exact values (a double quotient of these sizes is
+ * never a float rounding tie unless the exact value is one, so rounding it again to float is
+ * exact rounding).
+ */
+static float f32_of(uint32_t bits)
+{
+    float f;
+    memcpy(&f, &bits, 4);
+    return f;
+}
+
+float orc_row_gain(float alpha, uint32_t m2)
+{
+    if (m2 == 0 || alpha == 0.0f) return 0.0f;
+    float g = f32_of(orc_round_f32(896.0 / (double)m2));
+    return alpha < 0.0f ? -g : g;
+}
+
+float orc_row_sigma(float alpha, uint32_t m2)
+{
+    return f32_of(orc_round_f32(fabs((double)alpha) * (double)m2 / 896.0));
+}
+
+/* Decode tiles [t0, t1) (all when t1 < 0) into the E4M3 payload (rows x cols, contiguous; other
+ * tiles' elements untouched) and write every row's sigma (rows floats). */
+int orc_decompress_rowscaled_tiles(const uint8_t* blob, uint64_t len, int64_t t0, int64_t t1, uint8_t* out,
+                                   float* sigma)
+{
+    parsed P;
+    int rc = parse_blob(blob, len, &P);
+    if (rc) return rc;
+    if (t1 < 0 || t1 > P.ntiles) t1 = P.ntiles;
+    if (t0 < 0 || t0 > t1) return -1;
+    for (int64_t r = 0; r < P.rows; r++)
+        sigma[r] = orc_row_sigma(f32_of(get32(P.alpha + 4 * r)), get16(P.rowmax + 2 * r));
+    int64_t v0 = t0 * 32 * P.S, v1 = t1 * 32 * P.S < P.V ? t1 * 32 * P.S : P.V;
+    uint8_t* sym9 = (uint8_t*)calloc((size_t)(v1 - v0) * 9 + 9, 1);
+    int16_t* raw8 = (int16_t*)calloc((size_t)(v1 - v0) * 8 + 8, sizeof(int16_t));
+    rc = decode_tiles_to_symbols(&P, t0, t1, sym9, raw8);
+    if (rc == 0) {
+        for (int64_t v = v0; v < v1; v++) {
+            int64_t r = v / P.vpr, k = v % P.vpr;
+            int32_t f[8];
+            double y[8];
+            const uint8_t* sy9 = sym9 + 9 * (v - v0);
+            for (int j = 1; j <= 8; j++) {
+                int sy = sy9[j];
+                f[j - 1] = sy == ORC_ESC ? raw8[8 * (v - v0) + j - 1] : sy - ORC_R;
+            }
+            orc_fields_to_point(sy9[0], f, y);
+            float g = orc_row_gain(f32_of(get32(P.alpha + 4 * r)), get16(P.rowmax + 2 * r));
+            for (int i = 0; i < 8; i++) {
+                int64_t col = 8 * k + i;
+                if (col >= P.cols) continue;
+                out[r * P.cols + col] = (uint8_t)orc_f32_to_e4m3(orc_round_f32((double)g * y[i]));
+            }
+        }
+    }
+    free(sym9);
+    free(raw8);
+    return rc;
+}
+
 /* [DOC-ER]: the reported rate is 8 x every stored byte (metadata included) / element count. */
 double orc_actual_bpp(const uint8_t* blob, uint64_t len)
 {
@@ -1300,17 +1412,21 @@ double orc_actual_bpp(const uint8_t* blob, uint64_t len)
     return 8.0 * (double)len / ((double)P.rows * (double)P.cols);
 }
 
-/* Header fields, for tests: rows, cols, S, n_tiles, dtype, and the shared scale. */
-int orc_blob_info(const uint8_t* blob, uint64_t len, int64_t* info5, double* scale)
+/* Header fields, for tests: rows, cols, S, n_tiles, dtype, prob_bits, the byte offsets of the
+ * tile-offset and stream sections, and the shared scale. */
+int orc_blob_info(const uint8_t* blob, uint64_t len, int64_t* info8, double* scale)
 {
     parsed P;
     int rc = parse_blob(blob, len, &P);
     if (rc) return rc;
-    info5[0] = P.rows;
-    info5[1] = P.cols;
-    info5[2] = P.S;
-    info5[3] = P.ntiles;
-    info5[4] = P.dtype;
+    info8[0] = P.rows;
+    info8[1] = P.cols;
+    info8[2] = P.S;
+    info8[3] = P.ntiles;
+    info8[4] = P.dtype;
+    info8[5] = P.prob_bits;
+    info8[6] = (int64_t)P.off_offs;
+    info8[7] = (int64_t)P.off_stream;
     *scale = P.s;
     return 0;
 }
