@@ -53,6 +53,8 @@ def parse_args():
     ap.add_argument("--warmup", type=int, default=200)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--steps-per-tile", type=int, default=0, help="encoder S override (0 = default)")
+    ap.add_argument("--prob-bits", type=int, default=12, choices=[10, 12],
+                    help="frequency totals 2^prob_bits: 12 (the format's choice) or 10")
     ap.add_argument("--e2e-steps", type=int, default=50)
     ap.add_argument("--cpu-seconds", type=float, default=10.0, help="CPU-baseline sample length")
     ap.add_argument("--no-cpu-baseline", action="store_true")
@@ -274,7 +276,7 @@ def reference_arm(args, m, desc):
     if rank != 0:
         return
     import oracle
-    blob = oracle.compress(m.bits, m.dtype, m.target_bpp)
+    blob = oracle.compress(m.bits, m.dtype, m.target_bpp, prob_bits=args.prob_bits)
     info = oracle.blob_info(blob)
     # size each step's sample so that warm-up + steps take about a minute
     t = time.perf_counter()
@@ -357,7 +359,7 @@ def main():
             dist.barrier()
 
     # compress with the library's host encoder
-    cfg = ep.LatticeRANSConfig(mats[0].target_bpp, steps_per_tile=args.steps_per_tile)
+    cfg = ep.LatticeRANSConfig(mats[0].target_bpp, steps_per_tile=args.steps_per_tile, prob_bits=args.prob_bits)
     t = time.perf_counter()
     comps = [ep.compress(W.bits_to_torch(m.bits, m.dtype), cfg) for m in mats]
     enc_s = time.perf_counter() - t
@@ -496,7 +498,7 @@ def main():
                                               f"{psecs:.1f} s"}
         traffic = None
         if launches_per_step == 1:
-            traffic = measured_traffic(f"{args.workload}:{str(out_dts[0]).replace('torch.', '')}")
+            traffic = measured_traffic(f"{args.workload}:{str(out_dts[0]).replace('torch.', '')}:pb{args.prob_bits}")
         info = comps[0].info
         dt_names = [str(dt).replace("torch.", "") for dt in out_dts]
         config = {
@@ -505,6 +507,7 @@ def main():
             "matrices": n,
             "shapes": [list(c.shape) for c in comps],
             "target_bpp": mats[0].target_bpp,
+            "prob_bits": args.prob_bits,
             "actual_bpp": 8.0 * blob_bytes / sum(c.shape[0] * c.shape[1] for c in comps),
             "steps_per_tile": sorted({c.info.steps_per_tile for c in comps}),
             "n_tiles": sum(c.info.n_tiles for c in comps), "blob_bytes": blob_bytes, "out_bytes": out_bytes,

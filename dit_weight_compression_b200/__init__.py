@@ -43,12 +43,13 @@ class EpTensor(ctypes.Structure):
 
 class EpOptions(ctypes.Structure):
     _fields_ = [("steps_per_tile", _I), ("num_threads", _I), ("scale", _D), ("rd_refine", _I),
-                ("host_encoder", _I)]
+                ("host_encoder", _I), ("prob_bits", _I)]
 
 
 class EpBlobInfo(ctypes.Structure):
     _fields_ = [("rows", _I64), ("cols", _I64), ("dtype", _I), ("steps_per_tile", _I),
-                ("n_tiles", _I64), ("n_vectors", _I64), ("scale", _D), ("bytes", ctypes.c_uint64)]
+                ("n_tiles", _I64), ("n_vectors", _I64), ("scale", _D), ("bytes", ctypes.c_uint64),
+                ("prob_bits", _I)]
 
 
 SIGNATURES = {
@@ -132,11 +133,14 @@ class LatticeRANSConfig:
     num_threads: int = 0        # host encoder threads; 0 = all
     rd_refine: bool = False     # per-row rate-distortion refinement (slower encode; off by default)
     host_encoder: bool = False  # encode CUDA tensors on the host instead of on their GPU
+    prob_bits: int = 12         # frequency totals 2^prob_bits: 12 (the format's choice) or 10 (faster decode)
 
     def __post_init__(self):
         t = float(self.target_bpp)
         if not (t == t and 0.001 <= t <= 11.0):
             raise ValueError("target_bpp must be finite and in [0.001, 11]")
+        if self.prob_bits not in (10, 12):
+            raise ValueError("prob_bits must be 12 or 10")
 
 
 class CompressedTensor:
@@ -197,7 +201,7 @@ def compress(tensor: torch.Tensor, config, *, scale: float = 0.0) -> CompressedT
         t = t.contiguous()
     view = tensor_view(t)
     opts = EpOptions(cfg.steps_per_tile, cfg.num_threads, float(scale), int(bool(cfg.rd_refine)),
-                     int(bool(cfg.host_encoder)))
+                     int(bool(cfg.host_encoder)), int(cfg.prob_bits))
     h = ctypes.c_void_p()
     _check(lib().ep_compress_ex(ctypes.byref(view), cfg.target_bpp, ctypes.byref(opts), ctypes.byref(h)),
            "ep_compress")

@@ -50,12 +50,13 @@ extern "C" int ep_compress_ex(const ep_tensor* in, double target_bpp, const ep_o
     bool host_encoder = false;
     if (opt) {
         if (opt->steps_per_tile < 0 || opt->steps_per_tile > 1024 || opt->num_threads < 0 ||
-            !(opt->scale >= 0.0) || !std::isfinite(opt->scale))
+            !(opt->scale >= 0.0) || !std::isfinite(opt->scale) || (opt->prob_bits != 0 && !prob_bits_ok(opt->prob_bits)))
             return set_error(EP_ERR_ARG, "ep_compress: bad options");
         o.steps_per_tile = opt->steps_per_tile;
         o.threads = opt->num_threads;
         o.scale = opt->scale;
         o.rd_refine = opt->rd_refine != 0;
+        o.prob_bits = opt->prob_bits ? opt->prob_bits : kProbBitsDefault;
         host_encoder = opt->host_encoder != 0;
     }
     // A device tensor is encoded on its GPU (same bytes), unless the refinement or the caller asks
@@ -139,6 +140,7 @@ extern "C" int ep_get_info(const ep_blob* b, ep_blob_info* info) {
     info->n_vectors = L.n_vectors;
     info->scale = L.scale;
     info->bytes = b->bytes.size();
+    info->prob_bits = L.prob_bits;
     return EP_OK;
 }
 

@@ -38,13 +38,14 @@ const Launchers* launchers_for(int out_kind) {
 // One blob.  The 32-warp CTA runs only when there are more tiles than 16 warps per SM can hold at
 // once (the 16-warp kernel has twice the registers per thread) and every tile fits the smaller
 // buffer.
-int launch(const Params& p, int out_kind, bool vec, uint64_t max_tile, bool esc, const Ctl& ctl, cudaStream_t st,
-           int device, bool dependent) {
+int launch(const Params& p, int out_kind, const BlobLayout& L, bool vec, const Ctl& ctl, cudaStream_t st, int device,
+           bool dependent) {
     const LaunchCtx c{device, g_dev[device].sms};
-    const bool wide = max_tile <= Geo<kWarpsWide>::kBuf && p.n_tiles > uint32_t(kWarpsNarrow) * uint32_t(c.sms);
-    const Launchers* L = launchers_for(out_kind);
-    if (!L) return set_error(EP_ERR_DTYPE, "decode: unsupported output container");
-    return L->single(p, vec, wide, esc, ctl, st, c, dependent);
+    const bool wide = L.max_tile_bytes <= tile_buffer_bytes(kWarpsWide, L.prob_bits) &&
+                      p.n_tiles > uint32_t(kWarpsNarrow) * uint32_t(c.sms);
+    const Launchers* ln = launchers_for(out_kind);
+    if (!ln) return set_error(EP_ERR_DTYPE, "decode: unsupported output container");
+    return ln->single(p, L.prob_bits, vec, wide, L.has_escape != 0, ctl, st, c, dependent);
 }
 
 // Share `ctas` CTAs among blobs with tiles[i] tiles: every blob gets one, then each further CTA
@@ -109,6 +110,7 @@ Params make_params(const ep_blob* b, const uint8_t* dblob, const uint8_t* tables
     p.vec_per_row = uint32_t(L.vec_per_row);
     p.steps = L.steps;
     p.n_tiles = L.n_tiles;
+    p.joint_split = L.joint_split;
     return p;
 }
 
@@ -133,7 +135,8 @@ int ensure_device(ep_blob* b, int dev, cudaStream_t st) {
     uint8_t* blob = nullptr;
     uint8_t* tables = nullptr;
     uint32_t* status = nullptr;
-    if (cudaMalloc(&blob, b->bytes.size()) != cudaSuccess || cudaMalloc(&tables, kTableBytes) != cudaSuccess ||
+    const int pb = b->layout.prob_bits;
+    if (cudaMalloc(&blob, b->bytes.size()) != cudaSuccess || cudaMalloc(&tables, table_bytes(pb)) != cudaSuccess ||
         cudaMalloc(&status, 16) != cudaSuccess) {
         cudaFree(blob);
         cudaFree(tables);
@@ -145,10 +148,11 @@ int ensure_device(ep_blob* b, int dev, cudaStream_t st) {
     EP_CUDA(cudaMemsetAsync(status, 0, 16, st), "status clear");
     // expand the compact frequency tables once for this device copy
     const TableSrc ts = make_tablesrc(b, blob);
-    auto fn = expand_tables_kernel<kWarpsWide>;
-    EP_CUDA(cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, int(sizeof(ExpandSmem))),
+    auto fn = pb == 10 ? expand_tables_kernel<kWarpsWide, 10> : expand_tables_kernel<kWarpsWide, 12>;
+    const size_t smem = pb == 10 ? sizeof(ExpandSmem<10>) : sizeof(ExpandSmem<12>);
+    EP_CUDA(cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, int(smem)),
             "table expansion attribute");
-    fn<<<1, kWarpsWide * 32, sizeof(ExpandSmem), st>>>(ts, tables);
+    fn<<<1, kWarpsWide * 32, smem, st>>>(ts, tables);
     EP_CUDA(cudaGetLastError(), "table expansion launch");
     EP_CUDA(cudaStreamSynchronize(st), "blob upload");
     d.blob = blob;
@@ -218,7 +222,7 @@ extern "C" int ep_decompress(const ep_blob* cb, const ep_tensor* out, void* stre
         const DeviceCopy& d = b->dev[dev];
         const bool vec = vec_ok(L, out->data, out->row_stride, out->dtype);
         Params p = make_params(b, d.blob, d.tables, out->data, out->row_stride, d.status);
-        return launch(p, kind, vec, L.max_tile_bytes, L.has_escape, Ctl(), st, dev, true);
+        return launch(p, kind, L, vec, Ctl(), st, dev, true);
     }
 
     // Host output: upload the bytes, decode into a blob-owned buffer, copy back, synchronise.
@@ -252,7 +256,7 @@ extern "C" int ep_decompress(const ep_blob* cb, const ep_tensor* out, void* stre
             "ep_decompress: upload");
     const bool vec = vec_ok(L, d.stage_out, L.cols, out->dtype);
     Params p = make_params(b, d.stage_blob, d.tables, d.stage_out, L.cols, d.status);
-    rc = launch(p, kind, vec, L.max_tile_bytes, L.has_escape, Ctl(), st, dev, false);
+    rc = launch(p, kind, L, vec, Ctl(), st, dev, false);
     if (rc != EP_OK) return rc;
     EP_CUDA(cudaMemcpy2DAsync(out->data, size_t(out->row_stride) * es, d.stage_out, size_t(L.cols) * es,
                               size_t(L.cols) * es, size_t(L.rows), cudaMemcpyDeviceToHost, st),
@@ -289,36 +293,43 @@ extern "C" int ep_decompress_group(const ep_blob* const* blobs, const ep_tensor*
     }
     const int sms = g_dev[dev].sms;
     const int chunk = std::max(1, std::min(kMaxGroup, sms));
-    for (int c0 = 0; c0 < n; c0 += chunk) {
-        const int cn = std::min(chunk, n - c0);
-        std::vector<uint32_t> tiles(static_cast<size_t>(cn));
-        uint64_t total = 0, max_tile = 0;
-        for (int i = 0; i < cn; ++i) {
-            const BlobLayout& L = blobs[c0 + i]->layout;
-            tiles[size_t(i)] = L.n_tiles;
-            total += L.n_tiles;
-            max_tile = std::max<uint64_t>(max_tile, L.max_tile_bytes);
+    // one launch per chunk of blobs that share a frequency-total width
+    for (int pb : {12, 10}) {
+        std::vector<int> idx;
+        for (int i = 0; i < n; ++i)
+            if (blobs[i]->layout.prob_bits == pb) idx.push_back(i);
+        for (size_t c0 = 0; c0 < idx.size(); c0 += size_t(chunk)) {
+            const int cn = int(std::min(size_t(chunk), idx.size() - c0));
+            std::vector<uint32_t> tiles(static_cast<size_t>(cn));
+            uint64_t total = 0, max_tile = 0;
+            for (int i = 0; i < cn; ++i) {
+                const BlobLayout& L = blobs[idx[c0 + size_t(i)]]->layout;
+                tiles[size_t(i)] = L.n_tiles;
+                total += L.n_tiles;
+                max_tile = std::max<uint64_t>(max_tile, L.max_tile_bytes);
+            }
+            const std::vector<uint32_t> g = share_ctas(tiles, uint32_t(sms));
+            GroupParams gp = {};
+            gp.n = uint32_t(cn);
+            uint32_t cta = 0;
+            for (int i = 0; i < cn; ++i) {
+                const ep_blob* b = blobs[idx[c0 + size_t(i)]];
+                const ep_tensor& o = outs[idx[c0 + size_t(i)]];
+                const DeviceCopy& d = b->dev[dev];
+                const bool vec = vec_ok(b->layout, o.data, o.row_stride, dtype);
+                GroupEntry& e = gp.e[i];
+                e.p = make_params(b, d.blob, d.tables, o.data, o.row_stride, d.status);
+                e.cta0 = cta;
+                e.ncta = g[size_t(i)];
+                e.vec = vec ? 1u : 0u;
+                e.esc = b->layout.has_escape ? 1u : 0u;
+                cta += e.ncta;
+            }
+            const bool wide = max_tile <= tile_buffer_bytes(kWarpsWide, pb) &&
+                              total > uint64_t(kWarpsNarrow) * uint64_t(cta);
+            rc = launchers_for(kind)->group(gp, pb, cta, wide, st, LaunchCtx{dev, sms});
+            if (rc != EP_OK) return rc;
         }
-        const std::vector<uint32_t> g = share_ctas(tiles, uint32_t(sms));
-        GroupParams gp = {};
-        gp.n = uint32_t(cn);
-        uint32_t cta = 0;
-        for (int i = 0; i < cn; ++i) {
-            const ep_blob* b = blobs[c0 + i];
-            const ep_tensor& o = outs[c0 + i];
-            const DeviceCopy& d = b->dev[dev];
-            const bool vec = vec_ok(b->layout, o.data, o.row_stride, dtype);
-            GroupEntry& e = gp.e[i];
-            e.p = make_params(b, d.blob, d.tables, o.data, o.row_stride, d.status);
-            e.cta0 = cta;
-            e.ncta = g[size_t(i)];
-            e.vec = vec ? 1u : 0u;
-            e.esc = b->layout.has_escape ? 1u : 0u;
-            cta += e.ncta;
-        }
-        const bool wide = max_tile <= Geo<kWarpsWide>::kBuf && total > uint64_t(kWarpsNarrow) * uint64_t(cta);
-        rc = launchers_for(kind)->group(gp, cta, wide, st, LaunchCtx{dev, sms});
-        if (rc != EP_OK) return rc;
     }
     return EP_OK;
 }
@@ -334,7 +345,7 @@ extern "C" int ep_decode_fields(const ep_blob* cb, int16_t* fields, void* stream
     if (rc != EP_OK) return rc;
     const DeviceCopy& d = b->dev[dev];
     Params p = make_params(b, d.blob, d.tables, fields, b->layout.cols, d.status);
-    return launch(p, kOutFields, false, b->layout.max_tile_bytes, true, Ctl(), st, dev, false);
+    return launch(p, kOutFields, b->layout, false, Ctl(), st, dev, false);
 }
 
 extern "C" int ep_decode_wait_probe(const ep_blob* cb, uint32_t wait_spins, void* stream) {
@@ -352,7 +363,7 @@ extern "C" int ep_decode_wait_probe(const ep_blob* cb, uint32_t wait_spins, void
     Ctl ctl;
     ctl.wait_spins = wait_spins;
     ctl.probe_tx = 16;
-    return launch(p, kOutFields, false, b->layout.max_tile_bytes, true, ctl, st, dev, false);
+    return launch(p, kOutFields, b->layout, false, ctl, st, dev, false);
 }
 
 extern "C" int ep_decode_status(const ep_blob* cb, void* stream) {
@@ -446,7 +457,8 @@ extern "C" int ep_decompress_noalloc(const ep_blob* cb, const void* device_blob,
     Params p = make_params(cb, static_cast<const uint8_t*>(device_blob), nullptr, out->data, out->row_stride,
                            status);
     const TableSrc ts = make_tablesrc(cb, static_cast<const uint8_t*>(device_blob));
-    int rc = launchers_for(kind)->noalloc(p, ts, vec, L.has_escape, st, LaunchCtx{dev, g_noalloc[dev].sms});
+    int rc = launchers_for(kind)->noalloc(p, ts, L.prob_bits, vec, L.has_escape != 0, st,
+                                          LaunchCtx{dev, g_noalloc[dev].sms});
     if (rc != EP_OK || !wait) return rc;
     uint32_t s = 0;
     if (cudaMemcpyAsync(&s, status, sizeof s, cudaMemcpyDeviceToHost, st) != cudaSuccess ||

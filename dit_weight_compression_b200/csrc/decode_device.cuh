@@ -9,11 +9,14 @@
 //   * one warp per tile; the tile's 32 interleaved rANS states live one per lane;
 //   * one persistent CTA per SM (16 or 32 warps; grid = min(#SM, #tiles)); tile t goes to CTA
 //     t mod grid, so every SM gets an equal share even when there are few tiles;
-//   * decode tables: one packed 32-bit entry per slot of the 1024-slot range, {slot - cum(s), s
-//     (2 s for f8), escape flag, coset bit, q(s)}, for the joint (coset, f1) symbol and for f2..f8
-//     given each coset -- 15 tables, 60 KB -- so one shared-memory load per symbol gives everything
-//     the state update needs.  They are expanded once per blob and device by a small kernel into a
-//     block next to the device copy; every CTA stages that block into shared memory with bulk
+//   * decode tables, for the joint (coset, f1) symbol and for f2..f8 given each coset (15
+//     tables).  With 10-bit totals: one packed 32-bit entry per slot of the 1024-slot range,
+//     {slot - cum(s), s (2 s for f8), escape flag, coset bit, q(s)} -- 60 KB -- so one
+//     shared-memory load per symbol gives everything the state update needs.  With 12-bit totals
+//     the per-slot entries would take 240 KB, more than an SM has, so a symbol takes two loads:
+//     the slot's symbol byte (4096 per table, 60 KB), then that symbol's {cum(s), escape flag,
+//     q(s)} word (16 KB).  The tables are expanded once per blob and device by a small kernel into
+//     a block next to the device copy; every CTA stages that block into shared memory with bulk
 //     copies, overlapped with the fetch of its first tiles.  (The allocation-free entry point
 //     expands them inside each CTA instead.);
 //   * words: every lane reads its own word stream.  Lanes 2p and 2p+1 share region p of the tile
@@ -70,14 +73,38 @@ constexpr uint32_t kEntrySymShift = 10;
 constexpr uint32_t kEntryEsc = 1u << 19;
 constexpr uint32_t kEntryCosetShift = 20;
 constexpr uint32_t kEntryQShift = 21;
-static_assert(kProbBits == 10, "the packed entry holds 10-bit slots");
+constexpr uint32_t kSlots10 = 1024;
+
+// 12-bit totals.  Symbol byte of slot u of table t at [4096 t + u] (for the joint table the f1
+// symbol of the slot's coset half; the coset is u >= the coset-0 total).  Per-symbol word of
+// table t >= 1 at [kSlotBytes + 1024 (t + 1) + 4 s]; the joint table's at [kSlotBytes + 1024 c +
+// 4 s], its coset-1 cumulative frequencies following all of coset 0's:
+//   bits  0..11  cum(s)
+//   bit  12      s is the escape symbol
+//   bits 16..28  q(s)                 (<= 4096)
+// so the state update x <- q (x >> 12) + (x mod 4096) - cum(s) takes two field extractions.
+constexpr uint32_t kE12CumMask = 0xFFFu;
+constexpr uint32_t kE12Esc = 1u << 12;
+constexpr uint32_t kE12QShift = 16;
+
+// Shared addresses of the decode tables a step reads.
+template <int PB>
+struct Tab {
+    uint32_t t;        // 10-bit: the packed entries, 4 KB aligned
+};
+template <>
+struct Tab<12> {
+    uint32_t s1;       // symbol bytes, 4 KB aligned
+    uint32_t e2;       // per-symbol words
+    uint32_t split;    // slots of coset 0 in the joint table
+};
 
 // Scratch of the table expansion: frequencies and cumulative frequencies of every context.
 struct BuildScratch {
     uint16_t q[kFieldContexts][256];
     uint16_t cum[kFieldContexts][257];
 };
-static_assert(sizeof(BuildScratch) <= 16 * Geo<32>::kBuf, "expansion scratch fits the tile buffers");
+static_assert(sizeof(BuildScratch) <= 16 * Geo<32, 12>::kBuf, "expansion scratch fits the tile buffers");
 
 // ---- PTX wrappers ----------------------------------------------------------------------------
 __device__ __forceinline__ uint32_t smem_u32(const void* p) {
@@ -125,6 +152,12 @@ template <int OFF = 0>
 __device__ __forceinline__ uint32_t lds_u16(uint32_t a) {
     uint32_t v;
     asm volatile("ld.shared.u16 %0, [%1+%2];" : "=r"(v) : "r"(a), "n"(OFF));
+    return v;
+}
+template <int OFF = 0>
+__device__ __forceinline__ uint32_t lds_u8(uint32_t a) {
+    uint32_t v;
+    asm volatile("ld.shared.u8 %0, [%1+%2];" : "=r"(v) : "r"(a), "n"(OFF));
     return v;
 }
 template <int OFF = 0>
@@ -217,11 +250,12 @@ __device__ __forceinline__ uint32_t pack_entry(uint32_t bias, uint32_t s, uint32
            (coset << kEntryCosetShift) | (q << kEntryQShift);
 }
 
-// Fills tab[15][1024] from the blob's compact frequency tables (16 contexts; 0 and 8 together are
-// the joint (coset, f1) table).  `scr` is shared-memory scratch (BuildScratch) that the caller does
-// not use meanwhile.
-template <int WARPS>
-__device__ void build_tables(uint32_t (*tab)[kProbTotal], BuildScratch& scr, const TableSrc& p) {
+// Fills the decode tables at `tab` (shared memory, TableGeo<PB>::kBytes) from the blob's compact
+// frequency tables (16 contexts; 0 and 8 together are the joint (coset, f1) table).  `scr` is
+// shared-memory scratch (BuildScratch) that the caller does not use meanwhile.
+template <int WARPS, int PB>
+__device__ void build_tables(uint8_t* tab, BuildScratch& scr, const TableSrc& p) {
+    constexpr uint32_t M = 1u << PB;
     const uint32_t lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
     // (a) per context: frequencies of symbols 8*lane .. 8*lane+7 and their cumulative sums
     for (uint32_t ctx = warp; ctx < kFieldContexts; ctx += WARPS) {
@@ -252,14 +286,19 @@ __device__ void build_tables(uint32_t (*tab)[kProbTotal], BuildScratch& scr, con
         if (lane == 31) scr.cum[ctx][256] = uint16_t(min(c, 0xFFFFu));
     }
     __syncthreads();
-    // (b) slot -> packed entry.  Lane l of a warp writes slots it*32 + l of its part (one
-    // 128-byte run per store instruction); each lane walks its symbol forward as its slots grow.
+    // (b) slot -> entry (10-bit: the packed word; 12-bit: the symbol byte).  Lane l of a warp
+    // writes slots it*32 + l of its part (one contiguous run per store instruction); each lane
+    // walks its symbol forward as its slots grow.
     constexpr int P = WARPS >= 15 ? WARPS / 15 : 1;
-    constexpr uint32_t kSlotsPerPart = kProbTotal / P;
-    static_assert(kProbTotal % P == 0, "parts split the slots evenly");
+    constexpr uint32_t kSlotsPerPart = M / P;
+    static_assert(M % P == 0, "parts split the slots evenly");
+    uint32_t* tab32 = reinterpret_cast<uint32_t*>(tab);
+    auto put = [&](uint32_t ti, uint32_t slot, uint32_t bias, uint32_t sy, uint32_t q, uint32_t coset, uint32_t sh) {
+        if constexpr (PB == 10) tab32[ti * kSlots10 + slot] = pack_entry(bias, sy, q, coset, sh);
+        else tab[ti * kCtxBytes + slot] = uint8_t(sy);
+    };
     for (uint32_t item = warp; item < uint32_t(kDecodeTables * P); item += WARPS) {
         const uint32_t ti = item / P, part = item % P;
-        uint32_t* dst = tab[ti] + part * kSlotsPerPart;
         if (ti == 0) {  // the joint table: coset 0's slots, then coset 1's
             const uint32_t split = scr.cum[0][256];
             for (uint32_t w = lane; w < kSlotsPerPart; w += 32) {
@@ -268,7 +307,7 @@ __device__ void build_tables(uint32_t (*tab)[kProbTotal], BuildScratch& scr, con
                 const uint32_t local = slot - (c ? split : 0u);
                 const uint16_t* cum = scr.cum[8 * c];
                 const uint32_t sy = slot_symbol(cum, local);
-                dst[w] = pack_entry(local - cum[sy], sy, scr.q[8 * c][sy], c, kEntrySymShift);
+                put(0, slot, local - cum[sy], sy, scr.q[8 * c][sy], c, kEntrySymShift);
             }
             continue;
         }
@@ -276,8 +315,8 @@ __device__ void build_tables(uint32_t (*tab)[kProbTotal], BuildScratch& scr, con
         const uint16_t* cum = scr.cum[ctx];
         const uint16_t* qs = scr.q[ctx];
         const uint32_t sh = (ti - 1) % 7 == 6 ? kEntrySymShift + 1 : kEntrySymShift;  // field 8: 2 s
-        if (cum[256] != kProbTotal) {  // context never used by this blob (the host checked the rest)
-            for (uint32_t w = lane; w < kSlotsPerPart; w += 32) dst[w] = 0;
+        if (cum[256] != M) {  // context never used by this blob (the host checked the rest)
+            for (uint32_t w = lane; w < kSlotsPerPart; w += 32) put(ti, part * kSlotsPerPart + w, 0, 0, 0, 0, 0);
             continue;
         }
         const uint32_t first = part * kSlotsPerPart + lane;
@@ -290,7 +329,20 @@ __device__ void build_tables(uint32_t (*tab)[kProbTotal], BuildScratch& scr, con
                 c0 = next;
                 next = cum[sy + 1];
             }
-            dst[w] = pack_entry(slot - c0, sy, qs[sy], 0u, sh);
+            put(ti, slot, slot - c0, sy, qs[sy], 0u, sh);
+        }
+    }
+    if constexpr (PB == 12) {
+        // (c) the per-symbol words: row 0/1 the joint table's coset halves (coset 1's cumulative
+        // frequencies after coset 0's), row t + 1 table t >= 1
+        uint32_t* ent = reinterpret_cast<uint32_t*>(tab + kSlotBytes);
+        const uint32_t split = scr.cum[0][256];
+        for (uint32_t i = threadIdx.x; i < 16 * 256; i += WARPS * 32) {
+            const uint32_t row = i >> 8, sy = i & 255;
+            const uint32_t ctx = row == 0 ? 0u : row == 1 ? 8u : 8 * ((row - 2) / 7) + 1 + (row - 2) % 7;
+            const uint32_t q = scr.q[ctx][sy];
+            const uint32_t cum = scr.cum[ctx][sy] + (row == 1 ? split : 0u);
+            ent[i] = q ? ((q << kE12QShift) | (sy == uint32_t(kEscape) ? kE12Esc : 0u) | (cum & kE12CumMask)) : 0u;
         }
     }
 }
@@ -426,14 +478,14 @@ struct StepSyms {
 
 // ESC: the blob's tables give the escape symbol a frequency, so a field may be a raw word.
 template <bool ESC, bool FULL, class Reader>
-__device__ __forceinline__ void step_symbols(uint32_t tab, Reader& rd, uint32_t& x, bool active, StepSyms& s) {
+__device__ __forceinline__ void step_symbols10(uint32_t tab, Reader& rd, uint32_t& x, bool active, StepSyms& s) {
     if (FULL) active = true;
     // (coset, f1) as one symbol of the joint table, then f2..f8 from the 7 tables of that coset.
     // A lane past the last vector still loads (from its masked slot, inside the table) but keeps x.
     uint32_t* e = s.e;
     uint32_t acc = 0;
     e[0] = lds_u32<0>(slot_addr(x, tab));
-    if (active) x = (e[0] >> kEntryQShift) * (x >> kProbBits) + (e[0] & kEntryBiasMask);
+    if (active) x = (e[0] >> kEntryQShift) * (x >> 10) + (e[0] & kEntryBiasMask);
     renorm_step<FULL>(x, rd, active);
     if (ESC) acc = e[0];
     const uint32_t c = (e[0] >> kEntryCosetShift) & 1u;
@@ -442,7 +494,7 @@ __device__ __forceinline__ void step_symbols(uint32_t tab, Reader& rd, uint32_t&
 #define EP_FIELD(j)                                                                    \
     {                                                                                  \
         const uint32_t ent = lds_u32<((j) - 1) * kCtxBytes>(slot_addr(x, tb)); \
-        if (active) x = (ent >> kEntryQShift) * (x >> kProbBits) + (ent & kEntryBiasMask); \
+        if (active) x = (ent >> kEntryQShift) * (x >> 10) + (ent & kEntryBiasMask); \
         renorm_step<FULL>(x, rd, active);                                              \
         e[j] = ent;                                                                    \
         if (ESC) acc |= ent;                                                           \
@@ -467,7 +519,72 @@ __device__ __forceinline__ void step_symbols(uint32_t tab, Reader& rd, uint32_t&
     }
 }
 
-template <int OUT, bool VEC, bool ESC>
+// The same with 12-bit totals: per symbol the slot's symbol byte, then that symbol's word.  s.e[j]
+// holds the symbol s_j itself.
+template <bool ESC, bool FULL, class Reader>
+__device__ __forceinline__ void step_symbols12(const Tab<12>& T, Reader& rd, uint32_t& x, bool active, StepSyms& s) {
+    if (FULL) active = true;
+    uint32_t* e = s.e;
+    uint32_t acc = 0;
+    // (coset, f1): the slot's half of the joint table gives the coset (known before the loads
+    // return), its byte the f1 symbol.  A lane past the last vector still loads but keeps x.
+    uint32_t slot = x & 4095u;
+    const uint32_t c = slot >= T.split ? 1u : 0u;
+    {
+        const uint32_t sy = lds_u8<0>(T.s1 + slot);
+        const uint32_t en = lds_u32<0>(T.e2 + 1024u * c + 4u * sy);
+        if (active) x = (en >> kE12QShift) * (x >> 12) + slot - (en & kE12CumMask);
+        renorm_step<FULL>(x, rd, active);
+        e[0] = sy;
+        if (ESC) acc = en;
+    }
+    s.c = c;
+    const uint32_t b1 = T.s1 + kCtxBytes + c * (7u * kCtxBytes);  // field 2's symbol bytes given c
+    const uint32_t b2 = T.e2 + 2048u + c * (7u * 1024u);           // field 2's words given c
+#define EP_FIELD12(j)                                                                         \
+    {                                                                                         \
+        slot = x & 4095u;                                                                     \
+        const uint32_t sy = lds_u8<((j) - 1) * kCtxBytes>(b1 + slot);                         \
+        const uint32_t en = lds_u32<((j) - 1) * 1024>(b2 + 4u * sy);                          \
+        if (active) x = (en >> kE12QShift) * (x >> 12) + slot - (en & kE12CumMask);            \
+        renorm_step<FULL>(x, rd, active);                                                     \
+        e[j] = sy;                                                                            \
+        if (ESC) acc |= en;                                                                   \
+    }
+    EP_FIELD12(1) EP_FIELD12(2) EP_FIELD12(3) EP_FIELD12(4) EP_FIELD12(5) EP_FIELD12(6) EP_FIELD12(7)
+#undef EP_FIELD12
+
+    s.from_symbols = true;
+    if constexpr (ESC) {
+#pragma unroll
+        for (int j = 0; j < 8; ++j) s.f[j] = 0;
+    }
+    if (ESC && __any_sync(kFull, active && (acc & kE12Esc))) {
+        // escaped fields: the lane's raw words after its renormalisation words, by field
+#pragma unroll
+        for (int j = 0; j < 8; ++j) {
+            const bool mine = active && e[j] == uint32_t(kEscape);
+            s.f[j] = mine ? int32_t(int16_t(rd.wn)) : int32_t(e[j]) - kAlphabetR;
+            rd.consume_if(mine);
+        }
+        s.from_symbols = false;
+    }
+}
+
+template <int PB, bool ESC, bool FULL, class Reader>
+__device__ __forceinline__ void step_symbols(const Tab<PB>& tab, Reader& rd, uint32_t& x, bool active, StepSyms& s) {
+    if constexpr (PB == 10) step_symbols10<ESC, FULL>(tab.t, rd, x, active, s);
+    else step_symbols12<ESC, FULL>(tab, rd, x, active, s);
+}
+
+// Symbol s_j of a decoded step (entry layout of the total).
+template <int PB>
+__device__ __forceinline__ uint32_t sym_of(uint32_t e, int j) {
+    if constexpr (PB == 10) return (e >> (kEntrySymShift + (j == 7))) & 255u;
+    else return e;
+}
+
+template <int OUT, bool VEC, bool ESC, int PB>
 __device__ __forceinline__ void step_emit(const Params& p, const StepSyms& s, const Pos& pos) {
     const uint32_t* e = s.e;
     const uint32_t c = s.c;
@@ -480,7 +597,7 @@ __device__ __forceinline__ void step_emit(const Params& p, const StepSyms& s, co
         o[0] = int16_t(c);
 #pragma unroll
         for (int j = 0; j < 8; ++j)
-            o[1 + j] = int16_t(from_symbols ? int32_t((e[j] >> (kEntrySymShift + (j == 7))) & 255u) - kAlphabetR : f[j]);
+            o[1 + j] = int16_t(from_symbols ? int32_t(sym_of<PB>(e[j], j)) - kAlphabetR : f[j]);
         return;
     } else {
         // y_j = z_j + c/2, the lattice coordinate (z1..z7 = f1..f7, z8 = 2 f8 + parity of z1..z7),
@@ -502,8 +619,9 @@ __device__ __forceinline__ void step_emit(const Params& p, const StepSyms& s, co
             }
         };
         if (from_symbols) {
-            // Without escapes f_j = s_j - 127.  s_j sits in bits 10..17 of a field-1..7 entry and
-            // s_8 in bits 11..18 of a field-8 entry, so one mask and OR give
+            // Without escapes f_j = s_j - 127.  With 10-bit totals s_j sits in bits 10..17 of a
+            // field-1..7 entry and s_8 in bits 11..18 of a field-8 entry, so one mask and OR give
+            // (with 12-bit totals e_j is s_j, placed by one shift-and-add)
             //   T_j = 1.5 * 2^23 + 1024 s_j + 512 c:               T_j / 1024 - 12415 = s_j - 127 + c/2,
             //   T_8 = 1.5 * 2^23 + 2048 s_8 + 1024 par + 512 c:    T_8 / 1024 - 12542 = z_8 + c/2,
             // with par = (s_1 + ... + s_7 + 1) mod 2 (7 * 127 is odd), the complement of bit 10
@@ -511,9 +629,10 @@ __device__ __forceinline__ void step_emit(const Params& p, const StepSyms& s, co
             uint32_t t[8];
             const uint32_t km = kMagic | (c << 9);
 #pragma unroll
-            for (int j = 0; j < 7; ++j) t[j] = (e[j] & (0xFFu << kEntrySymShift)) | km;
+            for (int j = 0; j < 7; ++j)
+                t[j] = PB == 10 ? (e[j] & (0xFFu << kEntrySymShift)) | km : e[j] * 1024u + km;
             const uint32_t px = t[0] ^ t[1] ^ t[2] ^ t[3] ^ t[4] ^ t[5] ^ t[6];
-            t[7] = ((e[7] & (0xFFu << (kEntrySymShift + 1))) | km) | (~px & 0x400u);
+            t[7] = (PB == 10 ? (e[7] & (0xFFu << (kEntrySymShift + 1))) | km : e[7] * 2048u + km) | (~px & 0x400u);
             const float2 k = make_float2(1.0f / 1024, 1.0f / 1024), b = make_float2(-12415.0f, -12415.0f);
             scale(t, k, b, k, make_float2(-12415.0f, -12542.0f));
         } else {
@@ -540,14 +659,14 @@ __device__ __forceinline__ void step_emit(const Params& p, const StepSyms& s, co
 }
 
 
-template <int OUT, bool VEC, bool ESC, bool FULL, class Reader>
-__device__ __forceinline__ void decode_step(const Params& p, uint32_t tab, Reader& rd, uint32_t& x, bool active,
+template <int OUT, bool VEC, bool ESC, int PB, bool FULL, class Reader>
+__device__ __forceinline__ void decode_step(const Params& p, const Tab<PB>& tab, Reader& rd, uint32_t& x, bool active,
                                             const Pos& pos) {
     if (FULL) active = true;
     StepSyms s;
-    step_symbols<ESC, FULL>(tab, rd, x, active, s);
+    step_symbols<PB, ESC, FULL>(tab, rd, x, active, s);
     if (!active) return;
-    step_emit<OUT, VEC, ESC>(p, s, pos);
+    step_emit<OUT, VEC, ESC, PB>(p, s, pos);
 }
 
 // Decode `n` full steps, two between runaway checks (the tile buffer's slack covers what two
@@ -555,21 +674,21 @@ __device__ __forceinline__ void decode_step(const Params& p, uint32_t tab, Reade
 // Escape-free blobs are software-pipelined: the symbols of step k + 1 are decoded before step k
 // is written (blobs with escapes keep one step at a time, whose raw-field path would otherwise
 // hold two steps' fields in registers).
-template <int OUT, bool VEC, bool ESC, class Reader, class Guard, class Step>
-__device__ __forceinline__ uint32_t full_run(const Params& p, uint32_t tab, Reader& rd, uint32_t& x, Pos& pos,
+template <int OUT, bool VEC, bool ESC, int PB, class Reader, class Guard, class Step>
+__device__ __forceinline__ uint32_t full_run(const Params& p, const Tab<PB>& tab, Reader& rd, uint32_t& x, Pos& pos,
                                              uint32_t n, Guard in_range, Step walk) {
     if constexpr (ESC) {
         uint32_t k = 0;
         for (; k + 2 <= n; k += 2) {
             if (!__all_sync(kFull, in_range(rd))) return kStOverrun;  // a corrupt tile ran away
-            decode_step<OUT, VEC, ESC, true>(p, tab, rd, x, true, pos);
+            decode_step<OUT, VEC, ESC, PB, true>(p, tab, rd, x, true, pos);
             walk(pos);
-            decode_step<OUT, VEC, ESC, true>(p, tab, rd, x, true, pos);
+            decode_step<OUT, VEC, ESC, PB, true>(p, tab, rd, x, true, pos);
             walk(pos);
         }
         if (k < n) {
             if (!__all_sync(kFull, in_range(rd))) return kStOverrun;
-            decode_step<OUT, VEC, ESC, true>(p, tab, rd, x, true, pos);
+            decode_step<OUT, VEC, ESC, PB, true>(p, tab, rd, x, true, pos);
             walk(pos);
         }
         return 0;
@@ -577,35 +696,35 @@ __device__ __forceinline__ uint32_t full_run(const Params& p, uint32_t tab, Read
     if (n == 0) return 0;
     StepSyms a, b;
     if (!__all_sync(kFull, in_range(rd))) return kStOverrun;
-    step_symbols<ESC, true>(tab, rd, x, true, a);
+    step_symbols<PB, ESC, true>(tab, rd, x, true, a);
     uint32_t k = 1;
     for (; k + 2 <= n; k += 2) {
         if (!__all_sync(kFull, in_range(rd))) return kStOverrun;  // a corrupt tile ran away
-        step_symbols<ESC, true>(tab, rd, x, true, b);
-        step_emit<OUT, VEC, ESC>(p, a, pos);
+        step_symbols<PB, ESC, true>(tab, rd, x, true, b);
+        step_emit<OUT, VEC, ESC, PB>(p, a, pos);
         walk(pos);
-        step_symbols<ESC, true>(tab, rd, x, true, a);
-        step_emit<OUT, VEC, ESC>(p, b, pos);
+        step_symbols<PB, ESC, true>(tab, rd, x, true, a);
+        step_emit<OUT, VEC, ESC, PB>(p, b, pos);
         walk(pos);
     }
     if (k < n) {
         if (!__all_sync(kFull, in_range(rd))) return kStOverrun;
-        step_symbols<ESC, true>(tab, rd, x, true, b);
-        step_emit<OUT, VEC, ESC>(p, a, pos);
+        step_symbols<PB, ESC, true>(tab, rd, x, true, b);
+        step_emit<OUT, VEC, ESC, PB>(p, a, pos);
         walk(pos);
         a = b;
     }
-    step_emit<OUT, VEC, ESC>(p, a, pos);
+    step_emit<OUT, VEC, ESC, PB>(p, a, pos);
     walk(pos);
     return 0;
     }
 }
 
-template <int OUT, bool VEC, bool ESC, int WALK, class Reader, class Guard>
-__device__ __forceinline__ uint32_t full_steps(const Params& p, uint32_t tab, Reader& rd, uint32_t& x, Pos& pos,
+template <int OUT, bool VEC, bool ESC, int PB, int WALK, class Reader, class Guard>
+__device__ __forceinline__ uint32_t full_steps(const Params& p, const Tab<PB>& tab, Reader& rd, uint32_t& x, Pos& pos,
                                                uint32_t nfull, Guard in_range) {
     if constexpr (OUT == kOutFields) {
-        return full_run<OUT, VEC, ESC>(p, tab, rd, x, pos, nfull, in_range, [](Pos& s) { s.optr += 32 * 18; });
+        return full_run<OUT, VEC, ESC, PB>(p, tab, rd, x, pos, nfull, in_range, [](Pos& s) { s.optr += 32 * 18; });
     } else if constexpr (WALK == kWalkRows32) {
         constexpr int es = OutElem<OUT>::kBytes;
         const uint32_t per_row = p.vec_per_row / kLanes;
@@ -615,7 +734,7 @@ __device__ __forceinline__ uint32_t full_steps(const Params& p, uint32_t tab, Re
             // short rows: one run over the whole tile (the step pipeline does not restart at every
             // row), the row change a warp-uniform branch in the walk
             float a_next = pos.row + 1 < p.rows ? __ldg(p.alpha + pos.row + 1) : 0.0f;
-            return full_run<OUT, VEC, ESC>(p, tab, rd, x, pos, nfull, in_range, [&](Pos& s) {
+            return full_run<OUT, VEC, ESC, PB>(p, tab, rd, x, pos, nfull, in_range, [&](Pos& s) {
                 s.optr += 32 * 8 * es;
                 if (--left == 0) {
                     left = per_row;
@@ -631,7 +750,7 @@ __device__ __forceinline__ uint32_t full_steps(const Params& p, uint32_t tab, Re
             const uint32_t n = min(left, nfull - k);
             const float a_next = pos.row + 1 < p.rows ? __ldg(p.alpha + pos.row + 1) : 0.0f;
             const uint32_t st =
-                full_run<OUT, VEC, ESC>(p, tab, rd, x, pos, n, in_range, [](Pos& s) { s.optr += 32 * 8 * es; });
+                full_run<OUT, VEC, ESC, PB>(p, tab, rd, x, pos, n, in_range, [](Pos& s) { s.optr += 32 * 8 * es; });
             if (st) return st;
             k += n;
             left -= n;
@@ -644,7 +763,7 @@ __device__ __forceinline__ uint32_t full_steps(const Params& p, uint32_t tab, Re
         }
         return 0;
     } else {
-        return full_run<OUT, VEC, ESC>(p, tab, rd, x, pos, nfull, in_range,
+        return full_run<OUT, VEC, ESC, PB>(p, tab, rd, x, pos, nfull, in_range,
                                        [&p](Pos& s) { advance<OUT, WALK == kWalkWide>(p, s); });
     }
 }
@@ -652,8 +771,8 @@ __device__ __forceinline__ uint32_t full_steps(const Params& p, uint32_t tab, Re
 // Decode the steps of one tile with a given word reader; returns the status flags of the tile.
 // `pos` is the lane's first vector of the tile (first_pos), found by the caller before the tile's
 // words arrived.
-template <int OUT, bool VEC, bool ESC, class Reader, class Guard>
-__device__ __forceinline__ uint32_t decode_tile_steps(const Params& p, uint32_t tab, Reader& rd, uint32_t& x,
+template <int OUT, bool VEC, bool ESC, int PB, class Reader, class Guard>
+__device__ __forceinline__ uint32_t decode_tile_steps(const Params& p, const Tab<PB>& tab, Reader& rd, uint32_t& x,
                                                       uint32_t tile, uint32_t lane, Pos pos, Guard in_range) {
     const int64_t per_tile = int64_t(kLanes) * p.steps;
     const int64_t v0 = int64_t(tile) * per_tile;
@@ -661,16 +780,16 @@ __device__ __forceinline__ uint32_t decode_tile_steps(const Params& p, uint32_t 
     const uint32_t nfull = nv / kLanes, rem = nv % kLanes;
     uint32_t st;
     if (VEC && OUT != kOutFields && p.vec_per_row % kLanes == 0)
-        st = full_steps<OUT, VEC, ESC, (VEC && OUT != kOutFields) ? kWalkRows32 : kWalkWide>(p, tab, rd, x, pos, nfull,
+        st = full_steps<OUT, VEC, ESC, PB, (VEC && OUT != kOutFields) ? kWalkRows32 : kWalkWide>(p, tab, rd, x, pos, nfull,
                                                                                             in_range);
     else if (p.vec_per_row >= uint32_t(kLanes))
-        st = full_steps<OUT, VEC, ESC, kWalkWide>(p, tab, rd, x, pos, nfull, in_range);
+        st = full_steps<OUT, VEC, ESC, PB, kWalkWide>(p, tab, rd, x, pos, nfull, in_range);
     else
-        st = full_steps<OUT, VEC, ESC, kWalkNarrow>(p, tab, rd, x, pos, nfull, in_range);
+        st = full_steps<OUT, VEC, ESC, PB, kWalkNarrow>(p, tab, rd, x, pos, nfull, in_range);
     if (st) return st;
     if (rem) {
         if (!__all_sync(kFull, in_range(rd))) return kStOverrun;
-        decode_step<OUT, VEC, ESC, false>(p, tab, rd, x, lane < rem, pos);
+        decode_step<OUT, VEC, ESC, PB, false>(p, tab, rd, x, lane < rem, pos);
     }
     return 0;
 }
@@ -678,19 +797,19 @@ __device__ __forceinline__ uint32_t decode_tile_steps(const Params& p, uint32_t 
 // The CTA's layout inside its dynamic shared memory: shifted so that the table (and so every
 // context's 4 KB sub-table) starts on a 4 KB boundary of the shared window, which makes a
 // table address one OR of the slot into the sub-table's base.
-template <int WARPS>
-__device__ __forceinline__ Smem<WARPS>& smem_layout(uint8_t* raw) {
+template <int WARPS, int PB>
+__device__ __forceinline__ Smem<WARPS, PB>& smem_layout(uint8_t* raw) {
     const uint32_t pad = (kAlignSlack - (smem_u32(raw) & (kAlignSlack - 1))) & (kAlignSlack - 1);
-    return *reinterpret_cast<Smem<WARPS>*>(raw + pad);
+    return *reinterpret_cast<Smem<WARPS, PB>*>(raw + pad);
 }
 
 // The work of CTA `cta` of the `ncta` CTAs that decode one blob.
 // BUILD = false: stage the pre-expanded table from p.tables; true: expand it from `ts` in each CTA.
-template <int WARPS, int OUT, bool VEC, bool BUILD, bool ESC>
+template <int WARPS, int OUT, bool VEC, bool BUILD, bool ESC, int PB>
 __device__ __forceinline__ void decode_ctas(const Params& p, const TableSrc* ts, const Ctl& ctl, uint8_t* smem_raw,
                                             uint32_t cta, uint32_t ncta) {
-    Smem<WARPS>& sm = smem_layout<WARPS>(smem_raw);
-    constexpr uint32_t kBuf = Geo<WARPS>::kBuf;
+    Smem<WARPS, PB>& sm = smem_layout<WARPS, PB>(smem_raw);
+    constexpr uint32_t kBuf = Geo<WARPS, PB>::kBuf;
     constexpr uint64_t kMaxTile = 1ull << 22;  // above 160 B + 16 regions of 65535 words
     const uint32_t lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
     const bool fwd = (lane & 1) == 0;  // lanes 2p read forward, lanes 2p+1 backward
@@ -709,9 +828,9 @@ __device__ __forceinline__ void decode_ctas(const Params& p, const TableSrc* ts,
     }
     __syncthreads();  // barriers initialised before anyone uses them
     if (!BUILD && threadIdx.x == 0) {
-        mbar_expect_tx(&sm.tbar, kTableBytes);
-        for (uint32_t o = 0; o < kTableBytes; o += kTablePiece)
-            bulk_g2s(reinterpret_cast<uint8_t*>(&sm.tab[0][0]) + o, p.tables + o, kTablePiece, &sm.tbar);
+        mbar_expect_tx(&sm.tbar, TableGeo<PB>::kBytes);
+        for (uint32_t o = 0; o < TableGeo<PB>::kBytes; o += TableGeo<PB>::kPiece)
+            bulk_g2s(sm.tab + o, p.tables + o, TableGeo<PB>::kPiece, &sm.tbar);
     }
 
     const uint32_t tile_stride = ncta * WARPS;
@@ -749,7 +868,7 @@ __device__ __forceinline__ void decode_ctas(const Params& p, const TableSrc* ts,
     uint32_t tbytes = 0;
     bool first_ok = false, first_staged = false;
     if (BUILD) {  // expand the table first: its scratch lies in the tile buffers
-        build_tables<WARPS>(sm.tab, *reinterpret_cast<BuildScratch*>(&sm.tbuf[0][0]), *ts);
+        build_tables<WARPS, PB>(sm.tab, *reinterpret_cast<BuildScratch*>(&sm.tbuf[0][0]), *ts);
         __syncthreads();
     }
     if (tile < p.n_tiles) {  // the first tile's fetch overlaps the table staging
@@ -774,7 +893,14 @@ __device__ __forceinline__ void decode_ctas(const Params& p, const TableSrc* ts,
 
     asm volatile("griddepcontrol.wait;" ::: "memory");  // no-op unless launched as a dependent
     {
-        const uint32_t tab = smem_u32(&sm.tab[0][0]);
+        Tab<PB> tab;
+        if constexpr (PB == 10) {
+            tab.t = smem_u32(sm.tab);
+        } else {
+            tab.s1 = smem_u32(sm.tab);
+            tab.e2 = smem_u32(sm.tab + kSlotBytes);
+            tab.split = p.joint_split;
+        }
         bool first = true;
         for (; tile < p.n_tiles; tile += tile_stride) {
             bool ok = first_ok;
@@ -828,7 +954,7 @@ __device__ __forceinline__ void decode_ctas(const Params& p, const TableSrc* ts,
                 rd.wp = buf_a + uint32_t(min(max(o0, 0), int32_t(tbytes) - 2));
                 rd.wn = lds_u16(rd.wp);
                 const uint32_t wp0 = rd.wp, lo = buf_a, hi = buf_a + kBuf;
-                flags = decode_tile_steps<OUT, VEC, ESC>(p, tab, rd, x, tile, lane, pos,
+                flags = decode_tile_steps<OUT, VEC, ESC, PB>(p, tab, rd, x, tile, lane, pos,
                                                          [=](const SmemReader& r) { return r.wp - lo <= hi - lo; });
                 nread = rd.consumed(wp0);
             } else {
@@ -838,7 +964,7 @@ __device__ __forceinline__ void decode_ctas(const Params& p, const TableSrc* ts,
                 rd.hi = int32_t(tbytes) - 2;
                 rd.off = o0;
                 rd.wn = __ldg(reinterpret_cast<const uint16_t*>(tg + min(max(o0, 0), rd.hi)));
-                flags = decode_tile_steps<OUT, VEC, ESC>(p, tab, rd, x, tile, lane, pos,
+                flags = decode_tile_steps<OUT, VEC, ESC, PB>(p, tab, rd, x, tile, lane, pos,
                                                          [](const GlobalReader&) { return true; });
                 nread = rd.consumed(o0);
             }
@@ -863,15 +989,17 @@ drain:
 }
 
 // One blob over the whole grid.
-template <int WARPS, int OUT, bool VEC, bool BUILD, bool ESC>
+template <int WARPS, int OUT, bool VEC, bool BUILD, bool ESC, int PB>
 __global__ void __launch_bounds__(WARPS * 32, 1) decode_kernel(const __grid_constant__ Params p,
                                                                const __grid_constant__ TableSrc ts,
                                                                const __grid_constant__ Ctl ctl) {
     extern __shared__ __align__(128) uint8_t smem_raw[];
-    decode_ctas<WARPS, OUT, VEC, BUILD, ESC>(p, &ts, ctl, smem_raw, blockIdx.x, gridDim.x);
+    decode_ctas<WARPS, OUT, VEC, BUILD, ESC, PB>(p, &ts, ctl, smem_raw, blockIdx.x, gridDim.x);
 }
 
-template <int WARPS, int OUT>
+// A set of blobs (all with frequency totals 2^PB) in one launch: blob m owns CTAs
+// [cta0, cta0 + ncta) and stages only its own table.  Every blob picks its store and escape variant.
+template <int WARPS, int OUT, int PB>
 __global__ void __launch_bounds__(WARPS * 32, 1) group_kernel(const __grid_constant__ GroupParams g) {
     extern __shared__ __align__(128) uint8_t smem_raw[];
     uint32_t m = 0;
@@ -881,30 +1009,31 @@ __global__ void __launch_bounds__(WARPS * 32, 1) group_kernel(const __grid_const
     const uint32_t cta = blockIdx.x - e.cta0;
     const Ctl ctl;
     if (e.vec) {
-        if (e.esc) decode_ctas<WARPS, OUT, true, false, true>(e.p, nullptr, ctl, smem_raw, cta, e.ncta);
-        else decode_ctas<WARPS, OUT, true, false, false>(e.p, nullptr, ctl, smem_raw, cta, e.ncta);
+        if (e.esc) decode_ctas<WARPS, OUT, true, false, true, PB>(e.p, nullptr, ctl, smem_raw, cta, e.ncta);
+        else decode_ctas<WARPS, OUT, true, false, false, PB>(e.p, nullptr, ctl, smem_raw, cta, e.ncta);
     } else {
-        if (e.esc) decode_ctas<WARPS, OUT, false, false, true>(e.p, nullptr, ctl, smem_raw, cta, e.ncta);
-        else decode_ctas<WARPS, OUT, false, false, false>(e.p, nullptr, ctl, smem_raw, cta, e.ncta);
+        if (e.esc) decode_ctas<WARPS, OUT, false, false, true, PB>(e.p, nullptr, ctl, smem_raw, cta, e.ncta);
+        else decode_ctas<WARPS, OUT, false, false, false, PB>(e.p, nullptr, ctl, smem_raw, cta, e.ncta);
     }
 }
 
-// Expands the blob's compact frequency tables into the 64 KB packed decode table (one CTA).
+// Expands the blob's compact frequency tables into the decode tables (one CTA).
+template <int PB>
 struct ExpandSmem {
-    uint32_t tab[kDecodeTables][kProbTotal];
+    alignas(16) uint8_t tab[TableGeo<PB>::kBytes];
     BuildScratch scratch;
 };
 
-template <int WARPS>
+template <int WARPS, int PB>
 __global__ void __launch_bounds__(WARPS * 32, 1) expand_tables_kernel(const __grid_constant__ TableSrc p,
                                                                        uint8_t* tables) {
     extern __shared__ __align__(128) uint8_t smem_raw[];
-    ExpandSmem& sm = *reinterpret_cast<ExpandSmem*>(smem_raw);
-    build_tables<WARPS>(sm.tab, sm.scratch, p);
+    ExpandSmem<PB>& sm = *reinterpret_cast<ExpandSmem<PB>*>(smem_raw);
+    build_tables<WARPS, PB>(sm.tab, sm.scratch, p);
     __syncthreads();
-    const uint4* s = reinterpret_cast<const uint4*>(smem_raw);
+    const uint4* s = reinterpret_cast<const uint4*>(sm.tab);
     uint4* d = reinterpret_cast<uint4*>(tables);
-    for (uint32_t i = threadIdx.x; i < kTableBytes / 16; i += blockDim.x) d[i] = s[i];
+    for (uint32_t i = threadIdx.x; i < TableGeo<PB>::kBytes / 16; i += blockDim.x) d[i] = s[i];
 }
 
 // ---- launch functions (host side) ------------------------------------------------------------
@@ -922,10 +1051,10 @@ int ctas_per_sm(Fn fn, int threads, size_t smem, const LaunchCtx& c, int* cache,
     return cache[c.device];
 }
 
-template <int WARPS, int OUT, bool VEC, bool ESC>
+template <int WARPS, int OUT, bool VEC, bool ESC, int PB>
 int launch_one(const Params& p, const Ctl& ctl, cudaStream_t st, const LaunchCtx& c, bool dependent) {
-    auto fn = decode_kernel<WARPS, OUT, VEC, false, ESC>;
-    const size_t smem = sizeof(Smem<WARPS>) + kAlignSlack;
+    auto fn = decode_kernel<WARPS, OUT, VEC, false, ESC, PB>;
+    const size_t smem = sizeof(Smem<WARPS, PB>) + kAlignSlack;
     static std::mutex mu;
     static int per_sm[kMaxDevices] = {};
     const int n = ctas_per_sm(fn, WARPS * 32, smem, c, per_sm, mu);
@@ -950,32 +1079,39 @@ int launch_one(const Params& p, const Ctl& ctl, cudaStream_t st, const LaunchCtx
     return EP_OK;
 }
 
-template <int OUT, bool ESC>
+template <int OUT, bool ESC, int PB>
 int launch_width(const Params& p, bool vec, bool wide, const Ctl& ctl, cudaStream_t st, const LaunchCtx& c, bool dep) {
     if (wide)
-        return vec ? launch_one<kWarpsWide, OUT, true, ESC>(p, ctl, st, c, dep)
-                   : launch_one<kWarpsWide, OUT, false, ESC>(p, ctl, st, c, dep);
-    return vec ? launch_one<kWarpsNarrow, OUT, true, ESC>(p, ctl, st, c, dep)
-               : launch_one<kWarpsNarrow, OUT, false, ESC>(p, ctl, st, c, dep);
+        return vec ? launch_one<kWarpsWide, OUT, true, ESC, PB>(p, ctl, st, c, dep)
+                   : launch_one<kWarpsWide, OUT, false, ESC, PB>(p, ctl, st, c, dep);
+    return vec ? launch_one<kWarpsNarrow, OUT, true, ESC, PB>(p, ctl, st, c, dep)
+               : launch_one<kWarpsNarrow, OUT, false, ESC, PB>(p, ctl, st, c, dep);
+}
+
+template <int OUT, int PB>
+int launch_esc(const Params& p, bool vec, bool wide, bool esc, const Ctl& ctl, cudaStream_t st, const LaunchCtx& c,
+               bool dep) {
+    if constexpr (OUT == kOutFields) {  // test hook: the 16-warp kernel has the registers it needs
+        return launch_one<kWarpsNarrow, kOutFields, false, true, PB>(p, ctl, st, c, false);
+    } else {
+        return esc ? launch_width<OUT, true, PB>(p, vec, wide, ctl, st, c, dep)
+                   : launch_width<OUT, false, PB>(p, vec, wide, ctl, st, c, dep);
+    }
 }
 
 // One blob.  esc: the blob's tables give the escape symbol a frequency (else the escape-free
 // kernel runs).
 template <int OUT>
-int launch_single(const Params& p, bool vec, bool wide, bool esc, const Ctl& ctl, cudaStream_t st,
+int launch_single(const Params& p, int pb, bool vec, bool wide, bool esc, const Ctl& ctl, cudaStream_t st,
                   const LaunchCtx& c, bool dep) {
-    if constexpr (OUT == kOutFields) {  // test hook: the 16-warp kernel has the registers it needs
-        return launch_one<kWarpsNarrow, kOutFields, false, true>(p, ctl, st, c, false);
-    } else {
-        return esc ? launch_width<OUT, true>(p, vec, wide, ctl, st, c, dep)
-                   : launch_width<OUT, false>(p, vec, wide, ctl, st, c, dep);
-    }
+    return pb == 10 ? launch_esc<OUT, 10>(p, vec, wide, esc, ctl, st, c, dep)
+                    : launch_esc<OUT, 12>(p, vec, wide, esc, ctl, st, c, dep);
 }
 
-template <int WARPS, int OUT>
+template <int WARPS, int OUT, int PB>
 int group_launch_one(const GroupParams& g, uint32_t grid, cudaStream_t st, const LaunchCtx& c) {
-    auto fn = group_kernel<WARPS, OUT>;
-    const size_t smem = sizeof(Smem<WARPS>) + kAlignSlack;
+    auto fn = group_kernel<WARPS, OUT, PB>;
+    const size_t smem = sizeof(Smem<WARPS, PB>) + kAlignSlack;
     static std::mutex mu;
     static int per_sm[kMaxDevices] = {};
     if (ctas_per_sm(fn, WARPS * 32, smem, c, per_sm, mu) == 0)
@@ -996,19 +1132,22 @@ int group_launch_one(const GroupParams& g, uint32_t grid, cudaStream_t st, const
     return EP_OK;
 }
 
-// A set of blobs over `grid` CTAs.
+// A set of blobs (one total width pb) over `grid` CTAs.
 template <int OUT>
-int launch_group(const GroupParams& g, uint32_t grid, bool wide, cudaStream_t st, const LaunchCtx& c) {
-    return wide ? group_launch_one<kWarpsWide, OUT>(g, grid, st, c)
-                : group_launch_one<kWarpsNarrow, OUT>(g, grid, st, c);
+int launch_group(const GroupParams& g, int pb, uint32_t grid, bool wide, cudaStream_t st, const LaunchCtx& c) {
+    if (pb == 10)
+        return wide ? group_launch_one<kWarpsWide, OUT, 10>(g, grid, st, c)
+                    : group_launch_one<kWarpsNarrow, OUT, 10>(g, grid, st, c);
+    return wide ? group_launch_one<kWarpsWide, OUT, 12>(g, grid, st, c)
+                : group_launch_one<kWarpsNarrow, OUT, 12>(g, grid, st, c);
 }
 
 // The allocation-free decode: tables expanded in every CTA, the status word in caller-provided
 // device memory.  Error messages are static strings (no allocation).
-template <int WARPS, int OUT, bool VEC, bool ESC>
+template <int WARPS, int OUT, bool VEC, bool ESC, int PB>
 int noalloc_launch_one(const Params& p, const TableSrc& ts, cudaStream_t st, const LaunchCtx& c) {
-    auto fn = decode_kernel<WARPS, OUT, VEC, true, ESC>;
-    const size_t smem = sizeof(Smem<WARPS>) + kAlignSlack;
+    auto fn = decode_kernel<WARPS, OUT, VEC, true, ESC, PB>;
+    const size_t smem = sizeof(Smem<WARPS, PB>) + kAlignSlack;
     static std::mutex mu;
     static int per_sm[kMaxDevices] = {};
     const int n = ctas_per_sm(fn, WARPS * 32, smem, c, per_sm, mu);
@@ -1021,13 +1160,19 @@ int noalloc_launch_one(const Params& p, const TableSrc& ts, cudaStream_t st, con
     return EP_OK;
 }
 
-template <int OUT>
-int launch_noalloc(const Params& p, const TableSrc& ts, bool vec, bool esc, cudaStream_t st, const LaunchCtx& c) {
+template <int OUT, int PB>
+int noalloc_esc(const Params& p, const TableSrc& ts, bool vec, bool esc, cudaStream_t st, const LaunchCtx& c) {
     if (esc)
-        return vec ? noalloc_launch_one<kWarpsNarrow, OUT, true, true>(p, ts, st, c)
-                   : noalloc_launch_one<kWarpsNarrow, OUT, false, true>(p, ts, st, c);
-    return vec ? noalloc_launch_one<kWarpsNarrow, OUT, true, false>(p, ts, st, c)
-               : noalloc_launch_one<kWarpsNarrow, OUT, false, false>(p, ts, st, c);
+        return vec ? noalloc_launch_one<kWarpsNarrow, OUT, true, true, PB>(p, ts, st, c)
+                   : noalloc_launch_one<kWarpsNarrow, OUT, false, true, PB>(p, ts, st, c);
+    return vec ? noalloc_launch_one<kWarpsNarrow, OUT, true, false, PB>(p, ts, st, c)
+               : noalloc_launch_one<kWarpsNarrow, OUT, false, false, PB>(p, ts, st, c);
+}
+
+template <int OUT>
+int launch_noalloc(const Params& p, const TableSrc& ts, int pb, bool vec, bool esc, cudaStream_t st,
+                   const LaunchCtx& c) {
+    return pb == 10 ? noalloc_esc<OUT, 10>(p, ts, vec, esc, st, c) : noalloc_esc<OUT, 12>(p, ts, vec, esc, st, c);
 }
 
 // The launch table of one output container (each decode_<container>.cu defines one).

@@ -17,11 +17,22 @@ namespace ep {
 namespace dec {
 
 constexpr uint32_t kWaitSpins = 1u << 22;                     // bounded mbarrier wait (~0.3 s)
-constexpr uint32_t kCtxBytes = 4 * kProbTotal;                // one context's packed table: 4 KB
 // Decode tables: [0] the joint (coset, f1) symbol; [1 + 7c + (j - 2)] field j = 2..8 given coset c.
 constexpr int kDecodeTables = 15;
-constexpr uint32_t kTableBytes = kDecodeTables * kCtxBytes;   // 61440
-constexpr uint32_t kTablePiece = kTableBytes / 4;             // bytes per table bulk copy (15 KB)
+// 10-bit totals: one packed u32 entry per slot, 1024 slots per table (4 KB), 60 KB in all.
+// 12-bit totals: a u8 symbol per slot, 4096 slots per table (4 KB), then a u32 entry per symbol
+// -- 512 for the joint table, 256 for each other -- 60 KB + 16 KB.
+constexpr uint32_t kCtxBytes = 4096;                          // one table's slot block, either total
+constexpr uint32_t kSlotBytes = kDecodeTables * kCtxBytes;    // 61440
+constexpr uint32_t kSymEntryBytes = 16 * 256 * 4;             // 16384 (12-bit totals only)
+template <int PB>
+struct TableGeo {
+    static_assert(PB == 10 || PB == 12, "frequency totals are 10 or 12 bits");
+    static constexpr uint32_t kBytes = PB == 10 ? kSlotBytes : kSlotBytes + kSymEntryBytes;
+    static constexpr uint32_t kPiece = kBytes / 4;             // bytes per table bulk copy
+};
+constexpr uint32_t kMaxTableBytes = TableGeo<12>::kBytes;
+inline uint32_t table_bytes(int pb) { return pb == 10 ? TableGeo<10>::kBytes : TableGeo<12>::kBytes; }
 
 enum OutKind { kOutBF16 = 0, kOutFP16 = 1, kOutE4M3 = 2, kOutF32 = 3, kOutFields = 4, kOutI8 = 5 };
 
@@ -37,7 +48,7 @@ enum : uint32_t {
 // What the decode of one blob needs (small: a grouped launch passes up to kMaxGroup of them as
 // its kernel parameter).
 struct Params {
-    const uint8_t* tables;      // expanded decode table (kTableBytes), or null: expand in-kernel
+    const uint8_t* tables;      // expanded decode tables (TableGeo::kBytes), or null: expand in-kernel
     const uint32_t* tile_off;   // n_tiles + 1 offsets, 16-byte units
     const uint8_t* stream;      // stream section
     const float* alpha;         // per-row fp32 scales
@@ -47,6 +58,7 @@ struct Params {
     uint64_t stream_bytes;      // size of the stream section: every tile must lie inside it
     uint32_t vec_per_row;       // < 2^31 (checked when the blob is parsed)
     uint32_t steps, n_tiles;
+    uint32_t joint_split;       // slots of coset 0 in the joint (coset, f1) table
 };
 
 // Where the blob keeps the compact frequency tables the decode table is expanded from.
@@ -83,28 +95,36 @@ constexpr uint32_t kSmemOptin = 232448;  // 227 KB: the largest dynamic shared m
 constexpr uint32_t kAlignSlack = 4096;    // the table starts on a 4 KB boundary of the shared window
 constexpr uint32_t kBufSlack = 80;        // bytes after a tile buffer that two steps may over-read
 
-// CTA widths: 32 warps with 4992-byte tile buffers, or 16 warps with 10080-byte buffers; a tile
-// larger than its warp's buffer is read from global memory.
+// CTA widths: 32 or 16 warps, each warp with a tile buffer of Geo<WARPS, PB>::kBuf bytes (5120 or
+// 10336 with 10-bit totals, 4608 or 9312 with 12-bit ones); a tile larger than its warp's buffer is
+// read from global memory.
 constexpr int kWarpsWide = 32, kWarpsNarrow = 16;
 
-// Per-warp tile buffer size for a CTA of WARPS warps: what the 227 KB leave after the table.
-template <int WARPS>
+// Per-warp tile buffer size for a CTA of WARPS warps: what the 227 KB leave after the tables.
+template <int WARPS, int PB>
 struct Geo {
     static constexpr uint32_t kBuf =
-        ((kSmemOptin - kAlignSlack - kTableBytes - 64 - WARPS * (kBufSlack + 8) - 16) / WARPS) & ~15u;
+        ((kSmemOptin - kAlignSlack - TableGeo<PB>::kBytes - 64 - WARPS * (kBufSlack + 8) - 16) / WARPS) & ~15u;
 };
-
-template <int WARPS>
+template <int WARPS, int PB>
 struct Smem {
-    uint32_t tab[kDecodeTables][kProbTotal];                        // packed decode tables, 60 KB
-    alignas(16) uint8_t tbuf[WARPS][Geo<WARPS>::kBuf + kBufSlack];  // one staged tile per warp
-    unsigned long long bar[WARPS];                                  // tile staging, one per warp
-    unsigned long long tbar;                                        // the table's bulk copies
-    unsigned long long pbar;                                        // the wait-limit probe
+    alignas(16) uint8_t tab[TableGeo<PB>::kBytes];                      // decode tables
+    alignas(16) uint8_t tbuf[WARPS][Geo<WARPS, PB>::kBuf + kBufSlack];  // one staged tile per warp
+    unsigned long long bar[WARPS];                                      // tile staging, one per warp
+    unsigned long long tbar;                                            // the table's bulk copies
+    unsigned long long pbar;                                            // the wait-limit probe
 };
-static_assert(offsetof(Smem<32>, tbuf) == kTableBytes, "table block must be contiguous");
-static_assert(sizeof(Smem<32>) + kAlignSlack <= kSmemOptin && sizeof(Smem<16>) + kAlignSlack <= kSmemOptin,
+using Smem32x10 = Smem<32, 10>;
+using Smem32x12 = Smem<32, 12>;
+static_assert(offsetof(Smem32x10, tbuf) == TableGeo<10>::kBytes && offsetof(Smem32x12, tbuf) == TableGeo<12>::kBytes,
+              "table block must be contiguous");
+static_assert(sizeof(Smem<32, 10>) + kAlignSlack <= kSmemOptin && sizeof(Smem<16, 10>) + kAlignSlack <= kSmemOptin &&
+              sizeof(Smem<32, 12>) + kAlignSlack <= kSmemOptin && sizeof(Smem<16, 12>) + kAlignSlack <= kSmemOptin,
               "shared memory budget");
+inline uint32_t tile_buffer_bytes(int warps, int pb) {
+    if (pb == 10) return warps == 32 ? Geo<32, 10>::kBuf : Geo<16, 10>::kBuf;
+    return warps == 32 ? Geo<32, 12>::kBuf : Geo<16, 12>::kBuf;
+}
 
 // ---- launch functions, one table per output container ----------------------------------------
 struct LaunchCtx {
@@ -112,14 +132,16 @@ struct LaunchCtx {
     int sms;     // its SM count
 };
 
+// Every function takes the blob's frequency total width pb (10 or 12).
 struct Launchers {
     // one blob; `dependent`: launch as a programmatic dependent of the previous decode
-    int (*single)(const Params& p, bool vec, bool wide, bool esc, const Ctl& ctl, cudaStream_t st,
+    int (*single)(const Params& p, int pb, bool vec, bool wide, bool esc, const Ctl& ctl, cudaStream_t st,
                   const LaunchCtx& c, bool dependent);
-    // a set of blobs over `grid` CTAs
-    int (*group)(const GroupParams& g, uint32_t grid, bool wide, cudaStream_t st, const LaunchCtx& c);
+    // a set of blobs, all with the same pb, over `grid` CTAs
+    int (*group)(const GroupParams& g, int pb, uint32_t grid, bool wide, cudaStream_t st, const LaunchCtx& c);
     // one blob, tables expanded in every CTA, status in caller-provided memory; never allocates
-    int (*noalloc)(const Params& p, const TableSrc& ts, bool vec, bool esc, cudaStream_t st, const LaunchCtx& c);
+    int (*noalloc)(const Params& p, const TableSrc& ts, int pb, bool vec, bool esc, cudaStream_t st,
+                   const LaunchCtx& c);
 };
 
 extern const Launchers kLaunchBF16, kLaunchFP16, kLaunchE4M3, kLaunchF32, kLaunchI8, kLaunchFields;

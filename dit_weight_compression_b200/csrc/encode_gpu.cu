@@ -193,15 +193,17 @@ __global__ void __launch_bounds__(256) quant_kernel(const In in, const double* r
 // Per 32-column chunk of 32 rows (128 vectors), each lane takes 4 vectors: it reads the vector's
 // coset and fields once, rebuilds its 8 lattice coordinates (y = z + c/2, z8 = 2 f8 + parity) and
 // stages w y and y^2 for every real column; then every lane adds its row's terms in column order.
+// The row's largest |2 y| comes from its largest y^2 (exact for half-integers, and so is its root).
 __global__ void __launch_bounds__(kRowWarps * 32) alpha_kernel(const In in, const uint8_t* coset,
-                                                               const int16_t* fields, float* alpha) {
+                                                               const int16_t* fields, float* alpha,
+                                                               uint16_t* rowmax) {
     extern __shared__ double sh[];  // [kRowWarps][2][32][33]
     const int lane = threadIdx.x & 31, w = threadIdx.x >> 5;
     double (*wy)[33] = reinterpret_cast<double (*)[33]>(sh + size_t(w) * 2 * 32 * 33);
     double (*yy)[33] = reinterpret_cast<double (*)[33]>(sh + size_t(w) * 2 * 32 * 33 + 32 * 33);
     const int64_t r0 = (int64_t(blockIdx.x) * kRowWarps + w) * 32;
     if (r0 >= in.rows) return;
-    double swy = 0.0, syy = 0.0;
+    double swy = 0.0, syy = 0.0, ymax2 = 0.0;
     for (int64_t c0 = 0; c0 < in.cols; c0 += 32) {
 #pragma unroll
         for (int m = 0; m < 4; ++m) {
@@ -240,10 +242,14 @@ __global__ void __launch_bounds__(kRowWarps * 32) alpha_kernel(const In in, cons
         for (int j = 0; j < n; ++j) {
             swy = __dadd_rn(swy, wy[lane][j]);
             syy = __dadd_rn(syy, yy[lane][j]);
+            ymax2 = fmax(ymax2, yy[lane][j]);
         }
         __syncwarp();
     }
-    if (r0 + lane < in.rows) alpha[r0 + lane] = syy > 0.0 ? __double2float_rn(__ddiv_rn(swy, syy)) : 0.0f;
+    if (r0 + lane < in.rows) {
+        alpha[r0 + lane] = syy > 0.0 ? __double2float_rn(__ddiv_rn(swy, syy)) : 0.0f;
+        rowmax[r0 + lane] = uint16_t(2.0 * __dsqrt_rn(ymax2));
+    }
 }
 
 // ---- rANS tiles: one warp per tile, one lane per state --------------------------------------------
@@ -254,6 +260,7 @@ struct TileArgs {
     uint32_t steps, n_tiles;
     const uint16_t* q;          // [16][256]
     const uint32_t* cum;        // [16][257]
+    uint32_t prob_bits;         // totals M = 2^prob_bits
     uint32_t* lane_words;       // [n_tiles][32]: words of each lane (counting pass output)
     uint64_t* tile_bytes;       // [n_tiles] (counting pass output)
     const uint64_t* tile_off;   // [n_tiles] byte offsets in the stream (writing pass input)
@@ -311,11 +318,11 @@ __global__ void __launch_bounds__(kTileWarps * 32) tiles_kernel(const TileArgs a
     };
     uint32_t x = kStateLow;
     auto code = [&](uint32_t f, uint32_t c) {
-        if (uint64_t(x) >= (uint64_t(f) << (32 - kProbBits))) {  // renormalise: push 16 bits out
+        if (uint64_t(x) >= (uint64_t(f) << (32 - a.prob_bits))) {  // renormalise: push 16 bits out
             emit(x & 0xFFFFu);
             x >>= 16;
         }
-        x = (x / f) * kProbTotal + (x % f) + c;
+        x = (x / f) * (1u << a.prob_bits) + (x % f) + c;
     };
     for (int64_t k = steps - 1; k >= 0; --k) {
         const int64_t v = v0 + k * kLanes + lane;
@@ -391,7 +398,8 @@ int encode_gpu(const EncodeInput& in, double target, const EncodeOptions& opt, s
     uint8_t* coset = buf.alloc<uint8_t>(size_t(V));
     int16_t* fields = buf.alloc<int16_t>(size_t(V) * 8);
     float* alpha_d = buf.alloc<float>(size_t(rows));
-    if (!rms || !bad || !counts || !coset || !fields || !alpha_d) { why = "device memory"; return -7; }
+    uint16_t* rowmax_d = buf.alloc<uint16_t>(size_t(rows));
+    if (!rms || !bad || !counts || !coset || !fields || !alpha_d || !rowmax_d) { why = "device memory"; return -7; }
 
     const unsigned row_blocks = unsigned((rows + 32 * kRowWarps - 1) / (32 * kRowWarps));
     EPG(cudaMemsetAsync(bad, 0, 4, st), "encode: clear");
@@ -424,7 +432,7 @@ int encode_gpu(const EncodeInput& in, double target, const EncodeOptions& opt, s
     auto estimate = [&](double s) {
         Counts c;
         qrc = qrc ? qrc : quantise(s, n_sample, false, c);
-        return estimate_from_counts(c, rows, cols, n_sample, n_tiles);
+        return estimate_from_counts(c, rows, cols, n_sample, n_tiles, opt.prob_bits);
     };
     double s;
     if (opt.scale > 0.0) {
@@ -448,14 +456,16 @@ int encode_gpu(const EncodeInput& in, double target, const EncodeOptions& opt, s
     Counts all;
     if (int rc = quantise(s, 0, true, all)) return rc;
     Tables T;
-    T.build(all);
+    T.build(all, opt.prob_bits);
     constexpr size_t kAlphaSmem = size_t(kRowWarps) * 2 * 32 * 33 * sizeof(double);
     EPG(cudaFuncSetAttribute(alpha_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, int(kAlphaSmem)),
         "encode: row scales");
-    alpha_kernel<<<row_blocks, kRowWarps * 32, kAlphaSmem, st>>>(d, coset, fields, alpha_d);
+    alpha_kernel<<<row_blocks, kRowWarps * 32, kAlphaSmem, st>>>(d, coset, fields, alpha_d, rowmax_d);
     EPG(cudaGetLastError(), "encode: row scales");
     std::vector<float> alpha(static_cast<size_t>(rows));
+    std::vector<uint16_t> rowmax(static_cast<size_t>(rows));
     EPG(cudaMemcpyAsync(alpha.data(), alpha_d, 4 * size_t(rows), cudaMemcpyDeviceToHost, st), "encode: read back");
+    EPG(cudaMemcpyAsync(rowmax.data(), rowmax_d, 2 * size_t(rows), cudaMemcpyDeviceToHost, st), "encode: read back");
 
     // Tiles: count, lay out, write.
     uint16_t* q_d = buf.alloc<uint16_t>(16 * 256);
@@ -466,7 +476,8 @@ int encode_gpu(const EncodeInput& in, double target, const EncodeOptions& opt, s
     if (!q_d || !cum_d || !lane_words || !tbytes_d || !toff_d) { why = "device memory"; return -7; }
     EPG(cudaMemcpyAsync(q_d, &T.q[0][0], sizeof T.q, cudaMemcpyHostToDevice, st), "encode: tables");
     EPG(cudaMemcpyAsync(cum_d, &T.cum[0][0], sizeof T.cum, cudaMemcpyHostToDevice, st), "encode: tables");
-    TileArgs ta{coset, fields, V, uint32_t(S), uint32_t(n_tiles), q_d, cum_d, lane_words, tbytes_d, toff_d, nullptr};
+    TileArgs ta{coset, fields, V, uint32_t(S), uint32_t(n_tiles), q_d, cum_d, uint32_t(T.prob_bits), lane_words,
+                tbytes_d, toff_d, nullptr};
     const unsigned tile_blocks = unsigned((n_tiles + kTileWarps - 1) / kTileWarps);
     tiles_kernel<false><<<tile_blocks, kTileWarps * 32, 0, st>>>(ta);
     EPG(cudaGetLastError(), "encode: tile sizes");
@@ -479,7 +490,7 @@ int encode_gpu(const EncodeInput& in, double target, const EncodeOptions& opt, s
         stream_bytes += tbytes[size_t(t)];
     }
     uint64_t off_stream = 0;
-    if (!assemble_blob(in.dtype, rows, cols, S, s, T, alpha, tbytes, blob, &off_stream, why)) return -3;
+    if (!assemble_blob(in.dtype, rows, cols, S, s, T, alpha, rowmax, tbytes, blob, &off_stream, why)) return -3;
     uint8_t* stream_d = buf.alloc<uint8_t>(size_t(stream_bytes));
     if (!stream_d) { why = "device memory"; return -7; }
     EPG(cudaMemsetAsync(stream_d, 0, size_t(stream_bytes), st), "encode: clear");

@@ -188,11 +188,11 @@ static void encode_tile(const uint8_t* coset, const int16_t* fields, int64_t nve
     std::vector<uint16_t> lw[kLanes];  // emission order (reverse of reading order)
     const int64_t steps = (nvec + kLanes - 1) / kLanes;
     auto code = [&](uint32_t& st, std::vector<uint16_t>& w, uint32_t f, uint32_t c) {
-        if (uint64_t(st) >= (uint64_t(f) << (32 - kProbBits))) {  // renormalise: push 16 bits out
+        if (uint64_t(st) >= (uint64_t(f) << (32 - T.prob_bits))) {  // renormalise: push 16 bits out
             w.push_back(uint16_t(st));
             st >>= 16;
         }
-        st = (st / f) * kProbTotal + (st % f) + c;
+        st = (st / f) * T.M + (st % f) + c;
     };
     auto put = [&](uint32_t& st, std::vector<uint16_t>& w, int ctx, int sym) {
         code(st, w, T.q[ctx][sym], T.cum[ctx][sym]);
@@ -249,7 +249,8 @@ constexpr int kRdK[kRdCandidates] = {0, -1, 1, -2, 2};
 static double rd_resolution(double s, int ki) { return s * std::exp2(0.5 * kRdK[ki]); }
 
 static std::vector<int> rd_allocate(const ElementReader& rd, const Quantiser& Q, int64_t rows, int64_t cols,
-                                    int64_t vpr, double s, double target, int64_t n_tiles, int threads) {
+                                    int64_t vpr, double s, double target, int64_t n_tiles, int threads,
+                                    int prob_bits) {
     const size_t per = size_t(vpr) * 9, R5 = size_t(kRdCandidates);
     std::vector<uint8_t> sym(size_t(rows) * R5 * per);
     std::vector<uint64_t> nesc(size_t(rows) * R5);
@@ -316,12 +317,12 @@ static std::vector<int> rd_allocate(const ElementReader& rd, const Quantiser& Q,
             }
         }
         Tables T;
-        T.build(all);
+        T.build(all, prob_bits);
         double cost[16 * 256];
         for (int c = 0; c < 16; ++c)
             for (int sy = 0; sy < 256; ++sy)
-                cost[256 * c + sy] = T.q[c][sy] ? -std::log2(double(T.q[c][sy]) / double(kProbTotal))
-                                                : std::log2(double(kProbTotal));
+                cost[256 * c + sy] = T.q[c][sy] ? -std::log2(double(T.q[c][sy]) / double(T.M))
+                                                : std::log2(double(T.M));
         parallel_for(rows, threads, [&](int64_t a, int64_t b, int) {
             for (int64_t r = a; r < b; ++r)
                 for (int ki = 0; ki < kRdCandidates; ++ki) {
@@ -335,9 +336,7 @@ static std::vector<int> rd_allocate(const ElementReader& rd, const Quantiser& Q,
                     R[idx] = bits;
                 }
         });
-        const double meta = double(kHeaderBytes + round_up16(T.section_bytes()) + round_up16(4 * uint64_t(rows)) +
-                                   round_up16(4 * uint64_t(n_tiles + 1))) +
-                            double(n_tiles) * (160.0 + 8.0);
+        const double meta = metadata_bytes(T, rows, n_tiles);
         const double budget = target * double(rows) * double(cols) - 8.0 * meta;
         if (choose(0.0) > budget) {
             double lo = -100.0, hi = 40.0;
@@ -356,12 +355,14 @@ static std::vector<int> rd_allocate(const ElementReader& rd, const Quantiser& Q,
 
 
 bool assemble_blob(int dtype, int64_t rows, int64_t cols, int S, double s, const Tables& T,
-                   const std::vector<float>& alpha, const std::vector<uint64_t>& tile_bytes,
-                   std::vector<uint8_t>& blob, uint64_t* off_stream_out, std::string& why) {
+                   const std::vector<float>& alpha, const std::vector<uint16_t>& rowmax,
+                   const std::vector<uint64_t>& tile_bytes, std::vector<uint8_t>& blob, uint64_t* off_stream_out,
+                   std::string& why) {
     const int64_t n_tiles = int64_t(tile_bytes.size());
     uint64_t tab = T.section_bytes();
     uint64_t off_tab = kHeaderBytes, off_alpha = off_tab + round_up16(tab);
-    uint64_t off_offs = off_alpha + round_up16(4 * uint64_t(rows));
+    uint64_t off_rmax = off_alpha + round_up16(4 * uint64_t(rows));
+    uint64_t off_offs = off_rmax + round_up16(2 * uint64_t(rows));
     uint64_t off_stream = off_offs + round_up16(4 * uint64_t(n_tiles + 1));
     uint64_t stream = 0;
     for (uint64_t t : tile_bytes) stream += t;
@@ -382,6 +383,8 @@ bool assemble_blob(int dtype, int64_t rows, int64_t cols, int S, double s, const
     wr64(p + 56, off_alpha);
     wr64(p + 64, off_offs);
     wr64(p + 72, off_stream);
+    wr64(p + 80, off_rmax);
+    p[88] = uint8_t(T.prob_bits);
     uint8_t* t = p + off_tab;
     for (int c = 0; c < 16; ++c) {
         int lo, cnt;
@@ -396,6 +399,7 @@ bool assemble_blob(int dtype, int64_t rows, int64_t cols, int S, double s, const
         uint32_t bitsf;
         std::memcpy(&bitsf, &alpha[size_t(r)], 4);
         wr32(p + off_alpha + 4 * r, bitsf);
+        wr16(p + off_rmax + 2 * r, rowmax[size_t(r)]);
     }
     uint64_t acc = 0;
     for (int64_t i = 0; i <= n_tiles; ++i) {
@@ -450,7 +454,7 @@ int encode(const EncodeInput& in, double target, const EncodeOptions& opt, std::
         });
         Counts all;
         for (auto& p : part) all.merge(p);
-        return estimate_from_counts(all, rows, cols, n_sample, n_tiles);
+        return estimate_from_counts(all, rows, cols, n_sample, n_tiles, opt.prob_bits);
     };
 
     // Finest scale whose estimate meets the target: bisection on log2 s over [-24, 8].
@@ -473,17 +477,20 @@ int encode(const EncodeInput& in, double target, const EncodeOptions& opt, std::
 
     // Optional per-row resolutions (the rate-distortion refinement).
     std::vector<int> kr;
-    if (opt.rd_refine) kr = rd_allocate(rd, Q, rows, cols, vpr, s, target, n_tiles, threads);
+    if (opt.rd_refine) kr = rd_allocate(rd, Q, rows, cols, vpr, s, target, n_tiles, threads, opt.prob_bits);
 
-    // Full quantisation, least-squares row scales alpha_r = sum w y / sum y^2 (real columns).
+    // Full quantisation, least-squares row scales alpha_r = sum w y / sum y^2 (real columns), and
+    // each row's largest |2 y| (an integer: y is an integer or a half-integer) over real columns.
     std::vector<uint8_t> coset(static_cast<size_t>(V));
     std::vector<int16_t> fields(static_cast<size_t>(V) * 8);
     std::vector<float> alpha(static_cast<size_t>(rows));
+    std::vector<uint16_t> rowmax(static_cast<size_t>(rows));
     std::vector<Counts> part(static_cast<size_t>(threads));
     parallel_for(rows, threads, [&](int64_t a, int64_t b, int t) {
         QVec q;
         for (int64_t r = a; r < b; ++r) {
             double swy = 0.0, syy = 0.0;
+            uint32_t m2 = 0;
             const double sr = kr.empty() ? s : rd_resolution(s, kr[size_t(r)]);
             for (int64_t k = 0; k < vpr; ++k) {
                 Q.quantise(r, k, sr, q);
@@ -494,16 +501,18 @@ int encode(const EncodeInput& in, double target, const EncodeOptions& opt, std::
                     if (8 * k + i < cols) {
                         swy += rd.at(r, 8 * k + i) * q.y[i];
                         syy += q.y[i] * q.y[i];
+                        m2 = std::max(m2, uint32_t(std::fabs(2.0 * q.y[i])));
                     }
                 part[size_t(t)].add(q.coset, q.f);
             }
             alpha[size_t(r)] = syy > 0.0 ? float(swy / syy) : 0.0f;
+            rowmax[size_t(r)] = uint16_t(m2);
         }
     });
     Counts all;
     for (auto& p : part) all.merge(p);
     Tables T;
-    T.build(all);
+    T.build(all, opt.prob_bits);
 
     // Tiles.  (A region's word count is a u16: at most 2 * 17 * S words, fine for S <= 1024.)
     std::vector<std::vector<uint8_t>> tiles(static_cast<size_t>(n_tiles));
@@ -518,7 +527,7 @@ int encode(const EncodeInput& in, double target, const EncodeOptions& opt, std::
     std::vector<uint64_t> sizes(static_cast<size_t>(n_tiles));
     for (int64_t i = 0; i < n_tiles; ++i) sizes[size_t(i)] = tiles[size_t(i)].size();
     uint64_t off_stream = 0;
-    if (!assemble_blob(in.dtype, rows, cols, S, s, T, alpha, sizes, blob, &off_stream, why)) return -3;
+    if (!assemble_blob(in.dtype, rows, cols, S, s, T, alpha, rowmax, sizes, blob, &off_stream, why)) return -3;
     uint64_t acc = 0;
     for (auto& tb : tiles) {
         std::memcpy(blob.data() + off_stream + acc, tb.data(), tb.size());
@@ -532,7 +541,7 @@ int encode(const EncodeInput& in, double target, const EncodeOptions& opt, std::
 // ---------------------------------------------------------------------------------------------
 bool parse_blob(const uint8_t* d, size_t n, BlobLayout& L, std::string& why) {
     auto fail = [&](const char* m) { why = m; return false; };
-    if (n < kHeaderBytes) return fail("shorter than the 80-byte header");
+    if (n < kHeaderBytes) return fail("shorter than the 96-byte header");
     if (std::memcmp(d, "EPK1", 4) != 0) return fail("bad magic");
     if (rd16(d + 4) != kVersion) return fail("unknown version");
     L.dtype = d[6];
@@ -548,6 +557,10 @@ bool parse_blob(const uint8_t* d, size_t n, BlobLayout& L, std::string& why) {
     L.off_alpha = rd64(d + 56);
     L.off_offsets = rd64(d + 64);
     L.off_stream = rd64(d + 72);
+    L.off_rowmax = rd64(d + 80);
+    L.prob_bits = d[88];
+    if (!prob_bits_ok(L.prob_bits)) return fail("frequency total is neither 10 nor 12 bits");
+    const uint32_t M = 1u << L.prob_bits;
     if (L.total != n) return fail("stored size differs from the byte count");
     if (L.rows <= 0 || L.cols <= 0 || L.rows > (int64_t(1) << 40) || L.cols > (int64_t(1) << 33))
         return fail("bad shape");  // (the decoder keeps a row's vector index in 32 bits)
@@ -557,10 +570,11 @@ bool parse_blob(const uint8_t* d, size_t n, BlobLayout& L, std::string& why) {
     int64_t per = int64_t(kLanes) * L.steps;
     if (int64_t(L.n_tiles) != (L.n_vectors + per - 1) / per) return fail("tile count does not match the shape");
     auto aligned = [](uint64_t o) { return (o & 15) == 0; };
-    if (!aligned(L.off_tables) || !aligned(L.off_alpha) || !aligned(L.off_offsets) || !aligned(L.off_stream))
+    if (!aligned(L.off_tables) || !aligned(L.off_alpha) || !aligned(L.off_rowmax) || !aligned(L.off_offsets) ||
+        !aligned(L.off_stream))
         return fail("misaligned section");
     if (L.off_tables < kHeaderBytes || L.off_tables > L.off_alpha ||
-        L.off_alpha + 4 * uint64_t(L.rows) > L.off_offsets ||
+        L.off_alpha + 4 * uint64_t(L.rows) > L.off_rowmax || L.off_rowmax + 2 * uint64_t(L.rows) > L.off_offsets ||
         L.off_offsets + 4 * (uint64_t(L.n_tiles) + 1) > L.off_stream || L.off_stream > n)
         return fail("sections overlap or run past the end");
     uint64_t pos = L.off_tables;
@@ -577,10 +591,10 @@ bool parse_blob(const uint8_t* d, size_t n, BlobLayout& L, std::string& why) {
         uint32_t sum = L.esc_q[c];
         for (int i = 0; i < L.n[c]; ++i) sum += rd16(d + L.q_offset[c] + 2 * i);
         sums[c] = sum;
-        if (c != 0 && c != 8 && sum != 0 && sum != kProbTotal) return fail("field table does not sum to 1024");
+        if (c != 0 && c != 8 && sum != 0 && sum != M) return fail("field table does not sum to its total");
     }
     L.joint_split = sums[0];  // coset-0 half of the joint (coset, f1) table
-    if (sums[0] + sums[8] != kProbTotal) return fail("joint (coset, f1) table does not sum to 1024");
+    if (sums[0] + sums[8] != M) return fail("joint (coset, f1) table does not sum to its total");
     for (int c = 0; c < kFieldContexts; ++c)
         if (L.esc_q[c]) L.has_escape = 1;
     const uint8_t* off = d + L.off_offsets;

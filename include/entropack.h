@@ -75,6 +75,9 @@ typedef struct {
     int host_encoder;    /* nonzero: encode a device tensor on the host (it is copied there first);
                             by default a device tensor is encoded on its GPU -- the same bytes --
                             except with rd_refine, which runs on the host                    */
+    int prob_bits;       /* frequency totals M = 2^prob_bits: 12 (the format's fixed choice, also
+                            selected by 0) or 10 (a faster decode at a rate cost below 0.5% of the
+                            coded bits); anything else is EP_ERR_ARG                          */
 } ep_options;
 
 typedef struct ep_blob ep_blob;
@@ -88,6 +91,7 @@ typedef struct {
     int64_t n_vectors;   /* rows * ceil(cols / 8) */
     double scale;        /* the shared lattice scale s chosen by the rate search */
     uint64_t bytes;      /* stored bytes, including all metadata */
+    int prob_bits;       /* frequency totals 2^prob_bits (12 or 10) */
 } ep_blob_info;
 
 /*

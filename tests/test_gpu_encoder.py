@@ -40,10 +40,11 @@ CASES = [
 ]
 
 
+@pytest.mark.parametrize("pb", [12, 10])
 @pytest.mark.parametrize("name,make", CASES, ids=[c[0] for c in CASES])
-def test_gpu_encoder_equals_oracle(ep, name, make):
+def test_gpu_encoder_equals_oracle(ep, name, make, pb):
     m = make()
-    assert _gpu_blob(ep, m) == oracle.compress(m.bits, m.dtype, m.target_bpp)
+    assert _gpu_blob(ep, m, prob_bits=pb) == oracle.compress(m.bits, m.dtype, m.target_bpp, prob_bits=pb)
 
 
 def test_gpu_encoder_full_size_square(ep):

@@ -63,7 +63,7 @@ def test_group_dit_block_equals_single_decodes(ep):
 def _mixed_set(ep):
     """Blobs that take every variant of the kernel: tile lengths from 16 to 256 steps, an 11-bpp
     blob with escape words, ragged columns (element stores), a one-tile matrix, rows of fewer
-    than 32 vectors, FP16 and BF16 inputs."""
+    than 32 vectors, FP16 and BF16 inputs, 12-bit and 10-bit frequency totals."""
     specs = [
         (W.small(), None, {}),
         (W.square(rows=192, cols=1024), 4.0, {"steps_per_tile": 16}),
@@ -72,6 +72,9 @@ def _mixed_set(ep):
         (W.square(rows=8, cols=8), 4.0, {}),
         (W.dit(4, scale_down=8), None, {"steps_per_tile": 256}),
         (W.square(rows=300, cols=40), 3.0, {}),
+        # 10-bit totals: the call splits the set into one launch per total width
+        (W.square(rows=160, cols=768), 4.0, {"prob_bits": 10}),
+        (W.sweep(11.0, rows=40, cols=704), None, {"prob_bits": 10}),
     ]
     out = []
     for m, t, kw in specs:

@@ -24,6 +24,7 @@ pytestmark = pytest.mark.gpu
 TORCH = {W.BF16: torch.bfloat16, W.FP16: torch.float16, W.E4M3: torch.float8_e4m3fn, W.F32: torch.float32,
          W.INT8: torch.int8}
 NP = {W.BF16: np.uint16, W.FP16: np.uint16, W.E4M3: np.uint8, W.F32: np.uint32, W.INT8: np.uint8}
+PBS = (12, 10)   # frequency totals: 12-bit (the format's choice, default) and 10-bit
 
 
 @pytest.fixture(scope="module")
@@ -124,9 +125,11 @@ def _check_sampled(ep, c, m: W.Matrix, out_dtypes=None, seed=0):
 # GPU decodes oracle-encoded blobs (cross direction 1), every element.
 # ---------------------------------------------------------------------------------------------
 
-def test_small_oracle_blob_all_containers(ep):
+@pytest.mark.parametrize("pb", PBS)
+def test_small_oracle_blob_all_containers(ep, pb):
     m = W.small()
-    blob = oracle.compress(m.bits, m.dtype, m.target_bpp)
+    blob = oracle.compress(m.bits, m.dtype, m.target_bpp, prob_bits=pb)
+    assert oracle.blob_info(blob)["prob_bits"] == pb
     _check_full(ep, blob, m, [W.BF16, W.FP16, W.E4M3, W.F32, W.INT8])
 
 
@@ -148,65 +151,72 @@ def test_int8_container_oracle_blob(ep):
     assert c.dtype == torch.int8
 
 
-def test_square_full_size_oracle_blob(ep):
+@pytest.mark.parametrize("pb", PBS)
+def test_square_full_size_oracle_blob(ep, pb):
     m = W.square()
-    blob = oracle.compress(m.bits, m.dtype, m.target_bpp)
+    blob = oracle.compress(m.bits, m.dtype, m.target_bpp, prob_bits=pb)
     _check_full(ep, blob, m)
 
 
+@pytest.mark.parametrize("pb", PBS)
 @pytest.mark.parametrize("S", [1, 2, 3, 16, 33, 1024])
-def test_steps_per_tile_and_partial_tiles(ep, S):
+def test_steps_per_tile_and_partial_tiles(ep, S, pb):
     m = W.square(rows=97, cols=1000)
-    blob = oracle.compress(m.bits, m.dtype, 4.0, steps_per_tile=S)
+    blob = oracle.compress(m.bits, m.dtype, 4.0, steps_per_tile=S, prob_bits=pb)
     _check_full(ep, blob, m, [W.BF16, W.F32])
 
 
-@pytest.mark.parametrize("cols,S", [(256, 5), (512, 3), (768, 3), (768, 16), (1280, 5), (1536, 100), (1792, 7)])
-def test_short_rows_tiles_starting_mid_row(ep, cols, S):
+@pytest.mark.parametrize("cols,S,pb", [(256, 5, 12), (512, 3, 10), (768, 3, 12), (768, 16, 10), (1280, 5, 12),
+                                       (1536, 100, 12), (1792, 7, 10)])
+def test_short_rows_tiles_starting_mid_row(ep, cols, S, pb):
     """Rows of 1 to 7 steps (a multiple of 32 vectors per row, so a warp's lanes change rows
     together) with tile lengths that are not multiples of the row length: tiles start and end
     inside rows, the row change falls anywhere in a tile's run of steps, the last tile is
     partial."""
     m = W.square(rows=41, cols=cols)
-    blob = oracle.compress(m.bits, m.dtype, 4.0, steps_per_tile=S)
+    blob = oracle.compress(m.bits, m.dtype, 4.0, steps_per_tile=S, prob_bits=pb)
     _check_full(ep, blob, m, [W.BF16, W.FP16, W.E4M3])
 
 
+@pytest.mark.parametrize("pb", PBS)
 @pytest.mark.parametrize("S,rate", [(1, 11.0), (2, 4.0), (1, 0.5)])
-def test_many_tiles_per_warp(ep, S, rate):
+def test_many_tiles_per_warp(ep, S, rate, pb):
     """More tiles than resident warps (148 SMs x 32 warps), so warps decode several tiles one
     after another, each staged into the buffer the previous one used."""
     m = W.sweep(rate, rows=2400, cols=1024)
-    blob = oracle.compress(m.bits, m.dtype, rate, steps_per_tile=S)
+    blob = oracle.compress(m.bits, m.dtype, rate, steps_per_tile=S, prob_bits=pb)
     assert oracle.blob_info(blob)["n_tiles"] > 148 * 32
     _check_full(ep, blob, m)
 
 
+@pytest.mark.parametrize("pb", PBS)
 @pytest.mark.parametrize("shape", [(1, 1), (1, 8), (3, 13), (7, 9), (33, 7), (5, 1000), (17, 4100)])
-def test_ragged_shapes(ep, shape):
+def test_ragged_shapes(ep, shape, pb):
     g = np.random.Generator(np.random.PCG64(shape[0] * 1000 + shape[1]))
     m = W.Matrix(W.to_bf16_bits(g.normal(0, 0.02, shape)), W.BF16, 3.0)
-    blob = oracle.compress(m.bits, m.dtype, m.target_bpp)
+    blob = oracle.compress(m.bits, m.dtype, m.target_bpp, prob_bits=pb)
     _check_full(ep, blob, m, [W.BF16, W.FP16, W.E4M3, W.F32, W.INT8])
 
 
+@pytest.mark.parametrize("pb", PBS)
 @pytest.mark.parametrize("rate", [0.5, 2.0, 11.0])
-def test_rate_extremes_oracle_blob(ep, rate):
+def test_rate_extremes_oracle_blob(ep, rate, pb):
     m = W.sweep(rate, rows=128, cols=1376)
-    blob = oracle.compress(m.bits, m.dtype, rate)
+    blob = oracle.compress(m.bits, m.dtype, rate, prob_bits=pb)
     _check_full(ep, blob, m)
 
 
-def test_degenerate_tables(ep):
-    # constant rows: lone symbols (q = 4096) in most contexts; a zero row; FP16 input
+@pytest.mark.parametrize("pb", PBS)
+def test_degenerate_tables(ep, pb):
+    # constant rows: lone symbols (q = M) in most contexts; a zero row; FP16 input
     g = np.random.Generator(np.random.PCG64(5))
     x = g.normal(0, 0.05, (64, 1)) * np.ones((1, 1024))
     x[3] = 0.0
     m = W.Matrix(W.to_fp16_bits(x), W.FP16, 4.0)
-    blob = oracle.compress(m.bits, m.dtype, m.target_bpp)
+    blob = oracle.compress(m.bits, m.dtype, m.target_bpp, prob_bits=pb)
     _check_full(ep, blob, m)
     z = W.Matrix(W.to_bf16_bits(np.zeros((40, 64))), W.BF16, 1.0)
-    blob = oracle.compress(z.bits, z.dtype, z.target_bpp)
+    blob = oracle.compress(z.bits, z.dtype, z.target_bpp, prob_bits=pb)
     _check_full(ep, blob, z)
 
 

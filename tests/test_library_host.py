@@ -55,12 +55,14 @@ CASES = [
 ]
 
 
+@pytest.mark.parametrize("pb", [12, 10])
 @pytest.mark.parametrize("name,make", CASES, ids=[c[0] for c in CASES])
-def test_library_blob_equals_oracle_blob(ep, name, make):
+def test_library_blob_equals_oracle_blob(ep, name, make, pb):
     m = make()
-    lb = _lib_blob(ep, m).to_bytes()
-    ob = oracle.compress(m.bits, m.dtype, m.target_bpp)
+    lb = _lib_blob(ep, m, prob_bits=pb).to_bytes()
+    ob = oracle.compress(m.bits, m.dtype, m.target_bpp, prob_bits=pb)
     assert lb == ob
+    assert oracle.blob_info(lb)["prob_bits"] == pb
 
 
 @pytest.mark.parametrize("name,make", [CASES[1], CASES[2], CASES[4], ("ragged", lambda: W.small(rows=37, cols=203))],
@@ -69,9 +71,10 @@ def test_rd_refined_blob_equals_oracle_blob(ep, name, make):
     """The optional per-row rate-distortion refinement: library and oracle blobs byte-identical,
     and the thread count does not change the bytes."""
     m = make()
-    ob = oracle.compress(m.bits, m.dtype, m.target_bpp, rd_refine=True)
+    pb = 10 if name == "dit" else 12
+    ob = oracle.compress(m.bits, m.dtype, m.target_bpp, rd_refine=True, prob_bits=pb)
     for threads in (1, 5):
-        cfg = ep.LatticeRANSConfig(m.target_bpp, num_threads=threads, rd_refine=True)
+        cfg = ep.LatticeRANSConfig(m.target_bpp, num_threads=threads, rd_refine=True, prob_bits=pb)
         lb = ep.compress(W.bits_to_torch(m.bits, m.dtype), cfg).to_bytes()
         assert lb == ob
 

@@ -74,10 +74,11 @@ def _two_calls_match(ep, comp, out_dtype, make_out):
     assert free_after == free_before
 
 
-def test_noalloc_matches_decompress_twice(ep):
-    """BF16, vector stores, an escape-free blob."""
+@pytest.mark.parametrize("pb", [12, 10])
+def test_noalloc_matches_decompress_twice(ep, pb):
+    """BF16, vector stores, an escape-free blob; 12-bit and 10-bit frequency totals."""
     m = W.square(rows=1024, cols=2048)
-    comp = ep.compress(W.bits_to_torch(m.bits, m.dtype), m.target_bpp)
+    comp = ep.compress(W.bits_to_torch(m.bits, m.dtype), ep.LatticeRANSConfig(m.target_bpp, prob_bits=pb))
     _two_calls_match(ep, comp, W.BF16, lambda: torch.empty(comp.shape, dtype=torch.bfloat16, device="cuda"))
 
 
