@@ -309,20 +309,22 @@ def reference_arm(args, m, desc):
 # The CUDA arm.
 # ---------------------------------------------------------------------------------------------
 OUT_DTYPES = {"bf16": "bfloat16", "fp16": "float16", "e4m3": "float8_e4m3fn", "f32": "float32",
-              "int8": "int8"}
+              "int8": "int8", "e4m3row": "float8_e4m3fn"}
 
 
 def out_containers(arg: str, default):
-    """The torch dtypes each step decodes into, in order (the input's own by default)."""
+    """The containers each step decodes into, in order (the input's own by default), as
+    (name, torch dtype, row-scaled FP8?)."""
     import torch
     if not arg:
-        return [default]
+        return [(str(default).replace("torch.", ""), default, False)]
     out = []
     for name in arg.split(","):
         name = name.strip().lower()
         if name not in OUT_DTYPES:
             raise SystemExit(f"unknown output container {name!r} (one of {', '.join(OUT_DTYPES)})")
-        out.append(getattr(torch, OUT_DTYPES[name]))
+        out.append((name if name == "e4m3row" else OUT_DTYPES[name], getattr(torch, OUT_DTYPES[name]),
+                    name == "e4m3row"))
     return out
 
 
@@ -377,17 +379,18 @@ def main():
     n = len(comps)
     out_dts = out_containers(args.out_dtype, comps[0].dtype)
     nd = len(out_dts)
-    out_bytes = sum(c.shape[0] * c.shape[1] * torch.empty((), dtype=dt).element_size()
-                    for c in comps for dt in out_dts)
+    out_bytes = sum(c.shape[0] * c.shape[1] * torch.empty((), dtype=dt).element_size() + (4 * c.shape[0] if rs else 0)
+                    for c in comps for _, dt, rs in out_dts)
     blob_bytes = sum(len(b) for b in blobs)
     moved = nd * blob_bytes + out_bytes          # every decode reads its blob once
-    grouped = n > 1 and args.decode == "grouped"
+    grouped = n > 1 and args.decode == "grouped" and not any(rs for _, _, rs in out_dts)
 
     # R independent device copies of the whole set so that consecutive steps miss L2
     R = max(2, math.ceil(3 * L2_BYTES / moved))
     stream = torch.cuda.current_stream()
     copies = [[ep.CompressedTensor.from_bytes(b) for b in blobs] for _ in range(R)]
-    outs = [[[torch.empty(c.shape, dtype=dt, device="cuda") for c in comps] for dt in out_dts] for _ in range(R)]
+    outs = [[[torch.empty(c.shape, dtype=dt, device="cuda") for c in comps] for _, dt, _ in out_dts] for _ in range(R)]
+    sigmas = [[torch.empty(c.shape[0], dtype=torch.float32, device="cuda") for c in comps] for _ in range(R)]
     for cs in copies:
         for c in cs:
             c.prepare(stream=stream)
@@ -397,7 +400,8 @@ def main():
     g_handles = [(ctypes.c_void_p * n)(*[h.value for h in hs]) for hs in handles]
     g_views = [[(ep.EpTensor * n)(*vs) for vs in vd] for vd in views]
     sh = ctypes.c_void_p(stream.cuda_stream)
-    launches_per_step = nd * (math.ceil(n / 32) if grouped else n)
+    launches_per_step = nd * (math.ceil(n / 28) if grouped else n)
+    sig_ptrs = [[ctypes.c_void_p(t.data_ptr()) for t in ts] for ts in sigmas]
 
     def step(i):
         j = i % R
@@ -407,10 +411,14 @@ def main():
                 if rc != 0:
                     raise ep.EPError(rc, "ep_decompress_group")
                 continue
-            for h, v in zip(handles[j], views[j][d]):
-                rc = L.ep_decompress(h, ctypes.byref(v), sh)
+            rowscaled = out_dts[d][2]
+            for b, (h, v) in enumerate(zip(handles[j], views[j][d])):
+                if rowscaled:
+                    rc = L.ep_decompress_fp8_rowscaled(h, ctypes.byref(v), sig_ptrs[j][b], sh)
+                else:
+                    rc = L.ep_decompress(h, ctypes.byref(v), sh)
                 if rc != 0:
-                    raise ep.EPError(rc, "ep_decompress")
+                    raise ep.EPError(rc, "decode")
 
     # a first step, checked by the kernels' own integrity checks
     step(0)
@@ -455,12 +463,16 @@ def main():
     total_ms, avg_step_ms = max_over_ranks([total_ms, avg_step_ms], world)
 
     # end to end through the public call with host buffers: upload each blob, decode, download
-    host_outs = [[torch.empty(c.shape, dtype=dt).pin_memory() for c in comps] for dt in out_dts]
+    host_outs = [[torch.empty(c.shape, dtype=dt).pin_memory() for c in comps] for _, dt, _ in out_dts]
+    host_sig = [torch.empty(c.shape[0], dtype=torch.float32).pin_memory() for c in comps]
 
     def e2e_step():
-        for ho in host_outs:
-            for c, o in zip(comps, ho):
-                ep.decompress(c, out=o)
+        for (_, _, rowscaled), ho in zip(out_dts, host_outs):
+            for c, o, hs in zip(comps, ho, host_sig):
+                if rowscaled:
+                    ep.decompress_fp8_rowscaled(c, out=o, row_scale=hs)
+                else:
+                    ep.decompress(c, out=o)
 
     for _ in range(3):
         e2e_step()
@@ -498,9 +510,9 @@ def main():
                                               f"{psecs:.1f} s"}
         traffic = None
         if launches_per_step == 1:
-            traffic = measured_traffic(f"{args.workload}:{str(out_dts[0]).replace('torch.', '')}:pb{args.prob_bits}")
+            traffic = measured_traffic(f"{args.workload}:{out_dts[0][0]}:pb{args.prob_bits}")
         info = comps[0].info
-        dt_names = [str(dt).replace("torch.", "") for dt in out_dts]
+        dt_names = [name for name, _, _ in out_dts]
         config = {
             "workload": desc if not args.out_dtype else f"{desc.rsplit(', output', 1)[0]}, output "
                                                         f"{' then '.join(dt_names)}",

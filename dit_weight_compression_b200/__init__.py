@@ -66,6 +66,7 @@ SIGNATURES = {
     "ep_decode_fields": (_I, [_P, _P, _P]),
     "ep_decompress_noalloc": (_I, [_P, _P, _SZ, ctypes.POINTER(EpTensor), _P, _I]),
     "ep_decode_wait_probe": (_I, [_P, ctypes.c_uint32, _P]),
+    "ep_decompress_fp8_rowscaled": (_I, [_P, ctypes.POINTER(EpTensor), _P, _P]),
     "ep_blob_free": (None, [_P]),
     "ep_last_error": (ctypes.c_char_p, []),
 }
@@ -230,7 +231,7 @@ def decompress(compressed: CompressedTensor, config=None, *, out: torch.Tensor |
 def decompress_group(compressed: list, *, outs: list | None = None, dtype: torch.dtype | None = None,
                      device=None, stream=None) -> list:
     """Decode several blobs (e.g. one block's linear layers) with ep_decompress_group: one kernel
-    launch per 32 blobs, results bit-identical to decompress().  Outputs are CUDA tensors of one
+    launch per 28 blobs of one frequency-total width, results bit-identical to decompress().  Outputs are CUDA tensors of one
     dtype (the first blob's unless `dtype` or `outs` say otherwise), written asynchronously."""
     n = len(compressed)
     if outs is None:
@@ -251,6 +252,33 @@ def decompress_group(compressed: list, *, outs: list | None = None, dtype: torch
     return outs
 
 
+def decompress_fp8_rowscaled(compressed: CompressedTensor, *, out: torch.Tensor | None = None,
+                             row_scale: torch.Tensor | None = None, device=None, stream=None):
+    """The FP8 container with a per-row scale: returns (payload, row_scale), an E4M3 tensor of the
+    blob's shape normalised per row to +-448 and a float32 vector with one scale per row, such
+    that row_scale[:, None] * payload.float() restores the weights.  One kernel on `stream`."""
+    dev = torch.device("cuda", torch.cuda.current_device()) if device is None else torch.device(device)
+    if out is None:
+        out = torch.empty(compressed.shape, dtype=torch.float8_e4m3fn, device=dev)
+    if row_scale is None:
+        row_scale = torch.empty(compressed.shape[0], dtype=torch.float32, device=out.device)
+    if row_scale.dtype != torch.float32 or row_scale.numel() != compressed.shape[0] or not row_scale.is_contiguous():
+        raise ValueError("row_scale must be a contiguous float32 vector with one entry per row")
+    view = tensor_view(out)
+
+    def call():
+        _check(lib().ep_decompress_fp8_rowscaled(compressed.handle, ctypes.byref(view),
+                                                 ctypes.c_void_p(row_scale.data_ptr()), _stream_handle(stream)),
+               "ep_decompress_fp8_rowscaled")
+
+    if out.is_cuda:
+        with torch.cuda.device(out.device):
+            call()
+    else:  # rejected by the library (device outputs only)
+        call()
+    return out, row_scale
+
+
 def decode_status(compressed: CompressedTensor, stream=None) -> None:
     """Raise EPError if any decode of this blob on the current device found corrupt tiles."""
     _check(lib().ep_decode_status(compressed.handle, _stream_handle(stream)), "ep_decode_status")
@@ -264,5 +292,6 @@ def decode_fields(compressed: CompressedTensor, stream=None) -> torch.Tensor:
     return out
 
 
-__all__ = ["LatticeRANSConfig", "CompressedTensor", "compress", "decompress", "decompress_group", "decode_status",
+__all__ = ["LatticeRANSConfig", "CompressedTensor", "compress", "decompress", "decompress_group",
+           "decompress_fp8_rowscaled", "decode_status",
            "decode_fields", "EPError", "lib", "BF16", "FP16", "FP8_E4M3", "F32", "INT8"]

@@ -20,7 +20,7 @@ CSRC = os.path.join(PKG, "csrc")
 OBJ = os.path.join(PKG, "_build")
 LIB = os.path.join(PKG, "libentropack.so")
 SOURCES = ["api.cpp", "encoder.cpp", "decode.cu", "decode_bf16.cu", "decode_fp16.cu", "decode_e4m3.cu",
-           "decode_f32.cu", "decode_i8.cu", "decode_fields.cu", "encode_gpu.cu"]
+           "decode_f32.cu", "decode_i8.cu", "decode_fields.cu", "decode_e4m3row.cu", "encode_gpu.cu"]
 HEADERS = ["format.h", "blob.h", "tables.h", "decode_launch.h", "decode_device.cuh"]
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]
 

@@ -21,6 +21,7 @@ struct DeviceCopy {
     uint8_t* stage_blob = nullptr;  // host-output path: per-call upload target
     uint8_t* stage_out = nullptr;   // host-output path: decode target before the D2H copy
     size_t stage_out_bytes = 0;
+    float* stage_sigma = nullptr;   // host-output path of the row-scaled FP8 container: row scales
 };
 
 int set_error(int code, const std::string& msg);

@@ -31,6 +31,7 @@ const Launchers* launchers_for(int out_kind) {
         case kOutF32: return &kLaunchF32;
         case kOutI8: return &kLaunchI8;
         case kOutFields: return &kLaunchFields;
+        case kOutE4M3Row: return &kLaunchE4M3Row;
         default: return nullptr;
     }
 }
@@ -100,6 +101,8 @@ Params make_params(const ep_blob* b, const uint8_t* dblob, const uint8_t* tables
     p.tile_off = reinterpret_cast<const uint32_t*>(dblob + L.off_offsets);
     p.stream = dblob + L.off_stream;
     p.alpha = reinterpret_cast<const float*>(dblob + L.off_alpha);
+    p.rowmax = reinterpret_cast<const uint16_t*>(dblob + L.off_rowmax);
+    p.sigma = nullptr;
     p.out = out;
     p.status = status;
     p.rows = L.rows;
@@ -158,6 +161,33 @@ int ensure_device(ep_blob* b, int dev, cudaStream_t st) {
     d.blob = blob;
     d.tables = tables;
     d.status = status;
+    return EP_OK;
+}
+
+// Blob-owned staging buffers of the host-output path on `dev`: the per-call upload target, the
+// decoded output (at least out_bytes) and, for the row-scaled FP8 container, the row scales.
+int ensure_staging(ep_blob* b, int dev, size_t out_bytes, bool sigma) {
+    std::lock_guard<std::mutex> g(b->mu);
+    DeviceCopy& d = b->dev[dev];
+    if (!d.stage_blob && cudaMalloc(&d.stage_blob, b->bytes.size()) != cudaSuccess)
+        return set_error(EP_ERR_OOM, "host-output decode: staging copy of the blob");
+    if (d.stage_out_bytes < out_bytes) {
+        cudaFree(d.stage_out);
+        d.stage_out = nullptr;
+        d.stage_out_bytes = 0;
+        if (cudaMalloc(&d.stage_out, out_bytes) != cudaSuccess)
+            return set_error(EP_ERR_OOM, "host-output decode: staging output");
+        d.stage_out_bytes = out_bytes;
+    }
+    if (sigma && !d.stage_sigma && cudaMalloc(&d.stage_sigma, 4 * size_t(b->layout.rows)) != cudaSuccess)
+        return set_error(EP_ERR_OOM, "host-output decode: staging row scales");
+    if (!b->host_pinned) {
+        // best effort: page-locked host bytes make the per-call upload a direct DMA
+        if (cudaHostRegister(b->bytes.data(), b->bytes.size(), cudaHostRegisterDefault) == cudaSuccess)
+            b->host_pinned = true;
+        else
+            cudaGetLastError();
+    }
     return EP_OK;
 }
 
@@ -229,28 +259,8 @@ extern "C" int ep_decompress(const ep_blob* cb, const ep_tensor* out, void* stre
     rc = ensure_device(b, dev, st);
     if (rc != EP_OK) return rc;
     const size_t es = size_t(dtype_bytes(out->dtype));
-    const size_t out_bytes = size_t(L.rows) * size_t(L.cols) * es;
-    {
-        std::lock_guard<std::mutex> g(b->mu);
-        DeviceCopy& d = b->dev[dev];
-        if (!d.stage_blob && cudaMalloc(&d.stage_blob, b->bytes.size()) != cudaSuccess)
-            return set_error(EP_ERR_OOM, "ep_decompress: staging copy of the blob");
-        if (d.stage_out_bytes < out_bytes) {
-            cudaFree(d.stage_out);
-            d.stage_out = nullptr;
-            d.stage_out_bytes = 0;
-            if (cudaMalloc(&d.stage_out, out_bytes) != cudaSuccess)
-                return set_error(EP_ERR_OOM, "ep_decompress: staging output");
-            d.stage_out_bytes = out_bytes;
-        }
-        if (!b->host_pinned) {
-            // best effort: page-locked host bytes make the per-call upload a direct DMA
-            if (cudaHostRegister(b->bytes.data(), b->bytes.size(), cudaHostRegisterDefault) == cudaSuccess)
-                b->host_pinned = true;
-            else
-                cudaGetLastError();
-        }
-    }
+    rc = ensure_staging(b, dev, size_t(L.rows) * size_t(L.cols) * es, false);
+    if (rc != EP_OK) return rc;
     const DeviceCopy& d = b->dev[dev];
     EP_CUDA(cudaMemcpyAsync(d.stage_blob, b->bytes.data(), b->bytes.size(), cudaMemcpyHostToDevice, st),
             "ep_decompress: upload");
@@ -334,6 +344,55 @@ extern "C" int ep_decompress_group(const ep_blob* const* blobs, const ep_tensor*
     return EP_OK;
 }
 
+extern "C" int ep_decompress_fp8_rowscaled(const ep_blob* cb, const ep_tensor* out, float* row_scale, void* stream) {
+    clear_error();
+    if (!cb || !out || !out->data || !row_scale)
+        return set_error(EP_ERR_ARG, "ep_decompress_fp8_rowscaled: NULL argument");
+    ep_blob* b = const_cast<ep_blob*>(cb);
+    const BlobLayout& L = b->layout;
+    if (out->dtype != kE4M3) return set_error(EP_ERR_DTYPE, "ep_decompress_fp8_rowscaled: output must be FP8 E4M3");
+    if (out->rows != L.rows || out->cols != L.cols)
+        return set_error(EP_ERR_SHAPE, "ep_decompress_fp8_rowscaled: output shape differs from the blob's");
+    if (out->row_stride < out->cols) return set_error(EP_ERR_ARG, "ep_decompress_fp8_rowscaled: row_stride < cols");
+    if (reinterpret_cast<uintptr_t>(row_scale) % 4 != 0)
+        return set_error(EP_ERR_ARG, "ep_decompress_fp8_rowscaled: row_scale must be 4-byte aligned");
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    int dev = 0;
+    int rc = current_device(dev);
+    if (rc != EP_OK) return rc;
+    if (out->device >= 0) {
+        if (out->device != dev)
+            return set_error(EP_ERR_ARG, "ep_decompress_fp8_rowscaled: output is not on the current device");
+        rc = ensure_device(b, dev, st);
+        if (rc != EP_OK) return rc;
+        const DeviceCopy& d = b->dev[dev];
+        const bool vec = vec_ok(L, out->data, out->row_stride, kE4M3);
+        Params p = make_params(b, d.blob, d.tables, out->data, out->row_stride, d.status);
+        p.sigma = row_scale;
+        return launch(p, kOutE4M3Row, L, vec, Ctl(), st, dev, true);
+    }
+    // Host output and host row scales: upload the bytes, decode into blob-owned buffers, copy
+    // both back, synchronise.
+    rc = ensure_device(b, dev, st);
+    if (rc == EP_OK) rc = ensure_staging(b, dev, size_t(L.rows) * size_t(L.cols), true);
+    if (rc != EP_OK) return rc;
+    const DeviceCopy& d = b->dev[dev];
+    EP_CUDA(cudaMemcpyAsync(d.stage_blob, b->bytes.data(), b->bytes.size(), cudaMemcpyHostToDevice, st),
+            "ep_decompress_fp8_rowscaled: upload");
+    const bool vec = vec_ok(L, d.stage_out, L.cols, kE4M3);
+    Params p = make_params(b, d.stage_blob, d.tables, d.stage_out, L.cols, d.status);
+    p.sigma = d.stage_sigma;
+    rc = launch(p, kOutE4M3Row, L, vec, Ctl(), st, dev, false);
+    if (rc != EP_OK) return rc;
+    EP_CUDA(cudaMemcpy2DAsync(out->data, size_t(out->row_stride), d.stage_out, size_t(L.cols), size_t(L.cols),
+                              size_t(L.rows), cudaMemcpyDeviceToHost, st),
+            "ep_decompress_fp8_rowscaled: download");
+    EP_CUDA(cudaMemcpyAsync(row_scale, d.stage_sigma, 4 * size_t(L.rows), cudaMemcpyDeviceToHost, st),
+            "ep_decompress_fp8_rowscaled: download");
+    EP_CUDA(cudaStreamSynchronize(st), "ep_decompress_fp8_rowscaled: synchronise");
+    return EP_OK;
+}
+
 extern "C" int ep_decode_fields(const ep_blob* cb, int16_t* fields, void* stream) {
     clear_error();
     if (!cb || !fields) return set_error(EP_ERR_ARG, "ep_decode_fields: NULL argument");
@@ -402,6 +461,7 @@ extern "C" void ep_blob_free(ep_blob* b) {
         cudaFree(d.status);
         cudaFree(d.stage_blob);
         cudaFree(d.stage_out);
+        cudaFree(d.stage_sigma);
     }
     if (b->host_pinned) cudaHostUnregister(b->bytes.data());
     cudaSetDevice(prev);

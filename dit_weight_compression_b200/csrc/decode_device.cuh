@@ -350,7 +350,7 @@ __device__ void build_tables(uint8_t* tab, BuildScratch& scr, const TableSrc& p)
 // ---- output conversion -----------------------------------------------------------------------
 template <int OUT>
 struct OutElem {
-    static constexpr int kBytes = (OUT == kOutE4M3 || OUT == kOutI8) ? 1 : (OUT == kOutF32 ? 4 : 2);
+    static constexpr int kBytes = (OUT == kOutE4M3 || OUT == kOutE4M3Row || OUT == kOutI8) ? 1 : (OUT == kOutF32 ? 4 : 2);
 };
 
 // Eight values to eight consecutive elements at `dst` (aligned to the vector's size).
@@ -382,7 +382,7 @@ __device__ __forceinline__ void store_vec(uint8_t* dst, const float v[8]) {
         const uint32_t lo = __byte_perm(__byte_perm(q[0], q[1], 0x0040), __byte_perm(q[2], q[3], 0x0040), 0x5410);
         const uint32_t hi = __byte_perm(__byte_perm(q[4], q[5], 0x0040), __byte_perm(q[6], q[7], 0x0040), 0x5410);
         __stcs(reinterpret_cast<uint2*>(dst), make_uint2(lo, hi));
-    } else if constexpr (OUT == kOutE4M3) {
+    } else if constexpr (OUT == kOutE4M3 || OUT == kOutE4M3Row) {
         uint32_t w[4];
 #pragma unroll
         for (int i = 0; i < 4; ++i)
@@ -399,9 +399,32 @@ template <int OUT>
 __device__ __forceinline__ void store_one(uint8_t* dst, float v) {
     if constexpr (OUT == kOutBF16) *reinterpret_cast<__nv_bfloat16*>(dst) = __float2bfloat16_rn(v);
     else if constexpr (OUT == kOutFP16) *reinterpret_cast<__half*>(dst) = __float2half_rn(v);
-    else if constexpr (OUT == kOutE4M3) *dst = uint8_t(__nv_cvt_float_to_fp8(v, __NV_SATFINITE, __NV_E4M3));
+    else if constexpr (OUT == kOutE4M3 || OUT == kOutE4M3Row)
+        *dst = uint8_t(__nv_cvt_float_to_fp8(v, __NV_SATFINITE, __NV_E4M3));
     else if constexpr (OUT == kOutI8) *dst = uint8_t(max(-128, min(127, __float2int_rn(v))));
     else *reinterpret_cast<float*>(dst) = v;
+}
+
+// ---- the row factor a step multiplies the lattice coordinates by -------------------------------
+// The FP8 container with a per-row scale ("EntroPack: ... at Arbitrary Bitrates", abstract: FP8 is
+// one of the containers, and the stored rate is set apart from the restored precision): row r's
+// payload is E4M3(RNE_fp32(y * g_r)), g_r = RNE_fp32(896 / m_r) with alpha_r's sign (0 for an
+// all-zero row or alpha_r = 0), m_r the row's largest |2 y|, so the row's largest value meets 448;
+// sigma_r = RNE_fp32(|alpha_r| m_r / 896) restores it.  Every other container multiplies by alpha_r.
+__device__ __forceinline__ float row_gain(float a, uint32_t m2) {
+    const float g = __fdiv_rn(896.0f, float(m2));  // correctly rounded
+    return (m2 == 0 || a == 0.0f) ? 0.0f : (a < 0.0f ? -g : g);
+}
+// (the double quotient of these operands is never a float rounding tie unless the exact value is,
+// so rounding it to float is the correct rounding of |alpha| m / 896)
+__device__ __forceinline__ float row_sigma(float a, uint32_t m2) {
+    return __double2float_rn(__ddiv_rn(double(fabsf(a)) * double(m2), 896.0));
+}
+template <int OUT>
+__device__ __forceinline__ float row_factor(const Params& p, int64_t row) {
+    const float a = __ldg(p.alpha + row);
+    if constexpr (OUT == kOutE4M3Row) return row_gain(a, __ldg(p.rowmax + row));
+    else return a;
 }
 
 // ---- one step: every lane decodes (at most) one 8-vector --------------------------------------
@@ -426,7 +449,7 @@ __device__ __forceinline__ Pos first_pos(const Params& p, int64_t v) {
         s.row = v / p.vec_per_row;
         s.kcol = uint32_t(v - s.row * p.vec_per_row);
         s.optr = static_cast<uint8_t*>(p.out) + (s.row * p.row_stride + 8 * int64_t(s.kcol)) * OutElem<OUT>::kBytes;
-        s.a = v < p.n_vectors ? __ldg(p.alpha + s.row) : 0.0f;
+        s.a = v < p.n_vectors ? row_factor<OUT>(p, s.row) : 0.0f;
     }
     return s;
 }
@@ -447,14 +470,14 @@ __device__ __forceinline__ void advance(const Params& p, Pos& s) {
             s.kcol -= w ? p.vec_per_row : 0u;
             s.row += w ? 1 : 0;
             s.optr += w ? wrap : 0;
-            if (w && s.row < p.rows) s.a = __ldg(p.alpha + s.row);
+            if (w && s.row < p.rows) s.a = row_factor<OUT>(p, s.row);
         } else if (s.kcol >= p.vec_per_row) {
             do {
                 s.kcol -= p.vec_per_row;
                 ++s.row;
                 s.optr += wrap;
             } while (s.kcol >= p.vec_per_row);
-            s.a = s.row < p.rows ? __ldg(p.alpha + s.row) : 0.0f;
+            s.a = s.row < p.rows ? row_factor<OUT>(p, s.row) : 0.0f;
         }
     }
 }
@@ -733,7 +756,7 @@ __device__ __forceinline__ uint32_t full_steps(const Params& p, const Tab<PB>& t
         if (per_row < 8) {
             // short rows: one run over the whole tile (the step pipeline does not restart at every
             // row), the row change a warp-uniform branch in the walk
-            float a_next = pos.row + 1 < p.rows ? __ldg(p.alpha + pos.row + 1) : 0.0f;
+            float a_next = pos.row + 1 < p.rows ? row_factor<OUT>(p, pos.row + 1) : 0.0f;
             return full_run<OUT, VEC, ESC, PB>(p, tab, rd, x, pos, nfull, in_range, [&](Pos& s) {
                 s.optr += 32 * 8 * es;
                 if (--left == 0) {
@@ -741,14 +764,14 @@ __device__ __forceinline__ uint32_t full_steps(const Params& p, const Tab<PB>& t
                     s.optr += wrap;
                     ++s.row;
                     s.a = a_next;
-                    a_next = s.row + 1 < p.rows ? __ldg(p.alpha + s.row + 1) : 0.0f;
+                    a_next = s.row + 1 < p.rows ? row_factor<OUT>(p, s.row + 1) : 0.0f;
                 }
             });
         }
         // rows of 8 steps or more: one run per row, nothing but the output pointer moving inside it
         for (uint32_t k = 0; k < nfull;) {
             const uint32_t n = min(left, nfull - k);
-            const float a_next = pos.row + 1 < p.rows ? __ldg(p.alpha + pos.row + 1) : 0.0f;
+            const float a_next = pos.row + 1 < p.rows ? row_factor<OUT>(p, pos.row + 1) : 0.0f;
             const uint32_t st =
                 full_run<OUT, VEC, ESC, PB>(p, tab, rd, x, pos, n, in_range, [](Pos& s) { s.optr += 32 * 8 * es; });
             if (st) return st;
@@ -892,6 +915,10 @@ __device__ __forceinline__ void decode_ctas(const Params& p, const TableSrc* ts,
     }
 
     asm volatile("griddepcontrol.wait;" ::: "memory");  // no-op unless launched as a dependent
+    if constexpr (OUT == kOutE4M3Row) {  // the per-row scales, spread over the blob's CTAs
+        for (int64_t r = int64_t(cta) * blockDim.x + threadIdx.x; r < p.rows; r += int64_t(ncta) * blockDim.x)
+            p.sigma[r] = row_sigma(__ldg(p.alpha + r), __ldg(p.rowmax + r));
+    }
     {
         Tab<PB> tab;
         if constexpr (PB == 10) {
@@ -1176,9 +1203,10 @@ int launch_noalloc(const Params& p, const TableSrc& ts, int pb, bool vec, bool e
 }
 
 // The launch table of one output container (each decode_<container>.cu defines one).
+// (The fields test hook and the row-scaled FP8 container are single-blob launches only.)
 template <int OUT>
 constexpr Launchers make_launchers() {
-    if constexpr (OUT == kOutFields) return Launchers{&launch_single<OUT>, nullptr, nullptr};
+    if constexpr (OUT == kOutFields || OUT == kOutE4M3Row) return Launchers{&launch_single<OUT>, nullptr, nullptr};
     else return Launchers{&launch_single<OUT>, &launch_group<OUT>, &launch_noalloc<OUT>};
 }
 

@@ -34,7 +34,9 @@ struct TableGeo {
 constexpr uint32_t kMaxTableBytes = TableGeo<12>::kBytes;
 inline uint32_t table_bytes(int pb) { return pb == 10 ? TableGeo<10>::kBytes : TableGeo<12>::kBytes; }
 
-enum OutKind { kOutBF16 = 0, kOutFP16 = 1, kOutE4M3 = 2, kOutF32 = 3, kOutFields = 4, kOutI8 = 5 };
+// kOutE4M3Row: the FP8 container with a per-row scale -- an E4M3 payload normalised per row to
+// the format's range, plus one fp32 scale per row.
+enum OutKind { kOutBF16 = 0, kOutFP16 = 1, kOutE4M3 = 2, kOutF32 = 3, kOutFields = 4, kOutI8 = 5, kOutE4M3Row = 6 };
 
 // Status word bits (sticky, cleared by ep_decode_status).
 enum : uint32_t {
@@ -52,6 +54,8 @@ struct Params {
     const uint32_t* tile_off;   // n_tiles + 1 offsets, 16-byte units
     const uint8_t* stream;      // stream section
     const float* alpha;         // per-row fp32 scales
+    const uint16_t* rowmax;     // per-row largest |2 y| (row-scaled FP8 only)
+    float* sigma;               // per-row scale output (row-scaled FP8 only)
     void* out;
     uint32_t* status;
     int64_t rows, cols, row_stride, n_vectors;
@@ -78,7 +82,7 @@ struct Ctl {
 };
 
 // A set of blobs in one launch: blob m owns CTAs [cta0, cta0 + ncta).
-constexpr int kMaxGroup = 32;
+constexpr int kMaxGroup = 28;
 struct GroupEntry {
     Params p;
     uint32_t cta0, ncta;
@@ -144,7 +148,7 @@ struct Launchers {
                    const LaunchCtx& c);
 };
 
-extern const Launchers kLaunchBF16, kLaunchFP16, kLaunchE4M3, kLaunchF32, kLaunchI8, kLaunchFields;
+extern const Launchers kLaunchBF16, kLaunchFP16, kLaunchE4M3, kLaunchF32, kLaunchI8, kLaunchFields, kLaunchE4M3Row;
 
 }  // namespace dec
 }  // namespace ep

@@ -132,7 +132,7 @@ int ep_decompress(const ep_blob* b, const ep_tensor* out, void* stream);
 
 /*
  * Decompress a set of blobs -- for example the linear layers of one transformer block, decoded
- * just before they are used -- in as few kernel launches as possible: one per 32 blobs.  Each
+ * just before they are used -- in as few kernel launches as possible: one per 28 blobs that share a frequency-total width.  Each
  * blob is decoded exactly as ep_decompress would decode it (same arithmetic, bit-identical
  * results); the launch divides the GPU among the blobs in proportion to their tiles, so small
  * matrices that would each leave most SMs idle share the GPU instead.  (The pages motivate it:
@@ -149,6 +149,33 @@ int ep_decompress(const ep_blob* b, const ep_tensor* out, void* stream);
  * EP_ERR_DTYPE, EP_ERR_CUDA, EP_ERR_OOM; nothing is launched when an argument is invalid.
  */
 int ep_decompress_group(const ep_blob* const* blobs, const ep_tensor* outs, int n, void* stream);
+
+/*
+ * Decompress into the FP8 container with a per-row scale (the arXiv abstract lists FP8 among the
+ * containers and keeps the stored bitrate apart from the restored precision).  Row r is written
+ * as an E4M3 payload normalised to the format's range plus one fp32 scale sigma_r, so that
+ * sigma_r * payload restores alpha_r * y:
+ *   payload[r][c] = E4M3(RNE_fp32(y * g_r)), round to nearest even, saturating at +-448, with
+ *                   g_r = RNE_fp32(896 / m_r) carrying alpha_r's sign (0 when m_r = 0 or
+ *                   alpha_r = 0) and m_r the row's largest |2 y| (stored in the blob), so every
+ *                   nonzero row reaches +-448;
+ *   row_scale[r]  = RNE_fp32(|alpha_r| * m_r / 896) = rowmax |alpha_r * y| / 448.
+ * Unlike the plain E4M3 container, small weights keep E4M3's relative precision instead of
+ * falling into its subnormal range.
+ *   b          blob.
+ *   out        dtype EP_FP8_E4M3, rows x cols of the blob.  Device output (out->device >= 0,
+ *              the current device): one fused kernel launch on `stream`, asynchronous; the first
+ *              call on a device copies the blob there (allocates and synchronises once).  Host
+ *              output (out->device == -1): the end-to-end path of ep_decompress -- upload, decode
+ *              into blob-owned buffers, copy payload and scales back, synchronise `stream`.
+ *   row_scale  rows floats (4-byte aligned), written: device memory on the current device for a
+ *              device output, host memory for a host output.
+ *   stream     cudaStream_t as void*.
+ * Corrupt tiles are reported by ep_decode_status().  Returns EP_ERR_ARG (NULL pointers,
+ * misaligned row_scale, other-device output), EP_ERR_DTYPE (output not E4M3), EP_ERR_SHAPE,
+ * EP_ERR_CUDA, EP_ERR_OOM.
+ */
+int ep_decompress_fp8_rowscaled(const ep_blob* b, const ep_tensor* out, float* row_scale, void* stream);
 
 /* Stored bits per element: 8 * (stored bytes including metadata) / (rows * cols)
  * ("EntroPack lattice compression", section "Encoding and reconstruction": the reported rate
@@ -210,7 +237,10 @@ int ep_decode_fields(const ep_blob* b, int16_t* fields, void* stream);
  * (different streams, or several devices' host threads racing on one device) race on the status
  * word: serialise them or use ep_decompress.  The first call on each device looks up the array's
  * device address and sets the kernel's launch attributes; make that first call before any stream
- * capture.  Returns EP_ERR_ARG, EP_ERR_SHAPE, EP_ERR_DTYPE, EP_ERR_CUDA, EP_ERR_CORRUPT; messages
+ * capture.  The library allocates nothing, but the CUDA driver loads a kernel's code on its first
+ * launch (lazy module loading, the driver's default), which can take device memory: a caller that
+ * must see no allocation at all makes one call per output container and blob kind beforehand, or
+ * runs with CUDA_MODULE_LOADING=EAGER.  Returns EP_ERR_ARG, EP_ERR_SHAPE, EP_ERR_DTYPE, EP_ERR_CUDA, EP_ERR_CORRUPT; messages
  * from this call never allocate.
  */
 int ep_decompress_noalloc(const ep_blob* b, const void* device_blob, size_t device_blob_bytes, const ep_tensor* out,

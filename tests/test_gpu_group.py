@@ -10,6 +10,7 @@ import pytest
 import torch
 
 import oracle
+import oracle_parallel
 import workloads as W
 
 pytestmark = pytest.mark.gpu
@@ -48,7 +49,7 @@ def _status_all(ep, comps):
 def test_group_dit_block_equals_single_decodes(ep):
     """The six linear layers of a DiT block (four 3072x3072, 3072x8192, 8192x3072; Student-t
     weights with hot rows) at 2.5 bpp, decoded in one launch: bit-identical to six ep_decompress
-    calls."""
+    calls and to the oracle's decode of every tile."""
     comps = [_compress(ep, W.dit(j)) for j in range(len(W.DIT_SHAPES))]
     outs = ep.decompress_group(comps)
     _status_all(ep, comps)
@@ -58,6 +59,8 @@ def test_group_dit_block_equals_single_decodes(ep):
         ep.decode_status(c)
         assert o.shape == single.shape and o.dtype == torch.bfloat16
         assert torch.equal(o.view(torch.int16), single.view(torch.int16))
+        # and against the oracle, every tile
+        assert np.array_equal(_bits(o, W.BF16), oracle_parallel.decode(c.to_bytes(), "values", W.BF16))
 
 
 def _mixed_set(ep):

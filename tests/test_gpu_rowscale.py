@@ -1,0 +1,129 @@
+"""GPU parity of the FP8 container with a per-row scale (ep_decompress_fp8_rowscaled).
+
+The abstract ("EntroPack: ... at Arbitrary Bitrates") lists FP8 among the containers and keeps the
+stored rate apart from the restored precision.  The container is an E4M3 payload normalised per row
+to +-448 plus one fp32 scale per row; the oracle defines it (oracle.c, orc_decompress_rowscaled_tiles)
+and is pinned in test_oracle_pins.py.  Bars: payload bytes and scales bit-exact against the oracle,
+on oracle-encoded blobs (cross direction 1) and library blobs, for both frequency totals, every
+store path (vector, element, strided, misaligned) and blobs with escapes.
+"""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+import workloads as W
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(scope="module")
+def ep():
+    if not torch.cuda.is_available():
+        pytest.skip("no CUDA device")
+    from dit_weight_compression_b200 import build
+    build.build()
+    import dit_weight_compression_b200 as ep
+    return ep
+
+
+def _gpu(ep, c, out=None):
+    pay, sig = ep.decompress_fp8_rowscaled(c, out=out)
+    torch.cuda.synchronize()
+    ep.decode_status(c)
+    return pay.contiguous().view(torch.uint8).cpu().numpy(), sig.cpu().numpy()
+
+
+def _check(ep, blob):
+    c = ep.CompressedTensor.from_bytes(blob)
+    pay, sig = _gpu(ep, c)
+    opay, osig = oracle.decompress_rowscaled(blob)
+    assert np.array_equal(pay, opay)
+    assert np.array_equal(sig.view(np.uint32), osig.view(np.uint32))
+    return c, pay, sig
+
+
+@pytest.mark.parametrize("pb", [12, 10])
+def test_rowscaled_small_and_square_oracle_blobs(ep, pb):
+    for m in (W.small(), W.square(rows=1024, cols=2048)):
+        blob = oracle.compress(m.bits, m.dtype, m.target_bpp, prob_bits=pb)
+        _, pay, _ = _check(ep, blob)
+        p = torch.from_numpy(pay).view(torch.float8_e4m3fn).float()
+        assert torch.all(p.abs().amax(1) == 448.0)            # every row reaches the format's maximum
+
+
+def test_rowscaled_full_size_square(ep):
+    m = W.square()
+    blob = oracle.compress(m.bits, m.dtype, m.target_bpp)
+    _check(ep, blob)
+
+
+@pytest.mark.parametrize("shape,rate", [((37, 203), 3.5), ((5, 1000), 3.0), ((96, 704), 11.0), ((64, 1376), 0.5)])
+def test_rowscaled_ragged_and_rate_extremes(ep, shape, rate):
+    """Ragged columns (element stores), an 11-bpp blob full of escapes, a 0.5-bpp blob."""
+    g = np.random.Generator(np.random.PCG64(shape[0] * 131 + shape[1]))
+    m = W.Matrix(W.to_fp16_bits(g.normal(0, 0.02, shape)), W.FP16, rate)
+    blob = oracle.compress(m.bits, m.dtype, rate)
+    _check(ep, blob)
+
+
+def test_rowscaled_zero_rows_and_strided_outputs(ep):
+    """All-zero rows give a zero payload and a zero scale; outputs that are column windows of a
+    wider tensor, aligned and misaligned, get the same bytes."""
+    g = np.random.Generator(np.random.PCG64(3))
+    x = g.normal(0, 0.02, (64, 256))
+    x[[0, 5, 63]] = 0.0
+    m = W.Matrix(W.to_bf16_bits(x), W.BF16, 4.0)
+    blob = oracle.compress(m.bits, m.dtype, m.target_bpp)
+    c, pay, sig = _check(ep, blob)
+    assert np.all(pay[[0, 5, 63]] == 0) and np.all(sig[[0, 5, 63]] == 0.0)
+    for off in (0, 3):
+        big = torch.zeros((64, 256 + 16), dtype=torch.float8_e4m3fn, device="cuda")
+        view = big[:, off:off + 256]
+        p2, s2 = _gpu(ep, c, out=view)
+        assert np.array_equal(p2, pay) and np.array_equal(s2, sig)
+
+
+def test_rowscaled_library_blob_and_precision_vs_plain_e4m3(ep):
+    """A library-encoded layer shaped like the large-layer workload (N(0, 0.015^2) times column
+    scales in [0.5, 2]): bit-exact against the oracle, and sigma * payload restores the weights
+    with a lower relative L2 error than the plain E4M3 container, whose values of std ~0.015 sit
+    at and below E4M3's smallest normal 2^-6."""
+    m = W.large(0, rows=1024, cols=2048)
+    c = ep.compress(W.bits_to_torch(m.bits, m.dtype), m.target_bpp)
+    blob = c.to_bytes()
+    pay, sig = _gpu(ep, c)
+    opay, osig = oracle.decompress_rowscaled(blob)
+    assert np.array_equal(pay, opay) and np.array_equal(sig, osig)
+    w = oracle.dtype_to_f64(m.bits, m.dtype)
+    rs = sig[:, None].astype(np.float64) * torch.from_numpy(pay).view(torch.float8_e4m3fn).double().numpy()
+    plain = ep.decompress(c, dtype=torch.float8_e4m3fn)
+    torch.cuda.synchronize()
+    pl = plain.double().cpu().numpy()
+    bf = oracle.dtype_to_f64(oracle.decompress(blob, W.BF16), W.BF16)
+    rel = lambda a: np.linalg.norm(a - w) / np.linalg.norm(w)
+    assert rel(rs) < rel(pl)
+    assert rel(rs) < 1.05 * rel(bf) + 0.03          # near the BF16 restore: E4M3 adds ~2^-5 relative noise
+
+
+def test_rowscaled_argument_errors(ep):
+    m = W.small()
+    c = ep.compress(W.bits_to_torch(m.bits, m.dtype), m.target_bpp)
+    with pytest.raises(ep.EPError) as e:
+        ep.decompress_fp8_rowscaled(c, out=torch.empty(c.shape, dtype=torch.bfloat16, device="cuda"))
+    assert e.value.code == -2
+    with pytest.raises(ep.EPError) as e:
+        ep.decompress_fp8_rowscaled(c, out=torch.empty((255, 256), dtype=torch.float8_e4m3fn, device="cuda"),
+                                    row_scale=torch.empty(256, dtype=torch.float32, device="cuda"))
+    assert e.value.code == -3
+
+
+def test_rowscaled_host_output_path(ep):
+    """Host payload and host scales: the upload-decode-download path gives the device path's bytes."""
+    m = W.square(rows=256, cols=1024)
+    c = ep.compress(W.bits_to_torch(m.bits, m.dtype), m.target_bpp)
+    pay, sig = _gpu(ep, c)
+    hp = torch.empty(c.shape, dtype=torch.float8_e4m3fn).pin_memory()
+    hs = torch.empty(c.shape[0], dtype=torch.float32)
+    ep.decompress_fp8_rowscaled(c, out=hp, row_scale=hs)
+    assert np.array_equal(hp.view(torch.uint8).numpy(), pay) and np.array_equal(hs.numpy(), sig)

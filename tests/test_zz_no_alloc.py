@@ -8,8 +8,9 @@ in a fixed array inside the library instead of allocating one.
 
 This file checks that entry point against the ordinary ep_decompress on the same blob, bit for
 bit (the tolerance the parity tests use), on two calls in a row, for every kernel variant it can
-launch: vector and element stores, blobs with and without escape symbols, and each output
-container.  It also checks that the two calls leave the device's free memory unchanged, that a
+launch: vector and element stores, blobs with and without escape symbols, each output container
+and both frequency-total widths.  It also checks that the two calls leave the device's free memory
+unchanged (after a first call has let the driver load the kernel variant), that a
 corrupt tile is reported and the next clean call is not, and that a device buffer shorter than
 the blob is refused.  It is named so that pytest collects it after every other test file.
 """
@@ -52,7 +53,10 @@ def _noalloc(ep, comp, dev_blob, out, wait=1, nbytes=None):
 
 
 def _two_calls_match(ep, comp, out_dtype, make_out):
-    """Two allocation-free decodes in a row equal ep_decompress, with free memory unchanged."""
+    """Two allocation-free decodes in a row equal ep_decompress, with free memory unchanged.
+    One call comes first, unchecked: the first launch of a kernel variant lets the CUDA driver
+    load that kernel's code (lazy module loading), which can take device memory -- the driver's,
+    not the library's -- so the memory check starts after it."""
     ref = make_out()
     ep.decompress(comp, out=ref)
     torch.cuda.synchronize()
@@ -62,6 +66,8 @@ def _two_calls_match(ep, comp, out_dtype, make_out):
     outs = [make_out() for _ in range(2)]
     for o in outs:
         o.view(torch.uint8).fill_(0x7F)
+    warm = make_out()
+    assert _noalloc(ep, comp, dev_blob, warm) == 0, ep.lib().ep_last_error()
     torch.cuda.synchronize()
     free_before, _ = torch.cuda.mem_get_info()
     for o in outs:
