@@ -42,11 +42,12 @@ const Launchers* launchers_for(int out_kind) {
 int launch(const Params& p, int out_kind, const BlobLayout& L, bool vec, const Ctl& ctl, cudaStream_t st, int device,
            bool dependent) {
     const LaunchCtx c{device, g_dev[device].sms};
-    const bool wide = L.max_tile_bytes <= tile_buffer_bytes(kWarpsWide, L.prob_bits) &&
+    const int lay = table_layout(L.prob_bits, L.max_tile_bytes);
+    const bool wide = lay != 13 && L.max_tile_bytes <= tile_buffer_bytes(kWarpsWide, lay) &&
                       p.n_tiles > uint32_t(kWarpsNarrow) * uint32_t(c.sms);
     const Launchers* ln = launchers_for(out_kind);
     if (!ln) return set_error(EP_ERR_DTYPE, "decode: unsupported output container");
-    return ln->single(p, L.prob_bits, vec, wide, L.has_escape != 0, ctl, st, c, dependent);
+    return ln->single(p, lay, vec, wide, L.has_escape != 0, ctl, st, c, dependent);
 }
 
 // Share `ctas` CTAs among blobs with tiles[i] tiles: every blob gets one, then each further CTA
@@ -138,8 +139,8 @@ int ensure_device(ep_blob* b, int dev, cudaStream_t st) {
     uint8_t* blob = nullptr;
     uint8_t* tables = nullptr;
     uint32_t* status = nullptr;
-    const int pb = b->layout.prob_bits;
-    if (cudaMalloc(&blob, b->bytes.size()) != cudaSuccess || cudaMalloc(&tables, table_bytes(pb)) != cudaSuccess ||
+    const int lay = table_layout(b->layout.prob_bits, b->layout.max_tile_bytes);
+    if (cudaMalloc(&blob, b->bytes.size()) != cudaSuccess || cudaMalloc(&tables, table_bytes(lay)) != cudaSuccess ||
         cudaMalloc(&status, 16) != cudaSuccess) {
         cudaFree(blob);
         cudaFree(tables);
@@ -151,8 +152,9 @@ int ensure_device(ep_blob* b, int dev, cudaStream_t st) {
     EP_CUDA(cudaMemsetAsync(status, 0, 16, st), "status clear");
     // expand the compact frequency tables once for this device copy
     const TableSrc ts = make_tablesrc(b, blob);
-    auto fn = pb == 10 ? expand_tables_kernel<kWarpsWide, 10> : expand_tables_kernel<kWarpsWide, 12>;
-    const size_t smem = pb == 10 ? sizeof(ExpandSmem<10>) : sizeof(ExpandSmem<12>);
+    auto fn = lay == 10 ? expand_tables_kernel<kWarpsWide, 10>
+                        : lay == 12 ? expand_tables_kernel<kWarpsWide, 12> : expand_tables_kernel<kWarpsWide, 13>;
+    const size_t smem = lay == 10 ? sizeof(ExpandSmem<10>) : lay == 12 ? sizeof(ExpandSmem<12>) : sizeof(ExpandSmem<13>);
     EP_CUDA(cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, int(smem)),
             "table expansion attribute");
     fn<<<1, kWarpsWide * 32, smem, st>>>(ts, tables);
@@ -303,11 +305,11 @@ extern "C" int ep_decompress_group(const ep_blob* const* blobs, const ep_tensor*
     }
     const int sms = g_dev[dev].sms;
     const int chunk = std::max(1, std::min(kMaxGroup, sms));
-    // one launch per chunk of blobs that share a frequency-total width
-    for (int pb : {12, 10}) {
+    // one launch per chunk of blobs that share a table layout
+    for (int lay : {13, 12, 10}) {
         std::vector<int> idx;
         for (int i = 0; i < n; ++i)
-            if (blobs[i]->layout.prob_bits == pb) idx.push_back(i);
+            if (table_layout(blobs[i]->layout.prob_bits, blobs[i]->layout.max_tile_bytes) == lay) idx.push_back(i);
         for (size_t c0 = 0; c0 < idx.size(); c0 += size_t(chunk)) {
             const int cn = int(std::min(size_t(chunk), idx.size() - c0));
             std::vector<uint32_t> tiles(static_cast<size_t>(cn));
@@ -335,9 +337,9 @@ extern "C" int ep_decompress_group(const ep_blob* const* blobs, const ep_tensor*
                 e.esc = b->layout.has_escape ? 1u : 0u;
                 cta += e.ncta;
             }
-            const bool wide = max_tile <= tile_buffer_bytes(kWarpsWide, pb) &&
+            const bool wide = lay != 13 && max_tile <= tile_buffer_bytes(kWarpsWide, lay) &&
                               total > uint64_t(kWarpsNarrow) * uint64_t(cta);
-            rc = launchers_for(kind)->group(gp, pb, cta, wide, st, LaunchCtx{dev, sms});
+            rc = launchers_for(kind)->group(gp, lay, cta, wide, st, LaunchCtx{dev, sms});
             if (rc != EP_OK) return rc;
         }
     }
@@ -517,8 +519,8 @@ extern "C" int ep_decompress_noalloc(const ep_blob* cb, const void* device_blob,
     Params p = make_params(cb, static_cast<const uint8_t*>(device_blob), nullptr, out->data, out->row_stride,
                            status);
     const TableSrc ts = make_tablesrc(cb, static_cast<const uint8_t*>(device_blob));
-    int rc = launchers_for(kind)->noalloc(p, ts, L.prob_bits, vec, L.has_escape != 0, st,
-                                          LaunchCtx{dev, g_noalloc[dev].sms});
+    int rc = launchers_for(kind)->noalloc(p, ts, table_layout(L.prob_bits, L.max_tile_bytes), vec,
+                                          L.has_escape != 0, st, LaunchCtx{dev, g_noalloc[dev].sms});
     if (rc != EP_OK || !wait) return rc;
     uint32_t s = 0;
     if (cudaMemcpyAsync(&s, status, sizeof s, cudaMemcpyDeviceToHost, st) != cudaSuccess ||

@@ -14,8 +14,9 @@
 //     {slot - cum(s), s (2 s for f8), escape flag, coset bit, q(s)} -- 60 KB -- so one
 //     shared-memory load per symbol gives everything the state update needs.  With 12-bit totals
 //     the per-slot entries would take 240 KB, more than an SM has, so a symbol takes two loads:
-//     the slot's symbol byte (4096 per table, 60 KB), then that symbol's {cum(s), escape flag,
-//     q(s)} word (16 KB).  The tables are expanded once per blob and device by a small kernel into
+//     the slot's symbol byte (4096 per table, 60 KB), then that symbol's {q(s), -(cum(s) + the
+//     table's byte offset)} pair (32 KB), which turns the state update into one three-input add
+//     and one multiply-add on the slot's shared address.  The tables are expanded once per blob and device by a small kernel into
 //     a block next to the device copy; every CTA stages that block into shared memory with bulk
 //     copies, overlapped with the fetch of its first tiles.  (The allocation-free entry point
 //     expands them inside each CTA instead.);
@@ -76,28 +77,41 @@ constexpr uint32_t kEntryQShift = 21;
 constexpr uint32_t kSlots10 = 1024;
 
 // 12-bit totals.  Symbol byte of slot u of table t at [4096 t + u] (for the joint table the f1
-// symbol of the slot's coset half; the coset is u >= the coset-0 total).  Per-symbol word of
-// table t >= 1 at [kSlotBytes + 1024 (t + 1) + 4 s]; the joint table's at [kSlotBytes + 1024 c +
-// 4 s], its coset-1 cumulative frequencies following all of coset 0's:
-//   bits  0..11  cum(s)
-//   bit  12      s is the escape symbol
-//   bits 16..28  q(s)                 (<= 4096)
-// so the state update x <- q (x >> 12) + (x mod 4096) - cum(s) takes two field extractions.
-constexpr uint32_t kE12CumMask = 0xFFFu;
-constexpr uint32_t kE12Esc = 1u << 12;
-constexpr uint32_t kE12QShift = 16;
+// symbol of the slot's coset half; the coset is u >= the coset-0 total).  Per-symbol entry of
+// table t >= 1 at [kSlotBytes + 2048 (t + 1) + 8 s]; the joint table's at [kSlotBytes + 2048 c +
+// 8 s], its coset-1 cumulative frequencies following all of coset 0's:
+//   word 0  q(s)                      (<= 4096; 0 for a symbol the table does not hold)
+//   word 1  -(cum(s) + 4096 t) mod 2^32
+// With the slot's shared address a = base + 4096 t + u, the state update is
+// x <- q (x >> 12) + (a + word1 - base) = q (x >> 12) + u - cum(s).
 
 // Shared addresses of the decode tables a step reads.
-template <int PB>
+template <int LAY>
 struct Tab {
     uint32_t t;        // 10-bit: the packed entries, 4 KB aligned
 };
 template <>
 struct Tab<12> {
     uint32_t s1;       // symbol bytes, 4 KB aligned
-    uint32_t e2;       // per-symbol words
+    uint32_t e2;       // per-symbol entries
+    uint32_t s1split;  // s1 + the slots of coset 0 in the joint table
+};
+// Layout 13 (12-bit totals, hybrid), at `base` (4 KB aligned): the joint table's direct words at
+// base, f2 and f3 given coset c at base + kHDirect (1 + 2c + j - 2); symbol bytes of f4..f8 given c
+// at base + kHL1 + 4096 (5c + j - 4); their 8-byte entries (as in layout 12, with t = 5c + j - 4)
+// at base + kHL2 + 2048 (5c + j - 4).  A direct word of slot u holding symbol s:
+//   bits  0..11  u - cum(s)
+//   bits 12..19  s
+//   bits 20..31  q(s) - 1
+// so x <- (q - 1) (x >> 12) + (x >> 12) + (u - cum(s)).
+template <>
+struct Tab<13> {
+    uint32_t base;
     uint32_t split;    // slots of coset 0 in the joint table
 };
+__device__ __forceinline__ uint32_t pack_direct(uint32_t off, uint32_t s, uint32_t q) {
+    return q ? off | (s << 12) | ((q - 1) << 20) : 0u;
+}
 
 // Scratch of the table expansion: frequencies and cumulative frequencies of every context.
 struct BuildScratch {
@@ -164,6 +178,12 @@ template <int OFF = 0>
 __device__ __forceinline__ uint32_t lds_u32(uint32_t a) {
     uint32_t v;
     asm volatile("ld.shared.u32 %0, [%1+%2];" : "=r"(v) : "r"(a), "n"(OFF));
+    return v;
+}
+template <int OFF = 0>
+__device__ __forceinline__ uint2 lds_v2(uint32_t a) {
+    uint2 v;
+    asm volatile("ld.shared.v2.u32 {%0, %1}, [%2+%3];" : "=r"(v.x), "=r"(v.y) : "r"(a), "n"(OFF));
     return v;
 }
 // Shared address of slot (x mod M) of a 4 KB-aligned table at `base`: a mask and a multiply-add,
@@ -250,12 +270,73 @@ __device__ __forceinline__ uint32_t pack_entry(uint32_t bias, uint32_t s, uint32
            (coset << kEntryCosetShift) | (q << kEntryQShift);
 }
 
-// Fills the decode tables at `tab` (shared memory, TableGeo<PB>::kBytes) from the blob's compact
+// Layout 13 from the per-context frequencies and cumulative frequencies in `scr`: the 5 direct
+// tables, the 10 symbol-byte tables, then the 8-byte entries of those 10.
+template <int WARPS>
+__device__ void build_hybrid(uint8_t* tab, const BuildScratch& scr) {
+    const uint32_t lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+    constexpr int P = WARPS >= 15 ? WARPS / 15 : 1;
+    constexpr uint32_t kSlotsPerPart = 4096u / P;
+    const uint32_t split = scr.cum[0][256];
+    uint32_t* dir = reinterpret_cast<uint32_t*>(tab);
+    for (uint32_t item = warp; item < uint32_t(15 * P); item += WARPS) {
+        const uint32_t ti = item / P, part = item % P;
+        if (ti == 0) {  // the joint table, direct: coset 0's slots, then coset 1's
+            for (uint32_t w = lane; w < kSlotsPerPart; w += 32) {
+                const uint32_t slot = part * kSlotsPerPart + w;
+                const uint32_t c = slot < split ? 0u : 1u;
+                const uint32_t local = slot - (c ? split : 0u);
+                const uint16_t* cum = scr.cum[8 * c];
+                const uint32_t sy = slot_symbol(cum, local);
+                dir[slot] = pack_direct(local - cum[sy], sy, scr.q[8 * c][sy]);
+            }
+            continue;
+        }
+        // ti 1..4: f2, f3 given c (direct); ti 5..14: f4..f8 given c (symbol bytes)
+        const bool direct = ti < 5;
+        const uint32_t c = direct ? (ti - 1) / 2 : (ti - 5) / 5;
+        const uint32_t j = direct ? 2 + (ti - 1) % 2 : 4 + (ti - 5) % 5;
+        const uint32_t ctx = 8 * c + j - 1;
+        const uint16_t* cum = scr.cum[ctx];
+        const uint16_t* qs = scr.q[ctx];
+        uint32_t* dst32 = direct ? dir + ti * 4096u : nullptr;
+        uint8_t* dst8 = direct ? nullptr : tab + kHL1 + (ti - 5) * kCtxBytes;
+        if (cum[256] != 4096u) {  // context never used by this blob (the host checked the rest)
+            for (uint32_t w = lane; w < kSlotsPerPart; w += 32) {
+                if (direct) dst32[part * kSlotsPerPart + w] = 0;
+                else dst8[part * kSlotsPerPart + w] = 0;
+            }
+            continue;
+        }
+        const uint32_t first = part * kSlotsPerPart + lane;
+        uint32_t sy = slot_symbol(cum, first);
+        uint32_t c0 = cum[sy], next = cum[sy + 1];
+        for (uint32_t w = lane; w < kSlotsPerPart; w += 32) {
+            const uint32_t slot = part * kSlotsPerPart + w;
+            while (next <= slot) {
+                ++sy;
+                c0 = next;
+                next = cum[sy + 1];
+            }
+            if (direct) dst32[slot] = pack_direct(slot - c0, sy, qs[sy]);
+            else dst8[slot] = uint8_t(sy);
+        }
+    }
+    uint2* ent = reinterpret_cast<uint2*>(tab + kHL2);
+    for (uint32_t i = threadIdx.x; i < 10 * 256; i += WARPS * 32) {
+        const uint32_t row = i >> 8, sy = i & 255;
+        const uint32_t ctx = 8 * (row / 5) + 3 + row % 5;  // f4..f8 given coset row / 5
+        const uint32_t q = scr.q[ctx][sy];
+        ent[i] = q ? make_uint2(q, 0u - (uint32_t(scr.cum[ctx][sy]) + kCtxBytes * row)) : make_uint2(0u, 0u);
+    }
+}
+
+// Fills the decode tables at `tab` (shared memory, TableGeo<LAY>::kBytes) from the blob's compact
 // frequency tables (16 contexts; 0 and 8 together are the joint (coset, f1) table).  `scr` is
 // shared-memory scratch (BuildScratch) that the caller does not use meanwhile.
-template <int WARPS, int PB>
+template <int WARPS, int LAY>
 __device__ void build_tables(uint8_t* tab, BuildScratch& scr, const TableSrc& p) {
-    constexpr uint32_t M = 1u << PB;
+    constexpr uint32_t M = LAY == 10 ? 1024u : 4096u;
     const uint32_t lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
     // (a) per context: frequencies of symbols 8*lane .. 8*lane+7 and their cumulative sums
     for (uint32_t ctx = warp; ctx < kFieldContexts; ctx += WARPS) {
@@ -286,6 +367,10 @@ __device__ void build_tables(uint8_t* tab, BuildScratch& scr, const TableSrc& p)
         if (lane == 31) scr.cum[ctx][256] = uint16_t(min(c, 0xFFFFu));
     }
     __syncthreads();
+    if constexpr (LAY == 13) {
+        build_hybrid<WARPS>(tab, scr);
+        return;
+    }
     // (b) slot -> entry (10-bit: the packed word; 12-bit: the symbol byte).  Lane l of a warp
     // writes slots it*32 + l of its part (one contiguous run per store instruction); each lane
     // walks its symbol forward as its slots grow.
@@ -294,7 +379,7 @@ __device__ void build_tables(uint8_t* tab, BuildScratch& scr, const TableSrc& p)
     static_assert(M % P == 0, "parts split the slots evenly");
     uint32_t* tab32 = reinterpret_cast<uint32_t*>(tab);
     auto put = [&](uint32_t ti, uint32_t slot, uint32_t bias, uint32_t sy, uint32_t q, uint32_t coset, uint32_t sh) {
-        if constexpr (PB == 10) tab32[ti * kSlots10 + slot] = pack_entry(bias, sy, q, coset, sh);
+        if constexpr (LAY == 10) tab32[ti * kSlots10 + slot] = pack_entry(bias, sy, q, coset, sh);
         else tab[ti * kCtxBytes + slot] = uint8_t(sy);
     };
     for (uint32_t item = warp; item < uint32_t(kDecodeTables * P); item += WARPS) {
@@ -332,17 +417,18 @@ __device__ void build_tables(uint8_t* tab, BuildScratch& scr, const TableSrc& p)
             put(ti, slot, slot - c0, sy, qs[sy], 0u, sh);
         }
     }
-    if constexpr (PB == 12) {
-        // (c) the per-symbol words: row 0/1 the joint table's coset halves (coset 1's cumulative
-        // frequencies after coset 0's), row t + 1 table t >= 1
-        uint32_t* ent = reinterpret_cast<uint32_t*>(tab + kSlotBytes);
+    if constexpr (LAY == 12) {
+        // (c) the per-symbol entries: row 0/1 the joint table's coset halves (table 0; coset 1's
+        // cumulative frequencies after coset 0's), row t + 1 table t >= 1
+        uint2* ent = reinterpret_cast<uint2*>(tab + kSlotBytes);
         const uint32_t split = scr.cum[0][256];
         for (uint32_t i = threadIdx.x; i < 16 * 256; i += WARPS * 32) {
             const uint32_t row = i >> 8, sy = i & 255;
             const uint32_t ctx = row == 0 ? 0u : row == 1 ? 8u : 8 * ((row - 2) / 7) + 1 + (row - 2) % 7;
+            const uint32_t t = row < 2 ? 0u : row - 1;
             const uint32_t q = scr.q[ctx][sy];
             const uint32_t cum = scr.cum[ctx][sy] + (row == 1 ? split : 0u);
-            ent[i] = q ? ((q << kE12QShift) | (sy == uint32_t(kEscape) ? kE12Esc : 0u) | (cum & kE12CumMask)) : 0u;
+            ent[i] = q ? make_uint2(q, 0u - (cum + kCtxBytes * t)) : make_uint2(0u, 0u);
         }
     }
 }
@@ -542,37 +628,39 @@ __device__ __forceinline__ void step_symbols10(uint32_t tab, Reader& rd, uint32_
     }
 }
 
-// The same with 12-bit totals: per symbol the slot's symbol byte, then that symbol's word.  s.e[j]
-// holds the symbol s_j itself.
+// The same with 12-bit totals: per symbol the slot's symbol byte, then that symbol's entry.
+// s.e[j] holds the symbol s_j itself.
 template <bool ESC, bool FULL, class Reader>
 __device__ __forceinline__ void step_symbols12(const Tab<12>& T, Reader& rd, uint32_t& x, bool active, StepSyms& s) {
     if (FULL) active = true;
     uint32_t* e = s.e;
-    uint32_t acc = 0;
+    uint32_t acc = 0;                          // largest symbol: the escape symbol is the largest
+    const uint32_t ks = 0u - T.s1;             // (base of the symbol bytes, negated)
     // (coset, f1): the slot's half of the joint table gives the coset (known before the loads
     // return), its byte the f1 symbol.  A lane past the last vector still loads but keeps x.
-    uint32_t slot = x & 4095u;
-    const uint32_t c = slot >= T.split ? 1u : 0u;
+    uint32_t c;
     {
-        const uint32_t sy = lds_u8<0>(T.s1 + slot);
-        const uint32_t en = lds_u32<0>(T.e2 + 1024u * c + 4u * sy);
-        if (active) x = (en >> kE12QShift) * (x >> 12) + slot - (en & kE12CumMask);
+        const uint32_t a1 = (x & 4095u) | T.s1;
+        c = a1 >= T.s1split ? 1u : 0u;
+        const uint32_t sy = lds_u8<0>(a1);
+        const uint2 en = lds_v2<0>(T.e2 + 2048u * c + 8u * sy);
+        if (active) x = en.x * (x >> 12) + (a1 + en.y + ks);
         renorm_step<FULL>(x, rd, active);
         e[0] = sy;
-        if (ESC) acc = en;
+        if (ESC) acc = sy;
     }
     s.c = c;
     const uint32_t b1 = T.s1 + kCtxBytes + c * (7u * kCtxBytes);  // field 2's symbol bytes given c
-    const uint32_t b2 = T.e2 + 2048u + c * (7u * 1024u);           // field 2's words given c
+    const uint32_t b2 = T.e2 + 4096u + c * (7u * 2048u);           // field 2's entries given c
 #define EP_FIELD12(j)                                                                         \
     {                                                                                         \
-        slot = x & 4095u;                                                                     \
-        const uint32_t sy = lds_u8<((j) - 1) * kCtxBytes>(b1 + slot);                         \
-        const uint32_t en = lds_u32<((j) - 1) * 1024>(b2 + 4u * sy);                          \
-        if (active) x = (en >> kE12QShift) * (x >> 12) + slot - (en & kE12CumMask);            \
+        const uint32_t a1 = (x & 4095u) | b1;                                                 \
+        const uint32_t sy = lds_u8<((j) - 1) * kCtxBytes>(a1);                                \
+        const uint2 en = lds_v2<((j) - 1) * 2048>(b2 + 8u * sy);                              \
+        if (active) x = en.x * (x >> 12) + (a1 + en.y + (ks + ((j) - 1) * kCtxBytes));         \
         renorm_step<FULL>(x, rd, active);                                                     \
         e[j] = sy;                                                                            \
-        if (ESC) acc |= en;                                                                   \
+        if (ESC) acc = max(acc, sy);                                                          \
     }
     EP_FIELD12(1) EP_FIELD12(2) EP_FIELD12(3) EP_FIELD12(4) EP_FIELD12(5) EP_FIELD12(6) EP_FIELD12(7)
 #undef EP_FIELD12
@@ -582,7 +670,7 @@ __device__ __forceinline__ void step_symbols12(const Tab<12>& T, Reader& rd, uin
 #pragma unroll
         for (int j = 0; j < 8; ++j) s.f[j] = 0;
     }
-    if (ESC && __any_sync(kFull, active && (acc & kE12Esc))) {
+    if (ESC && __any_sync(kFull, active && acc == uint32_t(kEscape))) {
         // escaped fields: the lane's raw words after its renormalisation words, by field
 #pragma unroll
         for (int j = 0; j < 8; ++j) {
@@ -594,20 +682,71 @@ __device__ __forceinline__ void step_symbols12(const Tab<12>& T, Reader& rd, uin
     }
 }
 
-template <int PB, bool ESC, bool FULL, class Reader>
-__device__ __forceinline__ void step_symbols(const Tab<PB>& tab, Reader& rd, uint32_t& x, bool active, StepSyms& s) {
-    if constexpr (PB == 10) step_symbols10<ESC, FULL>(tab.t, rd, x, active, s);
-    else step_symbols12<ESC, FULL>(tab, rd, x, active, s);
+// Layout 13: (coset, f1), f2 and f3 from direct words (one load each), f4..f8 as in layout 12.
+template <bool ESC, bool FULL, class Reader>
+__device__ __forceinline__ void step_symbols13(const Tab<13>& T, Reader& rd, uint32_t& x, bool active, StepSyms& s) {
+    if (FULL) active = true;
+    uint32_t* e = s.e;
+    uint32_t acc = 0;                          // largest symbol: the escape symbol is the largest
+    // a direct word's state update; returns the symbol
+    auto direct = [&](uint32_t w) {
+        const uint32_t h = x >> 12;
+        if (active) x = (w >> 20) * h + (h + (w & 4095u));
+        return (w >> 12) & 255u;
+    };
+    uint32_t c;
+    {
+        const uint32_t slot = x & 4095u;
+        c = slot >= T.split ? 1u : 0u;
+        const uint32_t sy = direct(lds_u32<0>(T.base + 4u * slot));
+        renorm_step<FULL>(x, rd, active);
+        e[0] = sy;
+        if (ESC) acc = sy;
+    }
+    s.c = c;
+    const uint32_t bd = T.base + kHDirect + c * (2u * kHDirect);   // f2 given c; f3 follows
+#define EP_FIELD13D(j)                                                                            {                                                                                                 const uint32_t sy = direct(lds_u32<((j) - 1) * kHDirect>(bd + 4u * (x & 4095u)));             renorm_step<FULL>(x, rd, active);                                                             e[j] = sy;                                                                                    if (ESC) acc = max(acc, sy);                                                              }
+    EP_FIELD13D(1) EP_FIELD13D(2)
+#undef EP_FIELD13D
+    const uint32_t b1 = T.base + kHL1 + c * (5u * kCtxBytes);      // f4's symbol bytes given c
+    const uint32_t b2 = T.base + kHL2 + c * (5u * 2048u);          // f4's entries given c
+    const uint32_t ks = 0u - (T.base + kHL1);
+#define EP_FIELD13(j)                                                                             {                                                                                                 const uint32_t a1 = (x & 4095u) | b1;                                                         const uint32_t sy = lds_u8<((j) - 3) * kCtxBytes>(a1);                                        const uint2 en = lds_v2<((j) - 3) * 2048>(b2 + 8u * sy);                                      if (active) x = en.x * (x >> 12) + (a1 + en.y + (ks + ((j) - 3) * kCtxBytes));                 renorm_step<FULL>(x, rd, active);                                                             e[j] = sy;                                                                                    if (ESC) acc = max(acc, sy);                                                              }
+    EP_FIELD13(3) EP_FIELD13(4) EP_FIELD13(5) EP_FIELD13(6) EP_FIELD13(7)
+#undef EP_FIELD13
+
+    s.from_symbols = true;
+    if constexpr (ESC) {
+#pragma unroll
+        for (int j = 0; j < 8; ++j) s.f[j] = 0;
+    }
+    if (ESC && __any_sync(kFull, active && acc == uint32_t(kEscape))) {
+        // escaped fields: the lane's raw words after its renormalisation words, by field
+#pragma unroll
+        for (int j = 0; j < 8; ++j) {
+            const bool mine = active && e[j] == uint32_t(kEscape);
+            s.f[j] = mine ? int32_t(int16_t(rd.wn)) : int32_t(e[j]) - kAlphabetR;
+            rd.consume_if(mine);
+        }
+        s.from_symbols = false;
+    }
+}
+
+template <int LAY, bool ESC, bool FULL, class Reader>
+__device__ __forceinline__ void step_symbols(const Tab<LAY>& tab, Reader& rd, uint32_t& x, bool active, StepSyms& s) {
+    if constexpr (LAY == 10) step_symbols10<ESC, FULL>(tab.t, rd, x, active, s);
+    else if constexpr (LAY == 12) step_symbols12<ESC, FULL>(tab, rd, x, active, s);
+    else step_symbols13<ESC, FULL>(tab, rd, x, active, s);
 }
 
 // Symbol s_j of a decoded step (entry layout of the total).
-template <int PB>
+template <int LAY>
 __device__ __forceinline__ uint32_t sym_of(uint32_t e, int j) {
-    if constexpr (PB == 10) return (e >> (kEntrySymShift + (j == 7))) & 255u;
+    if constexpr (LAY == 10) return (e >> (kEntrySymShift + (j == 7))) & 255u;
     else return e;
 }
 
-template <int OUT, bool VEC, bool ESC, int PB>
+template <int OUT, bool VEC, bool ESC, int LAY>
 __device__ __forceinline__ void step_emit(const Params& p, const StepSyms& s, const Pos& pos) {
     const uint32_t* e = s.e;
     const uint32_t c = s.c;
@@ -620,7 +759,7 @@ __device__ __forceinline__ void step_emit(const Params& p, const StepSyms& s, co
         o[0] = int16_t(c);
 #pragma unroll
         for (int j = 0; j < 8; ++j)
-            o[1 + j] = int16_t(from_symbols ? int32_t(sym_of<PB>(e[j], j)) - kAlphabetR : f[j]);
+            o[1 + j] = int16_t(from_symbols ? int32_t(sym_of<LAY>(e[j], j)) - kAlphabetR : f[j]);
         return;
     } else {
         // y_j = z_j + c/2, the lattice coordinate (z1..z7 = f1..f7, z8 = 2 f8 + parity of z1..z7),
@@ -653,9 +792,9 @@ __device__ __forceinline__ void step_emit(const Params& p, const StepSyms& s, co
             const uint32_t km = kMagic | (c << 9);
 #pragma unroll
             for (int j = 0; j < 7; ++j)
-                t[j] = PB == 10 ? (e[j] & (0xFFu << kEntrySymShift)) | km : e[j] * 1024u + km;
+                t[j] = LAY == 10 ? (e[j] & (0xFFu << kEntrySymShift)) | km : e[j] * 1024u + km;
             const uint32_t px = t[0] ^ t[1] ^ t[2] ^ t[3] ^ t[4] ^ t[5] ^ t[6];
-            t[7] = (PB == 10 ? (e[7] & (0xFFu << (kEntrySymShift + 1))) | km : e[7] * 2048u + km) | (~px & 0x400u);
+            t[7] = (LAY == 10 ? (e[7] & (0xFFu << (kEntrySymShift + 1))) | km : e[7] * 2048u + km) | (~px & 0x400u);
             const float2 k = make_float2(1.0f / 1024, 1.0f / 1024), b = make_float2(-12415.0f, -12415.0f);
             scale(t, k, b, k, make_float2(-12415.0f, -12542.0f));
         } else {
@@ -682,14 +821,14 @@ __device__ __forceinline__ void step_emit(const Params& p, const StepSyms& s, co
 }
 
 
-template <int OUT, bool VEC, bool ESC, int PB, bool FULL, class Reader>
-__device__ __forceinline__ void decode_step(const Params& p, const Tab<PB>& tab, Reader& rd, uint32_t& x, bool active,
+template <int OUT, bool VEC, bool ESC, int LAY, bool FULL, class Reader>
+__device__ __forceinline__ void decode_step(const Params& p, const Tab<LAY>& tab, Reader& rd, uint32_t& x, bool active,
                                             const Pos& pos) {
     if (FULL) active = true;
     StepSyms s;
-    step_symbols<PB, ESC, FULL>(tab, rd, x, active, s);
+    step_symbols<LAY, ESC, FULL>(tab, rd, x, active, s);
     if (!active) return;
-    step_emit<OUT, VEC, ESC, PB>(p, s, pos);
+    step_emit<OUT, VEC, ESC, LAY>(p, s, pos);
 }
 
 // Decode `n` full steps, two between runaway checks (the tile buffer's slack covers what two
@@ -697,21 +836,21 @@ __device__ __forceinline__ void decode_step(const Params& p, const Tab<PB>& tab,
 // Escape-free blobs are software-pipelined: the symbols of step k + 1 are decoded before step k
 // is written (blobs with escapes keep one step at a time, whose raw-field path would otherwise
 // hold two steps' fields in registers).
-template <int OUT, bool VEC, bool ESC, int PB, class Reader, class Guard, class Step>
-__device__ __forceinline__ uint32_t full_run(const Params& p, const Tab<PB>& tab, Reader& rd, uint32_t& x, Pos& pos,
+template <int OUT, bool VEC, bool ESC, int LAY, class Reader, class Guard, class Step>
+__device__ __forceinline__ uint32_t full_run(const Params& p, const Tab<LAY>& tab, Reader& rd, uint32_t& x, Pos& pos,
                                              uint32_t n, Guard in_range, Step walk) {
     if constexpr (ESC) {
         uint32_t k = 0;
         for (; k + 2 <= n; k += 2) {
             if (!__all_sync(kFull, in_range(rd))) return kStOverrun;  // a corrupt tile ran away
-            decode_step<OUT, VEC, ESC, PB, true>(p, tab, rd, x, true, pos);
+            decode_step<OUT, VEC, ESC, LAY, true>(p, tab, rd, x, true, pos);
             walk(pos);
-            decode_step<OUT, VEC, ESC, PB, true>(p, tab, rd, x, true, pos);
+            decode_step<OUT, VEC, ESC, LAY, true>(p, tab, rd, x, true, pos);
             walk(pos);
         }
         if (k < n) {
             if (!__all_sync(kFull, in_range(rd))) return kStOverrun;
-            decode_step<OUT, VEC, ESC, PB, true>(p, tab, rd, x, true, pos);
+            decode_step<OUT, VEC, ESC, LAY, true>(p, tab, rd, x, true, pos);
             walk(pos);
         }
         return 0;
@@ -719,35 +858,35 @@ __device__ __forceinline__ uint32_t full_run(const Params& p, const Tab<PB>& tab
     if (n == 0) return 0;
     StepSyms a, b;
     if (!__all_sync(kFull, in_range(rd))) return kStOverrun;
-    step_symbols<PB, ESC, true>(tab, rd, x, true, a);
+    step_symbols<LAY, ESC, true>(tab, rd, x, true, a);
     uint32_t k = 1;
     for (; k + 2 <= n; k += 2) {
         if (!__all_sync(kFull, in_range(rd))) return kStOverrun;  // a corrupt tile ran away
-        step_symbols<PB, ESC, true>(tab, rd, x, true, b);
-        step_emit<OUT, VEC, ESC, PB>(p, a, pos);
+        step_symbols<LAY, ESC, true>(tab, rd, x, true, b);
+        step_emit<OUT, VEC, ESC, LAY>(p, a, pos);
         walk(pos);
-        step_symbols<PB, ESC, true>(tab, rd, x, true, a);
-        step_emit<OUT, VEC, ESC, PB>(p, b, pos);
+        step_symbols<LAY, ESC, true>(tab, rd, x, true, a);
+        step_emit<OUT, VEC, ESC, LAY>(p, b, pos);
         walk(pos);
     }
     if (k < n) {
         if (!__all_sync(kFull, in_range(rd))) return kStOverrun;
-        step_symbols<PB, ESC, true>(tab, rd, x, true, b);
-        step_emit<OUT, VEC, ESC, PB>(p, a, pos);
+        step_symbols<LAY, ESC, true>(tab, rd, x, true, b);
+        step_emit<OUT, VEC, ESC, LAY>(p, a, pos);
         walk(pos);
         a = b;
     }
-    step_emit<OUT, VEC, ESC, PB>(p, a, pos);
+    step_emit<OUT, VEC, ESC, LAY>(p, a, pos);
     walk(pos);
     return 0;
     }
 }
 
-template <int OUT, bool VEC, bool ESC, int PB, int WALK, class Reader, class Guard>
-__device__ __forceinline__ uint32_t full_steps(const Params& p, const Tab<PB>& tab, Reader& rd, uint32_t& x, Pos& pos,
+template <int OUT, bool VEC, bool ESC, int LAY, int WALK, class Reader, class Guard>
+__device__ __forceinline__ uint32_t full_steps(const Params& p, const Tab<LAY>& tab, Reader& rd, uint32_t& x, Pos& pos,
                                                uint32_t nfull, Guard in_range) {
     if constexpr (OUT == kOutFields) {
-        return full_run<OUT, VEC, ESC, PB>(p, tab, rd, x, pos, nfull, in_range, [](Pos& s) { s.optr += 32 * 18; });
+        return full_run<OUT, VEC, ESC, LAY>(p, tab, rd, x, pos, nfull, in_range, [](Pos& s) { s.optr += 32 * 18; });
     } else if constexpr (WALK == kWalkRows32) {
         constexpr int es = OutElem<OUT>::kBytes;
         const uint32_t per_row = p.vec_per_row / kLanes;
@@ -757,7 +896,7 @@ __device__ __forceinline__ uint32_t full_steps(const Params& p, const Tab<PB>& t
             // short rows: one run over the whole tile (the step pipeline does not restart at every
             // row), the row change a warp-uniform branch in the walk
             float a_next = pos.row + 1 < p.rows ? row_factor<OUT>(p, pos.row + 1) : 0.0f;
-            return full_run<OUT, VEC, ESC, PB>(p, tab, rd, x, pos, nfull, in_range, [&](Pos& s) {
+            return full_run<OUT, VEC, ESC, LAY>(p, tab, rd, x, pos, nfull, in_range, [&](Pos& s) {
                 s.optr += 32 * 8 * es;
                 if (--left == 0) {
                     left = per_row;
@@ -773,7 +912,7 @@ __device__ __forceinline__ uint32_t full_steps(const Params& p, const Tab<PB>& t
             const uint32_t n = min(left, nfull - k);
             const float a_next = pos.row + 1 < p.rows ? row_factor<OUT>(p, pos.row + 1) : 0.0f;
             const uint32_t st =
-                full_run<OUT, VEC, ESC, PB>(p, tab, rd, x, pos, n, in_range, [](Pos& s) { s.optr += 32 * 8 * es; });
+                full_run<OUT, VEC, ESC, LAY>(p, tab, rd, x, pos, n, in_range, [](Pos& s) { s.optr += 32 * 8 * es; });
             if (st) return st;
             k += n;
             left -= n;
@@ -786,7 +925,7 @@ __device__ __forceinline__ uint32_t full_steps(const Params& p, const Tab<PB>& t
         }
         return 0;
     } else {
-        return full_run<OUT, VEC, ESC, PB>(p, tab, rd, x, pos, nfull, in_range,
+        return full_run<OUT, VEC, ESC, LAY>(p, tab, rd, x, pos, nfull, in_range,
                                        [&p](Pos& s) { advance<OUT, WALK == kWalkWide>(p, s); });
     }
 }
@@ -794,8 +933,8 @@ __device__ __forceinline__ uint32_t full_steps(const Params& p, const Tab<PB>& t
 // Decode the steps of one tile with a given word reader; returns the status flags of the tile.
 // `pos` is the lane's first vector of the tile (first_pos), found by the caller before the tile's
 // words arrived.
-template <int OUT, bool VEC, bool ESC, int PB, class Reader, class Guard>
-__device__ __forceinline__ uint32_t decode_tile_steps(const Params& p, const Tab<PB>& tab, Reader& rd, uint32_t& x,
+template <int OUT, bool VEC, bool ESC, int LAY, class Reader, class Guard>
+__device__ __forceinline__ uint32_t decode_tile_steps(const Params& p, const Tab<LAY>& tab, Reader& rd, uint32_t& x,
                                                       uint32_t tile, uint32_t lane, Pos pos, Guard in_range) {
     const int64_t per_tile = int64_t(kLanes) * p.steps;
     const int64_t v0 = int64_t(tile) * per_tile;
@@ -803,16 +942,16 @@ __device__ __forceinline__ uint32_t decode_tile_steps(const Params& p, const Tab
     const uint32_t nfull = nv / kLanes, rem = nv % kLanes;
     uint32_t st;
     if (VEC && OUT != kOutFields && p.vec_per_row % kLanes == 0)
-        st = full_steps<OUT, VEC, ESC, PB, (VEC && OUT != kOutFields) ? kWalkRows32 : kWalkWide>(p, tab, rd, x, pos, nfull,
+        st = full_steps<OUT, VEC, ESC, LAY, (VEC && OUT != kOutFields) ? kWalkRows32 : kWalkWide>(p, tab, rd, x, pos, nfull,
                                                                                             in_range);
     else if (p.vec_per_row >= uint32_t(kLanes))
-        st = full_steps<OUT, VEC, ESC, PB, kWalkWide>(p, tab, rd, x, pos, nfull, in_range);
+        st = full_steps<OUT, VEC, ESC, LAY, kWalkWide>(p, tab, rd, x, pos, nfull, in_range);
     else
-        st = full_steps<OUT, VEC, ESC, PB, kWalkNarrow>(p, tab, rd, x, pos, nfull, in_range);
+        st = full_steps<OUT, VEC, ESC, LAY, kWalkNarrow>(p, tab, rd, x, pos, nfull, in_range);
     if (st) return st;
     if (rem) {
         if (!__all_sync(kFull, in_range(rd))) return kStOverrun;
-        decode_step<OUT, VEC, ESC, PB, false>(p, tab, rd, x, lane < rem, pos);
+        decode_step<OUT, VEC, ESC, LAY, false>(p, tab, rd, x, lane < rem, pos);
     }
     return 0;
 }
@@ -820,19 +959,19 @@ __device__ __forceinline__ uint32_t decode_tile_steps(const Params& p, const Tab
 // The CTA's layout inside its dynamic shared memory: shifted so that the table (and so every
 // context's 4 KB sub-table) starts on a 4 KB boundary of the shared window, which makes a
 // table address one OR of the slot into the sub-table's base.
-template <int WARPS, int PB>
-__device__ __forceinline__ Smem<WARPS, PB>& smem_layout(uint8_t* raw) {
+template <int WARPS, int LAY>
+__device__ __forceinline__ Smem<WARPS, LAY>& smem_layout(uint8_t* raw) {
     const uint32_t pad = (kAlignSlack - (smem_u32(raw) & (kAlignSlack - 1))) & (kAlignSlack - 1);
-    return *reinterpret_cast<Smem<WARPS, PB>*>(raw + pad);
+    return *reinterpret_cast<Smem<WARPS, LAY>*>(raw + pad);
 }
 
 // The work of CTA `cta` of the `ncta` CTAs that decode one blob.
 // BUILD = false: stage the pre-expanded table from p.tables; true: expand it from `ts` in each CTA.
-template <int WARPS, int OUT, bool VEC, bool BUILD, bool ESC, int PB>
+template <int WARPS, int OUT, bool VEC, bool BUILD, bool ESC, int LAY>
 __device__ __forceinline__ void decode_ctas(const Params& p, const TableSrc* ts, const Ctl& ctl, uint8_t* smem_raw,
                                             uint32_t cta, uint32_t ncta) {
-    Smem<WARPS, PB>& sm = smem_layout<WARPS, PB>(smem_raw);
-    constexpr uint32_t kBuf = Geo<WARPS, PB>::kBuf;
+    Smem<WARPS, LAY>& sm = smem_layout<WARPS, LAY>(smem_raw);
+    constexpr uint32_t kBuf = Geo<WARPS, LAY>::kBuf;
     constexpr uint64_t kMaxTile = 1ull << 22;  // above 160 B + 16 regions of 65535 words
     const uint32_t lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
     const bool fwd = (lane & 1) == 0;  // lanes 2p read forward, lanes 2p+1 backward
@@ -851,9 +990,9 @@ __device__ __forceinline__ void decode_ctas(const Params& p, const TableSrc* ts,
     }
     __syncthreads();  // barriers initialised before anyone uses them
     if (!BUILD && threadIdx.x == 0) {
-        mbar_expect_tx(&sm.tbar, TableGeo<PB>::kBytes);
-        for (uint32_t o = 0; o < TableGeo<PB>::kBytes; o += TableGeo<PB>::kPiece)
-            bulk_g2s(sm.tab + o, p.tables + o, TableGeo<PB>::kPiece, &sm.tbar);
+        mbar_expect_tx(&sm.tbar, TableGeo<LAY>::kBytes);
+        for (uint32_t o = 0; o < TableGeo<LAY>::kBytes; o += TableGeo<LAY>::kPiece)
+            bulk_g2s(sm.tab + o, p.tables + o, TableGeo<LAY>::kPiece, &sm.tbar);
     }
 
     const uint32_t tile_stride = ncta * WARPS;
@@ -891,7 +1030,7 @@ __device__ __forceinline__ void decode_ctas(const Params& p, const TableSrc* ts,
     uint32_t tbytes = 0;
     bool first_ok = false, first_staged = false;
     if (BUILD) {  // expand the table first: its scratch lies in the tile buffers
-        build_tables<WARPS, PB>(sm.tab, *reinterpret_cast<BuildScratch*>(&sm.tbuf[0][0]), *ts);
+        build_tables<WARPS, LAY>(sm.tab, *reinterpret_cast<BuildScratch*>(&sm.tbuf[0][0]), *ts);
         __syncthreads();
     }
     if (tile < p.n_tiles) {  // the first tile's fetch overlaps the table staging
@@ -920,13 +1059,16 @@ __device__ __forceinline__ void decode_ctas(const Params& p, const TableSrc* ts,
             p.sigma[r] = row_sigma(__ldg(p.alpha + r), __ldg(p.rowmax + r));
     }
     {
-        Tab<PB> tab;
-        if constexpr (PB == 10) {
+        Tab<LAY> tab;
+        if constexpr (LAY == 10) {
             tab.t = smem_u32(sm.tab);
+        } else if constexpr (LAY == 13) {
+            tab.base = smem_u32(sm.tab);
+            tab.split = p.joint_split;
         } else {
             tab.s1 = smem_u32(sm.tab);
             tab.e2 = smem_u32(sm.tab + kSlotBytes);
-            tab.split = p.joint_split;
+            tab.s1split = tab.s1 + p.joint_split;
         }
         bool first = true;
         for (; tile < p.n_tiles; tile += tile_stride) {
@@ -981,7 +1123,7 @@ __device__ __forceinline__ void decode_ctas(const Params& p, const TableSrc* ts,
                 rd.wp = buf_a + uint32_t(min(max(o0, 0), int32_t(tbytes) - 2));
                 rd.wn = lds_u16(rd.wp);
                 const uint32_t wp0 = rd.wp, lo = buf_a, hi = buf_a + kBuf;
-                flags = decode_tile_steps<OUT, VEC, ESC, PB>(p, tab, rd, x, tile, lane, pos,
+                flags = decode_tile_steps<OUT, VEC, ESC, LAY>(p, tab, rd, x, tile, lane, pos,
                                                          [=](const SmemReader& r) { return r.wp - lo <= hi - lo; });
                 nread = rd.consumed(wp0);
             } else {
@@ -991,7 +1133,7 @@ __device__ __forceinline__ void decode_ctas(const Params& p, const TableSrc* ts,
                 rd.hi = int32_t(tbytes) - 2;
                 rd.off = o0;
                 rd.wn = __ldg(reinterpret_cast<const uint16_t*>(tg + min(max(o0, 0), rd.hi)));
-                flags = decode_tile_steps<OUT, VEC, ESC, PB>(p, tab, rd, x, tile, lane, pos,
+                flags = decode_tile_steps<OUT, VEC, ESC, LAY>(p, tab, rd, x, tile, lane, pos,
                                                          [](const GlobalReader&) { return true; });
                 nread = rd.consumed(o0);
             }
@@ -1016,17 +1158,17 @@ drain:
 }
 
 // One blob over the whole grid.
-template <int WARPS, int OUT, bool VEC, bool BUILD, bool ESC, int PB>
+template <int WARPS, int OUT, bool VEC, bool BUILD, bool ESC, int LAY>
 __global__ void __launch_bounds__(WARPS * 32, 1) decode_kernel(const __grid_constant__ Params p,
                                                                const __grid_constant__ TableSrc ts,
                                                                const __grid_constant__ Ctl ctl) {
     extern __shared__ __align__(128) uint8_t smem_raw[];
-    decode_ctas<WARPS, OUT, VEC, BUILD, ESC, PB>(p, &ts, ctl, smem_raw, blockIdx.x, gridDim.x);
+    decode_ctas<WARPS, OUT, VEC, BUILD, ESC, LAY>(p, &ts, ctl, smem_raw, blockIdx.x, gridDim.x);
 }
 
-// A set of blobs (all with frequency totals 2^PB) in one launch: blob m owns CTAs
+// A set of blobs (all with frequency totals 2^LAY) in one launch: blob m owns CTAs
 // [cta0, cta0 + ncta) and stages only its own table.  Every blob picks its store and escape variant.
-template <int WARPS, int OUT, int PB>
+template <int WARPS, int OUT, int LAY>
 __global__ void __launch_bounds__(WARPS * 32, 1) group_kernel(const __grid_constant__ GroupParams g) {
     extern __shared__ __align__(128) uint8_t smem_raw[];
     uint32_t m = 0;
@@ -1036,31 +1178,31 @@ __global__ void __launch_bounds__(WARPS * 32, 1) group_kernel(const __grid_const
     const uint32_t cta = blockIdx.x - e.cta0;
     const Ctl ctl;
     if (e.vec) {
-        if (e.esc) decode_ctas<WARPS, OUT, true, false, true, PB>(e.p, nullptr, ctl, smem_raw, cta, e.ncta);
-        else decode_ctas<WARPS, OUT, true, false, false, PB>(e.p, nullptr, ctl, smem_raw, cta, e.ncta);
+        if (e.esc) decode_ctas<WARPS, OUT, true, false, true, LAY>(e.p, nullptr, ctl, smem_raw, cta, e.ncta);
+        else decode_ctas<WARPS, OUT, true, false, false, LAY>(e.p, nullptr, ctl, smem_raw, cta, e.ncta);
     } else {
-        if (e.esc) decode_ctas<WARPS, OUT, false, false, true, PB>(e.p, nullptr, ctl, smem_raw, cta, e.ncta);
-        else decode_ctas<WARPS, OUT, false, false, false, PB>(e.p, nullptr, ctl, smem_raw, cta, e.ncta);
+        if (e.esc) decode_ctas<WARPS, OUT, false, false, true, LAY>(e.p, nullptr, ctl, smem_raw, cta, e.ncta);
+        else decode_ctas<WARPS, OUT, false, false, false, LAY>(e.p, nullptr, ctl, smem_raw, cta, e.ncta);
     }
 }
 
 // Expands the blob's compact frequency tables into the decode tables (one CTA).
-template <int PB>
+template <int LAY>
 struct ExpandSmem {
-    alignas(16) uint8_t tab[TableGeo<PB>::kBytes];
+    alignas(16) uint8_t tab[TableGeo<LAY>::kBytes];
     BuildScratch scratch;
 };
 
-template <int WARPS, int PB>
+template <int WARPS, int LAY>
 __global__ void __launch_bounds__(WARPS * 32, 1) expand_tables_kernel(const __grid_constant__ TableSrc p,
                                                                        uint8_t* tables) {
     extern __shared__ __align__(128) uint8_t smem_raw[];
-    ExpandSmem<PB>& sm = *reinterpret_cast<ExpandSmem<PB>*>(smem_raw);
-    build_tables<WARPS, PB>(sm.tab, sm.scratch, p);
+    ExpandSmem<LAY>& sm = *reinterpret_cast<ExpandSmem<LAY>*>(smem_raw);
+    build_tables<WARPS, LAY>(sm.tab, sm.scratch, p);
     __syncthreads();
     const uint4* s = reinterpret_cast<const uint4*>(sm.tab);
     uint4* d = reinterpret_cast<uint4*>(tables);
-    for (uint32_t i = threadIdx.x; i < TableGeo<PB>::kBytes / 16; i += blockDim.x) d[i] = s[i];
+    for (uint32_t i = threadIdx.x; i < TableGeo<LAY>::kBytes / 16; i += blockDim.x) d[i] = s[i];
 }
 
 // ---- launch functions (host side) ------------------------------------------------------------
@@ -1078,10 +1220,10 @@ int ctas_per_sm(Fn fn, int threads, size_t smem, const LaunchCtx& c, int* cache,
     return cache[c.device];
 }
 
-template <int WARPS, int OUT, bool VEC, bool ESC, int PB>
+template <int WARPS, int OUT, bool VEC, bool ESC, int LAY>
 int launch_one(const Params& p, const Ctl& ctl, cudaStream_t st, const LaunchCtx& c, bool dependent) {
-    auto fn = decode_kernel<WARPS, OUT, VEC, false, ESC, PB>;
-    const size_t smem = sizeof(Smem<WARPS, PB>) + kAlignSlack;
+    auto fn = decode_kernel<WARPS, OUT, VEC, false, ESC, LAY>;
+    const size_t smem = sizeof(Smem<WARPS, LAY>) + kAlignSlack;
     static std::mutex mu;
     static int per_sm[kMaxDevices] = {};
     const int n = ctas_per_sm(fn, WARPS * 32, smem, c, per_sm, mu);
@@ -1106,39 +1248,40 @@ int launch_one(const Params& p, const Ctl& ctl, cudaStream_t st, const LaunchCtx
     return EP_OK;
 }
 
-template <int OUT, bool ESC, int PB>
+template <int OUT, bool ESC, int LAY>
 int launch_width(const Params& p, bool vec, bool wide, const Ctl& ctl, cudaStream_t st, const LaunchCtx& c, bool dep) {
-    if (wide)
-        return vec ? launch_one<kWarpsWide, OUT, true, ESC, PB>(p, ctl, st, c, dep)
-                   : launch_one<kWarpsWide, OUT, false, ESC, PB>(p, ctl, st, c, dep);
-    return vec ? launch_one<kWarpsNarrow, OUT, true, ESC, PB>(p, ctl, st, c, dep)
-               : launch_one<kWarpsNarrow, OUT, false, ESC, PB>(p, ctl, st, c, dep);
+    if (LAY != 13 && wide)
+        return vec ? launch_one<kWarpsWide, OUT, true, ESC, LAY>(p, ctl, st, c, dep)
+                   : launch_one<kWarpsWide, OUT, false, ESC, LAY>(p, ctl, st, c, dep);
+    return vec ? launch_one<kWarpsNarrow, OUT, true, ESC, LAY>(p, ctl, st, c, dep)
+               : launch_one<kWarpsNarrow, OUT, false, ESC, LAY>(p, ctl, st, c, dep);
 }
 
-template <int OUT, int PB>
+template <int OUT, int LAY>
 int launch_esc(const Params& p, bool vec, bool wide, bool esc, const Ctl& ctl, cudaStream_t st, const LaunchCtx& c,
                bool dep) {
     if constexpr (OUT == kOutFields) {  // test hook: the 16-warp kernel has the registers it needs
-        return launch_one<kWarpsNarrow, kOutFields, false, true, PB>(p, ctl, st, c, false);
+        return launch_one<kWarpsNarrow, kOutFields, false, true, LAY>(p, ctl, st, c, false);
     } else {
-        return esc ? launch_width<OUT, true, PB>(p, vec, wide, ctl, st, c, dep)
-                   : launch_width<OUT, false, PB>(p, vec, wide, ctl, st, c, dep);
+        return esc ? launch_width<OUT, true, LAY>(p, vec, wide, ctl, st, c, dep)
+                   : launch_width<OUT, false, LAY>(p, vec, wide, ctl, st, c, dep);
     }
 }
 
 // One blob.  esc: the blob's tables give the escape symbol a frequency (else the escape-free
 // kernel runs).
 template <int OUT>
-int launch_single(const Params& p, int pb, bool vec, bool wide, bool esc, const Ctl& ctl, cudaStream_t st,
+int launch_single(const Params& p, int lay, bool vec, bool wide, bool esc, const Ctl& ctl, cudaStream_t st,
                   const LaunchCtx& c, bool dep) {
-    return pb == 10 ? launch_esc<OUT, 10>(p, vec, wide, esc, ctl, st, c, dep)
-                    : launch_esc<OUT, 12>(p, vec, wide, esc, ctl, st, c, dep);
+    if (lay == 10) return launch_esc<OUT, 10>(p, vec, wide, esc, ctl, st, c, dep);
+    if (lay == 12) return launch_esc<OUT, 12>(p, vec, wide, esc, ctl, st, c, dep);
+    return launch_esc<OUT, 13>(p, vec, false, esc, ctl, st, c, dep);  // 16 warps only
 }
 
-template <int WARPS, int OUT, int PB>
+template <int WARPS, int OUT, int LAY>
 int group_launch_one(const GroupParams& g, uint32_t grid, cudaStream_t st, const LaunchCtx& c) {
-    auto fn = group_kernel<WARPS, OUT, PB>;
-    const size_t smem = sizeof(Smem<WARPS, PB>) + kAlignSlack;
+    auto fn = group_kernel<WARPS, OUT, LAY>;
+    const size_t smem = sizeof(Smem<WARPS, LAY>) + kAlignSlack;
     static std::mutex mu;
     static int per_sm[kMaxDevices] = {};
     if (ctas_per_sm(fn, WARPS * 32, smem, c, per_sm, mu) == 0)
@@ -1161,20 +1304,22 @@ int group_launch_one(const GroupParams& g, uint32_t grid, cudaStream_t st, const
 
 // A set of blobs (one total width pb) over `grid` CTAs.
 template <int OUT>
-int launch_group(const GroupParams& g, int pb, uint32_t grid, bool wide, cudaStream_t st, const LaunchCtx& c) {
-    if (pb == 10)
+int launch_group(const GroupParams& g, int lay, uint32_t grid, bool wide, cudaStream_t st, const LaunchCtx& c) {
+    if (lay == 10)
         return wide ? group_launch_one<kWarpsWide, OUT, 10>(g, grid, st, c)
                     : group_launch_one<kWarpsNarrow, OUT, 10>(g, grid, st, c);
-    return wide ? group_launch_one<kWarpsWide, OUT, 12>(g, grid, st, c)
-                : group_launch_one<kWarpsNarrow, OUT, 12>(g, grid, st, c);
+    if (lay == 12)
+        return wide ? group_launch_one<kWarpsWide, OUT, 12>(g, grid, st, c)
+                    : group_launch_one<kWarpsNarrow, OUT, 12>(g, grid, st, c);
+    return group_launch_one<kWarpsNarrow, OUT, 13>(g, grid, st, c);  // 16 warps only
 }
 
 // The allocation-free decode: tables expanded in every CTA, the status word in caller-provided
 // device memory.  Error messages are static strings (no allocation).
-template <int WARPS, int OUT, bool VEC, bool ESC, int PB>
+template <int WARPS, int OUT, bool VEC, bool ESC, int LAY>
 int noalloc_launch_one(const Params& p, const TableSrc& ts, cudaStream_t st, const LaunchCtx& c) {
-    auto fn = decode_kernel<WARPS, OUT, VEC, true, ESC, PB>;
-    const size_t smem = sizeof(Smem<WARPS, PB>) + kAlignSlack;
+    auto fn = decode_kernel<WARPS, OUT, VEC, true, ESC, LAY>;
+    const size_t smem = sizeof(Smem<WARPS, LAY>) + kAlignSlack;
     static std::mutex mu;
     static int per_sm[kMaxDevices] = {};
     const int n = ctas_per_sm(fn, WARPS * 32, smem, c, per_sm, mu);
@@ -1187,19 +1332,21 @@ int noalloc_launch_one(const Params& p, const TableSrc& ts, cudaStream_t st, con
     return EP_OK;
 }
 
-template <int OUT, int PB>
+template <int OUT, int LAY>
 int noalloc_esc(const Params& p, const TableSrc& ts, bool vec, bool esc, cudaStream_t st, const LaunchCtx& c) {
     if (esc)
-        return vec ? noalloc_launch_one<kWarpsNarrow, OUT, true, true, PB>(p, ts, st, c)
-                   : noalloc_launch_one<kWarpsNarrow, OUT, false, true, PB>(p, ts, st, c);
-    return vec ? noalloc_launch_one<kWarpsNarrow, OUT, true, false, PB>(p, ts, st, c)
-               : noalloc_launch_one<kWarpsNarrow, OUT, false, false, PB>(p, ts, st, c);
+        return vec ? noalloc_launch_one<kWarpsNarrow, OUT, true, true, LAY>(p, ts, st, c)
+                   : noalloc_launch_one<kWarpsNarrow, OUT, false, true, LAY>(p, ts, st, c);
+    return vec ? noalloc_launch_one<kWarpsNarrow, OUT, true, false, LAY>(p, ts, st, c)
+               : noalloc_launch_one<kWarpsNarrow, OUT, false, false, LAY>(p, ts, st, c);
 }
 
 template <int OUT>
-int launch_noalloc(const Params& p, const TableSrc& ts, int pb, bool vec, bool esc, cudaStream_t st,
+int launch_noalloc(const Params& p, const TableSrc& ts, int lay, bool vec, bool esc, cudaStream_t st,
                    const LaunchCtx& c) {
-    return pb == 10 ? noalloc_esc<OUT, 10>(p, ts, vec, esc, st, c) : noalloc_esc<OUT, 12>(p, ts, vec, esc, st, c);
+    if (lay == 10) return noalloc_esc<OUT, 10>(p, ts, vec, esc, st, c);
+    if (lay == 12) return noalloc_esc<OUT, 12>(p, ts, vec, esc, st, c);
+    return noalloc_esc<OUT, 13>(p, ts, vec, esc, st, c);
 }
 
 // The launch table of one output container (each decode_<container>.cu defines one).

@@ -20,19 +20,30 @@ constexpr uint32_t kWaitSpins = 1u << 22;                     // bounded mbarrie
 // Decode tables: [0] the joint (coset, f1) symbol; [1 + 7c + (j - 2)] field j = 2..8 given coset c.
 constexpr int kDecodeTables = 15;
 // 10-bit totals: one packed u32 entry per slot, 1024 slots per table (4 KB), 60 KB in all.
-// 12-bit totals: a u8 symbol per slot, 4096 slots per table (4 KB), then a u32 entry per symbol
-// -- 512 for the joint table, 256 for each other -- 60 KB + 16 KB.
+// 12-bit totals: a u8 symbol per slot, 4096 slots per table (4 KB), then an 8-byte entry per
+// symbol -- 512 for the joint table, 256 for each other -- 60 KB + 32 KB.
 constexpr uint32_t kCtxBytes = 4096;                          // one table's slot block, either total
 constexpr uint32_t kSlotBytes = kDecodeTables * kCtxBytes;    // 61440
-constexpr uint32_t kSymEntryBytes = 16 * 256 * 4;             // 16384 (12-bit totals only)
-template <int PB>
+constexpr uint32_t kSymEntryBytes = 16 * 256 * 8;             // 32768 (12-bit totals only)
+// 12-bit totals, hybrid: the joint table and f2, f3 given each coset as direct words, one u32 per
+// slot (5 tables of 16 KB), the other 10 tables as symbol bytes (4 KB each) and 8-byte entries
+// (2 KB each) -- 140 KB, which leaves 16-warp CTAs 5.2 KB tile buffers.
+constexpr uint32_t kHDirect = 4 * 4096;                       // one direct table: 16384
+constexpr uint32_t kHL1 = 5 * kHDirect;                       // 81920: symbol bytes of f4..f8
+constexpr uint32_t kHL2 = kHL1 + 10 * kCtxBytes;              // 122880: their 8-byte entries
+constexpr uint32_t kHybridBytes = kHL2 + 10 * 2048;           // 143360
+
+// Table layouts: 10 = 10-bit totals, one packed word per slot; 12 = 12-bit totals, two lookups
+// per symbol; 13 = 12-bit totals, hybrid (16-warp CTAs only).
+template <int LAY>
 struct TableGeo {
-    static_assert(PB == 10 || PB == 12, "frequency totals are 10 or 12 bits");
-    static constexpr uint32_t kBytes = PB == 10 ? kSlotBytes : kSlotBytes + kSymEntryBytes;
+    static_assert(LAY == 10 || LAY == 12 || LAY == 13, "table layouts are 10, 12 and 13");
+    static constexpr uint32_t kBytes = LAY == 10 ? kSlotBytes : LAY == 12 ? kSlotBytes + kSymEntryBytes : kHybridBytes;
     static constexpr uint32_t kPiece = kBytes / 4;             // bytes per table bulk copy
 };
-constexpr uint32_t kMaxTableBytes = TableGeo<12>::kBytes;
-inline uint32_t table_bytes(int pb) { return pb == 10 ? TableGeo<10>::kBytes : TableGeo<12>::kBytes; }
+inline uint32_t table_bytes(int lay) {
+    return lay == 10 ? TableGeo<10>::kBytes : lay == 12 ? TableGeo<12>::kBytes : TableGeo<13>::kBytes;
+}
 
 // kOutE4M3Row: the FP8 container with a per-row scale -- an E4M3 payload normalised per row to
 // the format's range, plus one fp32 scale per row.
@@ -99,21 +110,21 @@ constexpr uint32_t kSmemOptin = 232448;  // 227 KB: the largest dynamic shared m
 constexpr uint32_t kAlignSlack = 4096;    // the table starts on a 4 KB boundary of the shared window
 constexpr uint32_t kBufSlack = 80;        // bytes after a tile buffer that two steps may over-read
 
-// CTA widths: 32 or 16 warps, each warp with a tile buffer of Geo<WARPS, PB>::kBuf bytes (5120 or
-// 10336 with 10-bit totals, 4608 or 9312 with 12-bit ones); a tile larger than its warp's buffer is
-// read from global memory.
+// CTA widths: 32 or 16 warps, each warp with a tile buffer of Geo<WARPS, LAY>::kBuf bytes (5120 or
+// 10336 with layout 10, 4096 or 8288 with layout 12, 5216 with layout 13 and 16 warps); a tile
+// larger than its warp's buffer is read from global memory.
 constexpr int kWarpsWide = 32, kWarpsNarrow = 16;
 
 // Per-warp tile buffer size for a CTA of WARPS warps: what the 227 KB leave after the tables.
-template <int WARPS, int PB>
+template <int WARPS, int LAY>
 struct Geo {
     static constexpr uint32_t kBuf =
-        ((kSmemOptin - kAlignSlack - TableGeo<PB>::kBytes - 64 - WARPS * (kBufSlack + 8) - 16) / WARPS) & ~15u;
+        ((kSmemOptin - kAlignSlack - TableGeo<LAY>::kBytes - 64 - WARPS * (kBufSlack + 8) - 16) / WARPS) & ~15u;
 };
-template <int WARPS, int PB>
+template <int WARPS, int LAY>
 struct Smem {
-    alignas(16) uint8_t tab[TableGeo<PB>::kBytes];                      // decode tables
-    alignas(16) uint8_t tbuf[WARPS][Geo<WARPS, PB>::kBuf + kBufSlack];  // one staged tile per warp
+    alignas(16) uint8_t tab[TableGeo<LAY>::kBytes];                      // decode tables
+    alignas(16) uint8_t tbuf[WARPS][Geo<WARPS, LAY>::kBuf + kBufSlack];  // one staged tile per warp
     unsigned long long bar[WARPS];                                      // tile staging, one per warp
     unsigned long long tbar;                                            // the table's bulk copies
     unsigned long long pbar;                                            // the wait-limit probe
@@ -123,11 +134,19 @@ using Smem32x12 = Smem<32, 12>;
 static_assert(offsetof(Smem32x10, tbuf) == TableGeo<10>::kBytes && offsetof(Smem32x12, tbuf) == TableGeo<12>::kBytes,
               "table block must be contiguous");
 static_assert(sizeof(Smem<32, 10>) + kAlignSlack <= kSmemOptin && sizeof(Smem<16, 10>) + kAlignSlack <= kSmemOptin &&
-              sizeof(Smem<32, 12>) + kAlignSlack <= kSmemOptin && sizeof(Smem<16, 12>) + kAlignSlack <= kSmemOptin,
+              sizeof(Smem<32, 12>) + kAlignSlack <= kSmemOptin && sizeof(Smem<16, 12>) + kAlignSlack <= kSmemOptin &&
+              sizeof(Smem<16, 13>) + kAlignSlack <= kSmemOptin,
               "shared memory budget");
-inline uint32_t tile_buffer_bytes(int warps, int pb) {
-    if (pb == 10) return warps == 32 ? Geo<32, 10>::kBuf : Geo<16, 10>::kBuf;
-    return warps == 32 ? Geo<32, 12>::kBuf : Geo<16, 12>::kBuf;
+inline uint32_t tile_buffer_bytes(int warps, int lay) {
+    if (lay == 10) return warps == 32 ? Geo<32, 10>::kBuf : Geo<16, 10>::kBuf;
+    if (lay == 12) return warps == 32 ? Geo<32, 12>::kBuf : Geo<16, 12>::kBuf;
+    return Geo<16, 13>::kBuf;
+}
+// The layout a blob decodes with: 10-bit totals take layout 10; 12-bit totals take the hybrid
+// when every tile fits its 16-warp buffers, else layout 12.
+inline int table_layout(int prob_bits, uint64_t max_tile_bytes) {
+    if (prob_bits == 10) return 10;
+    return max_tile_bytes <= Geo<16, 13>::kBuf ? 13 : 12;
 }
 
 // ---- launch functions, one table per output container ----------------------------------------
@@ -136,15 +155,15 @@ struct LaunchCtx {
     int sms;     // its SM count
 };
 
-// Every function takes the blob's frequency total width pb (10 or 12).
+// Every function takes the blob's table layout lay (10, 12 or 13; 13 always runs 16 warps).
 struct Launchers {
     // one blob; `dependent`: launch as a programmatic dependent of the previous decode
-    int (*single)(const Params& p, int pb, bool vec, bool wide, bool esc, const Ctl& ctl, cudaStream_t st,
+    int (*single)(const Params& p, int lay, bool vec, bool wide, bool esc, const Ctl& ctl, cudaStream_t st,
                   const LaunchCtx& c, bool dependent);
-    // a set of blobs, all with the same pb, over `grid` CTAs
-    int (*group)(const GroupParams& g, int pb, uint32_t grid, bool wide, cudaStream_t st, const LaunchCtx& c);
+    // a set of blobs, all with the same layout, over `grid` CTAs
+    int (*group)(const GroupParams& g, int lay, uint32_t grid, bool wide, cudaStream_t st, const LaunchCtx& c);
     // one blob, tables expanded in every CTA, status in caller-provided memory; never allocates
-    int (*noalloc)(const Params& p, const TableSrc& ts, int pb, bool vec, bool esc, cudaStream_t st,
+    int (*noalloc)(const Params& p, const TableSrc& ts, int lay, bool vec, bool esc, cudaStream_t st,
                    const LaunchCtx& c);
 };
 
