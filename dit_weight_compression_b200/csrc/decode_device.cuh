@@ -78,8 +78,8 @@ constexpr uint32_t kSlots10 = 1024;
 
 // 12-bit totals.  Symbol byte of slot u of table t at [4096 t + u] (for the joint table the f1
 // symbol of the slot's coset half; the coset is u >= the coset-0 total).  Per-symbol entry of
-// table t >= 1 at [kSlotBytes + 2048 (t + 1) + 8 s]; the joint table's at [kSlotBytes + 2048 c +
-// 8 s], its coset-1 cumulative frequencies following all of coset 0's:
+// field j (1: the joint table, its coset-1 cumulative frequencies following all of coset 0's)
+// given coset c at [kSlotBytes + c (8 * 2048 + kCosetSkew) + 2048 (j - 1) + 8 s]:
 //   word 0  q(s)                      (<= 4096; 0 for a symbol the table does not hold)
 //   word 1  -(cum(s) + 4096 t) mod 2^32
 // With the slot's shared address a = base + 4096 t + u, the state update is
@@ -99,7 +99,7 @@ struct Tab<12> {
 // Layout 13 (12-bit totals, hybrid), at `base` (4 KB aligned): the joint table's direct words at
 // base, f2 and f3 given coset c at base + kHDirect (1 + 2c + j - 2); symbol bytes of f4..f8 given c
 // at base + kHL1 + 4096 (5c + j - 4); their 8-byte entries (as in layout 12, with t = 5c + j - 4)
-// at base + kHL2 + 2048 (5c + j - 4).  A direct word of slot u holding symbol s:
+// at base + kHL2 + c (5 * 2048 + kCosetSkew) + 2048 (j - 4).  A direct word of slot u holding s:
 //   bits  0..11  u - cum(s)
 //   bits 12..19  s
 //   bits 20..31  q(s) - 1
@@ -322,12 +322,12 @@ __device__ void build_hybrid(uint8_t* tab, const BuildScratch& scr) {
             else dst8[slot] = uint8_t(sy);
         }
     }
-    uint2* ent = reinterpret_cast<uint2*>(tab + kHL2);
     for (uint32_t i = threadIdx.x; i < 10 * 256; i += WARPS * 32) {
-        const uint32_t row = i >> 8, sy = i & 255;
-        const uint32_t ctx = 8 * (row / 5) + 3 + row % 5;  // f4..f8 given coset row / 5
+        const uint32_t row = i >> 8, sy = i & 255;        // row = 5c + j - 4
+        const uint32_t c = row / 5, ctx = 8 * c + 3 + row % 5;
         const uint32_t q = scr.q[ctx][sy];
-        ent[i] = q ? make_uint2(q, 0u - (uint32_t(scr.cum[ctx][sy]) + kCtxBytes * row)) : make_uint2(0u, 0u);
+        uint2* ent = reinterpret_cast<uint2*>(tab + kHL2 + c * kCosetSkew + 2048 * row);
+        ent[sy] = q ? make_uint2(q, 0u - (uint32_t(scr.cum[ctx][sy]) + kCtxBytes * row)) : make_uint2(0u, 0u);
     }
 }
 
@@ -418,17 +418,17 @@ __device__ void build_tables(uint8_t* tab, BuildScratch& scr, const TableSrc& p)
         }
     }
     if constexpr (LAY == 12) {
-        // (c) the per-symbol entries: row 0/1 the joint table's coset halves (table 0; coset 1's
-        // cumulative frequencies after coset 0's), row t + 1 table t >= 1
-        uint2* ent = reinterpret_cast<uint2*>(tab + kSlotBytes);
+        // (c) the per-symbol entries of field j (1..8) given coset c, table t (0 for the joint
+        // table, whose coset-1 cumulative frequencies follow coset 0's; else 1 + 7c + j - 2)
         const uint32_t split = scr.cum[0][256];
         for (uint32_t i = threadIdx.x; i < 16 * 256; i += WARPS * 32) {
-            const uint32_t row = i >> 8, sy = i & 255;
-            const uint32_t ctx = row == 0 ? 0u : row == 1 ? 8u : 8 * ((row - 2) / 7) + 1 + (row - 2) % 7;
-            const uint32_t t = row < 2 ? 0u : row - 1;
+            const uint32_t c = i >> 11, j = 1 + ((i >> 8) & 7), sy = i & 255;
+            const uint32_t ctx = 8 * c + j - 1;
+            const uint32_t t = j == 1 ? 0u : 1 + 7 * c + j - 2;
             const uint32_t q = scr.q[ctx][sy];
-            const uint32_t cum = scr.cum[ctx][sy] + (row == 1 ? split : 0u);
-            ent[i] = q ? make_uint2(q, 0u - (cum + kCtxBytes * t)) : make_uint2(0u, 0u);
+            const uint32_t cum = scr.cum[ctx][sy] + (j == 1 && c ? split : 0u);
+            uint2* ent = reinterpret_cast<uint2*>(tab + kSlotBytes + c * (8 * 2048 + kCosetSkew) + 2048 * (j - 1));
+            ent[sy] = q ? make_uint2(q, 0u - (cum + kCtxBytes * t)) : make_uint2(0u, 0u);
         }
     }
 }
@@ -643,7 +643,7 @@ __device__ __forceinline__ void step_symbols12(const Tab<12>& T, Reader& rd, uin
         const uint32_t a1 = (x & 4095u) | T.s1;
         c = a1 >= T.s1split ? 1u : 0u;
         const uint32_t sy = lds_u8<0>(a1);
-        const uint2 en = lds_v2<0>(T.e2 + 2048u * c + 8u * sy);
+        const uint2 en = lds_v2<0>(T.e2 + (8u * 2048u + kCosetSkew) * c + 8u * sy);
         if (active) x = en.x * (x >> 12) + (a1 + en.y + ks);
         renorm_step<FULL>(x, rd, active);
         e[0] = sy;
@@ -651,7 +651,7 @@ __device__ __forceinline__ void step_symbols12(const Tab<12>& T, Reader& rd, uin
     }
     s.c = c;
     const uint32_t b1 = T.s1 + kCtxBytes + c * (7u * kCtxBytes);  // field 2's symbol bytes given c
-    const uint32_t b2 = T.e2 + 4096u + c * (7u * 2048u);           // field 2's entries given c
+    const uint32_t b2 = T.e2 + 2048u + c * (8u * 2048u + kCosetSkew);  // field 2's entries given c
 #define EP_FIELD12(j)                                                                         \
     {                                                                                         \
         const uint32_t a1 = (x & 4095u) | b1;                                                 \
@@ -705,13 +705,28 @@ __device__ __forceinline__ void step_symbols13(const Tab<13>& T, Reader& rd, uin
     }
     s.c = c;
     const uint32_t bd = T.base + kHDirect + c * (2u * kHDirect);   // f2 given c; f3 follows
-#define EP_FIELD13D(j)                                                                            {                                                                                                 const uint32_t sy = direct(lds_u32<((j) - 1) * kHDirect>(bd + 4u * (x & 4095u)));             renorm_step<FULL>(x, rd, active);                                                             e[j] = sy;                                                                                    if (ESC) acc = max(acc, sy);                                                              }
+#define EP_FIELD13D(j)                                                                        \
+    {                                                                                         \
+        const uint32_t sy = direct(lds_u32<((j) - 1) * kHDirect>(bd + 4u * (x & 4095u)));     \
+        renorm_step<FULL>(x, rd, active);                                                     \
+        e[j] = sy;                                                                            \
+        if (ESC) acc = max(acc, sy);                                                          \
+    }
     EP_FIELD13D(1) EP_FIELD13D(2)
 #undef EP_FIELD13D
     const uint32_t b1 = T.base + kHL1 + c * (5u * kCtxBytes);      // f4's symbol bytes given c
-    const uint32_t b2 = T.base + kHL2 + c * (5u * 2048u);          // f4's entries given c
+    const uint32_t b2 = T.base + kHL2 + c * (5u * 2048u + kCosetSkew);  // f4's entries given c
     const uint32_t ks = 0u - (T.base + kHL1);
-#define EP_FIELD13(j)                                                                             {                                                                                                 const uint32_t a1 = (x & 4095u) | b1;                                                         const uint32_t sy = lds_u8<((j) - 3) * kCtxBytes>(a1);                                        const uint2 en = lds_v2<((j) - 3) * 2048>(b2 + 8u * sy);                                      if (active) x = en.x * (x >> 12) + (a1 + en.y + (ks + ((j) - 3) * kCtxBytes));                 renorm_step<FULL>(x, rd, active);                                                             e[j] = sy;                                                                                    if (ESC) acc = max(acc, sy);                                                              }
+#define EP_FIELD13(j)                                                                         \
+    {                                                                                         \
+        const uint32_t a1 = (x & 4095u) | b1;                                                 \
+        const uint32_t sy = lds_u8<((j) - 3) * kCtxBytes>(a1);                                \
+        const uint2 en = lds_v2<((j) - 3) * 2048>(b2 + 8u * sy);                              \
+        if (active) x = en.x * (x >> 12) + (a1 + en.y + (ks + ((j) - 3) * kCtxBytes));         \
+        renorm_step<FULL>(x, rd, active);                                                     \
+        e[j] = sy;                                                                            \
+        if (ESC) acc = max(acc, sy);                                                          \
+    }
     EP_FIELD13(3) EP_FIELD13(4) EP_FIELD13(5) EP_FIELD13(6) EP_FIELD13(7)
 #undef EP_FIELD13
 

@@ -24,14 +24,17 @@ constexpr int kDecodeTables = 15;
 // symbol -- 512 for the joint table, 256 for each other -- 60 KB + 32 KB.
 constexpr uint32_t kCtxBytes = 4096;                          // one table's slot block, either total
 constexpr uint32_t kSlotBytes = kDecodeTables * kCtxBytes;    // 61440
-constexpr uint32_t kSymEntryBytes = 16 * 256 * 8;             // 32768 (12-bit totals only)
+// The per-symbol entries of coset 1 start kCosetSkew bytes past a whole number of rows, so that a
+// warp whose lanes read the same symbol of the same field in both cosets hits different banks.
+constexpr uint32_t kCosetSkew = 64;
+constexpr uint32_t kSymEntryBytes = 16 * 256 * 8 + kCosetSkew;  // 32832 (12-bit totals only)
 // 12-bit totals, hybrid: the joint table and f2, f3 given each coset as direct words, one u32 per
 // slot (5 tables of 16 KB), the other 10 tables as symbol bytes (4 KB each) and 8-byte entries
 // (2 KB each) -- 140 KB, which leaves 16-warp CTAs 5.2 KB tile buffers.
 constexpr uint32_t kHDirect = 4 * 4096;                       // one direct table: 16384
 constexpr uint32_t kHL1 = 5 * kHDirect;                       // 81920: symbol bytes of f4..f8
 constexpr uint32_t kHL2 = kHL1 + 10 * kCtxBytes;              // 122880: their 8-byte entries
-constexpr uint32_t kHybridBytes = kHL2 + 10 * 2048;           // 143360
+constexpr uint32_t kHybridBytes = kHL2 + 10 * 2048 + kCosetSkew;  // 143424
 
 // Table layouts: 10 = 10-bit totals, one packed word per slot; 12 = 12-bit totals, two lookups
 // per symbol; 13 = 12-bit totals, hybrid (16-warp CTAs only).
@@ -111,7 +114,7 @@ constexpr uint32_t kAlignSlack = 4096;    // the table starts on a 4 KB boundary
 constexpr uint32_t kBufSlack = 80;        // bytes after a tile buffer that two steps may over-read
 
 // CTA widths: 32 or 16 warps, each warp with a tile buffer of Geo<WARPS, LAY>::kBuf bytes (5120 or
-// 10336 with layout 10, 4096 or 8288 with layout 12, 5216 with layout 13 and 16 warps); a tile
+// 10336 with layout 10, 4096 or 8272 with layout 12, 5200 with layout 13 and 16 warps); a tile
 // larger than its warp's buffer is read from global memory.
 constexpr int kWarpsWide = 32, kWarpsNarrow = 16;
 
