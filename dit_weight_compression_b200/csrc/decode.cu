@@ -23,6 +23,11 @@ struct DevInfo {
 std::mutex g_dev_mu;
 DevInfo g_dev[kMaxDevices];
 
+// The table layout of a blob's decodes on device `dev` (its SM count known: current_device ran).
+int blob_layout(const BlobLayout& L, int dev) {
+    return table_layout(L.prob_bits, L.max_tile_bytes, L.n_tiles, g_dev[dev].sms, true);
+}
+
 const Launchers* launchers_for(int out_kind) {
     switch (out_kind) {
         case kOutBF16: return &kLaunchBF16;
@@ -42,7 +47,7 @@ const Launchers* launchers_for(int out_kind) {
 int launch(const Params& p, int out_kind, const BlobLayout& L, bool vec, const Ctl& ctl, cudaStream_t st, int device,
            bool dependent) {
     const LaunchCtx c{device, g_dev[device].sms};
-    const int lay = table_layout(L.prob_bits, L.max_tile_bytes);
+    const int lay = blob_layout(L, device);
     const bool wide = lay != 13 && L.max_tile_bytes <= tile_buffer_bytes(kWarpsWide, lay) &&
                       p.n_tiles > uint32_t(kWarpsNarrow) * uint32_t(c.sms);
     const Launchers* ln = launchers_for(out_kind);
@@ -139,7 +144,7 @@ int ensure_device(ep_blob* b, int dev, cudaStream_t st) {
     uint8_t* blob = nullptr;
     uint8_t* tables = nullptr;
     uint32_t* status = nullptr;
-    const int lay = table_layout(b->layout.prob_bits, b->layout.max_tile_bytes);
+    const int lay = blob_layout(b->layout, dev);
     if (cudaMalloc(&blob, b->bytes.size()) != cudaSuccess || cudaMalloc(&tables, table_bytes(lay)) != cudaSuccess ||
         cudaMalloc(&status, 16) != cudaSuccess) {
         cudaFree(blob);
@@ -309,7 +314,7 @@ extern "C" int ep_decompress_group(const ep_blob* const* blobs, const ep_tensor*
     for (int lay : {13, 12, 10}) {
         std::vector<int> idx;
         for (int i = 0; i < n; ++i)
-            if (table_layout(blobs[i]->layout.prob_bits, blobs[i]->layout.max_tile_bytes) == lay) idx.push_back(i);
+            if (blob_layout(blobs[i]->layout, dev) == lay) idx.push_back(i);
         for (size_t c0 = 0; c0 < idx.size(); c0 += size_t(chunk)) {
             const int cn = int(std::min(size_t(chunk), idx.size() - c0));
             std::vector<uint32_t> tiles(static_cast<size_t>(cn));
@@ -519,7 +524,8 @@ extern "C" int ep_decompress_noalloc(const ep_blob* cb, const void* device_blob,
     Params p = make_params(cb, static_cast<const uint8_t*>(device_blob), nullptr, out->data, out->row_stride,
                            status);
     const TableSrc ts = make_tablesrc(cb, static_cast<const uint8_t*>(device_blob));
-    int rc = launchers_for(kind)->noalloc(p, ts, table_layout(L.prob_bits, L.max_tile_bytes), vec,
+    // 16-warp CTAs only, so the layout choice ignores the 32-warp rule
+    int rc = launchers_for(kind)->noalloc(p, ts, table_layout(L.prob_bits, L.max_tile_bytes, L.n_tiles, 0, false), vec,
                                           L.has_escape != 0, st, LaunchCtx{dev, g_noalloc[dev].sms});
     if (rc != EP_OK || !wait) return rc;
     uint32_t s = 0;

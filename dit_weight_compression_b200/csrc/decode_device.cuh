@@ -14,9 +14,9 @@
 //     {slot - cum(s), s (2 s for f8), escape flag, coset bit, q(s)} -- 60 KB -- so one
 //     shared-memory load per symbol gives everything the state update needs.  With 12-bit totals
 //     the per-slot entries would take 240 KB, more than an SM has, so a symbol takes two loads:
-//     the slot's symbol byte (4096 per table, 60 KB), then that symbol's {q(s), -(cum(s) + the
-//     table's byte offset)} pair (32 KB), which turns the state update into one three-input add
-//     and one multiply-add on the slot's shared address.  The tables are expanded once per blob and device by a small kernel into
+//     the slot's symbol byte (4096 per table, 60 KB), then that symbol's packed {q(s), cum(s)}
+//     word (16 KB), so the state update is two field extractions, a subtraction and a
+//     multiply-add.  The tables are expanded once per blob and device by a small kernel into
 //     a block next to the device copy; every CTA stages that block into shared memory with bulk
 //     copies, overlapped with the fetch of its first tiles.  (The allocation-free entry point
 //     expands them inside each CTA instead.);
@@ -79,11 +79,12 @@ constexpr uint32_t kSlots10 = 1024;
 // 12-bit totals.  Symbol byte of slot u of table t at [4096 t + u] (for the joint table the f1
 // symbol of the slot's coset half; the coset is u >= the coset-0 total).  Per-symbol entry of
 // field j (1: the joint table, its coset-1 cumulative frequencies following all of coset 0's)
-// given coset c at [kSlotBytes + c (8 * 2048 + kCosetSkew) + 2048 (j - 1) + 8 s]:
-//   word 0  q(s)                      (<= 4096; 0 for a symbol the table does not hold)
-//   word 1  -(cum(s) + 4096 t) mod 2^32
-// With the slot's shared address a = base + 4096 t + u, the state update is
-// x <- q (x >> 12) + (a + word1 - base) = q (x >> 12) + u - cum(s).
+// given coset c at [kSlotBytes + c (8 * 1024 + kCosetSkew) + 1024 (j - 1) + 4 s]:
+//   bits  0..12  cum(s)               (< 2^13; the joint table's coset-1 symbols follow coset 0's)
+//   bits 17..29  q(s)                 (<= 4096; 0 for a symbol the table does not hold)
+// With the slot u = x mod 4096, the state update is x <- q (x >> 12) + u - cum(s).
+constexpr uint32_t kE12CumMask = 0x1FFFu;
+constexpr uint32_t kE12QShift = 17;
 
 // Shared addresses of the decode tables a step reads.
 template <int LAY>
@@ -98,8 +99,9 @@ struct Tab<12> {
 };
 // Layout 13 (12-bit totals, hybrid), at `base` (4 KB aligned): the joint table's direct words at
 // base, f2 and f3 given coset c at base + kHDirect (1 + 2c + j - 2); symbol bytes of f4..f8 given c
-// at base + kHL1 + 4096 (5c + j - 4); their 8-byte entries (as in layout 12, with t = 5c + j - 4)
-// at base + kHL2 + c (5 * 2048 + kCosetSkew) + 2048 (j - 4).  A direct word of slot u holding s:
+// at base + kHL1 + 4096 (5c + j - 4); their 4-byte entries (as in layout 12) at
+// base + kHL2 + c (5 * 1024 + kCosetSkew) + 1024 (j - 4).  A direct word of
+// slot u holding s:
 //   bits  0..11  u - cum(s)
 //   bits 12..19  s
 //   bits 20..31  q(s) - 1
@@ -178,12 +180,6 @@ template <int OFF = 0>
 __device__ __forceinline__ uint32_t lds_u32(uint32_t a) {
     uint32_t v;
     asm volatile("ld.shared.u32 %0, [%1+%2];" : "=r"(v) : "r"(a), "n"(OFF));
-    return v;
-}
-template <int OFF = 0>
-__device__ __forceinline__ uint2 lds_v2(uint32_t a) {
-    uint2 v;
-    asm volatile("ld.shared.v2.u32 {%0, %1}, [%2+%3];" : "=r"(v.x), "=r"(v.y) : "r"(a), "n"(OFF));
     return v;
 }
 // Shared address of slot (x mod M) of a 4 KB-aligned table at `base`: a mask and a multiply-add,
@@ -271,7 +267,7 @@ __device__ __forceinline__ uint32_t pack_entry(uint32_t bias, uint32_t s, uint32
 }
 
 // Layout 13 from the per-context frequencies and cumulative frequencies in `scr`: the 5 direct
-// tables, the 10 symbol-byte tables, then the 8-byte entries of those 10.
+// tables, the 10 symbol-byte tables, then the 4-byte entries of those 10.
 template <int WARPS>
 __device__ void build_hybrid(uint8_t* tab, const BuildScratch& scr) {
     const uint32_t lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
@@ -326,8 +322,8 @@ __device__ void build_hybrid(uint8_t* tab, const BuildScratch& scr) {
         const uint32_t row = i >> 8, sy = i & 255;        // row = 5c + j - 4
         const uint32_t c = row / 5, ctx = 8 * c + 3 + row % 5;
         const uint32_t q = scr.q[ctx][sy];
-        uint2* ent = reinterpret_cast<uint2*>(tab + kHL2 + c * kCosetSkew + 2048 * row);
-        ent[sy] = q ? make_uint2(q, 0u - (uint32_t(scr.cum[ctx][sy]) + kCtxBytes * row)) : make_uint2(0u, 0u);
+        uint32_t* ent = reinterpret_cast<uint32_t*>(tab + kHL2 + c * kCosetSkew + 1024 * row);
+        ent[sy] = q ? (q << kE12QShift) | uint32_t(scr.cum[ctx][sy]) : 0u;
     }
 }
 
@@ -418,17 +414,16 @@ __device__ void build_tables(uint8_t* tab, BuildScratch& scr, const TableSrc& p)
         }
     }
     if constexpr (LAY == 12) {
-        // (c) the per-symbol entries of field j (1..8) given coset c, table t (0 for the joint
-        // table, whose coset-1 cumulative frequencies follow coset 0's; else 1 + 7c + j - 2)
+        // (c) the per-symbol entries of field j (1..8) given coset c (the joint table's coset-1
+        // cumulative frequencies follow coset 0's; a field's carry its table's offset in the block)
         const uint32_t split = scr.cum[0][256];
         for (uint32_t i = threadIdx.x; i < 16 * 256; i += WARPS * 32) {
             const uint32_t c = i >> 11, j = 1 + ((i >> 8) & 7), sy = i & 255;
             const uint32_t ctx = 8 * c + j - 1;
-            const uint32_t t = j == 1 ? 0u : 1 + 7 * c + j - 2;
             const uint32_t q = scr.q[ctx][sy];
             const uint32_t cum = scr.cum[ctx][sy] + (j == 1 && c ? split : 0u);
-            uint2* ent = reinterpret_cast<uint2*>(tab + kSlotBytes + c * (8 * 2048 + kCosetSkew) + 2048 * (j - 1));
-            ent[sy] = q ? make_uint2(q, 0u - (cum + kCtxBytes * t)) : make_uint2(0u, 0u);
+            uint32_t* ent = reinterpret_cast<uint32_t*>(tab + kSlotBytes + c * (8 * 1024 + kCosetSkew) + 1024 * (j - 1));
+            ent[sy] = q ? (q << kE12QShift) | cum : 0u;
         }
     }
 }
@@ -635,29 +630,28 @@ __device__ __forceinline__ void step_symbols12(const Tab<12>& T, Reader& rd, uin
     if (FULL) active = true;
     uint32_t* e = s.e;
     uint32_t acc = 0;                          // largest symbol: the escape symbol is the largest
-    const uint32_t ks = 0u - T.s1;             // (base of the symbol bytes, negated)
     // (coset, f1): the slot's half of the joint table gives the coset (known before the loads
     // return), its byte the f1 symbol.  A lane past the last vector still loads but keeps x.
     uint32_t c;
     {
-        const uint32_t a1 = (x & 4095u) | T.s1;
+        const uint32_t u = x & 4095u, a1 = u | T.s1;
         c = a1 >= T.s1split ? 1u : 0u;
         const uint32_t sy = lds_u8<0>(a1);
-        const uint2 en = lds_v2<0>(T.e2 + (8u * 2048u + kCosetSkew) * c + 8u * sy);
-        if (active) x = en.x * (x >> 12) + (a1 + en.y + ks);
+        const uint32_t en = lds_u32<0>(T.e2 + (8u * 1024u + kCosetSkew) * c + 4u * sy);
+        if (active) x = (en >> kE12QShift) * (x >> 12) + (u - (en & kE12CumMask));
         renorm_step<FULL>(x, rd, active);
         e[0] = sy;
         if (ESC) acc = sy;
     }
     s.c = c;
-    const uint32_t b1 = T.s1 + kCtxBytes + c * (7u * kCtxBytes);  // field 2's symbol bytes given c
-    const uint32_t b2 = T.e2 + 2048u + c * (8u * 2048u + kCosetSkew);  // field 2's entries given c
+    const uint32_t b1 = T.s1 + kCtxBytes + c * (7u * kCtxBytes);        // field 2's symbol bytes given c
+    const uint32_t b2 = T.e2 + 1024u + c * (8u * 1024u + kCosetSkew);   // field 2's entries given c
 #define EP_FIELD12(j)                                                                         \
     {                                                                                         \
-        const uint32_t a1 = (x & 4095u) | b1;                                                 \
-        const uint32_t sy = lds_u8<((j) - 1) * kCtxBytes>(a1);                                \
-        const uint2 en = lds_v2<((j) - 1) * 2048>(b2 + 8u * sy);                              \
-        if (active) x = en.x * (x >> 12) + (a1 + en.y + (ks + ((j) - 1) * kCtxBytes));         \
+        const uint32_t u = x & 4095u;                                                         \
+        const uint32_t sy = lds_u8<((j) - 1) * kCtxBytes>(u | b1);                            \
+        const uint32_t en = lds_u32<((j) - 1) * 1024>(b2 + 4u * sy);                          \
+        if (active) x = (en >> kE12QShift) * (x >> 12) + (u - (en & kE12CumMask));            \
         renorm_step<FULL>(x, rd, active);                                                     \
         e[j] = sy;                                                                            \
         if (ESC) acc = max(acc, sy);                                                          \
@@ -715,14 +709,13 @@ __device__ __forceinline__ void step_symbols13(const Tab<13>& T, Reader& rd, uin
     EP_FIELD13D(1) EP_FIELD13D(2)
 #undef EP_FIELD13D
     const uint32_t b1 = T.base + kHL1 + c * (5u * kCtxBytes);      // f4's symbol bytes given c
-    const uint32_t b2 = T.base + kHL2 + c * (5u * 2048u + kCosetSkew);  // f4's entries given c
-    const uint32_t ks = 0u - (T.base + kHL1);
+    const uint32_t b2 = T.base + kHL2 + c * (5u * 1024u + kCosetSkew);  // f4's entries given c
 #define EP_FIELD13(j)                                                                         \
     {                                                                                         \
-        const uint32_t a1 = (x & 4095u) | b1;                                                 \
-        const uint32_t sy = lds_u8<((j) - 3) * kCtxBytes>(a1);                                \
-        const uint2 en = lds_v2<((j) - 3) * 2048>(b2 + 8u * sy);                              \
-        if (active) x = en.x * (x >> 12) + (a1 + en.y + (ks + ((j) - 3) * kCtxBytes));         \
+        const uint32_t u = x & 4095u;                                                         \
+        const uint32_t sy = lds_u8<((j) - 3) * kCtxBytes>(u | b1);                            \
+        const uint32_t en = lds_u32<((j) - 3) * 1024>(b2 + 4u * sy);                          \
+        if (active) x = (en >> kE12QShift) * (x >> 12) + (u - (en & kE12CumMask));            \
         renorm_step<FULL>(x, rd, active);                                                     \
         e[j] = sy;                                                                            \
         if (ESC) acc = max(acc, sy);                                                          \

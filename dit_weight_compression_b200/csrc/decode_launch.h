@@ -20,21 +20,21 @@ constexpr uint32_t kWaitSpins = 1u << 22;                     // bounded mbarrie
 // Decode tables: [0] the joint (coset, f1) symbol; [1 + 7c + (j - 2)] field j = 2..8 given coset c.
 constexpr int kDecodeTables = 15;
 // 10-bit totals: one packed u32 entry per slot, 1024 slots per table (4 KB), 60 KB in all.
-// 12-bit totals: a u8 symbol per slot, 4096 slots per table (4 KB), then an 8-byte entry per
-// symbol -- 512 for the joint table, 256 for each other -- 60 KB + 32 KB.
+// 12-bit totals: a u8 symbol per slot, 4096 slots per table (4 KB), then a 4-byte entry per
+// symbol -- 512 for the joint table, 256 for each other -- 60 KB + 16 KB.
 constexpr uint32_t kCtxBytes = 4096;                          // one table's slot block, either total
 constexpr uint32_t kSlotBytes = kDecodeTables * kCtxBytes;    // 61440
 // The per-symbol entries of coset 1 start kCosetSkew bytes past a whole number of rows, so that a
 // warp whose lanes read the same symbol of the same field in both cosets hits different banks.
 constexpr uint32_t kCosetSkew = 64;
-constexpr uint32_t kSymEntryBytes = 16 * 256 * 8 + kCosetSkew;  // 32832 (12-bit totals only)
+constexpr uint32_t kSymEntryBytes = 16 * 256 * 4 + kCosetSkew;  // 16448 (12-bit totals only)
 // 12-bit totals, hybrid: the joint table and f2, f3 given each coset as direct words, one u32 per
-// slot (5 tables of 16 KB), the other 10 tables as symbol bytes (4 KB each) and 8-byte entries
-// (2 KB each) -- 140 KB, which leaves 16-warp CTAs 5.2 KB tile buffers.
+// slot (5 tables of 16 KB), the other 10 tables as symbol bytes (4 KB each) and 4-byte entries
+// (1 KB each) -- 130 KB, which leaves 16-warp CTAs 5.8 KB tile buffers.
 constexpr uint32_t kHDirect = 4 * 4096;                       // one direct table: 16384
 constexpr uint32_t kHL1 = 5 * kHDirect;                       // 81920: symbol bytes of f4..f8
-constexpr uint32_t kHL2 = kHL1 + 10 * kCtxBytes;              // 122880: their 8-byte entries
-constexpr uint32_t kHybridBytes = kHL2 + 10 * 2048 + kCosetSkew;  // 143424
+constexpr uint32_t kHL2 = kHL1 + 10 * kCtxBytes;              // 122880: their 4-byte entries
+constexpr uint32_t kHybridBytes = kHL2 + 10 * 1024 + kCosetSkew;  // 133184
 
 // Table layouts: 10 = 10-bit totals, one packed word per slot; 12 = 12-bit totals, two lookups
 // per symbol; 13 = 12-bit totals, hybrid (16-warp CTAs only).
@@ -114,7 +114,7 @@ constexpr uint32_t kAlignSlack = 4096;    // the table starts on a 4 KB boundary
 constexpr uint32_t kBufSlack = 80;        // bytes after a tile buffer that two steps may over-read
 
 // CTA widths: 32 or 16 warps, each warp with a tile buffer of Geo<WARPS, LAY>::kBuf bytes (5120 or
-// 10336 with layout 10, 4096 or 8272 with layout 12, 5200 with layout 13 and 16 warps); a tile
+// 10336 with layout 10, 4608 or 9296 with layout 12, 5840 with layout 13 and 16 warps); a tile
 // larger than its warp's buffer is read from global memory.
 constexpr int kWarpsWide = 32, kWarpsNarrow = 16;
 
@@ -145,10 +145,17 @@ inline uint32_t tile_buffer_bytes(int warps, int lay) {
     if (lay == 12) return warps == 32 ? Geo<32, 12>::kBuf : Geo<16, 12>::kBuf;
     return Geo<16, 13>::kBuf;
 }
-// The layout a blob decodes with: 10-bit totals take layout 10; 12-bit totals take the hybrid
-// when every tile fits its 16-warp buffers, else layout 12.
-inline int table_layout(int prob_bits, uint64_t max_tile_bytes) {
+// The layout a blob of n_tiles tiles decodes with on a device of `sms` SMs.  10-bit totals take
+// layout 10.  12-bit totals take layout 12 in 32-warp CTAs when there are more tiles than 16-warp
+// CTAs hold at once and every tile fits the 32-warp buffers (twice the independent rANS chains
+// per SM are worth the second lookup of three more symbols per vector); else the hybrid when every
+// tile fits its 16-warp buffers; else layout 12.  `wide_ok` false (a launch that runs 16-warp
+// CTAs only) skips the first rule.
+inline int table_layout(int prob_bits, uint64_t max_tile_bytes, uint64_t n_tiles, int sms, bool wide_ok) {
     if (prob_bits == 10) return 10;
+    if (wide_ok && n_tiles > uint64_t(kWarpsNarrow) * uint64_t(sms > 0 ? sms : 0) &&
+        max_tile_bytes <= Geo<kWarpsWide, 12>::kBuf)
+        return 12;
     return max_tile_bytes <= Geo<16, 13>::kBuf ? 13 : 12;
 }
 
