@@ -2,6 +2,8 @@
 // error message helpers shared by the host API (api.cpp) and the GPU API (decode.cu).
 #pragma once
 
+#include <cuda_runtime_api.h>
+
 #include <mutex>
 #include <string>
 #include <vector>
@@ -12,6 +14,7 @@
 namespace ep {
 
 constexpr int kMaxDevices = 64;
+constexpr int kMaxHostChunks = 8;   // host-output path: most chunks one call is split into
 
 // Device-side state of one blob on one GPU.
 struct DeviceCopy {
@@ -22,6 +25,7 @@ struct DeviceCopy {
     uint8_t* stage_out = nullptr;   // host-output path: decode target before the D2H copy
     size_t stage_out_bytes = 0;
     float* stage_sigma = nullptr;   // host-output path of the row-scaled FP8 container: row scales
+    cudaEvent_t chunk_done[kMaxHostChunks] = {};  // host-output path: chunk i decoded
 };
 
 int set_error(int code, const std::string& msg);

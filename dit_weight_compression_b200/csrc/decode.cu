@@ -4,6 +4,8 @@
 // container's instantiations are compiled in decode_<container>.cu.
 #include "decode_device.cuh"
 
+#include <numeric>
+#include <string>
 #include <vector>
 
 // Scratch of ep_decompress_noalloc: a fixed 256-byte array on every device that loads this
@@ -19,6 +21,8 @@ namespace {
 struct DevInfo {
     bool ready = false;
     int sms = 0;
+    cudaStream_t copyback = nullptr;  // host-output path: downloads run here (made on first use,
+                                      // kept for the life of the process)
 };
 std::mutex g_dev_mu;
 DevInfo g_dev[kMaxDevices];
@@ -188,6 +192,12 @@ int ensure_staging(ep_blob* b, int dev, size_t out_bytes, bool sigma) {
     }
     if (sigma && !d.stage_sigma && cudaMalloc(&d.stage_sigma, 4 * size_t(b->layout.rows)) != cudaSuccess)
         return set_error(EP_ERR_OOM, "host-output decode: staging row scales");
+    for (cudaEvent_t& e : d.chunk_done)
+        if (!e && cudaEventCreateWithFlags(&e, cudaEventDisableTiming) != cudaSuccess) {
+            e = nullptr;
+            cudaGetLastError();
+            return set_error(EP_ERR_CUDA, "host-output decode: chunk events");
+        }
     if (!b->host_pinned) {
         // best effort: page-locked host bytes make the per-call upload a direct DMA
         if (cudaHostRegister(b->bytes.data(), b->bytes.size(), cudaHostRegisterDefault) == cudaSuccess)
@@ -201,6 +211,109 @@ int ensure_staging(ep_blob* b, int dev, size_t out_bytes, bool sigma) {
 bool vec_ok(const BlobLayout& L, const void* out, int64_t row_stride, int dtype) {
     const uintptr_t align = (dtype == kE4M3 || dtype == kI8) ? 8 : 16;
     return L.cols % 8 == 0 && row_stride % 8 == 0 && (reinterpret_cast<uintptr_t>(out) % align) == 0;
+}
+
+// ---- host-output path ------------------------------------------------------------------------
+constexpr size_t kHostChunkBytes = size_t(4) << 20;  // output bytes per chunk, at least
+
+// The device's copy-back stream.
+int copyback_stream(int dev, cudaStream_t& out) {
+    std::lock_guard<std::mutex> g(g_dev_mu);
+    if (!g_dev[dev].copyback)
+        EP_CUDA(cudaStreamCreateWithFlags(&g_dev[dev].copyback, cudaStreamNonBlocking), "copy-back stream");
+    out = g_dev[dev].copyback;
+    return EP_OK;
+}
+
+// Tile boundaries of the host-output pipeline: chunk i holds tiles [t[i], t[i+1]).  Every chunk
+// starts on a row (its first vector is a multiple of the row's vector count), carries at least
+// kHostChunkBytes of output where the blob has that much, and there are at most kMaxHostChunks.
+// A small blob, or one whose tiles end on a row boundary only rarely, is one chunk.
+std::vector<uint32_t> host_chunks(const BlobLayout& L, size_t out_bytes) {
+    std::vector<uint32_t> t{0};
+    const uint64_t per = uint64_t(kLanes) * L.steps;                       // vectors per tile
+    const uint64_t vpr = uint64_t(L.vec_per_row);
+    const uint64_t unit = vpr / std::gcd(per, vpr);                        // tiles per row-aligned unit
+    const uint64_t n = std::min<uint64_t>(kMaxHostChunks, out_bytes / kHostChunkBytes);
+    if (n >= 2 && unit < L.n_tiles) {
+        const uint64_t units = (uint64_t(L.n_tiles) + unit - 1) / unit;
+        for (uint64_t i = 1; i < n; ++i) {
+            const uint64_t b = (units * i / n) * unit;
+            if (b > t.back() && b < L.n_tiles) t.push_back(uint32_t(b));
+        }
+    }
+    t.push_back(L.n_tiles);
+    return t;
+}
+
+// Decode into host memory (out->device == -1) and, for the row-scaled FP8 container, host row
+// scales.  The bytes before the stream section go up first; then chunk by chunk (whole rows
+// each), the chunk's stream bytes are uploaded and its tiles decoded on `st`, and the copy-back
+// stream waits for that decode and downloads the chunk's rows.  So the download of one chunk
+// overlaps the upload and decode of the next, and a call costs about its longer copy direction
+// instead of the sum of both.  A chunk is decoded as the blob restricted to its rows: the tile
+// offsets, scales, row maxima and output start at the chunk's first tile and row, which every
+// tile's decode already treats as its own origin.  Returns when every row is back.
+int decode_to_host(ep_blob* b, const ep_tensor* out, int kind, float* host_sigma, cudaStream_t st, int dev,
+                   const char* what) {
+    const BlobLayout& L = b->layout;
+    const size_t es = size_t(dtype_bytes(out->dtype));
+    const size_t row_bytes = size_t(L.cols) * es;
+    int rc = ensure_device(b, dev, st);
+    if (rc == EP_OK) rc = ensure_staging(b, dev, row_bytes * size_t(L.rows), host_sigma != nullptr);
+    cudaStream_t cb = nullptr;
+    if (rc == EP_OK) rc = copyback_stream(dev, cb);
+    if (rc != EP_OK) return rc;
+    const DeviceCopy& d = b->dev[dev];
+    const uint8_t* host = b->bytes.data();
+    const uint64_t stream_total = L.total - L.off_stream;
+    const uint64_t per = uint64_t(kLanes) * L.steps;
+    const std::vector<uint32_t> t = host_chunks(L, row_bytes * size_t(L.rows));
+    const std::string w(what);
+    EP_CUDA(cudaMemcpyAsync(d.stage_blob, host, L.off_stream, cudaMemcpyHostToDevice, st), w + ": upload");
+    uint64_t up = 0;  // stream bytes uploaded so far
+    for (size_t i = 0; i + 1 < t.size(); ++i) {
+        const uint32_t t0 = t[i], t1 = t[i + 1];
+        const bool last = i + 2 == t.size();
+        // tile offsets are checked to rise to the stream's end, so chunk i's tiles lie in [0, end)
+        const uint64_t end = last ? stream_total : std::min<uint64_t>(stream_total, 16ull * rd32(host + L.off_offsets + 4ull * t1));
+        if (end > up) {
+            EP_CUDA(cudaMemcpyAsync(d.stage_blob + L.off_stream + up, host + L.off_stream + up, end - up,
+                                    cudaMemcpyHostToDevice, st),
+                    w + ": upload");
+            up = end;
+        }
+        const int64_t v0 = int64_t(t0) * int64_t(per);
+        const int64_t v1 = last ? L.n_vectors : int64_t(t1) * int64_t(per);
+        const int64_t r0 = v0 / L.vec_per_row, r1 = last ? L.rows : v1 / L.vec_per_row;
+        uint8_t* dout = d.stage_out + size_t(r0) * row_bytes;
+        Params p = make_params(b, d.stage_blob, d.tables, dout, L.cols, d.status);
+        p.tile_off += t0;
+        p.alpha += r0;
+        p.rowmax += r0;
+        p.rows = r1 - r0;
+        p.n_vectors = v1 - v0;
+        p.n_tiles = t1 - t0;
+        if (host_sigma) p.sigma = d.stage_sigma + r0;
+        rc = launch(p, kind, L, vec_ok(L, dout, L.cols, out->dtype), Ctl(), st, dev, false);
+        if (rc != EP_OK) return rc;
+        EP_CUDA(cudaEventRecord(d.chunk_done[i], st), w + ": chunk event");
+        EP_CUDA(cudaStreamWaitEvent(cb, d.chunk_done[i], 0), w + ": chunk wait");
+        uint8_t* hout = static_cast<uint8_t*>(out->data) + size_t(r0) * size_t(out->row_stride) * es;
+        if (out->row_stride == L.cols)  // contiguous rows: one linear copy
+            EP_CUDA(cudaMemcpyAsync(hout, dout, size_t(r1 - r0) * row_bytes, cudaMemcpyDeviceToHost, cb),
+                    w + ": download");
+        else
+            EP_CUDA(cudaMemcpy2DAsync(hout, size_t(out->row_stride) * es, dout, row_bytes, row_bytes, size_t(r1 - r0),
+                                      cudaMemcpyDeviceToHost, cb),
+                    w + ": download");
+    }
+    if (host_sigma)
+        EP_CUDA(cudaMemcpyAsync(host_sigma, d.stage_sigma, 4 * size_t(L.rows), cudaMemcpyDeviceToHost, cb),
+                w + ": download");
+    EP_CUDA(cudaStreamSynchronize(cb), w + ": synchronise");
+    EP_CUDA(cudaStreamSynchronize(st), w + ": synchronise");
+    return EP_OK;
 }
 
 // ---- allocation-free decode (ep_decompress_noalloc) -------------------------------------------
@@ -262,24 +375,7 @@ extern "C" int ep_decompress(const ep_blob* cb, const ep_tensor* out, void* stre
         return launch(p, kind, L, vec, Ctl(), st, dev, true);
     }
 
-    // Host output: upload the bytes, decode into a blob-owned buffer, copy back, synchronise.
-    rc = ensure_device(b, dev, st);
-    if (rc != EP_OK) return rc;
-    const size_t es = size_t(dtype_bytes(out->dtype));
-    rc = ensure_staging(b, dev, size_t(L.rows) * size_t(L.cols) * es, false);
-    if (rc != EP_OK) return rc;
-    const DeviceCopy& d = b->dev[dev];
-    EP_CUDA(cudaMemcpyAsync(d.stage_blob, b->bytes.data(), b->bytes.size(), cudaMemcpyHostToDevice, st),
-            "ep_decompress: upload");
-    const bool vec = vec_ok(L, d.stage_out, L.cols, out->dtype);
-    Params p = make_params(b, d.stage_blob, d.tables, d.stage_out, L.cols, d.status);
-    rc = launch(p, kind, L, vec, Ctl(), st, dev, false);
-    if (rc != EP_OK) return rc;
-    EP_CUDA(cudaMemcpy2DAsync(out->data, size_t(out->row_stride) * es, d.stage_out, size_t(L.cols) * es,
-                              size_t(L.cols) * es, size_t(L.rows), cudaMemcpyDeviceToHost, st),
-            "ep_decompress: download");
-    EP_CUDA(cudaStreamSynchronize(st), "ep_decompress: synchronise");
-    return EP_OK;
+    return decode_to_host(b, out, kind, nullptr, st, dev, "ep_decompress");
 }
 
 extern "C" int ep_decompress_group(const ep_blob* const* blobs, const ep_tensor* outs, int n, void* stream) {
@@ -378,26 +474,7 @@ extern "C" int ep_decompress_fp8_rowscaled(const ep_blob* cb, const ep_tensor* o
         p.sigma = row_scale;
         return launch(p, kOutE4M3Row, L, vec, Ctl(), st, dev, true);
     }
-    // Host output and host row scales: upload the bytes, decode into blob-owned buffers, copy
-    // both back, synchronise.
-    rc = ensure_device(b, dev, st);
-    if (rc == EP_OK) rc = ensure_staging(b, dev, size_t(L.rows) * size_t(L.cols), true);
-    if (rc != EP_OK) return rc;
-    const DeviceCopy& d = b->dev[dev];
-    EP_CUDA(cudaMemcpyAsync(d.stage_blob, b->bytes.data(), b->bytes.size(), cudaMemcpyHostToDevice, st),
-            "ep_decompress_fp8_rowscaled: upload");
-    const bool vec = vec_ok(L, d.stage_out, L.cols, kE4M3);
-    Params p = make_params(b, d.stage_blob, d.tables, d.stage_out, L.cols, d.status);
-    p.sigma = d.stage_sigma;
-    rc = launch(p, kOutE4M3Row, L, vec, Ctl(), st, dev, false);
-    if (rc != EP_OK) return rc;
-    EP_CUDA(cudaMemcpy2DAsync(out->data, size_t(out->row_stride), d.stage_out, size_t(L.cols), size_t(L.cols),
-                              size_t(L.rows), cudaMemcpyDeviceToHost, st),
-            "ep_decompress_fp8_rowscaled: download");
-    EP_CUDA(cudaMemcpyAsync(row_scale, d.stage_sigma, 4 * size_t(L.rows), cudaMemcpyDeviceToHost, st),
-            "ep_decompress_fp8_rowscaled: download");
-    EP_CUDA(cudaStreamSynchronize(st), "ep_decompress_fp8_rowscaled: synchronise");
-    return EP_OK;
+    return decode_to_host(b, out, kOutE4M3Row, row_scale, st, dev, "ep_decompress_fp8_rowscaled");
 }
 
 extern "C" int ep_decode_fields(const ep_blob* cb, int16_t* fields, void* stream) {
@@ -469,6 +546,8 @@ extern "C" void ep_blob_free(ep_blob* b) {
         cudaFree(d.stage_blob);
         cudaFree(d.stage_out);
         cudaFree(d.stage_sigma);
+        for (cudaEvent_t e : d.chunk_done)
+            if (e) cudaEventDestroy(e);
     }
     if (b->host_pinned) cudaHostUnregister(b->bytes.data());
     cudaSetDevice(prev);

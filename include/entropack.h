@@ -122,11 +122,16 @@ int ep_compress_ex(const ep_tensor* in, double target_bpp, const ep_options* opt
  *           capture).  Later calls allocate nothing and do not synchronise.
  *           Host output (out->device == -1): end-to-end path on the current device -- copies the
  *           blob bytes host->device, decodes into a blob-owned device buffer, copies the result
- *           device->host into out->data, and synchronises `stream` before returning.
+ *           device->host into out->data, and returns when every row is there.  Blobs with 8 MB
+ *           of output or more go in up to 8 chunks of whole rows: uploads and decodes run on
+ *           `stream`, downloads on a copy-back stream the library keeps per device, so one
+ *           chunk's download overlaps the next chunk's upload and decode (page-locked host
+ *           memory lets the copies overlap; pageable memory works, slower).
  *   stream  cudaStream_t as void*.
  * Errors found on the GPU (corrupt tiles) are not returned here: read them with
  * ep_decode_status().  Returns EP_ERR_ARG, EP_ERR_SHAPE, EP_ERR_DTYPE, EP_ERR_CUDA, EP_ERR_OOM.
- * Not thread-safe for concurrent first calls on the same blob and device.
+ * Not thread-safe for concurrent first calls on the same blob and device, nor for concurrent
+ * host-output calls on the same blob (they share its staging buffers).
  */
 int ep_decompress(const ep_blob* b, const ep_tensor* out, void* stream);
 
@@ -167,7 +172,8 @@ int ep_decompress_group(const ep_blob* const* blobs, const ep_tensor* outs, int 
  *              the current device): one fused kernel launch on `stream`, asynchronous; the first
  *              call on a device copies the blob there (allocates and synchronises once).  Host
  *              output (out->device == -1): the end-to-end path of ep_decompress -- upload, decode
- *              into blob-owned buffers, copy payload and scales back, synchronise `stream`.
+ *              into blob-owned buffers, copy payload and scales back (in chunks of whole rows
+ *              like ep_decompress), return when both are there.
  *   row_scale  rows floats (4-byte aligned), written: device memory on the current device for a
  *              device output, host memory for a host output.
  *   stream     cudaStream_t as void*.

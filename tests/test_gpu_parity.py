@@ -310,6 +310,36 @@ def test_host_output_path_matches_device_path(ep):
     ep.decode_status(c)
 
 
+@pytest.mark.parametrize("rows,cols,dtype,rate,pinned,pad", [
+    (2048, 4096, W.BF16, 4.0, True, 0),     # 4 chunks; a tile is 2 rows, so every tile starts a row
+    (4104, 4099, W.BF16, 4.0, True, 0),     # ragged rows: a row-aligned unit is 513 tiles, the last
+                                            # chunk holds the 5 tiles left, the last one partial
+    (3072, 3072, W.FP16, 2.5, False, 24),   # 3 tiles per row-aligned unit; pageable, strided output
+])
+def test_host_output_chunks_match_device_path(ep, rows, cols, dtype, rate, pinned, pad):
+    """A host output of 8 MB or more comes back in chunks of whole rows, each downloaded while
+    the next is uploaded and decoded: the bytes equal the device path's for every chunk geometry,
+    and nothing outside the output's columns is written."""
+    g = np.random.Generator(np.random.PCG64(rows * 7 + cols))
+    x = g.normal(0, 0.02, (rows, cols))
+    bits = W.to_bf16_bits(x) if dtype == W.BF16 else W.to_fp16_bits(x)
+    c = ep.compress(W.bits_to_torch(bits, dtype), rate)
+    ref = _bits(_gpu_decode(ep, c), dtype)
+    tdt = TORCH[dtype]
+    big = torch.full((rows, cols + pad), 7.0, dtype=tdt)
+    if pinned:
+        big = big.pin_memory()
+    view = big[:, :cols]
+    ep.decompress(c, out=view)
+    ep.decode_status(c)
+    assert np.array_equal(_bits(view, dtype), ref)
+    if pad:
+        assert torch.all(big[:, cols:] == 7.0)
+    again = torch.empty((rows, cols), dtype=tdt).pin_memory()    # a second call reuses the staging
+    ep.decompress(c, out=again)
+    assert np.array_equal(_bits(again, dtype), ref)
+
+
 def test_side_stream(ep):
     m = W.small()
     c = ep.compress(W.bits_to_torch(m.bits, m.dtype), m.target_bpp)

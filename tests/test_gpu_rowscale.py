@@ -127,3 +127,16 @@ def test_rowscaled_host_output_path(ep):
     hs = torch.empty(c.shape[0], dtype=torch.float32)
     ep.decompress_fp8_rowscaled(c, out=hp, row_scale=hs)
     assert np.array_equal(hp.view(torch.uint8).numpy(), pay) and np.array_equal(hs.numpy(), sig)
+
+
+def test_rowscaled_host_output_in_chunks(ep):
+    """A 2048 x 4096 payload (8 MB) comes back in two chunks of whole rows: payload and scales
+    equal the device path's."""
+    m = W.square(rows=2048, cols=4096)
+    c = ep.compress(W.bits_to_torch(m.bits, m.dtype), m.target_bpp)
+    pay, sig = _gpu(ep, c)
+    hp = torch.empty(c.shape, dtype=torch.float8_e4m3fn).pin_memory()
+    hs = torch.empty(c.shape[0], dtype=torch.float32).pin_memory()
+    ep.decompress_fp8_rowscaled(c, out=hp, row_scale=hs)
+    ep.decode_status(c)
+    assert np.array_equal(hp.view(torch.uint8).numpy(), pay) and np.array_equal(hs.numpy(), sig)
