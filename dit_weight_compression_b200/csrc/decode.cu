@@ -45,18 +45,16 @@ const Launchers* launchers_for(int out_kind) {
     }
 }
 
-// One blob.  The 32-warp CTA runs only when there are more tiles than 16 warps per SM can hold at
-// once (the 16-warp kernel has twice the registers per thread) and every tile fits the smaller
-// buffer.
+// One blob, with the tables of its own layout (p.tables): 16-warp CTAs when they hold every tile
+// at once, else the widest whose buffers hold the largest tile.
 int launch(const Params& p, int out_kind, const BlobLayout& L, bool vec, const Ctl& ctl, cudaStream_t st, int device,
            bool dependent) {
     const LaunchCtx c{device, g_dev[device].sms};
     const int lay = blob_layout(L, device);
-    const bool wide = lay != 13 && L.max_tile_bytes <= tile_buffer_bytes(kWarpsWide, lay) &&
-                      p.n_tiles > uint32_t(kWarpsNarrow) * uint32_t(c.sms);
+    const int warps = cta_warps(lay, L.max_tile_bytes, p.n_tiles, uint64_t(c.sms));
     const Launchers* ln = launchers_for(out_kind);
     if (!ln) return set_error(EP_ERR_DTYPE, "decode: unsupported output container");
-    return ln->single(p, lay, vec, wide, L.has_escape != 0, ctl, st, c, dependent);
+    return ln->single(p, lay, vec, warps, L.has_escape != 0, ctl, st, c, dependent);
 }
 
 // Share `ctas` CTAs among blobs with tiles[i] tiles: every blob gets one, then each further CTA
@@ -140,39 +138,74 @@ TableSrc make_tablesrc(const ep_blob* b, const uint8_t* dblob) {
     return t;
 }
 
-// Device copy of the blob and its status word on `dev` (allocated and filled on first use).
+// The decode tables of layout `lay` in the device copy on `dev`, expanded on first use (one
+// allocation, one kernel on `st`, one synchronisation of `st`).  Call with b->mu held, after the
+// blob itself is on the device.
+int tables_locked(ep_blob* b, int dev, int lay, cudaStream_t st, const uint8_t*& out) {
+    DeviceCopy& d = b->dev[dev];
+    uint8_t*& slot = d.tables[layout_index(lay)];
+    if (!slot) {
+        uint8_t* tables = nullptr;
+        if (cudaMalloc(&tables, table_bytes(lay)) != cudaSuccess) {
+            cudaGetLastError();
+            return set_error(EP_ERR_OOM, "decode tables");
+        }
+        const TableSrc ts = make_tablesrc(b, d.blob);
+        auto fn = lay == 10 ? expand_tables_kernel<kWarpsWide, 10>
+                            : lay == 12 ? expand_tables_kernel<kWarpsWide, 12> : expand_tables_kernel<kWarpsWide, 13>;
+        const size_t smem =
+            lay == 10 ? sizeof(ExpandSmem<10>) : lay == 12 ? sizeof(ExpandSmem<12>) : sizeof(ExpandSmem<13>);
+        cudaError_t e = cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, int(smem));
+        if (e == cudaSuccess) {
+            fn<<<1, kWarpsWide * 32, smem, st>>>(ts, tables);
+            e = cudaGetLastError();
+        }
+        if (e == cudaSuccess) e = cudaStreamSynchronize(st);
+        if (e != cudaSuccess) {
+            cudaFree(tables);
+            return set_error(EP_ERR_CUDA, std::string("table expansion: ") + cudaGetErrorString(e));
+        }
+        slot = tables;
+    }
+    out = slot;
+    return EP_OK;
+}
+
+// Device copy of the blob, its status word and the tables of the layout its own decodes use on
+// `dev` (allocated and filled on first use).
 int ensure_device(ep_blob* b, int dev, cudaStream_t st) {
     std::lock_guard<std::mutex> g(b->mu);
     DeviceCopy& d = b->dev[dev];
-    if (d.blob) return EP_OK;
-    uint8_t* blob = nullptr;
-    uint8_t* tables = nullptr;
-    uint32_t* status = nullptr;
-    const int lay = blob_layout(b->layout, dev);
-    if (cudaMalloc(&blob, b->bytes.size()) != cudaSuccess || cudaMalloc(&tables, table_bytes(lay)) != cudaSuccess ||
-        cudaMalloc(&status, 16) != cudaSuccess) {
-        cudaFree(blob);
-        cudaFree(tables);
-        cudaFree(status);
-        cudaGetLastError();
-        return set_error(EP_ERR_OOM, "device copy of the blob");
+    if (!d.blob) {
+        uint8_t* blob = nullptr;
+        uint32_t* status = nullptr;
+        if (cudaMalloc(&blob, b->bytes.size()) != cudaSuccess || cudaMalloc(&status, 16) != cudaSuccess) {
+            cudaFree(blob);
+            cudaFree(status);
+            cudaGetLastError();
+            return set_error(EP_ERR_OOM, "device copy of the blob");
+        }
+        cudaError_t e = cudaMemcpyAsync(blob, b->bytes.data(), b->bytes.size(), cudaMemcpyHostToDevice, st);
+        if (e == cudaSuccess) e = cudaMemsetAsync(status, 0, 16, st);
+        if (e == cudaSuccess) e = cudaStreamSynchronize(st);
+        if (e != cudaSuccess) {
+            cudaFree(blob);
+            cudaFree(status);
+            return set_error(EP_ERR_CUDA, std::string("blob upload: ") + cudaGetErrorString(e));
+        }
+        d.blob = blob;
+        d.status = status;
     }
-    EP_CUDA(cudaMemcpyAsync(blob, b->bytes.data(), b->bytes.size(), cudaMemcpyHostToDevice, st), "blob upload");
-    EP_CUDA(cudaMemsetAsync(status, 0, 16, st), "status clear");
-    // expand the compact frequency tables once for this device copy
-    const TableSrc ts = make_tablesrc(b, blob);
-    auto fn = lay == 10 ? expand_tables_kernel<kWarpsWide, 10>
-                        : lay == 12 ? expand_tables_kernel<kWarpsWide, 12> : expand_tables_kernel<kWarpsWide, 13>;
-    const size_t smem = lay == 10 ? sizeof(ExpandSmem<10>) : lay == 12 ? sizeof(ExpandSmem<12>) : sizeof(ExpandSmem<13>);
-    EP_CUDA(cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, int(smem)),
-            "table expansion attribute");
-    fn<<<1, kWarpsWide * 32, smem, st>>>(ts, tables);
-    EP_CUDA(cudaGetLastError(), "table expansion launch");
-    EP_CUDA(cudaStreamSynchronize(st), "blob upload");
-    d.blob = blob;
-    d.tables = tables;
-    d.status = status;
-    return EP_OK;
+    const uint8_t* t = nullptr;
+    return tables_locked(b, dev, blob_layout(b->layout, dev), st, t);
+}
+
+// The device copy on `dev` and its tables of layout `lay`.
+int ensure_tables(ep_blob* b, int dev, int lay, cudaStream_t st, const uint8_t*& out) {
+    int rc = ensure_device(b, dev, st);
+    if (rc != EP_OK) return rc;
+    std::lock_guard<std::mutex> g(b->mu);
+    return tables_locked(b, dev, lay, st, out);
 }
 
 // Blob-owned staging buffers of the host-output path on `dev`: the per-call upload target, the
@@ -259,7 +292,8 @@ int decode_to_host(ep_blob* b, const ep_tensor* out, int kind, float* host_sigma
     const BlobLayout& L = b->layout;
     const size_t es = size_t(dtype_bytes(out->dtype));
     const size_t row_bytes = size_t(L.cols) * es;
-    int rc = ensure_device(b, dev, st);
+    const uint8_t* tables = nullptr;
+    int rc = ensure_tables(b, dev, blob_layout(L, dev), st, tables);
     if (rc == EP_OK) rc = ensure_staging(b, dev, row_bytes * size_t(L.rows), host_sigma != nullptr);
     cudaStream_t cb = nullptr;
     if (rc == EP_OK) rc = copyback_stream(dev, cb);
@@ -287,7 +321,7 @@ int decode_to_host(ep_blob* b, const ep_tensor* out, int kind, float* host_sigma
         const int64_t v1 = last ? L.n_vectors : int64_t(t1) * int64_t(per);
         const int64_t r0 = v0 / L.vec_per_row, r1 = last ? L.rows : v1 / L.vec_per_row;
         uint8_t* dout = d.stage_out + size_t(r0) * row_bytes;
-        Params p = make_params(b, d.stage_blob, d.tables, dout, L.cols, d.status);
+        Params p = make_params(b, d.stage_blob, tables, dout, L.cols, d.status);
         p.tile_off += t0;
         p.alpha += r0;
         p.rowmax += r0;
@@ -367,11 +401,12 @@ extern "C" int ep_decompress(const ep_blob* cb, const ep_tensor* out, void* stre
     if (out->device >= 0) {
         if (out->device != dev)
             return set_error(EP_ERR_ARG, "ep_decompress: output is not on the current device");
-        rc = ensure_device(b, dev, st);
+        const uint8_t* tables = nullptr;
+        rc = ensure_tables(b, dev, blob_layout(L, dev), st, tables);
         if (rc != EP_OK) return rc;
         const DeviceCopy& d = b->dev[dev];
         const bool vec = vec_ok(L, out->data, out->row_stride, out->dtype);
-        Params p = make_params(b, d.blob, d.tables, out->data, out->row_stride, d.status);
+        Params p = make_params(b, d.blob, tables, out->data, out->row_stride, d.status);
         return launch(p, kind, L, vec, Ctl(), st, dev, true);
     }
 
@@ -400,49 +435,65 @@ extern "C" int ep_decompress_group(const ep_blob* const* blobs, const ep_tensor*
             return set_error(EP_ERR_SHAPE, "ep_decompress_group: an output's shape differs from its blob's");
         if (o.row_stride < o.cols) return set_error(EP_ERR_ARG, "ep_decompress_group: row_stride < cols");
     }
-    for (int i = 0; i < n; ++i) {
-        rc = ensure_device(const_cast<ep_blob*>(blobs[i]), dev, st);
-        if (rc != EP_OK) return rc;
-    }
     const int sms = g_dev[dev].sms;
     const int chunk = std::max(1, std::min(kMaxGroup, sms));
-    // one launch per chunk of blobs that share a table layout
-    for (int lay : {13, 12, 10}) {
+    // Blobs of one frequency-total width go in chunks of up to `chunk` blobs, one launch each.  A
+    // chunk's layout and CTA width follow from its own tile count and largest tile, so every blob
+    // of the chunk needs that layout's tables: all are made ready before anything is launched.
+    struct Launch {
+        std::vector<int> idx;
+        int lay = 0, warps = 0;
+        uint32_t ctas = 0;
+        std::vector<uint32_t> share;
+        std::vector<const uint8_t*> tables;
+    };
+    std::vector<Launch> plan;
+    for (int pb : {12, 10}) {
         std::vector<int> idx;
         for (int i = 0; i < n; ++i)
-            if (blob_layout(blobs[i]->layout, dev) == lay) idx.push_back(i);
+            if (blobs[i]->layout.prob_bits == pb) idx.push_back(i);
         for (size_t c0 = 0; c0 < idx.size(); c0 += size_t(chunk)) {
-            const int cn = int(std::min(size_t(chunk), idx.size() - c0));
-            std::vector<uint32_t> tiles(static_cast<size_t>(cn));
+            Launch l;
+            l.idx.assign(idx.begin() + std::ptrdiff_t(c0), idx.begin() + std::ptrdiff_t(std::min(idx.size(), c0 + size_t(chunk))));
+            std::vector<uint32_t> tiles;
             uint64_t total = 0, max_tile = 0;
-            for (int i = 0; i < cn; ++i) {
-                const BlobLayout& L = blobs[idx[c0 + size_t(i)]]->layout;
-                tiles[size_t(i)] = L.n_tiles;
+            for (int i : l.idx) {
+                const BlobLayout& L = blobs[i]->layout;
+                tiles.push_back(L.n_tiles);
                 total += L.n_tiles;
                 max_tile = std::max<uint64_t>(max_tile, L.max_tile_bytes);
             }
-            const std::vector<uint32_t> g = share_ctas(tiles, uint32_t(sms));
-            GroupParams gp = {};
-            gp.n = uint32_t(cn);
-            uint32_t cta = 0;
-            for (int i = 0; i < cn; ++i) {
-                const ep_blob* b = blobs[idx[c0 + size_t(i)]];
-                const ep_tensor& o = outs[idx[c0 + size_t(i)]];
-                const DeviceCopy& d = b->dev[dev];
-                const bool vec = vec_ok(b->layout, o.data, o.row_stride, dtype);
-                GroupEntry& e = gp.e[i];
-                e.p = make_params(b, d.blob, d.tables, o.data, o.row_stride, d.status);
-                e.cta0 = cta;
-                e.ncta = g[size_t(i)];
-                e.vec = vec ? 1u : 0u;
-                e.esc = b->layout.has_escape ? 1u : 0u;
-                cta += e.ncta;
+            l.share = share_ctas(tiles, uint32_t(sms));
+            for (uint32_t g : l.share) l.ctas += g;
+            l.lay = table_layout(pb, max_tile, total, sms, true);
+            l.warps = cta_warps(l.lay, max_tile, total, l.ctas);
+            for (int i : l.idx) {
+                const uint8_t* t = nullptr;
+                rc = ensure_tables(const_cast<ep_blob*>(blobs[i]), dev, l.lay, st, t);
+                if (rc != EP_OK) return rc;
+                l.tables.push_back(t);
             }
-            const bool wide = lay != 13 && max_tile <= tile_buffer_bytes(kWarpsWide, lay) &&
-                              total > uint64_t(kWarpsNarrow) * uint64_t(cta);
-            rc = launchers_for(kind)->group(gp, lay, cta, wide, st, LaunchCtx{dev, sms});
-            if (rc != EP_OK) return rc;
+            plan.push_back(std::move(l));
         }
+    }
+    for (const Launch& l : plan) {
+        GroupParams gp = {};
+        gp.n = uint32_t(l.idx.size());
+        uint32_t cta = 0;
+        for (size_t k = 0; k < l.idx.size(); ++k) {
+            const ep_blob* b = blobs[l.idx[k]];
+            const ep_tensor& o = outs[l.idx[k]];
+            const DeviceCopy& d = b->dev[dev];
+            GroupEntry& e = gp.e[k];
+            e.p = make_params(b, d.blob, l.tables[k], o.data, o.row_stride, d.status);
+            e.cta0 = cta;
+            e.ncta = l.share[k];
+            e.vec = vec_ok(b->layout, o.data, o.row_stride, dtype) ? 1u : 0u;
+            e.esc = b->layout.has_escape ? 1u : 0u;
+            cta += e.ncta;
+        }
+        rc = launchers_for(kind)->group(gp, l.lay, cta, l.warps, st, LaunchCtx{dev, sms});
+        if (rc != EP_OK) return rc;
     }
     return EP_OK;
 }
@@ -466,11 +517,12 @@ extern "C" int ep_decompress_fp8_rowscaled(const ep_blob* cb, const ep_tensor* o
     if (out->device >= 0) {
         if (out->device != dev)
             return set_error(EP_ERR_ARG, "ep_decompress_fp8_rowscaled: output is not on the current device");
-        rc = ensure_device(b, dev, st);
+        const uint8_t* tables = nullptr;
+        rc = ensure_tables(b, dev, blob_layout(L, dev), st, tables);
         if (rc != EP_OK) return rc;
         const DeviceCopy& d = b->dev[dev];
         const bool vec = vec_ok(L, out->data, out->row_stride, kE4M3);
-        Params p = make_params(b, d.blob, d.tables, out->data, out->row_stride, d.status);
+        Params p = make_params(b, d.blob, tables, out->data, out->row_stride, d.status);
         p.sigma = row_scale;
         return launch(p, kOutE4M3Row, L, vec, Ctl(), st, dev, true);
     }
@@ -484,10 +536,11 @@ extern "C" int ep_decode_fields(const ep_blob* cb, int16_t* fields, void* stream
     cudaStream_t st = static_cast<cudaStream_t>(stream);
     int dev = 0;
     int rc = current_device(dev);
-    if (rc == EP_OK) rc = ensure_device(b, dev, st);
+    const uint8_t* tables = nullptr;
+    if (rc == EP_OK) rc = ensure_tables(b, dev, blob_layout(b->layout, dev), st, tables);
     if (rc != EP_OK) return rc;
     const DeviceCopy& d = b->dev[dev];
-    Params p = make_params(b, d.blob, d.tables, fields, b->layout.cols, d.status);
+    Params p = make_params(b, d.blob, tables, fields, b->layout.cols, d.status);
     return launch(p, kOutFields, b->layout, false, Ctl(), st, dev, false);
 }
 
@@ -498,11 +551,12 @@ extern "C" int ep_decode_wait_probe(const ep_blob* cb, uint32_t wait_spins, void
     cudaStream_t st = static_cast<cudaStream_t>(stream);
     int dev = 0;
     int rc = current_device(dev);
-    if (rc == EP_OK) rc = ensure_device(b, dev, st);
+    const uint8_t* tables = nullptr;
+    if (rc == EP_OK) rc = ensure_tables(b, dev, blob_layout(b->layout, dev), st, tables);
     if (rc != EP_OK) return rc;
     const DeviceCopy& d = b->dev[dev];
     // no tile is decoded and nothing is written: every CTA waits for bytes no copy delivers
-    Params p = make_params(b, d.blob, d.tables, nullptr, b->layout.cols, d.status);
+    Params p = make_params(b, d.blob, tables, nullptr, b->layout.cols, d.status);
     Ctl ctl;
     ctl.wait_spins = wait_spins;
     ctl.probe_tx = 16;
@@ -541,7 +595,7 @@ extern "C" void ep_blob_free(ep_blob* b) {
         if (!d.blob && !d.stage_blob && !d.stage_out) continue;
         cudaSetDevice(dv);
         cudaFree(d.blob);
-        cudaFree(d.tables);
+        for (uint8_t* t : d.tables) cudaFree(t);
         cudaFree(d.status);
         cudaFree(d.stage_blob);
         cudaFree(d.stage_out);

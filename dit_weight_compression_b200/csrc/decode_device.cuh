@@ -1256,34 +1256,40 @@ int launch_one(const Params& p, const Ctl& ctl, cudaStream_t st, const LaunchCtx
     return EP_OK;
 }
 
+template <int WARPS, int OUT, bool ESC, int LAY>
+int launch_vec(const Params& p, bool vec, const Ctl& ctl, cudaStream_t st, const LaunchCtx& c, bool dep) {
+    return vec ? launch_one<WARPS, OUT, true, ESC, LAY>(p, ctl, st, c, dep)
+               : launch_one<WARPS, OUT, false, ESC, LAY>(p, ctl, st, c, dep);
+}
+
 template <int OUT, bool ESC, int LAY>
-int launch_width(const Params& p, bool vec, bool wide, const Ctl& ctl, cudaStream_t st, const LaunchCtx& c, bool dep) {
-    if (LAY != 13 && wide)
-        return vec ? launch_one<kWarpsWide, OUT, true, ESC, LAY>(p, ctl, st, c, dep)
-                   : launch_one<kWarpsWide, OUT, false, ESC, LAY>(p, ctl, st, c, dep);
-    return vec ? launch_one<kWarpsNarrow, OUT, true, ESC, LAY>(p, ctl, st, c, dep)
-               : launch_one<kWarpsNarrow, OUT, false, ESC, LAY>(p, ctl, st, c, dep);
+int launch_width(const Params& p, bool vec, int warps, const Ctl& ctl, cudaStream_t st, const LaunchCtx& c, bool dep) {
+    if constexpr (LAY != 13) {
+        if (warps == kWarpsWide) return launch_vec<kWarpsWide, OUT, ESC, LAY>(p, vec, ctl, st, c, dep);
+        if (warps == kWarpsMid) return launch_vec<kWarpsMid, OUT, ESC, LAY>(p, vec, ctl, st, c, dep);
+    }
+    return launch_vec<kWarpsNarrow, OUT, ESC, LAY>(p, vec, ctl, st, c, dep);
 }
 
 template <int OUT, int LAY>
-int launch_esc(const Params& p, bool vec, bool wide, bool esc, const Ctl& ctl, cudaStream_t st, const LaunchCtx& c,
+int launch_esc(const Params& p, bool vec, int warps, bool esc, const Ctl& ctl, cudaStream_t st, const LaunchCtx& c,
                bool dep) {
     if constexpr (OUT == kOutFields) {  // test hook: the 16-warp kernel has the registers it needs
         return launch_one<kWarpsNarrow, kOutFields, false, true, LAY>(p, ctl, st, c, false);
     } else {
-        return esc ? launch_width<OUT, true, LAY>(p, vec, wide, ctl, st, c, dep)
-                   : launch_width<OUT, false, LAY>(p, vec, wide, ctl, st, c, dep);
+        return esc ? launch_width<OUT, true, LAY>(p, vec, warps, ctl, st, c, dep)
+                   : launch_width<OUT, false, LAY>(p, vec, warps, ctl, st, c, dep);
     }
 }
 
 // One blob.  esc: the blob's tables give the escape symbol a frequency (else the escape-free
 // kernel runs).
 template <int OUT>
-int launch_single(const Params& p, int lay, bool vec, bool wide, bool esc, const Ctl& ctl, cudaStream_t st,
+int launch_single(const Params& p, int lay, bool vec, int warps, bool esc, const Ctl& ctl, cudaStream_t st,
                   const LaunchCtx& c, bool dep) {
-    if (lay == 10) return launch_esc<OUT, 10>(p, vec, wide, esc, ctl, st, c, dep);
-    if (lay == 12) return launch_esc<OUT, 12>(p, vec, wide, esc, ctl, st, c, dep);
-    return launch_esc<OUT, 13>(p, vec, false, esc, ctl, st, c, dep);  // 16 warps only
+    if (lay == 10) return launch_esc<OUT, 10>(p, vec, warps, esc, ctl, st, c, dep);
+    if (lay == 12) return launch_esc<OUT, 12>(p, vec, warps, esc, ctl, st, c, dep);
+    return launch_esc<OUT, 13>(p, vec, kWarpsNarrow, esc, ctl, st, c, dep);  // 16 warps only
 }
 
 template <int WARPS, int OUT, int LAY>
@@ -1311,14 +1317,17 @@ int group_launch_one(const GroupParams& g, uint32_t grid, cudaStream_t st, const
 }
 
 // A set of blobs (one total width pb) over `grid` CTAs.
+template <int OUT, int LAY>
+int group_width(const GroupParams& g, uint32_t grid, int warps, cudaStream_t st, const LaunchCtx& c) {
+    if (warps == kWarpsWide) return group_launch_one<kWarpsWide, OUT, LAY>(g, grid, st, c);
+    if (warps == kWarpsMid) return group_launch_one<kWarpsMid, OUT, LAY>(g, grid, st, c);
+    return group_launch_one<kWarpsNarrow, OUT, LAY>(g, grid, st, c);
+}
+
 template <int OUT>
-int launch_group(const GroupParams& g, int lay, uint32_t grid, bool wide, cudaStream_t st, const LaunchCtx& c) {
-    if (lay == 10)
-        return wide ? group_launch_one<kWarpsWide, OUT, 10>(g, grid, st, c)
-                    : group_launch_one<kWarpsNarrow, OUT, 10>(g, grid, st, c);
-    if (lay == 12)
-        return wide ? group_launch_one<kWarpsWide, OUT, 12>(g, grid, st, c)
-                    : group_launch_one<kWarpsNarrow, OUT, 12>(g, grid, st, c);
+int launch_group(const GroupParams& g, int lay, uint32_t grid, int warps, cudaStream_t st, const LaunchCtx& c) {
+    if (lay == 10) return group_width<OUT, 10>(g, grid, warps, st, c);
+    if (lay == 12) return group_width<OUT, 12>(g, grid, warps, st, c);
     return group_launch_one<kWarpsNarrow, OUT, 13>(g, grid, st, c);  // 16 warps only
 }
 

@@ -113,10 +113,11 @@ constexpr uint32_t kSmemOptin = 232448;  // 227 KB: the largest dynamic shared m
 constexpr uint32_t kAlignSlack = 4096;    // the table starts on a 4 KB boundary of the shared window
 constexpr uint32_t kBufSlack = 80;        // bytes after a tile buffer that two steps may over-read
 
-// CTA widths: 32 or 16 warps, each warp with a tile buffer of Geo<WARPS, LAY>::kBuf bytes (5120 or
-// 10336 with layout 10, 4608 or 9296 with layout 12, 5840 with layout 13 and 16 warps); a tile
-// larger than its warp's buffer is read from global memory.
-constexpr int kWarpsWide = 32, kWarpsNarrow = 16;
+// CTA widths: 32, 24 or 16 warps, each warp with a tile buffer of Geo<WARPS, LAY>::kBuf bytes
+// (5120, 6848 or 10336 with layout 10; 4608, 6176 or 9296 with layout 12; 5840 with layout 13,
+// which leaves room for 16 warps only); a tile larger than its warp's buffer is read from global
+// memory.
+constexpr int kWarpsWide = 32, kWarpsMid = 24, kWarpsNarrow = 16;
 
 // Per-warp tile buffer size for a CTA of WARPS warps: what the 227 KB leave after the tables.
 template <int WARPS, int LAY>
@@ -136,27 +137,41 @@ using Smem32x10 = Smem<32, 10>;
 using Smem32x12 = Smem<32, 12>;
 static_assert(offsetof(Smem32x10, tbuf) == TableGeo<10>::kBytes && offsetof(Smem32x12, tbuf) == TableGeo<12>::kBytes,
               "table block must be contiguous");
-static_assert(sizeof(Smem<32, 10>) + kAlignSlack <= kSmemOptin && sizeof(Smem<16, 10>) + kAlignSlack <= kSmemOptin &&
-              sizeof(Smem<32, 12>) + kAlignSlack <= kSmemOptin && sizeof(Smem<16, 12>) + kAlignSlack <= kSmemOptin &&
+static_assert(sizeof(Smem<32, 10>) + kAlignSlack <= kSmemOptin && sizeof(Smem<24, 10>) + kAlignSlack <= kSmemOptin &&
+              sizeof(Smem<16, 10>) + kAlignSlack <= kSmemOptin && sizeof(Smem<32, 12>) + kAlignSlack <= kSmemOptin &&
+              sizeof(Smem<24, 12>) + kAlignSlack <= kSmemOptin && sizeof(Smem<16, 12>) + kAlignSlack <= kSmemOptin &&
               sizeof(Smem<16, 13>) + kAlignSlack <= kSmemOptin,
               "shared memory budget");
 inline uint32_t tile_buffer_bytes(int warps, int lay) {
-    if (lay == 10) return warps == 32 ? Geo<32, 10>::kBuf : Geo<16, 10>::kBuf;
-    if (lay == 12) return warps == 32 ? Geo<32, 12>::kBuf : Geo<16, 12>::kBuf;
+    if (lay == 10) return warps == 32 ? Geo<32, 10>::kBuf : warps == 24 ? Geo<24, 10>::kBuf : Geo<16, 10>::kBuf;
+    if (lay == 12) return warps == 32 ? Geo<32, 12>::kBuf : warps == 24 ? Geo<24, 12>::kBuf : Geo<16, 12>::kBuf;
     return Geo<16, 13>::kBuf;
 }
-// The layout a blob of n_tiles tiles decodes with on a device of `sms` SMs.  10-bit totals take
-// layout 10.  12-bit totals take layout 12 in 32-warp CTAs when there are more tiles than 16-warp
-// CTAs hold at once and every tile fits the 32-warp buffers (twice the independent rANS chains
-// per SM are worth the second lookup of three more symbols per vector); else the hybrid when every
-// tile fits its 16-warp buffers; else layout 12.  `wide_ok` false (a launch that runs 16-warp
-// CTAs only) skips the first rule.
+// Index of a layout's expanded tables in a device copy of a blob.
+inline int layout_index(int lay) { return lay == 10 ? 0 : lay == 12 ? 1 : 2; }
+constexpr int kLayouts = 3;
+
+// The layout a launch of n_tiles tiles (largest max_tile_bytes) decodes with on a device of `sms`
+// SMs.  10-bit totals take layout 10.  12-bit totals take layout 12 in 24- or 32-warp CTAs when
+// there are more tiles than 16-warp CTAs hold at once and every tile fits the 24-warp buffers
+// (more independent rANS chains per SM are worth the second lookup of three more symbols per
+// vector); else the hybrid when every tile fits its 16-warp buffers; else layout 12.  `wide_ok`
+// false (a launch that runs 16-warp CTAs only) skips the first rule.
 inline int table_layout(int prob_bits, uint64_t max_tile_bytes, uint64_t n_tiles, int sms, bool wide_ok) {
     if (prob_bits == 10) return 10;
     if (wide_ok && n_tiles > uint64_t(kWarpsNarrow) * uint64_t(sms > 0 ? sms : 0) &&
-        max_tile_bytes <= Geo<kWarpsWide, 12>::kBuf)
+        max_tile_bytes <= Geo<kWarpsMid, 12>::kBuf)
         return 12;
     return max_tile_bytes <= Geo<16, 13>::kBuf ? 13 : 12;
+}
+// The CTA width of such a launch over `ctas` CTAs: 16 warps when they hold every tile at once (the
+// 16-warp kernel has the most registers per thread); else the widest whose buffers hold the
+// largest tile (more chains per SM, fewer rounds of tiles); layout 13 runs 16 warps only.
+inline int cta_warps(int lay, uint64_t max_tile_bytes, uint64_t n_tiles, uint64_t ctas) {
+    if (lay == 13 || n_tiles <= uint64_t(kWarpsNarrow) * ctas) return kWarpsNarrow;
+    if (max_tile_bytes <= tile_buffer_bytes(kWarpsWide, lay)) return kWarpsWide;
+    if (max_tile_bytes <= tile_buffer_bytes(kWarpsMid, lay)) return kWarpsMid;
+    return kWarpsNarrow;
 }
 
 // ---- launch functions, one table per output container ----------------------------------------
@@ -165,13 +180,14 @@ struct LaunchCtx {
     int sms;     // its SM count
 };
 
-// Every function takes the blob's table layout lay (10, 12 or 13; 13 always runs 16 warps).
+// Every function takes the table layout lay (10, 12 or 13) and the CTA width in warps (16, 24 or
+// 32; layout 13 runs 16).
 struct Launchers {
     // one blob; `dependent`: launch as a programmatic dependent of the previous decode
-    int (*single)(const Params& p, int lay, bool vec, bool wide, bool esc, const Ctl& ctl, cudaStream_t st,
+    int (*single)(const Params& p, int lay, bool vec, int warps, bool esc, const Ctl& ctl, cudaStream_t st,
                   const LaunchCtx& c, bool dependent);
     // a set of blobs, all with the same layout, over `grid` CTAs
-    int (*group)(const GroupParams& g, int lay, uint32_t grid, bool wide, cudaStream_t st, const LaunchCtx& c);
+    int (*group)(const GroupParams& g, int lay, uint32_t grid, int warps, cudaStream_t st, const LaunchCtx& c);
     // one blob, tables expanded in every CTA, status in caller-provided memory; never allocates
     int (*noalloc)(const Params& p, const TableSrc& ts, int lay, bool vec, bool esc, cudaStream_t st,
                    const LaunchCtx& c);

@@ -149,7 +149,11 @@ int ep_decompress(const ep_blob* b, const ep_tensor* out, void* stream);
  *           same dtype.  Host outputs are not accepted.
  *   n       number of blobs; n == 0 does nothing.
  *   stream  cudaStream_t as void*; asynchronous like ep_decompress on device outputs.
- * The first call for a blob on a device copies it there (allocates and synchronises once).
+ * The first call for a blob on a device copies it there (allocates and synchronises once).  A
+ * launch's table layout and CTA width follow from the tile count and largest tile of the blobs it
+ * holds, so a set may need a blob's decode tables in a second layout: the first call that needs
+ * it expands them (one allocation and one synchronisation per blob, device and layout); repeat
+ * the call once before any stream capture.
  * Corrupt tiles are reported per blob by ep_decode_status().  Returns EP_ERR_ARG, EP_ERR_SHAPE,
  * EP_ERR_DTYPE, EP_ERR_CUDA, EP_ERR_OOM; nothing is launched when an argument is invalid.
  */
