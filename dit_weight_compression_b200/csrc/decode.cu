@@ -32,19 +32,6 @@ int blob_layout(const BlobLayout& L, int dev) {
     return table_layout(L.prob_bits, L.max_tile_bytes, L.n_tiles, g_dev[dev].sms, true);
 }
 
-const Launchers* launchers_for(int out_kind) {
-    switch (out_kind) {
-        case kOutBF16: return &kLaunchBF16;
-        case kOutFP16: return &kLaunchFP16;
-        case kOutE4M3: return &kLaunchE4M3;
-        case kOutF32: return &kLaunchF32;
-        case kOutI8: return &kLaunchI8;
-        case kOutFields: return &kLaunchFields;
-        case kOutE4M3Row: return &kLaunchE4M3Row;
-        default: return nullptr;
-    }
-}
-
 // One blob, with the tables of its own layout (p.tables): 16-warp CTAs when they hold every tile
 // at once, else the widest whose buffers hold the largest tile.
 int launch(const Params& p, int out_kind, const BlobLayout& L, bool vec, const Ctl& ctl, cudaStream_t st, int device,
@@ -52,9 +39,9 @@ int launch(const Params& p, int out_kind, const BlobLayout& L, bool vec, const C
     const LaunchCtx c{device, g_dev[device].sms};
     const int lay = blob_layout(L, device);
     const int warps = cta_warps(lay, L.max_tile_bytes, p.n_tiles, uint64_t(c.sms));
-    const Launchers* ln = launchers_for(out_kind);
-    if (!ln) return set_error(EP_ERR_DTYPE, "decode: unsupported output container");
-    return ln->single(p, lay, vec, warps, L.has_escape != 0, ctl, st, c, dependent);
+    const Launchers* ln = unit_launchers(out_kind, lay);
+    if (!ln || !ln->single) return set_error(EP_ERR_DTYPE, "decode: unsupported output container");
+    return ln->single(p, vec, warps, L.has_escape != 0, ctl, st, c, dependent);
 }
 
 // Share `ctas` CTAs among blobs with tiles[i] tiles: every blob gets one, then each further CTA
@@ -151,10 +138,12 @@ int tables_locked(ep_blob* b, int dev, int lay, cudaStream_t st, const uint8_t*&
             return set_error(EP_ERR_OOM, "decode tables");
         }
         const TableSrc ts = make_tablesrc(b, d.blob);
-        auto fn = lay == 10 ? expand_tables_kernel<kWarpsWide, 10>
-                            : lay == 12 ? expand_tables_kernel<kWarpsWide, 12> : expand_tables_kernel<kWarpsWide, 13>;
-        const size_t smem =
-            lay == 10 ? sizeof(ExpandSmem<10>) : lay == 12 ? sizeof(ExpandSmem<12>) : sizeof(ExpandSmem<13>);
+        auto fn = lay == 10   ? expand_tables_kernel<kWarpsWide, 10>
+                  : lay == 12 ? expand_tables_kernel<kWarpsWide, 12>
+                  : lay == 13 ? expand_tables_kernel<kWarpsWide, 13> : expand_tables_kernel<kWarpsWide, 14>;
+        const size_t smem = lay == 10   ? sizeof(ExpandSmem<10>)
+                            : lay == 12 ? sizeof(ExpandSmem<12>)
+                            : lay == 13 ? sizeof(ExpandSmem<13>) : sizeof(ExpandSmem<14>);
         cudaError_t e = cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, int(smem));
         if (e == cudaSuccess) {
             fn<<<1, kWarpsWide * 32, smem, st>>>(ts, tables);
@@ -492,7 +481,9 @@ extern "C" int ep_decompress_group(const ep_blob* const* blobs, const ep_tensor*
             e.esc = b->layout.has_escape ? 1u : 0u;
             cta += e.ncta;
         }
-        rc = launchers_for(kind)->group(gp, l.lay, cta, l.warps, st, LaunchCtx{dev, sms});
+        const Launchers* ln = unit_launchers(kind, l.lay);
+        if (!ln || !ln->group) return set_error(EP_ERR_DTYPE, "ep_decompress_group: unsupported output container");
+        rc = ln->group(gp, cta, l.warps, st, LaunchCtx{dev, sms});
         if (rc != EP_OK) return rc;
     }
     return EP_OK;
@@ -657,9 +648,10 @@ extern "C" int ep_decompress_noalloc(const ep_blob* cb, const void* device_blob,
     Params p = make_params(cb, static_cast<const uint8_t*>(device_blob), nullptr, out->data, out->row_stride,
                            status);
     const TableSrc ts = make_tablesrc(cb, static_cast<const uint8_t*>(device_blob));
-    // 16-warp CTAs only, so the layout choice ignores the 32-warp rule
-    int rc = launchers_for(kind)->noalloc(p, ts, table_layout(L.prob_bits, L.max_tile_bytes, L.n_tiles, 0, false), vec,
-                                          L.has_escape != 0, st, LaunchCtx{dev, g_noalloc[dev].sms});
+    // 16-warp CTAs only, and layouts 10, 12 and 13
+    const Launchers* ln = unit_launchers(kind, table_layout(L.prob_bits, L.max_tile_bytes, L.n_tiles, 1, false));
+    if (!ln || !ln->noalloc) return set_error_static(EP_ERR_DTYPE, "ep_decompress_noalloc: unsupported output dtype");
+    int rc = ln->noalloc(p, ts, vec, L.has_escape != 0, st, LaunchCtx{dev, g_noalloc[dev].sms});
     if (rc != EP_OK || !wait) return rc;
     uint32_t s = 0;
     if (cudaMemcpyAsync(&s, status, sizeof s, cudaMemcpyDeviceToHost, st) != cudaSuccess ||

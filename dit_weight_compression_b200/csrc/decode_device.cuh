@@ -97,20 +97,24 @@ struct Tab<12> {
     uint32_t e2;       // per-symbol entries
     uint32_t s1split;  // s1 + the slots of coset 0 in the joint table
 };
-// Layout 13 (12-bit totals, hybrid), at `base` (4 KB aligned): the joint table's direct words at
-// base, f2 and f3 given coset c at base + kHDirect (1 + 2c + j - 2); symbol bytes of f4..f8 given c
-// at base + kHL1 + 4096 (5c + j - 4); their 4-byte entries (as in layout 12) at
-// base + kHL2 + c (5 * 1024 + kCosetSkew) + 1024 (j - 4).  A direct word of
-// slot u holding s:
+// Layouts 13 and 14 (12-bit totals, hybrid with D = Hybrid<LAY>::kND direct fields per coset and
+// B = 7 - D two-lookup ones), at `base` (4 KB aligned): the joint table's direct words at base;
+// field j = 2 .. D + 1 given coset c at base + kHDirect (1 + D c + j - 2); symbol bytes of field
+// j = D + 2 .. 8 given c at base + kL1 + 4096 (B c + j - D - 2); their 4-byte entries (as in
+// layout 12) at base + kL2 + c (B * 1024 + kCosetSkew) + 1024 (j - D - 2).  A direct word of slot
+// u holding s:
 //   bits  0..11  u - cum(s)
 //   bits 12..19  s
 //   bits 20..31  q(s) - 1
 // so x <- (q - 1) (x >> 12) + (x >> 12) + (u - cum(s)).
-template <>
-struct Tab<13> {
+struct TabHybrid {
     uint32_t base;
     uint32_t split;    // slots of coset 0 in the joint table
 };
+template <>
+struct Tab<13> : TabHybrid {};
+template <>
+struct Tab<14> : TabHybrid {};
 __device__ __forceinline__ uint32_t pack_direct(uint32_t off, uint32_t s, uint32_t q) {
     return q ? off | (s << 12) | ((q - 1) << 20) : 0u;
 }
@@ -266,10 +270,11 @@ __device__ __forceinline__ uint32_t pack_entry(uint32_t bias, uint32_t s, uint32
            (coset << kEntryCosetShift) | (q << kEntryQShift);
 }
 
-// Layout 13 from the per-context frequencies and cumulative frequencies in `scr`: the 5 direct
-// tables, the 10 symbol-byte tables, then the 4-byte entries of those 10.
-template <int WARPS>
+// Layout 13 or 14 from the per-context frequencies and cumulative frequencies in `scr`: the
+// 1 + 2D direct tables, the 2B symbol-byte tables, then the 4-byte entries of those 2B.
+template <int WARPS, int LAY>
 __device__ void build_hybrid(uint8_t* tab, const BuildScratch& scr) {
+    constexpr uint32_t D = Hybrid<LAY>::kND, B = Hybrid<LAY>::kNB;
     const uint32_t lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
     constexpr int P = WARPS >= 15 ? WARPS / 15 : 1;
     constexpr uint32_t kSlotsPerPart = 4096u / P;
@@ -288,15 +293,16 @@ __device__ void build_hybrid(uint8_t* tab, const BuildScratch& scr) {
             }
             continue;
         }
-        // ti 1..4: f2, f3 given c (direct); ti 5..14: f4..f8 given c (symbol bytes)
-        const bool direct = ti < 5;
-        const uint32_t c = direct ? (ti - 1) / 2 : (ti - 5) / 5;
-        const uint32_t j = direct ? 2 + (ti - 1) % 2 : 4 + (ti - 5) % 5;
+        // ti 1..2D: f2..f(D+1) given c (direct); ti 2D+1..14: f(D+2)..f8 given c (symbol bytes)
+        const bool direct = ti <= 2 * D;
+        const uint32_t k = direct ? ti - 1 : ti - 1 - 2 * D;
+        const uint32_t c = direct ? k / D : k / B;
+        const uint32_t j = direct ? 2 + k % D : 2 + D + k % B;
         const uint32_t ctx = 8 * c + j - 1;
         const uint16_t* cum = scr.cum[ctx];
         const uint16_t* qs = scr.q[ctx];
         uint32_t* dst32 = direct ? dir + ti * 4096u : nullptr;
-        uint8_t* dst8 = direct ? nullptr : tab + kHL1 + (ti - 5) * kCtxBytes;
+        uint8_t* dst8 = direct ? nullptr : tab + Hybrid<LAY>::kL1 + k * kCtxBytes;
         if (cum[256] != 4096u) {  // context never used by this blob (the host checked the rest)
             for (uint32_t w = lane; w < kSlotsPerPart; w += 32) {
                 if (direct) dst32[part * kSlotsPerPart + w] = 0;
@@ -318,11 +324,11 @@ __device__ void build_hybrid(uint8_t* tab, const BuildScratch& scr) {
             else dst8[slot] = uint8_t(sy);
         }
     }
-    for (uint32_t i = threadIdx.x; i < 10 * 256; i += WARPS * 32) {
-        const uint32_t row = i >> 8, sy = i & 255;        // row = 5c + j - 4
-        const uint32_t c = row / 5, ctx = 8 * c + 3 + row % 5;
+    for (uint32_t i = threadIdx.x; i < 2 * B * 256; i += WARPS * 32) {
+        const uint32_t row = i >> 8, sy = i & 255;        // row = B c + j - D - 2
+        const uint32_t c = row / B, ctx = 8 * c + 1 + D + row % B;
         const uint32_t q = scr.q[ctx][sy];
-        uint32_t* ent = reinterpret_cast<uint32_t*>(tab + kHL2 + c * kCosetSkew + 1024 * row);
+        uint32_t* ent = reinterpret_cast<uint32_t*>(tab + Hybrid<LAY>::kL2 + c * kCosetSkew + 1024 * row);
         ent[sy] = q ? (q << kE12QShift) | uint32_t(scr.cum[ctx][sy]) : 0u;
     }
 }
@@ -363,8 +369,8 @@ __device__ void build_tables(uint8_t* tab, BuildScratch& scr, const TableSrc& p)
         if (lane == 31) scr.cum[ctx][256] = uint16_t(min(c, 0xFFFFu));
     }
     __syncthreads();
-    if constexpr (LAY == 13) {
-        build_hybrid<WARPS>(tab, scr);
+    if constexpr (is_hybrid(LAY)) {
+        build_hybrid<WARPS, LAY>(tab, scr);
         return;
     }
     // (b) slot -> entry (10-bit: the packed word; 12-bit: the symbol byte).  Lane l of a warp
@@ -676,9 +682,12 @@ __device__ __forceinline__ void step_symbols12(const Tab<12>& T, Reader& rd, uin
     }
 }
 
-// Layout 13: (coset, f1), f2 and f3 from direct words (one load each), f4..f8 as in layout 12.
-template <bool ESC, bool FULL, class Reader>
-__device__ __forceinline__ void step_symbols13(const Tab<13>& T, Reader& rd, uint32_t& x, bool active, StepSyms& s) {
+// Layouts 13 and 14: (coset, f1) and the next D fields from direct words (one load each), the
+// rest as in layout 12.
+template <int LAY, bool ESC, bool FULL, class Reader>
+__device__ __forceinline__ void step_symbols_hybrid(const Tab<LAY>& T, Reader& rd, uint32_t& x, bool active,
+                                                    StepSyms& s) {
+    constexpr uint32_t D = Hybrid<LAY>::kND, B = Hybrid<LAY>::kNB;
     if (FULL) active = true;
     uint32_t* e = s.e;
     uint32_t acc = 0;                          // largest symbol: the escape symbol is the largest
@@ -698,7 +707,7 @@ __device__ __forceinline__ void step_symbols13(const Tab<13>& T, Reader& rd, uin
         if (ESC) acc = sy;
     }
     s.c = c;
-    const uint32_t bd = T.base + kHDirect + c * (2u * kHDirect);   // f2 given c; f3 follows
+    const uint32_t bd = T.base + kHDirect + c * (D * kHDirect);    // f2 given c; f3 (f4) follow
 #define EP_FIELD13D(j)                                                                        \
     {                                                                                         \
         const uint32_t sy = direct(lds_u32<((j) - 1) * kHDirect>(bd + 4u * (x & 4095u)));     \
@@ -707,20 +716,22 @@ __device__ __forceinline__ void step_symbols13(const Tab<13>& T, Reader& rd, uin
         if (ESC) acc = max(acc, sy);                                                          \
     }
     EP_FIELD13D(1) EP_FIELD13D(2)
+    if constexpr (D == 3) EP_FIELD13D(3)
 #undef EP_FIELD13D
-    const uint32_t b1 = T.base + kHL1 + c * (5u * kCtxBytes);      // f4's symbol bytes given c
-    const uint32_t b2 = T.base + kHL2 + c * (5u * 1024u + kCosetSkew);  // f4's entries given c
+    const uint32_t b1 = T.base + Hybrid<LAY>::kL1 + c * (B * kCtxBytes);            // first two-lookup field's bytes
+    const uint32_t b2 = T.base + Hybrid<LAY>::kL2 + c * (B * 1024u + kCosetSkew);   // and its entries
 #define EP_FIELD13(j)                                                                         \
     {                                                                                         \
         const uint32_t u = x & 4095u;                                                         \
-        const uint32_t sy = lds_u8<((j) - 3) * kCtxBytes>(u | b1);                            \
-        const uint32_t en = lds_u32<((j) - 3) * 1024>(b2 + 4u * sy);                          \
+        const uint32_t sy = lds_u8<((j) - 1 - D) * kCtxBytes>(u | b1);                        \
+        const uint32_t en = lds_u32<((j) - 1 - D) * 1024>(b2 + 4u * sy);                      \
         if (active) x = (en >> kE12QShift) * (x >> 12) + (u - (en & kE12CumMask));            \
         renorm_step<FULL>(x, rd, active);                                                     \
         e[j] = sy;                                                                            \
         if (ESC) acc = max(acc, sy);                                                          \
     }
-    EP_FIELD13(3) EP_FIELD13(4) EP_FIELD13(5) EP_FIELD13(6) EP_FIELD13(7)
+    if constexpr (D == 2) EP_FIELD13(3)
+    EP_FIELD13(4) EP_FIELD13(5) EP_FIELD13(6) EP_FIELD13(7)
 #undef EP_FIELD13
 
     s.from_symbols = true;
@@ -744,7 +755,7 @@ template <int LAY, bool ESC, bool FULL, class Reader>
 __device__ __forceinline__ void step_symbols(const Tab<LAY>& tab, Reader& rd, uint32_t& x, bool active, StepSyms& s) {
     if constexpr (LAY == 10) step_symbols10<ESC, FULL>(tab.t, rd, x, active, s);
     else if constexpr (LAY == 12) step_symbols12<ESC, FULL>(tab, rd, x, active, s);
-    else step_symbols13<ESC, FULL>(tab, rd, x, active, s);
+    else step_symbols_hybrid<LAY, ESC, FULL>(tab, rd, x, active, s);
 }
 
 // Symbol s_j of a decoded step (entry layout of the total).
@@ -1070,7 +1081,7 @@ __device__ __forceinline__ void decode_ctas(const Params& p, const TableSrc* ts,
         Tab<LAY> tab;
         if constexpr (LAY == 10) {
             tab.t = smem_u32(sm.tab);
-        } else if constexpr (LAY == 13) {
+        } else if constexpr (is_hybrid(LAY)) {
             tab.base = smem_u32(sm.tab);
             tab.split = p.joint_split;
         } else {
@@ -1264,10 +1275,12 @@ int launch_vec(const Params& p, bool vec, const Ctl& ctl, cudaStream_t st, const
 
 template <int OUT, bool ESC, int LAY>
 int launch_width(const Params& p, bool vec, int warps, const Ctl& ctl, cudaStream_t st, const LaunchCtx& c, bool dep) {
-    if constexpr (LAY != 13) {
+    if constexpr (!is_hybrid(LAY)) {  // layout 13 leaves room for 16 or 20 warps, layout 14 for 16
         if (warps == kWarpsWide) return launch_vec<kWarpsWide, OUT, ESC, LAY>(p, vec, ctl, st, c, dep);
         if (warps == kWarpsMid) return launch_vec<kWarpsMid, OUT, ESC, LAY>(p, vec, ctl, st, c, dep);
     }
+    if constexpr (LAY != 14)
+        if (warps == kWarps20) return launch_vec<kWarps20, OUT, ESC, LAY>(p, vec, ctl, st, c, dep);
     return launch_vec<kWarpsNarrow, OUT, ESC, LAY>(p, vec, ctl, st, c, dep);
 }
 
@@ -1280,16 +1293,6 @@ int launch_esc(const Params& p, bool vec, int warps, bool esc, const Ctl& ctl, c
         return esc ? launch_width<OUT, true, LAY>(p, vec, warps, ctl, st, c, dep)
                    : launch_width<OUT, false, LAY>(p, vec, warps, ctl, st, c, dep);
     }
-}
-
-// One blob.  esc: the blob's tables give the escape symbol a frequency (else the escape-free
-// kernel runs).
-template <int OUT>
-int launch_single(const Params& p, int lay, bool vec, int warps, bool esc, const Ctl& ctl, cudaStream_t st,
-                  const LaunchCtx& c, bool dep) {
-    if (lay == 10) return launch_esc<OUT, 10>(p, vec, warps, esc, ctl, st, c, dep);
-    if (lay == 12) return launch_esc<OUT, 12>(p, vec, warps, esc, ctl, st, c, dep);
-    return launch_esc<OUT, 13>(p, vec, kWarpsNarrow, esc, ctl, st, c, dep);  // 16 warps only
 }
 
 template <int WARPS, int OUT, int LAY>
@@ -1319,16 +1322,13 @@ int group_launch_one(const GroupParams& g, uint32_t grid, cudaStream_t st, const
 // A set of blobs (one total width pb) over `grid` CTAs.
 template <int OUT, int LAY>
 int group_width(const GroupParams& g, uint32_t grid, int warps, cudaStream_t st, const LaunchCtx& c) {
-    if (warps == kWarpsWide) return group_launch_one<kWarpsWide, OUT, LAY>(g, grid, st, c);
-    if (warps == kWarpsMid) return group_launch_one<kWarpsMid, OUT, LAY>(g, grid, st, c);
+    if constexpr (!is_hybrid(LAY)) {
+        if (warps == kWarpsWide) return group_launch_one<kWarpsWide, OUT, LAY>(g, grid, st, c);
+        if (warps == kWarpsMid) return group_launch_one<kWarpsMid, OUT, LAY>(g, grid, st, c);
+    }
+    if constexpr (LAY != 14)
+        if (warps == kWarps20) return group_launch_one<kWarps20, OUT, LAY>(g, grid, st, c);
     return group_launch_one<kWarpsNarrow, OUT, LAY>(g, grid, st, c);
-}
-
-template <int OUT>
-int launch_group(const GroupParams& g, int lay, uint32_t grid, int warps, cudaStream_t st, const LaunchCtx& c) {
-    if (lay == 10) return group_width<OUT, 10>(g, grid, warps, st, c);
-    if (lay == 12) return group_width<OUT, 12>(g, grid, warps, st, c);
-    return group_launch_one<kWarpsNarrow, OUT, 13>(g, grid, st, c);  // 16 warps only
 }
 
 // The allocation-free decode: tables expanded in every CTA, the status word in caller-provided
@@ -1358,20 +1358,27 @@ int noalloc_esc(const Params& p, const TableSrc& ts, bool vec, bool esc, cudaStr
                : noalloc_launch_one<kWarpsNarrow, OUT, false, false, LAY>(p, ts, st, c);
 }
 
-template <int OUT>
-int launch_noalloc(const Params& p, const TableSrc& ts, int lay, bool vec, bool esc, cudaStream_t st,
-                   const LaunchCtx& c) {
-    if (lay == 10) return noalloc_esc<OUT, 10>(p, ts, vec, esc, st, c);
-    if (lay == 12) return noalloc_esc<OUT, 12>(p, ts, vec, esc, st, c);
-    return noalloc_esc<OUT, 13>(p, ts, vec, esc, st, c);
+// The launch table of one output container and one table layout (each unit compiled from
+// decode_unit.cu defines one).  esc: the blob's tables give the escape symbol a frequency (else
+// the escape-free kernel runs).
+template <int OUT, int LAY>
+int unit_single(const Params& p, bool vec, int warps, bool esc, const Ctl& ctl, cudaStream_t st, const LaunchCtx& c,
+                bool dep) {
+    return launch_esc<OUT, LAY>(p, vec, warps, esc, ctl, st, c, dep);
 }
-
-// The launch table of one output container (each decode_<container>.cu defines one).
-// (The fields test hook and the row-scaled FP8 container are single-blob launches only.)
-template <int OUT>
+template <int OUT, int LAY>
+int unit_group(const GroupParams& g, uint32_t grid, int warps, cudaStream_t st, const LaunchCtx& c) {
+    return group_width<OUT, LAY>(g, grid, warps, st, c);
+}
+template <int OUT, int LAY>
+int unit_noalloc(const Params& p, const TableSrc& ts, bool vec, bool esc, cudaStream_t st, const LaunchCtx& c) {
+    return noalloc_esc<OUT, LAY>(p, ts, vec, esc, st, c);
+}
+template <int OUT, int LAY>
 constexpr Launchers make_launchers() {
-    if constexpr (OUT == kOutFields || OUT == kOutE4M3Row) return Launchers{&launch_single<OUT>, nullptr, nullptr};
-    else return Launchers{&launch_single<OUT>, &launch_group<OUT>, &launch_noalloc<OUT>};
+    if constexpr (OUT == kOutFields || OUT == kOutE4M3Row) return Launchers{&unit_single<OUT, LAY>, nullptr, nullptr};
+    else if constexpr (LAY == 14) return Launchers{&unit_single<OUT, LAY>, &unit_group<OUT, LAY>, nullptr};
+    else return Launchers{&unit_single<OUT, LAY>, &unit_group<OUT, LAY>, &unit_noalloc<OUT, LAY>};
 }
 
 }  // namespace

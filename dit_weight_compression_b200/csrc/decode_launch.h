@@ -28,24 +28,35 @@ constexpr uint32_t kSlotBytes = kDecodeTables * kCtxBytes;    // 61440
 // warp whose lanes read the same symbol of the same field in both cosets hits different banks.
 constexpr uint32_t kCosetSkew = 64;
 constexpr uint32_t kSymEntryBytes = 16 * 256 * 4 + kCosetSkew;  // 16448 (12-bit totals only)
-// 12-bit totals, hybrid: the joint table and f2, f3 given each coset as direct words, one u32 per
-// slot (5 tables of 16 KB), the other 10 tables as symbol bytes (4 KB each) and 4-byte entries
-// (1 KB each) -- 130 KB, which leaves 16-warp CTAs 5.8 KB tile buffers.
+// 12-bit totals, hybrid layouts 13 and 14: the joint table and the next kND fields (f2, f3 for
+// layout 13; f2, f3, f4 for layout 14) given each coset as direct words, one u32 per slot (16 KB
+// a table); the other 7 - kND fields given each coset as symbol bytes (4 KB a table) and 4-byte
+// per-symbol entries (1 KB a table).  Layout 13 takes 130 KB, layout 14 152 KB.
 constexpr uint32_t kHDirect = 4 * 4096;                       // one direct table: 16384
-constexpr uint32_t kHL1 = 5 * kHDirect;                       // 81920: symbol bytes of f4..f8
-constexpr uint32_t kHL2 = kHL1 + 10 * kCtxBytes;              // 122880: their 4-byte entries
-constexpr uint32_t kHybridBytes = kHL2 + 10 * 1024 + kCosetSkew;  // 133184
+template <int LAY>
+struct Hybrid {
+    static constexpr uint32_t kND = LAY == 14 ? 3 : 2;         // direct fields per coset after the joint table
+    static constexpr uint32_t kNB = 7 - kND;                   // two-lookup fields per coset
+    static constexpr uint32_t kL1 = (1 + 2 * kND) * kHDirect;  // their symbol bytes (81920 / 114688)
+    static constexpr uint32_t kL2 = kL1 + 2 * kNB * kCtxBytes; // their 4-byte entries (122880 / 147456)
+    static constexpr uint32_t kBytes = kL2 + 2 * kNB * 1024 + kCosetSkew;  // 133184 / 155712
+};
+__host__ __device__ constexpr bool is_hybrid(int lay) { return lay == 13 || lay == 14; }
 
 // Table layouts: 10 = 10-bit totals, one packed word per slot; 12 = 12-bit totals, two lookups
-// per symbol; 13 = 12-bit totals, hybrid (16-warp CTAs only).
+// per symbol; 13 and 14 = 12-bit totals, hybrid.
 template <int LAY>
 struct TableGeo {
-    static_assert(LAY == 10 || LAY == 12 || LAY == 13, "table layouts are 10, 12 and 13");
-    static constexpr uint32_t kBytes = LAY == 10 ? kSlotBytes : LAY == 12 ? kSlotBytes + kSymEntryBytes : kHybridBytes;
+    static_assert(LAY == 10 || LAY == 12 || LAY == 13 || LAY == 14, "table layouts are 10, 12, 13 and 14");
+    static constexpr uint32_t kBytes =
+        LAY == 10 ? kSlotBytes : LAY == 12 ? kSlotBytes + kSymEntryBytes : Hybrid<LAY>::kBytes;
     static constexpr uint32_t kPiece = kBytes / 4;             // bytes per table bulk copy
+    static_assert(kPiece % 16 == 0, "bulk copies move multiples of 16 bytes");
 };
 inline uint32_t table_bytes(int lay) {
-    return lay == 10 ? TableGeo<10>::kBytes : lay == 12 ? TableGeo<12>::kBytes : TableGeo<13>::kBytes;
+    return lay == 10 ? TableGeo<10>::kBytes
+         : lay == 12 ? TableGeo<12>::kBytes
+         : lay == 13 ? TableGeo<13>::kBytes : TableGeo<14>::kBytes;
 }
 
 // kOutE4M3Row: the FP8 container with a per-row scale -- an E4M3 payload normalised per row to
@@ -113,11 +124,12 @@ constexpr uint32_t kSmemOptin = 232448;  // 227 KB: the largest dynamic shared m
 constexpr uint32_t kAlignSlack = 4096;    // the table starts on a 4 KB boundary of the shared window
 constexpr uint32_t kBufSlack = 80;        // bytes after a tile buffer that two steps may over-read
 
-// CTA widths: 32, 24 or 16 warps, each warp with a tile buffer of Geo<WARPS, LAY>::kBuf bytes
-// (5120, 6848 or 10336 with layout 10; 4608, 6176 or 9296 with layout 12; 5840 with layout 13,
-// which leaves room for 16 warps only); a tile larger than its warp's buffer is read from global
-// memory.
-constexpr int kWarpsWide = 32, kWarpsMid = 24, kWarpsNarrow = 16;
+// CTA widths: 16, 20, 24 or 32 warps, each warp with a tile buffer of Geo<WARPS, LAY>::kBuf bytes:
+//   layout 10: 10336, 8240, 6848, 5120;  layout 12: 9296, 7424, 6176, 4608;  layout 13: 5840, 4656;
+//   layout 14: 4432
+// (layout 13 leaves room for 16 or 20 warps, layout 14 for 16).  A tile larger than its warp's
+// buffer is read from global memory.
+constexpr int kWarpsNarrow = 16, kWarps20 = 20, kWarpsMid = 24, kWarpsWide = 32;
 
 // Per-warp tile buffer size for a CTA of WARPS warps: what the 227 KB leave after the tables.
 template <int WARPS, int LAY>
@@ -137,63 +149,137 @@ using Smem32x10 = Smem<32, 10>;
 using Smem32x12 = Smem<32, 12>;
 static_assert(offsetof(Smem32x10, tbuf) == TableGeo<10>::kBytes && offsetof(Smem32x12, tbuf) == TableGeo<12>::kBytes,
               "table block must be contiguous");
-static_assert(sizeof(Smem<32, 10>) + kAlignSlack <= kSmemOptin && sizeof(Smem<24, 10>) + kAlignSlack <= kSmemOptin &&
-              sizeof(Smem<16, 10>) + kAlignSlack <= kSmemOptin && sizeof(Smem<32, 12>) + kAlignSlack <= kSmemOptin &&
-              sizeof(Smem<24, 12>) + kAlignSlack <= kSmemOptin && sizeof(Smem<16, 12>) + kAlignSlack <= kSmemOptin &&
-              sizeof(Smem<16, 13>) + kAlignSlack <= kSmemOptin,
+template <int WARPS, int LAY>
+constexpr bool fits_smem() { return sizeof(Smem<WARPS, LAY>) + kAlignSlack <= kSmemOptin; }
+static_assert(fits_smem<16, 10>() && fits_smem<20, 10>() && fits_smem<24, 10>() && fits_smem<32, 10>() &&
+              fits_smem<16, 12>() && fits_smem<20, 12>() && fits_smem<24, 12>() && fits_smem<32, 12>() &&
+              fits_smem<16, 13>() && fits_smem<20, 13>() && fits_smem<16, 14>(),
               "shared memory budget");
+inline bool width_ok(int warps, int lay) {
+    if (lay == 14) return warps == kWarpsNarrow;
+    return warps == kWarpsNarrow || warps == kWarps20 || (lay != 13 && (warps == kWarpsMid || warps == kWarpsWide));
+}
 inline uint32_t tile_buffer_bytes(int warps, int lay) {
-    if (lay == 10) return warps == 32 ? Geo<32, 10>::kBuf : warps == 24 ? Geo<24, 10>::kBuf : Geo<16, 10>::kBuf;
-    if (lay == 12) return warps == 32 ? Geo<32, 12>::kBuf : warps == 24 ? Geo<24, 12>::kBuf : Geo<16, 12>::kBuf;
-    return Geo<16, 13>::kBuf;
+    switch (lay * 100 + warps) {
+        case 1016: return Geo<16, 10>::kBuf;
+        case 1020: return Geo<20, 10>::kBuf;
+        case 1024: return Geo<24, 10>::kBuf;
+        case 1032: return Geo<32, 10>::kBuf;
+        case 1216: return Geo<16, 12>::kBuf;
+        case 1220: return Geo<20, 12>::kBuf;
+        case 1224: return Geo<24, 12>::kBuf;
+        case 1232: return Geo<32, 12>::kBuf;
+        case 1316: return Geo<16, 13>::kBuf;
+        case 1320: return Geo<20, 13>::kBuf;
+        case 1416: return Geo<16, 14>::kBuf;
+        default: return 0;
+    }
 }
 // Index of a layout's expanded tables in a device copy of a blob.
-inline int layout_index(int lay) { return lay == 10 ? 0 : lay == 12 ? 1 : 2; }
-constexpr int kLayouts = 3;
+inline int layout_index(int lay) { return lay == 10 ? 0 : lay == 12 ? 1 : lay == 13 ? 2 : 3; }
+constexpr int kLayouts = 4;
 
-// The layout a launch of n_tiles tiles (largest max_tile_bytes) decodes with on a device of `sms`
-// SMs.  10-bit totals take layout 10.  12-bit totals take layout 12 in 24- or 32-warp CTAs when
-// there are more tiles than 16-warp CTAs hold at once and every tile fits the 24-warp buffers
-// (more independent rANS chains per SM are worth the second lookup of three more symbols per
-// vector); else the hybrid when every tile fits its 16-warp buffers; else layout 12.  `wide_ok`
-// false (a launch that runs 16-warp CTAs only) skips the first rule.
-inline int table_layout(int prob_bits, uint64_t max_tile_bytes, uint64_t n_tiles, int sms, bool wide_ok) {
-    if (prob_bits == 10) return 10;
-    if (wide_ok && n_tiles > uint64_t(kWarpsNarrow) * uint64_t(sms > 0 ? sms : 0) &&
-        max_tile_bytes <= Geo<kWarpsMid, 12>::kBuf)
-        return 12;
-    return max_tile_bytes <= Geo<16, 13>::kBuf ? 13 : 12;
+// ---- launch shape: table layout and CTA width ------------------------------------------------
+// A launch of n_tiles tiles over `ctas` CTAs (one per SM) runs in rounds: each warp decodes its
+// tiles one after another, so the time is about the number of rounds, ceil(n_tiles / (warps *
+// ctas)), times one tile's rANS chain, stretched by the warps that share the SM.  The chain of a
+// vector is 8 one-load symbols (layout 10), 4 one-load + 4 two-load (14), 3 + 5 (13) or 8
+// two-load (12): weights 8, 12, 13, 16 at ~45 cycles a one-load symbol.  Each warp past 16 adds
+// 1/64 (fitted to the measured choices between 16-, 24- and 32-warp CTAs).  A shape is usable when
+// its tile buffers hold the largest tile.  The cheapest usable shape wins; on a tie, the layout
+// with the shorter chain, then the narrower width when a single round suffices (more registers
+// per thread, no idle warps), else the wider (more chains per SM).
+struct LaunchShape {
+    int lay, warps;
+};
+inline uint32_t chain_weight(int lay) { return lay == 10 ? 8u : lay == 14 ? 12u : lay == 13 ? 13u : 16u; }
+inline uint64_t shape_cost(int lay, int warps, uint64_t n_tiles, uint64_t ctas) {
+    const uint64_t slots = uint64_t(warps) * (ctas ? ctas : 1);
+    return ((n_tiles + slots - 1) / slots) * chain_weight(lay) * uint64_t(48 + warps);
 }
-// The CTA width of such a launch over `ctas` CTAs: 16 warps when they hold every tile at once (the
-// 16-warp kernel has the most registers per thread); else the widest whose buffers hold the
-// largest tile (more chains per SM, fewer rounds of tiles); layout 13 runs 16 warps only.
+inline bool shape_better(LaunchShape a, LaunchShape b, uint64_t n_tiles, uint64_t ctas) {
+    const uint64_t ca = shape_cost(a.lay, a.warps, n_tiles, ctas), cb = shape_cost(b.lay, b.warps, n_tiles, ctas);
+    if (ca != cb) return ca < cb;
+    if (a.lay != b.lay) return chain_weight(a.lay) < chain_weight(b.lay);
+    const bool one_round = n_tiles <= uint64_t(a.warps) * ctas && n_tiles <= uint64_t(b.warps) * ctas;
+    return one_round ? a.warps < b.warps : a.warps > b.warps;
+}
+// The CTA width for tables already fixed to layout `lay`.
 inline int cta_warps(int lay, uint64_t max_tile_bytes, uint64_t n_tiles, uint64_t ctas) {
-    if (lay == 13 || n_tiles <= uint64_t(kWarpsNarrow) * ctas) return kWarpsNarrow;
-    if (max_tile_bytes <= tile_buffer_bytes(kWarpsWide, lay)) return kWarpsWide;
-    if (max_tile_bytes <= tile_buffer_bytes(kWarpsMid, lay)) return kWarpsMid;
-    return kWarpsNarrow;
+    LaunchShape best{lay, 0};
+    for (int w : {kWarpsNarrow, kWarps20, kWarpsMid, kWarpsWide}) {
+        if (!width_ok(w, lay) || max_tile_bytes > tile_buffer_bytes(w, lay)) continue;
+        if (!best.warps || shape_better(LaunchShape{lay, w}, best, n_tiles, ctas)) best.warps = w;
+    }
+    return best.warps ? best.warps : kWarpsNarrow;  // no buffer holds the largest tile: read it from global memory
+}
+// Layout and width of a launch for blobs with 2^prob_bits frequency totals.  `wide_ok` false (a
+// launch that runs 16-warp CTAs only) considers 16 warps alone, and layouts 10, 12 and 13.  When no buffer holds the largest
+// tile: layout 10, or layout 13 if its 16-warp buffers do, else 12, in 16-warp CTAs (the
+// oversized tiles are read from global memory).
+inline LaunchShape launch_shape(int prob_bits, uint64_t max_tile_bytes, uint64_t n_tiles, uint64_t ctas, bool wide_ok) {
+    LaunchShape best{0, 0};
+    const int lays12[3] = {14, 13, 12}, lays10[1] = {10};
+    const int* lays = prob_bits == 10 ? lays10 : lays12;
+    const int nl = prob_bits == 10 ? 1 : 3;
+    for (int k = 0; k < nl; ++k)
+        for (int w : {kWarpsNarrow, kWarps20, kWarpsMid, kWarpsWide}) {
+            if (!width_ok(w, lays[k]) || (!wide_ok && (w != kWarpsNarrow || lays[k] == 14))) continue;
+            if (max_tile_bytes > tile_buffer_bytes(w, lays[k])) continue;
+            const LaunchShape s{lays[k], w};
+            if (!best.warps || shape_better(s, best, n_tiles, ctas)) best = s;
+        }
+    if (best.warps) return best;
+    if (prob_bits == 10) return LaunchShape{10, kWarpsNarrow};
+    return LaunchShape{max_tile_bytes <= Geo<16, 13>::kBuf ? 13 : 12, kWarpsNarrow};
+}
+inline int table_layout(int prob_bits, uint64_t max_tile_bytes, uint64_t n_tiles, uint64_t ctas, bool wide_ok) {
+    return launch_shape(prob_bits, max_tile_bytes, n_tiles, ctas, wide_ok).lay;
 }
 
-// ---- launch functions, one table per output container ----------------------------------------
+// ---- launch functions, one table per output container and table layout ----------------------
 struct LaunchCtx {
     int device;  // CUDA ordinal (current device)
     int sms;     // its SM count
 };
 
-// Every function takes the table layout lay (10, 12 or 13) and the CTA width in warps (16, 24 or
-// 32; layout 13 runs 16).
+// The launches of one output container with one table layout; each (container, layout) pair is
+// compiled in a unit of its own (decode_unit.cu).  The CTA width is in warps: 16, 20, 24 or 32 for
+// layouts 10 and 12, 16 or 20 for layout 13, 16 for layout 14.  A null entry does not exist: the
+// fields test hook and the row-scaled FP8 container have single-blob launches only, and the
+// allocation-free launch takes layouts 10, 12 and 13.
 struct Launchers {
     // one blob; `dependent`: launch as a programmatic dependent of the previous decode
-    int (*single)(const Params& p, int lay, bool vec, int warps, bool esc, const Ctl& ctl, cudaStream_t st,
-                  const LaunchCtx& c, bool dependent);
-    // a set of blobs, all with the same layout, over `grid` CTAs
-    int (*group)(const GroupParams& g, int lay, uint32_t grid, int warps, cudaStream_t st, const LaunchCtx& c);
+    int (*single)(const Params& p, bool vec, int warps, bool esc, const Ctl& ctl, cudaStream_t st, const LaunchCtx& c,
+                  bool dependent);
+    // a set of blobs over `grid` CTAs
+    int (*group)(const GroupParams& g, uint32_t grid, int warps, cudaStream_t st, const LaunchCtx& c);
     // one blob, tables expanded in every CTA, status in caller-provided memory; never allocates
-    int (*noalloc)(const Params& p, const TableSrc& ts, int lay, bool vec, bool esc, cudaStream_t st,
-                   const LaunchCtx& c);
+    int (*noalloc)(const Params& p, const TableSrc& ts, bool vec, bool esc, cudaStream_t st, const LaunchCtx& c);
 };
 
-extern const Launchers kLaunchBF16, kLaunchFP16, kLaunchE4M3, kLaunchF32, kLaunchI8, kLaunchFields, kLaunchE4M3Row;
+// kLaunch_<container>_<layout>, one per unit.
+#define EP_DECLARE_UNITS(o) \
+    extern const Launchers kLaunch_##o##_10, kLaunch_##o##_12, kLaunch_##o##_13, kLaunch_##o##_14;
+EP_DECLARE_UNITS(0)
+EP_DECLARE_UNITS(1)
+EP_DECLARE_UNITS(2)
+EP_DECLARE_UNITS(3)
+EP_DECLARE_UNITS(4)
+EP_DECLARE_UNITS(5)
+EP_DECLARE_UNITS(6)
+#undef EP_DECLARE_UNITS
+static_assert(kOutBF16 == 0 && kOutFP16 == 1 && kOutE4M3 == 2 && kOutF32 == 3 && kOutFields == 4 && kOutI8 == 5 &&
+              kOutE4M3Row == 6, "unit names use the container numbers");
+
+inline const Launchers* unit_launchers(int out_kind, int lay) {
+#define EP_UNIT_ROW(o) {&kLaunch_##o##_10, &kLaunch_##o##_12, &kLaunch_##o##_13, &kLaunch_##o##_14}
+    static const Launchers* const table[7][kLayouts] = {EP_UNIT_ROW(0), EP_UNIT_ROW(1), EP_UNIT_ROW(2), EP_UNIT_ROW(3),
+                                                        EP_UNIT_ROW(4), EP_UNIT_ROW(5), EP_UNIT_ROW(6)};
+#undef EP_UNIT_ROW
+    if (out_kind < 0 || out_kind > 6 || !(lay == 10 || lay == 12 || is_hybrid(lay))) return nullptr;
+    return table[out_kind][layout_index(lay)];
+}
 
 }  // namespace dec
 }  // namespace ep
