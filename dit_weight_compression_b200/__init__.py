@@ -63,6 +63,7 @@ SIGNATURES = {
     "ep_blob_from_bytes": (_I, [_P, _SZ, ctypes.POINTER(_P)]),
     "ep_blob_prepare": (_I, [_P, _I, _P]),
     "ep_decode_status": (_I, [_P, _P]),
+    "ep_decode_shape": (_I, [_P, ctypes.POINTER(_I), ctypes.POINTER(_I)]),
     "ep_decode_fields": (_I, [_P, _P, _P]),
     "ep_decompress_noalloc": (_I, [_P, _P, _SZ, ctypes.POINTER(EpTensor), _P, _I]),
     "ep_decode_wait_probe": (_I, [_P, ctypes.c_uint32, _P]),
@@ -282,6 +283,13 @@ def decompress_fp8_rowscaled(compressed: CompressedTensor, *, out: torch.Tensor 
 def decode_status(compressed: CompressedTensor, stream=None) -> None:
     """Raise EPError if any decode of this blob on the current device found corrupt tiles."""
     _check(lib().ep_decode_status(compressed.handle, _stream_handle(stream)), "ep_decode_status")
+
+
+def decode_shape(compressed: CompressedTensor) -> tuple[int, int]:
+    """(table layout, CTA width in warps) of decompress() for this blob on the current device."""
+    lay, warps = _I(0), _I(0)
+    _check(lib().ep_decode_shape(compressed.handle, ctypes.byref(lay), ctypes.byref(warps)), "ep_decode_shape")
+    return lay.value, warps.value
 
 
 def decode_fields(compressed: CompressedTensor, stream=None) -> torch.Tensor:

@@ -554,6 +554,19 @@ extern "C" int ep_decode_wait_probe(const ep_blob* cb, uint32_t wait_spins, void
     return launch(p, kOutFields, b->layout, false, ctl, st, dev, false);
 }
 
+extern "C" int ep_decode_shape(const ep_blob* b, int* layout, int* warps) {
+    clear_error();
+    if (!b || !layout || !warps) return set_error(EP_ERR_ARG, "ep_decode_shape: NULL argument");
+    int dev = 0;
+    const int rc = current_device(dev);
+    if (rc != EP_OK) return rc;
+    const BlobLayout& L = b->layout;
+    const int lay = blob_layout(L, dev);  // as launch() decides for a whole-blob decode
+    *layout = lay;
+    *warps = cta_warps(lay, L.max_tile_bytes, L.n_tiles, uint64_t(g_dev[dev].sms));
+    return EP_OK;
+}
+
 extern "C" int ep_decode_status(const ep_blob* cb, void* stream) {
     clear_error();
     if (!cb) return set_error(EP_ERR_ARG, "ep_decode_status: NULL blob");

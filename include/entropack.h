@@ -213,6 +213,14 @@ int ep_blob_prepare(ep_blob* b, int device, void* stream);
  * not 2^16, unused words, bad tile extent, bulk-copy wait limit). */
 int ep_decode_status(const ep_blob* b, void* stream);
 
+/* The kernel variant ep_decompress uses for this blob on the current device: the layout of the
+ * decode tables in shared memory (10: 10-bit totals, one packed word per slot; 12, 13, 14: 12-bit
+ * totals, with 0, 3 or 4 of a vector's 8 symbols read in one lookup and the rest in two) and the
+ * CTA width in warps (16, 20, 24 or 32).  Both follow from the blob's tile count, its largest
+ * tile and the device's SM count; no decode is launched.  A diagnostic for tests and profiles:
+ * the method itself has no counterpart.  Returns EP_ERR_ARG (NULL pointer), EP_ERR_CUDA. */
+int ep_decode_shape(const ep_blob* b, int* layout, int* warps);
+
 /* Test hook: decode the fields of every vector into device memory `fields` (int16, n_vectors
  * x 9: column 0 the coset bit, columns 1..8 the fields f1..f8), asynchronously on `stream`.
  * Same kernel as ep_decompress up to the field inversion. */

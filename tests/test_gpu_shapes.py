@@ -1,0 +1,63 @@
+"""Every kernel variant the launch rule can pick, against the oracle on every tile.
+
+A decode launch picks the layout of its shared-memory tables and its CTA width from the blob's tile
+count, its largest tile and the SM count. The blobs here are sized to reach each (layout, width)
+pair the rule uses: layouts 14, 13, 12 (12-bit totals) and 10 (10-bit totals), CTAs of 16, 20, 24
+and 32 warps. For each one the test asserts that shape through ep_decode_shape, decodes, and
+compares every element with the oracle's tile-parallel decode.
+
+Tile sizes (i.i.d. N(0, 0.02^2) BF16, 8192 columns): 4.0 bpp with S = 32 gives tiles of at most
+4064 B, 2.5 bpp with S = 64 at most 5088 B, 4.0 bpp with S = 64 at most 8144 B. Tile counts are
+multiples of the SM count, so the cases hold on any GPU.
+"""
+import numpy as np
+import pytest
+import torch
+
+import oracle_parallel
+import workloads as W
+
+pytestmark = pytest.mark.gpu
+
+# (frequency-total bits, target bpp, S, tiles per SM, expected (layout, CTA warps))
+CASES = [
+    (12, 4.0, 32, 12, (14, 16)),   # tiles <= 4432 B: one round in 16-warp CTAs
+    (12, 2.5, 64, 12, (13, 16)),   # tiles too large for layout 14
+    (12, 4.0, 32, 18, (13, 20)),   # one round needs 20 warps: layout 13 has room for them
+    (12, 2.5, 64, 18, (12, 20)),   # ... but not for 5 KB tiles
+    (12, 2.5, 64, 22, (12, 24)),
+    (12, 4.0, 32, 28, (12, 32)),
+    (12, 4.0, 64, 4, (12, 16)),    # 8 KB tiles fit 16-warp layout-12 buffers only
+    (10, 4.0, 32, 12, (10, 16)),
+    (10, 4.0, 32, 18, (10, 20)),
+    (10, 4.0, 32, 22, (10, 24)),
+    (10, 4.0, 32, 28, (10, 32)),
+]
+
+
+@pytest.fixture(scope="module")
+def ep():
+    if not torch.cuda.is_available():
+        pytest.skip("no CUDA device")
+    from dit_weight_compression_b200 import build
+    build.build()
+    import dit_weight_compression_b200 as ep
+    return ep
+
+
+@pytest.mark.parametrize("pb,rate,S,per_sm,shape", CASES, ids=[f"L{c[4][0]}x{c[4][1]}" for c in CASES])
+def test_every_launch_shape_matches_oracle(ep, pb, rate, S, per_sm, shape):
+    sms = torch.cuda.get_device_properties(0).multi_processor_count
+    cols = 8192
+    rows = per_sm * sms * (32 * S) // (cols // 8)      # whole tiles: 32 S vectors, cols / 8 per row
+    g = np.random.Generator(np.random.PCG64(pb * 1000 + per_sm * 10 + S))
+    bits = W.to_bf16_bits(g.normal(0, 0.02, (rows, cols)))
+    c = ep.compress(W.bits_to_torch(bits, W.BF16).cuda(), ep.LatticeRANSConfig(rate, steps_per_tile=S, prob_bits=pb))
+    assert c.info.n_tiles == per_sm * sms
+    assert ep.decode_shape(c) == shape
+    out = ep.decompress(c)
+    torch.cuda.synchronize()
+    ep.decode_status(c)
+    got = out.view(torch.int16).cpu().numpy().view(np.uint16)
+    want = oracle_parallel.decode(c.to_bytes())
+    assert np.array_equal(got, want)
