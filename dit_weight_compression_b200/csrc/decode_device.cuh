@@ -80,11 +80,16 @@ constexpr uint32_t kSlots10 = 1024;
 // symbol of the slot's coset half; the coset is u >= the coset-0 total).  Per-symbol entry of
 // field j (1: the joint table, its coset-1 cumulative frequencies following all of coset 0's)
 // given coset c at [kSlotBytes + c (8 * 1024 + kCosetSkew) + 1024 (j - 1) + 4 s]:
-//   bits  0..12  cum(s)               (< 2^13; the joint table's coset-1 symbols follow coset 0's)
-//   bits 17..29  q(s)                 (<= 4096; 0 for a symbol the table does not hold)
-// With the slot u = x mod 4096, the state update is x <- q (x >> 12) + u - cum(s).
-constexpr uint32_t kE12CumMask = 0x1FFFu;
-constexpr uint32_t kE12QShift = 17;
+//   bits  0..12  q(s)                 (<= 4096; the whole entry is 0 for a symbol the table does not hold)
+//   bits 19..31  4096 - cum(s)        (1..4096; the joint table's coset-1 symbols follow coset 0's)
+// With the slot u = x mod 4096 and u' = x | 0xFFFFF000 (= u - 4096 mod 2^32, formed next to the
+// slot's address), the state update is x <- q (x >> 12) + (u' + (entry >> 19)), mod 2^32 equal to
+// q (x >> 12) + u - cum(s): one shift-add and one extraction after the load, then the multiply-add.
+constexpr uint32_t kE12QMask = 0x1FFFu;
+constexpr uint32_t kE12NegCumShift = 19;
+__device__ __forceinline__ uint32_t pack_entry12(uint32_t q, uint32_t cum) {
+    return q ? q | ((4096u - cum) << kE12NegCumShift) : 0u;
+}
 
 // Shared addresses of the decode tables a step reads.
 template <int LAY>
@@ -103,10 +108,11 @@ struct Tab<12> {
 // j = D + 2 .. 8 given c at base + kL1 + 4096 (B c + j - D - 2); their 4-byte entries (as in
 // layout 12) at base + kL2 + c (B * 1024 + kCosetSkew) + 1024 (j - D - 2).  A direct word of slot
 // u holding s:
-//   bits  0..11  u - cum(s)
+//   bits  0..11  q(s) - 1
 //   bits 12..19  s
-//   bits 20..31  q(s) - 1
-// so x <- (q - 1) (x >> 12) + (x >> 12) + (u - cum(s)).
+//   bits 20..31  u - cum(s)
+// so x <- (q - 1) (x >> 12) + ((x >> 12) + (word >> 20)): the shift-add and the extraction of
+// q - 1 run side by side after the load.
 struct TabHybrid {
     uint32_t base;
     uint32_t split;    // slots of coset 0 in the joint table
@@ -116,7 +122,7 @@ struct Tab<13> : TabHybrid {};
 template <>
 struct Tab<14> : TabHybrid {};
 __device__ __forceinline__ uint32_t pack_direct(uint32_t off, uint32_t s, uint32_t q) {
-    return q ? off | (s << 12) | ((q - 1) << 20) : 0u;
+    return q ? (q - 1) | (s << 12) | (off << 20) : 0u;
 }
 
 // Scratch of the table expansion: frequencies and cumulative frequencies of every context.
@@ -329,7 +335,7 @@ __device__ void build_hybrid(uint8_t* tab, const BuildScratch& scr) {
         const uint32_t c = row / B, ctx = 8 * c + 1 + D + row % B;
         const uint32_t q = scr.q[ctx][sy];
         uint32_t* ent = reinterpret_cast<uint32_t*>(tab + Hybrid<LAY>::kL2 + c * kCosetSkew + 1024 * row);
-        ent[sy] = q ? (q << kE12QShift) | uint32_t(scr.cum[ctx][sy]) : 0u;
+        ent[sy] = pack_entry12(q, uint32_t(scr.cum[ctx][sy]));
     }
 }
 
@@ -429,7 +435,7 @@ __device__ void build_tables(uint8_t* tab, BuildScratch& scr, const TableSrc& p)
             const uint32_t q = scr.q[ctx][sy];
             const uint32_t cum = scr.cum[ctx][sy] + (j == 1 && c ? split : 0u);
             uint32_t* ent = reinterpret_cast<uint32_t*>(tab + kSlotBytes + c * (8 * 1024 + kCosetSkew) + 1024 * (j - 1));
-            ent[sy] = q ? (q << kE12QShift) | cum : 0u;
+            ent[sy] = pack_entry12(q, cum);
         }
     }
 }
@@ -640,11 +646,11 @@ __device__ __forceinline__ void step_symbols12(const Tab<12>& T, Reader& rd, uin
     // return), its byte the f1 symbol.  A lane past the last vector still loads but keeps x.
     uint32_t c;
     {
-        const uint32_t u = x & 4095u, a1 = u | T.s1;
+        const uint32_t a1 = (x & 4095u) | T.s1, um = x | 0xFFFFF000u;
         c = a1 >= T.s1split ? 1u : 0u;
         const uint32_t sy = lds_u8<0>(a1);
         const uint32_t en = lds_u32<0>(T.e2 + (8u * 1024u + kCosetSkew) * c + 4u * sy);
-        if (active) x = (en >> kE12QShift) * (x >> 12) + (u - (en & kE12CumMask));
+        if (active) x = (en & kE12QMask) * (x >> 12) + (um + (en >> kE12NegCumShift));
         renorm_step<FULL>(x, rd, active);
         e[0] = sy;
         if (ESC) acc = sy;
@@ -654,10 +660,10 @@ __device__ __forceinline__ void step_symbols12(const Tab<12>& T, Reader& rd, uin
     const uint32_t b2 = T.e2 + 1024u + c * (8u * 1024u + kCosetSkew);   // field 2's entries given c
 #define EP_FIELD12(j)                                                                         \
     {                                                                                         \
-        const uint32_t u = x & 4095u;                                                         \
-        const uint32_t sy = lds_u8<((j) - 1) * kCtxBytes>(u | b1);                            \
+        const uint32_t um = x | 0xFFFFF000u;                                                  \
+        const uint32_t sy = lds_u8<((j) - 1) * kCtxBytes>((x & 4095u) | b1);                  \
         const uint32_t en = lds_u32<((j) - 1) * 1024>(b2 + 4u * sy);                          \
-        if (active) x = (en >> kE12QShift) * (x >> 12) + (u - (en & kE12CumMask));            \
+        if (active) x = (en & kE12QMask) * (x >> 12) + (um + (en >> kE12NegCumShift));        \
         renorm_step<FULL>(x, rd, active);                                                     \
         e[j] = sy;                                                                            \
         if (ESC) acc = max(acc, sy);                                                          \
@@ -694,7 +700,7 @@ __device__ __forceinline__ void step_symbols_hybrid(const Tab<LAY>& T, Reader& r
     // a direct word's state update; returns the symbol
     auto direct = [&](uint32_t w) {
         const uint32_t h = x >> 12;
-        if (active) x = (w >> 20) * h + (h + (w & 4095u));
+        if (active) x = (w & 4095u) * h + (h + (w >> 20));
         return (w >> 12) & 255u;
     };
     uint32_t c;
@@ -722,10 +728,10 @@ __device__ __forceinline__ void step_symbols_hybrid(const Tab<LAY>& T, Reader& r
     const uint32_t b2 = T.base + Hybrid<LAY>::kL2 + c * (B * 1024u + kCosetSkew);   // and its entries
 #define EP_FIELD13(j)                                                                         \
     {                                                                                         \
-        const uint32_t u = x & 4095u;                                                         \
-        const uint32_t sy = lds_u8<((j) - 1 - D) * kCtxBytes>(u | b1);                        \
+        const uint32_t um = x | 0xFFFFF000u;                                                  \
+        const uint32_t sy = lds_u8<((j) - 1 - D) * kCtxBytes>((x & 4095u) | b1);              \
         const uint32_t en = lds_u32<((j) - 1 - D) * 1024>(b2 + 4u * sy);                      \
-        if (active) x = (en >> kE12QShift) * (x >> 12) + (u - (en & kE12CumMask));            \
+        if (active) x = (en & kE12QMask) * (x >> 12) + (um + (en >> kE12NegCumShift));        \
         renorm_step<FULL>(x, rd, active);                                                     \
         e[j] = sy;                                                                            \
         if (ESC) acc = max(acc, sy);                                                          \
