@@ -293,49 +293,58 @@ int decode_to_host(ep_blob* b, const ep_tensor* out, int kind, float* host_sigma
     const uint64_t per = uint64_t(kLanes) * L.steps;
     const std::vector<uint32_t> t = host_chunks(L, row_bytes * size_t(L.rows));
     const std::string w(what);
-    EP_CUDA(cudaMemcpyAsync(d.stage_blob, host, L.off_stream, cudaMemcpyHostToDevice, st), w + ": upload");
-    uint64_t up = 0;  // stream bytes uploaded so far
-    for (size_t i = 0; i + 1 < t.size(); ++i) {
-        const uint32_t t0 = t[i], t1 = t[i + 1];
-        const bool last = i + 2 == t.size();
-        // tile offsets are checked to rise to the stream's end, so chunk i's tiles lie in [0, end)
-        const uint64_t end = last ? stream_total : std::min<uint64_t>(stream_total, 16ull * rd32(host + L.off_offsets + 4ull * t1));
-        if (end > up) {
-            EP_CUDA(cudaMemcpyAsync(d.stage_blob + L.off_stream + up, host + L.off_stream + up, end - up,
-                                    cudaMemcpyHostToDevice, st),
-                    w + ": upload");
-            up = end;
+    // Everything is issued first; whatever happens, both streams are drained before returning, so
+    // no download of an earlier chunk is still writing into the caller's buffer after an error.
+    auto issue = [&]() -> int {
+        EP_CUDA(cudaMemcpyAsync(d.stage_blob, host, L.off_stream, cudaMemcpyHostToDevice, st), w + ": upload");
+        uint64_t up = 0;  // stream bytes uploaded so far
+        for (size_t i = 0; i + 1 < t.size(); ++i) {
+            const uint32_t t0 = t[i], t1 = t[i + 1];
+            const bool last = i + 2 == t.size();
+            // tile offsets are checked to rise to the stream's end, so chunk i's tiles lie in [0, end)
+            const uint64_t end =
+                last ? stream_total : std::min<uint64_t>(stream_total, 16ull * rd32(host + L.off_offsets + 4ull * t1));
+            if (end > up) {
+                EP_CUDA(cudaMemcpyAsync(d.stage_blob + L.off_stream + up, host + L.off_stream + up, end - up,
+                                        cudaMemcpyHostToDevice, st),
+                        w + ": upload");
+                up = end;
+            }
+            const int64_t v0 = int64_t(t0) * int64_t(per);
+            const int64_t v1 = last ? L.n_vectors : int64_t(t1) * int64_t(per);
+            const int64_t r0 = v0 / L.vec_per_row, r1 = last ? L.rows : v1 / L.vec_per_row;
+            uint8_t* dout = d.stage_out + size_t(r0) * row_bytes;
+            Params p = make_params(b, d.stage_blob, tables, dout, L.cols, d.status);
+            p.tile_off += t0;
+            p.alpha += r0;
+            p.rowmax += r0;
+            p.rows = r1 - r0;
+            p.n_vectors = v1 - v0;
+            p.n_tiles = t1 - t0;
+            if (host_sigma) p.sigma = d.stage_sigma + r0;
+            const int lrc = launch(p, kind, L, vec_ok(L, dout, L.cols, out->dtype), Ctl(), st, dev, false);
+            if (lrc != EP_OK) return lrc;
+            EP_CUDA(cudaEventRecord(d.chunk_done[i], st), w + ": chunk event");
+            EP_CUDA(cudaStreamWaitEvent(cb, d.chunk_done[i], 0), w + ": chunk wait");
+            uint8_t* hout = static_cast<uint8_t*>(out->data) + size_t(r0) * size_t(out->row_stride) * es;
+            if (out->row_stride == L.cols)  // contiguous rows: one linear copy
+                EP_CUDA(cudaMemcpyAsync(hout, dout, size_t(r1 - r0) * row_bytes, cudaMemcpyDeviceToHost, cb),
+                        w + ": download");
+            else
+                EP_CUDA(cudaMemcpy2DAsync(hout, size_t(out->row_stride) * es, dout, row_bytes, row_bytes,
+                                          size_t(r1 - r0), cudaMemcpyDeviceToHost, cb),
+                        w + ": download");
         }
-        const int64_t v0 = int64_t(t0) * int64_t(per);
-        const int64_t v1 = last ? L.n_vectors : int64_t(t1) * int64_t(per);
-        const int64_t r0 = v0 / L.vec_per_row, r1 = last ? L.rows : v1 / L.vec_per_row;
-        uint8_t* dout = d.stage_out + size_t(r0) * row_bytes;
-        Params p = make_params(b, d.stage_blob, tables, dout, L.cols, d.status);
-        p.tile_off += t0;
-        p.alpha += r0;
-        p.rowmax += r0;
-        p.rows = r1 - r0;
-        p.n_vectors = v1 - v0;
-        p.n_tiles = t1 - t0;
-        if (host_sigma) p.sigma = d.stage_sigma + r0;
-        rc = launch(p, kind, L, vec_ok(L, dout, L.cols, out->dtype), Ctl(), st, dev, false);
-        if (rc != EP_OK) return rc;
-        EP_CUDA(cudaEventRecord(d.chunk_done[i], st), w + ": chunk event");
-        EP_CUDA(cudaStreamWaitEvent(cb, d.chunk_done[i], 0), w + ": chunk wait");
-        uint8_t* hout = static_cast<uint8_t*>(out->data) + size_t(r0) * size_t(out->row_stride) * es;
-        if (out->row_stride == L.cols)  // contiguous rows: one linear copy
-            EP_CUDA(cudaMemcpyAsync(hout, dout, size_t(r1 - r0) * row_bytes, cudaMemcpyDeviceToHost, cb),
+        if (host_sigma)
+            EP_CUDA(cudaMemcpyAsync(host_sigma, d.stage_sigma, 4 * size_t(L.rows), cudaMemcpyDeviceToHost, cb),
                     w + ": download");
-        else
-            EP_CUDA(cudaMemcpy2DAsync(hout, size_t(out->row_stride) * es, dout, row_bytes, row_bytes, size_t(r1 - r0),
-                                      cudaMemcpyDeviceToHost, cb),
-                    w + ": download");
-    }
-    if (host_sigma)
-        EP_CUDA(cudaMemcpyAsync(host_sigma, d.stage_sigma, 4 * size_t(L.rows), cudaMemcpyDeviceToHost, cb),
-                w + ": download");
-    EP_CUDA(cudaStreamSynchronize(cb), w + ": synchronise");
-    EP_CUDA(cudaStreamSynchronize(st), w + ": synchronise");
+        return EP_OK;
+    };
+    rc = issue();
+    const cudaError_t e1 = cudaStreamSynchronize(cb), e2 = cudaStreamSynchronize(st);
+    if (rc != EP_OK) return rc;
+    if (e1 != cudaSuccess || e2 != cudaSuccess)
+        return set_error(EP_ERR_CUDA, w + ": synchronise: " + cudaGetErrorString(e1 != cudaSuccess ? e1 : e2));
     return EP_OK;
 }
 
