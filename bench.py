@@ -29,6 +29,7 @@ import hashlib
 import json
 import math
 import os
+import re
 import statistics
 import subprocess
 import sys
@@ -166,10 +167,14 @@ TRAFFIC_FILE = os.path.join(ROOT, "profiles", "decode_traffic.json")
 
 
 def kernel_source_hash() -> str:
-    """Hash of the decode kernel's sources: a DRAM traffic figure is valid only for this code."""
+    """Hash of the decode kernel's code (comments and blank space removed): a DRAM traffic figure
+    is valid only for this code, and an edit to a comment does not change the kernel."""
     h = hashlib.sha256()
     for f in KERNEL_SOURCES:
-        h.update(open(os.path.join(ROOT, "dit_weight_compression_b200", "csrc", f), "rb").read())
+        text = open(os.path.join(ROOT, "dit_weight_compression_b200", "csrc", f), encoding="utf-8").read()
+        text = re.sub(r"/\*.*?\*/", " ", text, flags=re.S)
+        text = re.sub(r"//[^\n]*", " ", text)
+        h.update(" ".join(text.split()).encode())
     return h.hexdigest()[:16]
 
 

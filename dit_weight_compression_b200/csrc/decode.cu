@@ -1,7 +1,8 @@
-// decode.cu -- the GPU entry points of the C ABI: device copies of a blob, the decode launches
-// (ep_decompress, ep_decompress_group, ep_decode_fields), the status word, and the
-// allocation-free decode.  The kernels themselves are in decode_device.cuh; each output
-// container's instantiations are compiled in decode_<container>.cu.
+// decode.cu -- the GPU entry points of the C ABI: device copies of a blob and its decode tables,
+// the decode launches (ep_decompress, ep_decompress_group, ep_decompress_fp8_rowscaled,
+// ep_decode_fields), the host-output path, the status word, the launch-shape query and the
+// allocation-free decode.  The kernels themselves are in decode_device.cuh; the instantiations of
+// each (output container, table layout) pair are compiled from decode_unit.cu.
 #include "decode_device.cuh"
 
 #include <numeric>

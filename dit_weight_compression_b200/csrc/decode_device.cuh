@@ -7,16 +7,19 @@
 //
 // One kernel does the whole path.  Work split:
 //   * one warp per tile; the tile's 32 interleaved rANS states live one per lane;
-//   * one persistent CTA per SM (16 or 32 warps; grid = min(#SM, #tiles)); tile t goes to CTA
-//     t mod grid, so every SM gets an equal share even when there are few tiles;
+//   * one persistent CTA per SM (16, 20, 24 or 32 warps, with the table layout chosen per launch
+//     by launch_shape in decode_launch.h; grid = min(#SM, #tiles)); tile t goes to CTA t mod grid,
+//     so every SM gets an equal share even when there are few tiles;
 //   * decode tables, for the joint (coset, f1) symbol and for f2..f8 given each coset (15
 //     tables).  With 10-bit totals: one packed 32-bit entry per slot of the 1024-slot range,
 //     {slot - cum(s), s (2 s for f8), escape flag, coset bit, q(s)} -- 60 KB -- so one
 //     shared-memory load per symbol gives everything the state update needs.  With 12-bit totals
-//     the per-slot entries would take 240 KB, more than an SM has, so a symbol takes two loads:
-//     the slot's symbol byte (4096 per table, 60 KB), then that symbol's packed {q(s), cum(s)}
-//     word (16 KB), so the state update is two field extractions, a subtraction and a
-//     multiply-add.  The tables are expanded once per blob and device by a small kernel into
+//     the per-slot entries would take 240 KB, more than an SM has, so most symbols take two
+//     loads: the slot's symbol byte (4096 per table, 60 KB), then that symbol's packed
+//     {q(s), 4096 - cum(s)} word (16 KB).  Layouts 13 and 14 give the joint table and the next 2
+//     or 3 fields one packed word per slot instead, as far as shared memory allows.  Either way
+//     the state update is a shift-add and an extraction side by side, then one multiply-add.
+//     The tables are expanded once per blob, device and layout by a small kernel into
 //     a block next to the device copy; every CTA stages that block into shared memory with bulk
 //     copies, overlapped with the fetch of its first tiles.  (The allocation-free entry point
 //     expands them inside each CTA instead.);
@@ -35,8 +38,8 @@
 // No tensor cores: the path is table lookups and integer arithmetic, bound by HBM bytes and by
 // the latency and issue slots of that arithmetic, not by a contraction.
 //
-// Every output container instantiates these templates in a translation unit of its own
-// (decode_<container>.cu), which exports one Launchers table.
+// Every (output container, table layout) pair instantiates these templates in a translation unit
+// of its own (decode_unit.cu, compiled once per pair), which exports one Launchers table.
 #pragma once
 
 #include <cuda_bf16.h>

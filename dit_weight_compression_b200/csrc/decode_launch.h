@@ -1,9 +1,10 @@
-// decode_launch.h -- what the host side of the decode (decode.cu) and the per-container kernel
-// units (decode_<container>.cu) share: the kernel parameter blocks, the shared-memory geometry,
-// the status bits, and one table of launch functions per output container.
+// decode_launch.h -- what the host side of the decode (decode.cu) and the kernel units
+// (decode_unit.cu, one per output container and table layout) share: the kernel parameter
+// blocks, the shared-memory geometry of every table layout and CTA width, the rule that picks
+// them for a launch, the status bits, and one table of launch functions per unit.
 //
-// The kernels are templates over the output container; each container's instantiations live in
-// a translation unit of their own (decode_bf16.cu, ...), so the library builds in parallel.
+// The kernels are templates over the output container and the table layout; each pair's
+// instantiations live in a translation unit of their own, so the library builds in parallel.
 #pragma once
 
 #include <cuda_runtime.h>
