@@ -149,7 +149,7 @@ __device__ __forceinline__ void mbar_expect_tx(unsigned long long* bar, uint32_t
     asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(smem_u32(bar)), "r"(bytes)
                  : "memory");
 }
-// 1-D bulk copy global -> this CTA's shared memory, completing on `bar` (no multicast).
+// 1-D bulk copy global -> this CTA's own shared memory, completing on `bar`.
 __device__ __forceinline__ void bulk_g2s(void* dst, const void* src, uint32_t bytes, unsigned long long* bar) {
     asm volatile(
         "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(
