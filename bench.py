@@ -69,6 +69,9 @@ def parse_args():
     ap.add_argument("--decode", choices=["grouped", "single"], default="grouped",
                     help="for a set of matrices: one ep_decompress_group call per step, or one "
                          "ep_decompress call per matrix")
+    ap.add_argument("--matrices", type=int, default=0,
+                    help="for a set of matrices: use only the first K (0 = all), e.g. to keep a profiled "
+                         "case to a few GB on the device")
     return ap.parse_args()
 
 
@@ -351,8 +354,12 @@ def queue_delay_cycles(launches: int) -> int:
 def main():
     args = parse_args()
     mats, desc = workload(args.workload)
+    subset = ""
+    if 0 < args.matrices < len(mats):
+        subset = f"; the first {args.matrices} of its {len(mats)} matrices"
+        mats = mats[:args.matrices]
     if args.impl == "reference":
-        reference_arm(args, mats[0], desc)
+        reference_arm(args, mats[0], desc + subset)
         return
 
     import torch
@@ -527,8 +534,8 @@ def main():
         info = comps[0].info
         dt_names = [name for name, _, _ in out_dts]
         config = {
-            "workload": desc if not args.out_dtype else f"{desc.rsplit(', output', 1)[0]}, output "
-                                                        f"{' then '.join(dt_names)}",
+            "workload": (desc if not args.out_dtype else f"{desc.rsplit(', output', 1)[0]}, output "
+                                                         f"{' then '.join(dt_names)}") + subset,
             "matrices": n,
             "shapes": [list(c.shape) for c in comps],
             "target_bpp": mats[0].target_bpp,
