@@ -22,7 +22,7 @@ LIB = os.path.join(PKG, "libentropack.so")
 PLAIN = ["api.cpp", "encoder.cpp", "decode.cu", "encode_gpu.cu"]
 # The decode kernels: decode_unit.cu once per output container (OutKind 0..6) and table layout.
 UNIT_OUTS = range(7)
-UNIT_LAYS = (10, 12, 13, 14)
+UNIT_LAYS = (10, 11, 12, 13, 14)
 HEADERS = ["format.h", "blob.h", "tables.h", "decode_launch.h", "decode_device.cuh"]
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]
 
@@ -90,7 +90,7 @@ def build(verbose: bool = False, force: bool = False) -> str:
     if todo or not os.path.exists(LIB) or stale():
         os.makedirs(OBJ, exist_ok=True)
         # the largest units first, so the tail of the parallel build is short
-        todo.sort(key=lambda j: (j[1] != "decode_unit.cu", "_4_" in j[0], "_14" in j[0] or "_13" in j[0]))
+        todo.sort(key=lambda j: (j[1] != "decode_unit.cu", "_4_" in j[0], "_14." in j[0] or "_13." in j[0]))
         workers = max(1, min(len(todo), os.cpu_count() or 1))
 
         def run(job):

@@ -28,6 +28,9 @@ struct DevInfo {
 std::mutex g_dev_mu;
 DevInfo g_dev[kMaxDevices];
 
+static_assert(sizeof(DeviceCopy::tables) / sizeof(DeviceCopy::tables[0]) == kLayouts,
+              "one table block per table layout");
+
 // The table layout of a blob's decodes on device `dev` (its SM count known: current_device ran).
 int blob_layout(const BlobLayout& L, int dev) {
     return table_layout(L.prob_bits, L.max_tile_bytes, L.n_tiles, g_dev[dev].sms, true);
@@ -140,9 +143,11 @@ int tables_locked(ep_blob* b, int dev, int lay, cudaStream_t st, const uint8_t*&
         }
         const TableSrc ts = make_tablesrc(b, d.blob);
         auto fn = lay == 10   ? expand_tables_kernel<kWarpsWide, 10>
+                  : lay == 11 ? expand_tables_kernel<kWarpsWide, 11>
                   : lay == 12 ? expand_tables_kernel<kWarpsWide, 12>
                   : lay == 13 ? expand_tables_kernel<kWarpsWide, 13> : expand_tables_kernel<kWarpsWide, 14>;
         const size_t smem = lay == 10   ? sizeof(ExpandSmem<10>)
+                            : lay == 11 ? sizeof(ExpandSmem<11>)
                             : lay == 12 ? sizeof(ExpandSmem<12>)
                             : lay == 13 ? sizeof(ExpandSmem<13>) : sizeof(ExpandSmem<14>);
         cudaError_t e = cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, int(smem));

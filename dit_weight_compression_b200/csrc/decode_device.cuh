@@ -105,7 +105,7 @@ struct Tab<12> {
     uint32_t e2;       // per-symbol entries
     uint32_t s1split;  // s1 + the slots of coset 0 in the joint table
 };
-// Layouts 13 and 14 (12-bit totals, hybrid with D = Hybrid<LAY>::kND direct fields per coset and
+// Layouts 11, 13 and 14 (12-bit totals, hybrid with D = Hybrid<LAY>::kND direct fields per coset and
 // B = 7 - D two-lookup ones), at `base` (4 KB aligned): the joint table's direct words at base;
 // field j = 2 .. D + 1 given coset c at base + kHDirect (1 + D c + j - 2); symbol bytes of field
 // j = D + 2 .. 8 given c at base + kL1 + 4096 (B c + j - D - 2); their 4-byte entries (as in
@@ -120,6 +120,8 @@ struct TabHybrid {
     uint32_t base;
     uint32_t split;    // slots of coset 0 in the joint table
 };
+template <>
+struct Tab<11> : TabHybrid {};
 template <>
 struct Tab<13> : TabHybrid {};
 template <>
@@ -279,7 +281,7 @@ __device__ __forceinline__ uint32_t pack_entry(uint32_t bias, uint32_t s, uint32
            (coset << kEntryCosetShift) | (q << kEntryQShift);
 }
 
-// Layout 13 or 14 from the per-context frequencies and cumulative frequencies in `scr`: the
+// Layout 11, 13 or 14 from the per-context frequencies and cumulative frequencies in `scr`: the
 // 1 + 2D direct tables, the 2B symbol-byte tables, then the 4-byte entries of those 2B.
 template <int WARPS, int LAY>
 __device__ void build_hybrid(uint8_t* tab, const BuildScratch& scr) {
@@ -691,7 +693,7 @@ __device__ __forceinline__ void step_symbols12(const Tab<12>& T, Reader& rd, uin
     }
 }
 
-// Layouts 13 and 14: (coset, f1) and the next D fields from direct words (one load each), the
+// Layouts 11, 13 and 14: (coset, f1) and the next D fields from direct words (one load each), the
 // rest as in layout 12.
 template <int LAY, bool ESC, bool FULL, class Reader>
 __device__ __forceinline__ void step_symbols_hybrid(const Tab<LAY>& T, Reader& rd, uint32_t& x, bool active,
@@ -724,8 +726,9 @@ __device__ __forceinline__ void step_symbols_hybrid(const Tab<LAY>& T, Reader& r
         e[j] = sy;                                                                            \
         if (ESC) acc = max(acc, sy);                                                          \
     }
-    EP_FIELD13D(1) EP_FIELD13D(2)
-    if constexpr (D == 3) EP_FIELD13D(3)
+    if constexpr (D >= 1) EP_FIELD13D(1)
+    if constexpr (D >= 2) EP_FIELD13D(2)
+    if constexpr (D >= 3) EP_FIELD13D(3)
 #undef EP_FIELD13D
     const uint32_t b1 = T.base + Hybrid<LAY>::kL1 + c * (B * kCtxBytes);            // first two-lookup field's bytes
     const uint32_t b2 = T.base + Hybrid<LAY>::kL2 + c * (B * 1024u + kCosetSkew);   // and its entries
@@ -739,7 +742,9 @@ __device__ __forceinline__ void step_symbols_hybrid(const Tab<LAY>& T, Reader& r
         e[j] = sy;                                                                            \
         if (ESC) acc = max(acc, sy);                                                          \
     }
-    if constexpr (D == 2) EP_FIELD13(3)
+    if constexpr (D < 1) EP_FIELD13(1)
+    if constexpr (D < 2) EP_FIELD13(2)
+    if constexpr (D < 3) EP_FIELD13(3)
     EP_FIELD13(4) EP_FIELD13(5) EP_FIELD13(6) EP_FIELD13(7)
 #undef EP_FIELD13
 
@@ -1284,7 +1289,7 @@ int launch_vec(const Params& p, bool vec, const Ctl& ctl, cudaStream_t st, const
 
 template <int OUT, bool ESC, int LAY>
 int launch_width(const Params& p, bool vec, int warps, const Ctl& ctl, cudaStream_t st, const LaunchCtx& c, bool dep) {
-    if constexpr (!is_hybrid(LAY)) {  // layout 13 leaves room for 16 or 20 warps, layout 14 for 16
+    if constexpr (LAY != 13 && LAY != 14) {  // layout 13 leaves room for 16 or 20 warps, layout 14 for 16
         if (warps == kWarpsWide) return launch_vec<kWarpsWide, OUT, ESC, LAY>(p, vec, ctl, st, c, dep);
         if (warps == kWarpsMid) return launch_vec<kWarpsMid, OUT, ESC, LAY>(p, vec, ctl, st, c, dep);
     }
@@ -1331,7 +1336,7 @@ int group_launch_one(const GroupParams& g, uint32_t grid, cudaStream_t st, const
 // A set of blobs (one total width pb) over `grid` CTAs.
 template <int OUT, int LAY>
 int group_width(const GroupParams& g, uint32_t grid, int warps, cudaStream_t st, const LaunchCtx& c) {
-    if constexpr (!is_hybrid(LAY)) {
+    if constexpr (LAY != 13 && LAY != 14) {
         if (warps == kWarpsWide) return group_launch_one<kWarpsWide, OUT, LAY>(g, grid, st, c);
         if (warps == kWarpsMid) return group_launch_one<kWarpsMid, OUT, LAY>(g, grid, st, c);
     }

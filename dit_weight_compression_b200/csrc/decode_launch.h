@@ -29,26 +29,28 @@ constexpr uint32_t kSlotBytes = kDecodeTables * kCtxBytes;    // 61440
 // warp whose lanes read the same symbol of the same field in both cosets hits different banks.
 constexpr uint32_t kCosetSkew = 64;
 constexpr uint32_t kSymEntryBytes = 16 * 256 * 4 + kCosetSkew;  // 16448 (12-bit totals only)
-// 12-bit totals, hybrid layouts 13 and 14: the joint table and the next kND fields (f2, f3 for
-// layout 13; f2, f3, f4 for layout 14) given each coset as direct words, one u32 per slot (16 KB
-// a table); the other 7 - kND fields given each coset as symbol bytes (4 KB a table) and 4-byte
-// per-symbol entries (1 KB a table).  Layout 13 takes 130 KB, layout 14 152 KB.
+// 12-bit totals, hybrid layouts 11, 13 and 14: the joint table and the next kND fields (none for
+// layout 11; f2, f3 for layout 13; f2, f3, f4 for layout 14) given each coset as direct words, one
+// u32 per slot (16 KB a table); the other 7 - kND fields given each coset as symbol bytes (4 KB a
+// table) and 4-byte per-symbol entries (1 KB a table).  Layout 11 takes 86 KB, 13 130 KB, 14
+// 152 KB.
 constexpr uint32_t kHDirect = 4 * 4096;                       // one direct table: 16384
 template <int LAY>
 struct Hybrid {
-    static constexpr uint32_t kND = LAY == 14 ? 3 : 2;         // direct fields per coset after the joint table
+    static constexpr uint32_t kND = LAY == 14 ? 3 : LAY == 13 ? 2 : 0;  // direct fields per coset after the joint table
     static constexpr uint32_t kNB = 7 - kND;                   // two-lookup fields per coset
-    static constexpr uint32_t kL1 = (1 + 2 * kND) * kHDirect;  // their symbol bytes (81920 / 114688)
-    static constexpr uint32_t kL2 = kL1 + 2 * kNB * kCtxBytes; // their 4-byte entries (122880 / 147456)
-    static constexpr uint32_t kBytes = kL2 + 2 * kNB * 1024 + kCosetSkew;  // 133184 / 155712
+    static constexpr uint32_t kL1 = (1 + 2 * kND) * kHDirect;  // their symbol bytes (16384 / 81920 / 114688)
+    static constexpr uint32_t kL2 = kL1 + 2 * kNB * kCtxBytes; // their 4-byte entries
+    static constexpr uint32_t kBytes = kL2 + 2 * kNB * 1024 + kCosetSkew;  // 88128 / 133184 / 155712
 };
-__host__ __device__ constexpr bool is_hybrid(int lay) { return lay == 13 || lay == 14; }
+__host__ __device__ constexpr bool is_hybrid(int lay) { return lay == 11 || lay == 13 || lay == 14; }
 
 // Table layouts: 10 = 10-bit totals, one packed word per slot; 12 = 12-bit totals, two lookups
-// per symbol; 13 and 14 = 12-bit totals, hybrid.
+// per symbol; 11, 13 and 14 = 12-bit totals, hybrid.
 template <int LAY>
 struct TableGeo {
-    static_assert(LAY == 10 || LAY == 12 || LAY == 13 || LAY == 14, "table layouts are 10, 12, 13 and 14");
+    static_assert(LAY == 10 || LAY == 11 || LAY == 12 || LAY == 13 || LAY == 14,
+                  "table layouts are 10, 11, 12, 13 and 14");
     static constexpr uint32_t kBytes =
         LAY == 10 ? kSlotBytes : LAY == 12 ? kSlotBytes + kSymEntryBytes : Hybrid<LAY>::kBytes;
     static constexpr uint32_t kPiece = kBytes / 4;             // bytes per table bulk copy
@@ -56,6 +58,7 @@ struct TableGeo {
 };
 inline uint32_t table_bytes(int lay) {
     return lay == 10 ? TableGeo<10>::kBytes
+         : lay == 11 ? TableGeo<11>::kBytes
          : lay == 12 ? TableGeo<12>::kBytes
          : lay == 13 ? TableGeo<13>::kBytes : TableGeo<14>::kBytes;
 }
@@ -126,8 +129,8 @@ constexpr uint32_t kAlignSlack = 4096;    // the table starts on a 4 KB boundary
 constexpr uint32_t kBufSlack = 80;        // bytes after a tile buffer that two steps may over-read
 
 // CTA widths: 16, 20, 24 or 32 warps, each warp with a tile buffer of Geo<WARPS, LAY>::kBuf bytes:
-//   layout 10: 10336, 8240, 6848, 5120;  layout 12: 9296, 7424, 6176, 4608;  layout 13: 5840, 4656;
-//   layout 14: 4432
+//   layout 10: 10336, 8240, 6848, 5120;  layout 11: 8656, 6912, 5744, 4288;
+//   layout 12: 9296, 7424, 6176, 4608;   layout 13: 5840, 4656;  layout 14: 4432
 // (layout 13 leaves room for 16 or 20 warps, layout 14 for 16).  A tile larger than its warp's
 // buffer is read from global memory.
 constexpr int kWarpsNarrow = 16, kWarps20 = 20, kWarpsMid = 24, kWarpsWide = 32;
@@ -154,7 +157,8 @@ template <int WARPS, int LAY>
 constexpr bool fits_smem() { return sizeof(Smem<WARPS, LAY>) + kAlignSlack <= kSmemOptin; }
 static_assert(fits_smem<16, 10>() && fits_smem<20, 10>() && fits_smem<24, 10>() && fits_smem<32, 10>() &&
               fits_smem<16, 12>() && fits_smem<20, 12>() && fits_smem<24, 12>() && fits_smem<32, 12>() &&
-              fits_smem<16, 13>() && fits_smem<20, 13>() && fits_smem<16, 14>(),
+              fits_smem<16, 13>() && fits_smem<20, 13>() && fits_smem<16, 14>() && fits_smem<16, 11>() &&
+              fits_smem<20, 11>() && fits_smem<24, 11>() && fits_smem<32, 11>(),
               "shared memory budget");
 inline bool width_ok(int warps, int lay) {
     if (lay == 14) return warps == kWarpsNarrow;
@@ -166,6 +170,10 @@ inline uint32_t tile_buffer_bytes(int warps, int lay) {
         case 1020: return Geo<20, 10>::kBuf;
         case 1024: return Geo<24, 10>::kBuf;
         case 1032: return Geo<32, 10>::kBuf;
+        case 1116: return Geo<16, 11>::kBuf;
+        case 1120: return Geo<20, 11>::kBuf;
+        case 1124: return Geo<24, 11>::kBuf;
+        case 1132: return Geo<32, 11>::kBuf;
         case 1216: return Geo<16, 12>::kBuf;
         case 1220: return Geo<20, 12>::kBuf;
         case 1224: return Geo<24, 12>::kBuf;
@@ -177,15 +185,15 @@ inline uint32_t tile_buffer_bytes(int warps, int lay) {
     }
 }
 // Index of a layout's expanded tables in a device copy of a blob.
-inline int layout_index(int lay) { return lay == 10 ? 0 : lay == 12 ? 1 : lay == 13 ? 2 : 3; }
-constexpr int kLayouts = 4;
+inline int layout_index(int lay) { return lay == 10 ? 0 : lay == 12 ? 1 : lay == 13 ? 2 : lay == 14 ? 3 : 4; }
+constexpr int kLayouts = 5;
 
 // ---- launch shape: table layout and CTA width ------------------------------------------------
 // A launch of n_tiles tiles over `ctas` CTAs (one per SM) runs in rounds: each warp decodes its
 // tiles one after another, so the time is about the number of rounds, ceil(n_tiles / (warps *
 // ctas)), times one tile's rANS chain, stretched by the warps that share the SM.  The chain of a
-// vector is 8 one-load symbols (layout 10), 4 one-load + 4 two-load (14), 3 + 5 (13) or 8
-// two-load (12): weights 8, 12, 13, 16 at ~45 cycles a one-load symbol.  Each warp past 16 adds
+// vector is 8 one-load symbols (layout 10), 4 one-load + 4 two-load (14), 3 + 5 (13), 1 + 7 (11)
+// or 8 two-load (12): weights 8, 12, 13, 15, 16 at ~45 cycles a one-load symbol.  Each warp past 16 adds
 // 1/64 (fitted to the measured choices between 16-, 24- and 32-warp CTAs).  A shape is usable when
 // its tile buffers hold the largest tile.  The cheapest usable shape wins; on a tie, the layout
 // with the shorter chain, then the narrower width when a single round suffices (more registers
@@ -193,7 +201,9 @@ constexpr int kLayouts = 4;
 struct LaunchShape {
     int lay, warps;
 };
-inline uint32_t chain_weight(int lay) { return lay == 10 ? 8u : lay == 14 ? 12u : lay == 13 ? 13u : 16u; }
+inline uint32_t chain_weight(int lay) {
+    return lay == 10 ? 8u : lay == 14 ? 12u : lay == 13 ? 13u : lay == 11 ? 15u : 16u;
+}
 inline uint64_t shape_cost(int lay, int warps, uint64_t n_tiles, uint64_t ctas) {
     const uint64_t slots = uint64_t(warps) * (ctas ? ctas : 1);
     return ((n_tiles + slots - 1) / slots) * chain_weight(lay) * uint64_t(48 + warps);
@@ -215,14 +225,14 @@ inline int cta_warps(int lay, uint64_t max_tile_bytes, uint64_t n_tiles, uint64_
     return best.warps ? best.warps : kWarpsNarrow;  // no buffer holds the largest tile: read it from global memory
 }
 // Layout and width of a launch for blobs with 2^prob_bits frequency totals.  `wide_ok` false (a
-// launch that runs 16-warp CTAs only) considers 16 warps alone, and layouts 10, 12 and 13.  When no buffer holds the largest
+// launch that runs 16-warp CTAs only) considers 16 warps alone, and layouts 10 to 13.  When no buffer holds the largest
 // tile: layout 10, or layout 13 if its 16-warp buffers do, else 12, in 16-warp CTAs (the
 // oversized tiles are read from global memory).
 inline LaunchShape launch_shape(int prob_bits, uint64_t max_tile_bytes, uint64_t n_tiles, uint64_t ctas, bool wide_ok) {
     LaunchShape best{0, 0};
-    const int lays12[3] = {14, 13, 12}, lays10[1] = {10};
+    const int lays12[4] = {14, 13, 11, 12}, lays10[1] = {10};
     const int* lays = prob_bits == 10 ? lays10 : lays12;
-    const int nl = prob_bits == 10 ? 1 : 3;
+    const int nl = prob_bits == 10 ? 1 : 4;
     for (int k = 0; k < nl; ++k)
         for (int w : {kWarpsNarrow, kWarps20, kWarpsMid, kWarpsWide}) {
             if (!width_ok(w, lays[k]) || (!wide_ok && (w != kWarpsNarrow || lays[k] == 14))) continue;
@@ -246,9 +256,9 @@ struct LaunchCtx {
 
 // The launches of one output container with one table layout; each (container, layout) pair is
 // compiled in a unit of its own (decode_unit.cu).  The CTA width is in warps: 16, 20, 24 or 32 for
-// layouts 10 and 12, 16 or 20 for layout 13, 16 for layout 14.  A null entry does not exist: the
+// layouts 10, 11 and 12, 16 or 20 for layout 13, 16 for layout 14.  A null entry does not exist: the
 // fields test hook and the row-scaled FP8 container have single-blob launches only, and the
-// allocation-free launch takes layouts 10, 12 and 13.
+// allocation-free launch takes layouts 10 to 13.
 struct Launchers {
     // one blob; `dependent`: launch as a programmatic dependent of the previous decode
     int (*single)(const Params& p, bool vec, int warps, bool esc, const Ctl& ctl, cudaStream_t st, const LaunchCtx& c,
@@ -261,7 +271,7 @@ struct Launchers {
 
 // kLaunch_<container>_<layout>, one per unit.
 #define EP_DECLARE_UNITS(o) \
-    extern const Launchers kLaunch_##o##_10, kLaunch_##o##_12, kLaunch_##o##_13, kLaunch_##o##_14;
+    extern const Launchers kLaunch_##o##_10, kLaunch_##o##_12, kLaunch_##o##_13, kLaunch_##o##_14, kLaunch_##o##_11;
 EP_DECLARE_UNITS(0)
 EP_DECLARE_UNITS(1)
 EP_DECLARE_UNITS(2)
@@ -274,11 +284,11 @@ static_assert(kOutBF16 == 0 && kOutFP16 == 1 && kOutE4M3 == 2 && kOutF32 == 3 &&
               kOutE4M3Row == 6, "unit names use the container numbers");
 
 inline const Launchers* unit_launchers(int out_kind, int lay) {
-#define EP_UNIT_ROW(o) {&kLaunch_##o##_10, &kLaunch_##o##_12, &kLaunch_##o##_13, &kLaunch_##o##_14}
+#define EP_UNIT_ROW(o) {&kLaunch_##o##_10, &kLaunch_##o##_12, &kLaunch_##o##_13, &kLaunch_##o##_14, &kLaunch_##o##_11}
     static const Launchers* const table[7][kLayouts] = {EP_UNIT_ROW(0), EP_UNIT_ROW(1), EP_UNIT_ROW(2), EP_UNIT_ROW(3),
                                                         EP_UNIT_ROW(4), EP_UNIT_ROW(5), EP_UNIT_ROW(6)};
 #undef EP_UNIT_ROW
-    if (out_kind < 0 || out_kind > 6 || !(lay == 10 || lay == 12 || is_hybrid(lay))) return nullptr;
+    if (out_kind < 0 || out_kind > 6 || !(lay == 10 || lay == 12 || is_hybrid(lay))) return nullptr;  // 10..14
     return table[out_kind][layout_index(lay)];
 }
 
