@@ -22,7 +22,7 @@ LIB = os.path.join(PKG, "libentropack.so")
 PLAIN = ["api.cpp", "encoder.cpp", "decode.cu", "encode_gpu.cu"]
 # The decode kernels: decode_unit.cu once per output container (OutKind 0..6) and table layout.
 UNIT_OUTS = range(7)
-UNIT_LAYS = (10, 11, 12, 13, 14)
+UNIT_LAYS = (10, 11, 12, 13, 14, 15)
 HEADERS = ["format.h", "blob.h", "tables.h", "decode_launch.h", "decode_device.cuh"]
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]
 

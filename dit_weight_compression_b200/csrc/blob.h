@@ -19,8 +19,8 @@ constexpr int kMaxHostChunks = 8;   // host-output path: most chunks one call is
 // Device-side state of one blob on one GPU.
 struct DeviceCopy {
     uint8_t* blob = nullptr;        // copy of the serialised bytes (decode reads this)
-    uint8_t* tables[5] = {};        // decode tables expanded from the blob's frequency tables, one
-                                    // block per table layout (10, 12, 13, 14, 11), each made on first use
+    uint8_t* tables[6] = {};        // decode tables expanded from the blob's frequency tables, one
+                                    // block per table layout (10, 12, 13, 14, 11, 15), each made on first use
     uint32_t* status = nullptr;     // sticky error bits written by the decode kernel
     uint8_t* stage_blob = nullptr;  // host-output path: per-call upload target
     uint8_t* stage_out = nullptr;   // host-output path: decode target before the D2H copy

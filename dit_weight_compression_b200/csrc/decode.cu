@@ -145,11 +145,13 @@ int tables_locked(ep_blob* b, int dev, int lay, cudaStream_t st, const uint8_t*&
         auto fn = lay == 10   ? expand_tables_kernel<kWarpsWide, 10>
                   : lay == 11 ? expand_tables_kernel<kWarpsWide, 11>
                   : lay == 12 ? expand_tables_kernel<kWarpsWide, 12>
-                  : lay == 13 ? expand_tables_kernel<kWarpsWide, 13> : expand_tables_kernel<kWarpsWide, 14>;
+                  : lay == 13 ? expand_tables_kernel<kWarpsWide, 13>
+                  : lay == 14 ? expand_tables_kernel<kWarpsWide, 14> : expand_tables_kernel<kWarpsWide, 15>;
         const size_t smem = lay == 10   ? sizeof(ExpandSmem<10>)
                             : lay == 11 ? sizeof(ExpandSmem<11>)
                             : lay == 12 ? sizeof(ExpandSmem<12>)
-                            : lay == 13 ? sizeof(ExpandSmem<13>) : sizeof(ExpandSmem<14>);
+                            : lay == 13 ? sizeof(ExpandSmem<13>)
+                            : lay == 14 ? sizeof(ExpandSmem<14>) : sizeof(ExpandSmem<15>);
         cudaError_t e = cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, int(smem));
         if (e == cudaSuccess) {
             fn<<<1, kWarpsWide * 32, smem, st>>>(ts, tables);

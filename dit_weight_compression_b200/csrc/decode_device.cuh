@@ -105,7 +105,7 @@ struct Tab<12> {
     uint32_t e2;       // per-symbol entries
     uint32_t s1split;  // s1 + the slots of coset 0 in the joint table
 };
-// Layouts 11, 13 and 14 (12-bit totals, hybrid with D = Hybrid<LAY>::kND direct fields per coset and
+// Layouts 11, 15, 13 and 14 (12-bit totals, hybrid with D = Hybrid<LAY>::kND direct fields per coset and
 // B = 7 - D two-lookup ones), at `base` (4 KB aligned): the joint table's direct words at base;
 // field j = 2 .. D + 1 given coset c at base + kHDirect (1 + D c + j - 2); symbol bytes of field
 // j = D + 2 .. 8 given c at base + kL1 + 4096 (B c + j - D - 2); their 4-byte entries (as in
@@ -122,6 +122,8 @@ struct TabHybrid {
 };
 template <>
 struct Tab<11> : TabHybrid {};
+template <>
+struct Tab<15> : TabHybrid {};
 template <>
 struct Tab<13> : TabHybrid {};
 template <>
@@ -281,7 +283,7 @@ __device__ __forceinline__ uint32_t pack_entry(uint32_t bias, uint32_t s, uint32
            (coset << kEntryCosetShift) | (q << kEntryQShift);
 }
 
-// Layout 11, 13 or 14 from the per-context frequencies and cumulative frequencies in `scr`: the
+// Layout 11, 15, 13 or 14 from the per-context frequencies and cumulative frequencies in `scr`: the
 // 1 + 2D direct tables, the 2B symbol-byte tables, then the 4-byte entries of those 2B.
 template <int WARPS, int LAY>
 __device__ void build_hybrid(uint8_t* tab, const BuildScratch& scr) {
@@ -307,8 +309,9 @@ __device__ void build_hybrid(uint8_t* tab, const BuildScratch& scr) {
         // ti 1..2D: f2..f(D+1) given c (direct); ti 2D+1..14: f(D+2)..f8 given c (symbol bytes)
         const bool direct = ti <= 2 * D;
         const uint32_t k = direct ? ti - 1 : ti - 1 - 2 * D;
-        const uint32_t c = direct ? k / D : k / B;
-        const uint32_t j = direct ? 2 + k % D : 2 + D + k % B;
+        constexpr uint32_t Dd = D ? D : 1;  // layout 11 has no direct field after the joint table
+        const uint32_t c = direct ? k / Dd : k / B;
+        const uint32_t j = direct ? 2 + k % Dd : 2 + D + k % B;
         const uint32_t ctx = 8 * c + j - 1;
         const uint16_t* cum = scr.cum[ctx];
         const uint16_t* qs = scr.q[ctx];
@@ -693,7 +696,7 @@ __device__ __forceinline__ void step_symbols12(const Tab<12>& T, Reader& rd, uin
     }
 }
 
-// Layouts 11, 13 and 14: (coset, f1) and the next D fields from direct words (one load each), the
+// Layouts 11, 15, 13 and 14: (coset, f1) and the next D fields from direct words (one load each), the
 // rest as in layout 12.
 template <int LAY, bool ESC, bool FULL, class Reader>
 __device__ __forceinline__ void step_symbols_hybrid(const Tab<LAY>& T, Reader& rd, uint32_t& x, bool active,

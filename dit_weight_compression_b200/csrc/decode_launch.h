@@ -29,28 +29,27 @@ constexpr uint32_t kSlotBytes = kDecodeTables * kCtxBytes;    // 61440
 // warp whose lanes read the same symbol of the same field in both cosets hits different banks.
 constexpr uint32_t kCosetSkew = 64;
 constexpr uint32_t kSymEntryBytes = 16 * 256 * 4 + kCosetSkew;  // 16448 (12-bit totals only)
-// 12-bit totals, hybrid layouts 11, 13 and 14: the joint table and the next kND fields (none for
-// layout 11; f2, f3 for layout 13; f2, f3, f4 for layout 14) given each coset as direct words, one
-// u32 per slot (16 KB a table); the other 7 - kND fields given each coset as symbol bytes (4 KB a
-// table) and 4-byte per-symbol entries (1 KB a table).  Layout 11 takes 86 KB, 13 130 KB, 14
-// 152 KB.
+// 12-bit totals, hybrid layouts 11, 15, 13 and 14: the joint table and the next kND fields (none
+// for layout 11; f2 for layout 15; f2, f3 for layout 13; f2, f3, f4 for layout 14) given each
+// coset as direct words, one u32 per slot (16 KB a table); the other 7 - kND fields given each
+// coset as symbol bytes (4 KB a table) and 4-byte per-symbol entries (1 KB a table).  Layout 11
+// takes 86 KB, 15 108 KB, 13 130 KB, 14 152 KB.
 constexpr uint32_t kHDirect = 4 * 4096;                       // one direct table: 16384
 template <int LAY>
 struct Hybrid {
-    static constexpr uint32_t kND = LAY == 14 ? 3 : LAY == 13 ? 2 : 0;  // direct fields per coset after the joint table
+    static constexpr uint32_t kND = LAY == 14 ? 3 : LAY == 13 ? 2 : LAY == 15 ? 1 : 0;  // direct fields per coset after the joint table
     static constexpr uint32_t kNB = 7 - kND;                   // two-lookup fields per coset
     static constexpr uint32_t kL1 = (1 + 2 * kND) * kHDirect;  // their symbol bytes (16384 / 81920 / 114688)
     static constexpr uint32_t kL2 = kL1 + 2 * kNB * kCtxBytes; // their 4-byte entries
-    static constexpr uint32_t kBytes = kL2 + 2 * kNB * 1024 + kCosetSkew;  // 88128 / 133184 / 155712
+    static constexpr uint32_t kBytes = kL2 + 2 * kNB * 1024 + kCosetSkew;  // 88128 / 110656 / 133184 / 155712
 };
-__host__ __device__ constexpr bool is_hybrid(int lay) { return lay == 11 || lay == 13 || lay == 14; }
+__host__ __device__ constexpr bool is_hybrid(int lay) { return lay == 11 || lay == 13 || lay == 14 || lay == 15; }
 
 // Table layouts: 10 = 10-bit totals, one packed word per slot; 12 = 12-bit totals, two lookups
-// per symbol; 11, 13 and 14 = 12-bit totals, hybrid.
+// per symbol; 11, 13, 14 and 15 = 12-bit totals, hybrid.
 template <int LAY>
 struct TableGeo {
-    static_assert(LAY == 10 || LAY == 11 || LAY == 12 || LAY == 13 || LAY == 14,
-                  "table layouts are 10, 11, 12, 13 and 14");
+    static_assert(LAY >= 10 && LAY <= 15, "table layouts are 10 to 15");
     static constexpr uint32_t kBytes =
         LAY == 10 ? kSlotBytes : LAY == 12 ? kSlotBytes + kSymEntryBytes : Hybrid<LAY>::kBytes;
     static constexpr uint32_t kPiece = kBytes / 4;             // bytes per table bulk copy
@@ -60,7 +59,8 @@ inline uint32_t table_bytes(int lay) {
     return lay == 10 ? TableGeo<10>::kBytes
          : lay == 11 ? TableGeo<11>::kBytes
          : lay == 12 ? TableGeo<12>::kBytes
-         : lay == 13 ? TableGeo<13>::kBytes : TableGeo<14>::kBytes;
+         : lay == 13 ? TableGeo<13>::kBytes
+         : lay == 14 ? TableGeo<14>::kBytes : TableGeo<15>::kBytes;
 }
 
 // kOutE4M3Row: the FP8 container with a per-row scale -- an E4M3 payload normalised per row to
@@ -130,7 +130,8 @@ constexpr uint32_t kBufSlack = 80;        // bytes after a tile buffer that two 
 
 // CTA widths: 16, 20, 24 or 32 warps, each warp with a tile buffer of Geo<WARPS, LAY>::kBuf bytes:
 //   layout 10: 10336, 8240, 6848, 5120;  layout 11: 8656, 6912, 5744, 4288;
-//   layout 12: 9296, 7424, 6176, 4608;   layout 13: 5840, 4656;  layout 14: 4432
+//   layout 12: 9296, 7424, 6176, 4608;   layout 15: 7248, 5792, 4800, 3584;
+//   layout 13: 5840, 4656;  layout 14: 4432
 // (layout 13 leaves room for 16 or 20 warps, layout 14 for 16).  A tile larger than its warp's
 // buffer is read from global memory.
 constexpr int kWarpsNarrow = 16, kWarps20 = 20, kWarpsMid = 24, kWarpsWide = 32;
@@ -158,7 +159,8 @@ constexpr bool fits_smem() { return sizeof(Smem<WARPS, LAY>) + kAlignSlack <= kS
 static_assert(fits_smem<16, 10>() && fits_smem<20, 10>() && fits_smem<24, 10>() && fits_smem<32, 10>() &&
               fits_smem<16, 12>() && fits_smem<20, 12>() && fits_smem<24, 12>() && fits_smem<32, 12>() &&
               fits_smem<16, 13>() && fits_smem<20, 13>() && fits_smem<16, 14>() && fits_smem<16, 11>() &&
-              fits_smem<20, 11>() && fits_smem<24, 11>() && fits_smem<32, 11>(),
+              fits_smem<20, 11>() && fits_smem<24, 11>() && fits_smem<32, 11>() && fits_smem<16, 15>() &&
+              fits_smem<20, 15>() && fits_smem<24, 15>() && fits_smem<32, 15>(),
               "shared memory budget");
 inline bool width_ok(int warps, int lay) {
     if (lay == 14) return warps == kWarpsNarrow;
@@ -181,19 +183,25 @@ inline uint32_t tile_buffer_bytes(int warps, int lay) {
         case 1316: return Geo<16, 13>::kBuf;
         case 1320: return Geo<20, 13>::kBuf;
         case 1416: return Geo<16, 14>::kBuf;
+        case 1516: return Geo<16, 15>::kBuf;
+        case 1520: return Geo<20, 15>::kBuf;
+        case 1524: return Geo<24, 15>::kBuf;
+        case 1532: return Geo<32, 15>::kBuf;
         default: return 0;
     }
 }
 // Index of a layout's expanded tables in a device copy of a blob.
-inline int layout_index(int lay) { return lay == 10 ? 0 : lay == 12 ? 1 : lay == 13 ? 2 : lay == 14 ? 3 : 4; }
-constexpr int kLayouts = 5;
+inline int layout_index(int lay) {
+    return lay == 10 ? 0 : lay == 12 ? 1 : lay == 13 ? 2 : lay == 14 ? 3 : lay == 11 ? 4 : 5;
+}
+constexpr int kLayouts = 6;
 
 // ---- launch shape: table layout and CTA width ------------------------------------------------
 // A launch of n_tiles tiles over `ctas` CTAs (one per SM) runs in rounds: each warp decodes its
 // tiles one after another, so the time is about the number of rounds, ceil(n_tiles / (warps *
 // ctas)), times one tile's rANS chain, stretched by the warps that share the SM.  The chain of a
-// vector is 8 one-load symbols (layout 10), 4 one-load + 4 two-load (14), 3 + 5 (13), 1 + 7 (11)
-// or 8 two-load (12): weights 8, 12, 13, 15, 16 at ~45 cycles a one-load symbol.  Each warp past 16 adds
+// vector is 8 one-load symbols (layout 10), 4 one-load + 4 two-load (14), 3 + 5 (13), 2 + 6 (15),
+// 1 + 7 (11) or 8 two-load (12): weights 8, 12, 13, 14, 15, 16 at ~45 cycles a one-load symbol.  Each warp past 16 adds
 // 1/64 (fitted to the measured choices between 16-, 24- and 32-warp CTAs).  A shape is usable when
 // its tile buffers hold the largest tile.  The cheapest usable shape wins; on a tie, the layout
 // with the shorter chain, then the narrower width when a single round suffices (more registers
@@ -202,7 +210,7 @@ struct LaunchShape {
     int lay, warps;
 };
 inline uint32_t chain_weight(int lay) {
-    return lay == 10 ? 8u : lay == 14 ? 12u : lay == 13 ? 13u : lay == 11 ? 15u : 16u;
+    return lay == 10 ? 8u : lay == 14 ? 12u : lay == 13 ? 13u : lay == 15 ? 14u : lay == 11 ? 15u : 16u;
 }
 inline uint64_t shape_cost(int lay, int warps, uint64_t n_tiles, uint64_t ctas) {
     const uint64_t slots = uint64_t(warps) * (ctas ? ctas : 1);
@@ -230,9 +238,9 @@ inline int cta_warps(int lay, uint64_t max_tile_bytes, uint64_t n_tiles, uint64_
 // oversized tiles are read from global memory).
 inline LaunchShape launch_shape(int prob_bits, uint64_t max_tile_bytes, uint64_t n_tiles, uint64_t ctas, bool wide_ok) {
     LaunchShape best{0, 0};
-    const int lays12[4] = {14, 13, 11, 12}, lays10[1] = {10};
+    const int lays12[5] = {14, 13, 15, 11, 12}, lays10[1] = {10};
     const int* lays = prob_bits == 10 ? lays10 : lays12;
-    const int nl = prob_bits == 10 ? 1 : 4;
+    const int nl = prob_bits == 10 ? 1 : 5;
     for (int k = 0; k < nl; ++k)
         for (int w : {kWarpsNarrow, kWarps20, kWarpsMid, kWarpsWide}) {
             if (!width_ok(w, lays[k]) || (!wide_ok && (w != kWarpsNarrow || lays[k] == 14))) continue;
@@ -256,7 +264,7 @@ struct LaunchCtx {
 
 // The launches of one output container with one table layout; each (container, layout) pair is
 // compiled in a unit of its own (decode_unit.cu).  The CTA width is in warps: 16, 20, 24 or 32 for
-// layouts 10, 11 and 12, 16 or 20 for layout 13, 16 for layout 14.  A null entry does not exist: the
+// layouts 10, 11, 12 and 15, 16 or 20 for layout 13, 16 for layout 14.  A null entry does not exist: the
 // fields test hook and the row-scaled FP8 container have single-blob launches only, and the
 // allocation-free launch takes layouts 10 to 13.
 struct Launchers {
@@ -271,7 +279,8 @@ struct Launchers {
 
 // kLaunch_<container>_<layout>, one per unit.
 #define EP_DECLARE_UNITS(o) \
-    extern const Launchers kLaunch_##o##_10, kLaunch_##o##_12, kLaunch_##o##_13, kLaunch_##o##_14, kLaunch_##o##_11;
+    extern const Launchers kLaunch_##o##_10, kLaunch_##o##_12, kLaunch_##o##_13, kLaunch_##o##_14, kLaunch_##o##_11, \
+        kLaunch_##o##_15;
 EP_DECLARE_UNITS(0)
 EP_DECLARE_UNITS(1)
 EP_DECLARE_UNITS(2)
@@ -284,11 +293,12 @@ static_assert(kOutBF16 == 0 && kOutFP16 == 1 && kOutE4M3 == 2 && kOutF32 == 3 &&
               kOutE4M3Row == 6, "unit names use the container numbers");
 
 inline const Launchers* unit_launchers(int out_kind, int lay) {
-#define EP_UNIT_ROW(o) {&kLaunch_##o##_10, &kLaunch_##o##_12, &kLaunch_##o##_13, &kLaunch_##o##_14, &kLaunch_##o##_11}
+#define EP_UNIT_ROW(o) \
+    {&kLaunch_##o##_10, &kLaunch_##o##_12, &kLaunch_##o##_13, &kLaunch_##o##_14, &kLaunch_##o##_11, &kLaunch_##o##_15}
     static const Launchers* const table[7][kLayouts] = {EP_UNIT_ROW(0), EP_UNIT_ROW(1), EP_UNIT_ROW(2), EP_UNIT_ROW(3),
                                                         EP_UNIT_ROW(4), EP_UNIT_ROW(5), EP_UNIT_ROW(6)};
 #undef EP_UNIT_ROW
-    if (out_kind < 0 || out_kind > 6 || !(lay == 10 || lay == 12 || is_hybrid(lay))) return nullptr;  // 10..14
+    if (out_kind < 0 || out_kind > 6 || lay < 10 || lay > 15) return nullptr;
     return table[out_kind][layout_index(lay)];
 }
 

@@ -31,7 +31,7 @@ int main(int argc, char** argv) {
                                            strtoull(argv[i + 3], 0, 10), atoi(argv[i + 4]) != 0);
         printf("shape %d %d\n", s.lay, s.warps);
     }
-    for (int lay : {10, 11, 12, 13, 14})
+    for (int lay : {10, 11, 12, 13, 14, 15})
         for (int w : {16, 20, 24, 32}) printf("buf %d %d %u %d\n", lay, w, tile_buffer_bytes(w, lay), int(width_ok(w, lay)));
     return 0;
 }
@@ -44,11 +44,13 @@ TABLE_BYTES = {
     10: 15 * 4096,
     11: 1 * 16384 + 14 * 4096 + 14 * 1024 + 64,
     12: 15 * 4096 + 16 * 256 * 4 + 64,
+    15: 3 * 16384 + 12 * 4096 + 12 * 1024 + 64,
     13: 5 * 16384 + 10 * 4096 + 10 * 1024 + 64,
     14: 7 * 16384 + 8 * 4096 + 8 * 1024 + 64,
 }
-WIDTHS = {10: (16, 20, 24, 32), 11: (16, 20, 24, 32), 12: (16, 20, 24, 32), 13: (16, 20), 14: (16,)}
-WEIGHT = {10: 8, 14: 12, 13: 13, 11: 15, 12: 16}
+WIDTHS = {10: (16, 20, 24, 32), 11: (16, 20, 24, 32), 12: (16, 20, 24, 32), 13: (16, 20), 14: (16,),
+          15: (16, 20, 24, 32)}
+WEIGHT = {10: 8, 14: 12, 13: 13, 15: 14, 11: 15, 12: 16}
 
 
 def expected_buffer(lay, w):
@@ -78,7 +80,7 @@ def probe(tmp_path_factory):
 
 def test_buffer_sizes_follow_the_shared_memory_budget(probe):
     _, bufs = probe([])
-    for lay in (10, 11, 12, 13, 14):
+    for lay in (10, 11, 12, 13, 14, 15):
         for w in (16, 20, 24, 32):
             size, ok = bufs[(lay, w)]
             assert ok == (w in WIDTHS[lay]), (lay, w)
@@ -94,8 +96,8 @@ DOCUMENTED = [
     ("4096x11008 @2", 12, 4096, 2752, (13, 20)),
     ("4096x11008 @3.5", 12, 7152, 2752, (12, 20)),
     ("4096x11008 @6", 12, 6144, 5504, (11, 20)),
-    ("4096x11008 @11", 12, 5696, 11008, (11, 20)),
-    ("DiT set, grouped", 12, 5136, 5376, (11, 20)),
+    ("4096x11008 @11", 12, 5696, 11008, (15, 20)),
+    ("DiT set, grouped", 12, 5136, 5376, (15, 20)),
     ("DiT 3072x3072 alone", 12, 5136, 576, (13, 16)),
     ("large-layer stream, grouped", 12, 4080, 4 * 28672, (11, 32)),
     ("large-layer stream, 10-bit", 10, 4080, 4 * 28672, (10, 32)),
@@ -116,13 +118,13 @@ def _cost(lay, w, n, ctas):
 def test_choice_is_usable_and_cheapest(probe):
     cases = [(pb, tile, n, ctas, True)
              for pb in (10, 12)
-             for tile in (160, 2000, 4064, 4288, 4432, 4433, 4656, 4700, 5120, 5744, 5840, 6176, 6848, 6912, 7424, 8240,
-                 8656, 9296)
+             for tile in (160, 2000, 3584, 4064, 4288, 4432, 4433, 4656, 4700, 4800, 5120, 5744, 5792, 5840, 6176, 6848,
+                          6912, 7248, 7424, 8240, 8656, 9296)
              for n in (1, 4, 148, 2368, 2369, 2960, 3552, 4144, 4736, 10000, 114688)
              for ctas in (148, 132)]
     shapes, bufs = probe(cases)
     for (pb, tile, n, ctas, _), (lay, w) in zip(cases, shapes):
-        lays = (10,) if pb == 10 else (14, 13, 11, 12)
+        lays = (10,) if pb == 10 else (14, 13, 15, 11, 12)
         usable = [(l, x) for l in lays for x in WIDTHS[l] if bufs[(l, x)][0] >= tile]
         assert (lay == 10) == (pb == 10)
         if not usable:
@@ -132,14 +134,15 @@ def test_choice_is_usable_and_cheapest(probe):
 
 
 def test_sixteen_warp_launches_and_oversized_tiles(probe):
-    cases = list(itertools.product((10, 12), (4064, 5000, 6000, 9000, 12000), (100, 100000), (148,), (False,)))
+    cases = list(itertools.product((10, 12), (4064, 5000, 6000, 7000, 8000, 9000, 12000), (100, 100000), (148,), (False,)))
     cases += [(12, 12000, 100000, 148, True), (10, 12000, 100000, 148, True), (12, 9296, 100000, 148, True)]
     shapes, bufs = probe(cases)
     for (pb, tile, n, ctas, wide), (lay, w) in zip(cases, shapes):
         if not wide:
             assert w == 16 and lay != 14
             if pb == 12 and tile <= bufs[(12, 16)][0]:
-                assert lay == (13 if tile <= bufs[(13, 16)][0] else 11 if tile <= bufs[(11, 16)][0] else 12)
+                assert lay == (13 if tile <= bufs[(13, 16)][0] else 15 if tile <= bufs[(15, 16)][0]
+                               else 11 if tile <= bufs[(11, 16)][0] else 12)
         if tile > 10336:  # no buffer holds it: 16 warps, tiles read from global memory
             assert w == 16 and lay == (10 if pb == 10 else 12)
     assert shapes[-1] == (12, 16)   # fits 16-warp layout-12 buffers only

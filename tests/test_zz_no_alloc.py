@@ -88,11 +88,12 @@ def test_noalloc_matches_decompress_twice(ep, pb):
     _two_calls_match(ep, comp, W.BF16, lambda: torch.empty(comp.shape, dtype=torch.bfloat16, device="cuda"))
 
 
-@pytest.mark.parametrize("rate", [4.0, 4.3])
+@pytest.mark.parametrize("rate", [3.5, 4.0, 4.3])
 def test_noalloc_large_tiles(ep, rate):
-    """Tiles of about 8.1 and 8.8 KB (S = 64): too large for layout 13's buffers, so the
-    allocation-free kernel takes layout 11 (the joint table direct) and layout 12 (every symbol in
-    two lookups), each with its tables built inside every CTA."""
+    """Tiles of about 7.1, 8.1 and 8.8 KB (S = 64): too large for layout 13's buffers, so the
+    allocation-free kernel takes layout 15 (the joint table and f2 direct), layout 11 (the joint
+    table direct) and layout 12 (every symbol in two lookups), each with its tables built inside
+    every CTA."""
     g = np.random.Generator(np.random.PCG64(int(rate * 100)))
     bits = W.to_bf16_bits(g.normal(0, 0.02, (256, 8192)))
     comp = ep.compress(W.bits_to_torch(bits, W.BF16), ep.LatticeRANSConfig(rate, steps_per_tile=64))
