@@ -233,7 +233,7 @@ inline int cta_warps(int lay, uint64_t max_tile_bytes, uint64_t n_tiles, uint64_
     return best.warps ? best.warps : kWarpsNarrow;  // no buffer holds the largest tile: read it from global memory
 }
 // Layout and width of a launch for blobs with 2^prob_bits frequency totals.  `wide_ok` false (a
-// launch that runs 16-warp CTAs only) considers 16 warps alone, and layouts 10 to 13.  When no buffer holds the largest
+// launch that runs 16-warp CTAs only) considers 16 warps alone, and every layout but 14.  When no buffer holds the largest
 // tile: layout 10, or layout 13 if its 16-warp buffers do, else 12, in 16-warp CTAs (the
 // oversized tiles are read from global memory).
 inline LaunchShape launch_shape(int prob_bits, uint64_t max_tile_bytes, uint64_t n_tiles, uint64_t ctas, bool wide_ok) {
@@ -266,7 +266,7 @@ struct LaunchCtx {
 // compiled in a unit of its own (decode_unit.cu).  The CTA width is in warps: 16, 20, 24 or 32 for
 // layouts 10, 11, 12 and 15, 16 or 20 for layout 13, 16 for layout 14.  A null entry does not exist: the
 // fields test hook and the row-scaled FP8 container have single-blob launches only, and the
-// allocation-free launch takes layouts 10 to 13.
+// allocation-free launch takes every layout but 14.
 struct Launchers {
     // one blob; `dependent`: launch as a programmatic dependent of the previous decode
     int (*single)(const Params& p, bool vec, int warps, bool esc, const Ctl& ctl, cudaStream_t st, const LaunchCtx& c,
